@@ -1,0 +1,78 @@
+"""Per-token centering and quantizers -- oracle (test infrastructure).
+
+What the pages fix:
+- CentriQ §3, Eq. 1: symmetric b-bit per-token quantizer,
+  Q_a(x) = alpha * clip(round(x / alpha), -(2^(b-1) - 1), 2^(b-1) - 1), alpha = r / (2^(b-1) - 1),
+  with range r = ||x||_inf (absmax). b = 8 gives the A8 grid {-127..127}; b = 4 gives
+  {-7..7} (App. B.2: "quantizes to {-7,...,7}").
+- OrbitQuant PR #25, "Default changes": absmax INT8 at A8, Lloyd-Max codes below.
+- CentriQ §4.2 "Centering and exact re-injection": x_c = x - mean(x) * 1 over the n native
+  channels, one scalar stored beside the per-token scale.
+- FLUX.1-schnell-OrbitQuant-W4A4 model card, "Quantization": activation normalization
+  epsilon 1e-10.
+
+Readings where the pages are open:
+- round() is round-half-to-even; the range is floored at eps: alpha = max(r, eps) / qmax.
+- The Lloyd-Max scale is the token's RMS, sigma = max(sqrt(mean(z^2)), eps), which normalises
+  the rotated token to the unit-variance marginal the N(0, 1) codebook is built for.
+  The code of a value u = z / sigma is the number of thresholds strictly below u (nearest
+  centroid; a tie at a threshold goes to the lower index).
+- 4-bit codes are packed two per byte: element 2j in bits 0-3 of byte j, element 2j+1 in
+  bits 4-7. Absmax codes are two's-complement nibbles; Lloyd-Max codes are indices 0..15.
+
+Parity: pinned (tests/test_oracle_quant.py): the largest coordinate maps to +-qmax, the
+error bound |z - alpha q| <= alpha / 2, brute-force nearest grid point on small inputs,
+nearest-centroid brute force for Lloyd-Max codes, offset invariance of centered codes
+(CentriQ Eq. 6), pack/unpack round trip and hand-written byte examples.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+EPS = 1e-10
+
+
+def center(x: np.ndarray):
+    """(x - mean * 1, mean) with the mean over the native channels of each token."""
+    x = np.asarray(x, dtype=np.float64)
+    mean = x.sum(axis=1) / x.shape[1]
+    return x - mean[:, None], mean
+
+
+def absmax_quantize(z: np.ndarray, qmax: int, eps: float = EPS):
+    """Eq. 1 with r = ||z||_inf: returns (int64 codes [T, d], alpha float64 [T])."""
+    z = np.asarray(z, dtype=np.float64)
+    r = np.max(np.abs(z), axis=1)
+    alpha = np.maximum(r, eps) / qmax
+    q = np.clip(np.rint(z / alpha[:, None]), -qmax, qmax).astype(np.int64)
+    return q, alpha
+
+
+def lloyd_max_quantize(z: np.ndarray, thresholds: np.ndarray, eps: float = EPS):
+    """Nearest-centroid Lloyd-Max codes of z / sigma: (int64 codes [T, d], sigma [T])."""
+    z = np.asarray(z, dtype=np.float64)
+    sigma = np.maximum(np.sqrt(np.mean(z * z, axis=1)), eps)
+    u = z / sigma[:, None]
+    # number of thresholds strictly below u (searchsorted 'left' counts tau_k < u)
+    codes = np.searchsorted(np.asarray(thresholds, dtype=np.float64), u, side="left")
+    return codes.astype(np.int64), sigma
+
+
+def pack_nibbles(v: np.ndarray) -> np.ndarray:
+    """Pack 4-bit values (signed -8..7 or unsigned 0..15) of [R, d] into uint8 [R, d/2]."""
+    v = np.asarray(v, dtype=np.int64)
+    if v.shape[-1] % 2:
+        raise ValueError("even width required")
+    n = v & 0xF
+    return (n[..., 0::2] | (n[..., 1::2] << 4)).astype(np.uint8)
+
+
+def unpack_nibbles(b: np.ndarray, signed: bool) -> np.ndarray:
+    """Inverse of ``pack_nibbles``: uint8 [R, d/2] -> int64 [R, d]."""
+    b = np.asarray(b, dtype=np.int64)
+    lo, hi = b & 0xF, (b >> 4) & 0xF
+    out = np.empty(b.shape[:-1] + (2 * b.shape[-1],), dtype=np.int64)
+    out[..., 0::2], out[..., 1::2] = lo, hi
+    if signed:
+        out = np.where(out >= 8, out - 16, out)
+    return out

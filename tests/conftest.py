@@ -1,0 +1,24 @@
+"""Shared pytest configuration.
+
+Tests marked ``gpu`` need a CUDA device (a B200, sm_100a) and the built C-ABI library;
+everything else runs on the CPU. Select with ``-m gpu`` / ``-m "not gpu"``.
+"""
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+GOLDEN = os.path.join(ROOT, "tests", "golden")
+
+
+def pytest_configure(config):
+    config.addinivalue_line("markers", "gpu: needs a CUDA device and the built library")
+
+
+@pytest.fixture(scope="session")
+def golden_dir():
+    return GOLDEN

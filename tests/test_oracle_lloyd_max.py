@@ -1,0 +1,86 @@
+"""Pins for the oracle's 16-level N(0,1) Lloyd-Max codebook (CPU only).
+
+The optimality conditions are the definition of a Lloyd-Max quantizer; Max (1960) tabulates
+the 16-level Gaussian quantizer; scipy.optimize minimises the distortion by a different
+method (Nelder-Mead on the thresholds). OrbitQuant PR #25 "Default changes" names the
+codebook and its solvers.
+"""
+import os
+
+import numpy as np
+from scipy.optimize import minimize
+from scipy.special import ndtr
+
+import oracle
+from oracle import lloyd_max as L
+
+
+def _phi(x):
+    return np.exp(-0.5 * x * x) / np.sqrt(2 * np.pi)
+
+
+def check_conditions(c, t):
+    edges = np.concatenate(([-np.inf], t, [np.inf]))
+    p = ndtr(edges[1:]) - ndtr(edges[:-1])
+    phi = np.where(np.isfinite(edges), _phi(np.where(np.isfinite(edges), edges, 0.0)), 0.0)
+    with np.errstate(invalid="ignore", divide="ignore"):
+        cond_centroid = np.nanmax(np.abs(c - (phi[:-1] - phi[1:]) / p))
+    cond_mid = np.abs(t - 0.5 * (c[:-1] + c[1:])).max()
+    return cond_centroid < 1e-12 and cond_mid < 1e-15
+
+
+def load_max1960(golden_dir):
+    rows = [l.split() for l in open(os.path.join(golden_dir,
+                                                 "lloyd_max_16_gaussian_max1960.txt"))
+            if l.strip() and not l.startswith("#")]
+    return rows
+
+
+def check_max1960(c, t, golden_dir):
+    ok = True
+    for kind, idx, val in load_max1960(golden_dir):
+        got = (t if kind == "threshold" else c)[int(idx)]
+        ok &= abs(got - float(val)) <= 6e-4
+    return ok
+
+
+def test_optimality_conditions():
+    c, t = oracle.lloyd_max_gaussian()
+    assert check_conditions(c, t)
+
+
+def test_odd_symmetry():
+    c, t = oracle.lloyd_max_gaussian()
+    assert np.abs(c + c[::-1]).max() < 1e-13
+    assert np.abs(t + t[::-1]).max() < 1e-13
+    assert np.all(np.diff(c) > 0) and np.all(np.diff(t) > 0)
+
+
+def test_matches_max_1960_table(golden_dir):
+    c, t = oracle.lloyd_max_gaussian()
+    assert check_max1960(c, t, golden_dir)
+
+
+def test_agrees_with_direct_minimisation():
+    c, t = oracle.lloyd_max_gaussian()
+
+    def distortion(pos):
+        tt = np.sort(np.concatenate((-pos[::-1], [0.0], pos)))
+        e = np.concatenate(([-np.inf], tt, [np.inf]))
+        p = L._cell_prob(e[:-1], e[1:])
+        cc = (L._phi(e[:-1]) - L._phi(e[1:])) / p
+        return L.lloyd_max_mse(cc, tt)
+
+    r = minimize(distortion, t[8:] + 0.05, method="Nelder-Mead",
+                 options=dict(xatol=1e-12, fatol=1e-17, maxiter=50000, maxfev=100000))
+    assert np.abs(np.sort(r.x) - t[8:]).max() < 1e-6
+    assert abs(r.fun - L.lloyd_max_mse(c, t)) < 1e-13
+
+
+def test_mse_closed_form_matches_monte_carlo():
+    c, t = oracle.lloyd_max_gaussian()
+    x = np.random.default_rng(5).standard_normal(2_000_000)
+    q = c[np.searchsorted(t, x)]
+    mc = float(np.mean((x - q) ** 2))
+    assert abs(mc - L.lloyd_max_mse(c, t)) < 3e-4 * 1.0
+    assert 0.0094 < L.lloyd_max_mse(c, t) < 0.0096

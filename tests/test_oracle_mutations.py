@@ -1,0 +1,150 @@
+"""Planted mistakes in the oracle must be caught by its pins (CPU only).
+
+Each case swaps one oracle function for a copy with a plausible slip (a dropped term, a
+wrong sign or index, a transposed operand) and asserts that at least one pin of the
+matching test module now fails. Mistakes are planted only in the oracle, on the CPU.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from oracle import linear as Lm
+from oracle import lloyd_max as LL
+from oracle import quant as Qm
+from oracle import rpbh as R
+
+import test_oracle_linear as TL
+import test_oracle_lloyd_max as TLL
+import test_oracle_quant as TQ
+import test_oracle_rpbh as TR
+
+
+def _fails(fn, *a):
+    try:
+        return not fn(*a)
+    except Exception:
+        return True
+
+
+def _rot_mutant(kind):
+    def rotate(z, plan, h):
+        z = np.asarray(z, dtype=np.float64)
+        T, d = z.shape
+        H = R.sylvester_hadamard(h).astype(np.float64)
+        if kind != "no_norm":
+            H = H / np.sqrt(h)
+        for signs, perm in plan:
+            if kind == "sign_by_source":
+                u = (signs[None, :] * z)[:, perm]
+            elif kind == "scatter":
+                u = np.empty_like(z)
+                u[:, perm] = signs[None, :] * z
+            else:
+                u = signs[None, :] * z[:, perm]
+            if kind == "strided_blocks":
+                z = (u.reshape(T, h, d // h).transpose(0, 2, 1) @ H.T)
+                z = z.transpose(0, 2, 1).reshape(T, d)
+            else:
+                z = (u.reshape(T, d // h, h) @ H.T).reshape(T, d)
+        return z
+    return rotate
+
+
+@pytest.mark.parametrize("kind", ["no_norm", "sign_by_source", "scatter", "strided_blocks"])
+def test_rotation_mistakes_are_caught(monkeypatch, kind):
+    monkeypatch.setattr(R, "rotate", _rot_mutant(kind))
+    caught = (_fails(TR.check_orthogonal, 64, 16, 1)
+              or _fails(TR.check_basis_closed_form, 32, 8)
+              or _fails(TR.check_basis_closed_form, 64, 16))
+    assert caught
+
+
+def test_hadamard_sign_mistake_is_caught(monkeypatch):
+    def bad(h):
+        i = np.arange(h, dtype=np.uint64)
+        par = np.bitwise_count(i[:, None] | i[None, :]) & 1
+        return np.where(par == 1, -1, 1).astype(np.int64)
+    monkeypatch.setattr(R, "sylvester_hadamard", bad)
+    # (-1)^popcount(i|j) is D H D, still a Hadamard matrix: the Sylvester pins catch it
+    assert _fails(TR.check_sylvester, 8)
+
+
+def test_splitmix_mistake_is_caught(monkeypatch, golden_dir):
+    def bad_mix(z):
+        with np.errstate(over="ignore"):
+            z = (z ^ (z >> np.uint64(29))) * R._M1
+            z = (z ^ (z >> np.uint64(27))) * R._M2
+            return z ^ (z >> np.uint64(31))
+    monkeypatch.setattr(R, "_mix64", bad_mix)
+    assert _fails(TR.check_splitmix_vector, golden_dir)
+
+
+def test_absmax_mistakes_are_caught(monkeypatch):
+    z = np.random.default_rng(1).standard_normal((20, 64))
+
+    def off_by_one(z, qmax, eps=1e-10):
+        r = np.max(np.abs(z), axis=1)
+        alpha = np.maximum(r, eps) / (qmax + 1)
+        return np.clip(np.rint(z / alpha[:, None]), -qmax, qmax).astype(np.int64), alpha
+
+    def floor_round(z, qmax, eps=1e-10):
+        r = np.max(np.abs(z), axis=1)
+        alpha = np.maximum(r, eps) / qmax
+        return np.clip(np.floor(z / alpha[:, None]), -qmax, qmax).astype(np.int64), alpha
+
+    for m in (off_by_one, floor_round):
+        monkeypatch.setattr(Qm, "absmax_quantize", m)
+        assert _fails(TQ.check_absmax, z, 7)
+
+
+def test_lloyd_max_code_mistake_is_caught(monkeypatch):
+    z = np.random.default_rng(2).standard_normal((10, 64))
+
+    def shifted(z, thresholds, eps=1e-10):
+        sigma = np.maximum(np.sqrt(np.mean(z * z, axis=1)), eps)
+        codes = np.searchsorted(thresholds, z / sigma[:, None], side="left")
+        return np.minimum(codes + 1, 15), sigma
+
+    monkeypatch.setattr(Qm, "lloyd_max_quantize", shifted)
+    assert _fails(TQ.check_lloyd_max_codes, z)
+
+
+def test_lloyd_iteration_mistake_is_caught(monkeypatch, golden_dir):
+    def bad(levels=16, tol=1e-15, max_iter=2000):
+        c = np.linspace(-2.5, 2.5, levels)
+        for _ in range(max_iter):
+            t = 0.5 * (c[:-1] + c[1:])
+            e = np.concatenate(([-np.inf], t, [np.inf]))
+            c = (LL._phi(e[:-1]) - LL._phi(e[1:]))          # forgot / P(cell)
+        return c, 0.5 * (c[:-1] + c[1:])
+    c, t = bad()
+    assert _fails(TLL.check_conditions, c, t) and _fails(TLL.check_max1960, c, t, golden_dir)
+
+
+def test_gemm_transpose_mistake_is_caught(monkeypatch):
+    monkeypatch.setattr(Lm, "gemm_int", lambda a, w: np.asarray(a, float) @ np.asarray(w, float))
+    assert _fails(TL.check_gemm)
+
+
+def test_dropped_rank1_term_is_caught(monkeypatch):
+    def no_rank1(x, w, plan, h, center_tokens, bias=None):
+        x = np.asarray(x, dtype=np.float64)
+        xc = oracle.center(x)[0] if center_tokens else x
+        y = Lm.rotate(xc, plan, h) @ Lm.rotate(np.asarray(w, float), plan, h).T
+        return y + (0 if bias is None else np.asarray(bias)[None, :])
+    monkeypatch.setattr(Lm, "linear_unquantized", no_rank1)
+    assert _fails(TL.check_identity_quantizer, True, 1, False)
+
+
+def test_weight_rotation_transposed_is_caught(monkeypatch):
+    # weights rotated by Q instead of Q^T (rows through the inverse): W_R = W Q
+    def bad(x, w, plan, h, center_tokens, bias=None):
+        x = np.asarray(x, dtype=np.float64)
+        w = np.asarray(w, dtype=np.float64)
+        xc, mean = oracle.center(x) if center_tokens else (x, None)
+        y = Lm.rotate(xc, plan, h) @ oracle.unrotate(w, plan, h).T
+        if mean is not None:
+            y = y + mean[:, None] * w.sum(axis=1)[None, :]
+        return y + (0 if bias is None else np.asarray(bias)[None, :])
+    monkeypatch.setattr(Lm, "linear_unquantized", bad)
+    assert _fails(TL.check_identity_quantizer, False, 1, False)

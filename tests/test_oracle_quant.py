@@ -1,0 +1,102 @@
+"""Pins for the oracle's centering, quantizers and nibble packing (CPU only).
+
+CentriQ §3 Eq. 1 (symmetric per-token grid), §4.2 (centering), Eq. 6 (offset invariance);
+OrbitQuant PR #25 (absmax A8, Lloyd-Max below 8 bits).
+"""
+import numpy as np
+import pytest
+
+import oracle
+from oracle import quant as Qm
+
+
+def check_absmax(z, qmax):
+    q, alpha = Qm.absmax_quantize(z, qmax)
+    ok = True
+    # the largest coordinate lands on the end of the grid
+    j = np.argmax(np.abs(z), axis=1)
+    ok &= bool(np.all(np.abs(q[np.arange(len(z)), j]) == qmax))
+    # rounding error at most half a step, codes inside the grid
+    ok &= bool(np.all(np.abs(z - alpha[:, None] * q) <= alpha[:, None] * (0.5 + 1e-12)))
+    ok &= bool(np.all(np.abs(q) <= qmax))
+    # brute force: nearest grid point
+    grid = np.arange(-qmax, qmax + 1)
+    dist = np.abs(z[..., None] - alpha[:, None, None] * grid[None, None, :])
+    best = grid[np.argmin(dist, axis=-1)]
+    tie = np.sort(dist, axis=-1)
+    clear = (tie[..., 1] - tie[..., 0]) > 1e-12 * alpha[:, None]
+    ok &= bool(np.all(best[clear] == q[clear]))
+    return ok
+
+
+def check_lloyd_max_codes(z):
+    c, t = oracle.lloyd_max_gaussian()
+    codes, sigma = Qm.lloyd_max_quantize(z, t)
+    u = z / sigma[:, None]
+    dist = np.abs(u[..., None] - c[None, None, :])
+    srt = np.sort(dist, axis=-1)
+    clear = (srt[..., 1] - srt[..., 0]) > 1e-12
+    ok = bool(np.all(np.argmin(dist, axis=-1)[clear] == codes[clear]))
+    ok &= bool(np.allclose(sigma, np.sqrt((z * z).mean(axis=1)), rtol=1e-14))
+    return ok
+
+
+@pytest.mark.parametrize("qmax", [127, 7])
+def test_absmax_quantizer(qmax):
+    rng = np.random.default_rng(1)
+    z = rng.standard_normal((40, 96)) * rng.uniform(0.01, 100, (40, 1))
+    assert check_absmax(z, qmax)
+
+
+def test_absmax_zero_row_uses_eps():
+    q, alpha = Qm.absmax_quantize(np.zeros((2, 16)), 127)
+    assert np.all(q == 0) and np.allclose(alpha, 1e-10 / 127)
+
+
+def test_lloyd_max_codes_are_nearest_centroid():
+    rng = np.random.default_rng(2)
+    z = rng.standard_normal((30, 128)) * rng.uniform(0.1, 5, (30, 1))
+    assert check_lloyd_max_codes(z)
+
+
+def test_lloyd_max_threshold_tie_goes_low():
+    c, t = oracle.lloyd_max_gaussian()
+    # a token whose RMS is exactly 1 and that holds values exactly on thresholds
+    z = np.array([[t[3], -t[3], t[10], -t[10]]])
+    z = z / np.sqrt(np.mean(z * z))
+    codes, sigma = Qm.lloyd_max_quantize(z, t)
+    u = z / sigma[:, None]
+    assert np.all(codes == np.searchsorted(t, u[0], side="left"))
+
+
+def test_centering_and_offset_invariance():
+    # CentriQ Eq. 6: codes and scale of the centered token do not depend on x + c 1.
+    # x on a 2^-4 grid and c = 3/8 keep every sum exact in float64.
+    rng = np.random.default_rng(3)
+    x = np.round(rng.standard_normal((8, 256)) * 16) / 16
+    c = 3.0 / 8.0
+    xc1, m1 = Qm.center(x)
+    xc2, m2 = Qm.center(x + c)
+    assert np.array_equal(xc1, xc2) and np.array_equal(m2 - m1, np.full(8, c))
+    assert np.allclose(xc1.sum(axis=1), 0.0, atol=1e-12)
+    plan = oracle.rpbh_plan(256, 64, 1, 0)
+    z1 = oracle.rotate(xc1, plan, 64)
+    z2 = oracle.rotate(xc2, plan, 64)
+    q1, a1 = Qm.absmax_quantize(z1, 7)
+    q2, a2 = Qm.absmax_quantize(z2, 7)
+    assert np.array_equal(q1, q2) and np.array_equal(a1, a2)
+
+
+def test_pack_nibbles_hand_examples():
+    assert Qm.pack_nibbles(np.array([[1, -1]]))[0, 0] == 0xF1
+    assert Qm.pack_nibbles(np.array([[-7, 7]]))[0, 0] == 0x79
+    assert Qm.pack_nibbles(np.array([[0, 15]]))[0, 0] == 0xF0
+    assert Qm.pack_nibbles(np.array([[3, 0, -8, 2]])).tolist() == [[0x03, 0x28]]
+
+
+def test_pack_unpack_round_trip():
+    rng = np.random.default_rng(4)
+    s = rng.integers(-7, 8, (5, 64))
+    assert np.array_equal(Qm.unpack_nibbles(Qm.pack_nibbles(s), signed=True), s)
+    u = rng.integers(0, 16, (5, 64))
+    assert np.array_equal(Qm.unpack_nibbles(Qm.pack_nibbles(u), signed=False), u)
