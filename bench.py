@@ -1,0 +1,441 @@
+#!/usr/bin/env python
+"""Benchmark of the rotated, quantized linear layer on B200.
+
+One step = one pass of the whole hot path over one batch of tokens: the fused
+center + RPBH + quantize kernel followed by the tcgen05 low-bit GEMM with its dequant
+epilogue (weights are prepared once, offline, before timing). Default workload: the
+DiT-width W4A8 layer, T = 4096 tokens, d_in = d_out = 3072, block h = 1024, one round,
+absmax INT8 activations, INT4 per-channel weights.
+
+  python bench.py [--gpus N --steps K --warmup W] [--impl reference] [--workload NAME]
+
+Multi-GPU (launched by torchrun, one process per GPU): tokens are independent, so every rank
+runs its own batch with no collective on the data path (weak scaling); the only collectives
+are the barriers around the timed region and the max-over-ranks of the time.
+
+Timing: CUDA events on the launching stream over exactly K steps, a barrier and a
+synchronize on both sides. Inputs rotate over 4 independent sets (about 270 MB, more than
+the 126 MB L2), so no step reads data a previous step left in L2. Per-kernel durations
+come from events recorded between the two launches of every timed step. nvidia-smi
+samples the SM clock and throttle reasons during the timed region.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "rotate+quantize GB/s (% of HBM peak); W4A8/W4A4 linear TOPS (% tensor peak)"
+RING = 4
+# nominal dense int8 / bf16 tensor throughput ratio on B200 (4.5 / 2.25 PFLOP/s)
+INT8_PER_BF16 = 2.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# DRAM traffic per launch from an ncu capture, valid only for the kernel source it was taken
+# on (sha256 of the .cu file at capture time); null once the kernel has changed.
+NCU_TRAFFIC = {}
+
+
+def parse():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=4000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="dit_w4a8",
+                    choices=["tiny", "dit_w4a8", "narrow_lm", "mlp_up"])
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override the token count (small cases for profiler captures)")
+    ap.add_argument("--e2e-steps", type=int, default=100)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="CPU time budget of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def sha_of(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()
+
+
+# ---- clocks ---------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid, enabled=True):
+        self.uuid = uuid
+        self.proc = None
+        self.enabled = enabled
+        self.path = None
+
+    def __enter__(self):
+        if not self.enabled:
+            return self
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-f", self.path], stdout=subprocess.DEVNULL,
+                stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["not sampled"]}
+        rows = []
+        with open(self.path) as f:
+            for r in csv.reader(f):
+                r = [c.strip() for c in r]
+                if len(r) < 9:
+                    continue
+                if self.uuid and r[0] != self.uuid:
+                    continue
+                rows.append(r)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = sorted(float(r[1]) for r in rows if r[1].replace(".", "").isdigit())
+        mx = max(float(r[2]) for r in rows if r[2].replace(".", "").isdigit())
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": sm[len(sm) // 2] if sm else None, "sm_max_mhz": mx,
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max((float(r[3]) for r in rows
+                                    if r[3].replace(".", "").isdigit()), default=None)}
+
+
+# ---- CPU oracle legs ---------------------------------------------------------------------------
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def oracle_setup(wl, x_bits, w_bits):
+    import numpy as np
+    import oracle
+    import synth
+    plan = oracle.rpbh_plan(wl.d, wl.h, wl.rounds, wl.seed)
+    c, t = oracle.lloyd_max_gaussian()
+    w_codes, s_w, w1 = oracle.prepare_weights(synth.bf16_to_f64(w_bits), plan, wl.h)
+    return plan, c, t, w_codes, s_w, w1
+
+
+def oracle_pass(wl, setup, x_rows_f64):
+    import oracle
+    plan, c, t, w_codes, s_w, w1 = setup
+    qa = oracle.quantize_activations(x_rows_f64, plan, wl.h, wl.act, wl.center, t)
+    if wl.act == "int4_lloydmax":
+        acc = oracle.gemm_lloyd_max(qa["codes"], c, w_codes)
+    else:
+        acc = oracle.gemm_int(qa["codes"], w_codes)
+    return oracle.epilogue(acc, qa["scale"], s_w, qa["mean"] if wl.center else None,
+                           w1 if wl.center else None)
+
+
+def cpu_baseline(wl, x_bits, w_bits, seconds):
+    import synth
+    setup = oracle_setup(wl, x_bits, w_bits)
+    n = min(1024, wl.T)
+    xs = synth.bf16_to_f64(x_bits[:n])
+    done, t0 = 0, time.perf_counter()
+    while True:
+        oracle_pass(wl, setup, xs)
+        done += 1
+        el = time.perf_counter() - t0
+        if el >= seconds or done >= 64:
+            break
+    ops = 2.0 * n * wl.d * wl.n_out * done
+    return {"value": ops / el / 1e12, "unit": "TOPS", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{done} pass(es) of the oracle over {n} of the {wl.T} tokens "
+                      f"(float64 NumPy, weights prepared beforehand), {el:.1f} s"}
+
+
+def run_reference(args, wl, rank):
+    """--impl reference: the CPU oracle, as it stands, timed on the host cores."""
+    if rank != 0:
+        return None
+    import numpy as np
+    import synth
+    wl_, x_bits, w_bits = synth.make_inputs(wl.name, T=min(wl.T, 1024))
+    setup = oracle_setup(wl, x_bits, w_bits)
+    xs = synth.bf16_to_f64(x_bits)
+    # size each step so that warm-up + K steps take about two minutes in total
+    t0 = time.perf_counter()
+    oracle_pass(wl, setup, xs[:8])
+    per_tok = (time.perf_counter() - t0) / 8
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    n = int(max(1, min(len(xs), budget / max(per_tok, 1e-6))))
+    for i in range(args.warmup):
+        oracle_pass(wl, setup, xs[:n])
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        oracle_pass(wl, setup, xs[(i * n) % (len(xs) - n + 1):][:n])
+    el = time.perf_counter() - t0
+    ops = 2.0 * n * wl.d * wl.n_out * args.steps
+    v = ops / el / 1e12
+    sample = f"{n} tokens per step of the {wl.T}-token workload (float64 NumPy oracle)"
+    return {"metric": METRIC, "value": v, "unit": "TOPS", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": config_of(wl, wl.T, args.gpus),
+            "cpu_baseline": {"value": v, "unit": "TOPS", "cores": blas_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": v, "unit": "TOPS", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def config_of(wl, T, n):
+    return {"workload": wl.name, "T": T, "d_in": wl.d, "d_out": wl.n_out, "h": wl.h,
+            "rounds": wl.rounds, "act": wl.act, "center": wl.center, "weights": "int4",
+            "l2": f"inputs rotate over {RING} sets larger than L2 together",
+            "parallelism": "replicas" if n == 1 else f"dp{n} (tokens split, no collective)"}
+
+
+# ---- GPU leg ---------------------------------------------------------------------------------
+def main():
+    args = parse()
+    import synth
+    wl = synth.WORKLOADS[args.workload]
+    T = args.tokens or wl.T
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        line = run_reference(args, wl, rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return 0
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    import w4a8_ptq_linear_b200 as oq
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    _, _, w_bits = synth.make_inputs(wl.name, T=1)
+    plan = oq.Plan(wl.d, wl.h, wl.rounds, seed=wl.seed, center=wl.center, act=wl.act)
+    to_dev = lambda b: torch.from_numpy(np.ascontiguousarray(b)).view(torch.bfloat16).to(dev)
+
+    # RING independent sets: activations, prepared weights, codes, scales, outputs
+    sets = []
+    x_host_bits = None
+    for r in range(RING):
+        xb = synth.make_x(T, wl.d, mean_var=wl.mean_var, heavy_frac=wl.heavy_frac,
+                          outliers=wl.outliers, outlier_gain=wl.outlier_gain,
+                          seed=wl.seed + 1000 * rank + r)
+        if r == 0:
+            x_host_bits = xb
+        w = to_dev(w_bits)
+        wp, ws, w1 = oq.prepare_weights(plan, w)
+        del w
+        s = {"x": to_dev(xb), "wp": wp, "ws": ws, "w1": w1,
+             "codes": torch.empty((T, wl.d // 2 if plan.packed else wl.d),
+                                  dtype=torch.uint8 if plan.packed else torch.int8, device=dev),
+             "scale": torch.empty(T, dtype=torch.float32, device=dev),
+             "mean": torch.empty(T, dtype=torch.float32, device=dev) if wl.center else None,
+             "y": torch.empty((T, wl.n_out), dtype=torch.bfloat16, device=dev)}
+        sets.append(s)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+
+    def step(s):
+        oq.rotate_quantize(plan, s["x"], codes=s["codes"], scale=s["scale"], mean=s["mean"],
+                           stream=stream)
+
+    def gemm(s):
+        if wl.act == "int8_absmax":
+            oq.gemm_w4a8(s["codes"], s["scale"], s["wp"], s["ws"], mean=s["mean"],
+                         w_rowsum=s["w1"] if wl.center else None, out=s["y"], stream=stream)
+        else:
+            oq.gemm_w4a4(plan, wl.act, s["codes"], s["scale"], s["wp"], s["ws"],
+                         mean=s["mean"], w_rowsum=s["w1"] if wl.center else None, out=s["y"],
+                         stream=stream)
+
+    for i in range(max(3, args.warmup)):
+        s = sets[i % RING]
+        step(s)
+        gemm(s)
+    torch.cuda.synchronize()
+    st, code = oq.device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} code {code:#x} after warm-up")
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(uuid, enabled=not args.no_clocks) as clk:
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_start.record(stream)
+        for i in range(K):
+            s = sets[i % RING]
+            ev[i][0].record(stream)
+            step(s)
+            ev[i][1].record(stream)
+            gemm(s)
+            ev[i][2].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    rq_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / K
+    gm_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / K
+    st, code = oq.device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} code {code:#x} after timing")
+
+    t_max = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
+    elapsed_ms = float(t_max.item())
+    clocks = clk.summary()
+
+    # ---- end to end through the public API with host buffers ------------------------------
+    x_pin = torch.from_numpy(np.ascontiguousarray(x_host_bits)).view(torch.bfloat16).pin_memory()
+    y_pin = torch.empty((T, wl.n_out), dtype=torch.bfloat16).pin_memory()
+    s0 = sets[0]
+    ws_bytes = plan.workspace_bytes(T)
+    workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    x_dev = torch.empty_like(s0["x"])
+
+    def e2e_step():
+        x_dev.copy_(x_pin, non_blocking=True)
+        oq.linear(plan, x_dev, s0["wp"], s0["ws"], s0["w1"] if wl.center else None,
+                  workspace=workspace, out=s0["y"], stream=stream)
+        y_pin.copy_(s0["y"], non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = torch.tensor([e0.elapsed_time(e1) / args.e2e_steps], dtype=torch.float64,
+                          device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    e2e_ms = float(e2e_ms.item())
+    barrier()
+
+    # ---- numbers ------------------------------------------------------------------------------
+    ops = 2.0 * T * wl.d * wl.n_out
+    ms_per_step = elapsed_ms / K
+    value = ops * world / (ms_per_step * 1e-3) / 1e12
+    code_bytes = T * wl.d if wl.act == "int8_absmax" else T * wl.d // 2
+    rq_bytes = T * wl.d * 2 + code_bytes + 4 * T * (2 if wl.center else 1)
+    peaks, peak_kind = load_peaks()
+    long_region = elapsed_ms > 1000.0
+    bf16_peak = peaks.get("bf16_tflops_sustained" if long_region else "bf16_tflops",
+                          peaks["bf16_tflops"])
+    tensor_peak = bf16_peak * (INT8_PER_BF16 if wl.act != "int4_lloydmax" else 1.0)
+    hbm_peak = peaks["hbm_gbs"]
+    gemm_tops = ops / (gm_ms * 1e-3) / 1e12
+    rq_gbs = rq_bytes / (rq_ms * 1e-3) / 1e9
+    kfile = os.path.join(ROOT, "w4a8_ptq_linear_b200", "csrc", "k_gemm.cu")
+    tr = NCU_TRAFFIC.get((wl.name, "k_gemm"))
+    traffic = tr["bytes"] if tr and tr["sha"] == sha_of(kfile) else None
+    kfile_rq = os.path.join(ROOT, "w4a8_ptq_linear_b200", "csrc", "k_rotate_quant.cu")
+    tr_rq = NCU_TRAFFIC.get((wl.name, "k_rotate_quant"))
+    traffic_rq = tr_rq["bytes"] if tr_rq and tr_rq["sha"] == sha_of(kfile_rq) else None
+    peak_note = (f"{peak_kind} {'sustained' if long_region else 'burst'} bf16 "
+                 f"{bf16_peak} TFLOP/s" + (" x 2 (nominal int8/bf16 ratio)"
+                                           if wl.act != "int4_lloydmax" else ""))
+    gemm_roof = {"bound": "tensor", "achieved": gemm_tops, "peak": tensor_peak,
+                 "unit": "TOPS" if wl.act != "int4_lloydmax" else "TFLOP/s",
+                 "frac": gemm_tops / tensor_peak, "traffic": traffic, "kernel": "k_gemm",
+                 "peak_source": peak_note, "ms_per_launch": gm_ms}
+    rq_roof = {"bound": "hbm", "achieved": rq_gbs, "peak": hbm_peak, "unit": "GB/s",
+               "frac": rq_gbs / hbm_peak, "traffic": traffic_rq, "kernel": "k_rotate_quant",
+               "peak_source": f"{peak_kind} copy bandwidth", "ms_per_launch": rq_ms,
+               "algorithmic_bytes": rq_bytes}
+    dominant = gemm_roof if gm_ms >= rq_ms else rq_roof
+    other = rq_roof if dominant is gemm_roof else gemm_roof
+    line = {
+        "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8" if wl.act != "int4_lloydmax"
+        else "f16", "data": "synthetic", "config": config_of(wl, T, world),
+        "rotate_quantize_gbs": rq_gbs, "rotate_quantize_frac_hbm": rq_gbs / hbm_peak,
+        "gemm_tops": gemm_tops, "gemm_frac_tensor": gemm_tops / tensor_peak,
+        "roofline": dominant, "roofline_other": other,
+        "kernel_share": {"k_rotate_quant": rq_ms / (rq_ms + gm_ms),
+                         "k_gemm": gm_ms / (rq_ms + gm_ms)},
+        "e2e": {"value": ops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TOPS",
+                "h2d_bytes_per_step": T * wl.d * 2, "d2h_bytes_per_step": T * wl.n_out * 2,
+                "ms_per_step": e2e_ms, "steps": args.e2e_steps},
+        "gpu_launches": 2 * K,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, x_host_bits, w_bits, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    plan.close()
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

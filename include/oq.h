@@ -1,0 +1,204 @@
+/*
+ * oq.h -- C ABI of the rotated, quantized linear layer for NVIDIA B200 (sm_100a).
+ *
+ * The layer (CentriQ: Calibration-Free Quantization of Diffusion Transformers via Exact Mean
+ * Centering, §4.2 Eq. 5 and App. B.2 Eq. 9; OrbitQuant PR #25 "Default changes"):
+ *
+ *     y_t = s_w (.) W_hat_R  Q_a( R (x_t - mean_t 1) )  +  mean_t * w_1  +  b
+ *
+ *   - mean_t     per-token mean over the d native channels (optional centering, CentriQ §4.2);
+ *   - R          RPBH rotation: `rounds` independent rounds, each a gather by a random
+ *                permutation, random signs and the orthonormal Sylvester block Hadamard of
+ *                size h on consecutive blocks (OrbitQuant PR #25; CentriQ §3, §2);
+ *   - Q_a        per-token quantizer: absmax INT8 {-127..127}, absmax INT4 {-7..7}
+ *                (CentriQ §3 Eq. 1) or the 16-level N(0,1) Lloyd-Max codebook on x / RMS(x);
+ *   - W_hat_R    the weight pre-rotated by the same R (W_R = W R^T) and quantized to INT4
+ *                per output channel with scale s_w;
+ *   - w_1 = W 1  row sums of the unrotated, unquantized weight, kept in fp32 (CentriQ Eq. 4).
+ *
+ * Conventions for every call:
+ *   - Pointers named *_host are host memory; every other pointer is device memory on the
+ *     current CUDA device. The caller owns all buffers and streams; the library owns only
+ *     the plan.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream). Compute calls are
+ *     asynchronous on that stream and never synchronize the device.
+ *   - Row-major layouts; "ld" arguments are row pitches in elements.
+ *   - Argument errors are returned before anything is launched. Launch failures return
+ *     OQ_ERR_CUDA. Every device-side wait is bounded: a wait that gives up records a code in
+ *     a device error word and the kernel returns; oq_device_status() reads that word.
+ *   - oq_last_error() returns a human-readable message for the last failure on the calling
+ *     host thread.
+ *
+ * Data formats:
+ *   - activations / weights: bfloat16, row-major [rows, d];
+ *   - A8 codes: int8 [T, d];
+ *   - 4-bit codes: uint8 [rows, d/2], element 2j in bits 0-3 of byte j and element 2j+1 in
+ *     bits 4-7; absmax codes (and weight codes) are two's-complement nibbles in -7..7,
+ *     Lloyd-Max codes are indices 0..15 into the ascending codebook;
+ *   - per-token scale (alpha_t, or sigma_t for Lloyd-Max), per-token mean, per-channel s_w
+ *     and w_1: float32;
+ *   - bias: bfloat16 [d_out] or NULL;
+ *   - output: bfloat16 [T, d_out] (OQ_OUT_BF16) or raw accumulators [T, d_out] (OQ_OUT_ACC:
+ *     int32 for the integer GEMMs, float32 for the Lloyd-Max GEMM).
+ *
+ * Limits: d % 32 == 0, 32 <= d <= 32768; h a power of two, 1 <= h <= 1024, h | d;
+ * rounds in {1, 2}; T >= 0 (T == 0 launches nothing); d_out % 16 == 0; base pointers
+ * 16-byte aligned, row pitches multiples of 16 bytes.
+ */
+#ifndef OQ_H
+#define OQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  OQ_OK = 0,
+  OQ_ERR_INVALID_ARG = 1,    /* a size, enum or pointer is out of its documented range */
+  OQ_ERR_UNSUPPORTED = 2,    /* valid but outside this build (e.g. no sm_100 device)    */
+  OQ_ERR_MISALIGNED = 3,     /* a pointer or pitch breaks the 16-byte rule              */
+  OQ_ERR_CUDA = 4,           /* a CUDA runtime/driver call failed                       */
+  OQ_ERR_DEVICE_TIMEOUT = 5, /* a bounded device-side wait gave up                      */
+  OQ_ERR_NOMEM = 6           /* host or device allocation for a plan failed             */
+} oq_status;
+
+typedef enum {
+  OQ_ACT_INT8_ABSMAX = 0,    /* A8: alpha_t = max|z_t| / 127, codes in -127..127         */
+  OQ_ACT_INT4_ABSMAX = 1,    /* A4: alpha_t = max|z_t| / 7,   codes in -7..7             */
+  OQ_ACT_INT4_LLOYDMAX = 2   /* A4: sigma_t = RMS(z_t), nearest of 16 N(0,1) centroids   */
+} oq_act_kind;
+
+typedef enum {
+  OQ_OUT_BF16 = 0,           /* dequantised, rank-1 and bias added, rounded to bf16      */
+  OQ_OUT_ACC = 1             /* raw GEMM accumulators, no epilogue (test mode)           */
+} oq_out_kind;
+
+typedef struct oq_plan oq_plan; /* opaque, library-owned */
+
+/* ---- status ----------------------------------------------------------------------- */
+
+/* Static string naming a status code. */
+const char* oq_status_string(oq_status s);
+
+/* Message describing the last failure on the calling host thread ("" if none). */
+const char* oq_last_error(void);
+
+/* Synchronizes the current device, then returns OQ_ERR_DEVICE_TIMEOUT if a kernel recorded
+ * a bounded-wait failure since the last clear (its site code in *code_out if non-NULL),
+ * OQ_ERR_CUDA if the device reports an error, else OQ_OK. clear != 0 resets the word. */
+oq_status oq_device_status(int clear, uint64_t* code_out);
+
+/* ---- policies (host only) ---------------------------------------------------------- */
+
+/* Largest power of two dividing d, capped at 1024 (FLUX.1-schnell-OrbitQuant-W4A4 model card,
+ * "Quantization": block size policy largest_power_of_two_dividing_dim). 0 if d <= 0. */
+int oq_default_block(int d);
+
+/* 2 if h < 512 else 1 (OrbitQuant PR #25, "Default changes": rotation_rounds "auto"). */
+int oq_default_rounds(int h);
+
+/* ---- plan tables (host only, no device needed) ------------------------------------- */
+
+/* Signs (+1/-1) and permutation of RPBH round `round` (0-based) for width d and `seed`.
+ * The permutation is a gather: rotated position i reads channel perm_host[i].
+ * SplitMix64 in counter form: round r draws signs from key v(seed, 2r) and the
+ * permutation from key v(seed, 2r+1), with v(k, i) = mix64(k + (i+1) * 0x9E3779B97F4A7C15);
+ * sign i is -1 when bit 63 of v(k_sign, i) is set; perm sorts i by v(k_perm, i), ties by i.
+ * signs_host: int8[d], perm_host: int32[d], both caller-owned. */
+oq_status oq_rpbh_tables(int d, int round, uint64_t seed, int8_t* signs_host,
+                         int32_t* perm_host);
+
+/* 16-level Lloyd-Max codebook for N(0,1), solved by Newton's method on the centroid and
+ * midpoint conditions (OrbitQuant PR #25: codebook v3 uses a Newton solver).
+ * centroids16_host: double[16] ascending; thresholds15_host: double[15] midpoints. */
+oq_status oq_lloyd_max_codebook(double* centroids16_host, double* thresholds15_host);
+
+/* ---- plan ------------------------------------------------------------------------------ */
+
+/* Builds the RPBH tables and codebook on the host and uploads the tables (rounds * d
+ * uint16 entries, < 128 KiB) to the current device. The plan belongs to that device.
+ * center != 0 subtracts the per-token mean before the rotation (CentriQ §4.2). */
+oq_status oq_plan_create(oq_plan** out, int d, int h, int rounds, uint64_t seed,
+                         int center, oq_act_kind act);
+
+/* Frees the plan and its device tables. NULL is ignored. */
+void oq_plan_destroy(oq_plan* plan);
+
+/* Host copies of a plan's RPBH round (same layout as oq_rpbh_tables). */
+oq_status oq_plan_get_rpbh(const oq_plan* plan, int round, int8_t* signs_host,
+                           int32_t* perm_host);
+
+/* ---- compute ----------------------------------------------------------------------- */
+
+/* Fused center + RPBH + per-token scale + quantize (CentriQ §4.2 "Activation path",
+ * App. B.2 "the prologue ... subtracts its mean, applies ... H ... and quantizes";
+ * OrbitQuant PR #25 "Runtime work": the pre-rotation as one kernel).
+ *   x_bf16       [T, ldx] bf16, ldx >= d, (ldx * 2) % 16 == 0
+ *   codes        int8 [T, d] (A8) or uint8 [T, d/2] (A4 kinds)
+ *   scale        float [T]: alpha_t (absmax kinds) or sigma_t (Lloyd-Max)
+ *   mean         float [T] per-token mean; required iff the plan centers, else ignored
+ *   rotated_f32  float [T, d] normalised rotated (centered) values, or NULL (test output) */
+oq_status oq_rotate_quantize(const oq_plan* plan, const void* x_bf16, int64_t T, int64_t ldx,
+                             void* codes, float* scale, float* mean, float* rotated_f32,
+                             void* stream);
+
+/* Offline weight preparation (CentriQ §3 "Hadamard rotation": W x = (W R^T)(R x); §4.2
+ * Eq. 4: w_1 = W 1 in fp32 from the unquantized weight): every row of W goes through the
+ * plan's rotation without centering, is quantized to INT4 per output channel
+ * (s_w[o] = max|W_R[o,:]| / 7), and w_1[o] = sum_k W[o,k] (fp32, before rotation).
+ *   w_bf16    [n_out, ldw] bf16
+ *   w_packed  uint8 [n_out, d/2] two's-complement nibbles
+ *   w_scale   float [n_out];  w_rowsum float [n_out] */
+oq_status oq_prepare_weights(const oq_plan* plan, const void* w_bf16, int64_t n_out,
+                             int64_t ldw, uint8_t* w_packed, float* w_scale,
+                             float* w_rowsum, void* stream);
+
+/* W4A8 GEMM with the fused dequant epilogue (CentriQ Eq. 5 / Eq. 9):
+ *   acc[t,o] = sum_k a[t,k] * w[o,k]                     (exact int32)
+ *   y[t,o]   = bf16( a_scale[t] * w_scale[o] * acc + mean[t] * w_rowsum[o] + bias[o] )
+ *   a         int8 [T, d_in]; a_scale float [T]
+ *   mean      float [T] or NULL (no rank-1 term; w_rowsum may then be NULL)
+ *   w_packed  uint8 [d_out, d_in/2]; w_scale float [d_out]
+ *   bias_bf16 bf16 [d_out] or NULL
+ *   out       bf16 [T, d_out] (OQ_OUT_BF16) or int32 [T, d_out] (OQ_OUT_ACC) */
+oq_status oq_gemm_w4a8(const int8_t* a, const float* a_scale, const float* mean,
+                       const uint8_t* w_packed, const float* w_scale, const float* w_rowsum,
+                       const void* bias_bf16, int64_t T, int64_t d_in, int64_t d_out,
+                       oq_out_kind out_kind, void* out, void* stream);
+
+/* W4A4 GEMM, same epilogue. kind = OQ_ACT_INT4_ABSMAX (integer GEMM, exact int32
+ * accumulators) or OQ_ACT_INT4_LLOYDMAX (codes decoded through the plan's codebook to fp16,
+ * fp16 x fp16 -> fp32 GEMM; a_scale holds sigma_t; OQ_OUT_ACC gives float32). `plan` is
+ * required for Lloyd-Max (codebook) and ignored otherwise.
+ *   a_packed  uint8 [T, d_in/2] */
+oq_status oq_gemm_w4a4(const oq_plan* plan, oq_act_kind kind, const uint8_t* a_packed,
+                       const float* a_scale, const float* mean, const uint8_t* w_packed,
+                       const float* w_scale, const float* w_rowsum, const void* bias_bf16,
+                       int64_t T, int64_t d_in, int64_t d_out, oq_out_kind out_kind,
+                       void* out, void* stream);
+
+/* Bytes of device workspace oq_linear needs for T tokens (codes, scales, means). */
+size_t oq_linear_workspace_bytes(const oq_plan* plan, int64_t T);
+
+/* The whole layer: oq_rotate_quantize into `workspace`, then the GEMM for the plan's
+ * activation kind, on one stream. y_bf16 is [T, d_out] bf16. workspace must hold
+ * oq_linear_workspace_bytes(plan, T) bytes, 256-byte aligned; it is scratch owned by the
+ * caller and overwritten. */
+oq_status oq_linear(const oq_plan* plan, const void* x_bf16, int64_t T, int64_t ldx,
+                    const uint8_t* w_packed, const float* w_scale, const float* w_rowsum,
+                    const void* bias_bf16, int64_t d_out, void* y_bf16, void* workspace,
+                    size_t workspace_bytes, void* stream);
+
+/* Test hook for the bounded waits: launches one block that waits on an mbarrier nothing
+ * will arrive on, for at most timeout_ns, then records a timeout and returns. The next
+ * oq_device_status() reports OQ_ERR_DEVICE_TIMEOUT. The GPU stays usable. */
+oq_status oq_debug_wait_timeout(uint64_t timeout_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* OQ_H */

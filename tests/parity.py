@@ -1,0 +1,56 @@
+"""Comparison helpers for the parity tests (GPU results against the oracle).
+
+Tolerances (stated for this layer): rotated values <= 1e-5 relative to fp64 (Frobenius,
+per token); codes identical except where the oracle value lies within 1e-5 relative of a
+decision boundary; integer accumulators bit-exact given the same codes; final bf16 outputs
+<= 8e-3 relative (Frobenius over the whole output).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+ROT_TOL = 1e-5
+BOUNDARY_REL = 1e-5
+OUT_TOL = 8e-3
+
+
+def to_torch_bf16(bits: np.ndarray, device="cuda"):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(bits)).view(torch.bfloat16).to(device)
+
+
+def rel_fro(a, b) -> float:
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    nb = np.linalg.norm(b)
+    return float(np.linalg.norm(a - b) / nb) if nb > 0 else float(np.linalg.norm(a - b))
+
+
+def per_token_rel(a, b) -> np.ndarray:
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    nb = np.linalg.norm(b, axis=1)
+    return np.linalg.norm(a - b, axis=1) / np.where(nb > 0, nb, 1.0)
+
+
+def absmax_boundary_mask(z: np.ndarray, alpha: np.ndarray, qmax: int) -> np.ndarray:
+    """True where z / alpha lies within 1e-5 relative of a rounding boundary k + 1/2
+    (or of the clip edge qmax, whose neighbourhood both sides round identically)."""
+    v = z / alpha[:, None]
+    k = np.floor(v)
+    b = k + 0.5
+    near = np.abs(v - b) <= BOUNDARY_REL * np.maximum(np.abs(b), 0.5)
+    return near & (np.abs(b) < qmax)
+
+
+def lloyd_max_boundary_mask(z: np.ndarray, sigma: np.ndarray, thresholds) -> np.ndarray:
+    u = z / sigma[:, None]
+    t = np.asarray(thresholds, dtype=np.float64)
+    d = np.abs(u[..., None] - t[None, None, :])
+    return np.any(d <= BOUNDARY_REL * np.maximum(np.abs(t), 1.0)[None, None, :], axis=-1)
+
+
+def compare_codes(gpu_codes: np.ndarray, ref_codes: np.ndarray, exempt: np.ndarray):
+    """(number of differing codes outside the exemption, number of exempted positions)."""
+    diff = gpu_codes != ref_codes
+    return int(np.sum(diff & ~exempt)), int(np.sum(exempt))

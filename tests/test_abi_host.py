@@ -1,0 +1,78 @@
+"""The C-ABI library on the CPU: it loads, exports every declared entry point, and its
+host-side tables agree with the oracle (no GPU needed, no compute call is made)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+import w4a8_ptq_linear_b200 as oq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    src = open(os.path.join(ROOT, "include", "oq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(oq_[a-z0-9_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from w4a8_ptq_linear_b200 import build
+    build.build()
+    return oq.lib()
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = declared_symbols()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(lib, n), n
+    bound = {s[0] for s in oq.SIGNATURES}
+    assert set(names) == bound, "binding and header disagree"
+
+
+def test_status_strings(lib):
+    for code, name in [(0, "OQ_OK"), (1, "OQ_ERR_INVALID_ARG"), (5, "OQ_ERR_DEVICE_TIMEOUT")]:
+        assert lib.oq_status_string(code).decode() == name
+
+
+@pytest.mark.parametrize("d,rounds,seed", [(256, 1, 0), (3072, 2, 0), (1920, 2, 7),
+                                           (30720, 1, 123456789)])
+def test_rpbh_tables_match_oracle_bit_for_bit(lib, d, rounds, seed):
+    plan = oracle.rpbh_plan(d, oracle.default_block(d) if d % 1024 == 0 else 64, rounds, seed)
+    for r in range(rounds):
+        s, p = oq.rpbh_tables(d, r, seed)
+        assert np.array_equal(s.astype(np.float64), plan[r][0])
+        assert np.array_equal(p.astype(np.int64), plan[r][1])
+
+
+def test_newton_codebook_matches_lloyd_iteration(lib):
+    c_lib, t_lib = oq.lloyd_max_codebook()
+    c_or, t_or = oracle.lloyd_max_gaussian()
+    assert np.abs(c_lib - c_or).max() < 1e-10
+    assert np.abs(t_lib - t_or).max() < 1e-10
+
+
+def test_default_policies_match_oracle(lib):
+    for d in (256, 1152, 1920, 3072, 4096, 30720):
+        assert oq.default_block(d) == oracle.default_block(d)
+    for h in (64, 128, 256, 512, 1024):
+        assert oq.default_rounds(h) == oracle.default_rounds(h)
+
+
+def test_argument_validation_before_any_cuda_call(lib):
+    h = ctypes.c_void_p()
+    # h does not divide d, h not a power of two, bad rounds, bad d: rejected up front
+    for args in [(3072, 2048, 1), (3072, 96, 1), (3072, 1024, 3), (3000, 8, 1), (0, 8, 1)]:
+        st = lib.oq_plan_create(ctypes.byref(h), args[0], args[1], args[2], 0, 0, 0)
+        assert st == oq.OQ_ERR_INVALID_ARG, args
+    st = lib.oq_plan_create(ctypes.byref(h), 256, 64, 1, 0, 0, 9)
+    assert st == oq.OQ_ERR_INVALID_ARG
+    # GEMM shape checks happen before any launch
+    st = lib.oq_gemm_w4a8(None, None, None, None, None, None, None, 16, 100, 256, 0, None, None)
+    assert st == oq.OQ_ERR_INVALID_ARG
+    assert b"d_in" in lib.oq_last_error()

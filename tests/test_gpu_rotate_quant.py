@@ -1,0 +1,128 @@
+"""GPU parity of the fused center + RPBH + quantize kernel against the oracle.
+
+Each case runs oq_rotate_quantize through the C ABI on seeded synthetic tokens and compares
+element by element with the oracle: normalised rotated values (<= 1e-5 relative per token),
+per-token scales (<= 1e-5 relative), means, and codes (identical except within 1e-5
+relative of a decision boundary). Shapes span several CTAs' worth of tokens, ragged token
+counts, every block size from 1 to 1024, one and two rounds and the widest width.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from parity import (ROT_TOL, absmax_boundary_mask, compare_codes, lloyd_max_boundary_mask,
+                    per_token_rel, to_torch_bf16)
+
+pytestmark = pytest.mark.gpu
+
+QMAX = {"int8_absmax": 127, "int4_absmax": 7}
+
+CASES = [
+    # T, d, h, rounds, act, center
+    (64, 256, 64, 1, "int8_absmax", False),
+    (300, 3072, 1024, 1, "int8_absmax", False),
+    (257, 3072, 1024, 1, "int4_absmax", True),
+    (130, 1920, 128, 2, "int4_lloydmax", False),
+    (77, 4096, 512, 1, "int8_absmax", True),
+    (45, 4096, 256, 2, "int4_absmax", False),
+    (33, 256, 1, 1, "int8_absmax", False),
+    (40, 512, 8, 2, "int4_lloydmax", True),
+    (1, 3072, 1024, 1, "int8_absmax", True),
+    (9, 30720, 1024, 1, "int8_absmax", False),
+    (5, 30720, 64, 2, "int4_lloydmax", True),
+    (600, 1920, 64, 2, "int8_absmax", False),
+]
+
+
+def run_case(T, d, h, rounds, act, center, seed=0):
+    import torch
+    import w4a8_ptq_linear_b200 as oq
+    xb = synth.make_x(T, d, mean_var=3.0, heavy_frac=0.01, seed=seed)
+    plan = oq.Plan(d, h, rounds, seed=seed, center=center, act=act)
+    x = to_torch_bf16(xb)
+    codes, scale, mean, rot = oq.rotate_quantize(plan, x, rotated=True)
+    torch.cuda.synchronize()
+    st, code = oq.device_status()
+    assert st == 0, code
+    thresholds = oracle.lloyd_max_gaussian()[1]
+    ref = oracle.quantize_activations(synth.bf16_to_f64(xb), oracle.rpbh_plan(d, h, rounds, seed),
+                                      h, act, center, thresholds)
+    out = {
+        "codes": codes.cpu().numpy(), "scale": scale.cpu().numpy().astype(np.float64),
+        "mean": None if mean is None else mean.cpu().numpy().astype(np.float64),
+        "rot": rot.cpu().numpy().astype(np.float64),
+    }
+    plan.close()
+    return xb, ref, out
+
+
+@pytest.mark.parametrize("T,d,h,rounds,act,center", CASES)
+def test_rotate_quantize_matches_oracle(T, d, h, rounds, act, center):
+    xb, ref, out = run_case(T, d, h, rounds, act, center)
+    # rotated values
+    assert per_token_rel(out["rot"], ref["rotated"]).max() <= ROT_TOL
+    # scales and means
+    assert np.abs(out["scale"] / ref["scale"] - 1).max() <= ROT_TOL
+    if center:
+        x = synth.bf16_to_f64(xb)
+        tol = 1e-6 * np.abs(x).mean(axis=1) + 1e-30
+        assert np.all(np.abs(out["mean"] - ref["mean"]) <= tol)
+    # codes
+    if act == "int8_absmax":
+        gpu = out["codes"].view(np.int8).astype(np.int64)
+        ex = absmax_boundary_mask(ref["rotated"], ref["scale"], 127)
+    elif act == "int4_absmax":
+        gpu = oracle.unpack_nibbles(out["codes"], signed=True)
+        ex = absmax_boundary_mask(ref["rotated"], ref["scale"], 7)
+    else:
+        gpu = oracle.unpack_nibbles(out["codes"], signed=False)
+        ex = lloyd_max_boundary_mask(ref["rotated"], ref["scale"], oracle.lloyd_max_gaussian()[1])
+    bad, n_ex = compare_codes(gpu, ref["codes"], ex)
+    assert bad == 0, f"{bad} codes differ outside the boundary exemption ({n_ex} exempt)"
+
+
+def test_zero_and_constant_tokens():
+    import torch
+    import w4a8_ptq_linear_b200 as oq
+    d = 1024
+    xb = np.zeros((4, d), np.uint16)
+    xb[1] = synth.f64_to_bf16(np.full(d, 0.75))    # constant token
+    xb[2] = synth.f64_to_bf16(np.full(d, -3.0))
+    xb[3, 5] = synth.f64_to_bf16(np.array([2.0]))[0]   # one non-zero channel
+    for center in (False, True):
+        plan = oq.Plan(d, 256, 1, center=center, act="int8_absmax")
+        codes, scale, mean, _ = oq.rotate_quantize(plan, to_torch_bf16(xb))
+        c = codes.cpu().numpy().view(np.int8)
+        s = scale.cpu().numpy()
+        assert np.all(c[0] == 0) and abs(s[0] - 1e-10 / 127) < 1e-16
+        if center:
+            # a constant token centers to exactly zero: all codes 0, scale eps / qmax
+            m = mean.cpu().numpy()
+            assert m[1] == np.float32(0.75) and m[2] == np.float32(-3.0)
+            assert np.all(c[1] == 0) and np.all(c[2] == 0)
+        plan.close()
+    torch.cuda.synchronize()
+
+
+def test_empty_batch_launches_nothing():
+    import torch
+    import w4a8_ptq_linear_b200 as oq
+    plan = oq.Plan(256, 64, 1)
+    x = torch.empty((0, 256), dtype=torch.bfloat16, device="cuda")
+    codes, scale, _, _ = oq.rotate_quantize(plan, x)
+    assert codes.shape == (0, 256)
+    plan.close()
+
+
+def test_row_pitch_larger_than_width():
+    import torch
+    import w4a8_ptq_linear_b200 as oq
+    T, d = 50, 512
+    xb = synth.make_x(T, 640, mean_var=1.0, seed=4)
+    x = to_torch_bf16(xb)[:, :d]          # ldx = 640
+    plan = oq.Plan(d, 128, 2, act="int8_absmax")
+    codes, scale, _, _ = oq.rotate_quantize(plan, x)
+    codes2, scale2, _, _ = oq.rotate_quantize(plan, x.contiguous())
+    assert torch.equal(codes, codes2) and torch.equal(scale, scale2)
+    plan.close()

@@ -1,0 +1,363 @@
+// C ABI of the rotated, quantized linear layer (declarations and contracts: include/oq.h).
+// Host-side validation, plan lifecycle, the device error word and dispatch to the kernels.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <new>
+
+#include "oq_internal.h"
+#include "ptx.cuh"
+
+// Device error word: first bounded wait that gives up writes (1 << 63 | site << 32 | block).
+__device__ unsigned long long g_oq_error_word;
+
+namespace oq {
+
+static thread_local char g_last_error[512] = "";
+
+oq_status fail(oq_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  std::vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+oq_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(OQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+unsigned long long* device_error_word() {
+  constexpr int kMaxDev = 64;
+  static unsigned long long* ptrs[kMaxDev] = {};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_oq_error_word) != cudaSuccess) return nullptr;
+    ptrs[dev] = static_cast<unsigned long long*>(p);
+  }
+  return ptrs[dev];
+}
+
+namespace {
+
+__global__ void k_debug_wait(unsigned long long* err, unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    dev::mbar_init(dev::smem_u32(&bar), 1);
+    dev::fence_mbar_init();
+    // nothing ever arrives: the wait must give up by itself
+    dev::mbar_wait(dev::smem_u32(&bar), 0, err, kSiteDebug, limit_ns);
+  }
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool pow2(int v) { return v > 0 && (v & (v - 1)) == 0; }
+
+oq_status check_plan_device(const oq_plan* p) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev != p->device)
+    return fail(OQ_ERR_INVALID_ARG, "plan belongs to device %d, current device is %d",
+                p->device, dev);
+  return OQ_OK;
+}
+
+oq_status check_gemm_args(const void* a, const float* a_scale, const float* mean,
+                          const uint8_t* w, const float* w_scale, const float* w_rowsum,
+                          const void* bias, int64_t T, int64_t K, int64_t N, int out_kind,
+                          const void* out) {
+  if (T < 0 || T > 0x7FFFFFFF) return fail(OQ_ERR_INVALID_ARG, "T=%lld out of range", (long long)T);
+  if (K < 32 || K > 32768 || K % 32)
+    return fail(OQ_ERR_INVALID_ARG, "d_in=%lld must be a multiple of 32 in [32, 32768]",
+                (long long)K);
+  if (N < 16 || N > (1 << 24) || N % 16)
+    return fail(OQ_ERR_INVALID_ARG, "d_out=%lld must be a positive multiple of 16",
+                (long long)N);
+  if (out_kind != OQ_OUT_BF16 && out_kind != OQ_OUT_ACC)
+    return fail(OQ_ERR_INVALID_ARG, "unknown out_kind %d", out_kind);
+  if (!w || !w_scale || !out) return fail(OQ_ERR_INVALID_ARG, "NULL weight/scale/out pointer");
+  if (T > 0 && (!a || !a_scale)) return fail(OQ_ERR_INVALID_ARG, "NULL activation pointer");
+  if (mean && !w_rowsum) return fail(OQ_ERR_INVALID_ARG, "mean given without w_rowsum");
+  if ((T > 0 && !aligned16(a)) || !aligned16(w) || !aligned16(out))
+    return fail(OQ_ERR_MISALIGNED, "activation, weight and output must be 16-byte aligned");
+  (void)bias;
+  return OQ_OK;
+}
+
+}  // namespace
+}  // namespace oq
+
+using namespace oq;
+
+extern "C" {
+
+const char* oq_status_string(oq_status s) {
+  switch (s) {
+    case OQ_OK: return "OQ_OK";
+    case OQ_ERR_INVALID_ARG: return "OQ_ERR_INVALID_ARG";
+    case OQ_ERR_UNSUPPORTED: return "OQ_ERR_UNSUPPORTED";
+    case OQ_ERR_MISALIGNED: return "OQ_ERR_MISALIGNED";
+    case OQ_ERR_CUDA: return "OQ_ERR_CUDA";
+    case OQ_ERR_DEVICE_TIMEOUT: return "OQ_ERR_DEVICE_TIMEOUT";
+    case OQ_ERR_NOMEM: return "OQ_ERR_NOMEM";
+  }
+  return "OQ_STATUS_UNKNOWN";
+}
+
+const char* oq_last_error(void) { return g_last_error; }
+
+oq_status oq_device_status(int clear, uint64_t* code_out) {
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+  unsigned long long* w = device_error_word();
+  if (!w) return fail(OQ_ERR_CUDA, "device error word unavailable");
+  unsigned long long v = 0;
+  e = cudaMemcpy(&v, w, sizeof(v), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "read device error word");
+  if (code_out) *code_out = v;
+  if (clear && v) {
+    e = cudaMemset(w, 0, sizeof(v));
+    if (e != cudaSuccess) return cuda_fail(e, "clear device error word");
+  }
+  if (v) return fail(OQ_ERR_DEVICE_TIMEOUT, "device wait gave up: site %u block %u",
+                     (unsigned)((v >> 32) & 0xFFFF), (unsigned)(v & 0xFFFFFFFFu));
+  return OQ_OK;
+}
+
+int oq_default_block(int d) {
+  if (d <= 0) return 0;
+  int h = d & -d;
+  return h > 1024 ? 1024 : h;
+}
+
+int oq_default_rounds(int h) { return h < 512 ? 2 : 1; }
+
+oq_status oq_rpbh_tables(int d, int round, uint64_t seed, int8_t* signs_host,
+                         int32_t* perm_host) {
+  if (d <= 0 || d > 32768) return fail(OQ_ERR_INVALID_ARG, "d=%d out of range", d);
+  if (round < 0) return fail(OQ_ERR_INVALID_ARG, "round must be >= 0");
+  if (!signs_host || !perm_host) return fail(OQ_ERR_INVALID_ARG, "NULL output");
+  rpbh_round_tables(d, round, seed, signs_host, perm_host);
+  return OQ_OK;
+}
+
+oq_status oq_lloyd_max_codebook(double* centroids16_host, double* thresholds15_host) {
+  if (!centroids16_host || !thresholds15_host) return fail(OQ_ERR_INVALID_ARG, "NULL output");
+  lloyd_max_newton(centroids16_host, thresholds15_host);
+  return OQ_OK;
+}
+
+oq_status oq_plan_create(oq_plan** out, int d, int h, int rounds, uint64_t seed, int center,
+                         oq_act_kind act) {
+  if (!out) return fail(OQ_ERR_INVALID_ARG, "NULL plan output");
+  *out = nullptr;
+  if (d < 32 || d > 32768 || d % 32)
+    return fail(OQ_ERR_INVALID_ARG, "d=%d must be a multiple of 32 in [32, 32768]", d);
+  if (!pow2(h) || h > 1024 || d % h)
+    return fail(OQ_ERR_INVALID_ARG, "h=%d must be a power of two <= 1024 dividing d=%d", h, d);
+  if (rounds != 1 && rounds != 2) return fail(OQ_ERR_INVALID_ARG, "rounds=%d not in {1,2}", rounds);
+  if (act != OQ_ACT_INT8_ABSMAX && act != OQ_ACT_INT4_ABSMAX && act != OQ_ACT_INT4_LLOYDMAX)
+    return fail(OQ_ERR_INVALID_ARG, "unknown activation kind %d", (int)act);
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  int major = 0, minor = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  if (major != 10 || minor != 0)
+    return fail(OQ_ERR_UNSUPPORTED, "needs an sm_100 device (found sm_%d%d)", major, minor);
+
+  oq_plan* p = new (std::nothrow) oq_plan();
+  if (!p) return fail(OQ_ERR_NOMEM, "plan allocation");
+  p->d = d; p->h = h; p->rounds = rounds; p->center = center ? 1 : 0; p->act = act;
+  p->seed = seed; p->device = dev;
+  p->signs.resize((size_t)rounds * d);
+  p->perm.resize((size_t)rounds * d);
+  std::vector<uint16_t> tab((size_t)rounds * d);
+  for (int r = 0; r < rounds; ++r) {
+    rpbh_round_tables(d, r, seed, p->signs.data() + (size_t)r * d, p->perm.data() + (size_t)r * d);
+    for (int i = 0; i < d; ++i) {
+      const size_t k = (size_t)r * d + i;
+      tab[k] = (uint16_t)(p->perm[k] | (p->signs[k] < 0 ? 0x8000 : 0));
+    }
+  }
+  lloyd_max_newton(p->cb_c, p->cb_t);
+  e = cudaMalloc(&p->d_tab, tab.size() * sizeof(uint16_t));
+  if (e != cudaSuccess) {
+    delete p;
+    return fail(OQ_ERR_NOMEM, "cudaMalloc plan tables: %s", cudaGetErrorString(e));
+  }
+  e = cudaMemcpy(p->d_tab, tab.data(), tab.size() * sizeof(uint16_t), cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) {
+    cudaFree(p->d_tab);
+    delete p;
+    return cuda_fail(e, "upload plan tables");
+  }
+  if (!device_error_word()) {
+    cudaFree(p->d_tab);
+    delete p;
+    return fail(OQ_ERR_CUDA, "device error word unavailable");
+  }
+  *out = p;
+  return OQ_OK;
+}
+
+void oq_plan_destroy(oq_plan* plan) {
+  if (!plan) return;
+  if (plan->d_tab) {
+    int cur = -1;
+    cudaGetDevice(&cur);
+    if (cur != plan->device) cudaSetDevice(plan->device);
+    cudaFree(plan->d_tab);
+    if (cur != plan->device && cur >= 0) cudaSetDevice(cur);
+  }
+  delete plan;
+}
+
+oq_status oq_plan_get_rpbh(const oq_plan* plan, int round, int8_t* signs_host,
+                           int32_t* perm_host) {
+  if (!plan || !signs_host || !perm_host) return fail(OQ_ERR_INVALID_ARG, "NULL argument");
+  if (round < 0 || round >= plan->rounds) return fail(OQ_ERR_INVALID_ARG, "round out of range");
+  std::memcpy(signs_host, plan->signs.data() + (size_t)round * plan->d, plan->d);
+  std::memcpy(perm_host, plan->perm.data() + (size_t)round * plan->d, plan->d * sizeof(int32_t));
+  return OQ_OK;
+}
+
+static oq_status rotate_quantize_impl(const oq_plan* plan, const void* x, int64_t T, int64_t ldx,
+                                      void* codes, float* scale, float* mean, float* rotated,
+                                      float* rowsum, int mode, int center, cudaStream_t s) {
+  RqArgs a;
+  a.x = x; a.ldx = ldx; a.T = T; a.d = plan->d; a.h = plan->h; a.rounds = plan->rounds;
+  a.center = center; a.mode = mode; a.tab = plan->d_tab; a.codes = codes; a.scale = scale;
+  a.mean = mean; a.rotated = rotated; a.rowsum = rowsum;
+  for (int i = 0; i < 15; ++i) a.thr[i] = (float)plan->cb_t[i];
+  return launch_rotate_quant(a, s);
+}
+
+oq_status oq_rotate_quantize(const oq_plan* plan, const void* x_bf16, int64_t T, int64_t ldx,
+                             void* codes, float* scale, float* mean, float* rotated_f32,
+                             void* stream) {
+  if (!plan) return fail(OQ_ERR_INVALID_ARG, "NULL plan");
+  if (T < 0 || T > 0x7FFFFFFF) return fail(OQ_ERR_INVALID_ARG, "T out of range");
+  if (ldx < plan->d || (ldx * 2) % 16) return fail(OQ_ERR_MISALIGNED, "ldx must be >= d and a multiple of 8");
+  if (T > 0 && (!x_bf16 || !codes || !scale)) return fail(OQ_ERR_INVALID_ARG, "NULL x/codes/scale");
+  if (T > 0 && plan->center && !mean) return fail(OQ_ERR_INVALID_ARG, "centering plan needs mean");
+  if ((x_bf16 && !aligned16(x_bf16)) || (codes && !aligned16(codes)) ||
+      (rotated_f32 && !aligned16(rotated_f32)))
+    return fail(OQ_ERR_MISALIGNED, "x, codes and rotated must be 16-byte aligned");
+  oq_status st = check_plan_device(plan);
+  if (st != OQ_OK) return st;
+  const int mode = plan->act == OQ_ACT_INT8_ABSMAX ? kRqInt8
+                   : plan->act == OQ_ACT_INT4_ABSMAX ? kRqInt4 : kRqLloydMax;
+  return rotate_quantize_impl(plan, x_bf16, T, ldx, codes, scale, plan->center ? mean : nullptr,
+                              rotated_f32, nullptr, mode, plan->center,
+                              static_cast<cudaStream_t>(stream));
+}
+
+oq_status oq_prepare_weights(const oq_plan* plan, const void* w_bf16, int64_t n_out, int64_t ldw,
+                             uint8_t* w_packed, float* w_scale, float* w_rowsum, void* stream) {
+  if (!plan) return fail(OQ_ERR_INVALID_ARG, "NULL plan");
+  if (n_out < 0 || n_out > 0x7FFFFFFF) return fail(OQ_ERR_INVALID_ARG, "n_out out of range");
+  if (ldw < plan->d || (ldw * 2) % 16) return fail(OQ_ERR_MISALIGNED, "ldw must be >= d and a multiple of 8");
+  if (n_out > 0 && (!w_bf16 || !w_packed || !w_scale || !w_rowsum))
+    return fail(OQ_ERR_INVALID_ARG, "NULL weight argument");
+  if ((w_bf16 && !aligned16(w_bf16)) || (w_packed && !aligned16(w_packed)))
+    return fail(OQ_ERR_MISALIGNED, "w and w_packed must be 16-byte aligned");
+  oq_status st = check_plan_device(plan);
+  if (st != OQ_OK) return st;
+  return rotate_quantize_impl(plan, w_bf16, n_out, ldw, w_packed, w_scale, nullptr, nullptr,
+                              w_rowsum, kRqInt4, 0, static_cast<cudaStream_t>(stream));
+}
+
+oq_status oq_gemm_w4a8(const int8_t* a, const float* a_scale, const float* mean,
+                       const uint8_t* w_packed, const float* w_scale, const float* w_rowsum,
+                       const void* bias_bf16, int64_t T, int64_t d_in, int64_t d_out,
+                       oq_out_kind out_kind, void* out, void* stream) {
+  oq_status st = check_gemm_args(a, a_scale, mean, w_packed, w_scale, w_rowsum, bias_bf16, T,
+                                 d_in, d_out, (int)out_kind, out);
+  if (st != OQ_OK) return st;
+  GemmArgs g;
+  g.kind = kGemmA8; g.a = a; g.a_scale = a_scale; g.mean = mean; g.w = w_packed;
+  g.w_scale = w_scale; g.w_rowsum = w_rowsum; g.bias = bias_bf16; g.T = T; g.K = d_in;
+  g.N = d_out; g.out_acc = out_kind == OQ_OUT_ACC; g.out = out;
+  return launch_gemm(g, static_cast<cudaStream_t>(stream));
+}
+
+oq_status oq_gemm_w4a4(const oq_plan* plan, oq_act_kind kind, const uint8_t* a_packed,
+                       const float* a_scale, const float* mean, const uint8_t* w_packed,
+                       const float* w_scale, const float* w_rowsum, const void* bias_bf16,
+                       int64_t T, int64_t d_in, int64_t d_out, oq_out_kind out_kind, void* out,
+                       void* stream) {
+  if (kind != OQ_ACT_INT4_ABSMAX && kind != OQ_ACT_INT4_LLOYDMAX)
+    return fail(OQ_ERR_INVALID_ARG, "oq_gemm_w4a4 takes INT4_ABSMAX or INT4_LLOYDMAX");
+  if (kind == OQ_ACT_INT4_LLOYDMAX && !plan)
+    return fail(OQ_ERR_INVALID_ARG, "Lloyd-Max GEMM needs the plan's codebook");
+  oq_status st = check_gemm_args(a_packed, a_scale, mean, w_packed, w_scale, w_rowsum, bias_bf16,
+                                 T, d_in, d_out, (int)out_kind, out);
+  if (st != OQ_OK) return st;
+  GemmArgs g;
+  g.kind = kind == OQ_ACT_INT4_ABSMAX ? kGemmA4 : kGemmLloydMax;
+  g.a = a_packed; g.a_scale = a_scale; g.mean = mean; g.w = w_packed; g.w_scale = w_scale;
+  g.w_rowsum = w_rowsum; g.bias = bias_bf16; g.T = T; g.K = d_in; g.N = d_out;
+  g.out_acc = out_kind == OQ_OUT_ACC; g.out = out;
+  if (plan)
+    for (int i = 0; i < 16; ++i) g.centroids[i] = (float)plan->cb_c[i];
+  return launch_gemm(g, static_cast<cudaStream_t>(stream));
+}
+
+static size_t round256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+size_t oq_linear_workspace_bytes(const oq_plan* plan, int64_t T) {
+  if (!plan || T < 0) return 0;
+  const size_t code_bytes =
+      plan->act == OQ_ACT_INT8_ABSMAX ? (size_t)T * plan->d : (size_t)T * (plan->d / 2);
+  return round256(code_bytes) + 2 * round256((size_t)T * 4);
+}
+
+oq_status oq_linear(const oq_plan* plan, const void* x_bf16, int64_t T, int64_t ldx,
+                    const uint8_t* w_packed, const float* w_scale, const float* w_rowsum,
+                    const void* bias_bf16, int64_t d_out, void* y_bf16, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+  if (!plan) return fail(OQ_ERR_INVALID_ARG, "NULL plan");
+  if (T < 0) return fail(OQ_ERR_INVALID_ARG, "T out of range");
+  const size_t need = oq_linear_workspace_bytes(plan, T);
+  if (T > 0 && (!workspace || workspace_bytes < need))
+    return fail(OQ_ERR_INVALID_ARG, "workspace too small: need %zu bytes", need);
+  if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return fail(OQ_ERR_MISALIGNED, "workspace must be 256-byte aligned");
+  if (plan->center && !w_rowsum) return fail(OQ_ERR_INVALID_ARG, "centering needs w_rowsum");
+  const size_t code_bytes =
+      plan->act == OQ_ACT_INT8_ABSMAX ? (size_t)T * plan->d : (size_t)T * (plan->d / 2);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  void* codes = ws;
+  float* scale = reinterpret_cast<float*>(ws + round256(code_bytes));
+  float* mean = reinterpret_cast<float*>(ws + round256(code_bytes) + round256((size_t)T * 4));
+  oq_status st = oq_rotate_quantize(plan, x_bf16, T, ldx, codes, scale, mean, nullptr, stream);
+  if (st != OQ_OK) return st;
+  const float* m = plan->center ? mean : nullptr;
+  if (plan->act == OQ_ACT_INT8_ABSMAX)
+    return oq_gemm_w4a8(static_cast<const int8_t*>(codes), scale, m, w_packed, w_scale, w_rowsum,
+                        bias_bf16, T, plan->d, d_out, OQ_OUT_BF16, y_bf16, stream);
+  return oq_gemm_w4a4(plan, plan->act, static_cast<const uint8_t*>(codes), scale, m, w_packed,
+                      w_scale, w_rowsum, bias_bf16, T, plan->d, d_out, OQ_OUT_BF16, y_bf16,
+                      stream);
+}
+
+oq_status oq_debug_wait_timeout(uint64_t timeout_ns, void* stream) {
+  if (timeout_ns == 0 || timeout_ns > 10000000000ull)
+    return fail(OQ_ERR_INVALID_ARG, "timeout_ns must be in (0, 1e10]");
+  unsigned long long* w = device_error_word();
+  if (!w) return fail(OQ_ERR_CUDA, "device error word unavailable");
+  k_debug_wait<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(w, timeout_ns);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "launch debug wait");
+  return OQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,90 @@
+// Internal declarations shared by the host glue and the kernel translation units.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <string>
+#include <vector>
+
+#include <cuda_runtime.h>
+
+#include "../../include/oq.h"
+
+struct oq_plan {
+  int d = 0, h = 0, rounds = 0, center = 0;
+  oq_act_kind act = OQ_ACT_INT8_ABSMAX;
+  uint64_t seed = 0;
+  int device = -1;
+  std::vector<int8_t> signs;    // rounds * d
+  std::vector<int32_t> perm;    // rounds * d
+  uint16_t* d_tab = nullptr;    // device: rounds * d entries, perm | (sign < 0) << 15
+  double cb_c[16] = {}, cb_t[15] = {};
+};
+
+namespace oq {
+
+// ---- host tables -------------------------------------------------------------------------
+uint64_t splitmix64_at(uint64_t key, uint64_t i);
+void rpbh_round_tables(int d, int round, uint64_t seed, int8_t* signs, int32_t* perm);
+void lloyd_max_newton(double c16[16], double t15[15]);
+
+// ---- errors ------------------------------------------------------------------------------
+oq_status fail(oq_status s, const char* fmt, ...);
+oq_status cuda_fail(cudaError_t e, const char* what);
+// Device address of the error word of the current device (set up once per device).
+unsigned long long* device_error_word();
+
+// Device-side wait limit (nanoseconds of %globaltimer) for every bounded wait.
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+
+// Site codes written into the error word (bits 32..47) by a wait that gave up.
+enum : uint32_t {
+  kSiteRqRow = 1,          // rotate-quantize: row load
+  kSiteRqDrain = 2,        // rotate-quantize: drain of a row load after an abort
+  kSiteGemmEmpty = 16,     // GEMM producer: stage free
+  kSiteGemmFull = 17,      // GEMM converter: stage loaded
+  kSiteGemmConv = 18,      // GEMM MMA: stage converted
+  kSiteGemmAccum = 19,     // GEMM epilogue: accumulator ready
+  kSiteGemmDrain = 20,     // GEMM: drain after an abort
+  kSiteDebug = 99          // oq_debug_wait_timeout
+};
+
+// ---- rotate + quantize ---------------------------------------------------------------------
+enum RqMode : int { kRqInt8 = 0, kRqInt4 = 1, kRqLloydMax = 2 };
+
+struct RqArgs {
+  const void* x = nullptr;   // bf16 [T, ldx]
+  int64_t ldx = 0, T = 0;
+  int d = 0, h = 0, rounds = 0, center = 0, mode = 0;
+  const uint16_t* tab = nullptr;  // rounds * d
+  void* codes = nullptr;
+  float* scale = nullptr;
+  float* mean = nullptr;     // written when center (or when rowsum is wanted: see rowsum)
+  float* rotated = nullptr;  // optional [T, d]
+  float* rowsum = nullptr;   // optional [T]: sum of the row before centering/rotation
+  float thr[15] = {};        // Lloyd-Max thresholds (fp32)
+};
+oq_status launch_rotate_quant(const RqArgs& a, cudaStream_t s);
+
+// ---- GEMM ----------------------------------------------------------------------------------
+enum GemmKind : int { kGemmA8 = 0, kGemmA4 = 1, kGemmLloydMax = 2 };
+
+struct GemmArgs {
+  int kind = kGemmA8;
+  const void* a = nullptr;          // int8 [T, K] or uint8 [T, K/2]
+  const float* a_scale = nullptr;
+  const float* mean = nullptr;      // may be null
+  const uint8_t* w = nullptr;       // uint8 [N, K/2]
+  const float* w_scale = nullptr;
+  const float* w_rowsum = nullptr;  // may be null when mean is null
+  const void* bias = nullptr;       // bf16 [N] or null
+  int64_t T = 0, K = 0, N = 0;
+  int out_acc = 0;
+  void* out = nullptr;
+  float centroids[16] = {};
+};
+oq_status launch_gemm(const GemmArgs& g, cudaStream_t s);
+
+oq_status launch_debug_wait(unsigned long long timeout_ns, cudaStream_t s);
+
+}  // namespace oq

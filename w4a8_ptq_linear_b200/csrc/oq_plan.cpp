@@ -1,0 +1,105 @@
+// Host-side plan tables: RPBH signs/permutations and the N(0,1) Lloyd-Max codebook.
+//
+// RPBH (OrbitQuant PR #25 "Default changes"; FLUX.1-schnell-OrbitQuant-W4A4 model card,
+// "Quantization": rotation rpbh, rotation seed 0): the pages give no generator, so the
+// tables follow a fixed, documented rule built on SplitMix64 (Steele, Lea and Flood,
+// OOPSLA 2014) in counter form. The rule is stated in include/oq.h (oq_rpbh_tables).
+//
+// Lloyd-Max (OrbitQuant PR #25: codebook v3 is solved with Newton's method): the 16-level
+// quantizer of N(0,1) satisfies, for every cell k with edges (tau_{k-1}, tau_k),
+//     c_k = E[X | tau_{k-1} < X < tau_k],   tau_k = (c_k + c_{k+1}) / 2.
+// By odd symmetry tau_7 = 0 and only c_8..c_15 are unknown; Newton's method solves the
+// 8 centroid equations with the thresholds eliminated, using the analytic Jacobian.
+#include "oq_internal.h"
+
+#include <algorithm>
+#include <cmath>
+#include <utility>
+#include <vector>
+
+namespace oq {
+
+static inline uint64_t mix64(uint64_t z) {
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+uint64_t splitmix64_at(uint64_t key, uint64_t i) {
+  return mix64(key + (i + 1ull) * 0x9E3779B97F4A7C15ull);
+}
+
+void rpbh_round_tables(int d, int round, uint64_t seed, int8_t* signs, int32_t* perm) {
+  const uint64_t k_sign = splitmix64_at(seed, 2ull * (uint64_t)round);
+  const uint64_t k_perm = splitmix64_at(seed, 2ull * (uint64_t)round + 1ull);
+  std::vector<std::pair<uint64_t, int32_t>> keyed((size_t)d);
+  for (int i = 0; i < d; ++i) {
+    signs[i] = (splitmix64_at(k_sign, (uint64_t)i) >> 63) ? (int8_t)-1 : (int8_t)1;
+    keyed[(size_t)i] = {splitmix64_at(k_perm, (uint64_t)i), i};
+  }
+  std::sort(keyed.begin(), keyed.end());  // by key, then by index
+  for (int i = 0; i < d; ++i) perm[i] = keyed[(size_t)i].second;
+}
+
+// ---- Lloyd-Max ---------------------------------------------------------------------------
+
+static double pdf(double x) { return std::exp(-0.5 * x * x) * 0.39894228040143267794; }
+
+// P(a < X < b) for 0 <= a < b <= inf, from the upper tails (no cancellation).
+static double cell_prob_pos(double a, double b) {
+  const double ta = 0.5 * std::erfc(a * 0.70710678118654752440);
+  const double tb = std::isinf(b) ? 0.0 : 0.5 * std::erfc(b * 0.70710678118654752440);
+  return ta - tb;
+}
+
+void lloyd_max_newton(double c16[16], double t15[15]) {
+  // unknowns c[j] = c_{8+j}, j = 0..7; edges e_j = tau_{7+j}: e_0 = 0, e_j = (c_{j-1}+c_j)/2
+  double c[8];
+  for (int j = 0; j < 8; ++j) c[j] = 0.15 + 0.33 * j;
+  for (int it = 0; it < 100; ++it) {
+    double a[8], b[8], p[8], g[8], F[8];
+    for (int j = 0; j < 8; ++j) {
+      a[j] = (j == 0) ? 0.0 : 0.5 * (c[j - 1] + c[j]);
+      b[j] = (j == 7) ? INFINITY : 0.5 * (c[j] + c[j + 1]);
+      p[j] = cell_prob_pos(a[j], b[j]);
+      const double pb = std::isinf(b[j]) ? 0.0 : pdf(b[j]);
+      g[j] = (pdf(a[j]) - pb) / p[j];
+      F[j] = c[j] - g[j];
+    }
+    // Jacobian: dg/da = pdf(a)(g - a)/P, dg/db = pdf(b)(b - g)/P, da/dc = db/dc = 1/2
+    double J[8][9];
+    for (int j = 0; j < 8; ++j) {
+      for (int k = 0; k < 8; ++k) J[j][k] = (j == k) ? 1.0 : 0.0;
+      const double dga = (j == 0) ? 0.0 : pdf(a[j]) * (g[j] - a[j]) / p[j];
+      const double dgb = (j == 7) ? 0.0 : pdf(b[j]) * (b[j] - g[j]) / p[j];
+      if (j > 0) { J[j][j - 1] -= 0.5 * dga; J[j][j] -= 0.5 * dga; }
+      if (j < 7) { J[j][j] -= 0.5 * dgb; J[j][j + 1] -= 0.5 * dgb; }
+      J[j][8] = -F[j];
+    }
+    // Gaussian elimination with partial pivoting
+    for (int col = 0; col < 8; ++col) {
+      int piv = col;
+      for (int r = col + 1; r < 8; ++r)
+        if (std::fabs(J[r][col]) > std::fabs(J[piv][col])) piv = r;
+      for (int k = 0; k < 9; ++k) std::swap(J[col][k], J[piv][k]);
+      for (int r = col + 1; r < 8; ++r) {
+        const double f = J[r][col] / J[col][col];
+        for (int k = col; k < 9; ++k) J[r][k] -= f * J[col][k];
+      }
+    }
+    double dx[8];
+    for (int r = 7; r >= 0; --r) {
+      double s = J[r][8];
+      for (int k = r + 1; k < 8; ++k) s -= J[r][k] * dx[k];
+      dx[r] = s / J[r][r];
+    }
+    double step = 0.0;
+    for (int j = 0; j < 8; ++j) { c[j] += dx[j]; step = std::fmax(step, std::fabs(dx[j])); }
+    if (step < 1e-15) break;
+  }
+  for (int j = 0; j < 8; ++j) { c16[8 + j] = c[j]; c16[7 - j] = -c[j]; }
+  for (int k = 0; k < 15; ++k) t15[k] = 0.5 * (c16[k] + c16[k + 1]);
+  t15[7] = 0.0;
+}
+
+}  // namespace oq
