@@ -95,6 +95,14 @@ struct GemmParams {
 };
 
 // ---- converters --------------------------------------------------------------------------
+// prmt.b32 in its default mode: selector bit 3 replicates the sign of the chosen byte
+// (CUDA's __byte_perm only honours the low 3 bits of each selector nibble).
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
 // 8 two's-complement nibbles (element 2j low, 2j+1 high in byte j) -> 8 int8.
 __device__ __forceinline__ void nib8_to_i8(uint32_t w, uint32_t& o0, uint32_t& o1) {
   uint32_t lo = (w & 0x0F0F0F0Fu) ^ 0x08080808u;
@@ -132,7 +140,7 @@ __device__ __forceinline__ void lm4_to_f16(uint32_t s, const uint32_t (&lut)[8],
   const uint32_t hi_a = __byte_perm(lut[4], lut[5], s7);
   const uint32_t hi_b = __byte_perm(lut[6], lut[7], s7);
   // byte j of m = 0xFF when bit 3 of code j is set (prmt sign-replicate mode)
-  const uint32_t m = __byte_perm(s << 4, s, 0xD9C8);
+  const uint32_t m = prmt(s << 4, s, 0xD9C8);
   const uint32_t lo = (lo_a & ~m) | (lo_b & m);
   const uint32_t hi = (hi_a & ~m) | (hi_b & m);
   o0 = __byte_perm(lo, hi, 0x5140);
