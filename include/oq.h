@@ -133,9 +133,9 @@ oq_status oq_plan_get_rpbh(const oq_plan* plan, int round, int8_t* signs_host,
 
 /* ---- compute ----------------------------------------------------------------------- */
 
-/* Fused center + RPBH + per-token scale + quantize (CentriQ §4.2 "Activation path",
- * App. B.2 "the prologue ... subtracts its mean, applies ... H ... and quantizes";
- * OrbitQuant PR #25 "Runtime work": the pre-rotation as one kernel).
+/* Fused center + RPBH + per-token scale + quantize (CentriQ §4.2, activation path, and
+ * App. B.2, where one prologue centers each token, rotates it and quantizes it with one scale
+ * per token; OrbitQuant PR #25 "Runtime work": the pre-rotation runs as a single kernel).
  *   x_bf16       [T, ldx] bf16, ldx >= d, (ldx * 2) % 16 == 0
  *   codes        int8 [T, d] (A8) or uint8 [T, d/2] (A4 kinds)
  *   scale        float [T]: alpha_t (absmax kinds) or sigma_t (Lloyd-Max)
@@ -191,6 +191,29 @@ oq_status oq_linear(const oq_plan* plan, const void* x_bf16, int64_t T, int64_t 
                     const uint8_t* w_packed, const float* w_scale, const float* w_rowsum,
                     const void* bias_bf16, int64_t d_out, void* y_bf16, void* workspace,
                     size_t workspace_bytes, void* stream);
+
+/* Size in bytes of the library's static scratch array used by oq_linear_static_scratch. */
+#define OQ_STATIC_SCRATCH_BYTES (16u << 20)
+
+/* Allocation-free oq_linear. The pages have no counterpart: this entry point exists for
+ * callers that cannot allocate device memory, such as plug-ins running inside a framework
+ * that owns all device memory and gives them no allocator, or latency-critical paths that may
+ * not call cudaMalloc (it can synchronise the device). It computes exactly what oq_linear
+ * computes, with the same arguments except the workspace. Its scratch (codes, scales, means)
+ * comes from a 16 MiB array inside the library (OQ_STATIC_SCRATCH_BYTES). Every device that
+ * loads the library holds that array until the process exits. The call allocates nothing.
+ *   - Limit: oq_linear_workspace_bytes(plan, T) must be <= OQ_STATIC_SCRATCH_BYTES, e.g.
+ *     T <= 5447 tokens at d = 3072 with INT8 codes. Larger T returns OQ_ERR_INVALID_ARG
+ *     with a message; split the batch or use oq_linear.
+ *   - Set-up: the first call on a device looks up the array's device address (with that
+ *     device current). Make that first call before any stream capture.
+ *   - Sharing: all calls on a device use the same array and leave their contents in it.
+ *     Calls whose kernels overlap on the GPU (other streams, other host threads) race on it;
+ *     the caller must serialise them. Nothing in the array needs to start at zero. */
+oq_status oq_linear_static_scratch(const oq_plan* plan, const void* x_bf16, int64_t T,
+                                   int64_t ldx, const uint8_t* w_packed, const float* w_scale,
+                                   const float* w_rowsum, const void* bias_bf16, int64_t d_out,
+                                   void* y_bf16, void* stream);
 
 /* Test hook for the bounded waits: launches one block that waits on an mbarrier nothing
  * will arrive on, for at most timeout_ns, then records a timeout and returns. The next

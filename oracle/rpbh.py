@@ -7,7 +7,7 @@ What the pages fix:
   seed 0, block size = the largest power of two dividing the width.
 - CentriQ §3 "Hadamard rotation": H_n H_n^T = n I, so H_n / sqrt(n) is orthogonal and can be
   folded into the weight, W x = (W H^T)(H x); Sylvester matrices exist at every order 2^k.
-  CentriQ §2 describes OrbitQuant's basis as "randomly permuted block-Hadamard".
+  CentriQ §2 describes OrbitQuant's basis as block-Hadamard under a random permutation.
 
 What the pages leave open, and the reading taken here (the library follows the same spec):
 - One round is  z <- (I_{d/h} (x) H_h / sqrt(h)) . D_r . P_r . z,  with the permutation applied

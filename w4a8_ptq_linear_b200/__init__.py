@@ -46,6 +46,7 @@ SIGNATURES = [
     ("oq_linear_workspace_bytes", _SZ, [_P, _I64]),
     ("oq_linear", _I, [_P, _P, _I64, _I64, _P, _P, _P, _P, _I64, _P, _P, _SZ, _P]),
     ("oq_debug_wait_timeout", _I, [_U64, _P]),
+    ("oq_linear_static_scratch", _I, [_P, _P, _I64, _I64, _P, _P, _P, _P, _I64, _P, _P]),
 ]
 
 
@@ -263,6 +264,26 @@ def linear(plan: Plan, x, w_packed, w_scale, w_rowsum=None, bias=None, *, worksp
     _check(lib().oq_linear(plan.handle, _ptr(x), T, x.stride(0), _ptr(w_packed), _ptr(w_scale),
                            _ptr(w_rowsum), _ptr(bias), N, _ptr(out), _ptr(workspace),
                            workspace.numel() * workspace.element_size(), _stream(stream)))
+    return out
+
+
+def linear_static_scratch(plan: Plan, x, w_packed, w_scale, w_rowsum=None, bias=None, *,
+                          out=None, stream=None):
+    """oq_linear_static_scratch: the whole layer without a caller workspace.
+
+    For callers that cannot allocate device scratch (plug-ins inside a framework that owns all
+    device memory, or paths that may not call cudaMalloc). The scratch is a 16 MiB array inside
+    the library, shared by every call on the device; calls that overlap on the GPU race on it.
+    T is limited to what fits that array. Make the first call on a device before any capture.
+    """
+    import torch
+    T = x.shape[0]
+    N = w_packed.shape[0]
+    if out is None:
+        out = torch.empty((T, N), dtype=torch.bfloat16, device=x.device)
+    _check(lib().oq_linear_static_scratch(plan.handle, _ptr(x), T, x.stride(0), _ptr(w_packed),
+                                          _ptr(w_scale), _ptr(w_rowsum), _ptr(bias), N,
+                                          _ptr(out), _stream(stream)))
     return out
 
 
