@@ -43,7 +43,12 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM traffic per launch from an ncu capture, valid only for the kernel source it was taken
 # on (sha256 of the .cu file at capture time); null once the kernel has changed.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    # profiles/k_gemm_dit_w4a8.md: dram read 17.359 MB + write 0.006 MB
+    ("dit_w4a8", "k_gemm"): {"sha": "37195067d55c57cfbe889838ba1f474f2883566e86a789205fadd3e839751ac3", "bytes": 17364224},
+    # profiles/k_rotate_quant_dit_w4a8.md: dram read 25.239 MB + write 0
+    ("dit_w4a8", "k_rotate_quant"): {"sha": "dfa2d41a46719d9468b1d6b86521dcb2c85fd6a0f04fabe5558d3ecb8f91fd48", "bytes": 25239040},
+}
 
 
 def parse():
