@@ -1,22 +1,28 @@
 // Low-bit GEMM with the fused dequant epilogue, tcgen05 on sm_100a (CentriQ §4.2 Eq. 5 and
-// App. B.2 Eq. 9: y_t = W_hat Q_a(R x_t^c) + mean_t w_1 + b, rank-1 term and bias fused into
-// the epilogue; OrbitQuant PR #25: absmax INT8 activations at A8, Lloyd-Max codes below).
+// App. B.2 Eq. 9: y_t = W_hat Q_a(R x_t^c) + mean_t w_1 + b, with the rank-1 term and the bias
+// added in the GEMM epilogue; OrbitQuant PR #25: absmax INT8 activations at A8, Lloyd-Max
+// codes below).
 //
-// Orientation: the CTA computes D[o, t] = sum_k W[o, k] X[t, k] for 128 output channels o
-// (the MMA's M) and BN tokens t (the MMA's N), so the weight operand is the one that is
-// unpacked on chip and the activation tile is shared by all channel tiles through L2.
+// Orientation: a tile is D[o, t] = sum_k W[o, k] X[t, k] for 128 output channels o (the MMA's
+// M) and BN tokens t (the MMA's N). The weight operand is the one unpacked on chip, and the
+// activation tile is shared through L2 by every channel tile of the same token range.
 //
-// Warp roles (192 threads):
-//   warps 0-3  converters: packed INT4 weights (and 4-bit activations) -> INT8 / FP16 in the
-//              128-byte-swizzled K-major layout the tensor core reads; then the epilogue:
-//              TMEM -> registers -> scale, rank-1, bias -> bf16 -> shared -> TMA store.
-//   warp 4     producer: TMA loads of the packed weight tile and the activation tile.
-//   warp 5     TMEM allocator and MMA issuer (one elected thread issues tcgen05.mma).
-// Pipeline per stage s: full[s] (TMA landed) -> conv[s] (operands ready) -> empty[s]
-// (tcgen05.commit after the stage's MMAs). All waits are bounded.
+// Persistent CTAs (one per SM) walk the tiles in channel-fastest order. Warp roles (320 thr):
+//   warp 0     producer: TMA loads of the packed weight tile and of the activation tile into
+//              an S1-deep ring;
+//   warp 1     TMEM owner and MMA issuer (one thread issues tcgen05.mma, 4 per 128-byte K
+//              slice, into one of two TMEM accumulators of BN columns);
+//   warps 2-5  converters: packed INT4 weights (and 4-bit activations) -> INT8 / FP16 in the
+//              128-byte-swizzled K-major layout, into an S2-deep ring of operand tiles;
+//   warps 6-9  epilogue: TMEM -> registers -> alpha_t s_w acc + mean_t w_1 + b -> bf16 ->
+//              shared staging -> TMA store, 32 tokens at a time, double-buffered, while the
+//              MMA already accumulates the next tile into the other TMEM buffer.
+// Barriers: full[s] (TMA landed), xempty[s] (TMA slot free), wready[c] (operands converted),
+// wfree[c] (MMA done with them), tfull[b] / tempty[b] (accumulator handoff). All waits are
+// bounded; a wait that gives up records its site, sets an abort flag and the roles drain.
 //
 // Kinds:
-//   A8       X int8 via TMA, W int4 -> int8; tcgen05.mma.kind::i8, exact int32 in TMEM.
+//   A8       X int8 straight from TMA, W int4 -> int8; tcgen05.mma.kind::i8, exact int32.
 //   A4       X int4 -> int8, W int4 -> int8; kind::i8.
 //   LloydMax X code -> fp16 centroid (register table via prmt), W int4 -> fp16;
 //            kind::f16 with fp32 accumulation.
@@ -34,51 +40,39 @@
 namespace oq {
 namespace {
 
-constexpr int BM = 128;        // output channels per CTA (MMA M)
-constexpr int NCONV = 128;     // converter / epilogue threads
-constexpr int NTHREADS = 192;
-
-template <int KIND> struct KTraits;
-template <> struct KTraits<kGemmA8> {
-  static constexpr int BK = 128;           // K elements per stage (128 bytes of int8)
-  static constexpr bool X_PACKED = false;
-  static constexpr int STAGES = 3;
-};
-template <> struct KTraits<kGemmA4> {
-  static constexpr int BK = 128;
-  static constexpr bool X_PACKED = true;
-  static constexpr int STAGES = 3;
-};
-template <> struct KTraits<kGemmLloydMax> {
-  static constexpr int BK = 64;            // 64 fp16 = 128 bytes
-  static constexpr bool X_PACKED = true;
-  static constexpr int STAGES = 3;
-};
+constexpr int BM = 128;       // output channels per tile (MMA M)
+constexpr int NCONV = 128;    // converter threads (warps 2-5)
+constexpr int NEPI = 128;     // epilogue threads (warps 6-9)
+constexpr int NTHREADS = 320;
+constexpr int EPI_CHUNK = 32; // tokens per epilogue store
 
 template <int KIND, int BN>
-struct Layout {
-  static constexpr int BK = KTraits<KIND>::BK;
-  static constexpr int STAGES = KTraits<KIND>::STAGES;
-  static constexpr int W_TILE = BM * 128;                   // swizzled operand bytes
-  static constexpr int X_TILE = BN * 128;
-  static constexpr int WP_TILE = BM * (BK / 2);             // packed staging bytes
-  static constexpr int XP_TILE = KTraits<KIND>::X_PACKED ? BN * (BK / 2) : 0;
-  static constexpr int STAGE = W_TILE + X_TILE + WP_TILE + XP_TILE;
-  static constexpr int OFF_W = 0;
-  static constexpr int OFF_X = W_TILE;
-  static constexpr int OFF_WP = W_TILE + X_TILE;
-  static constexpr int OFF_XP = OFF_WP + WP_TILE;
-  static constexpr int PIPE = STAGES * STAGE;
-  static constexpr int OUT_BYTES_MAX = BN * BM * 4;          // epilogue staging (aliases PIPE)
-  static constexpr int MAIN = PIPE > OUT_BYTES_MAX ? PIPE : OUT_BYTES_MAX;
-  // small region: per-token scale/mean, barriers, TMEM address, abort flag
-  static constexpr int OFF_TOK = MAIN;
-  static constexpr int OFF_BAR = OFF_TOK + 2 * BN * 4;
-  static constexpr int NBARS = 3 * STAGES + 2;
-  static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
-  static constexpr int TOTAL = OFF_MISC + 16;
-  static constexpr int SMEM = TOTAL + 1024;                  // slack for 1024-B alignment
-  static_assert(STAGE % 1024 == 0, "stage tiles must keep 1024-byte alignment");
+struct Cfg {
+  static constexpr int BK = (KIND == kGemmLloydMax) ? 64 : 128;   // 128 bytes of K per stage
+  static constexpr bool XPACK = KIND != kGemmA8;
+  static constexpr int S1 = 4;                                     // TMA stages
+  static constexpr int S2 = (KIND == kGemmLloydMax) ? 3 : 2;       // converted stages
+  static constexpr int WT = BM * 128;                              // W operand tile
+  static constexpr int XT = BN * 128;                              // X operand tile
+  static constexpr int WP = BM * (BK / 2);                         // packed W per stage
+  static constexpr int XP = BN * (BK / 2);                         // packed X per stage
+  static constexpr int TMA_X = XPACK ? XP : XT;
+  static constexpr int TMA_STAGE = TMA_X + WP;
+  static constexpr int CONV_STAGE = WT + (XPACK ? XT : 0);
+  static constexpr int OFF_TMA = 0;
+  static constexpr int OFF_CONV = S1 * TMA_STAGE;
+  static constexpr int OFF_OUT = OFF_CONV + S2 * CONV_STAGE;
+  static constexpr int OUT_BYTES = 2 * EPI_CHUNK * BM * 2;         // two bf16 chunks or one acc
+  static constexpr int OFF_TOK = OFF_OUT + OUT_BYTES;              // float2 (scale, mean) [BN]
+  static constexpr int OFF_BAR = OFF_TOK + BN * 8;
+  static constexpr int NBAR = 2 * S1 + 2 * S2 + 4 + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM = OFF_MISC + 16 + 1024;                // + slack for alignment
+  static constexpr uint32_t TMA_BYTES = TMA_STAGE;
+  static_assert(TMA_STAGE % 1024 == 0 && CONV_STAGE % 1024 == 0 && TMA_X % 1024 == 0,
+                "operand tiles must stay 1024-byte aligned");
+  static_assert(BN % EPI_CHUNK == 0 && BN % 16 == 0 && BN <= 256, "MMA N");
+  static_assert(SMEM <= 232448, "shared memory");
 };
 
 struct GemmParams {
@@ -147,60 +141,69 @@ __device__ __forceinline__ void lm4_to_f16(uint32_t s, const uint32_t (&lut)[8],
   o1 = __byte_perm(lo, hi, 0x7362);
 }
 
-// Address of 16-byte chunk `c` (0..7) of row `r` in a 128-byte-swizzled K-major tile.
-__device__ __forceinline__ uint8_t* sw128(uint8_t* tile, int r, int c) {
-  return tile + r * 128 + ((c ^ (r & 7)) << 4);
-}
-
-// Packed INT4 rows of 64 bytes (128 elements) -> int8 swizzled rows.
+// Packed INT4 rows of 64 bytes -> int8 rows of 128 bytes in the 128-byte-swizzled layout
+// (16-byte chunk c of row r at r * 128 + ((c ^ (r & 7)) << 4)). Thread ctid takes the
+// 16-byte packed chunk q = ctid & 3 of rows ctid / 4 + 32 j; the swizzle phase r & 7 is the
+// same for all j, so every address is a constant offset from a per-thread base.
 template <int ROWS>
 __device__ __forceinline__ void convert_i4_i8(const uint8_t* src, uint8_t* dst, int ctid) {
-#pragma unroll 4
-  for (int c = ctid; c < ROWS * 4; c += NCONV) {
-    const int r = c >> 2, q = c & 3;
-    const uint4 in = *reinterpret_cast<const uint4*>(src + r * 64 + q * 16);
+  const int r0 = ctid >> 2, q = ctid & 3;
+  const uint8_t* s = src + r0 * 64 + q * 16;
+  uint8_t* da = dst + r0 * 128 + (((2 * q) ^ (r0 & 7)) << 4);
+  uint8_t* db = dst + r0 * 128 + (((2 * q + 1) ^ (r0 & 7)) << 4);
+#pragma unroll
+  for (int j = 0; j < ROWS / 32; ++j) {
+    const uint4 in = *reinterpret_cast<const uint4*>(s + j * 32 * 64);
     uint4 a, b;
     nib8_to_i8(in.x, a.x, a.y);
     nib8_to_i8(in.y, a.z, a.w);
     nib8_to_i8(in.z, b.x, b.y);
     nib8_to_i8(in.w, b.z, b.w);
-    *reinterpret_cast<uint4*>(sw128(dst, r, 2 * q)) = a;
-    *reinterpret_cast<uint4*>(sw128(dst, r, 2 * q + 1)) = b;
+    *reinterpret_cast<uint4*>(da + j * 32 * 128) = a;
+    *reinterpret_cast<uint4*>(db + j * 32 * 128) = b;
   }
 }
 
-// Packed INT4 rows of 32 bytes (64 elements) -> fp16 swizzled rows.
+// Packed INT4 rows of 32 bytes (64 elements) -> fp16 rows of 128 bytes, swizzled.
 template <int ROWS>
 __device__ __forceinline__ void convert_i4_f16(const uint8_t* src, uint8_t* dst, int ctid) {
-#pragma unroll 2
-  for (int c = ctid; c < ROWS * 2; c += NCONV) {
-    const int r = c >> 1, q = c & 1;
-    const uint4 in = *reinterpret_cast<const uint4*>(src + r * 32 + q * 16);
+  const int r0 = ctid >> 1, q = ctid & 1;
+  const uint8_t* s = src + r0 * 32 + q * 16;
+  uint8_t* d = dst + r0 * 128;
+  const int ph = r0 & 7;
+#pragma unroll
+  for (int j = 0; j < ROWS / 64; ++j) {
+    const uint4 in = *reinterpret_cast<const uint4*>(s + j * 64 * 32);
     const uint32_t w[4] = {in.x, in.y, in.z, in.w};
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
+    for (int k = 0; k < 4; ++k) {
       uint32_t o[4];
-      nib8_to_f16(w[j], o);
-      *reinterpret_cast<uint4*>(sw128(dst, r, 4 * q + j)) = make_uint4(o[0], o[1], o[2], o[3]);
+      nib8_to_f16(w[k], o);
+      *reinterpret_cast<uint4*>(d + j * 64 * 128 + (((4 * q + k) ^ ph) << 4)) =
+          make_uint4(o[0], o[1], o[2], o[3]);
     }
   }
 }
 
-// Lloyd-Max code rows of 32 bytes (64 codes) -> fp16 centroid swizzled rows.
+// Lloyd-Max code rows of 32 bytes (64 codes) -> fp16 centroid rows of 128 bytes, swizzled.
 template <int ROWS>
 __device__ __forceinline__ void convert_lm_f16(const uint8_t* src, uint8_t* dst, int ctid,
                                                const uint32_t (&lut)[8]) {
-#pragma unroll 2
-  for (int c = ctid; c < ROWS * 2; c += NCONV) {
-    const int r = c >> 1, q = c & 1;
-    const uint4 in = *reinterpret_cast<const uint4*>(src + r * 32 + q * 16);
+  const int r0 = ctid >> 1, q = ctid & 1;
+  const uint8_t* s = src + r0 * 32 + q * 16;
+  uint8_t* d = dst + r0 * 128;
+  const int ph = r0 & 7;
+#pragma unroll
+  for (int j = 0; j < ROWS / 64; ++j) {
+    const uint4 in = *reinterpret_cast<const uint4*>(s + j * 64 * 32);
     const uint32_t w[4] = {in.x, in.y, in.z, in.w};
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
+    for (int k = 0; k < 4; ++k) {
       uint32_t o0, o1, o2, o3;
-      lm4_to_f16(w[j] & 0xFFFFu, lut, o0, o1);
-      lm4_to_f16(w[j] >> 16, lut, o2, o3);
-      *reinterpret_cast<uint4*>(sw128(dst, r, 4 * q + j)) = make_uint4(o0, o1, o2, o3);
+      lm4_to_f16(w[k] & 0xFFFFu, lut, o0, o1);
+      lm4_to_f16(w[k] >> 16, lut, o2, o3);
+      *reinterpret_cast<uint4*>(d + j * 64 * 128 + (((4 * q + k) ^ ph) << 4)) =
+          make_uint4(o0, o1, o2, o3);
     }
   }
 }
@@ -209,205 +212,265 @@ template <int KIND, int BN>
 __global__ void __launch_bounds__(NTHREADS, 1)
     k_gemm(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
            const __grid_constant__ CUtensorMap tm_y, const GemmParams p) {
-  using L = Layout<KIND, BN>;
-  constexpr int BK = L::BK;
-  constexpr int STAGES = L::STAGES;
+  using C = Cfg<KIND, BN>;
+  constexpr int BK = C::BK, S1 = C::S1, S2 = C::S2;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  float* s_tok_scale = reinterpret_cast<float*>(smem + L::OFF_TOK);
-  float* s_tok_mean = s_tok_scale + BN;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
-  uint32_t* s_misc = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);  // [0] tmem, [1] abort
+  float2* s_tok = reinterpret_cast<float2*>(smem + C::OFF_TOK);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint32_t* s_misc = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);  // tmem, abort, epi flag
   volatile uint32_t* s_abort = s_misc + 1;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int o0 = blockIdx.x * BM;
-  const int t0 = blockIdx.y * BN;
+  const int n_o = (p.N + BM - 1) / BM;
+  const int n_tiles = n_o * ((p.T + BN - 1) / BN);
   const int nkb = (p.K + BK - 1) / BK;
 
-  auto full_bar = [&](int s) { return dev::smem_u32(&bars[s]); };
-  auto conv_bar = [&](int s) { return dev::smem_u32(&bars[STAGES + s]); };
-  auto empty_bar = [&](int s) { return dev::smem_u32(&bars[2 * STAGES + s]); };
-  const uint32_t accum_bar = dev::smem_u32(&bars[3 * STAGES]);
-  const uint32_t drain_bar = dev::smem_u32(&bars[3 * STAGES + 1]);
+  auto bar = [&](int i) { return dev::smem_u32(&bars[i]); };
+  auto full_bar = [&](int s) { return bar(s); };
+  auto xempty_bar = [&](int s) { return bar(S1 + s); };
+  auto wready_bar = [&](int c) { return bar(2 * S1 + c); };
+  auto wfree_bar = [&](int c) { return bar(2 * S1 + S2 + c); };
+  auto tfull_bar = [&](int b) { return bar(2 * S1 + 2 * S2 + b); };
+  auto tempty_bar = [&](int b) { return bar(2 * S1 + 2 * S2 + 2 + b); };
+  const uint32_t drain_bar = bar(2 * S1 + 2 * S2 + 4);
+  auto tma_stage = [&](int s) { return smem + C::OFF_TMA + s * C::TMA_STAGE; };
+  auto conv_stage = [&](int c) { return smem + C::OFF_CONV + c * C::CONV_STAGE; };
 
   if (tid == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < S1; ++s) {
       dev::mbar_init(full_bar(s), 1);
-      dev::mbar_init(conv_bar(s), NCONV);
-      dev::mbar_init(empty_bar(s), 1);
+      dev::mbar_init(xempty_bar(s), C::XPACK ? NCONV : 1);
     }
-    dev::mbar_init(accum_bar, 1);
+    for (int c = 0; c < S2; ++c) {
+      dev::mbar_init(wready_bar(c), NCONV);
+      dev::mbar_init(wfree_bar(c), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      dev::mbar_init(tfull_bar(b), 1);
+      dev::mbar_init(tempty_bar(b), NEPI);
+    }
     dev::mbar_init(drain_bar, 1);
     s_misc[1] = 0;
     dev::fence_mbar_init();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == 0 && lane == 0) {
     dev::prefetch_tmap(&tm_x);
     dev::prefetch_tmap(&tm_w);
     dev::prefetch_tmap(&tm_y);
   }
-  if (warp == 5) {
-    dev::tmem_alloc(dev::smem_u32(&s_misc[0]), BN);
+  if (warp == 1) {
+    dev::tmem_alloc(dev::smem_u32(&s_misc[0]), 2 * BN);
     dev::tmem_relinquish();
-  }
-  // per-token scale and mean of this tile (zero outside [0, T))
-  for (int i = tid; i < BN; i += NTHREADS) {
-    const int t = t0 + i;
-    s_tok_scale[i] = (t < p.T) ? p.a_scale[t] : 0.f;
-    s_tok_mean[i] = (t < p.T && p.mean) ? p.mean[t] : 0.f;
   }
   dev::tc_fence_before();
   __syncthreads();
   dev::tc_fence_after();
   const uint32_t tmem = s_misc[0];
 
-  if (warp == 4) {
+  auto give_up = [&]() { *s_abort = 1; };
+
+  if (warp == 0) {
     // ---------------- producer ----------------
     if (lane == 0) {
-      constexpr uint32_t bytes =
-          (uint32_t)(L::WP_TILE + (KTraits<KIND>::X_PACKED ? L::XP_TILE : L::X_TILE));
-      int kb = 0;
-      for (; kb < nkb; ++kb) {
-        const int s = kb % STAGES;
-        const uint32_t par = ((uint32_t)(kb / STAGES) & 1u) ^ 1u;
-        if (*s_abort) break;
-        if (!dev::mbar_wait(empty_bar(s), par, p.err, kSiteGemmEmpty, p.limit_ns)) {
-          *s_abort = 1;
-          break;
-        }
-        uint8_t* st = smem + s * L::STAGE;
-        dev::mbar_arrive_expect_tx(full_bar(s), bytes);
-        dev::tma_load_2d(dev::smem_u32(st + L::OFF_WP), &tm_w, kb * (BK / 2), o0, full_bar(s));
-        if constexpr (KTraits<KIND>::X_PACKED) {
-          dev::tma_load_2d(dev::smem_u32(st + L::OFF_XP), &tm_x, kb * (BK / 2), t0, full_bar(s));
-        } else {
-          dev::tma_load_2d(dev::smem_u32(st + L::OFF_X), &tm_x, kb * BK, t0, full_bar(s));
+      uint32_t j = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x) {
+        const int o0 = (tile % n_o) * BM, t0 = (tile / n_o) * BN;
+        for (int kb = 0; kb < nkb; ++kb, ++j) {
+          const int s = j % S1;
+          if (*s_abort ||
+              !dev::mbar_wait(xempty_bar(s), ((j / S1) & 1u) ^ 1u, p.err, kSiteGemmEmpty,
+                              p.limit_ns)) {
+            give_up();
+            ok = false;
+            break;
+          }
+          uint8_t* st = tma_stage(s);
+          dev::mbar_arrive_expect_tx(full_bar(s), C::TMA_BYTES);
+          dev::tma_load_2d(dev::smem_u32(st + C::TMA_X), &tm_w, kb * (BK / 2), o0, full_bar(s));
+          dev::tma_load_2d(dev::smem_u32(st), &tm_x, C::XPACK ? kb * (BK / 2) : kb * BK, t0,
+                           full_bar(s));
         }
       }
-      if (*s_abort) {
-        // drain: wait (bounded) for the loads of the last issued stages to land
-        for (int j = std::max(0, kb - STAGES); j < kb; ++j)
-          dev::mbar_wait(full_bar(j % STAGES), (uint32_t)(j / STAGES) & 1u, p.err, kSiteGemmDrain,
-                         p.limit_ns);
+      if (!ok) {  // let the loads already issued land before the block can exit
+        for (uint32_t i = (j >= (uint32_t)S1 ? j - S1 : 0); i < j; ++i)
+          dev::mbar_wait(full_bar(i % S1), (i / S1) & 1u, p.err, kSiteGemmDrain, p.limit_ns);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       constexpr uint32_t idesc =
           (KIND == kGemmLloydMax) ? dev::idesc_f16(BM, BN) : dev::idesc_i8(BM, BN);
-      bool issued_any = false;
-      for (int kb = 0; kb < nkb; ++kb) {
-        const int s = kb % STAGES;
-        if (*s_abort) break;
-        if (!dev::mbar_wait(conv_bar(s), (uint32_t)(kb / STAGES) & 1u, p.err, kSiteGemmConv,
-                            p.limit_ns)) {
-          *s_abort = 1;
+      uint32_t j = 0, it = 0;
+      bool ok = true, issued = false;
+      for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x, ++it) {
+        const int b = it & 1;
+        if (*s_abort || !dev::mbar_wait(tempty_bar(b), ((it >> 1) & 1u) ^ 1u, p.err,
+                                        kSiteGemmAccum, p.limit_ns)) {
+          give_up();
+          ok = false;
           break;
         }
         dev::tc_fence_after();
-        uint8_t* st = smem + s * L::STAGE;
-        const uint32_t aw = dev::smem_u32(st + L::OFF_W);
-        const uint32_t bx = dev::smem_u32(st + L::OFF_X);
+        const uint32_t dt = tmem + (uint32_t)(b * BN);
+        for (int kb = 0; kb < nkb; ++kb, ++j) {
+          const int s = j % S1, c = j % S2;
+          bool w = !*s_abort &&
+                   dev::mbar_wait(wready_bar(c), (j / S2) & 1u, p.err, kSiteGemmConv, p.limit_ns);
+          if (w && !C::XPACK)
+            w = dev::mbar_wait(full_bar(s), (j / S1) & 1u, p.err, kSiteGemmFull, p.limit_ns);
+          if (!w) {
+            give_up();
+            ok = false;
+            break;
+          }
+          dev::tc_fence_after();
+          const uint32_t aw = dev::smem_u32(conv_stage(c));
+          const uint32_t bx = C::XPACK ? dev::smem_u32(conv_stage(c) + C::WT)
+                                       : dev::smem_u32(tma_stage(s));
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t ad = dev::sdesc_sw128(aw + kk * 32);
-          const uint64_t bd = dev::sdesc_sw128(bx + kk * 32);
-          if constexpr (KIND == kGemmLloydMax)
-            dev::mma_f16(tmem, ad, bd, idesc, (kb | kk) != 0);
-          else
-            dev::mma_i8(tmem, ad, bd, idesc, (kb | kk) != 0);
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ad = dev::sdesc_sw128(aw + kk * 32);
+            const uint64_t bd = dev::sdesc_sw128(bx + kk * 32);
+            if constexpr (KIND == kGemmLloydMax)
+              dev::mma_f16(dt, ad, bd, idesc, (kb | kk) != 0);
+            else
+              dev::mma_i8(dt, ad, bd, idesc, (kb | kk) != 0);
+          }
+          issued = true;
+          dev::mma_commit(wfree_bar(c));
+          if (!C::XPACK) dev::mma_commit(xempty_bar(s));
         }
-        issued_any = true;
-        dev::mma_commit(empty_bar(s));
+        if (!ok) break;
+        dev::mma_commit(tfull_bar(b));
       }
-      if (!*s_abort) {
-        dev::mma_commit(accum_bar);
-      } else if (issued_any) {
+      if (!ok && issued) {  // wait for the MMAs in flight before TMEM is freed
         dev::mma_commit(drain_bar);
         dev::mbar_wait(drain_bar, 0, p.err, kSiteGemmDrain, p.limit_ns);
       }
     }
-  } else {
-    // ---------------- converters (warps 0-3) ----------------
-    const int ctid = tid;  // 0..127
+  } else if (warp < 6) {
+    // ---------------- converters ----------------
+    const int ctid = tid - 64;
     uint32_t lut[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) lut[i] = p.lut[i];
-    for (int kb = 0; kb < nkb; ++kb) {
-      const int s = kb % STAGES;
-      if (*s_abort) break;
-      if (!dev::mbar_wait(full_bar(s), (uint32_t)(kb / STAGES) & 1u, p.err, kSiteGemmFull,
-                          p.limit_ns)) {
-        *s_abort = 1;
-        break;
-      }
-      uint8_t* st = smem + s * L::STAGE;
-      if constexpr (KIND == kGemmLloydMax) {
-        convert_i4_f16<BM>(st + L::OFF_WP, st + L::OFF_W, ctid);
-        convert_lm_f16<BN>(st + L::OFF_XP, st + L::OFF_X, ctid, lut);
-      } else {
-        convert_i4_i8<BM>(st + L::OFF_WP, st + L::OFF_W, ctid);
-        if constexpr (KIND == kGemmA4) convert_i4_i8<BN>(st + L::OFF_XP, st + L::OFF_X, ctid);
-      }
-      dev::fence_async_smem();
-      dev::mbar_arrive(conv_bar(s));
-    }
-
-    // ---------------- epilogue ----------------
-    const int q = warp;                 // TMEM lane quarter 0..3
-    const int o_local = q * 32 + lane;  // output channel within the tile
-    const int o = o0 + o_local;
-    bool ok = !*s_abort;
-    if (ok && !dev::mbar_wait(accum_bar, 0, p.err, kSiteGemmAccum, p.limit_ns)) {
-      *s_abort = 1;
-      ok = false;
-    }
-    dev::tc_fence_after();
-    const bool has_o = o < p.N;
-    const float sw = has_o ? p.w_scale[o] : 0.f;
-    const float w1 = (has_o && p.mean) ? p.w_rowsum[o] : 0.f;
-    const float b = (has_o && p.bias) ? __bfloat162float(p.bias[o]) : 0.f;
-    if (ok) {
-      uint8_t* out = smem;  // pipeline stages are idle once the accumulator is complete
-#pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t r[32];
-        dev::tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(c * 32), r);
-        dev::tmem_wait_ld();
-        if (p.out_acc) {
-          uint32_t* o32 = reinterpret_cast<uint32_t*>(out);
-#pragma unroll
-          for (int j = 0; j < 32; ++j) o32[(c * 32 + j) * BM + o_local] = r[j];
+    uint32_t j = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x) {
+      for (int kb = 0; kb < nkb; ++kb, ++j) {
+        const int s = j % S1, c = j % S2;
+        bool w = !*s_abort &&
+                 dev::mbar_wait(full_bar(s), (j / S1) & 1u, p.err, kSiteGemmFull, p.limit_ns);
+        if (w)
+          w = dev::mbar_wait(wfree_bar(c), ((j / S2) & 1u) ^ 1u, p.err, kSiteGemmConv,
+                             p.limit_ns);
+        if (!w) {
+          give_up();
+          ok = false;
+          break;
+        }
+        const uint8_t* st = tma_stage(s);
+        uint8_t* cv = conv_stage(c);
+        if constexpr (KIND == kGemmLloydMax) {
+          convert_i4_f16<BM>(st + C::TMA_X, cv, ctid);
+          convert_lm_f16<BN>(st, cv + C::WT, ctid, lut);
         } else {
-          __nv_bfloat16* ob = reinterpret_cast<__nv_bfloat16*>(out);
+          convert_i4_i8<BM>(st + C::TMA_X, cv, ctid);
+          if constexpr (KIND == kGemmA4) convert_i4_i8<BN>(st, cv + C::WT, ctid);
+        }
+        dev::fence_async_smem();
+        dev::mbar_arrive(wready_bar(c));
+        if (C::XPACK) dev::mbar_arrive(xempty_bar(s));
+      }
+    }
+  } else {
+    // ---------------- epilogue ----------------
+    const int etid = tid - 192;          // 0..127
+    const int q = warp & 3;              // TMEM lane quarter of this warp
+    const int o_local = q * 32 + lane;
+    const bool leader = etid == 0;
+    const int nbuf = p.out_acc ? 1 : 2;
+    const int chunk_bytes = EPI_CHUNK * BM * (p.out_acc ? 4 : 2);
+    uint8_t* stage_out = smem + C::OFF_OUT;
+    uint32_t it = 0, g = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x, ++it) {
+      const int o0 = (tile % n_o) * BM, t0 = (tile / n_o) * BN;
+      const int b = it & 1;
+      const int o = o0 + o_local;
+      const bool has_o = o < p.N;
+      const float sw = has_o ? p.w_scale[o] : 0.f;
+      const float w1 = (has_o && p.mean) ? p.w_rowsum[o] : 0.f;
+      const float bb = (has_o && p.bias) ? __bfloat162float(p.bias[o]) : 0.f;
+      for (int i = etid; i < BN; i += NEPI) {
+        const int t = t0 + i;
+        s_tok[i] = make_float2((t < p.T) ? p.a_scale[t] : 0.f,
+                               (t < p.T && p.mean) ? p.mean[t] : 0.f);
+      }
+      // one thread waits for the accumulator; the verdict reaches all four warps through
+      // shared memory behind a named barrier, so every later barrier is reached uniformly
+      if (leader) {
+        const bool ready = !*s_abort && dev::mbar_wait(tfull_bar(b), (it >> 1) & 1u, p.err,
+                                                       kSiteGemmAccum, p.limit_ns);
+        if (!ready) give_up();
+        s_misc[2] = ready ? 1u : 0u;
+      }
+      dev::named_bar(1, NEPI);
+      ok = *reinterpret_cast<volatile uint32_t*>(&s_misc[2]) != 0;
+      if (ok) dev::tc_fence_after();
+#pragma unroll 1
+      for (int c = 0; ok && c < BN / EPI_CHUNK; ++c, ++g) {
+        uint32_t r[32];
+        dev::tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * BN + c * EPI_CHUNK), r);
+        dev::tmem_wait_ld();
+        if (c == BN / EPI_CHUNK - 1) {  // accumulator fully read: hand it back to the MMA
+          dev::tc_fence_before();
+          dev::mbar_arrive(tempty_bar(b));
+        }
+        const int buf = (int)(g % (uint32_t)nbuf);
+        if (g >= (uint32_t)nbuf) {  // the store that used this buffer must have read it
+          if (leader) {
+            if (nbuf == 2) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+            else dev::bulk_wait_all_read();
+          }
+          dev::named_bar(1, NEPI);
+        }
+        uint8_t* ob = stage_out + buf * chunk_bytes;
+        if (p.out_acc) {
+          uint32_t* o32 = reinterpret_cast<uint32_t*>(ob);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int tl = c * 32 + j;
-            const float acc = (KIND == kGemmLloydMax) ? __uint_as_float(r[j])
-                                                      : (float)(int32_t)r[j];
-            const float y = fmaf(acc, s_tok_scale[tl] * sw, fmaf(s_tok_mean[tl], w1, b));
-            ob[tl * BM + o_local] = __float2bfloat16_rn(y);
+          for (int jj = 0; jj < 32; ++jj) o32[jj * BM + o_local] = r[jj];
+        } else {
+          __nv_bfloat16* o16 = reinterpret_cast<__nv_bfloat16*>(ob);
+#pragma unroll
+          for (int jj = 0; jj < 32; ++jj) {
+            const float2 tk = s_tok[c * EPI_CHUNK + jj];
+            const float acc = (KIND == kGemmLloydMax) ? __uint_as_float(r[jj])
+                                                      : (float)(int32_t)r[jj];
+            o16[jj * BM + o_local] = __float2bfloat16_rn(fmaf(acc, tk.x * sw, fmaf(tk.y, w1, bb)));
           }
         }
+        dev::fence_async_smem();
+        dev::named_bar(1, NEPI);
+        if (leader) {
+          dev::tma_store_2d(&tm_y, dev::smem_u32(ob), o0, t0 + c * EPI_CHUNK);
+          dev::bulk_commit();
+        }
       }
-      dev::fence_async_smem();
-      dev::named_bar(1, NCONV);
-      if (tid == 0) {
-        dev::tma_store_2d(&tm_y, dev::smem_u32(out), o0, t0);
-        dev::bulk_commit();
-        dev::bulk_wait_all_read();
-      }
+      dev::named_bar(1, NEPI);  // s_tok of this tile is no longer read
     }
-    dev::tc_fence_before();
+    if (leader) dev::bulk_wait_all();
   }
 
+  dev::tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 1) {
     dev::tc_fence_after();
-    dev::tmem_dealloc(tmem, BN);
+    dev::tmem_dealloc(tmem, 2 * BN);
   }
 }
 
@@ -445,13 +508,24 @@ bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint6
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+int sm_count() {
+  static int n = 0;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  });
+  return n > 0 ? n : 148;
+}
+
 template <int KIND, int BN>
 oq_status run(const GemmArgs& g, const GemmParams& p, cudaStream_t s) {
-  using L = Layout<KIND, BN>;
-  constexpr int BK = L::BK;
+  using C = Cfg<KIND, BN>;
+  constexpr int BK = C::BK;
   CUtensorMap tx, tw, ty;
   bool ok = true;
-  if constexpr (KTraits<KIND>::X_PACKED)
+  if constexpr (C::XPACK)
     ok &= make_map_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.a, (uint64_t)g.K / 2, (uint64_t)g.T,
                       (uint64_t)g.K / 2, BK / 2, BN, CU_TENSOR_MAP_SWIZZLE_NONE);
   else
@@ -464,17 +538,21 @@ oq_status run(const GemmArgs& g, const GemmParams& p, cudaStream_t s) {
                                          : CU_TENSOR_MAP_DATA_TYPE_INT32)
                 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const uint64_t ysz = g.out_acc ? 4 : 2;
-  ok &= make_map_2d(&ty, ydt, g.out, (uint64_t)g.N, (uint64_t)g.T, (uint64_t)g.N * ysz, BM, BN,
-                    CU_TENSOR_MAP_SWIZZLE_NONE);
+  ok &= make_map_2d(&ty, ydt, g.out, (uint64_t)g.N, (uint64_t)g.T, (uint64_t)g.N * ysz, BM,
+                    EPI_CHUNK, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (!ok) return fail(OQ_ERR_CUDA, "cuTensorMapEncodeTiled failed or unavailable");
 
   auto kern = &k_gemm<KIND, BN>;
-  cudaError_t ce =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
-  if (ce != cudaSuccess) return cuda_fail(ce, "cudaFuncSetAttribute(gemm)");
-  const dim3 grid((unsigned)((g.N + BM - 1) / BM), (unsigned)((g.T + BN - 1) / BN));
-  kern<<<grid, NTHREADS, L::SMEM, s>>>(tx, tw, ty, p);
-  ce = cudaGetLastError();
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [&] {
+    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  });
+  if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute(gemm)");
+  const int64_t tiles = ((g.N + BM - 1) / BM) * ((g.T + BN - 1) / BN);
+  const int grid = (int)std::min<int64_t>(tiles, sm_count());
+  kern<<<grid, NTHREADS, C::SMEM, s>>>(tx, tw, ty, p);
+  cudaError_t ce = cudaGetLastError();
   if (ce != cudaSuccess) return cuda_fail(ce, "launch gemm");
   return OQ_OK;
 }
