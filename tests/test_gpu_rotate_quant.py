@@ -32,6 +32,10 @@ CASES = [
     (9, 30720, 1024, 1, "int8_absmax", False),
     (5, 30720, 64, 2, "int4_lloydmax", True),
     (600, 1920, 64, 2, "int8_absmax", False),
+    (4, 30720, 32, 1, "int4_absmax", True),
+    (3, 30720, 512, 2, "int8_absmax", False),
+    (70, 2048, 256, 1, "int4_lloydmax", True),
+    (20, 1280, 256, 2, "int8_absmax", True),
 ]
 
 

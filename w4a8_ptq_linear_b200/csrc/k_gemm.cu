@@ -509,13 +509,9 @@ bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint6
 }
 
 int sm_count() {
-  static int n = 0;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-  });
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
   return n > 0 ? n : 148;
 }
 
@@ -543,11 +539,7 @@ oq_status run(const GemmArgs& g, const GemmParams& p, cudaStream_t s) {
   if (!ok) return fail(OQ_ERR_CUDA, "cuTensorMapEncodeTiled failed or unavailable");
 
   auto kern = &k_gemm<KIND, BN>;
-  static std::once_flag attr_once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(attr_once, [&] {
-    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-  });
+  const cudaError_t attr_err = allow_max_dynamic_smem(reinterpret_cast<const void*>(kern));
   if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute(gemm)");
   const int64_t tiles = ((g.N + BM - 1) / BM) * ((g.T + BN - 1) / BN);
   const int grid = (int)std::min<int64_t>(tiles, sm_count());

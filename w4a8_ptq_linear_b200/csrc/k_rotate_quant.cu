@@ -1,26 +1,35 @@
 // Fused per-token center + RPBH rotation + scale + quantize (the activation path of CentriQ
 // §4.2 and App. B.2; OrbitQuant PR #25 "Runtime work": the pre-rotation as one kernel).
 //
-// Design (HBM-bound; one token row = d bf16 values):
-//  - Persistent CTAs. Each CTA walks tokens t = blockIdx.x, blockIdx.x + gridDim.x, ...; one
-//    thread streams whole rows into shared memory with 1-D bulk copies (TMA), `nbuf` rows
-//    ahead, each completing on its own mbarrier.
-//  - Thread i owns E consecutive rotated positions [i*E, i*E + E). Its entries of the plan
-//    table (permutation index | sign << 15, one uint16 per position and round) stay in
+// HBM-bound design, one token row (d bf16 values) at a time per CTA:
+//  - Persistent CTAs walk tokens t = blockIdx.x, blockIdx.x + gridDim.x, ...; one thread keeps
+//    whole rows streaming into shared memory with 1-D bulk copies (TMA) nbuf rows ahead.
+//  - Every thread owns 32 rotated positions per round. Its gather entries (source index |
+//    sign << 15, laid out on the host in the order the thread consumes them) stay in
 //    registers for the whole kernel.
-//  - Round r: gather u_k = s_k * z[pi_k] from shared memory, then the Sylvester transform on
-//    blocks of h: log2(E) butterfly stages inside the thread, then log2(h/E) stages across
-//    lanes with shuffles (h <= 32 E, so a block never leaves its warp). The second round
-//    gathers from an fp32 copy of the first round's output in shared memory.
-//  - Centering uses the sum of the gathered values (a permutation keeps the sum), so the
-//    mean costs one block reduction and no extra pass over the row.
-//  - Per-token absmax (or sum of squares for Lloyd-Max) by warp shuffles + one block
-//    reduction, then codes are written as packed int8 / nibbles with vector stores.
+//  - Block transform of size h = 2^L in three shapes:
+//      h <= 32        the thread holds whole blocks: L register butterfly stages;
+//      h = 64, 128    the thread holds 32 consecutive positions: 5 register stages, then
+//                     1-2 stages across lanes by shuffles;
+//      h >= 256       the gather fills a strided arrangement (the thread holds one column a of
+//                     a 32 x (h/32) view of its block), the high bits are transformed in
+//                     registers, one swizzled, bank-conflict-free shared-memory transpose per
+//                     warp brings 32 consecutive positions to each thread, and the low 5 bits
+//                     are transformed in registers.
+//    Butterflies past the first stage run on packed f32x2 adds.
+//  - A second round gathers from an fp32 copy of the first round's output, written in a
+//    swizzled layout whose indices the host folded into the round-2 entries.
+//  - Centering uses the sum of the gathered values (a permutation keeps the sum).
+//  - Per-token absmax (or sum of squares for Lloyd-Max) by shuffles and one block reduction;
+//    codes are rounded with one FMA against 1.5 * 2^23 and packed with byte permutes into
+//    one or two 16-byte stores per thread.
 #include <cuda_bf16.h>
 
 #include <algorithm>
 #include <cmath>
+#include <map>
 #include <mutex>
+#include <tuple>
 
 #include "oq_internal.h"
 #include "ptx.cuh"
@@ -28,11 +37,13 @@
 namespace oq {
 namespace {
 
+constexpr int EP = 32;  // positions per thread
+
 struct RqParams {
-  const __nv_bfloat16* x;
+  const uint16_t* x;   // bf16 bits
   int64_t ldx, T;
-  int d, hlog2, rounds, center, mode, nbuf, want_sum;
-  const uint16_t* tab;
+  int d, hlog2, center, mode, nbuf, want_sum;
+  const uint16_t* tab;   // rounds x d entries in kernel order
   void* codes;
   float* scale;
   float* mean;
@@ -44,29 +55,36 @@ struct RqParams {
   unsigned long long limit_ns;
 };
 
-template <int E>
-__device__ __forceinline__ void fwht_block(float (&v)[E], int lane, int hlog2) {
-  const int h = 1 << hlog2;
+// ---- packed fp32 pairs ------------------------------------------------------------------------
+__device__ __forceinline__ void bfly2(float& a0, float& a1, float& b0, float& b1) {
+  // (a, b) -> (a + b, a - b) on two independent pairs with f32x2 arithmetic
+  unsigned long long ra, rb, rs, rd;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(ra) : "f"(a0), "f"(a1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(rb) : "f"(b0), "f"(b1));
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(rs) : "l"(ra), "l"(rb));
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(rd) : "l"(ra), "l"(rb));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(rs));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(b0), "=f"(b1) : "l"(rd));
+}
+
+// butterfly stages over register-index bits [lo_bit, hi_bit)
+template <int LO, int HI>
+__device__ __forceinline__ void reg_stages(float (&v)[EP]) {
 #pragma unroll
-  for (int len = 1; len < E; len <<= 1) {
-    if (len >= h) break;
+  for (int bit = LO; bit < HI; ++bit) {
+    const int len = 1 << bit;
+    if (len == 1) {
 #pragma unroll
-    for (int i = 0; i < E; ++i) {
-      if (!(i & len)) {
-        const float a = v[i], b = v[i | len];
+      for (int i = 0; i < EP; i += 2) {
+        const float a = v[i], b = v[i + 1];
         v[i] = a + b;
-        v[i | len] = a - b;
+        v[i + 1] = a - b;
       }
-    }
-  }
+    } else {
 #pragma unroll
-  for (int m = 1; m < 32; m <<= 1) {
-    if (m * E >= h) break;
-    const bool upper = (lane & m) != 0;
-#pragma unroll
-    for (int i = 0; i < E; ++i) {
-      const float o = __shfl_xor_sync(0xffffffffu, v[i], m);
-      v[i] = upper ? (o - v[i]) : (v[i] + o);
+      for (int i = 0; i < EP; i += 2) {
+        if (!(i & len)) bfly2(v[i], v[i + 1], v[i | len], v[(i | len) + 1]);
+      }
     }
   }
 }
@@ -82,44 +100,113 @@ __device__ __forceinline__ float warp_max(float x) {
   return x;
 }
 
-__device__ __forceinline__ uint32_t tab_entry(const uint32_t* t, int i) {
-  return (t[i >> 1] >> ((i & 1) * 16)) & 0xFFFFu;
+__device__ __forceinline__ uint32_t entry(const uint32_t (&t)[EP / 2], int i) {
+  return (i & 1) ? (t[i >> 1] >> 16) : (t[i >> 1] & 0xFFFFu);
 }
 
-template <int E, int MAXT>
+__device__ __forceinline__ uint32_t byte_of(float f) { return __float_as_uint(f); }
+
+// Transposed index of (row, col) in a warp's 32 x 32 float tile: 16-byte chunk col/4 is
+// XORed with g(row) = (row & 7) ^ ((row / E2) * (E2 / 4) & 7). Writes of one register by all
+// lanes and 16-byte reads of 8 consecutive rows are both bank-conflict free.
+template <int E2>
+__device__ __forceinline__ int tsw(int row, int col) {
+  const int g = (row & 7) ^ (((row / E2) * (E2 / 4)) & 7);
+  return row * 32 + ((((col >> 2) ^ g) << 2) | (col & 3));
+}
+
+// Block transform of the 32 values a thread holds, for one of the three shapes.
+template <int HMODE>
+__device__ __forceinline__ void block_transform(float (&v)[EP], int hlog2, int lane,
+                                                float* warp_tile) {
+  if constexpr (HMODE == 0) {
+    // h <= 32: every block lies inside the thread
+    switch (hlog2) {
+      case 0: break;
+      case 1: reg_stages<0, 1>(v); break;
+      case 2: reg_stages<0, 2>(v); break;
+      case 3: reg_stages<0, 3>(v); break;
+      case 4: reg_stages<0, 4>(v); break;
+      default: reg_stages<0, 5>(v); break;
+    }
+  } else if constexpr (HMODE == 1) {
+    // h = 64 or 128: 5 stages in registers, then across 2 or 4 lanes
+    reg_stages<0, 5>(v);
+#pragma unroll
+    for (int m = 1; m <= 2; m <<= 1) {
+      if ((32 * m) >= (1 << hlog2)) break;
+      const float sgn = (lane & m) ? -1.f : 1.f;
+#pragma unroll
+      for (int i = 0; i < EP; ++i) {
+        const float o = __shfl_xor_sync(0xffffffffu, v[i], m);
+        v[i] = fmaf(v[i], sgn, o);  // lower lane: v + o; upper lane: o - v
+      }
+    }
+  } else {
+    // h = 256, 512, 1024: high bits in the strided arrangement, transpose, low bits
+    const int E2 = 1 << (hlog2 - 5);
+    auto run = [&](auto e2c) {
+      constexpr int E2c = decltype(e2c)::value;
+      constexpr int LB = (E2c == 8) ? 3 : (E2c == 16) ? 4 : 5;
+      reg_stages<0, LB>(v);
+      const int blk = lane / E2c, kB = lane % E2c;
+#pragma unroll
+      for (int i = 0; i < EP; ++i) {
+        const int ia = i / E2c, ib = i % E2c;
+        warp_tile[tsw<E2c>(blk * E2c + ib, kB + E2c * ia)] = v[i];
+      }
+      __syncwarp();
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        const float4 q = *reinterpret_cast<const float4*>(&warp_tile[tsw<E2c>(lane, 4 * m)]);
+        v[4 * m] = q.x; v[4 * m + 1] = q.y; v[4 * m + 2] = q.z; v[4 * m + 3] = q.w;
+      }
+      __syncwarp();
+      reg_stages<0, 5>(v);
+    };
+    if (E2 == 8) run(std::integral_constant<int, 8>{});
+    else if (E2 == 16) run(std::integral_constant<int, 16>{});
+    else run(std::integral_constant<int, 32>{});
+  }
+}
+
+template <int HMODE, int MAXT, int ROUNDS>
 __global__ void __launch_bounds__(MAXT) k_rotate_quant(const RqParams p) {
-  // The round-2 table stays in registers unless a 1024-thread block would spill it; then it
-  // is read per token from the L1-resident plan table.
-  constexpr bool kT1Regs = (E < 32) || (MAXT <= 256);
+  // Round-2 entries stay in registers unless a 1024-thread block would spill them.
+  constexpr bool kT1Regs = (ROUNDS == 2) && (MAXT <= 256);
   extern __shared__ __align__(1024) uint8_t smem[];
   const int d = p.d;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nwarps = blockDim.x >> 5;
-  const int base = tid * E;
+  const int base = tid * EP;
   const bool active = base < d;
   const uint32_t row_bytes = (uint32_t)d * 2u;
   const uint32_t row_stride = (row_bytes + 127u) & ~127u;
+  // With two rounds and h >= 256 the transpose tiles alias the fp32 round buffer: warp w's
+  // tile is exactly the range of positions warp w writes into that buffer.
+  constexpr bool kAlias = (ROUNDS == 2) && (HMODE == 2);
   uint8_t* rowbuf = smem;
   float* rbuf = reinterpret_cast<float*>(smem + (size_t)p.nbuf * row_stride);
-  float* red = rbuf + (p.rounds == 2 ? d : 0);   // [0,32) sums, [32,64) max / sumsq
+  float* tbuf = kAlias ? rbuf : rbuf + (ROUNDS == 2 ? nwarps * 1024 : 0);
+  float* red = tbuf + (HMODE == 2 ? nwarps * 1024 : 0);  // [0,32) sums, [32,64) statistic
   float* thr = red + 64;
   uint64_t* bars = reinterpret_cast<uint64_t*>(thr + 16);
+  float* warp_tile = tbuf + warp * 1024;
 
-  // plan entries of my positions, two uint16 per register
-  uint32_t t0[E / 2], t1[E / 2];
+  uint32_t t0[EP / 2], t1[EP / 2];
 #pragma unroll
-  for (int i = 0; i < E / 2; ++i) t0[i] = t1[i] = 0u;
+  for (int i = 0; i < EP / 2; ++i) t0[i] = t1[i] = 0u;
   if (active) {
     const uint4* s0 = reinterpret_cast<const uint4*>(p.tab + base);
 #pragma unroll
-    for (int i = 0; i < E / 8; ++i) {
+    for (int i = 0; i < 4; ++i) {
       const uint4 q = __ldg(s0 + i);
       t0[4 * i] = q.x; t0[4 * i + 1] = q.y; t0[4 * i + 2] = q.z; t0[4 * i + 3] = q.w;
     }
-    if (kT1Regs && p.rounds == 2) {
+    if constexpr (kT1Regs) {
       const uint4* s1 = reinterpret_cast<const uint4*>(p.tab + d + base);
 #pragma unroll
-      for (int i = 0; i < E / 8; ++i) {
+      for (int i = 0; i < 4; ++i) {
         const uint4 q = __ldg(s1 + i);
         t1[4 * i] = q.x; t1[4 * i + 1] = q.y; t1[4 * i + 2] = q.z; t1[4 * i + 3] = q.w;
       }
@@ -134,7 +221,6 @@ __global__ void __launch_bounds__(MAXT) k_rotate_quant(const RqParams p) {
 
   const int64_t T = p.T;
   const int64_t G = gridDim.x;
-  // thread 0 keeps the row loads nbuf tokens ahead
   if (tid == 0) {
     for (int b = 0; b < p.nbuf; ++b) {
       const int64_t tt = (int64_t)blockIdx.x + (int64_t)b * G;
@@ -154,18 +240,17 @@ __global__ void __launch_bounds__(MAXT) k_rotate_quant(const RqParams p) {
     const uint32_t parity = (uint32_t)(it / p.nbuf) & 1u;
     int fail = !dev::mbar_wait(dev::smem_u32(&bars[b]), parity, p.err, kSiteRqRow, p.limit_ns);
 
-    // ---- round 1: gather from the bf16 row, apply signs --------------------------------
-    float v[E];
+    // ---- round 1: gather from the bf16 row, apply signs ---------------------------------
+    float v[EP];
     float psum = 0.f;
-    const __nv_bfloat16* row =
-        reinterpret_cast<const __nv_bfloat16*>(rowbuf + (size_t)b * row_stride);
+    const uint16_t* row = reinterpret_cast<const uint16_t*>(rowbuf + (size_t)b * row_stride);
+    const bool take = active && !fail;
 #pragma unroll
-    for (int i = 0; i < E; ++i) {
-      float g = 0.f;
-      const uint32_t e = tab_entry(t0, i);
-      if (active && !fail) g = __bfloat162float(row[e & 0x7FFFu]);
-      psum += g;
-      v[i] = (e & 0x8000u) ? -g : g;
+    for (int i = 0; i < EP; ++i) {
+      const uint32_t e = entry(t0, i);
+      const uint32_t hb = take ? (uint32_t)row[e & 0x7FFFu] : 0u;
+      if (p.want_sum) psum += __uint_as_float(hb << 16);
+      v[i] = __uint_as_float((hb ^ (e & 0x8000u)) << 16);
     }
     if (p.want_sum) {
       psum = warp_sum(psum);
@@ -191,128 +276,114 @@ __global__ void __launch_bounds__(MAXT) k_rotate_quant(const RqParams p) {
       if (p.center) {
         const float mu = s / (float)d;
 #pragma unroll
-        for (int i = 0; i < E; ++i) v[i] -= (tab_entry(t0, i) & 0x8000u) ? -mu : mu;
+        for (int i = 0; i < EP; ++i) v[i] -= (entry(t0, i) & 0x8000u) ? -mu : mu;
         if (tid == 0) p.mean[t] = mu;
       }
       if (tid == 0 && p.rowsum) p.rowsum[t] = s;
     }
-    fwht_block<E>(v, lane, p.hlog2);
+    block_transform<HMODE>(v, p.hlog2, lane, warp_tile);
 
-    // ---- round 2: through an fp32 copy in shared memory --------------------------------
-    if (p.rounds == 2) {
+    // ---- round 2: through a swizzled fp32 copy in shared memory -------------------------
+    if constexpr (ROUNDS == 2) {
       if (active) {
-        float4* dst = reinterpret_cast<float4*>(rbuf + base);
 #pragma unroll
-        for (int i = 0; i < E / 4; ++i)
-          dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        for (int m = 0; m < 8; ++m)
+          *reinterpret_cast<float4*>(&rbuf[base + ((m ^ (tid & 7)) << 2)]) =
+              make_float4(v[4 * m], v[4 * m + 1], v[4 * m + 2], v[4 * m + 3]);
       }
       __syncthreads();
-      if (!kT1Regs && active) {
-        const uint4* s1 = reinterpret_cast<const uint4*>(p.tab + d + base);
+      if constexpr (!kT1Regs) {
+        if (active) {
+          const uint4* s1 = reinterpret_cast<const uint4*>(p.tab + d + base);
 #pragma unroll
-        for (int i = 0; i < E / 8; ++i) {
-          const uint4 q = __ldg(s1 + i);
-          t1[4 * i] = q.x; t1[4 * i + 1] = q.y; t1[4 * i + 2] = q.z; t1[4 * i + 3] = q.w;
+          for (int i = 0; i < 4; ++i) {
+            const uint4 q = __ldg(s1 + i);
+            t1[4 * i] = q.x; t1[4 * i + 1] = q.y; t1[4 * i + 2] = q.z; t1[4 * i + 3] = q.w;
+          }
         }
       }
 #pragma unroll
-      for (int i = 0; i < E; ++i) {
-        const uint32_t e = tab_entry(t1, i);
+      for (int i = 0; i < EP; ++i) {
+        const uint32_t e = entry(t1, i);
         const float g = active ? rbuf[e & 0x7FFFu] : 0.f;
-        v[i] = (e & 0x8000u) ? -g : g;
+        v[i] = __uint_as_float(__float_as_uint(g) ^ ((e & 0x8000u) << 16));
       }
-      fwht_block<E>(v, lane, p.hlog2);
+      if constexpr (kAlias) __syncthreads();  // every warp is done reading the round buffer
+      block_transform<HMODE>(v, p.hlog2, lane, warp_tile);
     }
 
-    // ---- per-token statistic ---------------------------------------------------------------
+    // ---- per-token statistic ------------------------------------------------------------
+    const bool lm = p.mode == kRqLloydMax;
     float stat = 0.f;
 #pragma unroll
-    for (int i = 0; i < E; ++i) {
-      v[i] *= p.inv_norm;
-      stat = (p.mode == kRqLloydMax) ? fmaf(v[i], v[i], stat) : fmaxf(stat, fabsf(v[i]));
-    }
-    stat = (p.mode == kRqLloydMax) ? warp_sum(stat) : warp_max(stat);
+    for (int i = 0; i < EP; ++i) stat = lm ? fmaf(v[i], v[i], stat) : fmaxf(stat, fabsf(v[i]));
+    stat = lm ? warp_sum(stat) : warp_max(stat);
     if (lane == 0) red[32 + warp] = stat;
     __syncthreads();
     stat = 0.f;
-    for (int w = 0; w < nwarps; ++w)
-      stat = (p.mode == kRqLloydMax) ? stat + red[32 + w] : fmaxf(stat, red[32 + w]);
+    for (int w = 0; w < nwarps; ++w) stat = lm ? stat + red[32 + w] : fmaxf(stat, red[32 + w]);
 
+    const float nrm = p.inv_norm;
     if (p.rotated && active) {
       float4* dst = reinterpret_cast<float4*>(p.rotated + t * (int64_t)d + base);
 #pragma unroll
-      for (int i = 0; i < E / 4; ++i)
-        dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+      for (int m = 0; m < 8; ++m)
+        dst[m] = make_float4(v[4 * m] * nrm, v[4 * m + 1] * nrm, v[4 * m + 2] * nrm,
+                             v[4 * m + 3] * nrm);
     }
 
-    // ---- quantize + store ---------------------------------------------------------------------
-    if (p.mode == kRqLloydMax) {
-      const float sigma = fmaxf(sqrtf(stat / (float)d), 1e-10f);
-      const float inv = 1.0f / sigma;
+    // ---- quantize + store --------------------------------------------------------------
+    if (lm) {
+      const float sigma = fmaxf(sqrtf(stat * nrm * nrm / (float)d), 1e-10f);
+      const float mult = nrm / sigma;
       if (tid == 0) p.scale[t] = sigma;
       if (active) {
-        uint32_t packed[E / 8];
+        uint32_t packed[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-        for (int j = 0; j < E / 8; ++j) packed[j] = 0u;
-#pragma unroll
-        for (int i = 0; i < E; ++i) {
-          const float u = v[i] * inv;
+        for (int i = 0; i < EP; ++i) {
+          const float u = v[i] * mult;
           int c = (u > thr[7]) ? 8 : 0;
           c += (u > thr[c + 3]) ? 4 : 0;
           c += (u > thr[c + 1]) ? 2 : 0;
           c += (u > thr[c]) ? 1 : 0;
           packed[i >> 3] |= (uint32_t)c << ((i & 7) * 4);
         }
-        uint8_t* dst = reinterpret_cast<uint8_t*>(p.codes) + t * (int64_t)(d / 2) + base / 2;
-        if constexpr (E == 8) {
-          *reinterpret_cast<uint32_t*>(dst) = packed[0];
-        } else if constexpr (E == 16) {
-          *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
-        } else {
-          *reinterpret_cast<uint4*>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-        }
+        *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(p.codes) + t * (int64_t)(d / 2) +
+                                  base / 2) = make_uint4(packed[0], packed[1], packed[2],
+                                                         packed[3]);
       }
     } else {
       const float qmax = (p.mode == kRqInt8) ? 127.f : 7.f;
-      const float a = fmaxf(stat, 1e-10f);
-      const float r = qmax / a;
+      const float a = fmaxf(stat * nrm, 1e-10f);
+      const float mult = nrm * (qmax / a);
       if (tid == 0) p.scale[t] = a / qmax;
       if (active) {
+        // fma against 1.5 * 2^23 rounds half-to-even to an integer held in the low mantissa
+        // bits; the low byte of each result is the two's-complement code
+        uint32_t w[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint32_t f0 = byte_of(fmaf(v[4 * k], mult, 12582912.f));
+          const uint32_t f1 = byte_of(fmaf(v[4 * k + 1], mult, 12582912.f));
+          const uint32_t f2 = byte_of(fmaf(v[4 * k + 2], mult, 12582912.f));
+          const uint32_t f3 = byte_of(fmaf(v[4 * k + 3], mult, 12582912.f));
+          w[k] = __byte_perm(__byte_perm(f0, f1, 0x0040), __byte_perm(f2, f3, 0x0040), 0x5410);
+        }
         if (p.mode == kRqInt8) {
-          uint32_t packed[E / 4];
-#pragma unroll
-          for (int j = 0; j < E / 4; ++j) packed[j] = 0u;
-#pragma unroll
-          for (int i = 0; i < E; ++i) {
-            const float q = fminf(fmaxf(rintf(v[i] * r), -qmax), qmax);
-            packed[i >> 2] |= ((uint32_t)(int32_t)q & 0xFFu) << ((i & 3) * 8);
-          }
           uint8_t* dst = reinterpret_cast<uint8_t*>(p.codes) + t * (int64_t)d + base;
-          if constexpr (E == 8) {
-            *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
-          } else {
-#pragma unroll
-            for (int j = 0; j < E / 16; ++j)
-              reinterpret_cast<uint4*>(dst)[j] =
-                  make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
-          }
+          reinterpret_cast<uint4*>(dst)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+          reinterpret_cast<uint4*>(dst)[1] = make_uint4(w[4], w[5], w[6], w[7]);
         } else {
-          uint32_t packed[E / 8];
+          uint32_t n[4];
 #pragma unroll
-          for (int j = 0; j < E / 8; ++j) packed[j] = 0u;
-#pragma unroll
-          for (int i = 0; i < E; ++i) {
-            const float q = fminf(fmaxf(rintf(v[i] * r), -qmax), qmax);
-            packed[i >> 3] |= ((uint32_t)(int32_t)q & 0xFu) << ((i & 7) * 4);
+          for (int k = 0; k < 4; ++k) {
+            uint32_t a0 = w[2 * k] & 0x0F0F0F0Fu, a1 = w[2 * k + 1] & 0x0F0F0F0Fu;
+            a0 |= a0 >> 4;   // byte 0: code0 | code1 << 4, byte 2: code2 | code3 << 4
+            a1 |= a1 >> 4;
+            n[k] = __byte_perm(a0, a1, 0x6420);
           }
-          uint8_t* dst = reinterpret_cast<uint8_t*>(p.codes) + t * (int64_t)(d / 2) + base / 2;
-          if constexpr (E == 8) {
-            *reinterpret_cast<uint32_t*>(dst) = packed[0];
-          } else if constexpr (E == 16) {
-            *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
-          } else {
-            *reinterpret_cast<uint4*>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-          }
+          *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(p.codes) + t * (int64_t)(d / 2) +
+                                    base / 2) = make_uint4(n[0], n[1], n[2], n[3]);
         }
       }
     }
@@ -322,68 +393,115 @@ __global__ void __launch_bounds__(MAXT) k_rotate_quant(const RqParams p) {
   // bulk copy lands in shared memory after the block has exited.
   if (aborted && tid == 0) {
     for (int k = 0; k < p.nbuf; ++k) {
-      const int j = it + k;  // iteration whose load may be outstanding
+      const int j = it + k;
       const int64_t tt = (int64_t)blockIdx.x + (int64_t)j * G;
       if (tt >= T) break;
-      const int b = j % p.nbuf;
-      dev::mbar_wait(dev::smem_u32(&bars[b]), (uint32_t)(j / p.nbuf) & 1u, p.err, kSiteRqDrain,
-                     p.limit_ns);
+      dev::mbar_wait(dev::smem_u32(&bars[j % p.nbuf]), (uint32_t)(j / p.nbuf) & 1u, p.err,
+                     kSiteRqDrain, p.limit_ns);
     }
   }
 }
 
-template <int E, int MAXT>
-void* rq_kernel() {
-  return reinterpret_cast<void*>(&k_rotate_quant<E, MAXT>);
+struct LaunchCfg {
+  void* fn = nullptr;
+  int nthr = 0, nbuf = 0, grid_per_sm = 0;
+  size_t smem = 0;
+};
+
+template <int HM, int MAXT, int R>
+void* kern() {
+  return reinterpret_cast<void*>(&k_rotate_quant<HM, MAXT, R>);
+}
+
+void* pick_kernel(int hmode, bool big, int rounds) {
+  if (rounds == 1) {
+    if (hmode == 0) return big ? kern<0, 1024, 1>() : kern<0, 256, 1>();
+    if (hmode == 1) return big ? kern<1, 1024, 1>() : kern<1, 256, 1>();
+    return big ? kern<2, 1024, 1>() : kern<2, 256, 1>();
+  }
+  if (hmode == 0) return big ? kern<0, 1024, 2>() : kern<0, 256, 2>();
+  if (hmode == 1) return big ? kern<1, 1024, 2>() : kern<1, 256, 2>();
+  return big ? kern<2, 1024, 2>() : kern<2, 256, 2>();
 }
 
 }  // namespace
+
+int rq_hmode(int h) { return h <= 32 ? 0 : (h <= 128 ? 1 : 2); }
+
+// Position (within the row) that thread t, register i of the round's gather holds.
+int64_t rq_gather_position(int h, int t, int i) {
+  if (rq_hmode(h) < 2) return (int64_t)t * EP + i;
+  const int E2 = h / 32;
+  const int warp = t / 32, lane = t % 32;
+  const int blk = lane / E2, kB = lane % E2, ia = i / E2, ib = i % E2;
+  return (int64_t)warp * 1024 + (int64_t)blk * h + kB + E2 * ia + 32 * ib;
+}
+
+// Index in the swizzled fp32 round buffer at which rotated position p is stored.
+int rq_round_buffer_index(int p) {
+  const int t = p / EP, m = (p % EP) / 4;
+  return t * EP + (((m ^ (t & 7)) << 2) | (p & 3));
+}
 
 oq_status launch_rotate_quant(const RqArgs& a, cudaStream_t s) {
   if (a.T == 0) return OQ_OK;
   int hlog2 = 0;
   while ((1 << hlog2) < a.h) ++hlog2;
-  int E;
-  if (a.h <= 256 && a.d <= 8192) E = 8;
-  else if (a.h <= 512 && a.d <= 16384) E = 16;
-  else E = 32;
-  const int nthr = ((a.d / E + 31) / 32) * 32;
+  const int hmode = rq_hmode(a.h);
+  const int active = a.d / EP;
+  const int nthr = ((active + 31) / 32) * 32;
+  const bool big = nthr > 256;
 
   int dev_id = 0;
   cudaError_t ce = cudaGetDevice(&dev_id);
   if (ce != cudaSuccess) return cuda_fail(ce, "cudaGetDevice");
-  int nsm = 0, max_smem = 0;
-  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev_id);
-  cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev_id);
 
-  const size_t row_stride = ((size_t)a.d * 2 + 127) & ~(size_t)127;
-  const size_t fixed = (a.rounds == 2 ? (size_t)a.d * 4 : 0) + 64 * 4 + 16 * 4;
-  int nbuf = 3;
-  while (nbuf > 1 && fixed + nbuf * row_stride + nbuf * 8 > (size_t)max_smem / 2) --nbuf;
-  const size_t smem = fixed + nbuf * row_stride + nbuf * 8;
-  if (smem > (size_t)max_smem) return fail(OQ_ERR_UNSUPPORTED, "rotate_quant: d too large");
-
-  void* fn = (E == 8)    ? rq_kernel<8, 1024>()
-             : (E == 16) ? rq_kernel<16, 1024>()
-             : (nthr <= 256) ? rq_kernel<32, 256>() : rq_kernel<32, 1024>();
-  ce = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (ce != cudaSuccess) return cuda_fail(ce, "cudaFuncSetAttribute(rotate_quant)");
-  int occ = 0;
-  ce = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, nthr, smem);
-  if (ce != cudaSuccess) return cuda_fail(ce, "occupancy(rotate_quant)");
-  occ = std::max(occ, 1);
-  const int64_t grid = std::min<int64_t>(a.T, (int64_t)nsm * occ);
+  // launch shape per (device, d, h mode, rounds), computed once
+  static std::mutex mu;
+  static std::map<std::tuple<int, int, int, int>, LaunchCfg> cache;
+  LaunchCfg cfg;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    auto key = std::make_tuple(dev_id, a.d, hmode, a.rounds);
+    auto itc = cache.find(key);
+    if (itc != cache.end()) {
+      cfg = itc->second;
+    } else {
+      int nsm = 0, max_smem = 0;
+      cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev_id);
+      cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev_id);
+      const size_t row_stride = ((size_t)a.d * 2 + 127) & ~(size_t)127;
+      // fp32 round buffer and transpose tiles (one region when both are needed), both sized
+      // in whole warps of 1024 positions
+      const size_t warps_bytes = (size_t)(nthr / 32) * 4096;
+      const size_t fixed = ((a.rounds == 2 || hmode == 2) ? warps_bytes : 0) + 64 * 4 + 16 * 4;
+      int nbuf = 3;
+      while (nbuf > 1 && fixed + nbuf * row_stride + nbuf * 8 > (size_t)max_smem / 3) --nbuf;
+      cfg.smem = fixed + nbuf * row_stride + nbuf * 8;
+      if (cfg.smem > (size_t)max_smem) return fail(OQ_ERR_UNSUPPORTED, "rotate_quant: d too large");
+      cfg.fn = pick_kernel(hmode, big, a.rounds);
+      cfg.nthr = nthr;
+      cfg.nbuf = nbuf;
+      ce = allow_max_dynamic_smem(cfg.fn);
+      if (ce != cudaSuccess) return cuda_fail(ce, "cudaFuncSetAttribute(rotate_quant)");
+      int occ = 0;
+      ce = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, cfg.fn, nthr, cfg.smem);
+      if (ce != cudaSuccess) return cuda_fail(ce, "occupancy(rotate_quant)");
+      cfg.grid_per_sm = std::max(occ, 1) * nsm;
+      cache[key] = cfg;
+    }
+  }
+  const int64_t grid = std::min<int64_t>(a.T, (int64_t)cfg.grid_per_sm);
 
   RqParams p{};
-  p.x = reinterpret_cast<const __nv_bfloat16*>(a.x);
+  p.x = reinterpret_cast<const uint16_t*>(a.x);
   p.ldx = a.ldx;
   p.T = a.T;
   p.d = a.d;
   p.hlog2 = hlog2;
-  p.rounds = a.rounds;
   p.center = a.center;
   p.mode = a.mode;
-  p.nbuf = nbuf;
+  p.nbuf = cfg.nbuf;
   p.want_sum = (a.center || a.rowsum) ? 1 : 0;
   p.tab = a.tab;
   p.codes = a.codes;
@@ -399,7 +517,7 @@ oq_status launch_rotate_quant(const RqArgs& a, cudaStream_t s) {
   p.limit_ns = kWaitLimitNs;
 
   void* args[] = {&p};
-  ce = cudaLaunchKernel(fn, dim3((unsigned)grid), dim3((unsigned)nthr), args, smem, s);
+  ce = cudaLaunchKernel(cfg.fn, dim3((unsigned)grid), dim3((unsigned)cfg.nthr), args, cfg.smem, s);
   if (ce != cudaSuccess) return cuda_fail(ce, "launch rotate_quant");
   return OQ_OK;
 }

@@ -5,6 +5,8 @@
 #include <cstring>
 #include <mutex>
 #include <new>
+#include <utility>
+#include <vector>
 
 #include "oq_internal.h"
 #include "ptx.cuh"
@@ -41,6 +43,23 @@ unsigned long long* device_error_word() {
     ptrs[dev] = static_cast<unsigned long long*>(p);
   }
   return ptrs[dev];
+}
+
+cudaError_t allow_max_dynamic_smem(const void* fn) {
+  static std::mutex mu;
+  static std::vector<std::pair<int, const void*>> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  for (const auto& d : done)
+    if (d.first == dev && d.second == fn) return cudaSuccess;
+  int max_smem = 0;
+  e = cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
+  if (e == cudaSuccess) done.emplace_back(dev, fn);
+  return e;
 }
 
 namespace {
@@ -179,12 +198,23 @@ oq_status oq_plan_create(oq_plan** out, int d, int h, int rounds, uint64_t seed,
   p->seed = seed; p->device = dev;
   p->signs.resize((size_t)rounds * d);
   p->perm.resize((size_t)rounds * d);
+  // Gather entries in the order the rotate-quantize kernel consumes them: thread t, register
+  // i of round r reads rotated position q = rq_gather_position(h, t, i), i.e. source index
+  // perm_r[q] with sign signs_r[q]. Round 1 reads the bf16 row, so the index is the channel;
+  // round 2 reads the fp32 round buffer, so the index is where that buffer keeps position
+  // perm_r[q].
   std::vector<uint16_t> tab((size_t)rounds * d);
-  for (int r = 0; r < rounds; ++r) {
+  for (int r = 0; r < rounds; ++r)
     rpbh_round_tables(d, r, seed, p->signs.data() + (size_t)r * d, p->perm.data() + (size_t)r * d);
-    for (int i = 0; i < d; ++i) {
-      const size_t k = (size_t)r * d + i;
-      tab[k] = (uint16_t)(p->perm[k] | (p->signs[k] < 0 ? 0x8000 : 0));
+  for (int r = 0; r < rounds; ++r) {
+    const int8_t* sg = p->signs.data() + (size_t)r * d;
+    const int32_t* pm = p->perm.data() + (size_t)r * d;
+    for (int t = 0; t < d / 32; ++t) {
+      for (int i = 0; i < 32; ++i) {
+        const int64_t q = rq_gather_position(h, t, i);
+        const int src = (r == 0) ? pm[q] : rq_round_buffer_index(pm[q]);
+        tab[(size_t)r * d + (size_t)t * 32 + i] = (uint16_t)(src | (sg[q] < 0 ? 0x8000 : 0));
+      }
     }
   }
   lloyd_max_newton(p->cb_c, p->cb_t);

@@ -17,7 +17,8 @@ struct oq_plan {
   int device = -1;
   std::vector<int8_t> signs;    // rounds * d
   std::vector<int32_t> perm;    // rounds * d
-  uint16_t* d_tab = nullptr;    // device: rounds * d entries, perm | (sign < 0) << 15
+  uint16_t* d_tab = nullptr;    // device: rounds * d gather entries in kernel order,
+                                // source index | (sign < 0) << 15
   double cb_c[16] = {}, cb_t[15] = {};
 };
 
@@ -27,6 +28,12 @@ namespace oq {
 uint64_t splitmix64_at(uint64_t key, uint64_t i);
 void rpbh_round_tables(int d, int round, uint64_t seed, int8_t* signs, int32_t* perm);
 void lloyd_max_newton(double c16[16], double t15[15]);
+
+// ---- launch helpers ----------------------------------------------------------------------
+// Raises a kernel's dynamic shared-memory ceiling to the device's opt-in maximum, once per
+// (device, kernel). The ceiling is a per-function attribute, so it must not depend on the
+// size of any one launch.
+cudaError_t allow_max_dynamic_smem(const void* fn);
 
 // ---- errors ------------------------------------------------------------------------------
 oq_status fail(oq_status s, const char* fmt, ...);
@@ -65,6 +72,10 @@ struct RqArgs {
   float thr[15] = {};        // Lloyd-Max thresholds (fp32)
 };
 oq_status launch_rotate_quant(const RqArgs& a, cudaStream_t s);
+// Kernel-order gather table helpers: the row position thread t, register i gathers in a
+// round, and where the fp32 round buffer keeps rotated position p.
+int64_t rq_gather_position(int h, int t, int i);
+int rq_round_buffer_index(int p);
 
 // ---- GEMM ----------------------------------------------------------------------------------
 enum GemmKind : int { kGemmA8 = 0, kGemmA4 = 1, kGemmLloydMax = 2 };
