@@ -7,19 +7,24 @@
 // M) and BN tokens t (the MMA's N). The weight operand is the one unpacked on chip, and the
 // activation tile is shared through L2 by every channel tile of the same token range.
 //
-// Persistent CTAs (one per SM) walk the tiles in channel-fastest order. Warp roles (320 thr):
-//   warp 0     producer: TMA loads of the packed weight tile and of the activation tile into
-//              an S1-deep ring;
+// Persistent CTAs (one per SM) walk the tiles in channel-fastest order. Warp roles (352 thr):
+//   warp 0     packed-operand producer: TMA loads of the packed weight tile (and, for 4-bit
+//              activations, the packed activation tile) into an SP-deep ring that the
+//              converters release as soon as they have unpacked it;
 //   warp 1     TMEM owner and MMA issuer (one thread issues tcgen05.mma, 4 per 128-byte K
 //              slice, into one of two TMEM accumulators of BN columns);
-//   warps 2-5  converters: packed INT4 weights (and 4-bit activations) -> INT8 / FP16 in the
+//   warp 2     activation producer (INT8 activations only): TMA loads of the activation tile
+//              into an SX-deep ring that only the MMA releases;
+//   warps 3-6  converters: packed INT4 weights (and 4-bit activations) -> INT8 / FP16 in the
 //              128-byte-swizzled K-major layout, into an S2-deep ring of operand tiles;
-//   warps 6-9  epilogue: TMEM -> registers -> alpha_t s_w acc + mean_t w_1 + b -> bf16 ->
-//              shared staging -> TMA store, 32 tokens at a time, double-buffered, while the
-//              MMA already accumulates the next tile into the other TMEM buffer.
-// Barriers: full[s] (TMA landed), xempty[s] (TMA slot free), wready[c] (operands converted),
-// wfree[c] (MMA done with them), tfull[b] / tempty[b] (accumulator handoff). All waits are
-// bounded; a wait that gives up records its site, sets an abort flag and the roles drain.
+//   warps 7-10 epilogue: TMEM -> registers -> alpha_t s_w acc + mean_t w_1 + b -> bf16 ->
+//              coalesced global stores (each warp writes 32 consecutive channels of a token),
+//              while the MMA already accumulates the next tile into the other TMEM buffer.
+// Keeping the large activation tile out of the conversion path matters: its ring slot is held
+// from the TMA issue to the end of its MMA, so the unpacking must not sit in that interval.
+// Barriers: xfull/xempty (activation ring), pfull/pempty (packed ring), wready/wfree
+// (converted operands), tfull/tempty (accumulators). All waits are bounded; a wait that gives
+// up records its site, sets an abort flag and the roles drain.
 //
 // Kinds:
 //   A8       X int8 straight from TMA, W int4 -> int8; tcgen05.mma.kind::i8, exact int32.
@@ -41,37 +46,36 @@ namespace oq {
 namespace {
 
 constexpr int BM = 128;       // output channels per tile (MMA M)
-constexpr int NCONV = 128;    // converter threads (warps 2-5)
-constexpr int NEPI = 128;     // epilogue threads (warps 6-9)
-constexpr int NTHREADS = 320;
-constexpr int EPI_CHUNK = 32; // tokens per epilogue store
+constexpr int NCONV = 128;    // converter threads (warps 3-6)
+constexpr int CONV0 = 96;     // first converter thread
+constexpr int NEPI = 128;     // epilogue threads (warps 7-10)
+constexpr int EPI0 = CONV0 + NCONV;  // first epilogue thread
+constexpr int NTHREADS = EPI0 + NEPI;
 
 template <int KIND, int BN>
 struct Cfg {
   static constexpr int BK = (KIND == kGemmLloydMax) ? 64 : 128;   // 128 bytes of K per stage
   static constexpr bool XPACK = KIND != kGemmA8;
-  static constexpr int S1 = 4;                                     // TMA stages
-  static constexpr int S2 = (KIND == kGemmLloydMax) ? 3 : 2;       // converted stages
+  static constexpr int SX = XPACK ? 0 : 4;                         // activation ring (A8)
+  static constexpr int SP = 4;                                     // packed ring
+  static constexpr int S2 = (KIND == kGemmA4) ? 2 : 3;             // converted ring
   static constexpr int WT = BM * 128;                              // W operand tile
   static constexpr int XT = BN * 128;                              // X operand tile
   static constexpr int WP = BM * (BK / 2);                         // packed W per stage
-  static constexpr int XP = BN * (BK / 2);                         // packed X per stage
-  static constexpr int TMA_X = XPACK ? XP : XT;
-  static constexpr int TMA_STAGE = TMA_X + WP;
-  static constexpr int CONV_STAGE = WT + (XPACK ? XT : 0);
-  static constexpr int OFF_TMA = 0;
-  static constexpr int OFF_CONV = S1 * TMA_STAGE;
-  static constexpr int OFF_OUT = OFF_CONV + S2 * CONV_STAGE;
-  static constexpr int OUT_BYTES = 2 * EPI_CHUNK * BM * 2;         // two bf16 chunks or one acc
-  static constexpr int OFF_TOK = OFF_OUT + OUT_BYTES;              // float2 (scale, mean) [BN]
+  static constexpr int XP = XPACK ? BN * (BK / 2) : 0;             // packed X per stage
+  static constexpr int P_STAGE = XP + WP;                          // [Xp][Wp]
+  static constexpr int CONV_STAGE = WT + (XPACK ? XT : 0);         // [W][X]
+  static constexpr int OFF_X = 0;
+  static constexpr int OFF_P = OFF_X + SX * XT;
+  static constexpr int OFF_CONV = OFF_P + SP * P_STAGE;
+  static constexpr int OFF_TOK = OFF_CONV + S2 * CONV_STAGE;       // float2 (scale, mean) [BN]
   static constexpr int OFF_BAR = OFF_TOK + BN * 8;
-  static constexpr int NBAR = 2 * S1 + 2 * S2 + 4 + 1;
+  static constexpr int NBAR = 2 * SX + 2 * SP + 2 * S2 + 4 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;                // + slack for alignment
-  static constexpr uint32_t TMA_BYTES = TMA_STAGE;
-  static_assert(TMA_STAGE % 1024 == 0 && CONV_STAGE % 1024 == 0 && TMA_X % 1024 == 0,
-                "operand tiles must stay 1024-byte aligned");
-  static_assert(BN % EPI_CHUNK == 0 && BN % 16 == 0 && BN <= 256, "MMA N");
+  static_assert(XT % 1024 == 0 && P_STAGE % 1024 == 0 && CONV_STAGE % 1024 == 0 &&
+                XP % 1024 == 0, "operand tiles must stay 1024-byte aligned");
+  static_assert(BN % 32 == 0 && BN <= 256, "MMA N");
   static_assert(SMEM <= 232448, "shared memory");
 };
 
@@ -81,6 +85,7 @@ struct GemmParams {
   const float* w_scale;
   const float* w_rowsum;
   const __nv_bfloat16* bias;
+  void* out;
   int T, K, N;
   int out_acc;
   uint32_t lut[8];     // Lloyd-Max: fp16 low bytes (0-3) and high bytes (4-7) of c_0..c_15
@@ -147,39 +152,41 @@ __device__ __forceinline__ void lm4_to_f16(uint32_t s, const uint32_t (&lut)[8],
 // same for all j, so every address is a constant offset from a per-thread base.
 template <int ROWS>
 __device__ __forceinline__ void convert_i4_i8(const uint8_t* src, uint8_t* dst, int ctid) {
+  constexpr int RSTEP = NCONV / 4;   // rows covered by one pass of all converter threads
   const int r0 = ctid >> 2, q = ctid & 3;
   const uint8_t* s = src + r0 * 64 + q * 16;
   uint8_t* da = dst + r0 * 128 + (((2 * q) ^ (r0 & 7)) << 4);
   uint8_t* db = dst + r0 * 128 + (((2 * q + 1) ^ (r0 & 7)) << 4);
 #pragma unroll
-  for (int j = 0; j < ROWS / 32; ++j) {
-    const uint4 in = *reinterpret_cast<const uint4*>(s + j * 32 * 64);
+  for (int j = 0; j < ROWS / RSTEP; ++j) {
+    const uint4 in = *reinterpret_cast<const uint4*>(s + j * RSTEP * 64);
     uint4 a, b;
     nib8_to_i8(in.x, a.x, a.y);
     nib8_to_i8(in.y, a.z, a.w);
     nib8_to_i8(in.z, b.x, b.y);
     nib8_to_i8(in.w, b.z, b.w);
-    *reinterpret_cast<uint4*>(da + j * 32 * 128) = a;
-    *reinterpret_cast<uint4*>(db + j * 32 * 128) = b;
+    *reinterpret_cast<uint4*>(da + j * RSTEP * 128) = a;
+    *reinterpret_cast<uint4*>(db + j * RSTEP * 128) = b;
   }
 }
 
 // Packed INT4 rows of 32 bytes (64 elements) -> fp16 rows of 128 bytes, swizzled.
 template <int ROWS>
 __device__ __forceinline__ void convert_i4_f16(const uint8_t* src, uint8_t* dst, int ctid) {
+  constexpr int RSTEP = NCONV / 2;
   const int r0 = ctid >> 1, q = ctid & 1;
   const uint8_t* s = src + r0 * 32 + q * 16;
   uint8_t* d = dst + r0 * 128;
   const int ph = r0 & 7;
 #pragma unroll
-  for (int j = 0; j < ROWS / 64; ++j) {
-    const uint4 in = *reinterpret_cast<const uint4*>(s + j * 64 * 32);
+  for (int j = 0; j < ROWS / RSTEP; ++j) {
+    const uint4 in = *reinterpret_cast<const uint4*>(s + j * RSTEP * 32);
     const uint32_t w[4] = {in.x, in.y, in.z, in.w};
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       uint32_t o[4];
       nib8_to_f16(w[k], o);
-      *reinterpret_cast<uint4*>(d + j * 64 * 128 + (((4 * q + k) ^ ph) << 4)) =
+      *reinterpret_cast<uint4*>(d + j * RSTEP * 128 + (((4 * q + k) ^ ph) << 4)) =
           make_uint4(o[0], o[1], o[2], o[3]);
     }
   }
@@ -189,31 +196,39 @@ __device__ __forceinline__ void convert_i4_f16(const uint8_t* src, uint8_t* dst,
 template <int ROWS>
 __device__ __forceinline__ void convert_lm_f16(const uint8_t* src, uint8_t* dst, int ctid,
                                                const uint32_t (&lut)[8]) {
+  constexpr int RSTEP = NCONV / 2;
   const int r0 = ctid >> 1, q = ctid & 1;
   const uint8_t* s = src + r0 * 32 + q * 16;
   uint8_t* d = dst + r0 * 128;
   const int ph = r0 & 7;
 #pragma unroll
-  for (int j = 0; j < ROWS / 64; ++j) {
-    const uint4 in = *reinterpret_cast<const uint4*>(s + j * 64 * 32);
+  for (int j = 0; j < ROWS / RSTEP; ++j) {
+    const uint4 in = *reinterpret_cast<const uint4*>(s + j * RSTEP * 32);
     const uint32_t w[4] = {in.x, in.y, in.z, in.w};
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       uint32_t o0, o1, o2, o3;
       lm4_to_f16(w[k] & 0xFFFFu, lut, o0, o1);
       lm4_to_f16(w[k] >> 16, lut, o2, o3);
-      *reinterpret_cast<uint4*>(d + j * 64 * 128 + (((4 * q + k) ^ ph) << 4)) =
+      *reinterpret_cast<uint4*>(d + j * RSTEP * 128 + (((4 * q + k) ^ ph) << 4)) =
           make_uint4(o0, o1, o2, o3);
     }
   }
 }
 
+// First K block of a tile. Tiles that run at the same time and share an activation tile
+// (neighbouring channel tiles) start their K loops at different blocks, so that they do not all
+// request the same L2 lines at the same moment. Integer accumulation is exact in any order.
+__device__ __forceinline__ int k_rotation(int tile, int n_o, int nkb) {
+  return (int)(((unsigned)(tile % n_o) * 7u) % (unsigned)nkb);
+}
+
 template <int KIND, int BN>
 __global__ void __launch_bounds__(NTHREADS, 1)
     k_gemm(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
-           const __grid_constant__ CUtensorMap tm_y, const GemmParams p) {
+           const GemmParams p) {
   using C = Cfg<KIND, BN>;
-  constexpr int BK = C::BK, S1 = C::S1, S2 = C::S2;
+  constexpr int BK = C::BK, SX = C::SX, SP = C::SP, S2 = C::S2;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -228,20 +243,27 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int nkb = (p.K + BK - 1) / BK;
 
   auto bar = [&](int i) { return dev::smem_u32(&bars[i]); };
-  auto full_bar = [&](int s) { return bar(s); };
-  auto xempty_bar = [&](int s) { return bar(S1 + s); };
-  auto wready_bar = [&](int c) { return bar(2 * S1 + c); };
-  auto wfree_bar = [&](int c) { return bar(2 * S1 + S2 + c); };
-  auto tfull_bar = [&](int b) { return bar(2 * S1 + 2 * S2 + b); };
-  auto tempty_bar = [&](int b) { return bar(2 * S1 + 2 * S2 + 2 + b); };
-  const uint32_t drain_bar = bar(2 * S1 + 2 * S2 + 4);
-  auto tma_stage = [&](int s) { return smem + C::OFF_TMA + s * C::TMA_STAGE; };
+  auto xfull_bar = [&](int s) { return bar(s); };
+  auto xempty_bar = [&](int s) { return bar(SX + s); };
+  auto pfull_bar = [&](int s) { return bar(2 * SX + s); };
+  auto pempty_bar = [&](int s) { return bar(2 * SX + SP + s); };
+  auto wready_bar = [&](int c) { return bar(2 * SX + 2 * SP + c); };
+  auto wfree_bar = [&](int c) { return bar(2 * SX + 2 * SP + S2 + c); };
+  auto tfull_bar = [&](int b) { return bar(2 * SX + 2 * SP + 2 * S2 + b); };
+  auto tempty_bar = [&](int b) { return bar(2 * SX + 2 * SP + 2 * S2 + 2 + b); };
+  const uint32_t drain_bar = bar(2 * SX + 2 * SP + 2 * S2 + 4);
+  auto x_stage = [&](int s) { return smem + C::OFF_X + s * C::XT; };
+  auto p_stage = [&](int s) { return smem + C::OFF_P + s * C::P_STAGE; };
   auto conv_stage = [&](int c) { return smem + C::OFF_CONV + c * C::CONV_STAGE; };
 
   if (tid == 0) {
-    for (int s = 0; s < S1; ++s) {
-      dev::mbar_init(full_bar(s), 1);
-      dev::mbar_init(xempty_bar(s), C::XPACK ? NCONV : 1);
+    for (int s = 0; s < SX; ++s) {
+      dev::mbar_init(xfull_bar(s), 1);
+      dev::mbar_init(xempty_bar(s), 1);
+    }
+    for (int s = 0; s < SP; ++s) {
+      dev::mbar_init(pfull_bar(s), 1);
+      dev::mbar_init(pempty_bar(s), NCONV);
     }
     for (int c = 0; c < S2; ++c) {
       dev::mbar_init(wready_bar(c), NCONV);
@@ -258,7 +280,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   if (warp == 0 && lane == 0) {
     dev::prefetch_tmap(&tm_x);
     dev::prefetch_tmap(&tm_w);
-    dev::prefetch_tmap(&tm_y);
   }
   if (warp == 1) {
     dev::tmem_alloc(dev::smem_u32(&s_misc[0]), 2 * BN);
@@ -271,32 +292,44 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
   auto give_up = [&]() { *s_abort = 1; };
 
-  if (warp == 0) {
-    // ---------------- producer ----------------
-    if (lane == 0) {
+  if (warp == 0 || warp == 2) {
+    // ---------------- producers ----------------
+    // warp 0: packed ring (W, and X for 4-bit activations); warp 2: INT8 activation ring
+    const bool packed_role = warp == 0;
+    if (lane == 0 && (packed_role || SX > 0)) {
+      const int ns = packed_role ? SP : SX;
       uint32_t j = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x) {
         const int o0 = (tile % n_o) * BM, t0 = (tile / n_o) * BN;
-        for (int kb = 0; kb < nkb; ++kb, ++j) {
-          const int s = j % S1;
-          if (*s_abort ||
-              !dev::mbar_wait(xempty_bar(s), ((j / S1) & 1u) ^ 1u, p.err, kSiteGemmEmpty,
-                              p.limit_ns)) {
+        const int krot = k_rotation(tile, n_o, nkb);
+        for (int step = 0; step < nkb; ++step, ++j) {
+          const int kb = (step + krot) % nkb;
+          const int s = j % ns;
+          const uint32_t empty_b = packed_role ? pempty_bar(s) : xempty_bar(s);
+          const uint32_t full_b = packed_role ? pfull_bar(s) : xfull_bar(s);
+          if (*s_abort || !dev::mbar_wait(empty_b, ((j / ns) & 1u) ^ 1u, p.err, kSiteGemmEmpty,
+                                          p.limit_ns)) {
             give_up();
             ok = false;
             break;
           }
-          uint8_t* st = tma_stage(s);
-          dev::mbar_arrive_expect_tx(full_bar(s), C::TMA_BYTES);
-          dev::tma_load_2d(dev::smem_u32(st + C::TMA_X), &tm_w, kb * (BK / 2), o0, full_bar(s));
-          dev::tma_load_2d(dev::smem_u32(st), &tm_x, C::XPACK ? kb * (BK / 2) : kb * BK, t0,
-                           full_bar(s));
+          if (packed_role) {
+            uint8_t* st = p_stage(s);
+            dev::mbar_arrive_expect_tx(full_b, (uint32_t)C::P_STAGE);
+            dev::tma_load_2d(dev::smem_u32(st + C::XP), &tm_w, kb * (BK / 2), o0, full_b);
+            if constexpr (C::XPACK)
+              dev::tma_load_2d(dev::smem_u32(st), &tm_x, kb * (BK / 2), t0, full_b);
+          } else {
+            dev::mbar_arrive_expect_tx(full_b, (uint32_t)C::XT);
+            dev::tma_load_2d(dev::smem_u32(x_stage(s)), &tm_x, kb * BK, t0, full_b);
+          }
         }
       }
       if (!ok) {  // let the loads already issued land before the block can exit
-        for (uint32_t i = (j >= (uint32_t)S1 ? j - S1 : 0); i < j; ++i)
-          dev::mbar_wait(full_bar(i % S1), (i / S1) & 1u, p.err, kSiteGemmDrain, p.limit_ns);
+        for (uint32_t i = (j >= (uint32_t)ns ? j - ns : 0); i < j; ++i)
+          dev::mbar_wait(packed_role ? pfull_bar(i % ns) : xfull_bar(i % ns), (i / ns) & 1u, p.err,
+                         kSiteGemmDrain, p.limit_ns);
       }
     }
   } else if (warp == 1) {
@@ -316,12 +349,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         dev::tc_fence_after();
         const uint32_t dt = tmem + (uint32_t)(b * BN);
-        for (int kb = 0; kb < nkb; ++kb, ++j) {
-          const int s = j % S1, c = j % S2;
+        for (int step = 0; step < nkb; ++step, ++j) {
+          const int c = j % S2;
+          const int sx = SX > 0 ? (int)(j % (uint32_t)(SX > 0 ? SX : 1)) : 0;
           bool w = !*s_abort &&
                    dev::mbar_wait(wready_bar(c), (j / S2) & 1u, p.err, kSiteGemmConv, p.limit_ns);
-          if (w && !C::XPACK)
-            w = dev::mbar_wait(full_bar(s), (j / S1) & 1u, p.err, kSiteGemmFull, p.limit_ns);
+          if constexpr (!C::XPACK) {
+            if (w)
+              w = dev::mbar_wait(xfull_bar(sx), (j / SX) & 1u, p.err, kSiteGemmFull, p.limit_ns);
+          }
           if (!w) {
             give_up();
             ok = false;
@@ -330,19 +366,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           dev::tc_fence_after();
           const uint32_t aw = dev::smem_u32(conv_stage(c));
           const uint32_t bx = C::XPACK ? dev::smem_u32(conv_stage(c) + C::WT)
-                                       : dev::smem_u32(tma_stage(s));
+                                       : dev::smem_u32(x_stage(sx));
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint64_t ad = dev::sdesc_sw128(aw + kk * 32);
             const uint64_t bd = dev::sdesc_sw128(bx + kk * 32);
             if constexpr (KIND == kGemmLloydMax)
-              dev::mma_f16(dt, ad, bd, idesc, (kb | kk) != 0);
+              dev::mma_f16(dt, ad, bd, idesc, (step | kk) != 0);
             else
-              dev::mma_i8(dt, ad, bd, idesc, (kb | kk) != 0);
+              dev::mma_i8(dt, ad, bd, idesc, (step | kk) != 0);
           }
           issued = true;
           dev::mma_commit(wfree_bar(c));
-          if (!C::XPACK) dev::mma_commit(xempty_bar(s));
+          if constexpr (!C::XPACK) dev::mma_commit(xempty_bar(sx));
         }
         if (!ok) break;
         dev::mma_commit(tfull_bar(b));
@@ -352,19 +388,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         dev::mbar_wait(drain_bar, 0, p.err, kSiteGemmDrain, p.limit_ns);
       }
     }
-  } else if (warp < 6) {
+  } else if (tid < EPI0) {
     // ---------------- converters ----------------
-    const int ctid = tid - 64;
+    const int ctid = tid - CONV0;
     uint32_t lut[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) lut[i] = p.lut[i];
     uint32_t j = 0;
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x) {
-      for (int kb = 0; kb < nkb; ++kb, ++j) {
-        const int s = j % S1, c = j % S2;
+      for (int step = 0; step < nkb; ++step, ++j) {
+        const int s = j % SP, c = j % S2;
         bool w = !*s_abort &&
-                 dev::mbar_wait(full_bar(s), (j / S1) & 1u, p.err, kSiteGemmFull, p.limit_ns);
+                 dev::mbar_wait(pfull_bar(s), (j / SP) & 1u, p.err, kSiteGemmFull, p.limit_ns);
         if (w)
           w = dev::mbar_wait(wfree_bar(c), ((j / S2) & 1u) ^ 1u, p.err, kSiteGemmConv,
                              p.limit_ns);
@@ -373,30 +409,30 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           ok = false;
           break;
         }
-        const uint8_t* st = tma_stage(s);
+        const uint8_t* st = p_stage(s);
         uint8_t* cv = conv_stage(c);
         if constexpr (KIND == kGemmLloydMax) {
-          convert_i4_f16<BM>(st + C::TMA_X, cv, ctid);
+          convert_i4_f16<BM>(st + C::XP, cv, ctid);
           convert_lm_f16<BN>(st, cv + C::WT, ctid, lut);
         } else {
-          convert_i4_i8<BM>(st + C::TMA_X, cv, ctid);
+          convert_i4_i8<BM>(st + C::XP, cv, ctid);
           if constexpr (KIND == kGemmA4) convert_i4_i8<BN>(st, cv + C::WT, ctid);
         }
         dev::fence_async_smem();
         dev::mbar_arrive(wready_bar(c));
-        if (C::XPACK) dev::mbar_arrive(xempty_bar(s));
+        dev::mbar_arrive(pempty_bar(s));
       }
     }
   } else {
     // ---------------- epilogue ----------------
-    const int etid = tid - 192;          // 0..127
+    // Thread (lane quarter q, lane) owns output channel o; a 32-column TMEM load gives it 32
+    // consecutive tokens of that channel. For each token the 32 lanes of a warp store 32
+    // consecutive channels, i.e. 64 (bf16) or 128 (raw accumulator) contiguous bytes.
+    const int etid = tid - EPI0;         // 0..127
     const int q = warp & 3;              // TMEM lane quarter of this warp
     const int o_local = q * 32 + lane;
     const bool leader = etid == 0;
-    const int nbuf = p.out_acc ? 1 : 2;
-    const int chunk_bytes = EPI_CHUNK * BM * (p.out_acc ? 4 : 2);
-    uint8_t* stage_out = smem + C::OFF_OUT;
-    uint32_t it = 0, g = 0;
+    uint32_t it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x, ++it) {
       const int o0 = (tile % n_o) * BM, t0 = (tile / n_o) * BN;
@@ -422,48 +458,38 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       dev::named_bar(1, NEPI);
       ok = *reinterpret_cast<volatile uint32_t*>(&s_misc[2]) != 0;
       if (ok) dev::tc_fence_after();
+      const int t_end = min(BN, p.T - t0);   // tokens of this tile inside [0, T)
 #pragma unroll 1
-      for (int c = 0; ok && c < BN / EPI_CHUNK; ++c, ++g) {
+      for (int c = 0; ok && c < BN / 32; ++c) {
         uint32_t r[32];
-        dev::tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * BN + c * EPI_CHUNK), r);
+        dev::tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * BN + c * 32), r);
         dev::tmem_wait_ld();
-        if (c == BN / EPI_CHUNK - 1) {  // accumulator fully read: hand it back to the MMA
+        if (c == BN / 32 - 1) {  // accumulator fully read: hand it back to the MMA
           dev::tc_fence_before();
           dev::mbar_arrive(tempty_bar(b));
         }
-        const int buf = (int)(g % (uint32_t)nbuf);
-        if (g >= (uint32_t)nbuf) {  // the store that used this buffer must have read it
-          if (leader) {
-            if (nbuf == 2) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-            else dev::bulk_wait_all_read();
-          }
-          dev::named_bar(1, NEPI);
-        }
-        uint8_t* ob = stage_out + buf * chunk_bytes;
+        if (!has_o) continue;
         if (p.out_acc) {
-          uint32_t* o32 = reinterpret_cast<uint32_t*>(ob);
+          uint32_t* dst = reinterpret_cast<uint32_t*>(p.out) + (int64_t)(t0 + c * 32) * p.N + o;
 #pragma unroll
-          for (int jj = 0; jj < 32; ++jj) o32[jj * BM + o_local] = r[jj];
+          for (int jj = 0; jj < 32; ++jj)
+            if (c * 32 + jj < t_end) dst[(int64_t)jj * p.N] = r[jj];
         } else {
-          __nv_bfloat16* o16 = reinterpret_cast<__nv_bfloat16*>(ob);
+          __nv_bfloat16* dst =
+              reinterpret_cast<__nv_bfloat16*>(p.out) + (int64_t)(t0 + c * 32) * p.N + o;
 #pragma unroll
           for (int jj = 0; jj < 32; ++jj) {
-            const float2 tk = s_tok[c * EPI_CHUNK + jj];
+            const float2 tk = s_tok[c * 32 + jj];
             const float acc = (KIND == kGemmLloydMax) ? __uint_as_float(r[jj])
                                                       : (float)(int32_t)r[jj];
-            o16[jj * BM + o_local] = __float2bfloat16_rn(fmaf(acc, tk.x * sw, fmaf(tk.y, w1, bb)));
+            if (c * 32 + jj < t_end)
+              dst[(int64_t)jj * p.N] =
+                  __float2bfloat16_rn(fmaf(acc, tk.x * sw, fmaf(tk.y, w1, bb)));
           }
-        }
-        dev::fence_async_smem();
-        dev::named_bar(1, NEPI);
-        if (leader) {
-          dev::tma_store_2d(&tm_y, dev::smem_u32(ob), o0, t0 + c * EPI_CHUNK);
-          dev::bulk_commit();
         }
       }
       dev::named_bar(1, NEPI);  // s_tok of this tile is no longer read
     }
-    if (leader) dev::bulk_wait_all();
   }
 
   dev::tc_fence_before();
@@ -519,7 +545,7 @@ template <int KIND, int BN>
 oq_status run(const GemmArgs& g, const GemmParams& p, cudaStream_t s) {
   using C = Cfg<KIND, BN>;
   constexpr int BK = C::BK;
-  CUtensorMap tx, tw, ty;
+  CUtensorMap tx, tw;
   bool ok = true;
   if constexpr (C::XPACK)
     ok &= make_map_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.a, (uint64_t)g.K / 2, (uint64_t)g.T,
@@ -529,13 +555,6 @@ oq_status run(const GemmArgs& g, const GemmParams& p, cudaStream_t s) {
                       (uint64_t)g.K, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B);
   ok &= make_map_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.w, (uint64_t)g.K / 2, (uint64_t)g.N,
                     (uint64_t)g.K / 2, BK / 2, BM, CU_TENSOR_MAP_SWIZZLE_NONE);
-  const CUtensorMapDataType ydt =
-      g.out_acc ? (KIND == kGemmLloydMax ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
-                                         : CU_TENSOR_MAP_DATA_TYPE_INT32)
-                : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  const uint64_t ysz = g.out_acc ? 4 : 2;
-  ok &= make_map_2d(&ty, ydt, g.out, (uint64_t)g.N, (uint64_t)g.T, (uint64_t)g.N * ysz, BM,
-                    EPI_CHUNK, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (!ok) return fail(OQ_ERR_CUDA, "cuTensorMapEncodeTiled failed or unavailable");
 
   auto kern = &k_gemm<KIND, BN>;
@@ -543,7 +562,7 @@ oq_status run(const GemmArgs& g, const GemmParams& p, cudaStream_t s) {
   if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute(gemm)");
   const int64_t tiles = ((g.N + BM - 1) / BM) * ((g.T + BN - 1) / BN);
   const int grid = (int)std::min<int64_t>(tiles, sm_count());
-  kern<<<grid, NTHREADS, C::SMEM, s>>>(tx, tw, ty, p);
+  kern<<<grid, NTHREADS, C::SMEM, s>>>(tx, tw, p);
   cudaError_t ce = cudaGetLastError();
   if (ce != cudaSuccess) return cuda_fail(ce, "launch gemm");
   return OQ_OK;
@@ -568,6 +587,7 @@ oq_status launch_gemm(const GemmArgs& g, cudaStream_t s) {
   p.K = (int)g.K;
   p.N = (int)g.N;
   p.out_acc = g.out_acc;
+  p.out = g.out;
   if (g.kind == kGemmLloydMax) {
     uint8_t lo[16], hi[16];
     for (int i = 0; i < 16; ++i) {

@@ -55,38 +55,44 @@ struct RqParams {
   unsigned long long limit_ns;
 };
 
-// ---- packed fp32 pairs ------------------------------------------------------------------------
-__device__ __forceinline__ void bfly2(float& a0, float& a1, float& b0, float& b1) {
-  // (a, b) -> (a + b, a - b) on two independent pairs with f32x2 arithmetic
-  unsigned long long ra, rb, rs, rd;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(ra) : "f"(a0), "f"(a1));
-  asm("mov.b64 %0, {%1, %2};" : "=l"(rb) : "f"(b0), "f"(b1));
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(rs) : "l"(ra), "l"(rb));
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(rd) : "l"(ra), "l"(rb));
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(rs));
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(b0), "=f"(b1) : "l"(rd));
-}
-
-// butterfly stages over register-index bits [lo_bit, hi_bit)
-template <int LO, int HI>
-__device__ __forceinline__ void reg_stages(float (&v)[EP]) {
+// ---- butterflies ------------------------------------------------------------------------------
+// A thread's 32 values live in float2 v[16] (v[k] = elements 2k, 2k+1) so that butterflies
+// whose partners sit in different pairs run as packed f32x2 operations.
+// Stage over element-index bit `bit`: (a, b) -> (a + b, a - b).
+template <int BIT>
+__device__ __forceinline__ void stage(float2 (&v)[EP / 2]) {
+  if constexpr (BIT == 0) {
 #pragma unroll
-  for (int bit = LO; bit < HI; ++bit) {
-    const int len = 1 << bit;
-    if (len == 1) {
+    for (int k = 0; k < EP / 2; ++k) {
+      const float a = v[k].x, b = v[k].y;
+      v[k] = make_float2(a + b, a - b);
+    }
+  } else {
+    constexpr int L = 1 << (BIT - 1);  // partner distance in pairs
+    const float2 m1 = make_float2(-1.f, -1.f);
 #pragma unroll
-      for (int i = 0; i < EP; i += 2) {
-        const float a = v[i], b = v[i + 1];
-        v[i] = a + b;
-        v[i + 1] = a - b;
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < EP; i += 2) {
-        if (!(i & len)) bfly2(v[i], v[i + 1], v[i | len], v[(i | len) + 1]);
+    for (int k = 0; k < EP / 2; ++k) {
+      if (!(k & L)) {
+        const float2 a = v[k], b = v[k | L];
+        v[k] = __fadd2_rn(a, b);
+        v[k | L] = __ffma2_rn(b, m1, a);
       }
     }
   }
+}
+
+// butterfly stages over element-index bits [0, HI)
+template <int HI>
+__device__ __forceinline__ void reg_stages(float2 (&v)[EP / 2]) {
+  if constexpr (HI > 0) stage<0>(v);
+  if constexpr (HI > 1) stage<1>(v);
+  if constexpr (HI > 2) stage<2>(v);
+  if constexpr (HI > 3) stage<3>(v);
+  if constexpr (HI > 4) stage<4>(v);
+}
+
+__device__ __forceinline__ float& el(float2 (&v)[EP / 2], int i) {
+  return (i & 1) ? v[i >> 1].y : v[i >> 1].x;
 }
 
 __device__ __forceinline__ float warp_sum(float x) {
@@ -106,40 +112,33 @@ __device__ __forceinline__ uint32_t entry(const uint32_t (&t)[EP / 2], int i) {
 
 __device__ __forceinline__ uint32_t byte_of(float f) { return __float_as_uint(f); }
 
-// Transposed index of (row, col) in a warp's 32 x 32 float tile: 16-byte chunk col/4 is
-// XORed with g(row) = (row & 7) ^ ((row / E2) * (E2 / 4) & 7). Writes of one register by all
-// lanes and 16-byte reads of 8 consecutive rows are both bank-conflict free.
-template <int E2>
-__device__ __forceinline__ int tsw(int row, int col) {
-  const int g = (row & 7) ^ (((row / E2) * (E2 / 4)) & 7);
-  return row * 32 + ((((col >> 2) ^ g) << 2) | (col & 3));
-}
-
 // Block transform of the 32 values a thread holds, for one of the three shapes.
 template <int HMODE>
-__device__ __forceinline__ void block_transform(float (&v)[EP], int hlog2, int lane,
+__device__ __forceinline__ void block_transform(float2 (&v)[EP / 2], int hlog2, int lane,
                                                 float* warp_tile) {
   if constexpr (HMODE == 0) {
     // h <= 32: every block lies inside the thread
     switch (hlog2) {
       case 0: break;
-      case 1: reg_stages<0, 1>(v); break;
-      case 2: reg_stages<0, 2>(v); break;
-      case 3: reg_stages<0, 3>(v); break;
-      case 4: reg_stages<0, 4>(v); break;
-      default: reg_stages<0, 5>(v); break;
+      case 1: reg_stages<1>(v); break;
+      case 2: reg_stages<2>(v); break;
+      case 3: reg_stages<3>(v); break;
+      case 4: reg_stages<4>(v); break;
+      default: reg_stages<5>(v); break;
     }
   } else if constexpr (HMODE == 1) {
     // h = 64 or 128: 5 stages in registers, then across 2 or 4 lanes
-    reg_stages<0, 5>(v);
+    reg_stages<5>(v);
 #pragma unroll
     for (int m = 1; m <= 2; m <<= 1) {
       if ((32 * m) >= (1 << hlog2)) break;
-      const float sgn = (lane & m) ? -1.f : 1.f;
+      const float sg = (lane & m) ? -1.f : 1.f;
+      const float2 sgn = make_float2(sg, sg);
 #pragma unroll
-      for (int i = 0; i < EP; ++i) {
-        const float o = __shfl_xor_sync(0xffffffffu, v[i], m);
-        v[i] = fmaf(v[i], sgn, o);  // lower lane: v + o; upper lane: o - v
+      for (int k = 0; k < EP / 2; ++k) {
+        const float2 o = make_float2(__shfl_xor_sync(0xffffffffu, v[k].x, m),
+                                     __shfl_xor_sync(0xffffffffu, v[k].y, m));
+        v[k] = __ffma2_rn(v[k], sgn, o);  // lower lane: v + o; upper lane: o - v
       }
     }
   } else {
@@ -148,21 +147,34 @@ __device__ __forceinline__ void block_transform(float (&v)[EP], int hlog2, int l
     auto run = [&](auto e2c) {
       constexpr int E2c = decltype(e2c)::value;
       constexpr int LB = (E2c == 8) ? 3 : (E2c == 16) ? 4 : 5;
-      reg_stages<0, LB>(v);
+      reg_stages<LB>(v);
+      // Element i of lane (blk, kB) goes to row blk*E2 + ib, column kB + E2*ia of the tile,
+      // stored at chunk (col/4) ^ g(row). With E2 >= 8 the chunk splits into a per-thread
+      // part (kB/4 ^ G(blk)) and a per-register part ((E2/4)*ia ^ (ib & 7)), so every
+      // address is a per-thread base plus one of 8 precomputed offsets and a constant.
       const int blk = lane / E2c, kB = lane % E2c;
+      const int R = (kB >> 2) ^ ((blk * (E2c / 4)) & 7);
+      float* tb = warp_tile + blk * E2c * 32 + (kB & 3);
+      int off[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) off[c] = (R ^ c) << 2;
 #pragma unroll
       for (int i = 0; i < EP; ++i) {
         const int ia = i / E2c, ib = i % E2c;
-        warp_tile[tsw<E2c>(blk * E2c + ib, kB + E2c * ia)] = v[i];
+        const int ci = (((E2c / 4) * ia) ^ (ib & 7)) & 7;
+        tb[ib * 32 + off[ci]] = el(v, i);
       }
       __syncwarp();
+      const int g = (lane & 7) ^ (((lane / E2c) * (E2c / 4)) & 7);
+      const float* rb = warp_tile + lane * 32;
 #pragma unroll
       for (int m = 0; m < 8; ++m) {
-        const float4 q = *reinterpret_cast<const float4*>(&warp_tile[tsw<E2c>(lane, 4 * m)]);
-        v[4 * m] = q.x; v[4 * m + 1] = q.y; v[4 * m + 2] = q.z; v[4 * m + 3] = q.w;
+        const float4 q = *reinterpret_cast<const float4*>(rb + ((m ^ g) << 2));
+        v[2 * m] = make_float2(q.x, q.y);
+        v[2 * m + 1] = make_float2(q.z, q.w);
       }
       __syncwarp();
-      reg_stages<0, 5>(v);
+      reg_stages<5>(v);
     };
     if (E2 == 8) run(std::integral_constant<int, 8>{});
     else if (E2 == 16) run(std::integral_constant<int, 16>{});
@@ -241,7 +253,7 @@ __global__ void __launch_bounds__(MAXT) k_rotate_quant(const RqParams p) {
     int fail = !dev::mbar_wait(dev::smem_u32(&bars[b]), parity, p.err, kSiteRqRow, p.limit_ns);
 
     // ---- round 1: gather from the bf16 row, apply signs ---------------------------------
-    float v[EP];
+    float2 v[EP / 2];
     float psum = 0.f;
     const uint16_t* row = reinterpret_cast<const uint16_t*>(rowbuf + (size_t)b * row_stride);
     const bool take = active && !fail;
@@ -250,7 +262,7 @@ __global__ void __launch_bounds__(MAXT) k_rotate_quant(const RqParams p) {
       const uint32_t e = entry(t0, i);
       const uint32_t hb = take ? (uint32_t)row[e & 0x7FFFu] : 0u;
       if (p.want_sum) psum += __uint_as_float(hb << 16);
-      v[i] = __uint_as_float((hb ^ (e & 0x8000u)) << 16);
+      el(v, i) = __uint_as_float((hb ^ (e & 0x8000u)) << 16);
     }
     if (p.want_sum) {
       psum = warp_sum(psum);
@@ -276,7 +288,7 @@ __global__ void __launch_bounds__(MAXT) k_rotate_quant(const RqParams p) {
       if (p.center) {
         const float mu = s / (float)d;
 #pragma unroll
-        for (int i = 0; i < EP; ++i) v[i] -= (entry(t0, i) & 0x8000u) ? -mu : mu;
+        for (int i = 0; i < EP; ++i) el(v, i) -= (entry(t0, i) & 0x8000u) ? -mu : mu;
         if (tid == 0) p.mean[t] = mu;
       }
       if (tid == 0 && p.rowsum) p.rowsum[t] = s;
@@ -289,7 +301,7 @@ __global__ void __launch_bounds__(MAXT) k_rotate_quant(const RqParams p) {
 #pragma unroll
         for (int m = 0; m < 8; ++m)
           *reinterpret_cast<float4*>(&rbuf[base + ((m ^ (tid & 7)) << 2)]) =
-              make_float4(v[4 * m], v[4 * m + 1], v[4 * m + 2], v[4 * m + 3]);
+              make_float4(v[2 * m].x, v[2 * m].y, v[2 * m + 1].x, v[2 * m + 1].y);
       }
       __syncthreads();
       if constexpr (!kT1Regs) {
@@ -306,7 +318,7 @@ __global__ void __launch_bounds__(MAXT) k_rotate_quant(const RqParams p) {
       for (int i = 0; i < EP; ++i) {
         const uint32_t e = entry(t1, i);
         const float g = active ? rbuf[e & 0x7FFFu] : 0.f;
-        v[i] = __uint_as_float(__float_as_uint(g) ^ ((e & 0x8000u) << 16));
+        el(v, i) = __uint_as_float(__float_as_uint(g) ^ ((e & 0x8000u) << 16));
       }
       if constexpr (kAlias) __syncthreads();  // every warp is done reading the round buffer
       block_transform<HMODE>(v, p.hlog2, lane, warp_tile);
@@ -316,7 +328,10 @@ __global__ void __launch_bounds__(MAXT) k_rotate_quant(const RqParams p) {
     const bool lm = p.mode == kRqLloydMax;
     float stat = 0.f;
 #pragma unroll
-    for (int i = 0; i < EP; ++i) stat = lm ? fmaf(v[i], v[i], stat) : fmaxf(stat, fabsf(v[i]));
+    for (int i = 0; i < EP; ++i) {
+      const float x = el(v, i);
+      stat = lm ? fmaf(x, x, stat) : fmaxf(stat, fabsf(x));
+    }
     stat = lm ? warp_sum(stat) : warp_max(stat);
     if (lane == 0) red[32 + warp] = stat;
     __syncthreads();
@@ -328,8 +343,8 @@ __global__ void __launch_bounds__(MAXT) k_rotate_quant(const RqParams p) {
       float4* dst = reinterpret_cast<float4*>(p.rotated + t * (int64_t)d + base);
 #pragma unroll
       for (int m = 0; m < 8; ++m)
-        dst[m] = make_float4(v[4 * m] * nrm, v[4 * m + 1] * nrm, v[4 * m + 2] * nrm,
-                             v[4 * m + 3] * nrm);
+        dst[m] = make_float4(v[2 * m].x * nrm, v[2 * m].y * nrm, v[2 * m + 1].x * nrm,
+                             v[2 * m + 1].y * nrm);
     }
 
     // ---- quantize + store --------------------------------------------------------------
@@ -341,7 +356,7 @@ __global__ void __launch_bounds__(MAXT) k_rotate_quant(const RqParams p) {
         uint32_t packed[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
         for (int i = 0; i < EP; ++i) {
-          const float u = v[i] * mult;
+          const float u = el(v, i) * mult;
           int c = (u > thr[7]) ? 8 : 0;
           c += (u > thr[c + 3]) ? 4 : 0;
           c += (u > thr[c + 1]) ? 2 : 0;
@@ -363,10 +378,12 @@ __global__ void __launch_bounds__(MAXT) k_rotate_quant(const RqParams p) {
         uint32_t w[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-          const uint32_t f0 = byte_of(fmaf(v[4 * k], mult, 12582912.f));
-          const uint32_t f1 = byte_of(fmaf(v[4 * k + 1], mult, 12582912.f));
-          const uint32_t f2 = byte_of(fmaf(v[4 * k + 2], mult, 12582912.f));
-          const uint32_t f3 = byte_of(fmaf(v[4 * k + 3], mult, 12582912.f));
+          const float2 magic = make_float2(12582912.f, 12582912.f);
+          const float2 mm = make_float2(mult, mult);
+          const float2 r0 = __ffma2_rn(v[2 * k], mm, magic);
+          const float2 r1 = __ffma2_rn(v[2 * k + 1], mm, magic);
+          const uint32_t f0 = byte_of(r0.x), f1 = byte_of(r0.y);
+          const uint32_t f2 = byte_of(r1.x), f3 = byte_of(r1.y);
           w[k] = __byte_perm(__byte_perm(f0, f1, 0x0040), __byte_perm(f2, f3, 0x0040), 0x5410);
         }
         if (p.mode == kRqInt8) {

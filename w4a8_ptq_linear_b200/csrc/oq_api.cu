@@ -57,7 +57,12 @@ cudaError_t allow_max_dynamic_smem(const void* fn) {
   int max_smem = 0;
   e = cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
+  cudaFuncAttributes fa{};
+  e = cudaFuncGetAttributes(&fa, fn);
+  if (e != cudaSuccess) return e;
+  // the ceiling covers dynamic shared memory only; static shared memory comes on top
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           max_smem - (int)fa.sharedSizeBytes);
   if (e == cudaSuccess) done.emplace_back(dev, fn);
   return e;
 }
