@@ -7,7 +7,7 @@
 // M) and BN tokens t (the MMA's N). The weight operand is the one unpacked on chip, and the
 // activation tile is shared through L2 by every channel tile of the same token range.
 //
-// Persistent CTAs (one per SM) walk the tiles in channel-fastest order. Warp roles (352 thr):
+// Persistent CTAs (one per SM) walk the tiles in channel-fastest order. Warp roles (608 thr):
 //   warp 0     packed-operand producer: TMA loads of the packed weight tile (and, for 4-bit
 //              activations, the packed activation tile) into an SP-deep ring that the
 //              converters release as soon as they have unpacked it;
@@ -15,9 +15,9 @@
 //              slice, into one of two TMEM accumulators of BN columns);
 //   warp 2     activation producer (INT8 activations only): TMA loads of the activation tile
 //              into an SX-deep ring that only the MMA releases;
-//   warps 3-6  converters: packed INT4 weights (and 4-bit activations) -> INT8 / FP16 in the
+//   warps 3-10 converters: packed INT4 weights (and 4-bit activations) -> INT8 / FP16 in the
 //              128-byte-swizzled K-major layout, into an S2-deep ring of operand tiles;
-//   warps 7-10 epilogue: TMEM -> registers -> alpha_t s_w acc + mean_t w_1 + b -> bf16 ->
+//   warps 11-18 epilogue: TMEM -> registers -> alpha_t s_w acc + mean_t w_1 + b -> bf16 ->
 //              coalesced global stores (each warp writes 32 consecutive channels of a token),
 //              while the MMA already accumulates the next tile into the other TMEM buffer.
 // Keeping the large activation tile out of the conversion path matters: its ring slot is held
@@ -46,9 +46,9 @@ namespace oq {
 namespace {
 
 constexpr int BM = 128;       // output channels per tile (MMA M)
-constexpr int NCONV = 128;    // converter threads (warps 3-6)
+constexpr int NCONV = 256;    // converter threads (warps 3-10)
 constexpr int CONV0 = 96;     // first converter thread
-constexpr int NEPI = 128;     // epilogue threads (warps 7-10)
+constexpr int NEPI = 256;     // epilogue threads (warps 11-18)
 constexpr int EPI0 = CONV0 + NCONV;  // first epilogue thread
 constexpr int NTHREADS = EPI0 + NEPI;
 
@@ -75,7 +75,7 @@ struct Cfg {
   static constexpr int SMEM = OFF_MISC + 16 + 1024;                // + slack for alignment
   static_assert(XT % 1024 == 0 && P_STAGE % 1024 == 0 && CONV_STAGE % 1024 == 0 &&
                 XP % 1024 == 0, "operand tiles must stay 1024-byte aligned");
-  static_assert(BN % 32 == 0 && BN <= 256, "MMA N");
+  static_assert(BN % 64 == 0 && BN <= 256, "MMA N");
   static_assert(SMEM <= 232448, "shared memory");
 };
 
@@ -428,10 +428,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     // Thread (lane quarter q, lane) owns output channel o; a 32-column TMEM load gives it 32
     // consecutive tokens of that channel. For each token the 32 lanes of a warp store 32
     // consecutive channels, i.e. 64 (bf16) or 128 (raw accumulator) contiguous bytes.
-    const int etid = tid - EPI0;         // 0..127
+    const int etid = tid - EPI0;         // 0..255
     const int q = warp & 3;              // TMEM lane quarter of this warp
+    const int half = etid >> 7;          // the two warps of a quarter split the columns
     const int o_local = q * 32 + lane;
     const bool leader = etid == 0;
+    constexpr int COLS = BN / 2;
     uint32_t it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x, ++it) {
@@ -460,11 +462,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (ok) dev::tc_fence_after();
       const int t_end = min(BN, p.T - t0);   // tokens of this tile inside [0, T)
 #pragma unroll 1
-      for (int c = 0; ok && c < BN / 32; ++c) {
+      for (int cc = 0; ok && cc < COLS / 32; ++cc) {
+        const int c = half * (COLS / 32) + cc;   // 32-column chunk of the tile
         uint32_t r[32];
         dev::tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * BN + c * 32), r);
         dev::tmem_wait_ld();
-        if (c == BN / 32 - 1) {  // accumulator fully read: hand it back to the MMA
+        if (cc == COLS / 32 - 1) {  // this thread's part of the accumulator is read
           dev::tc_fence_before();
           dev::mbar_arrive(tempty_bar(b));
         }
