@@ -4,9 +4,12 @@
 // HBM-bound design, one token row (d bf16 values) at a time per CTA:
 //  - Persistent CTAs walk tokens t = blockIdx.x, blockIdx.x + gridDim.x, ...; one thread keeps
 //    whole rows streaming into shared memory with 1-D bulk copies (TMA) nbuf rows ahead.
-//  - Every thread owns 32 rotated positions per round. Its gather entries (source index |
-//    sign << 15, laid out on the host in the order the thread consumes them) stay in
-//    registers for the whole kernel.
+//  - Every thread owns 32 rotated positions per round. Its gather entries (source indices,
+//    laid out on the host in the order the thread consumes them) stay in registers for the
+//    whole kernel.
+//  - Round-1 signs are moved to the source side (channel j takes the sign of the rotated
+//    position that gathers it) and applied by one coalesced 16-byte pass over the row in
+//    shared memory, so the random gather is only an index, a 2-byte load and a shift.
 //  - Block transform of size h = 2^L in three shapes:
 //      h <= 32        the thread holds whole blocks: L register butterfly stages;
 //      h = 64, 128    the thread holds 32 consecutive positions: 5 register stages, then
@@ -19,7 +22,8 @@
 //    Butterflies past the first stage run on packed f32x2 adds.
 //  - A second round gathers from an fp32 copy of the first round's output, written in a
 //    swizzled layout whose indices the host folded into the round-2 entries.
-//  - Centering uses the sum of the gathered values (a permutation keeps the sum).
+//  - Centering: the same pass sums the row; since a round is linear, the centered first round
+//    is R(x) - mean * R(1), with R(1) (unnormalised) a per-plan constant vector.
 //  - Per-token absmax (or sum of squares for Lloyd-Max) by shuffles and one block reduction;
 //    codes are rounded with one FMA against 1.5 * 2^23 and packed with byte permutes into
 //    one or two 16-byte stores per thread.
@@ -42,8 +46,10 @@ constexpr int EP = 32;  // positions per thread
 struct RqParams {
   const uint16_t* x;   // bf16 bits
   int64_t ldx, T;
-  int d, hlog2, center, mode, nbuf, want_sum;
+  int d, hlog2, center, mode, nbuf, want_sum, mask_smem;
   const uint16_t* tab;   // rounds x d entries in kernel order
+  const uint4* smask;    // round-1 source signs: bit 15 / 31 of word j/2 flips channel j
+  const float4* ones;    // c' = unnormalised round-1 transform of the all-ones vector
   void* codes;
   float* scale;
   float* mean;
@@ -112,26 +118,17 @@ __device__ __forceinline__ uint32_t entry(const uint32_t (&t)[EP / 2], int i) {
 
 __device__ __forceinline__ uint32_t byte_of(float f) { return __float_as_uint(f); }
 
-// Block transform of the 32 values a thread holds, for one of the three shapes.
-template <int HMODE>
-__device__ __forceinline__ void block_transform(float2 (&v)[EP / 2], int hlog2, int lane,
-                                                float* warp_tile) {
-  if constexpr (HMODE == 0) {
+// Block transform of the 32 values a thread holds, for h = 2^HLOG2 in one of three shapes.
+template <int HLOG2>
+__device__ __forceinline__ void block_transform(float2 (&v)[EP / 2], int lane, float* warp_tile) {
+  if constexpr (HLOG2 <= 5) {
     // h <= 32: every block lies inside the thread
-    switch (hlog2) {
-      case 0: break;
-      case 1: reg_stages<1>(v); break;
-      case 2: reg_stages<2>(v); break;
-      case 3: reg_stages<3>(v); break;
-      case 4: reg_stages<4>(v); break;
-      default: reg_stages<5>(v); break;
-    }
-  } else if constexpr (HMODE == 1) {
+    reg_stages<HLOG2>(v);
+  } else if constexpr (HLOG2 <= 7) {
     // h = 64 or 128: 5 stages in registers, then across 2 or 4 lanes
     reg_stages<5>(v);
 #pragma unroll
-    for (int m = 1; m <= 2; m <<= 1) {
-      if ((32 * m) >= (1 << hlog2)) break;
+    for (int m = 1; m < (1 << (HLOG2 - 5)); m <<= 1) {
       const float sg = (lane & m) ? -1.f : 1.f;
       const float2 sgn = make_float2(sg, sg);
 #pragma unroll
@@ -143,47 +140,40 @@ __device__ __forceinline__ void block_transform(float2 (&v)[EP / 2], int hlog2, 
     }
   } else {
     // h = 256, 512, 1024: high bits in the strided arrangement, transpose, low bits
-    const int E2 = 1 << (hlog2 - 5);
-    auto run = [&](auto e2c) {
-      constexpr int E2c = decltype(e2c)::value;
-      constexpr int LB = (E2c == 8) ? 3 : (E2c == 16) ? 4 : 5;
-      reg_stages<LB>(v);
-      // Element i of lane (blk, kB) goes to row blk*E2 + ib, column kB + E2*ia of the tile,
-      // stored at chunk (col/4) ^ g(row). With E2 >= 8 the chunk splits into a per-thread
-      // part (kB/4 ^ G(blk)) and a per-register part ((E2/4)*ia ^ (ib & 7)), so every
-      // address is a per-thread base plus one of 8 precomputed offsets and a constant.
-      const int blk = lane / E2c, kB = lane % E2c;
-      const int R = (kB >> 2) ^ ((blk * (E2c / 4)) & 7);
-      float* tb = warp_tile + blk * E2c * 32 + (kB & 3);
-      int off[8];
+    constexpr int E2 = 1 << (HLOG2 - 5);
+    reg_stages<HLOG2 - 5>(v);
+    // Element i of lane (blk, kB) goes to row blk*E2 + ib, column kB + E2*ia of the tile,
+    // stored at chunk (col/4) ^ g(row). With E2 >= 8 the chunk splits into a per-thread
+    // part (kB/4 ^ G(blk)) and a per-register part ((E2/4)*ia ^ (ib & 7)), so every
+    // address is a per-thread base plus one of 8 precomputed offsets and a constant.
+    const int blk = lane / E2, kB = lane % E2;
+    const int R = (kB >> 2) ^ ((blk * (E2 / 4)) & 7);
+    float* tb = warp_tile + blk * E2 * 32 + (kB & 3);
+    int off[8];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) off[c] = (R ^ c) << 2;
+    for (int c = 0; c < 8; ++c) off[c] = (R ^ c) << 2;
 #pragma unroll
-      for (int i = 0; i < EP; ++i) {
-        const int ia = i / E2c, ib = i % E2c;
-        const int ci = (((E2c / 4) * ia) ^ (ib & 7)) & 7;
-        tb[ib * 32 + off[ci]] = el(v, i);
-      }
-      __syncwarp();
-      const int g = (lane & 7) ^ (((lane / E2c) * (E2c / 4)) & 7);
-      const float* rb = warp_tile + lane * 32;
+    for (int i = 0; i < EP; ++i) {
+      const int ia = i / E2, ib = i % E2;
+      const int ci = (((E2 / 4) * ia) ^ (ib & 7)) & 7;
+      tb[ib * 32 + off[ci]] = el(v, i);
+    }
+    __syncwarp();
+    const int g = (lane & 7) ^ (((lane / E2) * (E2 / 4)) & 7);
+    const float* rb = warp_tile + lane * 32;
 #pragma unroll
-      for (int m = 0; m < 8; ++m) {
-        const float4 q = *reinterpret_cast<const float4*>(rb + ((m ^ g) << 2));
-        v[2 * m] = make_float2(q.x, q.y);
-        v[2 * m + 1] = make_float2(q.z, q.w);
-      }
-      __syncwarp();
-      reg_stages<5>(v);
-    };
-    if (E2 == 8) run(std::integral_constant<int, 8>{});
-    else if (E2 == 16) run(std::integral_constant<int, 16>{});
-    else run(std::integral_constant<int, 32>{});
+    for (int m = 0; m < 8; ++m) {
+      const float4 q = *reinterpret_cast<const float4*>(rb + ((m ^ g) << 2));
+      v[2 * m] = make_float2(q.x, q.y);
+      v[2 * m + 1] = make_float2(q.z, q.w);
+    }
+    __syncwarp();
+    reg_stages<5>(v);
   }
 }
 
-template <int HMODE, int MAXT, int ROUNDS>
-__global__ void __launch_bounds__(MAXT) k_rotate_quant(const RqParams p) {
+template <int HLOG2, int MAXT, int ROUNDS>
+__global__ void __launch_bounds__(MAXT, 1) k_rotate_quant(const RqParams p) {
   // Round-2 entries stay in registers unless a 1024-thread block would spill them.
   constexpr bool kT1Regs = (ROUNDS == 2) && (MAXT <= 256);
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -196,13 +186,16 @@ __global__ void __launch_bounds__(MAXT) k_rotate_quant(const RqParams p) {
   const uint32_t row_stride = (row_bytes + 127u) & ~127u;
   // With two rounds and h >= 256 the transpose tiles alias the fp32 round buffer: warp w's
   // tile is exactly the range of positions warp w writes into that buffer.
+  constexpr int HMODE = HLOG2 <= 5 ? 0 : (HLOG2 <= 7 ? 1 : 2);
   constexpr bool kAlias = (ROUNDS == 2) && (HMODE == 2);
   uint8_t* rowbuf = smem;
   float* rbuf = reinterpret_cast<float*>(smem + (size_t)p.nbuf * row_stride);
   float* tbuf = kAlias ? rbuf : rbuf + (ROUNDS == 2 ? nwarps * 1024 : 0);
   float* red = tbuf + (HMODE == 2 ? nwarps * 1024 : 0);  // [0,32) sums, [32,64) statistic
+  // round-1 sign masks, staged in shared memory when they fit beside the row buffers
+  uint4* s_mask = reinterpret_cast<uint4*>(red + 64 + 16 + 16);
   float* thr = red + 64;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(thr + 16);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(thr + 16);   // nbuf <= 3 barriers (16 floats)
   float* warp_tile = tbuf + warp * 1024;
 
   uint32_t t0[EP / 2], t1[EP / 2];
@@ -225,6 +218,11 @@ __global__ void __launch_bounds__(MAXT) k_rotate_quant(const RqParams p) {
     }
   }
   if (tid < 16) thr[tid] = p.thr[tid];
+  const uint4* mask = p.smask;
+  if (p.mask_smem) {
+    for (int c = tid; c < d / 8; c += blockDim.x) s_mask[c] = __ldg(p.smask + c);
+    mask = s_mask;
+  }
   if (tid == 0) {
     for (int b = 0; b < p.nbuf; ++b) dev::mbar_init(dev::smem_u32(&bars[b]), 1);
     dev::fence_mbar_init();
@@ -251,18 +249,27 @@ __global__ void __launch_bounds__(MAXT) k_rotate_quant(const RqParams p) {
     const int b = it % p.nbuf;
     const uint32_t parity = (uint32_t)(it / p.nbuf) & 1u;
     int fail = !dev::mbar_wait(dev::smem_u32(&bars[b]), parity, p.err, kSiteRqRow, p.limit_ns);
-
-    // ---- round 1: gather from the bf16 row, apply signs ---------------------------------
-    float2 v[EP / 2];
-    float psum = 0.f;
-    const uint16_t* row = reinterpret_cast<const uint16_t*>(rowbuf + (size_t)b * row_stride);
     const bool take = active && !fail;
+
+    // ---- source-side signs (and the row sum) in one coalesced pass ---------------------
+    uint4* rowv = reinterpret_cast<uint4*>(rowbuf + (size_t)b * row_stride);
+    const int nact = d / EP;          // threads that own positions; each takes 4 chunks
+    float psum = 0.f;
+    if (take) {
 #pragma unroll
-    for (int i = 0; i < EP; ++i) {
-      const uint32_t e = entry(t0, i);
-      const uint32_t hb = take ? (uint32_t)row[e & 0x7FFFu] : 0u;
-      if (p.want_sum) psum += __uint_as_float(hb << 16);
-      el(v, i) = __uint_as_float((hb ^ (e & 0x8000u)) << 16);
+      for (int m = 0; m < 4; ++m) {
+        const int c = tid + m * nact;
+        uint4 w = rowv[c];
+        const uint4 mk = mask[c];
+        if (p.want_sum) {
+          psum += __uint_as_float(w.x << 16) + __uint_as_float(w.x & 0xFFFF0000u);
+          psum += __uint_as_float(w.y << 16) + __uint_as_float(w.y & 0xFFFF0000u);
+          psum += __uint_as_float(w.z << 16) + __uint_as_float(w.z & 0xFFFF0000u);
+          psum += __uint_as_float(w.w << 16) + __uint_as_float(w.w & 0xFFFF0000u);
+        }
+        w.x ^= mk.x; w.y ^= mk.y; w.z ^= mk.z; w.w ^= mk.w;
+        rowv[c] = w;
+      }
     }
     if (p.want_sum) {
       psum = warp_sum(psum);
@@ -273,27 +280,35 @@ __global__ void __launch_bounds__(MAXT) k_rotate_quant(const RqParams p) {
       aborted = true;
       break;
     }
-    if (tid == 0) {  // row buffer b is free again
-      const int64_t tn = t + (int64_t)p.nbuf * G;
-      if (tn < T) {
-        const uint32_t bar = dev::smem_u32(&bars[b]);
-        dev::mbar_arrive_expect_tx(bar, row_bytes);
-        dev::bulk_g2s(dev::smem_u32(rowbuf + (size_t)b * row_stride), p.x + tn * p.ldx,
-                      row_bytes, bar);
-      }
-    }
-    if (p.want_sum) {
-      float s = 0.f;
-      for (int w = 0; w < nwarps; ++w) s += red[w];
-      if (p.center) {
-        const float mu = s / (float)d;
+
+    // ---- round 1: gather from the signed bf16 row ----------------------------------------
+    float2 v[EP / 2];
+    const uint16_t* row = reinterpret_cast<const uint16_t*>(rowbuf + (size_t)b * row_stride);
 #pragma unroll
-        for (int i = 0; i < EP; ++i) el(v, i) -= (entry(t0, i) & 0x8000u) ? -mu : mu;
-        if (tid == 0) p.mean[t] = mu;
-      }
-      if (tid == 0 && p.rowsum) p.rowsum[t] = s;
+    for (int i = 0; i < EP; ++i) {
+      const uint32_t hb = active ? (uint32_t)row[entry(t0, i)] : 0u;
+      el(v, i) = __uint_as_float(hb << 16);
     }
-    block_transform<HMODE>(v, p.hlog2, lane, warp_tile);
+    float mu = 0.f;
+    if (p.want_sum) {
+      float sum = 0.f;
+      for (int w = 0; w < nwarps; ++w) sum += red[w];
+      mu = sum / (float)d;
+      if (tid == 0) {
+        if (p.center) p.mean[t] = mu;
+        if (p.rowsum) p.rowsum[t] = sum;
+      }
+    }
+    block_transform<HLOG2>(v, lane, warp_tile);
+    if (p.center && active) {  // centered round = R(x) - mean * R(1)
+      const float2 nm = make_float2(-mu, -mu);
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        const float4 c1 = __ldg(p.ones + tid * 8 + m);
+        v[2 * m] = __ffma2_rn(make_float2(c1.x, c1.y), nm, v[2 * m]);
+        v[2 * m + 1] = __ffma2_rn(make_float2(c1.z, c1.w), nm, v[2 * m + 1]);
+      }
+    }
 
     // ---- round 2: through a swizzled fp32 copy in shared memory -------------------------
     if constexpr (ROUNDS == 2) {
@@ -321,7 +336,7 @@ __global__ void __launch_bounds__(MAXT) k_rotate_quant(const RqParams p) {
         el(v, i) = __uint_as_float(__float_as_uint(g) ^ ((e & 0x8000u) << 16));
       }
       if constexpr (kAlias) __syncthreads();  // every warp is done reading the round buffer
-      block_transform<HMODE>(v, p.hlog2, lane, warp_tile);
+      block_transform<HLOG2>(v, lane, warp_tile);
     }
 
     // ---- per-token statistic ------------------------------------------------------------
@@ -335,6 +350,15 @@ __global__ void __launch_bounds__(MAXT) k_rotate_quant(const RqParams p) {
     stat = lm ? warp_sum(stat) : warp_max(stat);
     if (lane == 0) red[32 + warp] = stat;
     __syncthreads();
+    if (tid == 0) {  // every thread is past its gathers: row buffer b can be refilled
+      const int64_t tn = t + (int64_t)p.nbuf * G;
+      if (tn < T) {
+        const uint32_t bar = dev::smem_u32(&bars[b]);
+        dev::mbar_arrive_expect_tx(bar, row_bytes);
+        dev::bulk_g2s(dev::smem_u32(rowbuf + (size_t)b * row_stride), p.x + tn * p.ldx,
+                      row_bytes, bar);
+      }
+    }
     stat = 0.f;
     for (int w = 0; w < nwarps; ++w) stat = lm ? stat + red[32 + w] : fmaxf(stat, red[32 + w]);
 
@@ -350,7 +374,7 @@ __global__ void __launch_bounds__(MAXT) k_rotate_quant(const RqParams p) {
     // ---- quantize + store --------------------------------------------------------------
     if (lm) {
       const float sigma = fmaxf(sqrtf(stat * nrm * nrm / (float)d), 1e-10f);
-      const float mult = nrm / sigma;
+      const float mult = nrm * __frcp_rn(sigma);
       if (tid == 0) p.scale[t] = sigma;
       if (active) {
         uint32_t packed[4] = {0u, 0u, 0u, 0u};
@@ -370,7 +394,7 @@ __global__ void __launch_bounds__(MAXT) k_rotate_quant(const RqParams p) {
     } else {
       const float qmax = (p.mode == kRqInt8) ? 127.f : 7.f;
       const float a = fmaxf(stat * nrm, 1e-10f);
-      const float mult = nrm * (qmax / a);
+      const float mult = nrm * qmax * __frcp_rn(a);
       if (tid == 0) p.scale[t] = a / qmax;
       if (active) {
         // fma against 1.5 * 2^23 rounds half-to-even to an integer held in the low mantissa
@@ -421,24 +445,35 @@ __global__ void __launch_bounds__(MAXT) k_rotate_quant(const RqParams p) {
 
 struct LaunchCfg {
   void* fn = nullptr;
-  int nthr = 0, nbuf = 0, grid_per_sm = 0;
+  int nthr = 0, nbuf = 0, grid_per_sm = 0, mask_smem = 0;
   size_t smem = 0;
 };
 
-template <int HM, int MAXT, int R>
+template <int HL, int MAXT, int R>
 void* kern() {
-  return reinterpret_cast<void*>(&k_rotate_quant<HM, MAXT, R>);
+  return reinterpret_cast<void*>(&k_rotate_quant<HL, MAXT, R>);
 }
 
-void* pick_kernel(int hmode, bool big, int rounds) {
-  if (rounds == 1) {
-    if (hmode == 0) return big ? kern<0, 1024, 1>() : kern<0, 256, 1>();
-    if (hmode == 1) return big ? kern<1, 1024, 1>() : kern<1, 256, 1>();
-    return big ? kern<2, 1024, 1>() : kern<2, 256, 1>();
+template <int MAXT, int R>
+void* kern_h(int hlog2) {
+  switch (hlog2) {
+    case 0: return kern<0, MAXT, R>();
+    case 1: return kern<1, MAXT, R>();
+    case 2: return kern<2, MAXT, R>();
+    case 3: return kern<3, MAXT, R>();
+    case 4: return kern<4, MAXT, R>();
+    case 5: return kern<5, MAXT, R>();
+    case 6: return kern<6, MAXT, R>();
+    case 7: return kern<7, MAXT, R>();
+    case 8: return kern<8, MAXT, R>();
+    case 9: return kern<9, MAXT, R>();
+    default: return kern<10, MAXT, R>();
   }
-  if (hmode == 0) return big ? kern<0, 1024, 2>() : kern<0, 256, 2>();
-  if (hmode == 1) return big ? kern<1, 1024, 2>() : kern<1, 256, 2>();
-  return big ? kern<2, 1024, 2>() : kern<2, 256, 2>();
+}
+
+void* pick_kernel(int hlog2, bool big, int rounds) {
+  if (rounds == 1) return big ? kern_h<1024, 1>(hlog2) : kern_h<256, 1>(hlog2);
+  return big ? kern_h<1024, 2>(hlog2) : kern_h<256, 2>(hlog2);
 }
 
 }  // namespace
@@ -479,7 +514,7 @@ oq_status launch_rotate_quant(const RqArgs& a, cudaStream_t s) {
   LaunchCfg cfg;
   {
     std::lock_guard<std::mutex> lock(mu);
-    auto key = std::make_tuple(dev_id, a.d, hmode, a.rounds);
+    auto key = std::make_tuple(dev_id, a.d, hlog2, a.rounds);
     auto itc = cache.find(key);
     if (itc != cache.end()) {
       cfg = itc->second;
@@ -491,12 +526,16 @@ oq_status launch_rotate_quant(const RqArgs& a, cudaStream_t s) {
       // fp32 round buffer and transpose tiles (one region when both are needed), both sized
       // in whole warps of 1024 positions
       const size_t warps_bytes = (size_t)(nthr / 32) * 4096;
-      const size_t fixed = ((a.rounds == 2 || hmode == 2) ? warps_bytes : 0) + 64 * 4 + 16 * 4;
-      int nbuf = 3;
-      while (nbuf > 1 && fixed + nbuf * row_stride + nbuf * 8 > (size_t)max_smem / 3) --nbuf;
-      cfg.smem = fixed + nbuf * row_stride + nbuf * 8;
+      // reductions, thresholds, barriers, then the sign masks (2 bytes per channel)
+      size_t fixed = ((a.rounds == 2 || hmode == 2) ? warps_bytes : 0) + 96 * 4;
+      const size_t mask_bytes = (size_t)a.d * 2;
+      cfg.mask_smem = fixed + mask_bytes + row_stride <= (size_t)max_smem / 3;
+      if (cfg.mask_smem) fixed += mask_bytes;
+      int nbuf = 2;
+      while (nbuf > 1 && fixed + nbuf * row_stride > (size_t)max_smem / 3) --nbuf;
+      cfg.smem = fixed + nbuf * row_stride;
       if (cfg.smem > (size_t)max_smem) return fail(OQ_ERR_UNSUPPORTED, "rotate_quant: d too large");
-      cfg.fn = pick_kernel(hmode, big, a.rounds);
+      cfg.fn = pick_kernel(hlog2, big, a.rounds);
       cfg.nthr = nthr;
       cfg.nbuf = nbuf;
       ce = allow_max_dynamic_smem(cfg.fn);
@@ -520,7 +559,10 @@ oq_status launch_rotate_quant(const RqArgs& a, cudaStream_t s) {
   p.mode = a.mode;
   p.nbuf = cfg.nbuf;
   p.want_sum = (a.center || a.rowsum) ? 1 : 0;
+  p.mask_smem = cfg.mask_smem;
   p.tab = a.tab;
+  p.smask = reinterpret_cast<const uint4*>(a.smask);
+  p.ones = reinterpret_cast<const float4*>(a.ones);
   p.codes = a.codes;
   p.scale = a.scale;
   p.mean = a.mean;

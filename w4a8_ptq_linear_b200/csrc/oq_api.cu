@@ -217,26 +217,56 @@ oq_status oq_plan_create(oq_plan** out, int d, int h, int rounds, uint64_t seed,
     for (int t = 0; t < d / 32; ++t) {
       for (int i = 0; i < 32; ++i) {
         const int64_t q = rq_gather_position(h, t, i);
-        const int src = (r == 0) ? pm[q] : rq_round_buffer_index(pm[q]);
-        tab[(size_t)r * d + (size_t)t * 32 + i] = (uint16_t)(src | (sg[q] < 0 ? 0x8000 : 0));
+        // round 1 carries no sign: it is applied to the source channel (see below)
+        const int src = (r == 0) ? pm[q] : (rq_round_buffer_index(pm[q]) | (sg[q] < 0 ? 0x8000 : 0));
+        tab[(size_t)r * d + (size_t)t * 32 + i] = (uint16_t)src;
       }
     }
   }
+  // Round-1 signs moved to the source side: channel pm[i] takes sign sg[i] (the rotated
+  // position that gathers it). Bit 15 (even channel) / 31 (odd channel) of word j/2.
+  std::vector<uint32_t> smask((size_t)d / 2, 0u);
+  for (int i = 0; i < d; ++i)
+    if (p->signs[i] < 0) smask[p->perm[i] / 2] |= 1u << (15 + 16 * (p->perm[i] & 1));
+  // c' = unnormalised round-1 transform of the all-ones vector = block Hadamard of the signs
+  std::vector<float> ones((size_t)d);
+  {
+    std::vector<int32_t> v(p->signs.begin(), p->signs.begin() + d);
+    for (int blk = 0; blk < d; blk += h)
+      for (int len = 1; len < h; len <<= 1)
+        for (int i = blk; i < blk + h; ++i)
+          if (!((i - blk) & len)) {
+            const int32_t a0 = v[i], b0 = v[i + len];
+            v[i] = a0 + b0;
+            v[i + len] = a0 - b0;
+          }
+    for (int i = 0; i < d; ++i) ones[i] = (float)v[i];
+  }
   lloyd_max_newton(p->cb_c, p->cb_t);
-  e = cudaMalloc(&p->d_tab, tab.size() * sizeof(uint16_t));
-  if (e != cudaSuccess) {
+  auto release = [&]() {
+    if (p->d_tab) cudaFree(p->d_tab);
+    if (p->d_smask) cudaFree(p->d_smask);
+    if (p->d_ones) cudaFree(p->d_ones);
     delete p;
-    return fail(OQ_ERR_NOMEM, "cudaMalloc plan tables: %s", cudaGetErrorString(e));
+  };
+  if (cudaMalloc(&p->d_tab, tab.size() * sizeof(uint16_t)) != cudaSuccess ||
+      cudaMalloc(&p->d_smask, smask.size() * sizeof(uint32_t)) != cudaSuccess ||
+      cudaMalloc(&p->d_ones, ones.size() * sizeof(float)) != cudaSuccess) {
+    release();
+    return fail(OQ_ERR_NOMEM, "cudaMalloc plan tables");
   }
   e = cudaMemcpy(p->d_tab, tab.data(), tab.size() * sizeof(uint16_t), cudaMemcpyHostToDevice);
+  if (e == cudaSuccess)
+    e = cudaMemcpy(p->d_smask, smask.data(), smask.size() * sizeof(uint32_t),
+                   cudaMemcpyHostToDevice);
+  if (e == cudaSuccess)
+    e = cudaMemcpy(p->d_ones, ones.data(), ones.size() * sizeof(float), cudaMemcpyHostToDevice);
   if (e != cudaSuccess) {
-    cudaFree(p->d_tab);
-    delete p;
+    release();
     return cuda_fail(e, "upload plan tables");
   }
   if (!device_error_word()) {
-    cudaFree(p->d_tab);
-    delete p;
+    release();
     return fail(OQ_ERR_CUDA, "device error word unavailable");
   }
   *out = p;
@@ -245,11 +275,13 @@ oq_status oq_plan_create(oq_plan** out, int d, int h, int rounds, uint64_t seed,
 
 void oq_plan_destroy(oq_plan* plan) {
   if (!plan) return;
-  if (plan->d_tab) {
+  if (plan->d_tab || plan->d_smask || plan->d_ones) {
     int cur = -1;
     cudaGetDevice(&cur);
     if (cur != plan->device) cudaSetDevice(plan->device);
-    cudaFree(plan->d_tab);
+    if (plan->d_tab) cudaFree(plan->d_tab);
+    if (plan->d_smask) cudaFree(plan->d_smask);
+    if (plan->d_ones) cudaFree(plan->d_ones);
     if (cur != plan->device && cur >= 0) cudaSetDevice(cur);
   }
   delete plan;
@@ -269,7 +301,8 @@ static oq_status rotate_quantize_impl(const oq_plan* plan, const void* x, int64_
                                       float* rowsum, int mode, int center, cudaStream_t s) {
   RqArgs a;
   a.x = x; a.ldx = ldx; a.T = T; a.d = plan->d; a.h = plan->h; a.rounds = plan->rounds;
-  a.center = center; a.mode = mode; a.tab = plan->d_tab; a.codes = codes; a.scale = scale;
+  a.center = center; a.mode = mode; a.tab = plan->d_tab; a.smask = plan->d_smask;
+  a.ones = plan->d_ones; a.codes = codes; a.scale = scale;
   a.mean = mean; a.rotated = rotated; a.rowsum = rowsum;
   for (int i = 0; i < 15; ++i) a.thr[i] = (float)plan->cb_t[i];
   return launch_rotate_quant(a, s);

@@ -18,7 +18,9 @@ struct oq_plan {
   std::vector<int8_t> signs;    // rounds * d
   std::vector<int32_t> perm;    // rounds * d
   uint16_t* d_tab = nullptr;    // device: rounds * d gather entries in kernel order,
-                                // source index | (sign < 0) << 15
+                                // source index (| (sign < 0) << 15 in round 2)
+  uint32_t* d_smask = nullptr;  // device: d/2 words, round-1 sign of channel j at bit 15 / 31
+  float* d_ones = nullptr;      // device: d floats, unnormalised round-1 transform of ones
   double cb_c[16] = {}, cb_t[15] = {};
 };
 
@@ -64,6 +66,8 @@ struct RqArgs {
   int64_t ldx = 0, T = 0;
   int d = 0, h = 0, rounds = 0, center = 0, mode = 0;
   const uint16_t* tab = nullptr;  // rounds * d
+  const uint32_t* smask = nullptr;  // d/2 words: round-1 signs moved to the source channels
+  const float* ones = nullptr;      // d floats: unnormalised round-1 transform of all ones
   void* codes = nullptr;
   float* scale = nullptr;
   float* mean = nullptr;     // written when center (or when rowsum is wanted: see rowsum)
