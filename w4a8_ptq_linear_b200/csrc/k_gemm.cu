@@ -3,28 +3,40 @@
 // added in the GEMM epilogue; OrbitQuant PR #25: absmax INT8 activations at A8, Lloyd-Max
 // codes below).
 //
-// Orientation: a tile is D[o, t] = sum_k W[o, k] X[t, k] for 128 output channels o (the MMA's
-// M) and BN tokens t (the MMA's N). The weight operand is the one unpacked on chip, and the
-// activation tile is shared through L2 by every channel tile of the same token range.
+// Orientation: a tile is D[o, t] = sum_k W[o, k] X[t, k] for 128 output channels o per CTA (the
+// MMA's M) and BN tokens t (the MMA's N). The weight operand is the one unpacked on chip, and
+// the activation tile is shared through L2 by every channel tile of the same token range.
 //
-// Persistent CTAs (one per SM) walk the tiles in channel-fastest order. Warp roles (608 thr):
+// Two shapes (template CG):
+//   CG = 1  one CTA per tile of 128 channels x BN tokens (small token counts);
+//   CG = 2  a cluster of two CTAs on neighbouring SMs computes 256 channels x BN tokens with
+//           tcgen05.mma.cta_group::2 (M = 256): each CTA stages and unpacks its own 128 weight
+//           rows and half of the activation tile, and the pair's leader issues the MMAs, whose
+//           completions are multicast to both CTAs. Every activation byte that crosses L2 and
+//           shared memory then feeds 256 channels instead of 128.
+//
+// Persistent CTAs (pairs) walk the tiles in channel-fastest order. Warp roles (608 thr):
 //   warp 0     packed-operand producer: TMA loads of the packed weight tile (and, for 4-bit
 //              activations, the packed activation tile) into an SP-deep ring that the
 //              converters release as soon as they have unpacked it;
-//   warp 1     TMEM owner and MMA issuer (one thread issues tcgen05.mma, 4 per 128-byte K
-//              slice, into one of two TMEM accumulators of BN columns);
+//   warp 1     TMEM owner and MMA issuer (one thread of the pair's leader issues tcgen05.mma,
+//              4 per 128-byte K slice, into one of two TMEM accumulators of BN columns);
 //   warp 2     activation producer (INT8 activations only): TMA loads of the activation tile
 //              into an SX-deep ring that only the MMA releases;
 //   warps 3-10 converters: packed INT4 weights (and 4-bit activations) -> INT8 / FP16 in the
-//              128-byte-swizzled K-major layout, into an S2-deep ring of operand tiles;
+//              128-byte-swizzled K-major layout, into an S2-deep ring of operand tiles; two
+//              groups of four warps take alternate K blocks, so that the hand-off latency of
+//              one block (barrier wait, proxy fence, arrive) overlaps the other's work;
 //   warps 11-18 epilogue: TMEM -> registers -> alpha_t s_w acc + mean_t w_1 + b -> bf16 ->
 //              coalesced global stores (each warp writes 32 consecutive channels of a token),
 //              while the MMA already accumulates the next tile into the other TMEM buffer.
 // Keeping the large activation tile out of the conversion path matters: its ring slot is held
 // from the TMA issue to the end of its MMA, so the unpacking must not sit in that interval.
 // Barriers: xfull/xempty (activation ring), pfull/pempty (packed ring), wready/wfree
-// (converted operands), tfull/tempty (accumulators). All waits are bounded; a wait that gives
-// up records its site, sets an abort flag and the roles drain.
+// (converted operands), tfull/tempty (accumulators). With CG = 2 the barriers the MMA waits on
+// (xfull, wready, tempty) are the leader's: the peer's activation loads complete on the
+// leader's xfull, and its converter and epilogue warps arrive there remotely. All waits are
+// bounded; a wait that gives up records its site, sets an abort flag and the roles drain.
 //
 // Kinds:
 //   A8       X int8 straight from TMA, W int4 -> int8; tcgen05.mma.kind::i8, exact int32.
@@ -37,6 +49,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstring>
+#include <map>
 #include <mutex>
 
 #include "oq_internal.h"
@@ -47,22 +60,27 @@ namespace {
 
 constexpr int BM = 128;       // output channels per tile (MMA M)
 constexpr int NCONV = 256;    // converter threads (warps 3-10)
+constexpr int NGROUP = 2;     // converter groups; group g converts the k-blocks j = g mod NGROUP
+constexpr int NCG = NCONV / NGROUP;  // threads per converter group
 constexpr int CONV0 = 96;     // first converter thread
 constexpr int NEPI = 256;     // epilogue threads (warps 11-18)
 constexpr int EPI0 = CONV0 + NCONV;  // first epilogue thread
 constexpr int NTHREADS = EPI0 + NEPI;
 
-template <int KIND, int BN>
+template <int KIND, int BN, int CG>
 struct Cfg {
   static constexpr int BK = (KIND == kGemmLloydMax) ? 64 : 128;   // 128 bytes of K per stage
   static constexpr bool XPACK = KIND != kGemmA8;
-  static constexpr int SX = XPACK ? 0 : 4;                         // activation ring (A8)
-  static constexpr int SP = 4;                                     // packed ring
-  static constexpr int S2 = (KIND == kGemmA4) ? 2 : 3;             // converted ring
+  static constexpr int XR = BN / CG;                               // activation rows per CTA
+  // Ring depths. Loads from L2 take a few thousand cycles, so the packed ring, which the
+  // converters free only after unpacking, must cover that latency at the MMA's pace.
+  static constexpr int SX = XPACK ? 0 : (CG == 2 ? 5 : 4);         // activation ring (A8)
+  static constexpr int SP = CG == 1 ? 4 : (KIND == kGemmA4 ? 6 : 8);  // packed ring
+  static constexpr int S2 = (KIND == kGemmA4) ? (CG == 2 ? 3 : 2) : (CG == 2 ? 4 : 3);
   static constexpr int WT = BM * 128;                              // W operand tile
-  static constexpr int XT = BN * 128;                              // X operand tile
+  static constexpr int XT = XR * 128;                              // X operand tile (this CTA)
   static constexpr int WP = BM * (BK / 2);                         // packed W per stage
-  static constexpr int XP = XPACK ? BN * (BK / 2) : 0;             // packed X per stage
+  static constexpr int XP = XPACK ? XR * (BK / 2) : 0;             // packed X per stage
   static constexpr int P_STAGE = XP + WP;                          // [Xp][Wp]
   static constexpr int CONV_STAGE = WT + (XPACK ? XT : 0);         // [W][X]
   static constexpr int OFF_X = 0;
@@ -77,6 +95,7 @@ struct Cfg {
                 XP % 1024 == 0, "operand tiles must stay 1024-byte aligned");
   static_assert(BN % 64 == 0 && BN <= 256, "MMA N");
   static_assert(SMEM <= 232448, "shared memory");
+  static_assert(NGROUP <= S2, "a converter group may run at most one ring phase ahead");
 };
 
 struct GemmParams {
@@ -147,12 +166,12 @@ __device__ __forceinline__ void lm4_to_f16(uint32_t s, const uint32_t (&lut)[8],
 }
 
 // Packed INT4 rows of 64 bytes -> int8 rows of 128 bytes in the 128-byte-swizzled layout
-// (16-byte chunk c of row r at r * 128 + ((c ^ (r & 7)) << 4)). Thread ctid takes the
-// 16-byte packed chunk q = ctid & 3 of rows ctid / 4 + 32 j; the swizzle phase r & 7 is the
-// same for all j, so every address is a constant offset from a per-thread base.
+// (16-byte chunk c of row r at r * 128 + ((c ^ (r & 7)) << 4)). Thread ctid of a group takes
+// the 16-byte packed chunk q = ctid & 3 of rows ctid / 4 + (NCG / 4) j; the swizzle phase r & 7
+// is the same for all j, so every address is a constant offset from a per-thread base.
 template <int ROWS>
 __device__ __forceinline__ void convert_i4_i8(const uint8_t* src, uint8_t* dst, int ctid) {
-  constexpr int RSTEP = NCONV / 4;   // rows covered by one pass of all converter threads
+  constexpr int RSTEP = NCG / 4;     // rows covered by one pass of the group's threads
   const int r0 = ctid >> 2, q = ctid & 3;
   const uint8_t* s = src + r0 * 64 + q * 16;
   uint8_t* da = dst + r0 * 128 + (((2 * q) ^ (r0 & 7)) << 4);
@@ -173,7 +192,7 @@ __device__ __forceinline__ void convert_i4_i8(const uint8_t* src, uint8_t* dst, 
 // Packed INT4 rows of 32 bytes (64 elements) -> fp16 rows of 128 bytes, swizzled.
 template <int ROWS>
 __device__ __forceinline__ void convert_i4_f16(const uint8_t* src, uint8_t* dst, int ctid) {
-  constexpr int RSTEP = NCONV / 2;
+  constexpr int RSTEP = NCG / 2;
   const int r0 = ctid >> 1, q = ctid & 1;
   const uint8_t* s = src + r0 * 32 + q * 16;
   uint8_t* d = dst + r0 * 128;
@@ -196,7 +215,7 @@ __device__ __forceinline__ void convert_i4_f16(const uint8_t* src, uint8_t* dst,
 template <int ROWS>
 __device__ __forceinline__ void convert_lm_f16(const uint8_t* src, uint8_t* dst, int ctid,
                                                const uint32_t (&lut)[8]) {
-  constexpr int RSTEP = NCONV / 2;
+  constexpr int RSTEP = NCG / 2;
   const int r0 = ctid >> 1, q = ctid & 1;
   const uint8_t* s = src + r0 * 32 + q * 16;
   uint8_t* d = dst + r0 * 128;
@@ -223,12 +242,12 @@ __device__ __forceinline__ int k_rotation(int tile, int n_o, int nkb) {
   return (int)(((unsigned)(tile % n_o) * 7u) % (unsigned)nkb);
 }
 
-template <int KIND, int BN>
+template <int KIND, int BN, int CG>
 __global__ void __launch_bounds__(NTHREADS, 1)
     k_gemm(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
            const GemmParams p) {
-  using C = Cfg<KIND, BN>;
-  constexpr int BK = C::BK, SX = C::SX, SP = C::SP, S2 = C::S2;
+  using C = Cfg<KIND, BN, CG>;
+  constexpr int BK = C::BK, SX = C::SX, SP = C::SP, S2 = C::S2, XR = C::XR;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -238,9 +257,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   volatile uint32_t* s_abort = s_misc + 1;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int n_o = (p.N + BM - 1) / BM;
+  const uint32_t rank = (CG == 2) ? dev::cluster_ctarank() : 0u;  // 0 = the pair's leader
+  constexpr int UNIT = BM * CG;                                    // channels per tile
+  const int n_o = (p.N + UNIT - 1) / UNIT;
   const int n_tiles = n_o * ((p.T + BN - 1) / BN);
   const int nkb = (p.K + BK - 1) / BK;
+  const int tile0 = (int)blockIdx.x / CG, tstep = (int)gridDim.x / CG;
 
   auto bar = [&](int i) { return dev::smem_u32(&bars[i]); };
   auto xfull_bar = [&](int s) { return bar(s); };
@@ -255,6 +277,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   auto x_stage = [&](int s) { return smem + C::OFF_X + s * C::XT; };
   auto p_stage = [&](int s) { return smem + C::OFF_P + s * C::P_STAGE; };
   auto conv_stage = [&](int c) { return smem + C::OFF_CONV + c * C::CONV_STAGE; };
+  // the leader's copy of one of this CTA's barriers, as a cluster address
+  auto lead = [&](uint32_t a) { return CG == 2 ? dev::map_to_cta(a, 0) : a; };
+  // arrive on the leader's copy of a barrier (a plain local arrive when CG = 1)
+  auto arrive_lead = [&](uint32_t a) {
+    if constexpr (CG == 2)
+      dev::mbar_arrive_cluster(lead(a));
+    else
+      dev::mbar_arrive(a);
+  };
 
   if (tid == 0) {
     for (int s = 0; s < SX; ++s) {
@@ -263,30 +294,41 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     for (int s = 0; s < SP; ++s) {
       dev::mbar_init(pfull_bar(s), 1);
-      dev::mbar_init(pempty_bar(s), NCONV);
+      dev::mbar_init(pempty_bar(s), NCG / 32);   // one arrive per converter warp
     }
     for (int c = 0; c < S2; ++c) {
-      dev::mbar_init(wready_bar(c), NCONV);
+      dev::mbar_init(wready_bar(c), CG * (NCG / 32));   // one arrive per converter warp
       dev::mbar_init(wfree_bar(c), 1);
     }
     for (int b = 0; b < 2; ++b) {
       dev::mbar_init(tfull_bar(b), 1);
-      dev::mbar_init(tempty_bar(b), NEPI);
+      dev::mbar_init(tempty_bar(b), CG * (NEPI / 32));  // one arrive per epilogue warp
     }
     dev::mbar_init(drain_bar, 1);
     s_misc[1] = 0;
-    dev::fence_mbar_init();
+    if constexpr (CG == 2)
+      dev::fence_mbar_init_cluster();
+    else
+      dev::fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
     dev::prefetch_tmap(&tm_x);
     dev::prefetch_tmap(&tm_w);
   }
   if (warp == 1) {
-    dev::tmem_alloc(dev::smem_u32(&s_misc[0]), 2 * BN);
-    dev::tmem_relinquish();
+    if constexpr (CG == 2) {
+      dev::tmem_alloc_pair(dev::smem_u32(&s_misc[0]), 2 * BN);
+      dev::tmem_relinquish_pair();
+    } else {
+      dev::tmem_alloc(dev::smem_u32(&s_misc[0]), 2 * BN);
+      dev::tmem_relinquish();
+    }
   }
   dev::tc_fence_before();
-  __syncthreads();
+  if constexpr (CG == 2)
+    dev::cluster_sync();  // barrier inits of both CTAs visible before any remote arrive
+  else
+    __syncthreads();
   dev::tc_fence_after();
   const uint32_t tmem = s_misc[0];
 
@@ -300,8 +342,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const int ns = packed_role ? SP : SX;
       uint32_t j = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x) {
-        const int o0 = (tile % n_o) * BM, t0 = (tile / n_o) * BN;
+      for (int tile = tile0; ok && tile < n_tiles; tile += tstep) {
+        const int o0 = (tile % n_o) * UNIT + (int)rank * BM;   // this CTA's weight rows
+        const int t0 = (tile / n_o) * BN + (int)rank * XR;     // this CTA's activation rows
         const int krot = k_rotation(tile, n_o, nkb);
         for (int step = 0; step < nkb; ++step, ++j) {
           const int kb = (step + krot) % nkb;
@@ -320,13 +363,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             dev::tma_load_2d(dev::smem_u32(st + C::XP), &tm_w, kb * (BK / 2), o0, full_b);
             if constexpr (C::XPACK)
               dev::tma_load_2d(dev::smem_u32(st), &tm_x, kb * (BK / 2), t0, full_b);
+          } else if constexpr (CG == 2) {
+            // both halves complete on the leader's barrier, which expects the bytes of both
+            if (rank == 0) dev::mbar_arrive_expect_tx(full_b, (uint32_t)(2 * C::XT));
+            dev::tma_load_2d_pair(dev::smem_u32(x_stage(s)), &tm_x, kb * BK, t0, lead(full_b));
           } else {
             dev::mbar_arrive_expect_tx(full_b, (uint32_t)C::XT);
             dev::tma_load_2d(dev::smem_u32(x_stage(s)), &tm_x, kb * BK, t0, full_b);
           }
         }
       }
-      if (!ok) {  // let the loads already issued land before the block can exit
+      // let the loads already issued land before the block can exit (activation loads of a
+      // pair complete on the leader's barriers, so only the leader can watch them)
+      if (!ok && (packed_role || rank == 0)) {
         for (uint32_t i = (j >= (uint32_t)ns ? j - ns : 0); i < j; ++i)
           dev::mbar_wait(packed_role ? pfull_bar(i % ns) : xfull_bar(i % ns), (i / ns) & 1u, p.err,
                          kSiteGemmDrain, p.limit_ns);
@@ -334,12 +383,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
-    if (lane == 0) {
+    if (lane == 0 && rank == 0) {
       constexpr uint32_t idesc =
-          (KIND == kGemmLloydMax) ? dev::idesc_f16(BM, BN) : dev::idesc_i8(BM, BN);
+          (KIND == kGemmLloydMax) ? dev::idesc_f16(UNIT, BN) : dev::idesc_i8(UNIT, BN);
+      auto commit = [&](uint32_t bar) {
+        if constexpr (CG == 2)
+          dev::mma_commit_pair(bar);
+        else
+          dev::mma_commit(bar);
+      };
       uint32_t j = 0, it = 0;
       bool ok = true, issued = false;
-      for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x, ++it) {
+      for (int tile = tile0; ok && tile < n_tiles; tile += tstep, ++it) {
         const int b = it & 1;
         if (*s_abort || !dev::mbar_wait(tempty_bar(b), ((it >> 1) & 1u) ^ 1u, p.err,
                                         kSiteGemmAccum, p.limit_ns)) {
@@ -371,39 +426,48 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           for (int kk = 0; kk < 4; ++kk) {
             const uint64_t ad = dev::sdesc_sw128(aw + kk * 32);
             const uint64_t bd = dev::sdesc_sw128(bx + kk * 32);
-            if constexpr (KIND == kGemmLloydMax)
-              dev::mma_f16(dt, ad, bd, idesc, (step | kk) != 0);
-            else
-              dev::mma_i8(dt, ad, bd, idesc, (step | kk) != 0);
+            if constexpr (CG == 2) {
+              if constexpr (KIND == kGemmLloydMax)
+                dev::mma_f16_pair(dt, ad, bd, idesc, (step | kk) != 0);
+              else
+                dev::mma_i8_pair(dt, ad, bd, idesc, (step | kk) != 0);
+            } else {
+              if constexpr (KIND == kGemmLloydMax)
+                dev::mma_f16(dt, ad, bd, idesc, (step | kk) != 0);
+              else
+                dev::mma_i8(dt, ad, bd, idesc, (step | kk) != 0);
+            }
           }
           issued = true;
-          dev::mma_commit(wfree_bar(c));
-          if constexpr (!C::XPACK) dev::mma_commit(xempty_bar(sx));
+          commit(wfree_bar(c));
+          if constexpr (!C::XPACK) commit(xempty_bar(sx));
         }
         if (!ok) break;
-        dev::mma_commit(tfull_bar(b));
+        commit(tfull_bar(b));
       }
       if (!ok && issued) {  // wait for the MMAs in flight before TMEM is freed
-        dev::mma_commit(drain_bar);
+        commit(drain_bar);
         dev::mbar_wait(drain_bar, 0, p.err, kSiteGemmDrain, p.limit_ns);
       }
     }
   } else if (tid < EPI0) {
     // ---------------- converters ----------------
-    const int ctid = tid - CONV0;
+    const int grp = (tid - CONV0) / NCG, ctid = (tid - CONV0) % NCG;
     uint32_t lut[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) lut[i] = p.lut[i];
     uint32_t j = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x) {
+    for (int tile = tile0; ok && tile < n_tiles; tile += tstep) {
       for (int step = 0; step < nkb; ++step, ++j) {
+        if ((int)(j % NGROUP) != grp) continue;
         const int s = j % SP, c = j % S2;
         bool w = !*s_abort &&
                  dev::mbar_wait(pfull_bar(s), (j / SP) & 1u, p.err, kSiteGemmFull, p.limit_ns);
         if (w)
           w = dev::mbar_wait(wfree_bar(c), ((j / S2) & 1u) ^ 1u, p.err, kSiteGemmConv,
                              p.limit_ns);
+        w = __all_sync(0xffffffffu, w);  // one verdict per warp: its lanes meet in __syncwarp
         if (!w) {
           give_up();
           ok = false;
@@ -413,14 +477,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         uint8_t* cv = conv_stage(c);
         if constexpr (KIND == kGemmLloydMax) {
           convert_i4_f16<BM>(st + C::XP, cv, ctid);
-          convert_lm_f16<BN>(st, cv + C::WT, ctid, lut);
+          convert_lm_f16<XR>(st, cv + C::WT, ctid, lut);
         } else {
           convert_i4_i8<BM>(st + C::XP, cv, ctid);
-          if constexpr (KIND == kGemmA4) convert_i4_i8<BN>(st, cv + C::WT, ctid);
+          if constexpr (KIND == kGemmA4) convert_i4_i8<XR>(st, cv + C::WT, ctid);
         }
-        dev::fence_async_smem();
-        dev::mbar_arrive(wready_bar(c));
-        dev::mbar_arrive(pempty_bar(s));
+        dev::fence_async_smem();  // this thread's tiles -> visible to the tensor cores
+        __syncwarp();             // the warp's reads of the packed stage and writes are done
+        if (lane == 0) {
+          dev::mbar_arrive(pempty_bar(s));
+          arrive_lead(wready_bar(c));
+        }
       }
     }
   } else {
@@ -432,12 +499,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int q = warp & 3;              // TMEM lane quarter of this warp
     const int half = etid >> 7;          // the two warps of a quarter split the columns
     const int o_local = q * 32 + lane;
-    const bool leader = etid == 0;
+    const bool ep_lead = etid == 0;
     constexpr int COLS = BN / 2;
     uint32_t it = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x, ++it) {
-      const int o0 = (tile % n_o) * BM, t0 = (tile / n_o) * BN;
+    for (int tile = tile0; ok && tile < n_tiles; tile += tstep, ++it) {
+      const int o0 = (tile % n_o) * UNIT + (int)rank * BM, t0 = (tile / n_o) * BN;
       const int b = it & 1;
       const int o = o0 + o_local;
       const bool has_o = o < p.N;
@@ -451,7 +518,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       // one thread waits for the accumulator; the verdict reaches all four warps through
       // shared memory behind a named barrier, so every later barrier is reached uniformly
-      if (leader) {
+      if (ep_lead) {
         const bool ready = !*s_abort && dev::mbar_wait(tfull_bar(b), (it >> 1) & 1u, p.err,
                                                        kSiteGemmAccum, p.limit_ns);
         if (!ready) give_up();
@@ -467,9 +534,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         uint32_t r[32];
         dev::tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * BN + c * 32), r);
         dev::tmem_wait_ld();
-        if (cc == COLS / 32 - 1) {  // this thread's part of the accumulator is read
+        if (cc == COLS / 32 - 1) {  // this warp's part of the accumulator is read
           dev::tc_fence_before();
-          dev::mbar_arrive(tempty_bar(b));
+          __syncwarp();
+          if (lane == 0) arrive_lead(tempty_bar(b));
         }
         if (!has_o) continue;
         if (p.out_acc) {
@@ -496,10 +564,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   }
 
   dev::tc_fence_before();
-  __syncthreads();
+  if constexpr (CG == 2)
+    dev::cluster_sync();  // no MMA, remote arrive or TMEM read of either CTA is still pending
+  else
+    __syncthreads();
   if (warp == 1) {
     dev::tc_fence_after();
-    dev::tmem_dealloc(tmem, 2 * BN);
+    if constexpr (CG == 2)
+      dev::tmem_dealloc_pair(tmem, 2 * BN);
+    else
+      dev::tmem_dealloc(tmem, 2 * BN);
   }
 }
 
@@ -544,28 +618,77 @@ int sm_count() {
   return n > 0 ? n : 148;
 }
 
-template <int KIND, int BN>
+// Clusters of two CTAs that can be resident at once for a kernel and its shared memory (0 if
+// the query fails), computed once per kernel and device.
+int active_pairs(const void* kern, size_t smem) {
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, int> cache;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = cache.find({kern, dev});
+  if (it != cache.end()) return it->second;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(2 * (unsigned)sm_count());
+  cfg.blockDim = dim3(NTHREADS);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  cache[{kern, dev}] = n;
+  return n;
+}
+
+template <int KIND, int BN, int CG>
 oq_status run(const GemmArgs& g, const GemmParams& p, cudaStream_t s) {
-  using C = Cfg<KIND, BN>;
+  using C = Cfg<KIND, BN, CG>;
   constexpr int BK = C::BK;
   CUtensorMap tx, tw;
   bool ok = true;
   if constexpr (C::XPACK)
     ok &= make_map_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.a, (uint64_t)g.K / 2, (uint64_t)g.T,
-                      (uint64_t)g.K / 2, BK / 2, BN, CU_TENSOR_MAP_SWIZZLE_NONE);
+                      (uint64_t)g.K / 2, BK / 2, C::XR, CU_TENSOR_MAP_SWIZZLE_NONE);
   else
     ok &= make_map_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.a, (uint64_t)g.K, (uint64_t)g.T,
-                      (uint64_t)g.K, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B);
+                      (uint64_t)g.K, BK, C::XR, CU_TENSOR_MAP_SWIZZLE_128B);
   ok &= make_map_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.w, (uint64_t)g.K / 2, (uint64_t)g.N,
                     (uint64_t)g.K / 2, BK / 2, BM, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (!ok) return fail(OQ_ERR_CUDA, "cuTensorMapEncodeTiled failed or unavailable");
 
-  auto kern = &k_gemm<KIND, BN>;
+  auto kern = &k_gemm<KIND, BN, CG>;
   const cudaError_t attr_err = allow_max_dynamic_smem(reinterpret_cast<const void*>(kern));
   if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute(gemm)");
-  const int64_t tiles = ((g.N + BM - 1) / BM) * ((g.T + BN - 1) / BN);
-  const int grid = (int)std::min<int64_t>(tiles, sm_count());
-  kern<<<grid, NTHREADS, C::SMEM, s>>>(tx, tw, p);
+  const int64_t tiles = ((g.N + BM * CG - 1) / (BM * CG)) * ((g.T + BN - 1) / BN);
+  if constexpr (CG == 1) {
+    const int grid = (int)std::min<int64_t>(tiles, sm_count());
+    kern<<<grid, NTHREADS, C::SMEM, s>>>(tx, tw, p);
+  } else {
+    const int pairs = active_pairs(reinterpret_cast<const void*>(kern), C::SMEM);
+    if (pairs <= 0) return fail(OQ_ERR_UNSUPPORTED, "gemm: no CTA pair fits on this device");
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)(2 * std::min<int64_t>(tiles, pairs)));
+    cfg.blockDim = dim3(NTHREADS);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t le = cudaLaunchKernelEx(&cfg, kern, tx, tw, p);
+    if (le != cudaSuccess) return cuda_fail(le, "launch gemm (CTA pairs)");
+  }
   cudaError_t ce = cudaGetLastError();
   if (ce != cudaSuccess) return cuda_fail(ce, "launch gemm");
   return OQ_OK;
@@ -604,12 +727,13 @@ oq_status launch_gemm(const GemmArgs& g, cudaStream_t s) {
   p.err = device_error_word();
   if (!p.err) return fail(OQ_ERR_CUDA, "device error word unavailable");
   p.limit_ns = kWaitLimitNs;
+  // up to 128 tokens: one CTA per 128 x 128 tile; beyond: CTA pairs on 256 x 256 tiles
   const bool small = g.T <= 128;
   switch (g.kind) {
-    case kGemmA8: return small ? run<kGemmA8, 128>(g, p, s) : run<kGemmA8, 256>(g, p, s);
-    case kGemmA4: return small ? run<kGemmA4, 128>(g, p, s) : run<kGemmA4, 256>(g, p, s);
+    case kGemmA8: return small ? run<kGemmA8, 128, 1>(g, p, s) : run<kGemmA8, 256, 2>(g, p, s);
+    case kGemmA4: return small ? run<kGemmA4, 128, 1>(g, p, s) : run<kGemmA4, 256, 2>(g, p, s);
     case kGemmLloydMax:
-      return small ? run<kGemmLloydMax, 128>(g, p, s) : run<kGemmLloydMax, 256>(g, p, s);
+      return small ? run<kGemmLloydMax, 128, 1>(g, p, s) : run<kGemmLloydMax, 256, 2>(g, p, s);
     default: return fail(OQ_ERR_INVALID_ARG, "unknown GEMM kind");
   }
 }

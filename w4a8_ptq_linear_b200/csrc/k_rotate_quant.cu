@@ -443,9 +443,409 @@ __global__ void __launch_bounds__(MAXT, 1) k_rotate_quant(const RqParams p) {
   }
 }
 
+
+// ================================================================================================
+// Two tokens per pass (widths up to 8192). Every value is a float2 holding the same rotated
+// position of tokens A and B, so all butterflies, the centering and the rounding FMAs run as
+// packed f32x2 operations, and one shared-memory gather fetches both tokens: a coalesced pass
+// applies the source-side signs and interleaves the two bf16 rows into one 32-bit word per
+// channel (A in the low half, B in the high half).
+// ================================================================================================
+
+template <int BIT>
+__device__ __forceinline__ void stage_pair(float2 (&v)[EP]) {
+  constexpr int L = 1 << BIT;
+  const float2 m1 = make_float2(-1.f, -1.f);
+#pragma unroll
+  for (int k = 0; k < EP; ++k) {
+    if (!(k & L)) {
+      const float2 a = v[k], b = v[k | L];
+      v[k] = __fadd2_rn(a, b);
+      v[k | L] = __ffma2_rn(b, m1, a);
+    }
+  }
+}
+
+template <int HI>
+__device__ __forceinline__ void reg_stages_pair(float2 (&v)[EP]) {
+  if constexpr (HI > 0) stage_pair<0>(v);
+  if constexpr (HI > 1) stage_pair<1>(v);
+  if constexpr (HI > 2) stage_pair<2>(v);
+  if constexpr (HI > 3) stage_pair<3>(v);
+  if constexpr (HI > 4) stage_pair<4>(v);
+}
+
+// One component (C = 0: token A, 1: token B) of the strided -> consecutive warp transpose used
+// for h >= 256 (same swizzle as the single-token kernel).
+template <int HLOG2, int C>
+__device__ __forceinline__ void transpose_component(float2 (&v)[EP], int lane, float* warp_tile) {
+  constexpr int E2 = 1 << (HLOG2 - 5);
+  const int blk = lane / E2, kB = lane % E2;
+  const int R = (kB >> 2) ^ ((blk * (E2 / 4)) & 7);
+  float* tb = warp_tile + blk * E2 * 32 + (kB & 3);
+  int off[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) off[c] = (R ^ c) << 2;
+#pragma unroll
+  for (int i = 0; i < EP; ++i) {
+    const int ia = i / E2, ib = i % E2;
+    const int ci = (((E2 / 4) * ia) ^ (ib & 7)) & 7;
+    tb[ib * 32 + off[ci]] = C ? v[i].y : v[i].x;
+  }
+  __syncwarp();
+  const int g = (lane & 7) ^ (((lane / E2) * (E2 / 4)) & 7);
+  const float* rb = warp_tile + lane * 32;
+#pragma unroll
+  for (int m = 0; m < 8; ++m) {
+    const float4 q = *reinterpret_cast<const float4*>(rb + ((m ^ g) << 2));
+    if (C) {
+      v[4 * m].y = q.x; v[4 * m + 1].y = q.y; v[4 * m + 2].y = q.z; v[4 * m + 3].y = q.w;
+    } else {
+      v[4 * m].x = q.x; v[4 * m + 1].x = q.y; v[4 * m + 2].x = q.z; v[4 * m + 3].x = q.w;
+    }
+  }
+  __syncwarp();
+}
+
+template <int HLOG2>
+__device__ __forceinline__ void block_transform_pair(float2 (&v)[EP], int lane, float* warp_tile) {
+  if constexpr (HLOG2 <= 5) {
+    reg_stages_pair<HLOG2>(v);
+  } else if constexpr (HLOG2 <= 7) {
+    reg_stages_pair<5>(v);
+#pragma unroll
+    for (int m = 1; m < (1 << (HLOG2 - 5)); m <<= 1) {
+      const float sg = (lane & m) ? -1.f : 1.f;
+      const float2 sgn = make_float2(sg, sg);
+#pragma unroll
+      for (int k = 0; k < EP; ++k) {
+        const float2 o = make_float2(__shfl_xor_sync(0xffffffffu, v[k].x, m),
+                                     __shfl_xor_sync(0xffffffffu, v[k].y, m));
+        v[k] = __ffma2_rn(v[k], sgn, o);  // lower lane: v + o; upper lane: o - v
+      }
+    }
+  } else {
+    reg_stages_pair<HLOG2 - 5>(v);
+    transpose_component<HLOG2, 0>(v, lane, warp_tile);
+    transpose_component<HLOG2, 1>(v, lane, warp_tile);
+    reg_stages_pair<5>(v);
+  }
+}
+
+__device__ __forceinline__ float2 warp_sum_pair(float2 x) {
+#pragma unroll
+  for (int m = 16; m > 0; m >>= 1)
+    x = __fadd2_rn(x, make_float2(__shfl_xor_sync(0xffffffffu, x.x, m),
+                                  __shfl_xor_sync(0xffffffffu, x.y, m)));
+  return x;
+}
+
+// sum of the 8 bf16 values of chunk a (token A) and chunk b (token B), as a float2
+__device__ __forceinline__ float2 chunk_sums(const uint4& a, const uint4& b) {
+  float2 s = make_float2(0.f, 0.f);
+  const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    s = __fadd2_rn(s, make_float2(__uint_as_float(wa[k] << 16), __uint_as_float(wb[k] << 16)));
+    s = __fadd2_rn(s, make_float2(__uint_as_float(wa[k] & 0xFFFF0000u),
+                                  __uint_as_float(wb[k] & 0xFFFF0000u)));
+  }
+  return s;
+}
+
+// low byte of every float of four rounded values, as one word
+__device__ __forceinline__ uint32_t pack4(float a, float b, float c, float e) {
+  return __byte_perm(__byte_perm(byte_of(a), byte_of(b), 0x0040),
+                     __byte_perm(byte_of(c), byte_of(e), 0x0040), 0x5410);
+}
+
+// two's-complement bytes of 8 codes -> 8 nibbles (element 2j in the low nibble of byte j)
+__device__ __forceinline__ uint32_t nibbles8(uint32_t w0, uint32_t w1) {
+  uint32_t a0 = w0 & 0x0F0F0F0Fu, a1 = w1 & 0x0F0F0F0Fu;
+  a0 |= a0 >> 4;
+  a1 |= a1 >> 4;
+  return __byte_perm(a0, a1, 0x6420);
+}
+
+template <int HLOG2, int ROUNDS>
+__global__ void __launch_bounds__(256, 2) k_rotate_quant_pair(const RqParams p) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int d = p.d;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nwarps = blockDim.x >> 5;
+  const int base = tid * EP;
+  const int nact = d / EP;  // threads that own positions
+  const bool active = tid < nact;
+  const uint32_t row_bytes = (uint32_t)d * 2u;
+  const uint32_t row_stride = (row_bytes + 127u) & ~127u;
+  const uint32_t pair_bytes = 2u * row_stride;
+  constexpr int HMODE = HLOG2 <= 5 ? 0 : (HLOG2 <= 7 ? 1 : 2);
+  // [nbuf landing pairs (row A | row B)] [interleaved words, later the transpose tiles]
+  // [round buffer, two rounds only] [reductions, thresholds, barriers]
+  uint8_t* land = smem;
+  uint32_t* wbuf = reinterpret_cast<uint32_t*>(smem + (size_t)p.nbuf * pair_bytes);
+  float2* rbuf = reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(wbuf) + nwarps * 4096);
+  float* red = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(rbuf) +
+                                        (ROUNDS == 2 ? nwarps * 8192 : 0));
+  float* thr = red + 32;                                     // [0,16) sums, [16,32) statistic
+  uint64_t* bars = reinterpret_cast<uint64_t*>(thr + 16);
+  float* warp_tile = reinterpret_cast<float*>(wbuf) + warp * 1024;
+
+  if (tid < 16) thr[tid] = p.thr[tid];
+  if (tid == 0) {
+    for (int b = 0; b < p.nbuf; ++b) dev::mbar_init(dev::smem_u32(&bars[b]), 1);
+    dev::fence_mbar_init();
+  }
+  __syncthreads();
+
+  const int64_t T = p.T;
+  const int64_t NP = (T + 1) / 2;  // token pairs; an odd tail loads its one row twice
+  const int64_t G = gridDim.x;
+  auto issue = [&](int b, int64_t q) {
+    const int64_t ta = 2 * q, tb = (2 * q + 1 < T) ? 2 * q + 1 : 2 * q;
+    const uint32_t bar = dev::smem_u32(&bars[b]);
+    uint8_t* dst = land + (size_t)b * pair_bytes;
+    dev::mbar_arrive_expect_tx(bar, 2u * row_bytes);
+    dev::bulk_g2s(dev::smem_u32(dst), p.x + ta * p.ldx, row_bytes, bar);
+    dev::bulk_g2s(dev::smem_u32(dst + row_stride), p.x + tb * p.ldx, row_bytes, bar);
+  };
+  if (tid == 0)
+    for (int b = 0; b < p.nbuf; ++b)
+      if ((int64_t)blockIdx.x + (int64_t)b * G < NP) issue(b, (int64_t)blockIdx.x + (int64_t)b * G);
+
+  const bool lm = p.mode == kRqLloydMax;
+  const float nrm = p.inv_norm;
+  int it = 0;
+  bool aborted = false;
+  for (int64_t q = blockIdx.x; q < NP; q += G, ++it) {
+    const int b = it % p.nbuf;
+    const int64_t ta = 2 * q;
+    const bool has_b = ta + 1 < T;
+    uint32_t t0[EP / 2];
+#pragma unroll
+    for (int i = 0; i < EP / 2; ++i) t0[i] = 0u;
+    if (active) {
+      const uint4* s0 = reinterpret_cast<const uint4*>(p.tab + base);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint4 w = __ldg(s0 + i);
+        t0[4 * i] = w.x; t0[4 * i + 1] = w.y; t0[4 * i + 2] = w.z; t0[4 * i + 3] = w.w;
+      }
+    }
+    int fail = !dev::mbar_wait(dev::smem_u32(&bars[b]), (uint32_t)(it / p.nbuf) & 1u, p.err,
+                               kSiteRqRow, p.limit_ns);
+
+    // ---- source-side signs, interleave A|B, row sums ----------------------------------
+    float2 psum = make_float2(0.f, 0.f);
+    if (active && !fail) {
+      const uint4* ra = reinterpret_cast<const uint4*>(land + (size_t)b * pair_bytes);
+      const uint4* rb = reinterpret_cast<const uint4*>(land + (size_t)b * pair_bytes + row_stride);
+      uint4* wv = reinterpret_cast<uint4*>(wbuf);
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int c = tid + m * nact;
+        uint4 a = ra[c], bb = rb[c];
+        const uint4 mk = __ldg(p.smask + c);
+        if (p.want_sum) psum = __fadd2_rn(psum, chunk_sums(a, bb));
+        a.x ^= mk.x; a.y ^= mk.y; a.z ^= mk.z; a.w ^= mk.w;
+        bb.x ^= mk.x; bb.y ^= mk.y; bb.z ^= mk.z; bb.w ^= mk.w;
+        // channels 8c..8c+3 -> words 4c..4c+3, channels 8c+4..8c+7 -> words d/2 + 4c..
+        wv[c] = make_uint4(__byte_perm(a.x, bb.x, 0x5410), __byte_perm(a.x, bb.x, 0x7632),
+                           __byte_perm(a.y, bb.y, 0x5410), __byte_perm(a.y, bb.y, 0x7632));
+        wv[d / 8 + c] = make_uint4(__byte_perm(a.z, bb.z, 0x5410), __byte_perm(a.z, bb.z, 0x7632),
+                                   __byte_perm(a.w, bb.w, 0x5410), __byte_perm(a.w, bb.w, 0x7632));
+      }
+    }
+    if (p.want_sum) {
+      psum = warp_sum_pair(psum);
+      if (lane == 0) { red[2 * warp] = psum.x; red[2 * warp + 1] = psum.y; }
+    }
+    fail = __syncthreads_or(fail);
+    if (fail) {
+      aborted = true;
+      break;
+    }
+    // every thread is past its reads of landing pair b: refill it
+    if (tid == 0 && q + (int64_t)p.nbuf * G < NP) issue(b, q + (int64_t)p.nbuf * G);
+
+    // ---- round 1: one gather for both tokens ---------------------------------------------
+    float2 v[EP];
+#pragma unroll
+    for (int i = 0; i < EP; ++i) {
+      const uint32_t w = active ? wbuf[entry(t0, i)] : 0u;
+      v[i] = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+    }
+    float2 mu = make_float2(0.f, 0.f);
+    if (p.want_sum) {
+      float2 sum = make_float2(0.f, 0.f);
+      for (int w = 0; w < nwarps; ++w) sum = __fadd2_rn(sum, make_float2(red[2 * w], red[2 * w + 1]));
+      mu = make_float2(sum.x / (float)d, sum.y / (float)d);
+      if (tid == 0) {
+        if (p.center) { p.mean[ta] = mu.x; if (has_b) p.mean[ta + 1] = mu.y; }
+        if (p.rowsum) { p.rowsum[ta] = sum.x; if (has_b) p.rowsum[ta + 1] = sum.y; }
+      }
+    }
+    if constexpr (HMODE == 2) __syncthreads();  // the transpose tiles reuse the gathered words
+    block_transform_pair<HLOG2>(v, lane, warp_tile);
+    if (p.center && active) {  // centered round = R(x) - mean * R(1)
+      const float2 nm = make_float2(-mu.x, -mu.y);
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        const float4 c1 = __ldg(p.ones + tid * 8 + m);
+        v[4 * m] = __ffma2_rn(make_float2(c1.x, c1.x), nm, v[4 * m]);
+        v[4 * m + 1] = __ffma2_rn(make_float2(c1.y, c1.y), nm, v[4 * m + 1]);
+        v[4 * m + 2] = __ffma2_rn(make_float2(c1.z, c1.z), nm, v[4 * m + 2]);
+        v[4 * m + 3] = __ffma2_rn(make_float2(c1.w, c1.w), nm, v[4 * m + 3]);
+      }
+    }
+
+    // ---- round 2: gather float2 pairs from the swizzled round buffer ----------------------
+    if constexpr (ROUNDS == 2) {
+      if (active) {
+        float4* rv = reinterpret_cast<float4*>(rbuf) + tid * 16;
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+          rv[k ^ (tid & 7)] = make_float4(v[2 * k].x, v[2 * k].y, v[2 * k + 1].x, v[2 * k + 1].y);
+      }
+      uint32_t t1[EP / 2];
+#pragma unroll
+      for (int i = 0; i < EP / 2; ++i) t1[i] = 0u;
+      if (active) {
+        const uint4* s1 = reinterpret_cast<const uint4*>(p.tab + d + base);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint4 w = __ldg(s1 + i);
+          t1[4 * i] = w.x; t1[4 * i + 1] = w.y; t1[4 * i + 2] = w.z; t1[4 * i + 3] = w.w;
+        }
+      }
+      __syncthreads();
+#pragma unroll
+      for (int i = 0; i < EP; ++i) {
+        const uint32_t e = entry(t1, i);
+        const float2 g = active ? rbuf[e & 0x7FFFu] : make_float2(0.f, 0.f);
+        const uint32_t sb = (e & 0x8000u) << 16;
+        v[i] = make_float2(__uint_as_float(__float_as_uint(g.x) ^ sb),
+                           __uint_as_float(__float_as_uint(g.y) ^ sb));
+      }
+      block_transform_pair<HLOG2>(v, lane, warp_tile);
+    }
+
+    // ---- per-token statistics --------------------------------------------------------------
+    float2 st = make_float2(0.f, 0.f);
+    if (lm) {
+#pragma unroll
+      for (int i = 0; i < EP; ++i) st = __ffma2_rn(v[i], v[i], st);
+      st = warp_sum_pair(st);
+    } else {
+#pragma unroll
+      for (int i = 0; i < EP; ++i) {
+        st.x = fmaxf(st.x, fabsf(v[i].x));
+        st.y = fmaxf(st.y, fabsf(v[i].y));
+      }
+      st.x = warp_max(st.x);
+      st.y = warp_max(st.y);
+    }
+    if (lane == 0) { red[16 + 2 * warp] = st.x; red[16 + 2 * warp + 1] = st.y; }
+    __syncthreads();
+    st = make_float2(0.f, 0.f);
+    for (int w = 0; w < nwarps; ++w) {
+      const float sa = red[16 + 2 * w], sb = red[16 + 2 * w + 1];
+      st = lm ? make_float2(st.x + sa, st.y + sb) : make_float2(fmaxf(st.x, sa), fmaxf(st.y, sb));
+    }
+
+    if (p.rotated && active) {
+#pragma unroll
+      for (int tk = 0; tk < 2; ++tk) {
+        if (tk == 1 && !has_b) break;
+        float4* dst = reinterpret_cast<float4*>(p.rotated + (ta + tk) * (int64_t)d + base);
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          const float2 a0 = v[4 * m], a1 = v[4 * m + 1], a2 = v[4 * m + 2], a3 = v[4 * m + 3];
+          dst[m] = tk ? make_float4(a0.y * nrm, a1.y * nrm, a2.y * nrm, a3.y * nrm)
+                      : make_float4(a0.x * nrm, a1.x * nrm, a2.x * nrm, a3.x * nrm);
+        }
+      }
+    }
+
+    // ---- quantize + store ------------------------------------------------------------------
+    uint8_t* codes = reinterpret_cast<uint8_t*>(p.codes);
+    if (lm) {
+      const float sa = fmaxf(sqrtf(st.x * nrm * nrm / (float)d), 1e-10f);
+      const float sb = fmaxf(sqrtf(st.y * nrm * nrm / (float)d), 1e-10f);
+      const float2 mult = make_float2(nrm * __frcp_rn(sa), nrm * __frcp_rn(sb));
+      if (tid == 0) { p.scale[ta] = sa; if (has_b) p.scale[ta + 1] = sb; }
+      if (active) {
+        uint32_t pa[4] = {0u, 0u, 0u, 0u}, pb[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+        for (int i = 0; i < EP; ++i) {
+          const float2 u = __fmul2_rn(v[i], mult);
+          int ca = (u.x > thr[7]) ? 8 : 0, cb = (u.y > thr[7]) ? 8 : 0;
+          ca += (u.x > thr[ca + 3]) ? 4 : 0; cb += (u.y > thr[cb + 3]) ? 4 : 0;
+          ca += (u.x > thr[ca + 1]) ? 2 : 0; cb += (u.y > thr[cb + 1]) ? 2 : 0;
+          ca += (u.x > thr[ca]) ? 1 : 0;     cb += (u.y > thr[cb]) ? 1 : 0;
+          pa[i >> 3] |= (uint32_t)ca << ((i & 7) * 4);
+          pb[i >> 3] |= (uint32_t)cb << ((i & 7) * 4);
+        }
+        *reinterpret_cast<uint4*>(codes + ta * (int64_t)(d / 2) + base / 2) =
+            make_uint4(pa[0], pa[1], pa[2], pa[3]);
+        if (has_b)
+          *reinterpret_cast<uint4*>(codes + (ta + 1) * (int64_t)(d / 2) + base / 2) =
+              make_uint4(pb[0], pb[1], pb[2], pb[3]);
+      }
+    } else {
+      const float qmax = (p.mode == kRqInt8) ? 127.f : 7.f;
+      const float aa = fmaxf(st.x * nrm, 1e-10f), ab = fmaxf(st.y * nrm, 1e-10f);
+      const float2 mult = make_float2(nrm * qmax * __frcp_rn(aa), nrm * qmax * __frcp_rn(ab));
+      if (tid == 0) { p.scale[ta] = aa / qmax; if (has_b) p.scale[ta + 1] = ab / qmax; }
+      if (active) {
+        // fma against 1.5 * 2^23 rounds half-to-even to an integer held in the low mantissa
+        // bits; the low byte of each result is the two's-complement code
+        const float2 magic = make_float2(12582912.f, 12582912.f);
+        uint32_t wa[8], wb[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const float2 r0 = __ffma2_rn(v[4 * k], mult, magic);
+          const float2 r1 = __ffma2_rn(v[4 * k + 1], mult, magic);
+          const float2 r2 = __ffma2_rn(v[4 * k + 2], mult, magic);
+          const float2 r3 = __ffma2_rn(v[4 * k + 3], mult, magic);
+          wa[k] = pack4(r0.x, r1.x, r2.x, r3.x);
+          wb[k] = pack4(r0.y, r1.y, r2.y, r3.y);
+        }
+        if (p.mode == kRqInt8) {
+          uint4* da = reinterpret_cast<uint4*>(codes + ta * (int64_t)d + base);
+          da[0] = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+          da[1] = make_uint4(wa[4], wa[5], wa[6], wa[7]);
+          if (has_b) {
+            uint4* db = reinterpret_cast<uint4*>(codes + (ta + 1) * (int64_t)d + base);
+            db[0] = make_uint4(wb[0], wb[1], wb[2], wb[3]);
+            db[1] = make_uint4(wb[4], wb[5], wb[6], wb[7]);
+          }
+        } else {
+          *reinterpret_cast<uint4*>(codes + ta * (int64_t)(d / 2) + base / 2) =
+              make_uint4(nibbles8(wa[0], wa[1]), nibbles8(wa[2], wa[3]), nibbles8(wa[4], wa[5]),
+                         nibbles8(wa[6], wa[7]));
+          if (has_b)
+            *reinterpret_cast<uint4*>(codes + (ta + 1) * (int64_t)(d / 2) + base / 2) =
+                make_uint4(nibbles8(wb[0], wb[1]), nibbles8(wb[2], wb[3]), nibbles8(wb[4], wb[5]),
+                           nibbles8(wb[6], wb[7]));
+        }
+      }
+    }
+  }
+
+  if (aborted && tid == 0) {
+    for (int k = 0; k < p.nbuf; ++k) {
+      const int j = it + k;
+      if ((int64_t)blockIdx.x + (int64_t)j * G >= NP) break;
+      dev::mbar_wait(dev::smem_u32(&bars[j % p.nbuf]), (uint32_t)(j / p.nbuf) & 1u, p.err,
+                     kSiteRqDrain, p.limit_ns);
+    }
+  }
+}
+
 struct LaunchCfg {
   void* fn = nullptr;
-  int nthr = 0, nbuf = 0, grid_per_sm = 0, mask_smem = 0;
+  int nthr = 0, nbuf = 0, grid_per_sm = 0, mask_smem = 0, pair = 0;
   size_t smem = 0;
 };
 
@@ -476,6 +876,31 @@ void* pick_kernel(int hlog2, bool big, int rounds) {
   return big ? kern_h<1024, 2>(hlog2) : kern_h<256, 2>(hlog2);
 }
 
+template <int HL, int R>
+void* kern_pair() {
+  return reinterpret_cast<void*>(&k_rotate_quant_pair<HL, R>);
+}
+
+template <int R>
+void* kern_pair_h(int hlog2) {
+  switch (hlog2) {
+    case 0: return kern_pair<0, R>();
+    case 1: return kern_pair<1, R>();
+    case 2: return kern_pair<2, R>();
+    case 3: return kern_pair<3, R>();
+    case 4: return kern_pair<4, R>();
+    case 5: return kern_pair<5, R>();
+    case 6: return kern_pair<6, R>();
+    case 7: return kern_pair<7, R>();
+    case 8: return kern_pair<8, R>();
+    case 9: return kern_pair<9, R>();
+    default: return kern_pair<10, R>();
+  }
+}
+
+// widths up to 8192 (at most 256 threads) run two tokens per pass
+constexpr int kPairMaxD = 8192;
+
 }  // namespace
 
 int rq_hmode(int h) { return h <= 32 ? 0 : (h <= 128 ? 1 : 2); }
@@ -489,9 +914,23 @@ int64_t rq_gather_position(int h, int t, int i) {
   return (int64_t)warp * 1024 + (int64_t)blk * h + kB + E2 * ia + 32 * ib;
 }
 
-// Index in the swizzled fp32 round buffer at which rotated position p is stored.
-int rq_round_buffer_index(int p) {
-  const int t = p / EP, m = (p % EP) / 4;
+// Word of the staged input row that holds channel j. The pair kernel keeps channels
+// 8c..8c+3 in words 4c..4c+3 and channels 8c+4..8c+7 in words d/2 + 4c.. (each word carries
+// the channel of both tokens); the single-token kernel reads the bf16 row as it is.
+int rq_round1_index(int d, int j) {
+  if (d > kPairMaxD) return j;
+  return ((j >> 3) << 2) + (j & 3) + ((j & 4) ? d / 2 : 0);
+}
+
+// Index in the swizzled round buffer at which rotated position p is stored: float2 slots
+// swizzled in pairs of positions for the pair kernel, floats swizzled in fours otherwise.
+int rq_round_buffer_index(int d, int p) {
+  const int t = p / EP;
+  if (d <= kPairMaxD) {
+    const int k = (p % EP) / 2;
+    return t * EP + (((k ^ (t & 7)) << 1) | (p & 1));
+  }
+  const int m = (p % EP) / 4;
   return t * EP + (((m ^ (t & 7)) << 2) | (p & 3));
 }
 
@@ -523,6 +962,23 @@ oq_status launch_rotate_quant(const RqArgs& a, cudaStream_t s) {
       cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev_id);
       cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev_id);
       const size_t row_stride = ((size_t)a.d * 2 + 127) & ~(size_t)127;
+      if (a.d <= kPairMaxD) {
+        // nbuf landing pairs, the interleaved words / transpose tiles, the round buffer,
+        // reductions + thresholds + barriers
+        cfg.pair = 1;
+        cfg.nbuf = 1;
+        cfg.smem = (size_t)cfg.nbuf * 2 * row_stride + (size_t)(nthr / 32) * 4096 +
+                   (a.rounds == 2 ? (size_t)(nthr / 32) * 8192 : 0) + 48 * 4 + 16 * 8;
+        cfg.fn = a.rounds == 1 ? kern_pair_h<1>(hlog2) : kern_pair_h<2>(hlog2);
+        cfg.nthr = nthr;
+        ce = allow_max_dynamic_smem(cfg.fn);
+        if (ce != cudaSuccess) return cuda_fail(ce, "cudaFuncSetAttribute(rotate_quant)");
+        int occ = 0;
+        ce = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, cfg.fn, nthr, cfg.smem);
+        if (ce != cudaSuccess) return cuda_fail(ce, "occupancy(rotate_quant)");
+        cfg.grid_per_sm = std::max(occ, 1) * nsm;
+        cache[key] = cfg;
+      } else {
       // fp32 round buffer and transpose tiles (one region when both are needed), both sized
       // in whole warps of 1024 positions
       const size_t warps_bytes = (size_t)(nthr / 32) * 4096;
@@ -545,9 +1001,11 @@ oq_status launch_rotate_quant(const RqArgs& a, cudaStream_t s) {
       if (ce != cudaSuccess) return cuda_fail(ce, "occupancy(rotate_quant)");
       cfg.grid_per_sm = std::max(occ, 1) * nsm;
       cache[key] = cfg;
+      }
     }
   }
-  const int64_t grid = std::min<int64_t>(a.T, (int64_t)cfg.grid_per_sm);
+  const int64_t units = cfg.pair ? (a.T + 1) / 2 : a.T;
+  const int64_t grid = std::min<int64_t>(units, (int64_t)cfg.grid_per_sm);
 
   RqParams p{};
   p.x = reinterpret_cast<const uint16_t*>(a.x);

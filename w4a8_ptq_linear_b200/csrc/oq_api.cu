@@ -205,9 +205,9 @@ oq_status oq_plan_create(oq_plan** out, int d, int h, int rounds, uint64_t seed,
   p->perm.resize((size_t)rounds * d);
   // Gather entries in the order the rotate-quantize kernel consumes them: thread t, register
   // i of round r reads rotated position q = rq_gather_position(h, t, i), i.e. source index
-  // perm_r[q] with sign signs_r[q]. Round 1 reads the bf16 row, so the index is the channel;
-  // round 2 reads the fp32 round buffer, so the index is where that buffer keeps position
-  // perm_r[q].
+  // perm_r[q] with sign signs_r[q]. Round 1 reads the staged row, so the index is where the
+  // kernel keeps that channel; round 2 reads the fp32 round buffer, so the index is where
+  // that buffer keeps position perm_r[q].
   std::vector<uint16_t> tab((size_t)rounds * d);
   for (int r = 0; r < rounds; ++r)
     rpbh_round_tables(d, r, seed, p->signs.data() + (size_t)r * d, p->perm.data() + (size_t)r * d);
@@ -218,7 +218,8 @@ oq_status oq_plan_create(oq_plan** out, int d, int h, int rounds, uint64_t seed,
       for (int i = 0; i < 32; ++i) {
         const int64_t q = rq_gather_position(h, t, i);
         // round 1 carries no sign: it is applied to the source channel (see below)
-        const int src = (r == 0) ? pm[q] : (rq_round_buffer_index(pm[q]) | (sg[q] < 0 ? 0x8000 : 0));
+        const int src = (r == 0) ? rq_round1_index(d, pm[q])
+                                 : (rq_round_buffer_index(d, pm[q]) | (sg[q] < 0 ? 0x8000 : 0));
         tab[(size_t)r * d + (size_t)t * 32 + i] = (uint16_t)src;
       }
     }

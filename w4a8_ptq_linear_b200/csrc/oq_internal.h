@@ -77,9 +77,11 @@ struct RqArgs {
 };
 oq_status launch_rotate_quant(const RqArgs& a, cudaStream_t s);
 // Kernel-order gather table helpers: the row position thread t, register i gathers in a
-// round, and where the fp32 round buffer keeps rotated position p.
+// round, where the staged input row keeps channel j, and where the fp32 round buffer keeps
+// rotated position p (the last two depend on which kernel shape width d uses).
 int64_t rq_gather_position(int h, int t, int i);
-int rq_round_buffer_index(int p);
+int rq_round1_index(int d, int j);
+int rq_round_buffer_index(int d, int p);
 
 // ---- GEMM ----------------------------------------------------------------------------------
 enum GemmKind : int { kGemmA8 = 0, kGemmA4 = 1, kGemmLloydMax = 2 };
