@@ -15,7 +15,9 @@
 //           completions are multicast to both CTAs. Every activation byte that crosses L2 and
 //           shared memory then feeds 256 channels instead of 128.
 //
-// Persistent CTAs (pairs) walk the tiles in channel-fastest order. Warp roles (608 thr):
+// Persistent CTAs (pairs) walk the tiles in channel-fastest order. Warp roles (608 thr; the
+// warp numbers are those of the 4-bit kinds, INT8 activations move the producers to warps 5
+// and 9 and the converters to 0, 2-4, 6-8, 10):
 //   warp 0     packed-operand producer: TMA loads of the packed weight tile (and, for 4-bit
 //              activations, the packed activation tile) into an SP-deep ring that the
 //              converters release as soon as they have unpacked it;
@@ -62,8 +64,12 @@ constexpr int BM = 128;       // output channels per tile (MMA M)
 constexpr int NCONV = 256;    // converter threads (warps 3-10)
 constexpr int NGROUP = 2;     // converter groups; group g converts the k-blocks j = g mod NGROUP
 constexpr int NCG = NCONV / NGROUP;  // threads per converter group
-constexpr int CONV0 = 96;     // first converter thread
-constexpr int NEPI = 256;     // epilogue threads (warps 11-18)
+constexpr int CONV0 = 96;     // threads before the epilogue that are not converters
+#ifndef OQ_GEMM_EPI_WARPS
+#define OQ_GEMM_EPI_WARPS 8
+#endif
+constexpr int NEPI = 32 * OQ_GEMM_EPI_WARPS;  // epilogue threads (warps from 11 on)
+constexpr int EPW = NEPI / 128;               // epilogue warps per TMEM lane quarter
 constexpr int EPI0 = CONV0 + NCONV;  // first epilogue thread
 constexpr int NTHREADS = EPI0 + NEPI;
 
@@ -311,7 +317,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     else
       dev::fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) {
+  // Warp roles. A warp's scheduler is warp % 4. With INT8 activations (light unpacking) the
+  // single MMA thread (warp 1) shares its scheduler only with the two TMA producers (warps 5
+  // and 9) and the two epilogue warps that must read TMEM lane quarter 1, while the eight
+  // converter warps (0, 2-4, 6-8, 10) use the other three schedulers. The 4-bit kinds unpack
+  // both operands and keep their converters (warps 3-10) on all four schedulers.
+  constexpr bool MMA_ALONE = KIND == kGemmA8;
+  constexpr int W_MMA = 1, W_PROD_P = MMA_ALONE ? 5 : 0, W_PROD_X = MMA_ALONE ? 9 : 2;
+  constexpr int W_EPI0 = EPI0 / 32;
+  const bool is_conv = warp < W_EPI0 && warp != W_MMA && warp != W_PROD_P && warp != W_PROD_X;
+  const int conv_idx = warp - (warp > W_MMA) - (warp > W_PROD_P) - (warp > W_PROD_X);
+  if (warp == W_PROD_P && lane == 0) {
     dev::prefetch_tmap(&tm_x);
     dev::prefetch_tmap(&tm_w);
   }
@@ -334,10 +350,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
   auto give_up = [&]() { *s_abort = 1; };
 
-  if (warp == 0 || warp == 2) {
+  if (warp == W_PROD_P || warp == W_PROD_X) {
     // ---------------- producers ----------------
     // warp 0: packed ring (W, and X for 4-bit activations); warp 2: INT8 activation ring
-    const bool packed_role = warp == 0;
+    const bool packed_role = warp == W_PROD_P;
     if (lane == 0 && (packed_role || SX > 0)) {
       const int ns = packed_role ? SP : SX;
       uint32_t j = 0;
@@ -381,7 +397,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                          kSiteGemmDrain, p.limit_ns);
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == W_MMA) {
     // ---------------- MMA issuer ----------------
     if (lane == 0 && rank == 0) {
       constexpr uint32_t idesc =
@@ -450,9 +466,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         dev::mbar_wait(drain_bar, 0, p.err, kSiteGemmDrain, p.limit_ns);
       }
     }
-  } else if (tid < EPI0) {
+  } else if (is_conv) {
     // ---------------- converters ----------------
-    const int grp = (tid - CONV0) / NCG, ctid = (tid - CONV0) % NCG;
+    const int cid = conv_idx * 32 + lane;   // 0 .. NCONV - 1
+    const int grp = cid / NCG, ctid = cid % NCG;
     uint32_t lut[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) lut[i] = p.lut[i];
@@ -497,10 +514,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     // consecutive channels, i.e. 64 (bf16) or 128 (raw accumulator) contiguous bytes.
     const int etid = tid - EPI0;         // 0..255
     const int q = warp & 3;              // TMEM lane quarter of this warp
-    const int half = etid >> 7;          // the two warps of a quarter split the columns
+    const int half = etid >> 7;          // the warps of a quarter split the columns
     const int o_local = q * 32 + lane;
     const bool ep_lead = etid == 0;
-    constexpr int COLS = BN / 2;
+    constexpr int COLS = BN / EPW;
     uint32_t it = 0;
     bool ok = true;
     for (int tile = tile0; ok && tile < n_tiles; tile += tstep, ++it) {
@@ -546,16 +563,25 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           for (int jj = 0; jj < 32; ++jj)
             if (c * 32 + jj < t_end) dst[(int64_t)jj * p.N] = r[jj];
         } else {
+          // two tokens at a time as f32x2: y = acc * (alpha_t s_w) + (mean_t w_1 + b)
           __nv_bfloat16* dst =
               reinterpret_cast<__nv_bfloat16*>(p.out) + (int64_t)(t0 + c * 32) * p.N + o;
+          const float4* tk4 = reinterpret_cast<const float4*>(s_tok + c * 32);
+          const float2 sw2 = make_float2(sw, sw), w12 = make_float2(w1, w1);
+          const float2 bb2 = make_float2(bb, bb);
+          const int n_valid = t_end - c * 32;   // tokens of this chunk inside [0, T)
+          const int64_t ld = p.N;
 #pragma unroll
-          for (int jj = 0; jj < 32; ++jj) {
-            const float2 tk = s_tok[c * 32 + jj];
-            const float acc = (KIND == kGemmLloydMax) ? __uint_as_float(r[jj])
-                                                      : (float)(int32_t)r[jj];
-            if (c * 32 + jj < t_end)
-              dst[(int64_t)jj * p.N] =
-                  __float2bfloat16_rn(fmaf(acc, tk.x * sw, fmaf(tk.y, w1, bb)));
+          for (int jj = 0; jj < 32; jj += 2) {
+            const float4 tk = tk4[jj / 2];    // (alpha, mean) of tokens jj and jj + 1
+            const float2 s2 = __fmul2_rn(make_float2(tk.x, tk.z), sw2);
+            const float2 c2 = __ffma2_rn(make_float2(tk.y, tk.w), w12, bb2);
+            const float2 a2 = (KIND == kGemmLloydMax)
+                                  ? make_float2(__uint_as_float(r[jj]), __uint_as_float(r[jj + 1]))
+                                  : make_float2((float)(int32_t)r[jj], (float)(int32_t)r[jj + 1]);
+            const __nv_bfloat162 y = __float22bfloat162_rn(__ffma2_rn(a2, s2, c2));
+            if (jj < n_valid) dst[(int64_t)jj * ld] = y.x;
+            if (jj + 1 < n_valid) dst[(int64_t)(jj + 1) * ld] = y.y;
           }
         }
       }
