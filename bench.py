@@ -8,6 +8,7 @@ DiT-width W4A8 layer, T = 4096 tokens, d_in = d_out = 3072, block h = 1024, one 
 absmax INT8 activations, INT4 per-channel weights.
 
   python bench.py [--gpus N --steps K --warmup W] [--impl reference] [--workload NAME]
+  python bench.py --sweep      # rotate+quantize bandwidth at every sweep point (one GPU)
 
 Multi-GPU (launched by torchrun, one process per GPU): tokens are independent, so every rank
 runs its own batch with no collective on the data path (weak scaling); the only collectives
@@ -44,10 +45,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic per launch from an ncu capture, valid only for the kernel source it was taken
 # on (sha256 of the .cu file at capture time); null once the kernel has changed.
 NCU_TRAFFIC = {
-    # profiles/k_gemm_dit_w4a8.md: dram read 17.359 MB + write 0.006 MB
-    ("dit_w4a8", "k_gemm"): {"sha": "37195067d55c57cfbe889838ba1f474f2883566e86a789205fadd3e839751ac3", "bytes": 17364224},
-    # profiles/k_rotate_quant_dit_w4a8.md: dram read 25.239 MB + write 0
-    ("dit_w4a8", "k_rotate_quant"): {"sha": "dfa2d41a46719d9468b1d6b86521dcb2c85fd6a0f04fabe5558d3ecb8f91fd48", "bytes": 25239040},
+    # ncu --set full of the CTA-pair kernel: dram read 17.374 MB + write 24.320 MB
+    ("dit_w4a8", "k_gemm"): {"sha": "402528d7ec8390a691189c53177761c6b535dcdc74d45c9685e55c477e83ab4e", "bytes": 41693952},
+    # ncu --set full of the two-token kernel: dram read 25.243 MB + write 0
+    ("dit_w4a8", "k_rotate_quant"): {"sha": "0b7b5e1f15f6098c7567802bbe7e835898250ee0c98ef022d4bec4e3b69953b3", "bytes": 25242880},
 }
 
 
@@ -66,6 +67,10 @@ def parse():
                     help="CPU time budget of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="time rotate+quantize alone at every point of the bandwidth sweep "
+                         "(T x d x h x rounds x output), one JSON line per point")
+    ap.add_argument("--sweep-iters", type=int, default=10)
     return ap.parse_args()
 
 
@@ -76,6 +81,27 @@ def load_peaks():
             d = json.load(f)
         return d, "measured"
     return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---- multi-rank host logic (one process per GPU; each rank runs the whole path on its own
+# shard of independent token batches, so there is no collective on the data path) ----------
+def input_seed(base_seed, rank, r):
+    """Seed of input set r on `rank`: every rank draws different tokens of the same shape."""
+    return base_seed + 1000 * rank + r
+
+
+def max_over_ranks(x, world, dist=None, device=None):
+    """The largest value of the scalar x over all ranks (one all-reduce when world > 1)."""
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank, world, ms):
+    """Units per second of the whole job: every rank processed units_per_rank in at most ms."""
+    return units_per_rank * world / (ms * 1e-3)
 
 
 def sha_of(path):
@@ -237,8 +263,55 @@ def config_of(wl, T, n):
 
 
 # ---- GPU leg ---------------------------------------------------------------------------------
+def run_sweep(args):
+    """Rotate+quantize alone at every sweep point. Inputs are drawn on the device (N(0,1) plus
+    a per-token mean of variance 3, bf16); the L2 is flushed by writing a 256 MB buffer before
+    every timed launch, and each launch is timed by CUDA events on its stream."""
+    import torch
+    import synth
+    import w4a8_ptq_linear_b200 as oq
+    peaks, peak_kind = load_peaks()
+    hbm = peaks["hbm_gbs"]
+    dev = torch.device("cuda", 0)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    gen = torch.Generator(device=dev)
+    for (T, d, h, rounds, act) in synth.sweep_points():
+        plan = oq.Plan(d, h, rounds, seed=0, center=False, act=act)
+        gen.manual_seed(1000003 * T + d)
+        x = (torch.randn((T, d), generator=gen, device=dev) +
+             3.0 ** 0.5 * torch.randn((T, 1), generator=gen, device=dev)).to(torch.bfloat16)
+        codes, scale, _, _ = oq.rotate_quantize(plan, x)
+        times = []
+        for i in range(args.warmup + args.sweep_iters):
+            flush.fill_(i & 0xFF)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            oq.rotate_quantize(plan, x, codes=codes, scale=scale)
+            e1.record()
+            torch.cuda.synchronize()
+            if i >= args.warmup:
+                times.append(e0.elapsed_time(e1))
+        st, code = oq.device_status()
+        if st != 0:
+            raise RuntimeError(f"device status {st} code {code:#x} at sweep point {T, d, h}")
+        ms = sum(times) / len(times)
+        nbytes = T * d * 2 + (T * d if act == "int8_absmax" else T * d // 2) + 4 * T
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        print(json.dumps({"sweep": {"T": T, "d": d, "h": h, "rounds": rounds, "act": act},
+                          "us": ms * 1e3, "gbs": gbs, "frac_hbm": gbs / hbm,
+                          "peak": f"{peak_kind} copy bandwidth {hbm} GB/s",
+                          "l2": "flushed before every launch", "iters": len(times)}),
+              flush=True)
+        del x, codes, scale
+        plan.close()
+    return 0
+
+
 def main():
     args = parse()
+    if args.sweep:
+        return run_sweep(args)
     import synth
     wl = synth.WORKLOADS[args.workload]
     T = args.tokens or wl.T
@@ -277,7 +350,7 @@ def main():
     for r in range(RING):
         xb = synth.make_x(T, wl.d, mean_var=wl.mean_var, heavy_frac=wl.heavy_frac,
                           outliers=wl.outliers, outlier_gain=wl.outlier_gain,
-                          seed=wl.seed + 1000 * rank + r)
+                          seed=input_seed(wl.seed, rank, r))
         if r == 0:
             x_host_bits = xb
         w = to_dev(w_bits)
@@ -345,10 +418,7 @@ def main():
     if st != 0:
         raise RuntimeError(f"device status {st} code {code:#x} after timing")
 
-    t_max = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
-    elapsed_ms = float(t_max.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, world, dist, dev)
     clocks = clk.summary()
 
     # ---- end to end through the public API with host buffers ------------------------------
@@ -376,17 +446,13 @@ def main():
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = torch.tensor([e0.elapsed_time(e1) / args.e2e_steps], dtype=torch.float64,
-                          device=dev)
-    if world > 1:
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
-    e2e_ms = float(e2e_ms.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, world, dist, dev)
     barrier()
 
     # ---- numbers ------------------------------------------------------------------------------
     ops = 2.0 * T * wl.d * wl.n_out
     ms_per_step = elapsed_ms / K
-    value = ops * world / (ms_per_step * 1e-3) / 1e12
+    value = whole_job_rate(ops, world, ms_per_step) / 1e12
     code_bytes = T * wl.d if wl.act == "int8_absmax" else T * wl.d // 2
     rq_bytes = T * wl.d * 2 + code_bytes + 4 * T * (2 if wl.center else 1)
     peaks, peak_kind = load_peaks()
@@ -426,7 +492,7 @@ def main():
         "roofline": dominant, "roofline_other": other,
         "kernel_share": {"k_rotate_quant": rq_ms / (rq_ms + gm_ms),
                          "k_gemm": gm_ms / (rq_ms + gm_ms)},
-        "e2e": {"value": ops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TOPS",
+        "e2e": {"value": whole_job_rate(ops, world, e2e_ms) / 1e12, "unit": "TOPS",
                 "h2d_bytes_per_step": T * wl.d * 2, "d2h_bytes_per_step": T * wl.n_out * 2,
                 "ms_per_step": e2e_ms, "steps": args.e2e_steps},
         "gpu_launches": 2 * K,

@@ -86,6 +86,17 @@ def test_rotate_quantize_matches_oracle(T, d, h, rounds, act, center):
     assert bad == 0, f"{bad} codes differ outside the boundary exemption ({n_ex} exempt)"
 
 
+# Every (width, block, rounds, output) point of the rotate+quantize bandwidth sweep, at a
+# small odd token count (the two-token kernel's tail pass included): the sweep's token counts
+# only change how many passes each CTA makes.
+SWEEP = sorted({(d, h, rounds, act) for (_, d, h, rounds, act) in synth.sweep_points()})
+
+
+@pytest.mark.parametrize("d,h,rounds,act", SWEEP)
+def test_sweep_grid_matches_oracle(d, h, rounds, act):
+    test_rotate_quantize_matches_oracle(9, d, h, rounds, act, False)
+
+
 def test_zero_and_constant_tokens():
     import torch
     import w4a8_ptq_linear_b200 as oq
