@@ -422,28 +422,57 @@ def main():
     clocks = clk.summary()
 
     # ---- end to end through the public API with host buffers ------------------------------
+    # Every step copies its input from pinned host memory, runs oq_linear and copies the
+    # result back. Three streams (host->device, the layer, device->host) and two device buffer
+    # sets let step i's input copy overlap step i-1's layer and step i-2's output copy, as a
+    # serving loop would; events order each buffer's reuse.
+    NB = 2
     x_pin = torch.from_numpy(np.ascontiguousarray(x_host_bits)).view(torch.bfloat16).pin_memory()
-    y_pin = torch.empty((T, wl.n_out), dtype=torch.bfloat16).pin_memory()
+    y_pins = [torch.empty((T, wl.n_out), dtype=torch.bfloat16).pin_memory() for _ in range(NB)]
     s0 = sets[0]
     ws_bytes = plan.workspace_bytes(T)
     workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
-    x_dev = torch.empty_like(s0["x"])
+    x_devs = [torch.empty_like(s0["x"]) for _ in range(NB)]
+    y_devs = [torch.empty_like(s0["y"]) for _ in range(NB)]
+    s_in = torch.cuda.Stream(device=dev)
+    s_out = torch.cuda.Stream(device=dev)
+    ev_in = [torch.cuda.Event() for _ in range(NB)]     # input k copied to the device
+    ev_done = [torch.cuda.Event() for _ in range(NB)]   # layer on buffer set k finished
+    ev_out = [torch.cuda.Event() for _ in range(NB)]    # output k copied to the host
 
-    def e2e_step():
-        x_dev.copy_(x_pin, non_blocking=True)
-        oq.linear(plan, x_dev, s0["wp"], s0["ws"], s0["w1"] if wl.center else None,
-                  workspace=workspace, out=s0["y"], stream=stream)
-        y_pin.copy_(s0["y"], non_blocking=True)
+    def e2e_step(i):
+        k = i % NB
+        s_in.wait_event(ev_done[k])          # step i - NB no longer reads x_devs[k]
+        with torch.cuda.stream(s_in):
+            x_devs[k].copy_(x_pin, non_blocking=True)
+        ev_in[k].record(s_in)
+        stream.wait_event(ev_in[k])
+        stream.wait_event(ev_out[k])         # step i - NB's output has left y_devs[k]
+        oq.linear(plan, x_devs[k], s0["wp"], s0["ws"], s0["w1"] if wl.center else None,
+                  workspace=workspace, out=y_devs[k], stream=stream)
+        ev_done[k].record(stream)
+        s_out.wait_event(ev_done[k])
+        with torch.cuda.stream(s_out):
+            y_pins[k].copy_(y_devs[k], non_blocking=True)
+        ev_out[k].record(s_out)
 
-    for _ in range(3):
-        e2e_step()
+    def drain():
+        for k in range(NB):
+            stream.wait_event(ev_out[k])
+
+    for i in range(3):
+        e2e_step(i)
+    drain()
     torch.cuda.synchronize()
     barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(args.e2e_steps):
-        e2e_step()
+    s_in.wait_stream(stream)
+    s_out.wait_stream(stream)
+    for i in range(args.e2e_steps):
+        e2e_step(i)
+    drain()
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, world, dist, dev)

@@ -31,6 +31,7 @@
 
 #include <algorithm>
 #include <cmath>
+#include <cstring>
 #include <map>
 #include <mutex>
 #include <tuple>
@@ -55,7 +56,7 @@ struct RqParams {
   float* mean;
   float* rotated;
   float* rowsum;
-  float thr[16];
+  float2 cells[32];    // Lloyd-Max code cells (see lm_code)
   float inv_norm;
   unsigned long long* err;
   unsigned long long limit_ns;
@@ -117,6 +118,20 @@ __device__ __forceinline__ uint32_t entry(const uint32_t (&t)[EP / 2], int i) {
 }
 
 __device__ __forceinline__ uint32_t byte_of(float f) { return __float_as_uint(f); }
+
+// Lloyd-Max code of u = z / sigma, i.e. the number of thresholds below u. The 32 cells of width
+// 1/4 over [-4, 4) hold at most one threshold each (the 16-level N(0,1) thresholds are more than
+// 1/4 apart); cell j keeps (its threshold or +inf, the number of thresholds below the cell), so
+// the code is that count plus one comparison. The cell index is floor(4u + 16): 4u + 15.5
+// rounded to an integer by adding 2^23. The count is exact unless u lies within 2^-22 of a
+// cell edge with a threshold between them, i.e. within 2^-22 of a decision boundary. Values
+// outside [-4, 4) clamp to the end cells, which hold no threshold beyond their range.
+__device__ __forceinline__ uint32_t lm_code(float u, const float2* cells) {
+  int j = __float_as_int(fmaf(u, 4.f, 15.5f) + 8388608.f) - 0x4B000000;
+  j = min(max(j, 0), 31);
+  const float2 c = cells[j];
+  return (uint32_t)__float_as_int(c.y) + (u > c.x ? 1u : 0u);
+}
 
 // Block transform of the 32 values a thread holds, for h = 2^HLOG2 in one of three shapes.
 template <int HLOG2>
@@ -192,10 +207,10 @@ __global__ void __launch_bounds__(MAXT, 1) k_rotate_quant(const RqParams p) {
   float* rbuf = reinterpret_cast<float*>(smem + (size_t)p.nbuf * row_stride);
   float* tbuf = kAlias ? rbuf : rbuf + (ROUNDS == 2 ? nwarps * 1024 : 0);
   float* red = tbuf + (HMODE == 2 ? nwarps * 1024 : 0);  // [0,32) sums, [32,64) statistic
+  float2* cells = reinterpret_cast<float2*>(red + 64);     // 32 Lloyd-Max code cells
+  uint64_t* bars = reinterpret_cast<uint64_t*>(red + 128);  // nbuf <= 3 barriers (16 floats)
   // round-1 sign masks, staged in shared memory when they fit beside the row buffers
-  uint4* s_mask = reinterpret_cast<uint4*>(red + 64 + 16 + 16);
-  float* thr = red + 64;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(thr + 16);   // nbuf <= 3 barriers (16 floats)
+  uint4* s_mask = reinterpret_cast<uint4*>(red + 144);
   float* warp_tile = tbuf + warp * 1024;
 
   uint32_t t0[EP / 2], t1[EP / 2];
@@ -217,7 +232,7 @@ __global__ void __launch_bounds__(MAXT, 1) k_rotate_quant(const RqParams p) {
       }
     }
   }
-  if (tid < 16) thr[tid] = p.thr[tid];
+  if (tid < 32) cells[tid] = p.cells[tid];
   const uint4* mask = p.smask;
   if (p.mask_smem) {
     for (int c = tid; c < d / 8; c += blockDim.x) s_mask[c] = __ldg(p.smask + c);
@@ -379,14 +394,8 @@ __global__ void __launch_bounds__(MAXT, 1) k_rotate_quant(const RqParams p) {
       if (active) {
         uint32_t packed[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-        for (int i = 0; i < EP; ++i) {
-          const float u = el(v, i) * mult;
-          int c = (u > thr[7]) ? 8 : 0;
-          c += (u > thr[c + 3]) ? 4 : 0;
-          c += (u > thr[c + 1]) ? 2 : 0;
-          c += (u > thr[c]) ? 1 : 0;
-          packed[i >> 3] |= (uint32_t)c << ((i & 7) * 4);
-        }
+        for (int i = 0; i < EP; ++i)
+          packed[i >> 3] |= lm_code(el(v, i) * mult, cells) << ((i & 7) * 4);
         *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(p.codes) + t * (int64_t)(d / 2) +
                                   base / 2) = make_uint4(packed[0], packed[1], packed[2],
                                                          packed[3]);
@@ -587,11 +596,12 @@ __global__ void __launch_bounds__(256, 2) k_rotate_quant_pair(const RqParams p) 
   float2* rbuf = reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(wbuf) + nwarps * 4096);
   float* red = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(rbuf) +
                                         (ROUNDS == 2 ? nwarps * 8192 : 0));
-  float* thr = red + 32;                                     // [0,16) sums, [16,32) statistic
-  uint64_t* bars = reinterpret_cast<uint64_t*>(thr + 16);
+  // red: [0,16) sums, [16,32) statistic; then 32 Lloyd-Max code cells and the barriers
+  float2* cells = reinterpret_cast<float2*>(red + 32);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(red + 96);
   float* warp_tile = reinterpret_cast<float*>(wbuf) + warp * 1024;
 
-  if (tid < 16) thr[tid] = p.thr[tid];
+  if (tid < 32) cells[tid] = p.cells[tid];
   if (tid == 0) {
     for (int b = 0; b < p.nbuf; ++b) dev::mbar_init(dev::smem_u32(&bars[b]), 1);
     dev::fence_mbar_init();
@@ -779,12 +789,8 @@ __global__ void __launch_bounds__(256, 2) k_rotate_quant_pair(const RqParams p) 
 #pragma unroll
         for (int i = 0; i < EP; ++i) {
           const float2 u = __fmul2_rn(v[i], mult);
-          int ca = (u.x > thr[7]) ? 8 : 0, cb = (u.y > thr[7]) ? 8 : 0;
-          ca += (u.x > thr[ca + 3]) ? 4 : 0; cb += (u.y > thr[cb + 3]) ? 4 : 0;
-          ca += (u.x > thr[ca + 1]) ? 2 : 0; cb += (u.y > thr[cb + 1]) ? 2 : 0;
-          ca += (u.x > thr[ca]) ? 1 : 0;     cb += (u.y > thr[cb]) ? 1 : 0;
-          pa[i >> 3] |= (uint32_t)ca << ((i & 7) * 4);
-          pb[i >> 3] |= (uint32_t)cb << ((i & 7) * 4);
+          pa[i >> 3] |= lm_code(u.x, cells) << ((i & 7) * 4);
+          pb[i >> 3] |= lm_code(u.y, cells) << ((i & 7) * 4);
         }
         *reinterpret_cast<uint4*>(codes + ta * (int64_t)(d / 2) + base / 2) =
             make_uint4(pa[0], pa[1], pa[2], pa[3]);
@@ -968,7 +974,7 @@ oq_status launch_rotate_quant(const RqArgs& a, cudaStream_t s) {
         cfg.pair = 1;
         cfg.nbuf = 1;
         cfg.smem = (size_t)cfg.nbuf * 2 * row_stride + (size_t)(nthr / 32) * 4096 +
-                   (a.rounds == 2 ? (size_t)(nthr / 32) * 8192 : 0) + 48 * 4 + 16 * 8;
+                   (a.rounds == 2 ? (size_t)(nthr / 32) * 8192 : 0) + 96 * 4 + 16 * 8;
         cfg.fn = a.rounds == 1 ? kern_pair_h<1>(hlog2) : kern_pair_h<2>(hlog2);
         cfg.nthr = nthr;
         ce = allow_max_dynamic_smem(cfg.fn);
@@ -983,7 +989,7 @@ oq_status launch_rotate_quant(const RqArgs& a, cudaStream_t s) {
       // in whole warps of 1024 positions
       const size_t warps_bytes = (size_t)(nthr / 32) * 4096;
       // reductions, thresholds, barriers, then the sign masks (2 bytes per channel)
-      size_t fixed = ((a.rounds == 2 || hmode == 2) ? warps_bytes : 0) + 96 * 4;
+      size_t fixed = ((a.rounds == 2 || hmode == 2) ? warps_bytes : 0) + 144 * 4;
       const size_t mask_bytes = (size_t)a.d * 2;
       cfg.mask_smem = fixed + mask_bytes + row_stride <= (size_t)max_smem / 3;
       if (cfg.mask_smem) fixed += mask_bytes;
@@ -1026,8 +1032,23 @@ oq_status launch_rotate_quant(const RqArgs& a, cudaStream_t s) {
   p.mean = a.mean;
   p.rotated = a.rotated;
   p.rowsum = a.rowsum;
-  for (int i = 0; i < 15; ++i) p.thr[i] = a.thr[i];
-  p.thr[15] = INFINITY;
+  if (a.mode == kRqLloydMax) {
+    // cell j covers [-4 + j/4, -4 + (j+1)/4): its threshold (at most one) and the count below
+    for (int j = 0; j < 32; ++j) {
+      const float lo = -4.f + 0.25f * (float)j, hi = lo + 0.25f;
+      int below = 0, inside = 0;
+      float theta = INFINITY;
+      for (int k = 0; k < 15; ++k) {
+        if (a.thr[k] < lo) ++below;
+        else if (a.thr[k] < hi) { theta = a.thr[k]; ++inside; }
+      }
+      if (inside > 1 || a.thr[0] < -4.f || a.thr[14] >= 4.f)
+        return fail(OQ_ERR_UNSUPPORTED, "rotate_quant: codebook thresholds closer than 1/4");
+      float below_bits;
+      std::memcpy(&below_bits, &below, sizeof(float));   // the count, as the bits of .y
+      p.cells[j] = make_float2(theta, below_bits);
+    }
+  }
   p.inv_norm = (float)std::pow(1.0 / std::sqrt((double)a.h), (double)a.rounds);
   p.err = device_error_word();
   if (!p.err) return fail(OQ_ERR_CUDA, "device error word unavailable");
