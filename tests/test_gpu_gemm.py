@@ -16,7 +16,9 @@ from parity import OUT_TOL, absmax_boundary_mask, compare_codes, rel_fro, to_tor
 pytestmark = pytest.mark.gpu
 
 SHAPES = [(64, 256, 256), (200, 384, 272), (513, 3072, 3072), (129, 1920, 1920),
-          (7, 128, 16), (300, 256, 4096)]
+          (7, 128, 16), (300, 256, 4096),
+          # 100 CTA-pair tiles: more than one wave of pairs on a 148-SM part
+          (2560, 1536, 2560)]
 
 
 def _codes(rng, T, K, N, amax):
@@ -59,7 +61,8 @@ def test_w4a4_absmax_accumulators_bit_exact(T, K, N):
     assert np.array_equal(acc.cpu().numpy().astype(np.int64), ref)
 
 
-@pytest.mark.parametrize("T,K,N", [(64, 256, 256), (200, 384, 272), (130, 1920, 1920)])
+@pytest.mark.parametrize("T,K,N", [(64, 256, 256), (200, 384, 272), (130, 1920, 1920),
+                                   (2560, 1536, 2560)])
 def test_lloyd_max_accumulators(T, K, N):
     import torch
     import w4a8_ptq_linear_b200 as oq
