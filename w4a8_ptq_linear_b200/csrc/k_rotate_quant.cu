@@ -1,32 +1,35 @@
 // Fused per-token center + RPBH rotation + scale + quantize (the activation path of CentriQ
 // §4.2 and App. B.2; OrbitQuant PR #25 "Runtime work": the pre-rotation as one kernel).
 //
-// HBM-bound design, one token row (d bf16 values) at a time per CTA:
-//  - Persistent CTAs walk tokens t = blockIdx.x, blockIdx.x + gridDim.x, ...; one thread keeps
-//    whole rows streaming into shared memory with 1-D bulk copies (TMA) nbuf rows ahead.
-//  - Every thread owns 32 rotated positions per round. Its gather entries (source indices,
-//    laid out on the host in the order the thread consumes them) stay in registers for the
-//    whole kernel.
-//  - Round-1 signs are moved to the source side (channel j takes the sign of the rotated
-//    position that gathers it) and applied by one coalesced 16-byte pass over the row in
-//    shared memory, so the random gather is only an index, a 2-byte load and a shift.
+// HBM-bound design; persistent CTAs of d/32 threads, every thread owning 32 rotated positions
+// per round. Two kernel shapes share the building blocks below:
+//  - k_rotate_quant_pair (d <= 8192): one pass handles two tokens. A 1-D bulk copy (TMA) lands
+//    both bf16 rows in shared memory; one coalesced 16-byte pass applies the round-1 signs on
+//    the source side (channel j takes the sign of the rotated position that gathers it) and
+//    interleaves the rows into one 32-bit word per channel, so that one random gather per
+//    position serves both tokens. Every value is then a float2 (token A, token B) and all
+//    butterflies, the centering FMA and the rounding FMA run as packed f32x2 operations.
+//  - k_rotate_quant (wider rows, up to 1024 threads): the same steps one token at a time, the
+//    row streaming 1-3 rows ahead and the signs applied in place.
+// Common steps:
+//  - Gather entries (where the staged row keeps the source of each position) are laid out on
+//    the host in the order the threads consume them.
 //  - Block transform of size h = 2^L in three shapes:
 //      h <= 32        the thread holds whole blocks: L register butterfly stages;
 //      h = 64, 128    the thread holds 32 consecutive positions: 5 register stages, then
 //                     1-2 stages across lanes by shuffles;
-//      h >= 256       the gather fills a strided arrangement (the thread holds one column a of
+//      h >= 256       the gather fills a strided arrangement (the thread holds one column of
 //                     a 32 x (h/32) view of its block), the high bits are transformed in
 //                     registers, one swizzled, bank-conflict-free shared-memory transpose per
-//                     warp brings 32 consecutive positions to each thread, and the low 5 bits
-//                     are transformed in registers.
-//    Butterflies past the first stage run on packed f32x2 adds.
+//                     warp (per token) brings 32 consecutive positions to each thread, and
+//                     the low 5 bits are transformed in registers.
 //  - A second round gathers from an fp32 copy of the first round's output, written in a
 //    swizzled layout whose indices the host folded into the round-2 entries.
-//  - Centering: the same pass sums the row; since a round is linear, the centered first round
-//    is R(x) - mean * R(1), with R(1) (unnormalised) a per-plan constant vector.
+//  - Centering: the interleave / sign pass sums the row; since a round is linear, the centered
+//    first round is R(x) - mean * R(1), with R(1) (unnormalised) a per-plan constant vector.
 //  - Per-token absmax (or sum of squares for Lloyd-Max) by shuffles and one block reduction;
-//    codes are rounded with one FMA against 1.5 * 2^23 and packed with byte permutes into
-//    one or two 16-byte stores per thread.
+//    absmax codes are rounded with one FMA against 1.5 * 2^23 and packed with byte permutes
+//    into 16-byte stores; Lloyd-Max codes come from a 32-cell table (lm_code).
 #include <cuda_bf16.h>
 
 #include <algorithm>
