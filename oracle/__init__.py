@@ -15,7 +15,8 @@ Sources (pages are cited by title and section):
   second independent RPBH round, absmax INT8 at A8, Lloyd-Max codebooks.
 - CentriQ: Calibration-Free Quantization of Diffusion Transformers via Exact Mean Centering
   (§3 "Quantizers", Eq. 1; "Hadamard rotation", Lemma 1; §4.2 "Centering and exact
-  re-injection", Eq. 4, Eq. 5, Eq. 6; App. B.1, B.2 Eq. 9; App. C.5 "Exactness").
+  re-injection", Eq. 4, Eq. 5, Eq. 6; "Scale and grid"; App. B.1, B.2 Eq. 9, B.3 Tab. 3;
+  App. C.5 "Exactness").
 - FLUX.1-schnell-OrbitQuant-W4A4 model card ("Quantization" settings: activation
   normalization epsilon 1e-10, rotation rpbh, rotation seed 0, block-size policy).
 
@@ -24,15 +25,16 @@ Parity status per function is listed in each module header.
 from .rpbh import (splitmix64_at, rpbh_plan, sylvester_hadamard, rotate, unrotate,
                    rpbh_matrix, default_block, default_rounds)
 from .lloyd_max import lloyd_max_gaussian, lloyd_max_mse
-from .quant import (EPS, center, absmax_quantize, lloyd_max_quantize, pack_nibbles,
-                    unpack_nibbles)
+from .quant import (EPS, PCT_RHO, PCT_GAMMA, center, absmax_quantize, lloyd_max_quantize,
+                    percentile_quantize, pack_nibbles, unpack_nibbles)
 from .linear import (quantize_activations, prepare_weights, gemm_int, gemm_lloyd_max,
                      epilogue, linear_forward, linear_unquantized)
 
 __all__ = [
     "splitmix64_at", "rpbh_plan", "sylvester_hadamard", "rotate", "unrotate", "rpbh_matrix",
     "default_block", "default_rounds", "lloyd_max_gaussian", "lloyd_max_mse", "EPS", "center",
-    "absmax_quantize", "lloyd_max_quantize", "pack_nibbles", "unpack_nibbles",
+    "absmax_quantize", "lloyd_max_quantize", "percentile_quantize", "PCT_RHO", "PCT_GAMMA",
+    "pack_nibbles", "unpack_nibbles",
     "quantize_activations", "prepare_weights", "gemm_int", "gemm_lloyd_max", "epilogue",
     "linear_forward", "linear_unquantized",
 ]

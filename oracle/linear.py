@@ -23,7 +23,7 @@ from __future__ import annotations
 
 import numpy as np
 
-from .quant import EPS, center, absmax_quantize, lloyd_max_quantize
+from .quant import EPS, center, absmax_quantize, lloyd_max_quantize, percentile_quantize
 from .rpbh import rotate
 
 QMAX = {"int8_absmax": 127, "int4_absmax": 7}
@@ -46,6 +46,8 @@ def quantize_activations(x: np.ndarray, plan, h: int, act: str, center_tokens: b
         codes, scale = absmax_quantize(z, QMAX[act])
     elif act == "int4_lloydmax":
         codes, scale = lloyd_max_quantize(z, thresholds)
+    elif act == "int4_percentile":
+        codes, scale = percentile_quantize(z, 7)
     else:
         raise ValueError(act)
     return {"rotated": z, "codes": codes, "scale": scale, "mean": mean}

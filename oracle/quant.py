@@ -10,6 +10,11 @@ What the pages fix:
   channels, one scalar stored beside the per-token scale.
 - FLUX.1-schnell-OrbitQuant-W4A4 model card, "Quantization": activation normalization
   epsilon 1e-10.
+- CentriQ §4.2 "Scale and grid" and App. B.3 (Tab. 3): the percentile scale. The spread of the
+  rotated token is sigma_hat = q_rho(|z|) / Phi^-1((1 + rho) / 2), the empirical rho-quantile
+  of the magnitudes over the half-normal quantile, and alpha = gamma * sigma_hat / (2^(b-1) - 1)
+  with rho = 0.9995 and gamma = 2.5591 (Tab. 3; §4.2 rounds it to 2.56), values beyond the
+  range clipping to the end of the grid.
 
 Readings where the pages are open:
 - round() is round-half-to-even; the range is floored at eps: alpha = max(r, eps) / qmax.
@@ -19,17 +24,26 @@ Readings where the pages are open:
   centroid; a tie at a threshold goes to the lower index).
 - 4-bit codes are packed two per byte: element 2j in bits 0-3 of byte j, element 2j+1 in
   bits 4-7. Absmax codes are two's-complement nibbles; Lloyd-Max codes are indices 0..15.
+- The percentile scale's "empirical quantile" is the linear interpolation between order
+  statistics at position rho (n - 1) (NumPy's and PyTorch's default); its range
+  gamma * sigma_hat takes the same eps floor as the absmax range.
 
 Parity: pinned (tests/test_oracle_quant.py): the largest coordinate maps to +-qmax, the
 error bound |z - alpha q| <= alpha / 2, brute-force nearest grid point on small inputs,
 nearest-centroid brute force for Lloyd-Max codes, offset invariance of centered codes
-(CentriQ Eq. 6), pack/unpack round trip and hand-written byte examples.
+(CentriQ Eq. 6), pack/unpack round trip and hand-written byte examples; for the percentile
+scale, the inverse normal CDF against an independent erfc, the quantile against order
+statistics interpolated by hand, sigma_hat of Gaussian tokens against their standard
+deviation, and clipping of outliers.
 """
 from __future__ import annotations
 
 import numpy as np
+from scipy.special import ndtri
 
 EPS = 1e-10
+PCT_RHO = 0.9995      # CentriQ Tab. 3: activation quantile
+PCT_GAMMA = 2.5591    # CentriQ Tab. 3: clip factor gamma*
 
 
 def center(x: np.ndarray):
@@ -56,6 +70,21 @@ def lloyd_max_quantize(z: np.ndarray, thresholds: np.ndarray, eps: float = EPS):
     # number of thresholds strictly below u (searchsorted 'left' counts tau_k < u)
     codes = np.searchsorted(np.asarray(thresholds, dtype=np.float64), u, side="left")
     return codes.astype(np.int64), sigma
+
+
+def percentile_quantize(z: np.ndarray, qmax: int, rho: float = PCT_RHO,
+                        gamma: float = PCT_GAMMA, eps: float = EPS):
+    """Eq. 1 with the percentile range (CentriQ §4.2, App. B.3): (int64 codes, alpha [T]).
+
+    sigma_hat = q_rho(|z|) / Phi^-1((1 + rho) / 2); alpha = max(gamma sigma_hat, eps) / qmax;
+    codes = clip(round(z / alpha), -qmax, qmax).
+    """
+    z = np.asarray(z, dtype=np.float64)
+    q = np.quantile(np.abs(z), rho, axis=1)          # linear between order statistics
+    sigma_hat = q / ndtri((1.0 + rho) / 2.0)
+    alpha = np.maximum(gamma * sigma_hat, eps) / qmax
+    codes = np.clip(np.rint(z / alpha[:, None]), -qmax, qmax).astype(np.int64)
+    return codes, alpha
 
 
 def pack_nibbles(v: np.ndarray) -> np.ndarray:

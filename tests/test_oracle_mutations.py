@@ -109,6 +109,29 @@ def test_lloyd_max_code_mistake_is_caught(monkeypatch):
     assert _fails(TQ.check_lloyd_max_codes, z)
 
 
+def test_percentile_mistakes_are_caught(monkeypatch):
+    z = np.random.default_rng(5).standard_normal((8, 3072)) * 2.0
+    orig = Qm.percentile_quantize
+
+    def no_normalisation(z, qmax, rho=Qm.PCT_RHO, gamma=Qm.PCT_GAMMA, eps=Qm.EPS):
+        q = np.quantile(np.abs(z), rho, axis=1)
+        alpha = np.maximum(gamma * q, eps) / qmax
+        return np.clip(np.rint(z / alpha[:, None]), -qmax, qmax).astype(np.int64), alpha
+
+    def order_statistic(z, qmax, rho=Qm.PCT_RHO, gamma=Qm.PCT_GAMMA, eps=Qm.EPS):
+        q = np.quantile(np.abs(z), rho, axis=1, method="inverted_cdf")
+        alpha = np.maximum(gamma * q / Qm.ndtri((1 + rho) / 2), eps) / qmax
+        return np.clip(np.rint(z / alpha[:, None]), -qmax, qmax).astype(np.int64), alpha
+
+    def no_clip(z, qmax, rho=Qm.PCT_RHO, gamma=Qm.PCT_GAMMA, eps=Qm.EPS):
+        codes, alpha = orig(z, qmax, rho, gamma, eps)
+        return np.rint(z / alpha[:, None]).astype(np.int64), alpha
+
+    for m in (no_normalisation, order_statistic, no_clip):
+        monkeypatch.setattr(Qm, "percentile_quantize", m)
+        assert _fails(TQ.check_percentile, z)
+
+
 def test_lloyd_iteration_mistake_is_caught(monkeypatch, golden_dir):
     def bad(levels=16, tol=1e-15, max_iter=2000):
         c = np.linspace(-2.5, 2.5, levels)

@@ -1,8 +1,11 @@
 """Pins for the oracle's centering, quantizers and nibble packing (CPU only).
 
-CentriQ §3 Eq. 1 (symmetric per-token grid), §4.2 (centering), Eq. 6 (offset invariance);
+CentriQ §3 Eq. 1 (symmetric per-token grid), §4.2 (centering; "Scale and grid": the
+percentile scale), Eq. 6 (offset invariance), App. B.3 Tab. 3 (rho, gamma*);
 OrbitQuant PR #25 (absmax A8, Lloyd-Max below 8 bits).
 """
+import math
+
 import numpy as np
 import pytest
 
@@ -100,3 +103,74 @@ def test_pack_unpack_round_trip():
     assert np.array_equal(Qm.unpack_nibbles(Qm.pack_nibbles(s), signed=True), s)
     u = rng.integers(0, 16, (5, 64))
     assert np.array_equal(Qm.unpack_nibbles(Qm.pack_nibbles(u), signed=False), u)
+
+
+def half_normal_quantile(p):
+    """x with Phi(x) = p, by bisection on Phi(x) = erfc(-x / sqrt 2) / 2 (no SciPy)."""
+    lo, hi = 0.0, 20.0
+    for _ in range(200):
+        mid = (lo + hi) / 2
+        if 0.5 * math.erfc(-mid / math.sqrt(2.0)) < p:
+            lo = mid
+        else:
+            hi = mid
+    return (lo + hi) / 2
+
+
+def check_percentile(z, qmax=7):
+    """The percentile quantizer against its definition written out by hand."""
+    q, alpha = Qm.percentile_quantize(z, qmax)
+    n = z.shape[1]
+    s = np.sort(np.abs(z), axis=1)
+    pos = Qm.PCT_RHO * (n - 1)
+    k = int(math.floor(pos))
+    qv = s[:, k] + (pos - k) * (s[:, min(k + 1, n - 1)] - s[:, k])
+    sigma_hat = qv / half_normal_quantile((1 + Qm.PCT_RHO) / 2)
+    alpha_ref = np.maximum(Qm.PCT_GAMMA * sigma_hat, Qm.EPS) / qmax
+    ok = bool(np.allclose(alpha, alpha_ref, rtol=1e-12, atol=0))
+    # codes: the nearest point of the grid {-qmax..qmax} (values past the range clip)
+    grid = np.arange(-qmax, qmax + 1)
+    dist = np.abs(z[..., None] - alpha[:, None, None] * grid[None, None, :])
+    best = grid[np.argmin(dist, axis=-1)]
+    tie = np.sort(dist, axis=-1)
+    clear = (tie[..., 1] - tie[..., 0]) > 1e-12 * alpha[:, None]
+    ok &= bool(np.all(best[clear] == q[clear]))
+    return ok
+
+
+def test_half_normal_quantile_pin():
+    # the table value of the standard normal 0.99975 quantile, and SciPy agrees with erfc
+    x = half_normal_quantile(0.99975)
+    assert abs(x - 3.4807564) < 1e-6
+    assert abs(Qm.ndtri(0.99975) - x) < 1e-12
+
+
+@pytest.mark.parametrize("n", [256, 1920, 3072, 4096, 30720])
+def test_percentile_quantizer_definition(n):
+    z = np.random.default_rng(n).standard_normal((6, n)) * np.array([[0.5], [1], [2], [3], [7], [1e-3]])
+    assert check_percentile(z)
+
+
+def test_percentile_scale_of_gaussian_tokens():
+    # sigma_hat estimates the standard deviation of a Gaussian token (the Phi^-1 normalisation)
+    rng = np.random.default_rng(3)
+    for sd in (0.1, 1.0, 5.0):
+        z = rng.normal(0, sd, (2, 400000))
+        _, alpha = Qm.percentile_quantize(z, 7)
+        sigma_hat = alpha * 7 / Qm.PCT_GAMMA
+        assert np.all(np.abs(sigma_hat / sd - 1) < 0.04)
+
+
+def test_percentile_clips_outliers():
+    # one huge coordinate moves the quantile by at most one rank of the clean magnitudes (unlike
+    # an absmax range, which it would set) and clips to the end of the grid
+    n = 4096
+    z = np.random.default_rng(4).standard_normal((1, n))
+    s = np.sort(np.abs(z[0]))
+    k = int(math.floor(Qm.PCT_RHO * (n - 1)))
+    z[0, 17] = 1000.0
+    q, a1 = Qm.percentile_quantize(z, 7)
+    quantile = a1[0] * 7 / Qm.PCT_GAMMA * half_normal_quantile((1 + Qm.PCT_RHO) / 2)
+    assert s[k] <= quantile <= s[k + 2]
+    assert q[0, 17] == 7
+    assert q.min() >= -7 and q.max() <= 7
