@@ -32,9 +32,13 @@
  * Data formats:
  *   - activations / weights: bfloat16, row-major [rows, d];
  *   - A8 codes: int8 [T, d];
- *   - 4-bit codes: uint8 [rows, d/2], element 2j in bits 0-3 of byte j and element 2j+1 in
- *     bits 4-7; absmax codes (and weight codes) are two's-complement nibbles in -7..7,
+ *   - 4-bit activation codes: uint8 [rows, d/2], element 2j in bits 0-3 of byte j and
+ *     element 2j+1 in bits 4-7; absmax codes are two's-complement nibbles in -7..7,
  *     Lloyd-Max codes are indices 0..15 into the ascending codebook;
+ *   - prepared INT4 weights (the GEMM layout): uint8 [d_out, d_in/2] of two's-complement
+ *     nibbles in -7..7; every row is split into 16-byte groups, and byte j of group g holds
+ *     element 32g + j in bits 0-3 and element 32g + 16 + j in bits 4-7. The GEMM widens a
+ *     nibble to the int8 16 n by masking alone;
  *   - per-token scale (alpha_t, or sigma_t for Lloyd-Max), per-token mean, per-channel s_w
  *     and w_1: float32;
  *   - bias: bfloat16 [d_out] or NULL;
@@ -150,7 +154,7 @@ oq_status oq_rotate_quantize(const oq_plan* plan, const void* x_bf16, int64_t T,
  * plan's rotation without centering, is quantized to INT4 per output channel
  * (s_w[o] = max|W_R[o,:]| / 7), and w_1[o] = sum_k W[o,k] (fp32, before rotation).
  *   w_bf16    [n_out, ldw] bf16
- *   w_packed  uint8 [n_out, d/2] two's-complement nibbles
+ *   w_packed  uint8 [n_out, d/2] in the GEMM layout (see "Data formats")
  *   w_scale   float [n_out];  w_rowsum float [n_out] */
 oq_status oq_prepare_weights(const oq_plan* plan, const void* w_bf16, int64_t n_out,
                              int64_t ldw, uint8_t* w_packed, float* w_scale,
@@ -161,7 +165,7 @@ oq_status oq_prepare_weights(const oq_plan* plan, const void* w_bf16, int64_t n_
  *   y[t,o]   = bf16( a_scale[t] * w_scale[o] * acc + mean[t] * w_rowsum[o] + bias[o] )
  *   a         int8 [T, d_in]; a_scale float [T]
  *   mean      float [T] or NULL (no rank-1 term; w_rowsum may then be NULL)
- *   w_packed  uint8 [d_out, d_in/2]; w_scale float [d_out]
+ *   w_packed  uint8 [d_out, d_in/2] in the GEMM layout; w_scale float [d_out]
  *   bias_bf16 bf16 [d_out] or NULL
  *   out       bf16 [T, d_out] (OQ_OUT_BF16) or int32 [T, d_out] (OQ_OUT_ACC) */
 oq_status oq_gemm_w4a8(const int8_t* a, const float* a_scale, const float* mean,

@@ -14,6 +14,27 @@ BOUNDARY_REL = 1e-5
 OUT_TOL = 8e-3
 
 
+def pack_w4_gemm(w) -> np.ndarray:
+    """INT4 weight codes [N, K] (-8..7) -> the prepared-weight GEMM layout of include/oq.h:
+    every row in 16-byte groups, byte j of group g holding element 32g + j in bits 0-3 and
+    element 32g + 16 + j in bits 4-7."""
+    w = np.asarray(w, dtype=np.int64)
+    n, k = w.shape
+    if k % 32:
+        raise ValueError("K must be a multiple of 32")
+    g = (w & 0xF).reshape(n, k // 32, 32)
+    return (g[..., :16] | (g[..., 16:] << 4)).reshape(n, k // 2).astype(np.uint8)
+
+
+def unpack_w4_gemm(b) -> np.ndarray:
+    """Inverse of ``pack_w4_gemm``: uint8 [N, K/2] -> signed int64 [N, K]."""
+    b = np.asarray(b, dtype=np.int64)
+    n, kb = b.shape
+    g = b.reshape(n, kb // 16, 16)
+    out = np.concatenate([g & 0xF, (g >> 4) & 0xF], axis=-1).reshape(n, kb * 2)
+    return np.where(out >= 8, out - 16, out)
+
+
 def to_torch_bf16(bits: np.ndarray, device="cuda"):
     import torch
     return torch.from_numpy(np.ascontiguousarray(bits)).view(torch.bfloat16).to(device)

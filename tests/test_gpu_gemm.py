@@ -11,7 +11,8 @@ import pytest
 
 import oracle
 import synth
-from parity import OUT_TOL, absmax_boundary_mask, compare_codes, rel_fro, to_torch_bf16
+from parity import (OUT_TOL, absmax_boundary_mask, compare_codes, pack_w4_gemm, rel_fro,
+                    to_torch_bf16, unpack_w4_gemm)
 
 pytestmark = pytest.mark.gpu
 
@@ -37,7 +38,7 @@ def test_w4a8_accumulators_bit_exact(T, K, N):
     rng = np.random.default_rng(T + K + N)
     a, w = _codes(rng, T, K, N, 127)
     at = torch.from_numpy(a.astype(np.int8)).cuda()
-    wp = torch.from_numpy(oracle.pack_nibbles(w)).cuda()
+    wp = torch.from_numpy(pack_w4_gemm(w)).cuda()
     ones = torch.ones(max(T, N), dtype=torch.float32, device="cuda")
     acc = oq.gemm_w4a8(at, ones[:T], wp, ones[:N], out_kind=oq.OUT_ACC)
     torch.cuda.synchronize()
@@ -53,7 +54,7 @@ def test_w4a4_absmax_accumulators_bit_exact(T, K, N):
     rng = np.random.default_rng(7 * T + K + N)
     a, w = _codes(rng, T, K, N, 7)
     ap = torch.from_numpy(oracle.pack_nibbles(a)).cuda()
-    wp = torch.from_numpy(oracle.pack_nibbles(w)).cuda()
+    wp = torch.from_numpy(pack_w4_gemm(w)).cuda()
     ones = torch.ones(max(T, N), dtype=torch.float32, device="cuda")
     acc = oq.gemm_w4a4(None, "int4_absmax", ap, ones[:T], wp, ones[:N], out_kind=oq.OUT_ACC)
     torch.cuda.synchronize()
@@ -71,7 +72,7 @@ def test_lloyd_max_accumulators(T, K, N):
     w = rng.integers(-7, 8, (N, K))
     plan = oq.Plan(K, 64, 1, act="int4_lloydmax")
     ap = torch.from_numpy(oracle.pack_nibbles(codes)).cuda()
-    wp = torch.from_numpy(oracle.pack_nibbles(w)).cuda()
+    wp = torch.from_numpy(pack_w4_gemm(w)).cuda()
     ones = torch.ones(max(T, N), dtype=torch.float32, device="cuda")
     acc = oq.gemm_w4a4(plan, "int4_lloydmax", ap, ones[:T], wp, ones[:N], out_kind=oq.OUT_ACC)
     acc = acc.cpu().numpy().astype(np.float64)
@@ -107,7 +108,7 @@ def test_epilogue_matches_oracle(kind, with_mean, with_bias):
     mean_t = cuda(mean) if with_mean else None
     w1_t = cuda(w1) if with_mean else None
     bias_t = to_torch_bf16(bias_bits) if with_bias else None
-    wp = cuda(oracle.pack_nibbles(w))
+    wp = cuda(pack_w4_gemm(w))
     if kind == "int8_absmax":
         y = oq.gemm_w4a8(cuda(a.astype(np.int8)), cuda(scale), wp, cuda(s_w), mean=mean_t,
                          w_rowsum=w1_t, bias=bias_t)
@@ -142,7 +143,7 @@ def test_prepare_weights_matches_oracle(n_out, d, h, rounds):
     codes, s_w, w1_ref = oracle.prepare_weights(w, op, h)
     assert np.abs(ws.cpu().numpy() / s_w - 1).max() <= 1e-5
     assert np.all(np.abs(w1.cpu().numpy() - w1_ref) <= 1e-5 * np.abs(w).sum(axis=1))
-    gpu = oracle.unpack_nibbles(wp.cpu().numpy(), signed=True)
+    gpu = unpack_w4_gemm(wp.cpu().numpy())
     ex = absmax_boundary_mask(oracle.rotate(w, op, h), s_w, 7)
     bad, _ = compare_codes(gpu, codes, ex)
     assert bad == 0

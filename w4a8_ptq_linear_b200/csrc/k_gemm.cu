@@ -4,27 +4,32 @@
 // codes below).
 //
 // Orientation: a tile is D[o, t] = sum_k W[o, k] X[t, k] for 128 output channels o per CTA (the
-// MMA's M) and BN tokens t (the MMA's N). The weight operand is the one unpacked on chip, and
+// MMA's M) and N tokens t (the MMA's N). The weight operand is the one unpacked on chip, and
 // the activation tile is shared through L2 by every channel tile of the same token range.
 //
 // Two shapes (template CG):
-//   CG = 1  one CTA per tile of 128 channels x BN tokens (small token counts);
-//   CG = 2  a cluster of two CTAs on neighbouring SMs computes 256 channels x BN tokens with
-//           tcgen05.mma.cta_group::2 (M = 256): each CTA stages and unpacks its own 128 weight
-//           rows and half of the activation tile, and the pair's leader issues the MMAs, whose
-//           completions are multicast to both CTAs. Every activation byte that crosses L2 and
-//           shared memory then feeds 256 channels instead of 128.
+//   CG = 1  one CTA per tile of 128 channels x N <= 128 tokens (small token counts);
+//   CG = 2  a cluster of two CTAs on neighbouring SMs computes 256 channels x N <= 256 tokens
+//           with tcgen05.mma.cta_group::2 (M = 256): each CTA stages and unpacks its own 128
+//           weight rows and half of the activation rows, and the pair's leader issues the MMAs,
+//           whose completions are multicast to both CTAs. Every activation byte that crosses L2
+//           and shared memory then feeds 256 channels instead of 128.
 //
-// Persistent CTAs (pairs) walk the tiles in channel-fastest order. Warp roles (608 thr; the
-// warp numbers are those of the 4-bit kinds, INT8 activations move the producers to warps 5
-// and 9 and the converters to 0, 2-4, 6-8, 10):
+// Schedule: persistent CTAs (pairs) take the tiles round robin in channel-tile-fastest order,
+// so that the pairs running at the same time share activation rows through L2. Tiles are 256
+// (CG = 2) or 128 (CG = 1) tokens wide; only the last token tile of a ragged T is narrower,
+// and its MMAs run with an N cut to the next multiple of 32.
+//
+// Warp roles (608 thr; the warp numbers are those of the 4-bit kinds, INT8 activations move
+// the producers to warps 5 and 9 and the converters to 0, 2-4, 6-8, 10):
 //   warp 0     packed-operand producer: TMA loads of the packed weight tile (and, for 4-bit
-//              activations, the packed activation tile) into an SP-deep ring that the
+//              activations, the packed activation rows) into an SP-deep ring that the
 //              converters release as soon as they have unpacked it;
 //   warp 1     TMEM owner and MMA issuer (one thread of the pair's leader issues tcgen05.mma,
-//              4 per 128-byte K slice, into one of two TMEM accumulators of BN columns);
-//   warp 2     activation producer (INT8 activations only): TMA loads of the activation tile
-//              into an SX-deep ring that only the MMA releases;
+//              4 per 128-byte K slice, into one of two TMEM accumulators of up to 256 columns);
+//   warp 2     activation producer (INT8 activations only): TMA loads of the activation rows
+//              (boxes of 16 rows, exactly the tile's width) into an SX-deep ring that only the
+//              MMA releases;
 //   warps 3-10 converters: packed INT4 weights (and 4-bit activations) -> INT8 / FP16 in the
 //              128-byte-swizzled K-major layout, into an S2-deep ring of operand tiles; two
 //              groups of four warps take alternate K blocks, so that the hand-off latency of
@@ -32,18 +37,25 @@
 //   warps 11-18 epilogue: TMEM -> registers -> alpha_t s_w acc + mean_t w_1 + b -> bf16 ->
 //              coalesced global stores (each warp writes 32 consecutive channels of a token),
 //              while the MMA already accumulates the next tile into the other TMEM buffer.
-// Keeping the large activation tile out of the conversion path matters: its ring slot is held
-// from the TMA issue to the end of its MMA, so the unpacking must not sit in that interval.
 // Barriers: xfull/xempty (activation ring), pfull/pempty (packed ring), wready/wfree
 // (converted operands), tfull/tempty (accumulators). With CG = 2 the barriers the MMA waits on
 // (xfull, wready, tempty) are the leader's: the peer's activation loads complete on the
 // leader's xfull, and its converter and epilogue warps arrive there remotely. All waits are
 // bounded; a wait that gives up records its site, sets an abort flag and the roles drain.
 //
+// Integer widening. The weights arrive in the GEMM layout of the prepared weights: in every
+// 16-byte group of a row, byte j holds element j in its low nibble and element 16 + j in its
+// high nibble. A two's-complement nibble moved to the high half of a byte is the int8 16 n,
+// so a group widens to two 16-byte int8 chunks with one shift and two masks per word. The
+// 4-bit activations (element 2j low, 2j + 1 high in byte j) widen the same way plus two byte
+// permutes. The products are then 16 or 256 times the true ones; the int32 sums stay exact
+// (|16 * 127 * 7| K < 2^31 for K <= 32768) and the epilogue folds 1/16 or 1/256 into its
+// scale, which is exact in floating point.
+//
 // Kinds:
-//   A8       X int8 straight from TMA, W int4 -> int8; tcgen05.mma.kind::i8, exact int32.
-//   A4       X int4 -> int8, W int4 -> int8; kind::i8.
-//   LloydMax X code -> fp16 centroid (register table via prmt), W int4 -> fp16;
+//   A8       X int8 straight from TMA, W int4 -> 16 W int8; tcgen05.mma.kind::i8, exact int32.
+//   A4       X int4 -> 16 X int8, W int4 -> 16 W int8; kind::i8.
+//   LloydMax X code -> fp16 centroid (register table via prmt), W int4 -> 16 W fp16 (exact);
 //            kind::f16 with fp32 accumulation.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -60,7 +72,8 @@
 namespace oq {
 namespace {
 
-constexpr int BM = 128;       // output channels per tile (MMA M)
+constexpr int BM = 128;       // output channels per CTA (MMA M per CTA)
+constexpr int CH = 32;        // tokens per schedule chunk (MMA N granularity)
 constexpr int NCONV = 256;    // converter threads (warps 3-10)
 constexpr int NGROUP = 2;     // converter groups; group g converts the k-blocks j = g mod NGROUP
 constexpr int NCG = NCONV / NGROUP;  // threads per converter group
@@ -73,11 +86,13 @@ constexpr int EPW = NEPI / 128;               // epilogue warps per TMEM lane qu
 constexpr int EPI0 = CONV0 + NCONV;  // first epilogue thread
 constexpr int NTHREADS = EPI0 + NEPI;
 
-template <int KIND, int BN, int CG>
+template <int KIND, int CG>
 struct Cfg {
   static constexpr int BK = (KIND == kGemmLloydMax) ? 64 : 128;   // 128 bytes of K per stage
   static constexpr bool XPACK = KIND != kGemmA8;
-  static constexpr int XR = BN / CG;                               // activation rows per CTA
+  static constexpr int BNMAX = 128 * CG;                           // tokens per tile, at most
+  static constexpr int MAXCH = BNMAX / CH;                         // chunks per tile, at most
+  static constexpr int XR = 128;                                   // activation rows per CTA
   // Ring depths. Loads from L2 take a few thousand cycles, so the packed ring, which the
   // converters free only after unpacking, must cover that latency at the MMA's pace.
   static constexpr int SX = XPACK ? 0 : (CG == 2 ? 5 : 4);         // activation ring (A8)
@@ -92,14 +107,15 @@ struct Cfg {
   static constexpr int OFF_X = 0;
   static constexpr int OFF_P = OFF_X + SX * XT;
   static constexpr int OFF_CONV = OFF_P + SP * P_STAGE;
-  static constexpr int OFF_TOK = OFF_CONV + S2 * CONV_STAGE;       // float2 (scale, mean) [BN]
-  static constexpr int OFF_BAR = OFF_TOK + BN * 8;
+  static constexpr int OFF_TOK = OFF_CONV + S2 * CONV_STAGE;       // float2 (scale, mean)
+  static constexpr int OFF_BAR = OFF_TOK + BNMAX * 8;
   static constexpr int NBAR = 2 * SX + 2 * SP + 2 * S2 + 4 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;                // + slack for alignment
+  // 1/16 per widened INT4 operand (see "Integer widening")
+  static constexpr float ACC_SCALE = KIND == kGemmA4 ? 1.f / 256.f : 1.f / 16.f;
   static_assert(XT % 1024 == 0 && P_STAGE % 1024 == 0 && CONV_STAGE % 1024 == 0 &&
                 XP % 1024 == 0, "operand tiles must stay 1024-byte aligned");
-  static_assert(BN % 64 == 0 && BN <= 256, "MMA N");
   static_assert(SMEM <= 232448, "shared memory");
   static_assert(NGROUP <= S2, "a converter group may run at most one ring phase ahead");
 };
@@ -118,6 +134,33 @@ struct GemmParams {
   unsigned long long limit_ns;
 };
 
+// ---- schedule ----------------------------------------------------------------------------------
+// The tiles of one CTA (pair), round robin over the grid in channel-tile-fastest order, so that
+// the pairs running at the same time share activation rows through L2. A tile is 256 (or 128)
+// tokens of one channel tile; only the last token tile of a ragged T is narrower, and its MMAs
+// run with the narrower N. Every role walks the same sequence.
+template <int MAXCH>
+struct TileIter {
+  int tile, n_tiles, step, n_o, cpm;
+  __device__ TileIter(int T, int n_o_, int unit_index, int n_units) {
+    cpm = (T + CH - 1) / CH;
+    n_o = n_o_;
+    n_tiles = n_o * ((cpm + MAXCH - 1) / MAXCH);
+    tile = unit_index;
+    step = n_units;
+  }
+  // channel tile m, first token t0, chunks of 32 tokens nch of the next tile
+  __device__ bool next(int& m, int& t0, int& nch) {
+    if (tile >= n_tiles) return false;
+    m = tile % n_o;
+    const int tt = tile / n_o;
+    t0 = tt * MAXCH * CH;
+    nch = min(MAXCH, cpm - tt * MAXCH);
+    tile += step;
+    return true;
+  }
+};
+
 // ---- converters --------------------------------------------------------------------------
 // prmt.b32 in its default mode: selector bit 3 replicates the sign of the chosen byte
 // (CUDA's __byte_perm only honours the low 3 bits of each selector nibble).
@@ -127,32 +170,12 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   return d;
 }
 
-// 8 two's-complement nibbles (element 2j low, 2j+1 high in byte j) -> 8 int8.
-__device__ __forceinline__ void nib8_to_i8(uint32_t w, uint32_t& o0, uint32_t& o1) {
-  uint32_t lo = (w & 0x0F0F0F0Fu) ^ 0x08080808u;
-  uint32_t hi = ((w >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
-  lo = (lo + 0x78787878u) ^ 0x80808080u;     // per-byte sign extension, no carries
-  hi = (hi + 0x78787878u) ^ 0x80808080u;
+// 8 two's-complement nibbles (element 2j low, 2j+1 high in byte j) -> 8 int8 of 16 n.
+__device__ __forceinline__ void nib8_to_i8x16(uint32_t w, uint32_t& o0, uint32_t& o1) {
+  const uint32_t lo = (w << 4) & 0xF0F0F0F0u;   // 16 * even elements
+  const uint32_t hi = w & 0xF0F0F0F0u;          // 16 * odd elements
   o0 = __byte_perm(lo, hi, 0x5140);
   o1 = __byte_perm(lo, hi, 0x7362);
-}
-
-// 8 two's-complement nibbles -> 8 fp16 (exact): (n ^ 8) | 0x6400 is the half 1024 + n + 8.
-__device__ __forceinline__ void nib8_to_f16(uint32_t w, uint32_t (&o)[4]) {
-  const uint32_t t = w ^ 0x88888888u;
-  const uint32_t h0 = (t & 0x000F000Fu) | 0x64006400u;
-  const uint32_t h1 = ((t >> 4) & 0x000F000Fu) | 0x64006400u;
-  const uint32_t h2 = ((t >> 8) & 0x000F000Fu) | 0x64006400u;
-  const uint32_t h3 = ((t >> 12) & 0x000F000Fu) | 0x64006400u;
-  const uint32_t p[4] = {__byte_perm(h0, h1, 0x5410), __byte_perm(h2, h3, 0x5410),
-                         __byte_perm(h0, h1, 0x7632), __byte_perm(h2, h3, 0x7632)};
-  const __half2 bias = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    __half2 v = *reinterpret_cast<const __half2*>(&p[i]);
-    v = __hsub2(v, bias);
-    o[i] = *reinterpret_cast<uint32_t*>(&v);
-  }
 }
 
 // 4 Lloyd-Max codes (nibbles of s, code 0 in bits 0-3) -> 4 fp16 centroids (2 words).
@@ -171,63 +194,109 @@ __device__ __forceinline__ void lm4_to_f16(uint32_t s, const uint32_t (&lut)[8],
   o1 = __byte_perm(lo, hi, 0x7362);
 }
 
-// Packed INT4 rows of 64 bytes -> int8 rows of 128 bytes in the 128-byte-swizzled layout
-// (16-byte chunk c of row r at r * 128 + ((c ^ (r & 7)) << 4)). Thread ctid of a group takes
-// the 16-byte packed chunk q = ctid & 3 of rows ctid / 4 + (NCG / 4) j; the swizzle phase r & 7
-// is the same for all j, so every address is a constant offset from a per-thread base.
-template <int ROWS>
-__device__ __forceinline__ void convert_i4_i8(const uint8_t* src, uint8_t* dst, int ctid) {
+// Weight rows in the GEMM layout (64 packed bytes = 128 elements per stage) -> int8 rows of
+// 128 bytes in the 128-byte-swizzled layout (16-byte chunk c of row r at
+// r * 128 + ((c ^ (r & 7)) << 4)). Thread ctid of a group takes packed group q = ctid & 3 of
+// rows ctid / 4 + (NCG / 4) j: its low nibbles are chunk 2q, its high nibbles chunk 2q + 1.
+// The swizzle phase r & 7 is the same for all j, so every address is a constant offset from a
+// per-thread base.
+__device__ __forceinline__ void convert_w_i8(const uint8_t* src, uint8_t* dst, int ctid) {
   constexpr int RSTEP = NCG / 4;     // rows covered by one pass of the group's threads
   const int r0 = ctid >> 2, q = ctid & 3;
   const uint8_t* s = src + r0 * 64 + q * 16;
   uint8_t* da = dst + r0 * 128 + (((2 * q) ^ (r0 & 7)) << 4);
   uint8_t* db = dst + r0 * 128 + (((2 * q + 1) ^ (r0 & 7)) << 4);
 #pragma unroll
-  for (int j = 0; j < ROWS / RSTEP; ++j) {
+  for (int j = 0; j < BM / RSTEP; ++j) {
+    const uint4 in = *reinterpret_cast<const uint4*>(s + j * RSTEP * 64);
+    const uint4 lo = make_uint4((in.x << 4) & 0xF0F0F0F0u, (in.y << 4) & 0xF0F0F0F0u,
+                                (in.z << 4) & 0xF0F0F0F0u, (in.w << 4) & 0xF0F0F0F0u);
+    const uint4 hi = make_uint4(in.x & 0xF0F0F0F0u, in.y & 0xF0F0F0F0u, in.z & 0xF0F0F0F0u,
+                                in.w & 0xF0F0F0F0u);
+    *reinterpret_cast<uint4*>(da + j * RSTEP * 128) = lo;
+    *reinterpret_cast<uint4*>(db + j * RSTEP * 128) = hi;
+  }
+}
+
+// 4-bit activation rows (natural nibble order, 64 packed bytes per stage) -> int8 rows, the
+// first `rows` rows (rounded up to a pass of the group).
+__device__ __forceinline__ void convert_x_i8(const uint8_t* src, uint8_t* dst, int ctid, int rows) {
+  constexpr int RSTEP = NCG / 4;
+  const int r0 = ctid >> 2, q = ctid & 3;
+  const uint8_t* s = src + r0 * 64 + q * 16;
+  uint8_t* da = dst + r0 * 128 + (((2 * q) ^ (r0 & 7)) << 4);
+  uint8_t* db = dst + r0 * 128 + (((2 * q + 1) ^ (r0 & 7)) << 4);
+#pragma unroll 1
+  for (int j = 0; j * RSTEP < rows; ++j) {
     const uint4 in = *reinterpret_cast<const uint4*>(s + j * RSTEP * 64);
     uint4 a, b;
-    nib8_to_i8(in.x, a.x, a.y);
-    nib8_to_i8(in.y, a.z, a.w);
-    nib8_to_i8(in.z, b.x, b.y);
-    nib8_to_i8(in.w, b.z, b.w);
+    nib8_to_i8x16(in.x, a.x, a.y);
+    nib8_to_i8x16(in.y, a.z, a.w);
+    nib8_to_i8x16(in.z, b.x, b.y);
+    nib8_to_i8x16(in.w, b.z, b.w);
     *reinterpret_cast<uint4*>(da + j * RSTEP * 128) = a;
     *reinterpret_cast<uint4*>(db + j * RSTEP * 128) = b;
   }
 }
 
-// Packed INT4 rows of 32 bytes (64 elements) -> fp16 rows of 128 bytes, swizzled.
-template <int ROWS>
-__device__ __forceinline__ void convert_i4_f16(const uint8_t* src, uint8_t* dst, int ctid) {
+// Half-precision lane pairs of 16 n from two bytes of a GEMM-layout word (bytes b0, b1 moved
+// to the low byte of each 16-bit lane by prmt): the low nibble n gives the half
+// 1024 + (n + 8) (n xor 8 is n + 8), scaled by 16 and shifted by FMA; the high nibble gives
+// 1024 + 16 (n + 8) directly. Both results are exact.
+__device__ __forceinline__ void w_pair_f16(uint32_t x, uint32_t& lo16, uint32_t& hi16) {
+  const uint32_t l = (x & 0x000F000Fu) ^ 0x64086408u;
+  const uint32_t h = (x & 0x00F000F0u) ^ 0x64806480u;
+  const __half2 sixteen = __halves2half2(__ushort_as_half(0x4C00), __ushort_as_half(0x4C00));
+  const __half2 off_l = __halves2half2(__ushort_as_half(0xF408), __ushort_as_half(0xF408));
+  const __half2 off_h = __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480));
+  __half2 vl = __hfma2(*reinterpret_cast<const __half2*>(&l), sixteen, off_l);  // 16 v - 16512
+  __half2 vh = __hsub2(*reinterpret_cast<const __half2*>(&h), off_h);           // v - 1152
+  lo16 = *reinterpret_cast<uint32_t*>(&vl);
+  hi16 = *reinterpret_cast<uint32_t*>(&vh);
+}
+
+// Weight rows in the GEMM layout (32 packed bytes = 64 elements per stage) -> fp16 rows of 128
+// bytes (16 n), swizzled. Thread ctid takes packed group q = ctid & 1 of its rows: chunks
+// 4q, 4q + 1 hold its low nibbles (elements 0-15 of the group), 4q + 2, 4q + 3 its high ones.
+__device__ __forceinline__ void convert_w_f16(const uint8_t* src, uint8_t* dst, int ctid) {
   constexpr int RSTEP = NCG / 2;
   const int r0 = ctid >> 1, q = ctid & 1;
   const uint8_t* s = src + r0 * 32 + q * 16;
   uint8_t* d = dst + r0 * 128;
   const int ph = r0 & 7;
 #pragma unroll
-  for (int j = 0; j < ROWS / RSTEP; ++j) {
+  for (int j = 0; j < BM / RSTEP; ++j) {
     const uint4 in = *reinterpret_cast<const uint4*>(s + j * RSTEP * 32);
     const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+    uint32_t P[4][2], Q[4][2];   // [word][byte pair]: low-nibble and high-nibble lanes
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      uint32_t o[4];
-      nib8_to_f16(w[k], o);
-      *reinterpret_cast<uint4*>(d + j * RSTEP * 128 + (((4 * q + k) ^ ph) << 4)) =
-          make_uint4(o[0], o[1], o[2], o[3]);
+    for (int m = 0; m < 4; ++m) {
+      w_pair_f16(__byte_perm(w[m], 0u, 0x4140), P[m][0], Q[m][0]);
+      w_pair_f16(__byte_perm(w[m], 0u, 0x4342), P[m][1], Q[m][1]);
     }
+    uint8_t* row = d + j * RSTEP * 128;
+    *reinterpret_cast<uint4*>(row + (((4 * q + 0) ^ ph) << 4)) =
+        make_uint4(P[0][0], P[0][1], P[1][0], P[1][1]);
+    *reinterpret_cast<uint4*>(row + (((4 * q + 1) ^ ph) << 4)) =
+        make_uint4(P[2][0], P[2][1], P[3][0], P[3][1]);
+    *reinterpret_cast<uint4*>(row + (((4 * q + 2) ^ ph) << 4)) =
+        make_uint4(Q[0][0], Q[0][1], Q[1][0], Q[1][1]);
+    *reinterpret_cast<uint4*>(row + (((4 * q + 3) ^ ph) << 4)) =
+        make_uint4(Q[2][0], Q[2][1], Q[3][0], Q[3][1]);
   }
 }
 
-// Lloyd-Max code rows of 32 bytes (64 codes) -> fp16 centroid rows of 128 bytes, swizzled.
-template <int ROWS>
+// Lloyd-Max code rows of 32 bytes (64 codes) -> fp16 centroid rows of 128 bytes, swizzled; the
+// first `rows` rows (rounded up to a pass of the group).
 __device__ __forceinline__ void convert_lm_f16(const uint8_t* src, uint8_t* dst, int ctid,
-                                               const uint32_t (&lut)[8]) {
+                                               const uint32_t (&lut)[8], int rows) {
   constexpr int RSTEP = NCG / 2;
   const int r0 = ctid >> 1, q = ctid & 1;
   const uint8_t* s = src + r0 * 32 + q * 16;
   uint8_t* d = dst + r0 * 128;
   const int ph = r0 & 7;
-#pragma unroll
-  for (int j = 0; j < ROWS / RSTEP; ++j) {
+#pragma unroll 1
+  for (int j = 0; j * RSTEP < rows; ++j) {
     const uint4 in = *reinterpret_cast<const uint4*>(s + j * RSTEP * 32);
     const uint32_t w[4] = {in.x, in.y, in.z, in.w};
 #pragma unroll
@@ -241,19 +310,19 @@ __device__ __forceinline__ void convert_lm_f16(const uint8_t* src, uint8_t* dst,
   }
 }
 
-// First K block of a tile. Tiles that run at the same time and share an activation tile
+// First K block of a tile. Tiles that run at the same time and share an activation range
 // (neighbouring channel tiles) start their K loops at different blocks, so that they do not all
 // request the same L2 lines at the same moment. Integer accumulation is exact in any order.
-__device__ __forceinline__ int k_rotation(int tile, int n_o, int nkb) {
-  return (int)(((unsigned)(tile % n_o) * 7u) % (unsigned)nkb);
+__device__ __forceinline__ int k_rotation(int m, int nkb) {
+  return (int)(((unsigned)m * 7u) % (unsigned)nkb);
 }
 
-template <int KIND, int BN, int CG>
+template <int KIND, int CG>
 __global__ void __launch_bounds__(NTHREADS, 1)
     k_gemm(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
            const GemmParams p) {
-  using C = Cfg<KIND, BN, CG>;
-  constexpr int BK = C::BK, SX = C::SX, SP = C::SP, S2 = C::S2, XR = C::XR;
+  using C = Cfg<KIND, CG>;
+  constexpr int BK = C::BK, SX = C::SX, SP = C::SP, S2 = C::S2, MAXCH = C::MAXCH;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -266,9 +335,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const uint32_t rank = (CG == 2) ? dev::cluster_ctarank() : 0u;  // 0 = the pair's leader
   constexpr int UNIT = BM * CG;                                    // channels per tile
   const int n_o = (p.N + UNIT - 1) / UNIT;
-  const int n_tiles = n_o * ((p.T + BN - 1) / BN);
   const int nkb = (p.K + BK - 1) / BK;
-  const int tile0 = (int)blockIdx.x / CG, tstep = (int)gridDim.x / CG;
+  const int unit_index = (int)blockIdx.x / CG, n_units = (int)gridDim.x / CG;
+  auto tiles = [&]() { return TileIter<MAXCH>(p.T, n_o, unit_index, n_units); };
 
   auto bar = [&](int i) { return dev::smem_u32(&bars[i]); };
   auto xfull_bar = [&](int s) { return bar(s); };
@@ -333,10 +402,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   }
   if (warp == 1) {
     if constexpr (CG == 2) {
-      dev::tmem_alloc_pair(dev::smem_u32(&s_misc[0]), 2 * BN);
+      dev::tmem_alloc_pair(dev::smem_u32(&s_misc[0]), 2 * C::BNMAX);
       dev::tmem_relinquish_pair();
     } else {
-      dev::tmem_alloc(dev::smem_u32(&s_misc[0]), 2 * BN);
+      dev::tmem_alloc(dev::smem_u32(&s_misc[0]), 2 * C::BNMAX);
       dev::tmem_relinquish();
     }
   }
@@ -352,16 +421,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
   if (warp == W_PROD_P || warp == W_PROD_X) {
     // ---------------- producers ----------------
-    // warp 0: packed ring (W, and X for 4-bit activations); warp 2: INT8 activation ring
+    // W_PROD_P: packed ring (W, and X for 4-bit activations); W_PROD_X: INT8 activation ring
     const bool packed_role = warp == W_PROD_P;
     if (lane == 0 && (packed_role || SX > 0)) {
       const int ns = packed_role ? SP : SX;
       uint32_t j = 0;
       bool ok = true;
-      for (int tile = tile0; ok && tile < n_tiles; tile += tstep) {
-        const int o0 = (tile % n_o) * UNIT + (int)rank * BM;   // this CTA's weight rows
-        const int t0 = (tile / n_o) * BN + (int)rank * XR;     // this CTA's activation rows
-        const int krot = k_rotation(tile, n_o, nkb);
+      auto it = tiles();
+      int m, t0, nch;
+      while (ok && it.next(m, t0, nch)) {
+        const int o0 = m * UNIT + (int)rank * BM;          // this CTA's weight rows
+        // this CTA's activation rows start at x0; one box brings XR rows (a narrower last
+        // tile reads rows past it, or past T as zeros, that its MMAs do not use)
+        const int x0 = t0 + (int)rank * (nch * CH / CG);
+        const int krot = k_rotation(m, nkb);
         for (int step = 0; step < nkb; ++step, ++j) {
           const int kb = (step + krot) % nkb;
           const int s = j % ns;
@@ -378,14 +451,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             dev::mbar_arrive_expect_tx(full_b, (uint32_t)C::P_STAGE);
             dev::tma_load_2d(dev::smem_u32(st + C::XP), &tm_w, kb * (BK / 2), o0, full_b);
             if constexpr (C::XPACK)
-              dev::tma_load_2d(dev::smem_u32(st), &tm_x, kb * (BK / 2), t0, full_b);
+              dev::tma_load_2d(dev::smem_u32(st), &tm_x, kb * (BK / 2), x0, full_b);
           } else if constexpr (CG == 2) {
             // both halves complete on the leader's barrier, which expects the bytes of both
             if (rank == 0) dev::mbar_arrive_expect_tx(full_b, (uint32_t)(2 * C::XT));
-            dev::tma_load_2d_pair(dev::smem_u32(x_stage(s)), &tm_x, kb * BK, t0, lead(full_b));
+            dev::tma_load_2d_pair(dev::smem_u32(x_stage(s)), &tm_x, kb * BK, x0, lead(full_b));
           } else {
             dev::mbar_arrive_expect_tx(full_b, (uint32_t)C::XT);
-            dev::tma_load_2d(dev::smem_u32(x_stage(s)), &tm_x, kb * BK, t0, full_b);
+            dev::tma_load_2d(dev::smem_u32(x_stage(s)), &tm_x, kb * BK, x0, full_b);
           }
         }
       }
@@ -400,26 +473,28 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   } else if (warp == W_MMA) {
     // ---------------- MMA issuer ----------------
     if (lane == 0 && rank == 0) {
-      constexpr uint32_t idesc =
-          (KIND == kGemmLloydMax) ? dev::idesc_f16(UNIT, BN) : dev::idesc_i8(UNIT, BN);
       auto commit = [&](uint32_t bar) {
         if constexpr (CG == 2)
           dev::mma_commit_pair(bar);
         else
           dev::mma_commit(bar);
       };
-      uint32_t j = 0, it = 0;
+      uint32_t j = 0, it_n = 0;
       bool ok = true, issued = false;
-      for (int tile = tile0; ok && tile < n_tiles; tile += tstep, ++it) {
-        const int b = it & 1;
-        if (*s_abort || !dev::mbar_wait(tempty_bar(b), ((it >> 1) & 1u) ^ 1u, p.err,
+      auto it = tiles();
+      int m, t0, nch;
+      for (; ok && it.next(m, t0, nch); ++it_n) {
+        const uint32_t idesc = (KIND == kGemmLloydMax) ? dev::idesc_f16(UNIT, nch * CH)
+                                                       : dev::idesc_i8(UNIT, nch * CH);
+        const int b = it_n & 1;
+        if (*s_abort || !dev::mbar_wait(tempty_bar(b), ((it_n >> 1) & 1u) ^ 1u, p.err,
                                         kSiteGemmAccum, p.limit_ns)) {
           give_up();
           ok = false;
           break;
         }
         dev::tc_fence_after();
-        const uint32_t dt = tmem + (uint32_t)(b * BN);
+        const uint32_t dt = tmem + (uint32_t)(b * C::BNMAX);
         for (int step = 0; step < nkb; ++step, ++j) {
           const int c = j % S2;
           const int sx = SX > 0 ? (int)(j % (uint32_t)(SX > 0 ? SX : 1)) : 0;
@@ -475,7 +550,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     for (int i = 0; i < 8; ++i) lut[i] = p.lut[i];
     uint32_t j = 0;
     bool ok = true;
-    for (int tile = tile0; ok && tile < n_tiles; tile += tstep) {
+    auto it = tiles();
+    int m, t0, nch;
+    while (ok && it.next(m, t0, nch)) {
+      const int rows = nch * CH / CG;   // activation rows of this CTA
       for (int step = 0; step < nkb; ++step, ++j) {
         if ((int)(j % NGROUP) != grp) continue;
         const int s = j % SP, c = j % S2;
@@ -493,11 +571,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const uint8_t* st = p_stage(s);
         uint8_t* cv = conv_stage(c);
         if constexpr (KIND == kGemmLloydMax) {
-          convert_i4_f16<BM>(st + C::XP, cv, ctid);
-          convert_lm_f16<XR>(st, cv + C::WT, ctid, lut);
+          convert_w_f16(st + C::XP, cv, ctid);
+          convert_lm_f16(st, cv + C::WT, ctid, lut, rows);
         } else {
-          convert_i4_i8<BM>(st + C::XP, cv, ctid);
-          if constexpr (KIND == kGemmA4) convert_i4_i8<XR>(st, cv + C::WT, ctid);
+          convert_w_i8(st + C::XP, cv, ctid);
+          if constexpr (KIND == kGemmA4) convert_x_i8(st, cv + C::WT, ctid, rows);
         }
         dev::fence_async_smem();  // this thread's tiles -> visible to the tensor cores
         __syncwarp();             // the warp's reads of the packed stage and writes are done
@@ -511,32 +589,35 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     // ---------------- epilogue ----------------
     // Thread (lane quarter q, lane) owns output channel o; a 32-column TMEM load gives it 32
     // consecutive tokens of that channel. For each token the 32 lanes of a warp store 32
-    // consecutive channels, i.e. 64 (bf16) or 128 (raw accumulator) contiguous bytes.
-    const int etid = tid - EPI0;         // 0..255
+    // consecutive channels, i.e. 64 (bf16) or 128 (raw accumulator) contiguous bytes. The
+    // EPW warps of a lane quarter take the tile's 32-column chunks in turn.
+    const int etid = tid - EPI0;         // 0..NEPI-1
     const int q = warp & 3;              // TMEM lane quarter of this warp
-    const int half = etid >> 7;          // the warps of a quarter split the columns
+    const int half = etid >> 7;          // index among the warps of the quarter
     const int o_local = q * 32 + lane;
     const bool ep_lead = etid == 0;
-    constexpr int COLS = BN / EPW;
-    uint32_t it = 0;
+    uint32_t it_n = 0;
     bool ok = true;
-    for (int tile = tile0; ok && tile < n_tiles; tile += tstep, ++it) {
-      const int o0 = (tile % n_o) * UNIT + (int)rank * BM, t0 = (tile / n_o) * BN;
-      const int b = it & 1;
+    auto it = tiles();
+    int m, t0, nch;
+    for (; ok && it.next(m, t0, nch); ++it_n) {
+      const int o0 = m * UNIT + (int)rank * BM;
+      const int b = it_n & 1;
       const int o = o0 + o_local;
       const bool has_o = o < p.N;
-      const float sw = has_o ? p.w_scale[o] : 0.f;
+      const float sw = has_o ? p.w_scale[o] * C::ACC_SCALE : 0.f;
       const float w1 = (has_o && p.mean) ? p.w_rowsum[o] : 0.f;
       const float bb = (has_o && p.bias) ? __bfloat162float(p.bias[o]) : 0.f;
-      for (int i = etid; i < BN; i += NEPI) {
+      const int ncols = nch * CH;
+      for (int i = etid; i < ncols; i += NEPI) {
         const int t = t0 + i;
         s_tok[i] = make_float2((t < p.T) ? p.a_scale[t] : 0.f,
                                (t < p.T && p.mean) ? p.mean[t] : 0.f);
       }
-      // one thread waits for the accumulator; the verdict reaches all four warps through
+      // one thread waits for the accumulator; the verdict reaches all epilogue warps through
       // shared memory behind a named barrier, so every later barrier is reached uniformly
       if (ep_lead) {
-        const bool ready = !*s_abort && dev::mbar_wait(tfull_bar(b), (it >> 1) & 1u, p.err,
+        const bool ready = !*s_abort && dev::mbar_wait(tfull_bar(b), (it_n >> 1) & 1u, p.err,
                                                        kSiteGemmAccum, p.limit_ns);
         if (!ready) give_up();
         s_misc[2] = ready ? 1u : 0u;
@@ -544,24 +625,38 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       dev::named_bar(1, NEPI);
       ok = *reinterpret_cast<volatile uint32_t*>(&s_misc[2]) != 0;
       if (ok) dev::tc_fence_after();
-      const int t_end = min(BN, p.T - t0);   // tokens of this tile inside [0, T)
+      const int t_end = min(ncols, p.T - t0);   // tokens of this tile inside [0, T)
+      const int nmine = (nch - half + EPW - 1) / EPW;   // chunks half, half + EPW, ...
+      if (ok && nmine == 0) {
+        dev::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) arrive_lead(tempty_bar(b));
+      }
 #pragma unroll 1
-      for (int cc = 0; ok && cc < COLS / 32; ++cc) {
-        const int c = half * (COLS / 32) + cc;   // 32-column chunk of the tile
+      for (int cc = 0; ok && cc < nmine; ++cc) {
+        const int c = half + cc * EPW;   // 32-column chunk of the tile
         uint32_t r[32];
-        dev::tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * BN + c * 32), r);
+        dev::tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * C::BNMAX + c * 32), r);
         dev::tmem_wait_ld();
-        if (cc == COLS / 32 - 1) {  // this warp's part of the accumulator is read
+        if (cc == nmine - 1) {  // this warp's part of the accumulator is read
           dev::tc_fence_before();
           __syncwarp();
           if (lane == 0) arrive_lead(tempty_bar(b));
         }
         if (!has_o) continue;
+        const int n_valid = t_end - c * 32;   // tokens of this chunk inside [0, T)
         if (p.out_acc) {
-          uint32_t* dst = reinterpret_cast<uint32_t*>(p.out) + (int64_t)(t0 + c * 32) * p.N + o;
+          if constexpr (KIND == kGemmLloydMax) {
+            float* dst = reinterpret_cast<float*>(p.out) + (int64_t)(t0 + c * 32) * p.N + o;
 #pragma unroll
-          for (int jj = 0; jj < 32; ++jj)
-            if (c * 32 + jj < t_end) dst[(int64_t)jj * p.N] = r[jj];
+            for (int jj = 0; jj < 32; ++jj)
+              if (jj < n_valid) dst[(int64_t)jj * p.N] = __uint_as_float(r[jj]) * C::ACC_SCALE;
+          } else {
+            int32_t* dst = reinterpret_cast<int32_t*>(p.out) + (int64_t)(t0 + c * 32) * p.N + o;
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj)
+              if (jj < n_valid) dst[(int64_t)jj * p.N] = (int32_t)r[jj] >> (KIND == kGemmA4 ? 8 : 4);
+          }
         } else {
           // two tokens at a time as f32x2: y = acc * (alpha_t s_w) + (mean_t w_1 + b)
           __nv_bfloat16* dst =
@@ -569,7 +664,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           const float4* tk4 = reinterpret_cast<const float4*>(s_tok + c * 32);
           const float2 sw2 = make_float2(sw, sw), w12 = make_float2(w1, w1);
           const float2 bb2 = make_float2(bb, bb);
-          const int n_valid = t_end - c * 32;   // tokens of this chunk inside [0, T)
           const int64_t ld = p.N;
 #pragma unroll
           for (int jj = 0; jj < 32; jj += 2) {
@@ -597,9 +691,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   if (warp == 1) {
     dev::tc_fence_after();
     if constexpr (CG == 2)
-      dev::tmem_dealloc_pair(tmem, 2 * BN);
+      dev::tmem_dealloc_pair(tmem, 2 * C::BNMAX);
     else
-      dev::tmem_dealloc(tmem, 2 * BN);
+      dev::tmem_dealloc(tmem, 2 * C::BNMAX);
   }
 }
 
@@ -674,9 +768,9 @@ int active_pairs(const void* kern, size_t smem) {
   return n;
 }
 
-template <int KIND, int BN, int CG>
+template <int KIND, int CG>
 oq_status run(const GemmArgs& g, const GemmParams& p, cudaStream_t s) {
-  using C = Cfg<KIND, BN, CG>;
+  using C = Cfg<KIND, CG>;
   constexpr int BK = C::BK;
   CUtensorMap tx, tw;
   bool ok = true;
@@ -690,10 +784,11 @@ oq_status run(const GemmArgs& g, const GemmParams& p, cudaStream_t s) {
                     (uint64_t)g.K / 2, BK / 2, BM, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (!ok) return fail(OQ_ERR_CUDA, "cuTensorMapEncodeTiled failed or unavailable");
 
-  auto kern = &k_gemm<KIND, BN, CG>;
+  auto kern = &k_gemm<KIND, CG>;
   const cudaError_t attr_err = allow_max_dynamic_smem(reinterpret_cast<const void*>(kern));
   if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute(gemm)");
-  const int64_t tiles = ((g.N + BM * CG - 1) / (BM * CG)) * ((g.T + BN - 1) / BN);
+  // tiles of 128 * CG tokens of one channel tile; no more CTAs (pairs) than tiles
+  const int64_t tiles = ((g.N + BM * CG - 1) / (BM * CG)) * ((g.T + 128 * CG - 1) / (128 * CG));
   if constexpr (CG == 1) {
     const int grid = (int)std::min<int64_t>(tiles, sm_count());
     kern<<<grid, NTHREADS, C::SMEM, s>>>(tx, tw, p);
@@ -753,13 +848,13 @@ oq_status launch_gemm(const GemmArgs& g, cudaStream_t s) {
   p.err = device_error_word();
   if (!p.err) return fail(OQ_ERR_CUDA, "device error word unavailable");
   p.limit_ns = kWaitLimitNs;
-  // up to 128 tokens: one CTA per 128 x 128 tile; beyond: CTA pairs on 256 x 256 tiles
+  // up to 128 tokens: single CTAs on 128-channel tiles; beyond: CTA pairs on 256 channels
   const bool small = g.T <= 128;
   switch (g.kind) {
-    case kGemmA8: return small ? run<kGemmA8, 128, 1>(g, p, s) : run<kGemmA8, 256, 2>(g, p, s);
-    case kGemmA4: return small ? run<kGemmA4, 128, 1>(g, p, s) : run<kGemmA4, 256, 2>(g, p, s);
+    case kGemmA8: return small ? run<kGemmA8, 1>(g, p, s) : run<kGemmA8, 2>(g, p, s);
+    case kGemmA4: return small ? run<kGemmA4, 1>(g, p, s) : run<kGemmA4, 2>(g, p, s);
     case kGemmLloydMax:
-      return small ? run<kGemmLloydMax, 128, 1>(g, p, s) : run<kGemmLloydMax, 256, 2>(g, p, s);
+      return small ? run<kGemmLloydMax, 1>(g, p, s) : run<kGemmLloydMax, 2>(g, p, s);
     default: return fail(OQ_ERR_INVALID_ARG, "unknown GEMM kind");
   }
 }

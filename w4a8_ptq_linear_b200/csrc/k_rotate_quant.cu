@@ -51,6 +51,7 @@ struct RqParams {
   const uint16_t* x;   // bf16 bits
   int64_t ldx, T;
   int d, hlog2, center, mode, nbuf, want_sum, mask_smem;
+  int wlayout;         // 4-bit absmax codes in the GEMM weight layout (see gemm_layout4)
   const uint16_t* tab;   // rounds x d entries in kernel order
   const uint4* smask;    // round-1 source signs: bit 15 / 31 of word j/2 flips channel j
   const float4* ones;    // c' = unnormalised round-1 transform of the all-ones vector
@@ -110,6 +111,13 @@ __device__ __forceinline__ float warp_sum(float x) {
   for (int m = 16; m > 0; m >>= 1) x += __shfl_xor_sync(0xffffffffu, x, m);
   return x;
 }
+// max(a, b, c) in one instruction (three-input max.f32, sm_100)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 __device__ __forceinline__ float warp_max(float x) {
 #pragma unroll
   for (int m = 16; m > 0; m >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, m));
@@ -134,6 +142,16 @@ __device__ __forceinline__ uint32_t lm_code(float u, const float2* cells) {
   j = min(max(j, 0), 31);
   const float2 c = cells[j];
   return (uint32_t)__float_as_int(c.y) + (u > c.x ? 1u : 0u);
+}
+
+// Two's-complement bytes of a thread's 32 consecutive codes (w[k] = codes 4k..4k+3) -> one
+// 16-byte group of the GEMM weight layout: byte j holds code j in its low nibble and code
+// 16 + j in its high nibble.
+__device__ __forceinline__ uint4 gemm_layout4(const uint32_t (&w)[8]) {
+  uint32_t o[4];
+#pragma unroll
+  for (int m = 0; m < 4; ++m) o[m] = (w[m] & 0x0F0F0F0Fu) | ((w[m + 4] << 4) & 0xF0F0F0F0u);
+  return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 // Block transform of the 32 values a thread holds, for h = 2^HLOG2 in one of three shapes.
@@ -360,10 +378,12 @@ __global__ void __launch_bounds__(MAXT, 1) k_rotate_quant(const RqParams p) {
     // ---- per-token statistic ------------------------------------------------------------
     const bool lm = p.mode == kRqLloydMax;
     float stat = 0.f;
+    if (lm) {
 #pragma unroll
-    for (int i = 0; i < EP; ++i) {
-      const float x = el(v, i);
-      stat = lm ? fmaf(x, x, stat) : fmaxf(stat, fabsf(x));
+      for (int i = 0; i < EP; ++i) stat = fmaf(el(v, i), el(v, i), stat);
+    } else {
+#pragma unroll
+      for (int i = 0; i < EP; i += 2) stat = fmax3(stat, fabsf(el(v, i)), fabsf(el(v, i + 1)));
     }
     stat = lm ? warp_sum(stat) : warp_max(stat);
     if (lane == 0) red[32 + warp] = stat;
@@ -426,6 +446,9 @@ __global__ void __launch_bounds__(MAXT, 1) k_rotate_quant(const RqParams p) {
           uint8_t* dst = reinterpret_cast<uint8_t*>(p.codes) + t * (int64_t)d + base;
           reinterpret_cast<uint4*>(dst)[0] = make_uint4(w[0], w[1], w[2], w[3]);
           reinterpret_cast<uint4*>(dst)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        } else if (p.wlayout) {
+          *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(p.codes) + t * (int64_t)(d / 2) +
+                                    base / 2) = gemm_layout4(w);
         } else {
           uint32_t n[4];
 #pragma unroll
@@ -751,9 +774,9 @@ __global__ void __launch_bounds__(256, 2) k_rotate_quant_pair(const RqParams p) 
       st = warp_sum_pair(st);
     } else {
 #pragma unroll
-      for (int i = 0; i < EP; ++i) {
-        st.x = fmaxf(st.x, fabsf(v[i].x));
-        st.y = fmaxf(st.y, fabsf(v[i].y));
+      for (int i = 0; i < EP; i += 2) {
+        st.x = fmax3(st.x, fabsf(v[i].x), fabsf(v[i + 1].x));
+        st.y = fmax3(st.y, fabsf(v[i].y), fabsf(v[i + 1].y));
       }
       st.x = warp_max(st.x);
       st.y = warp_max(st.y);
@@ -829,6 +852,11 @@ __global__ void __launch_bounds__(256, 2) k_rotate_quant_pair(const RqParams p) 
             db[0] = make_uint4(wb[0], wb[1], wb[2], wb[3]);
             db[1] = make_uint4(wb[4], wb[5], wb[6], wb[7]);
           }
+        } else if (p.wlayout) {
+          *reinterpret_cast<uint4*>(codes + ta * (int64_t)(d / 2) + base / 2) = gemm_layout4(wa);
+          if (has_b)
+            *reinterpret_cast<uint4*>(codes + (ta + 1) * (int64_t)(d / 2) + base / 2) =
+                gemm_layout4(wb);
         } else {
           *reinterpret_cast<uint4*>(codes + ta * (int64_t)(d / 2) + base / 2) =
               make_uint4(nibbles8(wa[0], wa[1]), nibbles8(wa[2], wa[3]), nibbles8(wa[4], wa[5]),
@@ -975,17 +1003,26 @@ oq_status launch_rotate_quant(const RqArgs& a, cudaStream_t s) {
         // nbuf landing pairs, the interleaved words / transpose tiles, the round buffer,
         // reductions + thresholds + barriers
         cfg.pair = 1;
-        cfg.nbuf = 1;
-        cfg.smem = (size_t)cfg.nbuf * 2 * row_stride + (size_t)(nthr / 32) * 4096 +
-                   (a.rounds == 2 ? (size_t)(nthr / 32) * 8192 : 0) + 96 * 4 + 16 * 8;
         cfg.fn = a.rounds == 1 ? kern_pair_h<1>(hlog2) : kern_pair_h<2>(hlog2);
         cfg.nthr = nthr;
         ce = allow_max_dynamic_smem(cfg.fn);
         if (ce != cudaSuccess) return cuda_fail(ce, "cudaFuncSetAttribute(rotate_quant)");
-        int occ = 0;
-        ce = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, cfg.fn, nthr, cfg.smem);
-        if (ce != cudaSuccess) return cuda_fail(ce, "occupancy(rotate_quant)");
-        cfg.grid_per_sm = std::max(occ, 1) * nsm;
+        // a second landing pair lets each CTA have the next pair's rows in flight for a whole
+        // pass; it is taken when it costs no resident CTA
+        int best_occ = 0;
+        for (int nb = 1; nb <= 2; ++nb) {
+          const size_t smem = (size_t)nb * 2 * row_stride + (size_t)(nthr / 32) * 4096 +
+                              (a.rounds == 2 ? (size_t)(nthr / 32) * 8192 : 0) + 96 * 4 + 16 * 8;
+          int occ = 0;
+          ce = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, cfg.fn, nthr, smem);
+          if (ce != cudaSuccess) return cuda_fail(ce, "occupancy(rotate_quant)");
+          if (nb == 1 || occ >= best_occ) {
+            best_occ = occ;
+            cfg.nbuf = nb;
+            cfg.smem = smem;
+          }
+        }
+        cfg.grid_per_sm = std::max(best_occ, 1) * nsm;
         cache[key] = cfg;
       } else {
       // fp32 round buffer and transpose tiles (one region when both are needed), both sized
@@ -1027,6 +1064,7 @@ oq_status launch_rotate_quant(const RqArgs& a, cudaStream_t s) {
   p.nbuf = cfg.nbuf;
   p.want_sum = (a.center || a.rowsum) ? 1 : 0;
   p.mask_smem = cfg.mask_smem;
+  p.wlayout = a.wlayout;
   p.tab = a.tab;
   p.smask = reinterpret_cast<const uint4*>(a.smask);
   p.ones = reinterpret_cast<const float4*>(a.ones);

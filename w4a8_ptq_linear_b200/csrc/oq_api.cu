@@ -299,12 +299,13 @@ oq_status oq_plan_get_rpbh(const oq_plan* plan, int round, int8_t* signs_host,
 
 static oq_status rotate_quantize_impl(const oq_plan* plan, const void* x, int64_t T, int64_t ldx,
                                       void* codes, float* scale, float* mean, float* rotated,
-                                      float* rowsum, int mode, int center, cudaStream_t s) {
+                                      float* rowsum, int mode, int center, int wlayout,
+                                      cudaStream_t s) {
   RqArgs a;
   a.x = x; a.ldx = ldx; a.T = T; a.d = plan->d; a.h = plan->h; a.rounds = plan->rounds;
   a.center = center; a.mode = mode; a.tab = plan->d_tab; a.smask = plan->d_smask;
   a.ones = plan->d_ones; a.codes = codes; a.scale = scale;
-  a.mean = mean; a.rotated = rotated; a.rowsum = rowsum;
+  a.mean = mean; a.rotated = rotated; a.rowsum = rowsum; a.wlayout = wlayout;
   for (int i = 0; i < 15; ++i) a.thr[i] = (float)plan->cb_t[i];
   return launch_rotate_quant(a, s);
 }
@@ -325,7 +326,7 @@ oq_status oq_rotate_quantize(const oq_plan* plan, const void* x_bf16, int64_t T,
   const int mode = plan->act == OQ_ACT_INT8_ABSMAX ? kRqInt8
                    : plan->act == OQ_ACT_INT4_ABSMAX ? kRqInt4 : kRqLloydMax;
   return rotate_quantize_impl(plan, x_bf16, T, ldx, codes, scale, plan->center ? mean : nullptr,
-                              rotated_f32, nullptr, mode, plan->center,
+                              rotated_f32, nullptr, mode, plan->center, 0,
                               static_cast<cudaStream_t>(stream));
 }
 
@@ -341,7 +342,7 @@ oq_status oq_prepare_weights(const oq_plan* plan, const void* w_bf16, int64_t n_
   oq_status st = check_plan_device(plan);
   if (st != OQ_OK) return st;
   return rotate_quantize_impl(plan, w_bf16, n_out, ldw, w_packed, w_scale, nullptr, nullptr,
-                              w_rowsum, kRqInt4, 0, static_cast<cudaStream_t>(stream));
+                              w_rowsum, kRqInt4, 0, 1, static_cast<cudaStream_t>(stream));
 }
 
 oq_status oq_gemm_w4a8(const int8_t* a, const float* a_scale, const float* mean,

@@ -74,6 +74,7 @@ struct RqArgs {
   float* rotated = nullptr;  // optional [T, d]
   float* rowsum = nullptr;   // optional [T]: sum of the row before centering/rotation
   float thr[15] = {};        // Lloyd-Max thresholds (fp32)
+  int wlayout = 0;           // kRqInt4 only: write the codes in the GEMM weight layout
 };
 oq_status launch_rotate_quant(const RqArgs& a, cudaStream_t s);
 // Kernel-order gather table helpers: the row position thread t, register i gathers in a
