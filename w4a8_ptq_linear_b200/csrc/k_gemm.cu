@@ -96,7 +96,7 @@ struct Cfg {
   // Ring depths. Loads from L2 take a few thousand cycles, so the packed ring, which the
   // converters free only after unpacking, must cover that latency at the MMA's pace.
   static constexpr int SX = XPACK ? 0 : (CG == 2 ? 5 : 4);         // activation ring (A8)
-  static constexpr int SP = CG == 1 ? 4 : (KIND == kGemmA4 ? 6 : 8);  // packed ring
+  static constexpr int SP = CG == 1 ? 4 : (KIND == kGemmA8 ? 6 : (KIND == kGemmA4 ? 6 : 8));
   static constexpr int S2 = (KIND == kGemmA4) ? (CG == 2 ? 3 : 2) : (CG == 2 ? 4 : 3);
   static constexpr int WT = BM * 128;                              // W operand tile
   static constexpr int XT = XR * 128;                              // X operand tile (this CTA)
@@ -107,7 +107,9 @@ struct Cfg {
   static constexpr int OFF_X = 0;
   static constexpr int OFF_P = OFF_X + SX * XT;
   static constexpr int OFF_CONV = OFF_P + SP * P_STAGE;
-  static constexpr int OFF_TOK = OFF_CONV + S2 * CONV_STAGE;       // float2 (scale, mean)
+  static constexpr int OFF_STG = OFF_CONV + S2 * CONV_STAGE;       // epilogue staging tiles
+  static constexpr int STG = 32 * 32 * 2;                          // bf16 [32 tokens][32 ch]
+  static constexpr int OFF_TOK = OFF_STG + (NEPI / 32) * STG;      // float2 (scale, mean)
   static constexpr int OFF_BAR = OFF_TOK + BNMAX * 8;
   static constexpr int NBAR = 2 * SX + 2 * SP + 2 * S2 + 4 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
@@ -320,7 +322,7 @@ __device__ __forceinline__ int k_rotation(int m, int nkb) {
 template <int KIND, int CG>
 __global__ void __launch_bounds__(NTHREADS, 1)
     k_gemm(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
-           const GemmParams p) {
+           const __grid_constant__ CUtensorMap tm_y, const GemmParams p) {
   using C = Cfg<KIND, CG>;
   constexpr int BK = C::BK, SX = C::SX, SP = C::SP, S2 = C::S2, MAXCH = C::MAXCH;
   extern __shared__ uint8_t smem_raw[];
@@ -400,6 +402,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     dev::prefetch_tmap(&tm_x);
     dev::prefetch_tmap(&tm_w);
   }
+  if (warp == W_EPI0 && lane == 0 && !p.out_acc) dev::prefetch_tmap(&tm_y);
   if (warp == 1) {
     if constexpr (CG == 2) {
       dev::tmem_alloc_pair(dev::smem_u32(&s_misc[0]), 2 * C::BNMAX);
@@ -592,6 +595,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     // consecutive channels, i.e. 64 (bf16) or 128 (raw accumulator) contiguous bytes. The
     // EPW warps of a lane quarter take the tile's 32-column chunks in turn.
     const int etid = tid - EPI0;         // 0..NEPI-1
+    uint8_t* stg = smem + C::OFF_STG + (warp - W_EPI0) * C::STG;
     const int q = warp & 3;              // TMEM lane quarter of this warp
     const int half = etid >> 7;          // index among the warps of the quarter
     const int o_local = q * 32 + lane;
@@ -643,28 +647,28 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           __syncwarp();
           if (lane == 0) arrive_lead(tempty_bar(b));
         }
-        if (!has_o) continue;
+        if (o0 + q * 32 >= p.N) continue;    // this warp's channels all lie past N
         const int n_valid = t_end - c * 32;   // tokens of this chunk inside [0, T)
         if (p.out_acc) {
           if constexpr (KIND == kGemmLloydMax) {
             float* dst = reinterpret_cast<float*>(p.out) + (int64_t)(t0 + c * 32) * p.N + o;
 #pragma unroll
             for (int jj = 0; jj < 32; ++jj)
-              if (jj < n_valid) dst[(int64_t)jj * p.N] = __uint_as_float(r[jj]) * C::ACC_SCALE;
+              if (has_o && jj < n_valid) dst[(int64_t)jj * p.N] = __uint_as_float(r[jj]) * C::ACC_SCALE;
           } else {
             int32_t* dst = reinterpret_cast<int32_t*>(p.out) + (int64_t)(t0 + c * 32) * p.N + o;
 #pragma unroll
             for (int jj = 0; jj < 32; ++jj)
-              if (jj < n_valid) dst[(int64_t)jj * p.N] = (int32_t)r[jj] >> (KIND == kGemmA4 ? 8 : 4);
+              if (has_o && jj < n_valid) dst[(int64_t)jj * p.N] = (int32_t)r[jj] >> (KIND == kGemmA4 ? 8 : 4);
           }
         } else {
-          // two tokens at a time as f32x2: y = acc * (alpha_t s_w) + (mean_t w_1 + b)
-          __nv_bfloat16* dst =
-              reinterpret_cast<__nv_bfloat16*>(p.out) + (int64_t)(t0 + c * 32) * p.N + o;
+          // two tokens at a time as f32x2: y = acc * (alpha_t s_w) + (mean_t w_1 + b), into
+          // this warp's staging tile [32 tokens][32 channels]; one TMA store writes the tile
+          // (the store clips tokens past T and channels past N)
           const float4* tk4 = reinterpret_cast<const float4*>(s_tok + c * 32);
           const float2 sw2 = make_float2(sw, sw), w12 = make_float2(w1, w1);
           const float2 bb2 = make_float2(bb, bb);
-          const int64_t ld = p.N;
+          uint32_t yb[16];
 #pragma unroll
           for (int jj = 0; jj < 32; jj += 2) {
             const float4 tk = tk4[jj / 2];    // (alpha, mean) of tokens jj and jj + 1
@@ -674,13 +678,26 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                                   ? make_float2(__uint_as_float(r[jj]), __uint_as_float(r[jj + 1]))
                                   : make_float2((float)(int32_t)r[jj], (float)(int32_t)r[jj + 1]);
             const __nv_bfloat162 y = __float22bfloat162_rn(__ffma2_rn(a2, s2, c2));
-            if (jj < n_valid) dst[(int64_t)jj * ld] = y.x;
-            if (jj + 1 < n_valid) dst[(int64_t)(jj + 1) * ld] = y.y;
+            yb[jj / 2] = *reinterpret_cast<const uint32_t*>(&y);
+          }
+          if (lane == 0) dev::bulk_wait_all_read();   // the previous store has read the tile
+          __syncwarp();
+#pragma unroll
+          for (int jj = 0; jj < 32; jj += 2) {
+            *reinterpret_cast<uint16_t*>(stg + jj * 64 + lane * 2) = (uint16_t)(yb[jj / 2] & 0xFFFFu);
+            *reinterpret_cast<uint16_t*>(stg + (jj + 1) * 64 + lane * 2) = (uint16_t)(yb[jj / 2] >> 16);
+          }
+          dev::fence_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            dev::tma_store_2d(&tm_y, dev::smem_u32(stg), o0 + q * 32, t0 + c * 32);
+            dev::bulk_commit();
           }
         }
       }
       dev::named_bar(1, NEPI);  // s_tok of this tile is no longer read
     }
+    if (lane == 0) dev::bulk_wait_all();   // this warp's output stores are complete
   }
 
   dev::tc_fence_before();
@@ -772,8 +789,13 @@ template <int KIND, int CG>
 oq_status run(const GemmArgs& g, const GemmParams& p, cudaStream_t s) {
   using C = Cfg<KIND, CG>;
   constexpr int BK = C::BK;
-  CUtensorMap tx, tw;
+  CUtensorMap tx, tw, ty;
   bool ok = true;
+  if (!g.out_acc)
+    ok &= make_map_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.out, (uint64_t)g.N, (uint64_t)g.T,
+                      (uint64_t)g.N * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE);
+  else
+    std::memset(&ty, 0, sizeof(ty));
   if constexpr (C::XPACK)
     ok &= make_map_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.a, (uint64_t)g.K / 2, (uint64_t)g.T,
                       (uint64_t)g.K / 2, BK / 2, C::XR, CU_TENSOR_MAP_SWIZZLE_NONE);
@@ -791,7 +813,7 @@ oq_status run(const GemmArgs& g, const GemmParams& p, cudaStream_t s) {
   const int64_t tiles = ((g.N + BM * CG - 1) / (BM * CG)) * ((g.T + 128 * CG - 1) / (128 * CG));
   if constexpr (CG == 1) {
     const int grid = (int)std::min<int64_t>(tiles, sm_count());
-    kern<<<grid, NTHREADS, C::SMEM, s>>>(tx, tw, p);
+    kern<<<grid, NTHREADS, C::SMEM, s>>>(tx, tw, ty, p);
   } else {
     const int pairs = active_pairs(reinterpret_cast<const void*>(kern), C::SMEM);
     if (pairs <= 0) return fail(OQ_ERR_UNSUPPORTED, "gemm: no CTA pair fits on this device");
@@ -807,7 +829,7 @@ oq_status run(const GemmArgs& g, const GemmParams& p, cudaStream_t s) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    const cudaError_t le = cudaLaunchKernelEx(&cfg, kern, tx, tw, p);
+    const cudaError_t le = cudaLaunchKernelEx(&cfg, kern, tx, tw, ty, p);
     if (le != cudaSuccess) return cuda_fail(le, "launch gemm (CTA pairs)");
   }
   cudaError_t ce = cudaGetLastError();

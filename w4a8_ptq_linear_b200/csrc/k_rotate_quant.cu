@@ -603,7 +603,10 @@ __device__ __forceinline__ uint32_t nibbles8(uint32_t w0, uint32_t w1) {
 }
 
 template <int HLOG2, int ROUNDS>
-__global__ void __launch_bounds__(256, 2) k_rotate_quant_pair(const RqParams p) {
+#ifndef OQ_RQ_PAIR_MINB
+#define OQ_RQ_PAIR_MINB 2
+#endif
+__global__ void __launch_bounds__(256, OQ_RQ_PAIR_MINB) k_rotate_quant_pair(const RqParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const int d = p.d;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -1010,7 +1013,10 @@ oq_status launch_rotate_quant(const RqArgs& a, cudaStream_t s) {
         // a second landing pair lets each CTA have the next pair's rows in flight for a whole
         // pass; it is taken when it costs no resident CTA
         int best_occ = 0;
-        for (int nb = 1; nb <= 2; ++nb) {
+#ifndef OQ_RQ_MAXNBUF
+#define OQ_RQ_MAXNBUF 2
+#endif
+        for (int nb = 1; nb <= OQ_RQ_MAXNBUF; ++nb) {
           const size_t smem = (size_t)nb * 2 * row_stride + (size_t)(nthr / 32) * 4096 +
                               (a.rounds == 2 ? (size_t)(nthr / 32) * 8192 : 0) + 96 * 4 + 16 * 8;
           int occ = 0;
