@@ -59,7 +59,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="dit_w4a8",
-                    choices=["tiny", "dit_w4a8", "narrow_lm", "mlp_up"])
+                    choices=["tiny", "dit_w4a8", "narrow_lm", "mlp_up", "mlp_up_pct"])
     ap.add_argument("--tokens", type=int, default=None,
                     help="override the token count (small cases for profiler captures)")
     ap.add_argument("--e2e-steps", type=int, default=100)

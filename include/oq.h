@@ -72,8 +72,16 @@ typedef enum {
 typedef enum {
   OQ_ACT_INT8_ABSMAX = 0,    /* A8: alpha_t = max|z_t| / 127, codes in -127..127         */
   OQ_ACT_INT4_ABSMAX = 1,    /* A4: alpha_t = max|z_t| / 7,   codes in -7..7             */
-  OQ_ACT_INT4_LLOYDMAX = 2   /* A4: sigma_t = RMS(z_t), nearest of 16 N(0,1) centroids   */
+  OQ_ACT_INT4_LLOYDMAX = 2,  /* A4: sigma_t = RMS(z_t), nearest of 16 N(0,1) centroids   */
+  OQ_ACT_INT4_PERCENTILE = 3 /* A4: percentile range (below), codes clipped to -7..7     */
 } oq_act_kind;
+/* OQ_ACT_INT4_PERCENTILE (CentriQ §4.2 "Scale and grid", App. B.3 Tab. 3): the spread of the
+ * rotated token is sigma_hat_t = q_rho(|z_t|) / Phi^-1((1 + rho) / 2) with rho = 0.9995, where
+ * q_rho is the empirical quantile, linear between the order statistics around position
+ * rho (d - 1); alpha_t = max(gamma sigma_hat_t, 1e-10) / 7 with gamma = 2.5591, and
+ * codes = clip(round(z / alpha_t), -7, 7). The codes and the GEMM are those of
+ * OQ_ACT_INT4_ABSMAX; only the scale differs. Limit: d <= 8192 (the quantile needs the
+ * d - floor(rho (d - 1)) <= 6 largest magnitudes, kept per thread). */
 
 typedef enum {
   OQ_OUT_BF16 = 0,           /* dequantised, rank-1 and bias added, rounded to bf16      */
@@ -173,9 +181,10 @@ oq_status oq_gemm_w4a8(const int8_t* a, const float* a_scale, const float* mean,
                        const void* bias_bf16, int64_t T, int64_t d_in, int64_t d_out,
                        oq_out_kind out_kind, void* out, void* stream);
 
-/* W4A4 GEMM, same epilogue. kind = OQ_ACT_INT4_ABSMAX (integer GEMM, exact int32
- * accumulators) or OQ_ACT_INT4_LLOYDMAX (codes decoded through the plan's codebook to fp16,
- * fp16 x fp16 -> fp32 GEMM; a_scale holds sigma_t; OQ_OUT_ACC gives float32). `plan` is
+/* W4A4 GEMM, same epilogue. kind = OQ_ACT_INT4_ABSMAX or OQ_ACT_INT4_PERCENTILE (integer
+ * GEMM, exact int32 accumulators) or OQ_ACT_INT4_LLOYDMAX (codes decoded through the plan's
+ * codebook to fp16, fp16 x fp16 -> fp32 GEMM; a_scale holds sigma_t; OQ_OUT_ACC gives
+ * float32). `plan` is
  * required for Lloyd-Max (codebook) and ignored otherwise.
  *   a_packed  uint8 [T, d_in/2] */
 oq_status oq_gemm_w4a4(const oq_plan* plan, oq_act_kind kind, const uint8_t* a_packed,

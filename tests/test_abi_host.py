@@ -72,6 +72,10 @@ def test_argument_validation_before_any_cuda_call(lib):
         assert st == oq.OQ_ERR_INVALID_ARG, args
     st = lib.oq_plan_create(ctypes.byref(h), 256, 64, 1, 0, 0, 9)
     assert st == oq.OQ_ERR_INVALID_ARG
+    # the percentile scale keeps at most 6 order statistics per token: d <= 8192
+    st = lib.oq_plan_create(ctypes.byref(h), 16384, 1024, 1, 0, 0, 3)
+    assert st == oq.OQ_ERR_UNSUPPORTED
+    assert b"percentile" in lib.oq_last_error()
     # GEMM shape checks happen before any launch
     st = lib.oq_gemm_w4a8(None, None, None, None, None, None, None, 16, 100, 256, 0, None, None)
     assert st == oq.OQ_ERR_INVALID_ARG

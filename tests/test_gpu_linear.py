@@ -40,7 +40,7 @@ def _gpu_layer(wl, xb, wb, bias_bits=None):
 
 
 @pytest.mark.parametrize("name,T", [("tiny", 64), ("dit_w4a8", 300), ("narrow_lm", 257),
-                                    ("mlp_up", 130)])
+                                    ("mlp_up", 130), ("mlp_up_pct", 130)])
 def test_layer_matches_oracle(name, T):
     wl, xb, wb = synth.make_inputs(name, T=T)
     y = _gpu_layer(wl, xb, wb)
@@ -56,7 +56,7 @@ def test_layer_with_bias():
     assert rel_fro(y, ref) <= OUT_TOL
 
 
-@pytest.mark.parametrize("name", ["dit_w4a8", "narrow_lm", "mlp_up"])
+@pytest.mark.parametrize("name", ["dit_w4a8", "narrow_lm", "mlp_up", "mlp_up_pct"])
 def test_full_size_layer_on_sampled_rows(name):
     wl, xb, wb = synth.make_inputs(name)
     y = _gpu_layer(wl, xb, wb)

@@ -36,6 +36,14 @@ CASES = [
     (3, 30720, 512, 2, "int8_absmax", False),
     (70, 2048, 256, 1, "int4_lloydmax", True),
     (20, 1280, 256, 2, "int8_absmax", True),
+    # CentriQ percentile scale: the quantile needs the R = d - floor(0.9995 (d - 1)) largest
+    # magnitudes, R = 2 (d < 2000), 3, 4, 5, 6 (d = 8192)
+    (257, 3072, 1024, 1, "int4_percentile", True),
+    (130, 1920, 128, 2, "int4_percentile", False),
+    (45, 4096, 256, 2, "int4_percentile", False),
+    (31, 6144, 1024, 1, "int4_percentile", True),
+    (20, 8192, 512, 1, "int4_percentile", True),
+    (7, 256, 64, 1, "int4_percentile", False),
 ]
 
 
@@ -76,7 +84,7 @@ def test_rotate_quantize_matches_oracle(T, d, h, rounds, act, center):
     if act == "int8_absmax":
         gpu = out["codes"].view(np.int8).astype(np.int64)
         ex = absmax_boundary_mask(ref["rotated"], ref["scale"], 127)
-    elif act == "int4_absmax":
+    elif act in ("int4_absmax", "int4_percentile"):
         gpu = oracle.unpack_nibbles(out["codes"], signed=True)
         ex = absmax_boundary_mask(ref["rotated"], ref["scale"], 7)
     else:
@@ -141,3 +149,36 @@ def test_row_pitch_larger_than_width():
     codes2, scale2, _, _ = oq.rotate_quantize(plan, x.contiguous())
     assert torch.equal(codes, codes2) and torch.equal(scale, scale2)
     plan.close()
+
+
+def test_percentile_clips_outliers_and_handles_flat_tokens():
+    # CentriQ §4.2: the percentile range leaves the largest magnitudes past +-7 alpha, which
+    # clip to +-7; tokens with few distinct magnitudes exercise ties in the order statistics
+    import torch
+    import w4a8_ptq_linear_b200 as oq
+    d, h = 3072, 1024
+    xb = synth.make_x(6, d, mean_var=0.0, seed=3)
+    x = synth.bf16_to_f64(xb)
+    x[0, 17] = 900.0                    # one huge channel
+    x[1, :40] = 300.0                   # a block of equal outliers
+    x[2] = 0.0                          # zero token
+    x[3] = 0.0
+    x[3, 5] = 2.0                       # one non-zero channel
+    x[4] = np.where(np.arange(d) % 2 == 0, 1.0, -1.0)   # flat magnitudes
+    xb = synth.f64_to_bf16(x)
+    plan = oq.Plan(d, h, 1, act="int4_percentile")
+    codes, scale, _, rot = oq.rotate_quantize(plan, to_torch_bf16(xb), rotated=True)
+    torch.cuda.synchronize()
+    ref = oracle.quantize_activations(synth.bf16_to_f64(xb), oracle.rpbh_plan(d, h, 1, 0), h,
+                                      "int4_percentile", False)
+    s = scale.cpu().numpy().astype(np.float64)
+    nz = ref["scale"] > 1e-9
+    assert np.all(np.abs(s[nz] / ref["scale"][nz] - 1) <= ROT_TOL)
+    assert np.all(np.abs(s[~nz] - ref["scale"][~nz]) <= 1e-16)
+    gpu = oracle.unpack_nibbles(codes.cpu().numpy(), signed=True)
+    ex = absmax_boundary_mask(ref["rotated"], ref["scale"], 7)
+    bad, _ = compare_codes(gpu, ref["codes"], ex)
+    assert bad == 0
+    assert np.abs(gpu[0]).max() == 7 and np.all(gpu[2] == 0)
+    plan.close()
+

@@ -22,7 +22,7 @@ LIB_PATH = os.path.join(_PKG, "lib", "liboq.so")
 
 OQ_OK, OQ_ERR_INVALID_ARG, OQ_ERR_UNSUPPORTED, OQ_ERR_MISALIGNED = 0, 1, 2, 3
 OQ_ERR_CUDA, OQ_ERR_DEVICE_TIMEOUT, OQ_ERR_NOMEM = 4, 5, 6
-ACT_KINDS = {"int8_absmax": 0, "int4_absmax": 1, "int4_lloydmax": 2}
+ACT_KINDS = {"int8_absmax": 0, "int4_absmax": 1, "int4_lloydmax": 2, "int4_percentile": 3}
 OUT_BF16, OUT_ACC = 0, 1
 
 # (name, restype, argtypes) of every exported entry point

@@ -52,6 +52,9 @@ struct RqParams {
   int64_t ldx, T;
   int d, hlog2, center, mode, nbuf, want_sum, mask_smem;
   int wlayout;         // 4-bit absmax codes in the GEMM weight layout (see gemm_layout4)
+  int pct_r;           // percentile: order statistics needed from the top (2..6)
+  float pct_frac;      // percentile: interpolation weight between ranks pct_r-1 and pct_r-2
+  float pct_mult;      // percentile: gamma / Phi^-1((1 + rho) / 2)
   const uint16_t* tab;   // rounds x d entries in kernel order
   const uint4* smask;    // round-1 source signs: bit 15 / 31 of word j/2 flips channel j
   const float4* ones;    // c' = unnormalised round-1 transform of the all-ones vector
@@ -588,6 +591,12 @@ __device__ __forceinline__ float2 chunk_sums(const uint4& a, const uint4& b) {
   return s;
 }
 
+// a rounded value (1.5 * 2^23 + q) clipped to q in [-7, 7] (exact: integers in this range)
+__device__ __forceinline__ float2 clamp_code(float2 r) {
+  return make_float2(fminf(fmaxf(r.x, 12582905.f), 12582919.f),
+                     fminf(fmaxf(r.y, 12582905.f), 12582919.f));
+}
+
 // low byte of every float of four rounded values, as one word
 __device__ __forceinline__ uint32_t pack4(float a, float b, float c, float e) {
   return __byte_perm(__byte_perm(byte_of(a), byte_of(b), 0x0040),
@@ -602,11 +611,94 @@ __device__ __forceinline__ uint32_t nibbles8(uint32_t w0, uint32_t w1) {
   return __byte_perm(a0, a1, 0x6420);
 }
 
+// ---- percentile scale (CentriQ §4.2 "Scale and grid", App. B.3) ---------------------------
+// The rho-quantile of |z| over the d positions, linear between the order statistics around
+// position rho (d - 1), needs the R = d - floor(rho (d - 1)) largest magnitudes (R <= 6 for
+// d <= 8192). Every thread keeps the R largest of its values in a descending list (one max/min
+// insertion per value), the warp merges its lanes' lists by R rounds of max extraction, and
+// every warp merges the warps' lists (through shared memory) the same way.
+
+// insert x into the descending list m, keeping the R largest (a multiset: ties are kept)
+template <int R>
+__device__ __forceinline__ void topr_insert(float (&m)[R], float x) {
+#pragma unroll
+  for (int k = 0; k < R; ++k) {
+    const float hi = fmaxf(m[k], x);
+    x = fminf(m[k], x);
+    m[k] = hi;
+  }
+}
+
+// the R largest of the union of the lanes' descending lists, in every lane (out descending)
+template <int R>
+__device__ __forceinline__ void warp_topr(float (&m)[R], int lane, float (&out)[R]) {
+#pragma unroll
+  for (int k = 0; k < R; ++k) {
+    const float top = warp_max(m[0]);
+    const unsigned who = __ballot_sync(0xffffffffu, m[0] == top);
+    const bool pop = lane == __ffs(who) - 1;   // exactly one lane gives up its head
+#pragma unroll
+    for (int j = 0; j < R - 1; ++j) m[j] = pop ? m[j + 1] : m[j];
+    m[R - 1] = pop ? -1.f : m[R - 1];
+    out[k] = top;
+  }
+}
+
+// Phase 1 of the two tokens' percentile statistic: the warp's R largest |v| of token A (x) and
+// token B (y), written to lists[warp][token][0..R) in shared memory.
+template <int R>
+__device__ __forceinline__ void pct_warp_lists(const float2 (&v)[EP], bool active, int lane,
+                                               int warp, float* lists) {
+  float ma[R], mb[R];
+#pragma unroll
+  for (int k = 0; k < R; ++k) ma[k] = mb[k] = -1.f;
+  if (active) {
+#pragma unroll
+    for (int i = 0; i < EP; ++i) {
+      topr_insert<R>(ma, fabsf(v[i].x));
+      topr_insert<R>(mb, fabsf(v[i].y));
+    }
+  }
+  float oa[R], ob[R];
+  warp_topr<R>(ma, lane, oa);
+  warp_topr<R>(mb, lane, ob);
+  if (lane == 0) {
+#pragma unroll
+    for (int k = 0; k < R; ++k) {
+      lists[(2 * warp) * R + k] = oa[k];
+      lists[(2 * warp + 1) * R + k] = ob[k];
+    }
+  }
+}
+
+// Phase 2 (after a block barrier): the interpolated quantile of both tokens from every warp's
+// lists; every warp computes the same result.
+template <int R>
+__device__ __forceinline__ float2 pct_quantiles(const float* lists, int nwarps, int lane,
+                                                float frac) {
+  float ma[R], mb[R];
+#pragma unroll
+  for (int k = 0; k < R; ++k) ma[k] = mb[k] = -1.f;
+  // lane l takes list entries l and l + 32 of each token (nwarps * R <= 48)
+#pragma unroll
+  for (int rep = 0; rep < 2; ++rep) {
+    const int e = lane + 32 * rep;
+    if (e < nwarps * R) {
+      const int w = e / R, k = e % R;
+      topr_insert<R>(ma, lists[(2 * w) * R + k]);
+      topr_insert<R>(mb, lists[(2 * w + 1) * R + k]);
+    }
+  }
+  float oa[R], ob[R];
+  warp_topr<R>(ma, lane, oa);
+  warp_topr<R>(mb, lane, ob);
+  // order statistic floor(pos) is rank R-1 from the top, floor(pos) + 1 is rank R-2
+  return make_float2(fmaf(frac, oa[R - 2] - oa[R - 1], oa[R - 1]),
+                     fmaf(frac, ob[R - 2] - ob[R - 1], ob[R - 1]));
+}
+
 template <int HLOG2, int ROUNDS>
-#ifndef OQ_RQ_PAIR_MINB
-#define OQ_RQ_PAIR_MINB 2
-#endif
-__global__ void __launch_bounds__(256, OQ_RQ_PAIR_MINB) k_rotate_quant_pair(const RqParams p) {
+__global__ void __launch_bounds__(256, 2) k_rotate_quant_pair(const RqParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const int d = p.d;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -628,6 +720,7 @@ __global__ void __launch_bounds__(256, OQ_RQ_PAIR_MINB) k_rotate_quant_pair(cons
   // red: [0,16) sums, [16,32) statistic; then 32 Lloyd-Max code cells and the barriers
   float2* cells = reinterpret_cast<float2*>(red + 32);
   uint64_t* bars = reinterpret_cast<uint64_t*>(red + 96);
+  float* pct_lists = red + 128;   // percentile: up to 8 warps x 2 tokens x 6 ranks
   float* warp_tile = reinterpret_cast<float*>(wbuf) + warp * 1024;
 
   if (tid < 32) cells[tid] = p.cells[tid];
@@ -771,7 +864,16 @@ __global__ void __launch_bounds__(256, OQ_RQ_PAIR_MINB) k_rotate_quant_pair(cons
 
     // ---- per-token statistics --------------------------------------------------------------
     float2 st = make_float2(0.f, 0.f);
-    if (lm) {
+    const bool pct = p.mode == kRqPercentile;
+    if (pct) {
+      switch (p.pct_r) {
+        case 2: pct_warp_lists<2>(v, active, lane, warp, pct_lists); break;
+        case 3: pct_warp_lists<3>(v, active, lane, warp, pct_lists); break;
+        case 4: pct_warp_lists<4>(v, active, lane, warp, pct_lists); break;
+        case 5: pct_warp_lists<5>(v, active, lane, warp, pct_lists); break;
+        default: pct_warp_lists<6>(v, active, lane, warp, pct_lists); break;
+      }
+    } else if (lm) {
 #pragma unroll
       for (int i = 0; i < EP; ++i) st = __ffma2_rn(v[i], v[i], st);
       st = warp_sum_pair(st);
@@ -784,12 +886,22 @@ __global__ void __launch_bounds__(256, OQ_RQ_PAIR_MINB) k_rotate_quant_pair(cons
       st.x = warp_max(st.x);
       st.y = warp_max(st.y);
     }
-    if (lane == 0) { red[16 + 2 * warp] = st.x; red[16 + 2 * warp + 1] = st.y; }
+    if (lane == 0 && !pct) { red[16 + 2 * warp] = st.x; red[16 + 2 * warp + 1] = st.y; }
     __syncthreads();
     st = make_float2(0.f, 0.f);
-    for (int w = 0; w < nwarps; ++w) {
-      const float sa = red[16 + 2 * w], sb = red[16 + 2 * w + 1];
-      st = lm ? make_float2(st.x + sa, st.y + sb) : make_float2(fmaxf(st.x, sa), fmaxf(st.y, sb));
+    if (pct) {
+      switch (p.pct_r) {
+        case 2: st = pct_quantiles<2>(pct_lists, nwarps, lane, p.pct_frac); break;
+        case 3: st = pct_quantiles<3>(pct_lists, nwarps, lane, p.pct_frac); break;
+        case 4: st = pct_quantiles<4>(pct_lists, nwarps, lane, p.pct_frac); break;
+        case 5: st = pct_quantiles<5>(pct_lists, nwarps, lane, p.pct_frac); break;
+        default: st = pct_quantiles<6>(pct_lists, nwarps, lane, p.pct_frac); break;
+      }
+    } else {
+      for (int w = 0; w < nwarps; ++w) {
+        const float sa = red[16 + 2 * w], sb = red[16 + 2 * w + 1];
+        st = lm ? make_float2(st.x + sa, st.y + sb) : make_float2(fmaxf(st.x, sa), fmaxf(st.y, sb));
+      }
     }
 
     if (p.rotated && active) {
@@ -829,20 +941,27 @@ __global__ void __launch_bounds__(256, OQ_RQ_PAIR_MINB) k_rotate_quant_pair(cons
       }
     } else {
       const float qmax = (p.mode == kRqInt8) ? 127.f : 7.f;
-      const float aa = fmaxf(st.x * nrm, 1e-10f), ab = fmaxf(st.y * nrm, 1e-10f);
+      // range: absmax, or gamma * sigma_hat for the percentile scale (its quantile times
+      // gamma / Phi^-1((1 + rho) / 2)); both floored at eps
+      const float rs = pct ? p.pct_mult : 1.f;
+      const float aa = fmaxf(st.x * nrm * rs, 1e-10f), ab = fmaxf(st.y * nrm * rs, 1e-10f);
       const float2 mult = make_float2(nrm * qmax * __frcp_rn(aa), nrm * qmax * __frcp_rn(ab));
       if (tid == 0) { p.scale[ta] = aa / qmax; if (has_b) p.scale[ta + 1] = ab / qmax; }
       if (active) {
         // fma against 1.5 * 2^23 rounds half-to-even to an integer held in the low mantissa
-        // bits; the low byte of each result is the two's-complement code
+        // bits; the low byte of each result is the two's-complement code. The percentile range
+        // can leave values past +-qmax: clamping the rounded value to magic +- qmax clips them
         const float2 magic = make_float2(12582912.f, 12582912.f);
         uint32_t wa[8], wb[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-          const float2 r0 = __ffma2_rn(v[4 * k], mult, magic);
-          const float2 r1 = __ffma2_rn(v[4 * k + 1], mult, magic);
-          const float2 r2 = __ffma2_rn(v[4 * k + 2], mult, magic);
-          const float2 r3 = __ffma2_rn(v[4 * k + 3], mult, magic);
+          float2 r0 = __ffma2_rn(v[4 * k], mult, magic);
+          float2 r1 = __ffma2_rn(v[4 * k + 1], mult, magic);
+          float2 r2 = __ffma2_rn(v[4 * k + 2], mult, magic);
+          float2 r3 = __ffma2_rn(v[4 * k + 3], mult, magic);
+          if (pct) {
+            r0 = clamp_code(r0); r1 = clamp_code(r1); r2 = clamp_code(r2); r3 = clamp_code(r3);
+          }
           wa[k] = pack4(r0.x, r1.x, r2.x, r3.x);
           wb[k] = pack4(r0.y, r1.y, r2.y, r3.y);
         }
@@ -941,6 +1060,20 @@ void* kern_pair_h(int hlog2) {
 // widths up to 8192 (at most 256 threads) run two tokens per pass
 constexpr int kPairMaxD = 8192;
 
+// CentriQ App. B.3 (Tab. 3): activation quantile rho and clip factor gamma*
+constexpr double kPctRho = 0.9995;
+constexpr double kPctGamma = 2.5591;
+
+// Phi^-1(p) for the standard normal, by bisection on Phi(x) = erfc(-x / sqrt 2) / 2 (monotone)
+double inv_normal_cdf(double prob) {
+  double lo = -40.0, hi = 40.0;
+  for (int i = 0; i < 200; ++i) {
+    const double mid = 0.5 * (lo + hi);
+    if (0.5 * std::erfc(-mid / std::sqrt(2.0)) < prob) lo = mid; else hi = mid;
+  }
+  return 0.5 * (lo + hi);
+}
+
 }  // namespace
 
 int rq_hmode(int h) { return h <= 32 ? 0 : (h <= 128 ? 1 : 2); }
@@ -1010,24 +1143,12 @@ oq_status launch_rotate_quant(const RqArgs& a, cudaStream_t s) {
         cfg.nthr = nthr;
         ce = allow_max_dynamic_smem(cfg.fn);
         if (ce != cudaSuccess) return cuda_fail(ce, "cudaFuncSetAttribute(rotate_quant)");
-        // a second landing pair lets each CTA have the next pair's rows in flight for a whole
-        // pass; it is taken when it costs no resident CTA
+        cfg.nbuf = 1;
+        cfg.smem = (size_t)cfg.nbuf * 2 * row_stride + (size_t)(nthr / 32) * 4096 +
+                   (a.rounds == 2 ? (size_t)(nthr / 32) * 8192 : 0) + 224 * 4 + 16 * 8;
         int best_occ = 0;
-#ifndef OQ_RQ_MAXNBUF
-#define OQ_RQ_MAXNBUF 2
-#endif
-        for (int nb = 1; nb <= OQ_RQ_MAXNBUF; ++nb) {
-          const size_t smem = (size_t)nb * 2 * row_stride + (size_t)(nthr / 32) * 4096 +
-                              (a.rounds == 2 ? (size_t)(nthr / 32) * 8192 : 0) + 96 * 4 + 16 * 8;
-          int occ = 0;
-          ce = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, cfg.fn, nthr, smem);
-          if (ce != cudaSuccess) return cuda_fail(ce, "occupancy(rotate_quant)");
-          if (nb == 1 || occ >= best_occ) {
-            best_occ = occ;
-            cfg.nbuf = nb;
-            cfg.smem = smem;
-          }
-        }
+        ce = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&best_occ, cfg.fn, nthr, cfg.smem);
+        if (ce != cudaSuccess) return cuda_fail(ce, "occupancy(rotate_quant)");
         cfg.grid_per_sm = std::max(best_occ, 1) * nsm;
         cache[key] = cfg;
       } else {
@@ -1071,6 +1192,17 @@ oq_status launch_rotate_quant(const RqArgs& a, cudaStream_t s) {
   p.want_sum = (a.center || a.rowsum) ? 1 : 0;
   p.mask_smem = cfg.mask_smem;
   p.wlayout = a.wlayout;
+  if (a.mode == kRqPercentile) {
+    if (!cfg.pair) return fail(OQ_ERR_UNSUPPORTED, "percentile scale supports d <= %d", kPairMaxD);
+    // linear interpolation between order statistics at pos = rho (d - 1) (ascending order):
+    // ranks floor(pos) and floor(pos) + 1 are the (R-1)-th and (R-2)-th largest, R = d - floor(pos)
+    const double pos = kPctRho * (double)(a.d - 1);
+    const double lo = std::floor(pos);
+    p.pct_r = a.d - (int)lo;
+    p.pct_frac = (float)(pos - lo);
+    p.pct_mult = (float)(kPctGamma / inv_normal_cdf(0.5 * (1.0 + kPctRho)));
+    if (p.pct_r < 2 || p.pct_r > 6) return fail(OQ_ERR_UNSUPPORTED, "percentile rank out of range");
+  }
   p.tab = a.tab;
   p.smask = reinterpret_cast<const uint4*>(a.smask);
   p.ones = reinterpret_cast<const float4*>(a.ones);

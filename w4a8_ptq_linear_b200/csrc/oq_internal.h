@@ -59,7 +59,7 @@ enum : uint32_t {
 };
 
 // ---- rotate + quantize ---------------------------------------------------------------------
-enum RqMode : int { kRqInt8 = 0, kRqInt4 = 1, kRqLloydMax = 2 };
+enum RqMode : int { kRqInt8 = 0, kRqInt4 = 1, kRqLloydMax = 2, kRqPercentile = 3 };
 
 struct RqArgs {
   const void* x = nullptr;   // bf16 [T, ldx]
