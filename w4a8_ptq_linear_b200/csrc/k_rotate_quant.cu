@@ -712,6 +712,8 @@ __global__ void __launch_bounds__(256, 2) k_rotate_quant_pair(const RqParams p) 
   constexpr int HMODE = HLOG2 <= 5 ? 0 : (HLOG2 <= 7 ? 1 : 2);
   // [nbuf landing pairs (row A | row B)] [interleaved words, later the transpose tiles]
   // [round buffer, two rounds only] [reductions, thresholds, barriers]
+  // [transpose tiles, h >= 256 only: their own region, so that no block barrier separates the
+  // gather from the transposes] [round-1 sign masks]
   uint8_t* land = smem;
   uint32_t* wbuf = reinterpret_cast<uint32_t*>(smem + (size_t)p.nbuf * pair_bytes);
   float2* rbuf = reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(wbuf) + nwarps * 4096);
@@ -721,9 +723,12 @@ __global__ void __launch_bounds__(256, 2) k_rotate_quant_pair(const RqParams p) 
   float2* cells = reinterpret_cast<float2*>(red + 32);
   uint64_t* bars = reinterpret_cast<uint64_t*>(red + 96);
   float* pct_lists = red + 128;   // percentile: up to 8 warps x 2 tokens x 6 ranks
-  float* warp_tile = reinterpret_cast<float*>(wbuf) + warp * 1024;
+  float* tiles = red + 224;       // h >= 256: nwarps x 1024 floats
+  uint4* s_mask = reinterpret_cast<uint4*>(tiles + (HMODE == 2 ? nwarps * 1024 : 0));
+  float* warp_tile = tiles + warp * 1024;
 
   if (tid < 32) cells[tid] = p.cells[tid];
+  for (int c = tid; c < d / 8; c += blockDim.x) s_mask[c] = __ldg(p.smask + c);
   if (tid == 0) {
     for (int b = 0; b < p.nbuf; ++b) dev::mbar_init(dev::smem_u32(&bars[b]), 1);
     dev::fence_mbar_init();
@@ -777,7 +782,7 @@ __global__ void __launch_bounds__(256, 2) k_rotate_quant_pair(const RqParams p) 
       for (int m = 0; m < 4; ++m) {
         const int c = tid + m * nact;
         uint4 a = ra[c], bb = rb[c];
-        const uint4 mk = __ldg(p.smask + c);
+        const uint4 mk = s_mask[c];
         if (p.want_sum) psum = __fadd2_rn(psum, chunk_sums(a, bb));
         a.x ^= mk.x; a.y ^= mk.y; a.z ^= mk.z; a.w ^= mk.w;
         bb.x ^= mk.x; bb.y ^= mk.y; bb.z ^= mk.z; bb.w ^= mk.w;
@@ -817,7 +822,6 @@ __global__ void __launch_bounds__(256, 2) k_rotate_quant_pair(const RqParams p) 
         if (p.rowsum) { p.rowsum[ta] = sum.x; if (has_b) p.rowsum[ta + 1] = sum.y; }
       }
     }
-    if constexpr (HMODE == 2) __syncthreads();  // the transpose tiles reuse the gathered words
     block_transform_pair<HLOG2>(v, lane, warp_tile);
     if (p.center && active) {  // centered round = R(x) - mean * R(1)
       const float2 nm = make_float2(-mu.x, -mu.y);
@@ -1058,7 +1062,10 @@ void* kern_pair_h(int hlog2) {
 }
 
 // widths up to 8192 (at most 256 threads) run two tokens per pass
-constexpr int kPairMaxD = 8192;
+#ifndef OQ_RQ_PAIR_MAXD
+#define OQ_RQ_PAIR_MAXD 8192
+#endif
+constexpr int kPairMaxD = OQ_RQ_PAIR_MAXD;
 
 // CentriQ App. B.3 (Tab. 3): activation quantile rho and clip factor gamma*
 constexpr double kPctRho = 0.9995;
@@ -1145,7 +1152,8 @@ oq_status launch_rotate_quant(const RqArgs& a, cudaStream_t s) {
         if (ce != cudaSuccess) return cuda_fail(ce, "cudaFuncSetAttribute(rotate_quant)");
         cfg.nbuf = 1;
         cfg.smem = (size_t)cfg.nbuf * 2 * row_stride + (size_t)(nthr / 32) * 4096 +
-                   (a.rounds == 2 ? (size_t)(nthr / 32) * 8192 : 0) + 224 * 4 + 16 * 8;
+                   (a.rounds == 2 ? (size_t)(nthr / 32) * 8192 : 0) + 224 * 4 +
+                   (hmode == 2 ? (size_t)(nthr / 32) * 4096 : 0) + (size_t)a.d * 2;
         int best_occ = 0;
         ce = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&best_occ, cfg.fn, nthr, cfg.smem);
         if (ce != cudaSuccess) return cuda_fail(ce, "occupancy(rotate_quant)");
