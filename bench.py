@@ -45,10 +45,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic per launch from an ncu capture, valid only for the kernel source it was taken
 # on (sha256 of the .cu file at capture time); null once the kernel has changed.
 NCU_TRAFFIC = {
-    # ncu --set full of the CTA-pair kernel: dram read 17.374 MB + write 24.320 MB
-    ("dit_w4a8", "k_gemm"): {"sha": "402528d7ec8390a691189c53177761c6b535dcdc74d45c9685e55c477e83ab4e", "bytes": 41693952},
-    # ncu --set full of the two-token kernel: dram read 25.243 MB + write 0
-    ("dit_w4a8", "k_rotate_quant"): {"sha": "0b7b5e1f15f6098c7567802bbe7e835898250ee0c98ef022d4bec4e3b69953b3", "bytes": 25242880},
+    # ncu --set full of the CTA-pair kernel (TMA-store epilogue): dram read 17.373 MB + write 0.054 MB
+    ("dit_w4a8", "k_gemm"): {"sha": "46b41ab8fd129e4f0fffd487415f4d4283bb4672db876a2bdf3f7277377eb82b", "bytes": 17427456},
+    # ncu --set full of the two-token kernel: dram read 25.258 MB + write 0
+    ("dit_w4a8", "k_rotate_quant"): {"sha": "93e26d57a081f54e998e6a60544702af974645ab4a8686ba7cf31504ab486b2c", "bytes": 25258496},
 }
 
 
