@@ -84,3 +84,70 @@ def test_mse_closed_form_matches_monte_carlo():
     mc = float(np.mean((x - q) ** 2))
     assert abs(mc - L.lloyd_max_mse(c, t)) < 3e-4 * 1.0
     assert 0.0094 < L.lloyd_max_mse(c, t) < 0.0096
+
+
+# ---- per-width tables: the width-d post-rotation marginal f_d -----------------------------
+
+def test_sphere_d3_is_the_uniform_quantizer():
+    # f_3 is uniform on [-sqrt 3, sqrt 3]: the Lloyd-Max quantizer of a uniform density has
+    # equal cells, centroids at the cell midpoints (closed form)
+    d, L16 = 3, 16
+    c, t = oracle.lloyd_max_sphere(d)
+    r = np.sqrt(3.0)
+    edges = -r + 2 * r * np.arange(L16 + 1) / L16
+    assert np.allclose(t, edges[1:-1], atol=1e-12)
+    assert np.allclose(c, 0.5 * (edges[:-1] + edges[1:]), atol=1e-12)
+
+
+def test_sphere_conditions_by_quadrature():
+    # centroid and midpoint conditions, with the cell integrals of f_d done by adaptive
+    # quadrature of the density itself (not the incomplete-beta / closed-form pair)
+    from scipy.integrate import quad
+    for d in (32, 256, 1920):
+        pdf, _, _ = oracle.sphere_marginal(d)
+        f = lambda y: float(pdf(np.array([y]))[0])
+        c, t = oracle.lloyd_max_sphere(d)
+        r = min(np.sqrt(d), 12.0)      # f_d < 1e-30 beyond 12 for these widths
+        edges = np.concatenate(([-r], t, [r]))
+        total = 0.0
+        for k in range(16):
+            a, b = edges[k], edges[k + 1]
+            p = quad(f, a, b, epsabs=1e-14, epsrel=1e-13, limit=200)[0]
+            mom = quad(lambda y: y * f(y), a, b, epsabs=1e-14, epsrel=1e-13, limit=200)[0]
+            total += p
+            assert abs(mom / p - c[k]) < 1e-9, (d, k)
+        assert abs(total - 1.0) < 1e-10
+        assert np.abs(t - 0.5 * (c[:-1] + c[1:])).max() < 1e-15
+        assert np.allclose(c, -c[::-1], atol=1e-12)
+
+
+def test_sphere_tables_tend_to_the_gaussian_table():
+    # the gap to the N(0, 1) table closes like 1/d
+    cg, tg = oracle.lloyd_max_gaussian()
+    scaled = []
+    for d in (1024, 16384, 262144):
+        c, _ = oracle.lloyd_max_sphere(d)
+        scaled.append(np.abs(c - cg).max() * d)
+    assert max(scaled) / min(scaled) < 1.01
+    assert scaled[-1] / 262144 < 3e-5
+
+
+def test_sphere_distortion_monte_carlo():
+    # quantize sqrt(d) u_1 for random directions u: the empirical MSE matches the table's
+    # distortion computed by quadrature, and beats the Gaussian table on the same samples
+    from scipy.integrate import quad
+    d = 64
+    c, t = oracle.lloyd_max_sphere(d)
+    pdf, _, _ = oracle.sphere_marginal(d)
+    r = np.sqrt(d)
+    edges = np.concatenate(([-r], t, [r]))
+    mse = sum(quad(lambda y: (y - c[k]) ** 2 * float(pdf(np.array([y]))[0]), edges[k],
+                   edges[k + 1], epsabs=1e-14, limit=200)[0] for k in range(16))
+    rng = np.random.default_rng(7)
+    u = rng.standard_normal((200000, d))
+    y = np.sqrt(d) * u[:, 0] / np.linalg.norm(u, axis=1)
+    q = c[np.searchsorted(t, y)]
+    emp = np.mean((y - q) ** 2)
+    assert abs(emp - mse) < 4e-4 * 3
+    cg, tg = oracle.lloyd_max_gaussian()
+    assert emp < np.mean((y - cg[np.searchsorted(tg, y)]) ** 2)
