@@ -59,7 +59,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="dit_w4a8",
-                    choices=["tiny", "dit_w4a8", "narrow_lm", "mlp_up", "mlp_up_pct"])
+                    choices=["tiny", "dit_w4a8", "narrow_lm", "narrow_lm_w", "mlp_up", "mlp_up_pct"])
     ap.add_argument("--tokens", type=int, default=None,
                     help="override the token count (small cases for profiler captures)")
     ap.add_argument("--e2e-steps", type=int, default=100)
@@ -185,7 +185,8 @@ def oracle_setup(wl, x_bits, w_bits):
     import oracle
     import synth
     plan = oracle.rpbh_plan(wl.d, wl.h, wl.rounds, wl.seed)
-    c, t = oracle.lloyd_max_gaussian()
+    c, t = (oracle.lloyd_max_sphere(wl.d) if wl.act == "int4_lloydmax_width"
+            else oracle.lloyd_max_gaussian())
     w_codes, s_w, w1 = oracle.prepare_weights(synth.bf16_to_f64(w_bits), plan, wl.h)
     return plan, c, t, w_codes, s_w, w1
 
@@ -194,7 +195,7 @@ def oracle_pass(wl, setup, x_rows_f64):
     import oracle
     plan, c, t, w_codes, s_w, w1 = setup
     qa = oracle.quantize_activations(x_rows_f64, plan, wl.h, wl.act, wl.center, t)
-    if wl.act == "int4_lloydmax":
+    if wl.act.startswith("int4_lloydmax"):
         acc = oracle.gemm_lloyd_max(qa["codes"], c, w_codes)
     else:
         acc = oracle.gemm_int(qa["codes"], w_codes)
@@ -488,7 +489,7 @@ def main():
     long_region = elapsed_ms > 1000.0
     bf16_peak = peaks.get("bf16_tflops_sustained" if long_region else "bf16_tflops",
                           peaks["bf16_tflops"])
-    tensor_peak = bf16_peak * (INT8_PER_BF16 if wl.act != "int4_lloydmax" else 1.0)
+    tensor_peak = bf16_peak * (INT8_PER_BF16 if not wl.act.startswith("int4_lloydmax") else 1.0)
     hbm_peak = peaks["hbm_gbs"]
     gemm_tops = ops / (gm_ms * 1e-3) / 1e12
     rq_gbs = rq_bytes / (rq_ms * 1e-3) / 1e9
@@ -500,9 +501,9 @@ def main():
     traffic_rq = tr_rq["bytes"] if tr_rq and tr_rq["sha"] == sha_of(kfile_rq) else None
     peak_note = (f"{peak_kind} {'sustained' if long_region else 'burst'} bf16 "
                  f"{bf16_peak} TFLOP/s" + (" x 2 (nominal int8/bf16 ratio)"
-                                           if wl.act != "int4_lloydmax" else ""))
+                                           if not wl.act.startswith("int4_lloydmax") else ""))
     gemm_roof = {"bound": "tensor", "achieved": gemm_tops, "peak": tensor_peak,
-                 "unit": "TOPS" if wl.act != "int4_lloydmax" else "TFLOP/s",
+                 "unit": "TOPS" if not wl.act.startswith("int4_lloydmax") else "TFLOP/s",
                  "frac": gemm_tops / tensor_peak, "traffic": traffic, "kernel": "k_gemm",
                  "peak_source": peak_note, "ms_per_launch": gm_ms}
     rq_roof = {"bound": "hbm", "achieved": rq_gbs, "peak": hbm_peak, "unit": "GB/s",
@@ -514,7 +515,7 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "int8" if wl.act != "int4_lloydmax"
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8" if not wl.act.startswith("int4_lloydmax")
         else "f16", "data": "synthetic", "config": config_of(wl, T, world),
         "rotate_quantize_gbs": rq_gbs, "rotate_quantize_frac_hbm": rq_gbs / hbm_peak,
         "gemm_tops": gemm_tops, "gemm_frac_tensor": gemm_tops / tensor_peak,

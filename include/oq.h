@@ -73,8 +73,15 @@ typedef enum {
   OQ_ACT_INT8_ABSMAX = 0,    /* A8: alpha_t = max|z_t| / 127, codes in -127..127         */
   OQ_ACT_INT4_ABSMAX = 1,    /* A4: alpha_t = max|z_t| / 7,   codes in -7..7             */
   OQ_ACT_INT4_LLOYDMAX = 2,  /* A4: sigma_t = RMS(z_t), nearest of 16 N(0,1) centroids   */
-  OQ_ACT_INT4_PERCENTILE = 3 /* A4: percentile range (below), codes clipped to -7..7     */
+  OQ_ACT_INT4_PERCENTILE = 3, /* A4: percentile range (below), codes clipped to -7..7    */
+  OQ_ACT_INT4_LLOYDMAX_WIDTH = 4 /* A4: as LLOYDMAX with the width-d codebook (below)    */
 } oq_act_kind;
+/* OQ_ACT_INT4_LLOYDMAX_WIDTH (OrbitQuant PR #25 "Default changes": codebook v3 is one table
+ * per width d, solved by Newton's method; CentriQ §2: the codebook is derived from the
+ * post-rotation marginal): codes and GEMM as OQ_ACT_INT4_LLOYDMAX, with the 16-level
+ * MSE-optimal codebook of the marginal of one coordinate of a width-d token normalised to unit
+ * RMS, f_d(y) = c_d (1 - y^2/d)^((d-3)/2) on |y| < sqrt(d) (uniformly random direction; the
+ * N(0,1) codebook is its d -> inf limit). See oq_lloyd_max_codebook_width. */
 /* OQ_ACT_INT4_PERCENTILE (CentriQ §4.2 "Scale and grid", App. B.3 Tab. 3): the spread of the
  * rotated token is sigma_hat_t = q_rho(|z_t|) / Phi^-1((1 + rho) / 2) with rho = 0.9995, where
  * q_rho is the empirical quantile, linear between the order statistics around position
@@ -127,6 +134,12 @@ oq_status oq_rpbh_tables(int d, int round, uint64_t seed, int8_t* signs_host,
  * midpoint conditions (OrbitQuant PR #25: codebook v3 uses a Newton solver).
  * centroids16_host: double[16] ascending; thresholds15_host: double[15] midpoints. */
 oq_status oq_lloyd_max_codebook(double* centroids16_host, double* thresholds15_host);
+
+/* The 16-level Lloyd-Max codebook of the width-d marginal f_d (see OQ_ACT_INT4_LLOYDMAX_WIDTH),
+ * solved by Newton's method on the centroid and midpoint conditions; cell probabilities by
+ * composite Simpson integration of f_d, cell first moments in closed form. Host only.
+ * 32 <= d <= 32768, else OQ_ERR_INVALID_ARG. */
+oq_status oq_lloyd_max_codebook_width(int d, double* centroids16_host, double* thresholds15_host);
 
 /* ---- plan ------------------------------------------------------------------------------ */
 

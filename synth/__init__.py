@@ -64,6 +64,7 @@ class Workload:
     h: int
     rounds: int
     act: str            # "int8_absmax" | "int4_absmax" | "int4_lloydmax" | "int4_percentile"
+                        # | "int4_lloydmax_width"
     center: bool
     mean_var: float     # variance of the per-token mean offset
     outliers: int = 0   # channels scaled by outlier_gain (tiny workload)
@@ -79,6 +80,9 @@ WORKLOADS = {
                          heavy_frac=0.01),
     "narrow_lm": Workload("narrow_lm", 8192, 1920, 1920, 128, 2, "int4_lloydmax", False, 3.0,
                           heavy_frac=0.01),
+    # the same layer with the width-d codebook (per-width tables, codebook v3)
+    "narrow_lm_w": Workload("narrow_lm_w", 8192, 1920, 1920, 128, 2, "int4_lloydmax_width", False,
+                            3.0, heavy_frac=0.01),
     "mlp_up": Workload("mlp_up", 4096, 3072, 12288, 1024, 1, "int4_absmax", True, 5.0),
     # the same layer with CentriQ's percentile per-token scale (§4.2 "Scale and grid")
     "mlp_up_pct": Workload("mlp_up_pct", 4096, 3072, 12288, 1024, 1, "int4_percentile", True,

@@ -57,6 +57,16 @@ def test_newton_codebook_matches_lloyd_iteration(lib):
     assert np.abs(t_lib - t_or).max() < 1e-10
 
 
+def test_width_codebook_matches_lloyd_iteration(lib):
+    # library: Newton with Simpson cell probabilities; oracle: Lloyd iteration with the
+    # incomplete beta function
+    for d in (32, 256, 1920, 3072, 30720):
+        c, t = oq.lloyd_max_codebook_width(d)
+        c_or, t_or = oracle.lloyd_max_sphere(d)
+        assert np.abs(c - c_or).max() < 1e-8 and np.abs(t - t_or).max() < 1e-8, d
+    assert lib.oq_lloyd_max_codebook_width(16, None, None) == oq.OQ_ERR_INVALID_ARG
+
+
 def test_default_policies_match_oracle(lib):
     for d in (256, 1152, 1920, 3072, 4096, 30720):
         assert oq.default_block(d) == oracle.default_block(d)

@@ -16,7 +16,8 @@ pytestmark = pytest.mark.gpu
 
 
 def _oracle_rows(wl, xb_rows, wb, bias=None):
-    c, t = oracle.lloyd_max_gaussian()
+    c, t = (oracle.lloyd_max_sphere(wl.d) if wl.act == "int4_lloydmax_width"
+            else oracle.lloyd_max_gaussian())
     plan = oracle.rpbh_plan(wl.d, wl.h, wl.rounds, wl.seed)
     y, _, _ = oracle.linear_forward(synth.bf16_to_f64(xb_rows), synth.bf16_to_f64(wb), plan,
                                     wl.h, wl.act, wl.center, bias=bias, centroids=c,
@@ -40,7 +41,7 @@ def _gpu_layer(wl, xb, wb, bias_bits=None):
 
 
 @pytest.mark.parametrize("name,T", [("tiny", 64), ("dit_w4a8", 300), ("narrow_lm", 257),
-                                    ("mlp_up", 130), ("mlp_up_pct", 130)])
+                                    ("narrow_lm_w", 257), ("mlp_up", 130), ("mlp_up_pct", 130)])
 def test_layer_matches_oracle(name, T):
     wl, xb, wb = synth.make_inputs(name, T=T)
     y = _gpu_layer(wl, xb, wb)
@@ -56,7 +57,7 @@ def test_layer_with_bias():
     assert rel_fro(y, ref) <= OUT_TOL
 
 
-@pytest.mark.parametrize("name", ["dit_w4a8", "narrow_lm", "mlp_up", "mlp_up_pct"])
+@pytest.mark.parametrize("name", ["dit_w4a8", "narrow_lm", "narrow_lm_w", "mlp_up", "mlp_up_pct"])
 def test_full_size_layer_on_sampled_rows(name):
     wl, xb, wb = synth.make_inputs(name)
     y = _gpu_layer(wl, xb, wb)

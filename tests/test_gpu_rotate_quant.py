@@ -44,6 +44,10 @@ CASES = [
     (31, 6144, 1024, 1, "int4_percentile", True),
     (20, 8192, 512, 1, "int4_percentile", True),
     (7, 256, 64, 1, "int4_percentile", False),
+    # the width-d Lloyd-Max codebook (codebook v3 tables per width)
+    (130, 1920, 128, 2, "int4_lloydmax_width", False),
+    (33, 256, 32, 1, "int4_lloydmax_width", True),
+    (5, 30720, 1024, 1, "int4_lloydmax_width", False),
 ]
 
 
@@ -57,7 +61,8 @@ def run_case(T, d, h, rounds, act, center, seed=0):
     torch.cuda.synchronize()
     st, code = oq.device_status()
     assert st == 0, code
-    thresholds = oracle.lloyd_max_gaussian()[1]
+    thresholds = (oracle.lloyd_max_sphere(d)[1] if act == "int4_lloydmax_width"
+                  else oracle.lloyd_max_gaussian()[1])
     ref = oracle.quantize_activations(synth.bf16_to_f64(xb), oracle.rpbh_plan(d, h, rounds, seed),
                                       h, act, center, thresholds)
     out = {
@@ -89,7 +94,9 @@ def test_rotate_quantize_matches_oracle(T, d, h, rounds, act, center):
         ex = absmax_boundary_mask(ref["rotated"], ref["scale"], 7)
     else:
         gpu = oracle.unpack_nibbles(out["codes"], signed=False)
-        ex = lloyd_max_boundary_mask(ref["rotated"], ref["scale"], oracle.lloyd_max_gaussian()[1])
+        thr = (oracle.lloyd_max_sphere(d)[1] if act == "int4_lloydmax_width"
+               else oracle.lloyd_max_gaussian()[1])
+        ex = lloyd_max_boundary_mask(ref["rotated"], ref["scale"], thr)
     bad, n_ex = compare_codes(gpu, ref["codes"], ex)
     assert bad == 0, f"{bad} codes differ outside the boundary exemption ({n_ex} exempt)"
 

@@ -22,7 +22,8 @@ LIB_PATH = os.path.join(_PKG, "lib", "liboq.so")
 
 OQ_OK, OQ_ERR_INVALID_ARG, OQ_ERR_UNSUPPORTED, OQ_ERR_MISALIGNED = 0, 1, 2, 3
 OQ_ERR_CUDA, OQ_ERR_DEVICE_TIMEOUT, OQ_ERR_NOMEM = 4, 5, 6
-ACT_KINDS = {"int8_absmax": 0, "int4_absmax": 1, "int4_lloydmax": 2, "int4_percentile": 3}
+ACT_KINDS = {"int8_absmax": 0, "int4_absmax": 1, "int4_lloydmax": 2, "int4_percentile": 3,
+             "int4_lloydmax_width": 4}
 OUT_BF16, OUT_ACC = 0, 1
 
 # (name, restype, argtypes) of every exported entry point
@@ -36,6 +37,7 @@ SIGNATURES = [
     ("oq_default_rounds", _I, [_I]),
     ("oq_rpbh_tables", _I, [_I, _I, _U64, _P, _P]),
     ("oq_lloyd_max_codebook", _I, [_P, _P]),
+    ("oq_lloyd_max_codebook_width", _I, [_I, _P, _P]),
     ("oq_plan_create", _I, [ctypes.POINTER(_P), _I, _I, _I, _U64, _I, _I]),
     ("oq_plan_destroy", None, [_P]),
     ("oq_plan_get_rpbh", _I, [_P, _I, _P, _P]),
@@ -126,6 +128,14 @@ def lloyd_max_codebook():
     c = np.empty(16, np.float64)
     t = np.empty(15, np.float64)
     _check(lib().oq_lloyd_max_codebook(c.ctypes.data, t.ctypes.data))
+    return c, t
+
+
+def lloyd_max_codebook_width(d: int):
+    """The library's Newton-solved codebook of the width-d marginal: (centroids, thresholds)."""
+    c = np.empty(16, np.float64)
+    t = np.empty(15, np.float64)
+    _check(lib().oq_lloyd_max_codebook_width(d, c.ctypes.data, t.ctypes.data))
     return c, t
 
 

@@ -177,6 +177,14 @@ oq_status oq_lloyd_max_codebook(double* centroids16_host, double* thresholds15_h
   return OQ_OK;
 }
 
+oq_status oq_lloyd_max_codebook_width(int d, double* centroids16_host,
+                                      double* thresholds15_host) {
+  if (!centroids16_host || !thresholds15_host) return fail(OQ_ERR_INVALID_ARG, "NULL output");
+  if (d < 32 || d > 32768) return fail(OQ_ERR_INVALID_ARG, "d=%d outside [32, 32768]", d);
+  lloyd_max_newton_width(d, centroids16_host, thresholds15_host);
+  return OQ_OK;
+}
+
 oq_status oq_plan_create(oq_plan** out, int d, int h, int rounds, uint64_t seed, int center,
                          oq_act_kind act) {
   if (!out) return fail(OQ_ERR_INVALID_ARG, "NULL plan output");
@@ -187,7 +195,7 @@ oq_status oq_plan_create(oq_plan** out, int d, int h, int rounds, uint64_t seed,
     return fail(OQ_ERR_INVALID_ARG, "h=%d must be a power of two <= 1024 dividing d=%d", h, d);
   if (rounds != 1 && rounds != 2) return fail(OQ_ERR_INVALID_ARG, "rounds=%d not in {1,2}", rounds);
   if (act != OQ_ACT_INT8_ABSMAX && act != OQ_ACT_INT4_ABSMAX && act != OQ_ACT_INT4_LLOYDMAX &&
-      act != OQ_ACT_INT4_PERCENTILE)
+      act != OQ_ACT_INT4_PERCENTILE && act != OQ_ACT_INT4_LLOYDMAX_WIDTH)
     return fail(OQ_ERR_INVALID_ARG, "unknown activation kind %d", (int)act);
   if (act == OQ_ACT_INT4_PERCENTILE && d > 8192)
     return fail(OQ_ERR_UNSUPPORTED, "the percentile scale supports d <= 8192 (d=%d)", d);
@@ -246,7 +254,10 @@ oq_status oq_plan_create(oq_plan** out, int d, int h, int rounds, uint64_t seed,
           }
     for (int i = 0; i < d; ++i) ones[i] = (float)v[i];
   }
-  lloyd_max_newton(p->cb_c, p->cb_t);
+  if (act == OQ_ACT_INT4_LLOYDMAX_WIDTH)
+    lloyd_max_newton_width(d, p->cb_c, p->cb_t);
+  else
+    lloyd_max_newton(p->cb_c, p->cb_t);
   auto release = [&]() {
     if (p->d_tab) cudaFree(p->d_tab);
     if (p->d_smask) cudaFree(p->d_smask);
@@ -326,10 +337,10 @@ oq_status oq_rotate_quantize(const oq_plan* plan, const void* x_bf16, int64_t T,
     return fail(OQ_ERR_MISALIGNED, "x, codes and rotated must be 16-byte aligned");
   oq_status st = check_plan_device(plan);
   if (st != OQ_OK) return st;
-  const int mode = plan->act == OQ_ACT_INT8_ABSMAX     ? kRqInt8
-                   : plan->act == OQ_ACT_INT4_ABSMAX   ? kRqInt4
-                   : plan->act == OQ_ACT_INT4_LLOYDMAX ? kRqLloydMax
-                                                       : kRqPercentile;
+  const int mode = plan->act == OQ_ACT_INT8_ABSMAX       ? kRqInt8
+                   : plan->act == OQ_ACT_INT4_ABSMAX     ? kRqInt4
+                   : plan->act == OQ_ACT_INT4_PERCENTILE ? kRqPercentile
+                                                         : kRqLloydMax;   // either codebook
   return rotate_quantize_impl(plan, x_bf16, T, ldx, codes, scale, plan->center ? mean : nullptr,
                               rotated_f32, nullptr, mode, plan->center, 0,
                               static_cast<cudaStream_t>(stream));
@@ -370,16 +381,17 @@ oq_status oq_gemm_w4a4(const oq_plan* plan, oq_act_kind kind, const uint8_t* a_p
                        int64_t T, int64_t d_in, int64_t d_out, oq_out_kind out_kind, void* out,
                        void* stream) {
   if (kind != OQ_ACT_INT4_ABSMAX && kind != OQ_ACT_INT4_LLOYDMAX &&
-      kind != OQ_ACT_INT4_PERCENTILE)
+      kind != OQ_ACT_INT4_PERCENTILE && kind != OQ_ACT_INT4_LLOYDMAX_WIDTH)
     return fail(OQ_ERR_INVALID_ARG,
-                "oq_gemm_w4a4 takes INT4_ABSMAX, INT4_LLOYDMAX or INT4_PERCENTILE");
-  if (kind == OQ_ACT_INT4_LLOYDMAX && !plan)
+                "oq_gemm_w4a4 takes INT4_ABSMAX, INT4_PERCENTILE or a Lloyd-Max kind");
+  const bool lm = kind == OQ_ACT_INT4_LLOYDMAX || kind == OQ_ACT_INT4_LLOYDMAX_WIDTH;
+  if (lm && !plan)
     return fail(OQ_ERR_INVALID_ARG, "Lloyd-Max GEMM needs the plan's codebook");
   oq_status st = check_gemm_args(a_packed, a_scale, mean, w_packed, w_scale, w_rowsum, bias_bf16,
                                  T, d_in, d_out, (int)out_kind, out);
   if (st != OQ_OK) return st;
   GemmArgs g;
-  g.kind = kind == OQ_ACT_INT4_LLOYDMAX ? kGemmLloydMax : kGemmA4;   // percentile codes: A4
+  g.kind = lm ? kGemmLloydMax : kGemmA4;   // percentile codes run through the A4 GEMM
   g.a = a_packed; g.a_scale = a_scale; g.mean = mean; g.w = w_packed; g.w_scale = w_scale;
   g.w_rowsum = w_rowsum; g.bias = bias_bf16; g.T = T; g.K = d_in; g.N = d_out;
   g.out_acc = out_kind == OQ_OUT_ACC; g.out = out;

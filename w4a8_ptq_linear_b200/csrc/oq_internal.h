@@ -30,6 +30,8 @@ namespace oq {
 uint64_t splitmix64_at(uint64_t key, uint64_t i);
 void rpbh_round_tables(int d, int round, uint64_t seed, int8_t* signs, int32_t* perm);
 void lloyd_max_newton(double c16[16], double t15[15]);
+// 16-level Lloyd-Max codebook of the width-d post-rotation marginal (d >= 4)
+void lloyd_max_newton_width(int d, double c16[16], double t15[15]);
 
 // ---- launch helpers ----------------------------------------------------------------------
 // Raises a kernel's dynamic shared-memory ceiling to the device's opt-in maximum, once per

@@ -102,4 +102,89 @@ void lloyd_max_newton(double c16[16], double t15[15]) {
   t15[7] = 0.0;
 }
 
+// ---- per-width Lloyd-Max -------------------------------------------------------------------
+// OrbitQuant PR #25 solves one codebook per width d (codebook v3). The quantized variable is a
+// coordinate of the token normalised to unit RMS after the rotation; for a uniformly random
+// direction it is y = sqrt(d) u_1, u uniform on the sphere S^(d-1), with density
+//     f_d(y) = c_d (1 - y^2 / d)^((d - 3) / 2),  c_d = Gamma(d/2) / (sqrt(pi d) Gamma((d-1)/2)),
+// on |y| < sqrt(d) (the N(0,1) limit as d grows). Its first moment over a cell is closed form,
+// int_a^b y f_d = m(a) - m(b) with m(t) = c_d d / (d - 1) (1 - t^2 / d)^((d - 1) / 2); cell
+// probabilities are integrated numerically (composite Simpson, steps of 1/2048).
+namespace {
+struct SphereMarginal {
+  double d, r, log_c;
+  explicit SphereMarginal(int dd)
+      : d((double)dd), r(std::sqrt((double)dd)),
+        log_c(std::lgamma(0.5 * dd) - 0.5 * std::log(3.14159265358979323846 * dd) -
+              std::lgamma(0.5 * (dd - 1))) {}
+  double pdf(double y) const {
+    const double q = y * y / d;
+    return q < 1.0 ? std::exp(log_c + 0.5 * (d - 3.0) * std::log1p(-q)) : 0.0;
+  }
+  double tail_moment(double t) const {   // int_t^r y f_d(y) dy, t >= 0
+    const double q = t * t / d;
+    return q < 1.0 ? std::exp(log_c + 0.5 * (d - 1.0) * std::log1p(-q)) * d / (d - 1.0) : 0.0;
+  }
+  double cell_prob(double a, double b) const {   // 0 <= a < b; f_d < 1e-40 beyond 16
+    b = std::min(b, std::min(r, 16.0));
+    if (b <= a) return 0.0;
+    int n = (int)std::ceil((b - a) * 2048.0);
+    n += n & 1;
+    if (n < 2) n = 2;
+    const double h = (b - a) / n;
+    double sum = pdf(a) + pdf(b);
+    for (int i = 1; i < n; ++i) sum += pdf(a + i * h) * ((i & 1) ? 4.0 : 2.0);
+    return sum * h / 3.0;
+  }
+};
+}  // namespace
+
+void lloyd_max_newton_width(int d, double c16[16], double t15[15]) {
+  const SphereMarginal f(d);
+  double c[8];
+  for (int j = 0; j < 8; ++j) c[j] = 0.15 + 0.3 * j;
+  for (int it = 0; it < 100; ++it) {
+    double a[8], b[8], p[8], g[8], F[8];
+    for (int j = 0; j < 8; ++j) {
+      a[j] = (j == 0) ? 0.0 : 0.5 * (c[j - 1] + c[j]);
+      b[j] = (j == 7) ? f.r : 0.5 * (c[j] + c[j + 1]);
+      p[j] = f.cell_prob(a[j], b[j]);
+      g[j] = (f.tail_moment(a[j]) - f.tail_moment(b[j])) / p[j];
+      F[j] = c[j] - g[j];
+    }
+    // Jacobian: dg/da = f(a)(g - a)/P, dg/db = f(b)(b - g)/P, da/dc = db/dc = 1/2
+    double J[8][9];
+    for (int j = 0; j < 8; ++j) {
+      for (int k = 0; k < 8; ++k) J[j][k] = (j == k) ? 1.0 : 0.0;
+      const double dga = (j == 0) ? 0.0 : f.pdf(a[j]) * (g[j] - a[j]) / p[j];
+      const double dgb = (j == 7) ? 0.0 : f.pdf(b[j]) * (b[j] - g[j]) / p[j];
+      if (j > 0) { J[j][j - 1] -= 0.5 * dga; J[j][j] -= 0.5 * dga; }
+      if (j < 7) { J[j][j] -= 0.5 * dgb; J[j][j + 1] -= 0.5 * dgb; }
+      J[j][8] = -F[j];
+    }
+    for (int col = 0; col < 8; ++col) {
+      int piv = col;
+      for (int rr = col + 1; rr < 8; ++rr)
+        if (std::fabs(J[rr][col]) > std::fabs(J[piv][col])) piv = rr;
+      for (int k = 0; k < 9; ++k) std::swap(J[col][k], J[piv][k]);
+      for (int rr = col + 1; rr < 8; ++rr) {
+        const double m = J[rr][col] / J[col][col];
+        for (int k = col; k < 9; ++k) J[rr][k] -= m * J[col][k];
+      }
+    }
+    double dx[8];
+    for (int rr = 7; rr >= 0; --rr) {
+      double sum = J[rr][8];
+      for (int k = rr + 1; k < 8; ++k) sum -= J[rr][k] * dx[k];
+      dx[rr] = sum / J[rr][rr];
+    }
+    double step = 0.0;
+    for (int j = 0; j < 8; ++j) { c[j] += dx[j]; step = std::fmax(step, std::fabs(dx[j])); }
+    if (step < 1e-15) break;
+  }
+  for (int j = 0; j < 8; ++j) { c16[8 + j] = c[j]; c16[7 - j] = -c[j]; }
+  for (int k = 0; k < 15; ++k) t15[k] = 0.5 * (c16[k] + c16[k + 1]);
+  t15[7] = 0.0;
+}
+
 }  // namespace oq
