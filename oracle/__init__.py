@@ -24,7 +24,8 @@ Parity status per function is listed in each module header.
 """
 from .rpbh import (splitmix64_at, rpbh_plan, sylvester_hadamard, rotate, unrotate,
                    rpbh_matrix, default_block, default_rounds)
-from .lloyd_max import lloyd_max_gaussian, lloyd_max_mse, lloyd_max_sphere, sphere_marginal
+from .lloyd_max import (lloyd_max_gaussian, lloyd_max_gaussian_8bit, lloyd_max_mse,
+                        lloyd_max_sphere, sphere_marginal)
 from .quant import (EPS, PCT_RHO, PCT_GAMMA, center, absmax_quantize, lloyd_max_quantize,
                     percentile_quantize, pack_nibbles, unpack_nibbles)
 from .linear import (quantize_activations, prepare_weights, gemm_int, gemm_lloyd_max,
@@ -32,7 +33,8 @@ from .linear import (quantize_activations, prepare_weights, gemm_int, gemm_lloyd
 
 __all__ = [
     "splitmix64_at", "rpbh_plan", "sylvester_hadamard", "rotate", "unrotate", "rpbh_matrix",
-    "default_block", "default_rounds", "lloyd_max_gaussian", "lloyd_max_mse", "lloyd_max_sphere",
+    "default_block", "default_rounds", "lloyd_max_gaussian", "lloyd_max_gaussian_8bit",
+    "lloyd_max_mse", "lloyd_max_sphere",
     "sphere_marginal", "EPS", "center",
     "absmax_quantize", "lloyd_max_quantize", "percentile_quantize", "PCT_RHO", "PCT_GAMMA",
     "pack_nibbles", "unpack_nibbles",

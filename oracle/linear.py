@@ -44,7 +44,7 @@ def quantize_activations(x: np.ndarray, plan, h: int, act: str, center_tokens: b
     z = rotate(xc, plan, h)
     if act in QMAX:
         codes, scale = absmax_quantize(z, QMAX[act])
-    elif act in ("int4_lloydmax", "int4_lloydmax_width"):
+    elif act in ("int4_lloydmax", "int4_lloydmax_width", "int8_lloydmax"):
         codes, scale = lloyd_max_quantize(z, thresholds)
     elif act == "int4_percentile":
         codes, scale = percentile_quantize(z, 7)
@@ -96,7 +96,7 @@ def linear_forward(x, w, plan, h, act, center_tokens, bias=None, centroids=None,
     """The whole quantized layer in float64. Returns (y, activation dict, weight tuple)."""
     qa = quantize_activations(x, plan, h, act, center_tokens, thresholds)
     w_codes, s_w, w1 = prepare_weights(w, plan, h)
-    if act in ("int4_lloydmax", "int4_lloydmax_width"):
+    if act in ("int4_lloydmax", "int4_lloydmax_width", "int8_lloydmax"):
         acc = gemm_lloyd_max(qa["codes"], centroids, w_codes)
     else:
         acc = gemm_int(qa["codes"], w_codes)

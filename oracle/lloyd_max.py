@@ -35,6 +35,8 @@ table; and the distortion against a Monte Carlo of random directions.
 """
 from __future__ import annotations
 
+import functools
+
 import numpy as np
 from scipy.special import betainc, gammaln, ndtr
 
@@ -130,4 +132,15 @@ def lloyd_max_sphere(d: int, levels: int = 16, tol: float = 1e-15, max_iter: int
             break
         c = c_new
     return c, 0.5 * (c[:-1] + c[1:])
+
+
+@functools.lru_cache(maxsize=None)
+def lloyd_max_gaussian_8bit():
+    """(centroids[256], thresholds[255]) of the 256-level N(0, 1) Lloyd-Max quantizer (the
+    A8 Lloyd-Max codes of OrbitQuant PR #25's comparison). Lloyd's iteration converges slowly
+    at 256 levels; it stops when no centroid moves by 1e-13."""
+    c, t = lloyd_max_gaussian(levels=256, tol=1e-13, max_iter=2000000)
+    c.setflags(write=False)
+    t.setflags(write=False)
+    return c, t
 

@@ -151,3 +151,27 @@ def test_sphere_distortion_monte_carlo():
     assert abs(emp - mse) < 4e-4 * 3
     cg, tg = oracle.lloyd_max_gaussian()
     assert emp < np.mean((y - cg[np.searchsorted(tg, y)]) ** 2)
+
+
+# ---- 256 levels: the A8 Lloyd-Max codebook -----------------------------------------------
+
+def test_gaussian_256_levels():
+    from scipy.integrate import quad
+    c, t = oracle.lloyd_max_gaussian_8bit()
+    assert c.shape == (256,) and t.shape == (255,)
+    assert np.all(np.diff(c) > 0) and np.allclose(c, -c[::-1], atol=1e-12)
+    assert np.abs(t - 0.5 * (c[:-1] + c[1:])).max() < 1e-15
+    # centroid condition on sample cells by adaptive quadrature (not the closed form)
+    edges = np.concatenate(([-12.0], t, [12.0]))
+    for k in (0, 40, 127, 128, 200, 255):
+        a, b = edges[k], edges[k + 1]
+        p = quad(_phi, a, b, epsabs=1e-16, epsrel=1e-13)[0]
+        m = quad(lambda x: x * _phi(x), a, b, epsabs=1e-16, epsrel=1e-13)[0]
+        assert abs(m / p - c[k]) < 1e-9 * max(1.0, abs(c[k])), k
+    # Panter and Dite (1951): high-resolution distortion sqrt(3) pi / (2 L^2) for N(0, 1)
+    mse = L.lloyd_max_mse(c, t)
+    assert abs(mse / (np.sqrt(3.0) * np.pi / 2.0 / 256 ** 2) - 1.0) < 0.02
+    # Monte Carlo distortion
+    x = np.random.default_rng(3).standard_normal(2_000_000)
+    emp = np.mean((x - c[np.searchsorted(t, x)]) ** 2)
+    assert abs(emp / mse - 1.0) < 0.04   # tail cells dominate the sampling error
