@@ -59,7 +59,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="dit_w4a8",
-                    choices=["tiny", "dit_w4a8", "narrow_lm", "narrow_lm_w", "mlp_up", "mlp_up_pct"])
+                    choices=["tiny", "dit_w4a8", "dit_lm8", "narrow_lm", "narrow_lm_w", "mlp_up",
+                             "mlp_up_pct"])
     ap.add_argument("--tokens", type=int, default=None,
                     help="override the token count (small cases for profiler captures)")
     ap.add_argument("--e2e-steps", type=int, default=100)
@@ -186,6 +187,7 @@ def oracle_setup(wl, x_bits, w_bits):
     import synth
     plan = oracle.rpbh_plan(wl.d, wl.h, wl.rounds, wl.seed)
     c, t = (oracle.lloyd_max_sphere(wl.d) if wl.act == "int4_lloydmax_width"
+            else oracle.lloyd_max_gaussian_8bit() if wl.act == "int8_lloydmax"
             else oracle.lloyd_max_gaussian())
     w_codes, s_w, w1 = oracle.prepare_weights(synth.bf16_to_f64(w_bits), plan, wl.h)
     return plan, c, t, w_codes, s_w, w1
@@ -195,7 +197,7 @@ def oracle_pass(wl, setup, x_rows_f64):
     import oracle
     plan, c, t, w_codes, s_w, w1 = setup
     qa = oracle.quantize_activations(x_rows_f64, plan, wl.h, wl.act, wl.center, t)
-    if wl.act.startswith("int4_lloydmax"):
+    if "lloydmax" in wl.act:
         acc = oracle.gemm_lloyd_max(qa["codes"], c, w_codes)
     else:
         acc = oracle.gemm_int(qa["codes"], w_codes)
@@ -359,7 +361,8 @@ def main():
         del w
         s = {"x": to_dev(xb), "wp": wp, "ws": ws, "w1": w1,
              "codes": torch.empty((T, wl.d // 2 if plan.packed else wl.d),
-                                  dtype=torch.uint8 if plan.packed else torch.int8, device=dev),
+                                  dtype=torch.int8 if wl.act == "int8_absmax" else torch.uint8,
+                                  device=dev),
              "scale": torch.empty(T, dtype=torch.float32, device=dev),
              "mean": torch.empty(T, dtype=torch.float32, device=dev) if wl.center else None,
              "y": torch.empty((T, wl.n_out), dtype=torch.bfloat16, device=dev)}
@@ -375,6 +378,10 @@ def main():
         if wl.act == "int8_absmax":
             oq.gemm_w4a8(s["codes"], s["scale"], s["wp"], s["ws"], mean=s["mean"],
                          w_rowsum=s["w1"] if wl.center else None, out=s["y"], stream=stream)
+        elif wl.act == "int8_lloydmax":
+            oq.gemm_w4a8_lloydmax(plan, s["codes"], s["scale"], s["wp"], s["ws"], mean=s["mean"],
+                                  w_rowsum=s["w1"] if wl.center else None, out=s["y"],
+                                  stream=stream)
         else:
             oq.gemm_w4a4(plan, wl.act, s["codes"], s["scale"], s["wp"], s["ws"],
                          mean=s["mean"], w_rowsum=s["w1"] if wl.center else None, out=s["y"],
@@ -483,13 +490,13 @@ def main():
     ops = 2.0 * T * wl.d * wl.n_out
     ms_per_step = elapsed_ms / K
     value = whole_job_rate(ops, world, ms_per_step) / 1e12
-    code_bytes = T * wl.d if wl.act == "int8_absmax" else T * wl.d // 2
+    code_bytes = T * wl.d if wl.act.startswith("int8") else T * wl.d // 2
     rq_bytes = T * wl.d * 2 + code_bytes + 4 * T * (2 if wl.center else 1)
     peaks, peak_kind = load_peaks()
     long_region = elapsed_ms > 1000.0
     bf16_peak = peaks.get("bf16_tflops_sustained" if long_region else "bf16_tflops",
                           peaks["bf16_tflops"])
-    tensor_peak = bf16_peak * (INT8_PER_BF16 if not wl.act.startswith("int4_lloydmax") else 1.0)
+    tensor_peak = bf16_peak * (INT8_PER_BF16 if "lloydmax" not in wl.act else 1.0)
     hbm_peak = peaks["hbm_gbs"]
     gemm_tops = ops / (gm_ms * 1e-3) / 1e12
     rq_gbs = rq_bytes / (rq_ms * 1e-3) / 1e9
@@ -501,9 +508,9 @@ def main():
     traffic_rq = tr_rq["bytes"] if tr_rq and tr_rq["sha"] == sha_of(kfile_rq) else None
     peak_note = (f"{peak_kind} {'sustained' if long_region else 'burst'} bf16 "
                  f"{bf16_peak} TFLOP/s" + (" x 2 (nominal int8/bf16 ratio)"
-                                           if not wl.act.startswith("int4_lloydmax") else ""))
+                                           if "lloydmax" not in wl.act else ""))
     gemm_roof = {"bound": "tensor", "achieved": gemm_tops, "peak": tensor_peak,
-                 "unit": "TOPS" if not wl.act.startswith("int4_lloydmax") else "TFLOP/s",
+                 "unit": "TOPS" if "lloydmax" not in wl.act else "TFLOP/s",
                  "frac": gemm_tops / tensor_peak, "traffic": traffic, "kernel": "k_gemm",
                  "peak_source": peak_note, "ms_per_launch": gm_ms}
     rq_roof = {"bound": "hbm", "achieved": rq_gbs, "peak": hbm_peak, "unit": "GB/s",
@@ -515,7 +522,7 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "int8" if not wl.act.startswith("int4_lloydmax")
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8" if "lloydmax" not in wl.act
         else "f16", "data": "synthetic", "config": config_of(wl, T, world),
         "rotate_quantize_gbs": rq_gbs, "rotate_quantize_frac_hbm": rq_gbs / hbm_peak,
         "gemm_tops": gemm_tops, "gemm_frac_tensor": gemm_tops / tensor_peak,

@@ -74,8 +74,14 @@ typedef enum {
   OQ_ACT_INT4_ABSMAX = 1,    /* A4: alpha_t = max|z_t| / 7,   codes in -7..7             */
   OQ_ACT_INT4_LLOYDMAX = 2,  /* A4: sigma_t = RMS(z_t), nearest of 16 N(0,1) centroids   */
   OQ_ACT_INT4_PERCENTILE = 3, /* A4: percentile range (below), codes clipped to -7..7    */
-  OQ_ACT_INT4_LLOYDMAX_WIDTH = 4 /* A4: as LLOYDMAX with the width-d codebook (below)    */
+  OQ_ACT_INT4_LLOYDMAX_WIDTH = 4, /* A4: as LLOYDMAX with the width-d codebook (below)   */
+  OQ_ACT_INT8_LLOYDMAX = 5   /* A8: sigma_t = RMS(z_t), nearest of 256 N(0,1) centroids  */
 } oq_act_kind;
+/* OQ_ACT_INT8_LLOYDMAX (OrbitQuant PR #25 "Default changes": the 8-bit Lloyd-Max activations
+ * that absmax INT8 replaced as the A8 default): codes are uint8 [T, d] indices 0..255 into the
+ * 256-level N(0,1) codebook (oq_lloyd_max_codebook_8bit), code = the number of thresholds
+ * strictly below z / sigma_t; the GEMM (oq_gemm_w4a8_lloydmax) decodes them to fp16 centroids
+ * through a table and runs fp16 x fp16 -> fp32. Limit: d <= 8192. */
 /* OQ_ACT_INT4_LLOYDMAX_WIDTH (OrbitQuant PR #25 "Default changes": codebook v3 is one table
  * per width d, solved by Newton's method; CentriQ §2: the codebook is derived from the
  * post-rotation marginal): codes and GEMM as OQ_ACT_INT4_LLOYDMAX, with the 16-level
@@ -135,6 +141,11 @@ oq_status oq_rpbh_tables(int d, int round, uint64_t seed, int8_t* signs_host,
  * centroids16_host: double[16] ascending; thresholds15_host: double[15] midpoints. */
 oq_status oq_lloyd_max_codebook(double* centroids16_host, double* thresholds15_host);
 
+/* The 256-level N(0,1) Lloyd-Max codebook (OQ_ACT_INT8_LLOYDMAX), solved by Newton's method
+ * on the centroid conditions (tridiagonal Jacobian) from the high-resolution point density.
+ * centroids256_host: double[256] ascending; thresholds255_host: double[255]. Host only. */
+oq_status oq_lloyd_max_codebook_8bit(double* centroids256_host, double* thresholds255_host);
+
 /* The 16-level Lloyd-Max codebook of the width-d marginal f_d (see OQ_ACT_INT4_LLOYDMAX_WIDTH),
  * solved by Newton's method on the centroid and midpoint conditions; cell probabilities by
  * composite Simpson integration of f_d, cell first moments in closed form. Host only.
@@ -162,7 +173,8 @@ oq_status oq_plan_get_rpbh(const oq_plan* plan, int round, int8_t* signs_host,
  * App. B.2, where one prologue centers each token, rotates it and quantizes it with one scale
  * per token; OrbitQuant PR #25 "Runtime work": the pre-rotation runs as a single kernel).
  *   x_bf16       [T, ldx] bf16, ldx >= d, (ldx * 2) % 16 == 0
- *   codes        int8 [T, d] (A8) or uint8 [T, d/2] (A4 kinds)
+ *   codes        int8 [T, d] (A8 absmax), uint8 [T, d] (8-bit Lloyd-Max) or uint8 [T, d/2]
+ *                (A4 kinds)
  *   scale        float [T]: alpha_t (absmax kinds) or sigma_t (Lloyd-Max)
  *   mean         float [T] per-token mean; required iff the plan centers, else ignored
  *   rotated_f32  float [T, d] normalised rotated (centered) values, or NULL (test output) */
@@ -205,6 +217,18 @@ oq_status oq_gemm_w4a4(const oq_plan* plan, oq_act_kind kind, const uint8_t* a_p
                        const float* w_scale, const float* w_rowsum, const void* bias_bf16,
                        int64_t T, int64_t d_in, int64_t d_out, oq_out_kind out_kind,
                        void* out, void* stream);
+
+/* W4A8 GEMM for 8-bit Lloyd-Max codes (OQ_ACT_INT8_LLOYDMAX), same epilogue with
+ * a_scale = sigma_t:
+ *   acc[t,o] = sum_k c[codes[t,k]] * w[o,k]    (fp16 centroids and weights, fp32 accumulation)
+ *   codes     uint8 [T, d_in]; sigma float [T]; `plan` supplies the 256-level codebook and must
+ *             have been created with OQ_ACT_INT8_LLOYDMAX (else OQ_ERR_INVALID_ARG)
+ *   other arguments and out as for oq_gemm_w4a8 (OQ_OUT_ACC gives float32). */
+oq_status oq_gemm_w4a8_lloydmax(const oq_plan* plan, const uint8_t* codes, const float* sigma,
+                                const float* mean, const uint8_t* w_packed, const float* w_scale,
+                                const float* w_rowsum, const void* bias_bf16, int64_t T,
+                                int64_t d_in, int64_t d_out, oq_out_kind out_kind, void* out,
+                                void* stream);
 
 /* Bytes of device workspace oq_linear needs for T tokens (codes, scales, means). */
 size_t oq_linear_workspace_bytes(const oq_plan* plan, int64_t T);

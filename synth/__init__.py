@@ -64,7 +64,7 @@ class Workload:
     h: int
     rounds: int
     act: str            # "int8_absmax" | "int4_absmax" | "int4_lloydmax" | "int4_percentile"
-                        # | "int4_lloydmax_width"
+                        # | "int4_lloydmax_width" | "int8_lloydmax"
     center: bool
     mean_var: float     # variance of the per-token mean offset
     outliers: int = 0   # channels scaled by outlier_gain (tiny workload)
@@ -78,6 +78,10 @@ WORKLOADS = {
     "tiny": Workload("tiny", 64, 256, 256, 64, 1, "int8_absmax", False, 2.0, outliers=4),
     "dit_w4a8": Workload("dit_w4a8", 4096, 3072, 3072, 1024, 1, "int8_absmax", False, 3.0,
                          heavy_frac=0.01),
+    # the DiT-width layer with 8-bit Lloyd-Max activations (the A8 alternative that OrbitQuant
+    # PR #25 compares absmax INT8 against)
+    "dit_lm8": Workload("dit_lm8", 4096, 3072, 3072, 1024, 1, "int8_lloydmax", False, 3.0,
+                        heavy_frac=0.01),
     "narrow_lm": Workload("narrow_lm", 8192, 1920, 1920, 128, 2, "int4_lloydmax", False, 3.0,
                           heavy_frac=0.01),
     # the same layer with the width-d codebook (per-width tables, codebook v3)

@@ -67,6 +67,14 @@ def test_width_codebook_matches_lloyd_iteration(lib):
     assert lib.oq_lloyd_max_codebook_width(16, None, None) == oq.OQ_ERR_INVALID_ARG
 
 
+def test_codebook_256_matches_lloyd_iteration(lib):
+    c, t = oq.lloyd_max_codebook_8bit()
+    c_or, t_or = oracle.lloyd_max_gaussian_8bit()
+    assert np.abs(c - c_or).max() < 1e-8 and np.abs(t - t_or).max() < 1e-8
+    h = ctypes.c_void_p()
+    assert lib.oq_plan_create(ctypes.byref(h), 16384, 1024, 1, 0, 0, 5) == oq.OQ_ERR_UNSUPPORTED
+
+
 def test_default_policies_match_oracle(lib):
     for d in (256, 1152, 1920, 3072, 4096, 30720):
         assert oq.default_block(d) == oracle.default_block(d)

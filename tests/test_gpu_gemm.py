@@ -148,3 +148,39 @@ def test_prepare_weights_matches_oracle(n_out, d, h, rounds):
     bad, _ = compare_codes(gpu, codes, ex)
     assert bad == 0
     plan.close()
+
+
+@pytest.mark.parametrize("T,K,N", [(64, 256, 256), (200, 384, 272), (300, 3072, 3072),
+                                   (2560, 1536, 2560)])
+def test_lloyd_max_8bit_accumulators_and_epilogue(T, K, N):
+    import torch
+    import w4a8_ptq_linear_b200 as oq
+    rng = np.random.default_rng(5 * T + K)
+    codes = rng.integers(0, 256, (T, K))
+    w = rng.integers(-7, 8, (N, K))
+    plan = oq.Plan(K, 64, 1, act="int8_lloydmax")
+    cu = lambda v: torch.from_numpy(np.ascontiguousarray(v)).cuda()
+    ap, wp = cu(codes.astype(np.uint8)), cu(pack_w4_gemm(w))
+    ones = torch.ones(max(T, N), dtype=torch.float32, device="cuda")
+    acc = oq.gemm_w4a8_lloydmax(plan, ap, ones[:T], wp, ones[:N], out_kind=oq.OUT_ACC)
+    acc = acc.cpu().numpy().astype(np.float64)
+    c, _ = oq.lloyd_max_codebook_8bit()
+    c16 = c.astype(np.float16).astype(np.float64)
+    # the same fp16 centroids: only the fp32 accumulation order differs
+    assert rel_fro(acc, oracle.gemm_lloyd_max(codes, c16, w)) < 1e-6
+    c_or, _ = oracle.lloyd_max_gaussian_8bit()
+    assert rel_fro(acc, oracle.gemm_lloyd_max(codes, c_or, w)) < 1e-3
+    # epilogue with scales, rank-1 term and bias
+    scale = rng.uniform(0.001, 0.1, T).astype(np.float32)
+    s_w = rng.uniform(0.001, 0.05, N).astype(np.float32)
+    mean = rng.normal(0, 3, T).astype(np.float32)
+    w1 = rng.normal(0, 1, N).astype(np.float32)
+    bias_bits = synth.make_bias(N, seed=4)
+    y = oq.gemm_w4a8_lloydmax(plan, ap, cu(scale), wp, cu(s_w), mean=cu(mean), w_rowsum=cu(w1),
+                              bias=to_torch_bf16(bias_bits))
+    ref = oracle.epilogue(oracle.gemm_lloyd_max(codes, c_or, w), scale.astype(np.float64),
+                          s_w.astype(np.float64), mean.astype(np.float64), w1.astype(np.float64),
+                          synth.bf16_to_f64(bias_bits))
+    assert rel_fro(y.float().cpu().numpy().astype(np.float64), ref) <= OUT_TOL
+    plan.close()
+

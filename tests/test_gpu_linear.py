@@ -17,6 +17,7 @@ pytestmark = pytest.mark.gpu
 
 def _oracle_rows(wl, xb_rows, wb, bias=None):
     c, t = (oracle.lloyd_max_sphere(wl.d) if wl.act == "int4_lloydmax_width"
+            else oracle.lloyd_max_gaussian_8bit() if wl.act == "int8_lloydmax"
             else oracle.lloyd_max_gaussian())
     plan = oracle.rpbh_plan(wl.d, wl.h, wl.rounds, wl.seed)
     y, _, _ = oracle.linear_forward(synth.bf16_to_f64(xb_rows), synth.bf16_to_f64(wb), plan,
@@ -40,7 +41,8 @@ def _gpu_layer(wl, xb, wb, bias_bits=None):
     return out
 
 
-@pytest.mark.parametrize("name,T", [("tiny", 64), ("dit_w4a8", 300), ("narrow_lm", 257),
+@pytest.mark.parametrize("name,T", [("tiny", 64), ("dit_w4a8", 300), ("dit_lm8", 300),
+                                    ("narrow_lm", 257),
                                     ("narrow_lm_w", 257), ("mlp_up", 130), ("mlp_up_pct", 130)])
 def test_layer_matches_oracle(name, T):
     wl, xb, wb = synth.make_inputs(name, T=T)
@@ -57,7 +59,8 @@ def test_layer_with_bias():
     assert rel_fro(y, ref) <= OUT_TOL
 
 
-@pytest.mark.parametrize("name", ["dit_w4a8", "narrow_lm", "narrow_lm_w", "mlp_up", "mlp_up_pct"])
+@pytest.mark.parametrize("name", ["dit_w4a8", "dit_lm8", "narrow_lm", "narrow_lm_w", "mlp_up",
+                                  "mlp_up_pct"])
 def test_full_size_layer_on_sampled_rows(name):
     wl, xb, wb = synth.make_inputs(name)
     y = _gpu_layer(wl, xb, wb)

@@ -48,6 +48,10 @@ CASES = [
     (130, 1920, 128, 2, "int4_lloydmax_width", False),
     (33, 256, 32, 1, "int4_lloydmax_width", True),
     (5, 30720, 1024, 1, "int4_lloydmax_width", False),
+    # 8-bit Lloyd-Max codes (255 thresholds, binary search)
+    (300, 3072, 1024, 1, "int8_lloydmax", False),
+    (45, 4096, 256, 2, "int8_lloydmax", True),
+    (7, 256, 64, 1, "int8_lloydmax", False),
 ]
 
 
@@ -62,6 +66,7 @@ def run_case(T, d, h, rounds, act, center, seed=0):
     st, code = oq.device_status()
     assert st == 0, code
     thresholds = (oracle.lloyd_max_sphere(d)[1] if act == "int4_lloydmax_width"
+                  else oracle.lloyd_max_gaussian_8bit()[1] if act == "int8_lloydmax"
                   else oracle.lloyd_max_gaussian()[1])
     ref = oracle.quantize_activations(synth.bf16_to_f64(xb), oracle.rpbh_plan(d, h, rounds, seed),
                                       h, act, center, thresholds)
@@ -89,6 +94,10 @@ def test_rotate_quantize_matches_oracle(T, d, h, rounds, act, center):
     if act == "int8_absmax":
         gpu = out["codes"].view(np.int8).astype(np.int64)
         ex = absmax_boundary_mask(ref["rotated"], ref["scale"], 127)
+    elif act == "int8_lloydmax":
+        gpu = out["codes"].view(np.uint8).astype(np.int64)
+        ex = lloyd_max_boundary_mask(ref["rotated"], ref["scale"],
+                                     oracle.lloyd_max_gaussian_8bit()[1])
     elif act in ("int4_absmax", "int4_percentile"):
         gpu = oracle.unpack_nibbles(out["codes"], signed=True)
         ex = absmax_boundary_mask(ref["rotated"], ref["scale"], 7)

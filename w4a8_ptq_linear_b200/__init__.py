@@ -23,7 +23,7 @@ LIB_PATH = os.path.join(_PKG, "lib", "liboq.so")
 OQ_OK, OQ_ERR_INVALID_ARG, OQ_ERR_UNSUPPORTED, OQ_ERR_MISALIGNED = 0, 1, 2, 3
 OQ_ERR_CUDA, OQ_ERR_DEVICE_TIMEOUT, OQ_ERR_NOMEM = 4, 5, 6
 ACT_KINDS = {"int8_absmax": 0, "int4_absmax": 1, "int4_lloydmax": 2, "int4_percentile": 3,
-             "int4_lloydmax_width": 4}
+             "int4_lloydmax_width": 4, "int8_lloydmax": 5}
 OUT_BF16, OUT_ACC = 0, 1
 
 # (name, restype, argtypes) of every exported entry point
@@ -38,6 +38,7 @@ SIGNATURES = [
     ("oq_rpbh_tables", _I, [_I, _I, _U64, _P, _P]),
     ("oq_lloyd_max_codebook", _I, [_P, _P]),
     ("oq_lloyd_max_codebook_width", _I, [_I, _P, _P]),
+    ("oq_lloyd_max_codebook_8bit", _I, [_P, _P]),
     ("oq_plan_create", _I, [ctypes.POINTER(_P), _I, _I, _I, _U64, _I, _I]),
     ("oq_plan_destroy", None, [_P]),
     ("oq_plan_get_rpbh", _I, [_P, _I, _P, _P]),
@@ -45,6 +46,7 @@ SIGNATURES = [
     ("oq_prepare_weights", _I, [_P, _P, _I64, _I64, _P, _P, _P, _P]),
     ("oq_gemm_w4a8", _I, [_P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _P, _P]),
     ("oq_gemm_w4a4", _I, [_P, _I, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _P, _P]),
+    ("oq_gemm_w4a8_lloydmax", _I, [_P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _P, _P]),
     ("oq_linear_workspace_bytes", _SZ, [_P, _I64]),
     ("oq_linear", _I, [_P, _P, _I64, _I64, _P, _P, _P, _P, _I64, _P, _P, _SZ, _P]),
     ("oq_debug_wait_timeout", _I, [_U64, _P]),
@@ -131,6 +133,14 @@ def lloyd_max_codebook():
     return c, t
 
 
+def lloyd_max_codebook_8bit():
+    """The library's Newton-solved 256-level N(0,1) codebook: (centroids, thresholds)."""
+    c = np.empty(256, np.float64)
+    t = np.empty(255, np.float64)
+    _check(lib().oq_lloyd_max_codebook_8bit(c.ctypes.data, t.ctypes.data))
+    return c, t
+
+
 def lloyd_max_codebook_width(d: int):
     """The library's Newton-solved codebook of the width-d marginal: (centroids, thresholds)."""
     c = np.empty(16, np.float64)
@@ -184,7 +194,7 @@ class Plan:
 
     @property
     def packed(self) -> bool:
-        return self.act != "int8_absmax"
+        return self.act not in ("int8_absmax", "int8_lloydmax")
 
     def workspace_bytes(self, T: int) -> int:
         return int(lib().oq_linear_workspace_bytes(self._h, T))
@@ -200,7 +210,8 @@ def rotate_quantize(plan: Plan, x, *, codes=None, scale=None, mean=None, rotated
     dev = x.device
     if codes is None:
         codes = torch.empty((T, plan.d // 2 if plan.packed else plan.d),
-                            dtype=torch.uint8 if plan.packed else torch.int8, device=dev)
+                            dtype=torch.int8 if plan.act == "int8_absmax" else torch.uint8,
+                            device=dev)
     if scale is None:
         scale = torch.empty(T, dtype=torch.float32, device=dev)
     if plan.center and mean is None:
@@ -251,12 +262,25 @@ def gemm_w4a4(plan, kind, a_packed, a_scale, w_packed, w_scale, *, mean=None, w_
     import torch
     T, K = a_packed.shape[0], a_packed.shape[1] * 2
     N = w_packed.shape[0]
-    acc_dt = torch.float32 if kind == "int4_lloydmax" else torch.int32
+    acc_dt = torch.float32 if kind.startswith("int4_lloydmax") else torch.int32
     out = _out(T, N, out_kind, acc_dt, a_packed.device, out)
     _check(lib().oq_gemm_w4a4(plan.handle if plan is not None else None, ACT_KINDS[kind],
                               _ptr(a_packed), _ptr(a_scale), _ptr(mean), _ptr(w_packed),
                               _ptr(w_scale), _ptr(w_rowsum), _ptr(bias), T, K, N, out_kind,
                               _ptr(out), _stream(stream)))
+    return out
+
+
+def gemm_w4a8_lloydmax(plan, codes, sigma, w_packed, w_scale, *, mean=None, w_rowsum=None,
+                       bias=None, out_kind=OUT_BF16, out=None, stream=None):
+    """oq_gemm_w4a8_lloydmax: uint8 [T, K] 8-bit Lloyd-Max codes x packed INT4."""
+    import torch
+    T, K = codes.shape
+    N = w_packed.shape[0]
+    out = _out(T, N, out_kind, torch.float32, codes.device, out)
+    _check(lib().oq_gemm_w4a8_lloydmax(plan.handle, _ptr(codes), _ptr(sigma), _ptr(mean),
+                                       _ptr(w_packed), _ptr(w_scale), _ptr(w_rowsum), _ptr(bias),
+                                       T, K, N, out_kind, _ptr(out), _stream(stream)))
     return out
 
 

@@ -57,6 +57,8 @@
 //   A4       X int4 -> 16 X int8, W int4 -> 16 W int8; kind::i8.
 //   LloydMax X code -> fp16 centroid (register table via prmt), W int4 -> 16 W fp16 (exact);
 //            kind::f16 with fp32 accumulation.
+//   LloydMax8 X 8-bit code -> fp16 centroid through a 256-entry table in shared memory, W as
+//            LloydMax; kind::f16.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -88,20 +90,22 @@ constexpr int NTHREADS = EPI0 + NEPI;
 
 template <int KIND, int CG>
 struct Cfg {
-  static constexpr int BK = (KIND == kGemmLloydMax) ? 64 : 128;   // 128 bytes of K per stage
+  static constexpr bool FP = KIND == kGemmLloydMax || KIND == kGemmLloydMax8;  // kind::f16
+  static constexpr int BK = FP ? 64 : 128;                          // 128 bytes of K per stage
   static constexpr bool XPACK = KIND != kGemmA8;
+  static constexpr int XB = KIND == kGemmLloydMax8 ? BK : BK / 2;  // activation bytes per row
   static constexpr int BNMAX = 128 * CG;                           // tokens per tile, at most
   static constexpr int MAXCH = BNMAX / CH;                         // chunks per tile, at most
   static constexpr int XR = 128;                                   // activation rows per CTA
   // Ring depths. Loads from L2 take a few thousand cycles, so the packed ring, which the
   // converters free only after unpacking, must cover that latency at the MMA's pace.
   static constexpr int SX = XPACK ? 0 : (CG == 2 ? 5 : 4);         // activation ring (A8)
-  static constexpr int SP = CG == 1 ? 4 : (KIND == kGemmA8 ? 6 : (KIND == kGemmA4 ? 6 : 8));
+  static constexpr int SP = CG == 1 ? 4 : (KIND == kGemmLloydMax ? 8 : 6);
   static constexpr int S2 = (KIND == kGemmA4) ? (CG == 2 ? 3 : 2) : (CG == 2 ? 4 : 3);
   static constexpr int WT = BM * 128;                              // W operand tile
   static constexpr int XT = XR * 128;                              // X operand tile (this CTA)
   static constexpr int WP = BM * (BK / 2);                         // packed W per stage
-  static constexpr int XP = XPACK ? XR * (BK / 2) : 0;             // packed X per stage
+  static constexpr int XP = XPACK ? XR * XB : 0;                   // staged X per stage
   static constexpr int P_STAGE = XP + WP;                          // [Xp][Wp]
   static constexpr int CONV_STAGE = WT + (XPACK ? XT : 0);         // [W][X]
   static constexpr int OFF_X = 0;
@@ -113,7 +117,8 @@ struct Cfg {
   static constexpr int OFF_BAR = OFF_TOK + BNMAX * 8;
   static constexpr int NBAR = 2 * SX + 2 * SP + 2 * S2 + 4 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  static constexpr int SMEM = OFF_MISC + 16 + 1024;                // + slack for alignment
+  static constexpr int OFF_LUT8 = OFF_MISC + 16;                   // 8-bit code -> fp16 table
+  static constexpr int SMEM = OFF_LUT8 + (KIND == kGemmLloydMax8 ? 512 : 0) + 1024;
   // 1/16 per widened INT4 operand (see "Integer widening")
   static constexpr float ACC_SCALE = KIND == kGemmA4 ? 1.f / 256.f : 1.f / 16.f;
   static_assert(XT % 1024 == 0 && P_STAGE % 1024 == 0 && CONV_STAGE % 1024 == 0 &&
@@ -132,6 +137,7 @@ struct GemmParams {
   int T, K, N;
   int out_acc;
   uint32_t lut[8];     // Lloyd-Max: fp16 low bytes (0-3) and high bytes (4-7) of c_0..c_15
+  uint32_t lut8[128];  // 8-bit Lloyd-Max: fp16 centroids c_0..c_255, two per word
   unsigned long long* err;
   unsigned long long limit_ns;
 };
@@ -312,6 +318,31 @@ __device__ __forceinline__ void convert_lm_f16(const uint8_t* src, uint8_t* dst,
   }
 }
 
+// 8-bit Lloyd-Max code rows (64 codes per stage) -> fp16 centroid rows of 128 bytes, swizzled,
+// through a 256-entry table in shared memory; the first `rows` rows (rounded up to a pass).
+// Thread ctid takes 16 codes (16-byte group q = ctid & 3) of its rows: chunks 2q and 2q + 1.
+__device__ __forceinline__ void convert_lm8_f16(const uint8_t* src, uint8_t* dst, int ctid,
+                                                const uint16_t* lut, int rows) {
+  constexpr int RSTEP = NCG / 4;
+  const int r0 = ctid >> 2, q = ctid & 3;
+  const uint8_t* s = src + r0 * 64 + q * 16;
+  uint8_t* da = dst + r0 * 128 + (((2 * q) ^ (r0 & 7)) << 4);
+  uint8_t* db = dst + r0 * 128 + (((2 * q + 1) ^ (r0 & 7)) << 4);
+#pragma unroll 1
+  for (int j = 0; j * RSTEP < rows; ++j) {
+    const uint4 in = *reinterpret_cast<const uint4*>(s + j * RSTEP * 64);
+    const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+    uint32_t o[8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      o[2 * k] = (uint32_t)lut[w[k] & 0xFF] | ((uint32_t)lut[(w[k] >> 8) & 0xFF] << 16);
+      o[2 * k + 1] = (uint32_t)lut[(w[k] >> 16) & 0xFF] | ((uint32_t)lut[w[k] >> 24] << 16);
+    }
+    *reinterpret_cast<uint4*>(da + j * RSTEP * 128) = make_uint4(o[0], o[1], o[2], o[3]);
+    *reinterpret_cast<uint4*>(db + j * RSTEP * 128) = make_uint4(o[4], o[5], o[6], o[7]);
+  }
+}
+
 // First K block of a tile. Tiles that run at the same time and share an activation range
 // (neighbouring channel tiles) start their K loops at different blocks, so that they do not all
 // request the same L2 lines at the same moment. Integer accumulation is exact in any order.
@@ -332,6 +363,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint32_t* s_misc = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);  // tmem, abort, epi flag
   volatile uint32_t* s_abort = s_misc + 1;
+  const uint16_t* s_lut8 = reinterpret_cast<const uint16_t*>(smem + C::OFF_LUT8);
+  if constexpr (KIND == kGemmLloydMax8)
+    for (int i = threadIdx.x; i < 128; i += blockDim.x)
+      reinterpret_cast<uint32_t*>(smem + C::OFF_LUT8)[i] = p.lut8[i];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = (CG == 2) ? dev::cluster_ctarank() : 0u;  // 0 = the pair's leader
@@ -454,7 +489,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             dev::mbar_arrive_expect_tx(full_b, (uint32_t)C::P_STAGE);
             dev::tma_load_2d(dev::smem_u32(st + C::XP), &tm_w, kb * (BK / 2), o0, full_b);
             if constexpr (C::XPACK)
-              dev::tma_load_2d(dev::smem_u32(st), &tm_x, kb * (BK / 2), x0, full_b);
+              dev::tma_load_2d(dev::smem_u32(st), &tm_x, kb * C::XB, x0, full_b);
           } else if constexpr (CG == 2) {
             // both halves complete on the leader's barrier, which expects the bytes of both
             if (rank == 0) dev::mbar_arrive_expect_tx(full_b, (uint32_t)(2 * C::XT));
@@ -487,7 +522,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       auto it = tiles();
       int m, t0, nch;
       for (; ok && it.next(m, t0, nch); ++it_n) {
-        const uint32_t idesc = (KIND == kGemmLloydMax) ? dev::idesc_f16(UNIT, nch * CH)
+        const uint32_t idesc = C::FP ? dev::idesc_f16(UNIT, nch * CH)
                                                        : dev::idesc_i8(UNIT, nch * CH);
         const int b = it_n & 1;
         if (*s_abort || !dev::mbar_wait(tempty_bar(b), ((it_n >> 1) & 1u) ^ 1u, p.err,
@@ -521,12 +556,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const uint64_t ad = dev::sdesc_sw128(aw + kk * 32);
             const uint64_t bd = dev::sdesc_sw128(bx + kk * 32);
             if constexpr (CG == 2) {
-              if constexpr (KIND == kGemmLloydMax)
+              if constexpr (C::FP)
                 dev::mma_f16_pair(dt, ad, bd, idesc, (step | kk) != 0);
               else
                 dev::mma_i8_pair(dt, ad, bd, idesc, (step | kk) != 0);
             } else {
-              if constexpr (KIND == kGemmLloydMax)
+              if constexpr (C::FP)
                 dev::mma_f16(dt, ad, bd, idesc, (step | kk) != 0);
               else
                 dev::mma_i8(dt, ad, bd, idesc, (step | kk) != 0);
@@ -576,6 +611,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if constexpr (KIND == kGemmLloydMax) {
           convert_w_f16(st + C::XP, cv, ctid);
           convert_lm_f16(st, cv + C::WT, ctid, lut, rows);
+        } else if constexpr (KIND == kGemmLloydMax8) {
+          convert_w_f16(st + C::XP, cv, ctid);
+          convert_lm8_f16(st, cv + C::WT, ctid, s_lut8, rows);
         } else {
           convert_w_i8(st + C::XP, cv, ctid);
           if constexpr (KIND == kGemmA4) convert_x_i8(st, cv + C::WT, ctid, rows);
@@ -650,7 +688,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (o0 + q * 32 >= p.N) continue;    // this warp's channels all lie past N
         const int n_valid = t_end - c * 32;   // tokens of this chunk inside [0, T)
         if (p.out_acc) {
-          if constexpr (KIND == kGemmLloydMax) {
+          if constexpr (C::FP) {
             float* dst = reinterpret_cast<float*>(p.out) + (int64_t)(t0 + c * 32) * p.N + o;
 #pragma unroll
             for (int jj = 0; jj < 32; ++jj)
@@ -674,7 +712,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const float4 tk = tk4[jj / 2];    // (alpha, mean) of tokens jj and jj + 1
             const float2 s2 = __fmul2_rn(make_float2(tk.x, tk.z), sw2);
             const float2 c2 = __ffma2_rn(make_float2(tk.y, tk.w), w12, bb2);
-            const float2 a2 = (KIND == kGemmLloydMax)
+            const float2 a2 = C::FP
                                   ? make_float2(__uint_as_float(r[jj]), __uint_as_float(r[jj + 1]))
                                   : make_float2((float)(int32_t)r[jj], (float)(int32_t)r[jj + 1]);
             const __nv_bfloat162 y = __float22bfloat162_rn(__ffma2_rn(a2, s2, c2));
@@ -796,9 +834,11 @@ oq_status run(const GemmArgs& g, const GemmParams& p, cudaStream_t s) {
                       (uint64_t)g.N * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE);
   else
     std::memset(&ty, 0, sizeof(ty));
-  if constexpr (C::XPACK)
-    ok &= make_map_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.a, (uint64_t)g.K / 2, (uint64_t)g.T,
-                      (uint64_t)g.K / 2, BK / 2, C::XR, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if constexpr (C::XPACK) {
+    const uint64_t xrow = (uint64_t)g.K * C::XB / BK;   // activation bytes per token
+    ok &= make_map_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.a, xrow, (uint64_t)g.T, xrow, C::XB,
+                      C::XR, CU_TENSOR_MAP_SWIZZLE_NONE);
+  }
   else
     ok &= make_map_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.a, (uint64_t)g.K, (uint64_t)g.T,
                       (uint64_t)g.K, BK, C::XR, CU_TENSOR_MAP_SWIZZLE_128B);
@@ -857,6 +897,10 @@ oq_status launch_gemm(const GemmArgs& g, cudaStream_t s) {
   p.N = (int)g.N;
   p.out_acc = g.out_acc;
   p.out = g.out;
+  if (g.kind == kGemmLloydMax8)
+    for (int i = 0; i < 128; ++i)
+      p.lut8[i] = (uint32_t)f16_bits(g.centroids8[2 * i]) |
+                  ((uint32_t)f16_bits(g.centroids8[2 * i + 1]) << 16);
   if (g.kind == kGemmLloydMax) {
     uint8_t lo[16], hi[16];
     for (int i = 0; i < 16; ++i) {
@@ -877,6 +921,8 @@ oq_status launch_gemm(const GemmArgs& g, cudaStream_t s) {
     case kGemmA4: return small ? run<kGemmA4, 1>(g, p, s) : run<kGemmA4, 2>(g, p, s);
     case kGemmLloydMax:
       return small ? run<kGemmLloydMax, 1>(g, p, s) : run<kGemmLloydMax, 2>(g, p, s);
+    case kGemmLloydMax8:
+      return small ? run<kGemmLloydMax8, 1>(g, p, s) : run<kGemmLloydMax8, 2>(g, p, s);
     default: return fail(OQ_ERR_INVALID_ARG, "unknown GEMM kind");
   }
 }

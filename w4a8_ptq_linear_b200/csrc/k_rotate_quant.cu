@@ -52,6 +52,7 @@ struct RqParams {
   int64_t ldx, T;
   int d, hlog2, center, mode, nbuf, want_sum, mask_smem;
   int wlayout;         // 4-bit absmax codes in the GEMM weight layout (see gemm_layout4)
+  const float* thr8;   // 8-bit Lloyd-Max: 255 ascending thresholds (+ one pad), device
   int pct_r;           // percentile: order statistics needed from the top (2..6)
   float pct_frac;      // percentile: interpolation weight between ranks pct_r-1 and pct_r-2
   float pct_mult;      // percentile: gamma / Phi^-1((1 + rho) / 2)
@@ -155,6 +156,16 @@ __device__ __forceinline__ uint4 gemm_layout4(const uint32_t (&w)[8]) {
 #pragma unroll
   for (int m = 0; m < 4; ++m) o[m] = (w[m] & 0x0F0F0F0Fu) | ((w[m + 4] << 4) & 0xF0F0F0F0u);
   return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// 8-bit Lloyd-Max code of u: the number of the 255 ascending thresholds strictly below u, by a
+// branch-free binary search (the thresholds in shared memory; a tie goes to the lower code).
+__device__ __forceinline__ uint32_t lm8_code(float u, const float* thr) {
+  uint32_t lo = 0;
+#pragma unroll
+  for (uint32_t step = 128; step > 0; step >>= 1)
+    if (thr[lo + step - 1] < u) lo += step;
+  return lo;
 }
 
 // Block transform of the 32 values a thread holds, for h = 2^HLOG2 in one of three shapes.
@@ -725,10 +736,13 @@ __global__ void __launch_bounds__(256, 2) k_rotate_quant_pair(const RqParams p) 
   float* pct_lists = red + 128;   // percentile: up to 8 warps x 2 tokens x 6 ranks
   float* tiles = red + 224;       // h >= 256: nwarps x 1024 floats
   uint4* s_mask = reinterpret_cast<uint4*>(tiles + (HMODE == 2 ? nwarps * 1024 : 0));
+  float* s_thr8 = reinterpret_cast<float*>(s_mask + d / 8);   // 8-bit Lloyd-Max thresholds
   float* warp_tile = tiles + warp * 1024;
 
   if (tid < 32) cells[tid] = p.cells[tid];
   for (int c = tid; c < d / 8; c += blockDim.x) s_mask[c] = __ldg(p.smask + c);
+  if (p.mode == kRqLloydMax8)
+    for (int k = tid; k < 256; k += blockDim.x) s_thr8[k] = __ldg(p.thr8 + k);
   if (tid == 0) {
     for (int b = 0; b < p.nbuf; ++b) dev::mbar_init(dev::smem_u32(&bars[b]), 1);
     dev::fence_mbar_init();
@@ -750,7 +764,8 @@ __global__ void __launch_bounds__(256, 2) k_rotate_quant_pair(const RqParams p) 
     for (int b = 0; b < p.nbuf; ++b)
       if ((int64_t)blockIdx.x + (int64_t)b * G < NP) issue(b, (int64_t)blockIdx.x + (int64_t)b * G);
 
-  const bool lm = p.mode == kRqLloydMax;
+  const bool lm8 = p.mode == kRqLloydMax8;
+  const bool lm = p.mode == kRqLloydMax || lm8;   // RMS scale
   const float nrm = p.inv_norm;
   int it = 0;
   bool aborted = false;
@@ -929,7 +944,31 @@ __global__ void __launch_bounds__(256, 2) k_rotate_quant_pair(const RqParams p) 
       const float sb = fmaxf(sqrtf(st.y * nrm * nrm / (float)d), 1e-10f);
       const float2 mult = make_float2(nrm * __frcp_rn(sa), nrm * __frcp_rn(sb));
       if (tid == 0) { p.scale[ta] = sa; if (has_b) p.scale[ta + 1] = sb; }
-      if (active) {
+      if (active && lm8) {
+        // 8-bit codes: the number of the 255 thresholds below u, by binary search in shared
+        // memory; one byte per code, 32 consecutive codes per thread and token
+        uint32_t wa[8], wb[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          uint32_t ca[4], cb[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 u = __fmul2_rn(v[4 * k + e], mult);
+            ca[e] = lm8_code(u.x, s_thr8);
+            cb[e] = lm8_code(u.y, s_thr8);
+          }
+          wa[k] = ca[0] | (ca[1] << 8) | (ca[2] << 16) | (ca[3] << 24);
+          wb[k] = cb[0] | (cb[1] << 8) | (cb[2] << 16) | (cb[3] << 24);
+        }
+        uint4* da = reinterpret_cast<uint4*>(codes + ta * (int64_t)d + base);
+        da[0] = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+        da[1] = make_uint4(wa[4], wa[5], wa[6], wa[7]);
+        if (has_b) {
+          uint4* db = reinterpret_cast<uint4*>(codes + (ta + 1) * (int64_t)d + base);
+          db[0] = make_uint4(wb[0], wb[1], wb[2], wb[3]);
+          db[1] = make_uint4(wb[4], wb[5], wb[6], wb[7]);
+        }
+      } else if (active) {
         uint32_t pa[4] = {0u, 0u, 0u, 0u}, pb[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
         for (int i = 0; i < EP; ++i) {
@@ -1153,7 +1192,7 @@ oq_status launch_rotate_quant(const RqArgs& a, cudaStream_t s) {
         cfg.nbuf = 1;
         cfg.smem = (size_t)cfg.nbuf * 2 * row_stride + (size_t)(nthr / 32) * 4096 +
                    (a.rounds == 2 ? (size_t)(nthr / 32) * 8192 : 0) + 224 * 4 +
-                   (hmode == 2 ? (size_t)(nthr / 32) * 4096 : 0) + (size_t)a.d * 2;
+                   (hmode == 2 ? (size_t)(nthr / 32) * 4096 : 0) + (size_t)a.d * 2 + 1024;
         int best_occ = 0;
         ce = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&best_occ, cfg.fn, nthr, cfg.smem);
         if (ce != cudaSuccess) return cuda_fail(ce, "occupancy(rotate_quant)");
@@ -1200,6 +1239,9 @@ oq_status launch_rotate_quant(const RqArgs& a, cudaStream_t s) {
   p.want_sum = (a.center || a.rowsum) ? 1 : 0;
   p.mask_smem = cfg.mask_smem;
   p.wlayout = a.wlayout;
+  p.thr8 = a.thr8;
+  if (a.mode == kRqLloydMax8 && !cfg.pair)
+    return fail(OQ_ERR_UNSUPPORTED, "8-bit Lloyd-Max codes support d <= %d", kPairMaxD);
   if (a.mode == kRqPercentile) {
     if (!cfg.pair) return fail(OQ_ERR_UNSUPPORTED, "percentile scale supports d <= %d", kPairMaxD);
     // linear interpolation between order statistics at pos = rho (d - 1) (ascending order):

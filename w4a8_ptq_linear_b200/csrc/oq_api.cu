@@ -177,6 +177,12 @@ oq_status oq_lloyd_max_codebook(double* centroids16_host, double* thresholds15_h
   return OQ_OK;
 }
 
+oq_status oq_lloyd_max_codebook_8bit(double* centroids256_host, double* thresholds255_host) {
+  if (!centroids256_host || !thresholds255_host) return fail(OQ_ERR_INVALID_ARG, "NULL output");
+  lloyd_max_newton_256(centroids256_host, thresholds255_host);
+  return OQ_OK;
+}
+
 oq_status oq_lloyd_max_codebook_width(int d, double* centroids16_host,
                                       double* thresholds15_host) {
   if (!centroids16_host || !thresholds15_host) return fail(OQ_ERR_INVALID_ARG, "NULL output");
@@ -195,10 +201,13 @@ oq_status oq_plan_create(oq_plan** out, int d, int h, int rounds, uint64_t seed,
     return fail(OQ_ERR_INVALID_ARG, "h=%d must be a power of two <= 1024 dividing d=%d", h, d);
   if (rounds != 1 && rounds != 2) return fail(OQ_ERR_INVALID_ARG, "rounds=%d not in {1,2}", rounds);
   if (act != OQ_ACT_INT8_ABSMAX && act != OQ_ACT_INT4_ABSMAX && act != OQ_ACT_INT4_LLOYDMAX &&
-      act != OQ_ACT_INT4_PERCENTILE && act != OQ_ACT_INT4_LLOYDMAX_WIDTH)
+      act != OQ_ACT_INT4_PERCENTILE && act != OQ_ACT_INT4_LLOYDMAX_WIDTH &&
+      act != OQ_ACT_INT8_LLOYDMAX)
     return fail(OQ_ERR_INVALID_ARG, "unknown activation kind %d", (int)act);
   if (act == OQ_ACT_INT4_PERCENTILE && d > 8192)
     return fail(OQ_ERR_UNSUPPORTED, "the percentile scale supports d <= 8192 (d=%d)", d);
+  if (act == OQ_ACT_INT8_LLOYDMAX && d > 8192)
+    return fail(OQ_ERR_UNSUPPORTED, "8-bit Lloyd-Max codes support d <= 8192 (d=%d)", d);
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
@@ -258,10 +267,12 @@ oq_status oq_plan_create(oq_plan** out, int d, int h, int rounds, uint64_t seed,
     lloyd_max_newton_width(d, p->cb_c, p->cb_t);
   else
     lloyd_max_newton(p->cb_c, p->cb_t);
+  if (act == OQ_ACT_INT8_LLOYDMAX) lloyd_max_newton_256(p->cb8_c, p->cb8_t);
   auto release = [&]() {
     if (p->d_tab) cudaFree(p->d_tab);
     if (p->d_smask) cudaFree(p->d_smask);
     if (p->d_ones) cudaFree(p->d_ones);
+    if (p->d_thr8) cudaFree(p->d_thr8);
     delete p;
   };
   if (cudaMalloc(&p->d_tab, tab.size() * sizeof(uint16_t)) != cudaSuccess ||
@@ -276,6 +287,13 @@ oq_status oq_plan_create(oq_plan** out, int d, int h, int rounds, uint64_t seed,
                    cudaMemcpyHostToDevice);
   if (e == cudaSuccess)
     e = cudaMemcpy(p->d_ones, ones.data(), ones.size() * sizeof(float), cudaMemcpyHostToDevice);
+  if (e == cudaSuccess && act == OQ_ACT_INT8_LLOYDMAX) {
+    float thr[256];
+    for (int k = 0; k < 255; ++k) thr[k] = (float)p->cb8_t[k];
+    thr[255] = INFINITY;
+    e = cudaMalloc(&p->d_thr8, sizeof(thr));
+    if (e == cudaSuccess) e = cudaMemcpy(p->d_thr8, thr, sizeof(thr), cudaMemcpyHostToDevice);
+  }
   if (e != cudaSuccess) {
     release();
     return cuda_fail(e, "upload plan tables");
@@ -290,13 +308,14 @@ oq_status oq_plan_create(oq_plan** out, int d, int h, int rounds, uint64_t seed,
 
 void oq_plan_destroy(oq_plan* plan) {
   if (!plan) return;
-  if (plan->d_tab || plan->d_smask || plan->d_ones) {
+  if (plan->d_tab || plan->d_smask || plan->d_ones || plan->d_thr8) {
     int cur = -1;
     cudaGetDevice(&cur);
     if (cur != plan->device) cudaSetDevice(plan->device);
     if (plan->d_tab) cudaFree(plan->d_tab);
     if (plan->d_smask) cudaFree(plan->d_smask);
     if (plan->d_ones) cudaFree(plan->d_ones);
+    if (plan->d_thr8) cudaFree(plan->d_thr8);
     if (cur != plan->device && cur >= 0) cudaSetDevice(cur);
   }
   delete plan;
@@ -320,6 +339,7 @@ static oq_status rotate_quantize_impl(const oq_plan* plan, const void* x, int64_
   a.center = center; a.mode = mode; a.tab = plan->d_tab; a.smask = plan->d_smask;
   a.ones = plan->d_ones; a.codes = codes; a.scale = scale;
   a.mean = mean; a.rotated = rotated; a.rowsum = rowsum; a.wlayout = wlayout;
+  a.thr8 = plan->d_thr8;
   for (int i = 0; i < 15; ++i) a.thr[i] = (float)plan->cb_t[i];
   return launch_rotate_quant(a, s);
 }
@@ -340,6 +360,7 @@ oq_status oq_rotate_quantize(const oq_plan* plan, const void* x_bf16, int64_t T,
   const int mode = plan->act == OQ_ACT_INT8_ABSMAX       ? kRqInt8
                    : plan->act == OQ_ACT_INT4_ABSMAX     ? kRqInt4
                    : plan->act == OQ_ACT_INT4_PERCENTILE ? kRqPercentile
+                   : plan->act == OQ_ACT_INT8_LLOYDMAX   ? kRqLloydMax8
                                                          : kRqLloydMax;   // either codebook
   return rotate_quantize_impl(plan, x_bf16, T, ldx, codes, scale, plan->center ? mean : nullptr,
                               rotated_f32, nullptr, mode, plan->center, 0,
@@ -400,12 +421,35 @@ oq_status oq_gemm_w4a4(const oq_plan* plan, oq_act_kind kind, const uint8_t* a_p
   return launch_gemm(g, static_cast<cudaStream_t>(stream));
 }
 
+oq_status oq_gemm_w4a8_lloydmax(const oq_plan* plan, const uint8_t* codes, const float* sigma,
+                                const float* mean, const uint8_t* w_packed, const float* w_scale,
+                                const float* w_rowsum, const void* bias_bf16, int64_t T,
+                                int64_t d_in, int64_t d_out, oq_out_kind out_kind, void* out,
+                                void* stream) {
+  if (!plan || plan->act != OQ_ACT_INT8_LLOYDMAX)
+    return fail(OQ_ERR_INVALID_ARG, "the 8-bit Lloyd-Max GEMM needs an INT8_LLOYDMAX plan");
+  oq_status st = check_gemm_args(codes, sigma, mean, w_packed, w_scale, w_rowsum, bias_bf16, T,
+                                 d_in, d_out, (int)out_kind, out);
+  if (st != OQ_OK) return st;
+  GemmArgs g;
+  g.kind = kGemmLloydMax8;
+  g.a = codes; g.a_scale = sigma; g.mean = mean; g.w = w_packed; g.w_scale = w_scale;
+  g.w_rowsum = w_rowsum; g.bias = bias_bf16; g.T = T; g.K = d_in; g.N = d_out;
+  g.out_acc = out_kind == OQ_OUT_ACC; g.out = out;
+  for (int i = 0; i < 256; ++i) g.centroids8[i] = (float)plan->cb8_c[i];
+  return launch_gemm(g, static_cast<cudaStream_t>(stream));
+}
+
 static size_t round256(size_t v) { return (v + 255) & ~(size_t)255; }
+// one byte per code (A8 absmax and 8-bit Lloyd-Max) or two codes per byte
+static bool codes8(const oq_plan* plan) {
+  return plan->act == OQ_ACT_INT8_ABSMAX || plan->act == OQ_ACT_INT8_LLOYDMAX;
+}
 
 size_t oq_linear_workspace_bytes(const oq_plan* plan, int64_t T) {
   if (!plan || T < 0) return 0;
   const size_t code_bytes =
-      plan->act == OQ_ACT_INT8_ABSMAX ? (size_t)T * plan->d : (size_t)T * (plan->d / 2);
+      codes8(plan) ? (size_t)T * plan->d : (size_t)T * (plan->d / 2);
   return round256(code_bytes) + 2 * round256((size_t)T * 4);
 }
 
@@ -422,7 +466,7 @@ oq_status oq_linear(const oq_plan* plan, const void* x_bf16, int64_t T, int64_t 
     return fail(OQ_ERR_MISALIGNED, "workspace must be 256-byte aligned");
   if (plan->center && !w_rowsum) return fail(OQ_ERR_INVALID_ARG, "centering needs w_rowsum");
   const size_t code_bytes =
-      plan->act == OQ_ACT_INT8_ABSMAX ? (size_t)T * plan->d : (size_t)T * (plan->d / 2);
+      codes8(plan) ? (size_t)T * plan->d : (size_t)T * (plan->d / 2);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   void* codes = ws;
   float* scale = reinterpret_cast<float*>(ws + round256(code_bytes));
@@ -433,6 +477,10 @@ oq_status oq_linear(const oq_plan* plan, const void* x_bf16, int64_t T, int64_t 
   if (plan->act == OQ_ACT_INT8_ABSMAX)
     return oq_gemm_w4a8(static_cast<const int8_t*>(codes), scale, m, w_packed, w_scale, w_rowsum,
                         bias_bf16, T, plan->d, d_out, OQ_OUT_BF16, y_bf16, stream);
+  if (plan->act == OQ_ACT_INT8_LLOYDMAX)
+    return oq_gemm_w4a8_lloydmax(plan, static_cast<const uint8_t*>(codes), scale, m, w_packed,
+                                 w_scale, w_rowsum, bias_bf16, T, plan->d, d_out, OQ_OUT_BF16,
+                                 y_bf16, stream);
   return oq_gemm_w4a4(plan, plan->act, static_cast<const uint8_t*>(codes), scale, m, w_packed,
                       w_scale, w_rowsum, bias_bf16, T, plan->d, d_out, OQ_OUT_BF16, y_bf16,
                       stream);

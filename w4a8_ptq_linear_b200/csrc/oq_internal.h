@@ -22,6 +22,8 @@ struct oq_plan {
   uint32_t* d_smask = nullptr;  // device: d/2 words, round-1 sign of channel j at bit 15 / 31
   float* d_ones = nullptr;      // device: d floats, unnormalised round-1 transform of ones
   double cb_c[16] = {}, cb_t[15] = {};
+  double cb8_c[256] = {}, cb8_t[255] = {};   // 8-bit Lloyd-Max codebook
+  float* d_thr8 = nullptr;      // device: its 255 thresholds (fp32) + one pad
 };
 
 namespace oq {
@@ -32,6 +34,8 @@ void rpbh_round_tables(int d, int round, uint64_t seed, int8_t* signs, int32_t* 
 void lloyd_max_newton(double c16[16], double t15[15]);
 // 16-level Lloyd-Max codebook of the width-d post-rotation marginal (d >= 4)
 void lloyd_max_newton_width(int d, double c16[16], double t15[15]);
+// 256-level N(0,1) Lloyd-Max codebook (8-bit Lloyd-Max activations)
+void lloyd_max_newton_256(double c256[256], double t255[255]);
 
 // ---- launch helpers ----------------------------------------------------------------------
 // Raises a kernel's dynamic shared-memory ceiling to the device's opt-in maximum, once per
@@ -61,7 +65,8 @@ enum : uint32_t {
 };
 
 // ---- rotate + quantize ---------------------------------------------------------------------
-enum RqMode : int { kRqInt8 = 0, kRqInt4 = 1, kRqLloydMax = 2, kRqPercentile = 3 };
+enum RqMode : int { kRqInt8 = 0, kRqInt4 = 1, kRqLloydMax = 2, kRqPercentile = 3,
+                     kRqLloydMax8 = 4 };
 
 struct RqArgs {
   const void* x = nullptr;   // bf16 [T, ldx]
@@ -77,6 +82,7 @@ struct RqArgs {
   float* rowsum = nullptr;   // optional [T]: sum of the row before centering/rotation
   float thr[15] = {};        // Lloyd-Max thresholds (fp32)
   int wlayout = 0;           // kRqInt4 only: write the codes in the GEMM weight layout
+  const float* thr8 = nullptr;  // kRqLloydMax8: 256 floats (255 thresholds + pad), device
 };
 oq_status launch_rotate_quant(const RqArgs& a, cudaStream_t s);
 // Kernel-order gather table helpers: the row position thread t, register i gathers in a
@@ -87,7 +93,7 @@ int rq_round1_index(int d, int j);
 int rq_round_buffer_index(int d, int p);
 
 // ---- GEMM ----------------------------------------------------------------------------------
-enum GemmKind : int { kGemmA8 = 0, kGemmA4 = 1, kGemmLloydMax = 2 };
+enum GemmKind : int { kGemmA8 = 0, kGemmA4 = 1, kGemmLloydMax = 2, kGemmLloydMax8 = 3 };
 
 struct GemmArgs {
   int kind = kGemmA8;
@@ -102,6 +108,7 @@ struct GemmArgs {
   int out_acc = 0;
   void* out = nullptr;
   float centroids[16] = {};
+  float centroids8[256] = {};   // kGemmLloydMax8
 };
 oq_status launch_gemm(const GemmArgs& g, cudaStream_t s);
 

@@ -187,4 +187,58 @@ void lloyd_max_newton_width(int d, double c16[16], double t15[15]) {
   t15[7] = 0.0;
 }
 
+// ---- 256-level N(0,1) Lloyd-Max ----------------------------------------------------------------
+// The same centroid conditions with 128 unknowns (the positive centroids); the Jacobian is
+// tridiagonal and solved by the Thomas algorithm. The start is the high-resolution
+// (Panter-Dite) point density, proportional to phi^(1/3), i.e. quantiles of N(0, 3).
+static double inv_phi(double prob) {   // Phi^-1 by bisection on erfc
+  double lo = -40.0, hi = 40.0;
+  for (int i = 0; i < 200; ++i) {
+    const double mid = 0.5 * (lo + hi);
+    if (0.5 * std::erfc(-mid * 0.70710678118654752440) < prob) lo = mid; else hi = mid;
+  }
+  return 0.5 * (lo + hi);
+}
+
+void lloyd_max_newton_256(double c256[256], double t255[255]) {
+  constexpr int H = 128;
+  double c[H];
+  for (int j = 0; j < H; ++j) c[j] = std::sqrt(3.0) * inv_phi((H + j + 0.5) / (2.0 * H));
+  for (int it = 0; it < 200; ++it) {
+    double a[H], b[H], p[H], g[H], F[H], lo[H], di[H], up[H];
+    for (int j = 0; j < H; ++j) {
+      a[j] = (j == 0) ? 0.0 : 0.5 * (c[j - 1] + c[j]);
+      b[j] = (j == H - 1) ? INFINITY : 0.5 * (c[j] + c[j + 1]);
+      p[j] = cell_prob_pos(a[j], b[j]);
+      const double pb = std::isinf(b[j]) ? 0.0 : pdf(b[j]);
+      g[j] = (pdf(a[j]) - pb) / p[j];
+      F[j] = c[j] - g[j];
+    }
+    for (int j = 0; j < H; ++j) {
+      const double dga = (j == 0) ? 0.0 : pdf(a[j]) * (g[j] - a[j]) / p[j];
+      const double dgb = (j == H - 1) ? 0.0 : pdf(b[j]) * (b[j] - g[j]) / p[j];
+      lo[j] = -0.5 * dga;
+      di[j] = 1.0 - 0.5 * dga - 0.5 * dgb;
+      up[j] = -0.5 * dgb;
+    }
+    // Thomas algorithm for J dx = -F
+    double cp[H], dp[H], dx[H];
+    cp[0] = up[0] / di[0];
+    dp[0] = -F[0] / di[0];
+    for (int j = 1; j < H; ++j) {
+      const double m = di[j] - lo[j] * cp[j - 1];
+      cp[j] = up[j] / m;
+      dp[j] = (-F[j] - lo[j] * dp[j - 1]) / m;
+    }
+    dx[H - 1] = dp[H - 1];
+    for (int j = H - 2; j >= 0; --j) dx[j] = dp[j] - cp[j] * dx[j + 1];
+    double step = 0.0;
+    for (int j = 0; j < H; ++j) { c[j] += dx[j]; step = std::fmax(step, std::fabs(dx[j])); }
+    if (step < 1e-15) break;
+  }
+  for (int j = 0; j < H; ++j) { c256[H + j] = c[j]; c256[H - 1 - j] = -c[j]; }
+  for (int k = 0; k < 255; ++k) t255[k] = 0.5 * (c256[k] + c256[k + 1]);
+  t255[H - 1] = 0.0;
+}
+
 }  // namespace oq
