@@ -80,10 +80,7 @@ constexpr int NCONV = 256;    // converter threads (warps 3-10)
 constexpr int NGROUP = 2;     // converter groups; group g converts the k-blocks j = g mod NGROUP
 constexpr int NCG = NCONV / NGROUP;  // threads per converter group
 constexpr int CONV0 = 96;     // threads before the epilogue that are not converters
-#ifndef OQ_GEMM_EPI_WARPS
-#define OQ_GEMM_EPI_WARPS 8
-#endif
-constexpr int NEPI = 32 * OQ_GEMM_EPI_WARPS;  // epilogue threads (warps from 11 on)
+constexpr int NEPI = 256;     // epilogue threads (warps 11-18), two per TMEM lane quarter
 constexpr int EPW = NEPI / 128;               // epilogue warps per TMEM lane quarter
 constexpr int EPI0 = CONV0 + NCONV;  // first epilogue thread
 constexpr int NTHREADS = EPI0 + NEPI;

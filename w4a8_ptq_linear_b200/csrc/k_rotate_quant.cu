@@ -1101,10 +1101,7 @@ void* kern_pair_h(int hlog2) {
 }
 
 // widths up to 8192 (at most 256 threads) run two tokens per pass
-#ifndef OQ_RQ_PAIR_MAXD
-#define OQ_RQ_PAIR_MAXD 8192
-#endif
-constexpr int kPairMaxD = OQ_RQ_PAIR_MAXD;
+constexpr int kPairMaxD = 8192;
 
 // CentriQ App. B.3 (Tab. 3): activation quantile rho and clip factor gamma*
 constexpr double kPctRho = 0.9995;
