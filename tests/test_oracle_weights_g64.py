@@ -1,0 +1,70 @@
+"""Pins for the oracle's asymmetric grouped INT4 weights (CentriQ Eq. 2, §4.3, App. B.2)."""
+import itertools
+
+import numpy as np
+
+from oracle import weights_g64 as G
+
+
+def _w(n=6, d=256, seed=0):
+    rng = np.random.default_rng(seed)
+    w = rng.standard_normal((n, d))
+    w[0, :64] += 3.0                    # a shifted group
+    w[1, 64:128] *= 0.01                # a narrow group
+    w[2, 128:192] = 0.25                # a constant group
+    return w
+
+
+def test_reconstruction_error_and_extremes():
+    w = _w()
+    q, s, z = G.asym_group_quantize(w)
+    assert q.min() >= 0 and q.max() <= 15
+    wh = G.dequantize(q, s, z)
+    err = np.abs(w - wh).reshape(6, 4, 64)
+    assert np.all(err <= s[..., None] / 2 * (1 + 1e-12) + 1e-15)
+    wg = w.reshape(6, 4, 64)
+    whg = wh.reshape(6, 4, 64)
+    # the minimum and maximum of every group reconstruct exactly (up to rounding)
+    i_lo, i_hi = wg.argmin(axis=2), wg.argmax(axis=2)
+    for r, g in itertools.product(range(6), range(4)):
+        assert abs(whg[r, g, i_lo[r, g]] - wg[r, g, i_lo[r, g]]) <= 1e-12 * (1 + abs(wg[r, g].max()))
+        if wg[r, g].max() > wg[r, g].min():
+            assert abs(whg[r, g, i_hi[r, g]] - wg[r, g, i_hi[r, g]]) <= 1e-12 * (1 + abs(wg[r, g].max()))
+    # a constant group reconstructs exactly
+    assert np.allclose(wh[2, 128:192], 0.25, atol=1e-15)
+
+
+def test_codes_are_the_nearest_grid_point():
+    rng = np.random.default_rng(3)
+    w = rng.uniform(-2, 2, (5, 64))
+    q, s, z = G.asym_group_quantize(w)
+    for r in range(5):
+        grid = s[r, 0] * (np.arange(16) - z[r, 0])
+        best = np.abs(w[r][:, None] - grid[None, :]).argmin(axis=1)
+        d_best = np.abs(w[r] - grid[best])
+        d_q = np.abs(w[r] - grid[q[r]])
+        assert np.all(d_q <= d_best + 1e-12)
+
+
+def test_zero_point_correction_identity():
+    # App. B.2: the Q - 8 integer product with the correction -sigma z' p equals the product
+    # with the dequantized weights
+    rng = np.random.default_rng(5)
+    w = _w(n=7, d=192, seed=2)
+    q, s, z = G.asym_group_quantize(w)
+    a = rng.integers(-7, 8, (9, 192))
+    ref = a.astype(np.float64) @ G.dequantize(q, s, z).T
+    got = G.corrected_product(a, q, s, z)
+    assert np.abs(got - ref).max() <= 1e-10 * np.abs(ref).max()
+
+
+def test_mutation_dropped_correction_is_caught():
+    rng = np.random.default_rng(6)
+    w = _w(n=4, d=128, seed=4)
+    q, s, z = G.asym_group_quantize(w)
+    a = rng.integers(-7, 8, (5, 128))
+    ref = a.astype(np.float64) @ G.dequantize(q, s, z).T
+    ag = a.reshape(5, 2, 64).astype(np.float64)
+    qs = (q.astype(np.float64) - 8).reshape(4, 2, 64)
+    no_corr = np.einsum("tgk,ngk,ng->tn", ag, qs, s)   # plants the slip: no z' p term
+    assert np.abs(no_corr - ref).max() > 1e-3 * np.abs(ref).max()
