@@ -68,3 +68,45 @@ def test_mutation_dropped_correction_is_caught():
     qs = (q.astype(np.float64) - 8).reshape(4, 2, 64)
     no_corr = np.einsum("tgk,ngk,ng->tn", ag, qs, s)   # plants the slip: no z' p term
     assert np.abs(no_corr - ref).max() > 1e-3 * np.abs(ref).max()
+
+
+def test_fp16_storage_codes_nearest_on_stored_grid():
+    # with 16-bit storage the codes are the nearest point of the grid that is decoded
+    rng = np.random.default_rng(8)
+    w = rng.standard_normal((7, 128)) * 0.03
+    w[3, :64] += 0.2                       # a group away from zero (negative shift)
+    w[4, 64:] *= 1e-3                      # a group below the sigma floor
+    q, s, z = G.asym_group_quantize(w, store=np.float16)
+    assert np.array_equal(s.astype(np.float16).astype(np.float64), s)
+    assert np.array_equal(z.astype(np.float16).astype(np.float64), z)
+    assert s.min() >= G.SIGMA_MIN_F16
+    for r in range(7):
+        for g in range(2):
+            grid = s[r, g] * (np.arange(16) - z[r, g])
+            seg = w[r, 64 * g:64 * (g + 1)]
+            d_best = np.abs(seg[:, None] - grid[None, :]).min(axis=1)
+            d_q = np.abs(seg - grid[q[r, 64 * g:64 * (g + 1)]])
+            assert np.all(d_q <= d_best + 1e-12)
+            # and the stored grid still covers the group (error within one step)
+            assert np.all(d_q <= s[r, g] * (0.5 + 2.0 ** -11 * max(1.0, abs(z[r, g]))) + 1e-15)
+
+
+def test_layer_reduces_to_unquantized_for_fine_weights():
+    # the layer oracle with g64 weights, against the unquantized layer: the weight error is
+    # bounded by sigma / 2 per element, so |y - y_exact| <= alpha sum_k |a_k| sigma_k / 2 +
+    # the activation rounding; checked with the activation quantizer error removed by using
+    # the codes' own dequantized activations as input to the exact path
+    from oracle import rpbh_plan, rotate
+    rng = np.random.default_rng(9)
+    d, n, t = 256, 16, 5
+    plan = rpbh_plan(d, 64, 1, 0)
+    x = rng.standard_normal((t, d))
+    w = rng.standard_normal((n, d)) * 0.05
+    y, qa, (q, s, z, w1) = G.linear_forward_g64(x, w, plan, 64, "int4_absmax", True)
+    a = qa["codes"] * qa["scale"][:, None]                # dequantized activations
+    w_r = rotate(w, plan, 64)
+    y_exact = a @ w_r.T + qa["mean"][:, None] * w1[None, :]
+    sig = np.repeat(s, 64, axis=1)                        # [n, d]
+    bound = np.abs(a) @ (sig / 2 + 1e-15).T
+    assert np.all(np.abs(y - y_exact) <= bound * (1 + 1e-9))
+    assert np.abs(y - y_exact).max() > 0                  # the weights really are quantized
