@@ -59,6 +59,25 @@ def asym_group_quantize(w: np.ndarray, g: int = GROUP, bits: int = 4, store=None
     return q.reshape(n, d), sigma, z
 
 
+def asym_group_quantize_f32(w: np.ndarray, g: int = GROUP):
+    """The same codes, sigma and z with every step taken in float32, one IEEE operation at a
+    time (range, division by 15, the fp16 floor and rounding, -min / sigma, w / sigma + z,
+    round half to even): the precision in which the CUDA path takes these integer decisions.
+    Returns (Q int64 [N, d], sigma fp16-valued float64 [N, d/g], z likewise)."""
+    w = np.asarray(w, dtype=np.float32)
+    n, d = w.shape
+    if d % g:
+        raise ValueError("d must be a multiple of the group size")
+    wg = w.reshape(n, d // g, g)
+    lo, hi = wg.min(axis=2), wg.max(axis=2)
+    s = np.maximum((hi - lo) / np.float32(15), np.float32(SIGMA_MIN_F16))
+    sf = s.astype(np.float16).astype(np.float32)
+    zf = (-lo / sf).astype(np.float16).astype(np.float32)
+    v = np.rint(wg / sf[..., None] + zf[..., None])
+    q = np.clip(v, 0, 15).astype(np.int64)
+    return q.reshape(n, d), sf.astype(np.float64), zf.astype(np.float64)
+
+
 def dequantize(q: np.ndarray, sigma: np.ndarray, z: np.ndarray, g: int = GROUP) -> np.ndarray:
     """W_hat = sigma (Q - z) per group (float64)."""
     n, d = q.shape

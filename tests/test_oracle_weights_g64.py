@@ -110,3 +110,17 @@ def test_layer_reduces_to_unquantized_for_fine_weights():
     bound = np.abs(a) @ (sig / 2 + 1e-15).T
     assert np.all(np.abs(y - y_exact) <= bound * (1 + 1e-9))
     assert np.abs(y - y_exact).max() > 0                  # the weights really are quantized
+
+
+def test_f32_decision_agrees_with_the_definition():
+    # the float32 restatement gives the fp64 definition's codes except where the value sits
+    # within float32 rounding of a tie; sigma and z equal unless a fp16 boundary intervenes
+    rng = np.random.default_rng(10)
+    w = (rng.standard_normal((64, 512)) * 0.02).astype(np.float32).astype(np.float64)
+    q64, s64, z64 = G.asym_group_quantize(w, store=np.float16)
+    q32, s32, z32 = G.asym_group_quantize_f32(w)
+    same_grid = (s64 == s32) & (z64 == z32)
+    assert same_grid.mean() > 0.99
+    mask = np.repeat(same_grid, 64, axis=1)
+    assert np.mean(q64[mask] != q32[mask]) < 1e-4
+    assert q32.min() >= 0 and q32.max() <= 15
