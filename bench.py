@@ -60,7 +60,7 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="dit_w4a8",
                     choices=["tiny", "dit_w4a8", "dit_lm8", "narrow_lm", "narrow_lm_w", "mlp_up",
-                             "mlp_up_pct"])
+                             "mlp_up_pct", "mlp_up_g64"])
     ap.add_argument("--tokens", type=int, default=None,
                     help="override the token count (small cases for profiler captures)")
     ap.add_argument("--e2e-steps", type=int, default=100)
@@ -189,6 +189,10 @@ def oracle_setup(wl, x_bits, w_bits):
     c, t = (oracle.lloyd_max_sphere(wl.d) if wl.act == "int4_lloydmax_width"
             else oracle.lloyd_max_gaussian_8bit() if wl.act == "int8_lloydmax"
             else oracle.lloyd_max_gaussian())
+    if wl.weights == "int4_g64":
+        from oracle import weights_g64
+        q, sg, z, w1 = weights_g64.prepare_weights_g64(synth.bf16_to_f64(w_bits), plan, wl.h)
+        return plan, c, t, weights_g64.dequantize(q, sg, z), np.ones(wl.n_out), w1
     w_codes, s_w, w1 = oracle.prepare_weights(synth.bf16_to_f64(w_bits), plan, wl.h)
     return plan, c, t, w_codes, s_w, w1
 
@@ -199,6 +203,8 @@ def oracle_pass(wl, setup, x_rows_f64):
     qa = oracle.quantize_activations(x_rows_f64, plan, wl.h, wl.act, wl.center, t)
     if "lloydmax" in wl.act:
         acc = oracle.gemm_lloyd_max(qa["codes"], c, w_codes)
+    elif wl.weights == "int4_g64":   # w_codes holds the dequantized grouped weights
+        acc = qa["codes"].astype(float) @ w_codes.T
     else:
         acc = oracle.gemm_int(qa["codes"], w_codes)
     return oracle.epilogue(acc, qa["scale"], s_w, qa["mean"] if wl.center else None,
@@ -260,7 +266,8 @@ def run_reference(args, wl, rank):
 
 def config_of(wl, T, n):
     return {"workload": wl.name, "T": T, "d_in": wl.d, "d_out": wl.n_out, "h": wl.h,
-            "rounds": wl.rounds, "act": wl.act, "center": wl.center, "weights": "int4",
+            "rounds": wl.rounds, "act": wl.act, "center": wl.center,
+            "weights": "int4" if wl.weights == "int4_channel" else wl.weights,
             "l2": f"inputs rotate over {RING} sets larger than L2 together",
             "parallelism": "replicas" if n == 1 else f"dp{n} (tokens split, no collective)"}
 
@@ -344,6 +351,7 @@ def main():
             dist.barrier()
 
     _, _, w_bits = synth.make_inputs(wl.name, T=1)
+    g64 = wl.weights == "int4_g64"
     plan = oq.Plan(wl.d, wl.h, wl.rounds, seed=wl.seed, center=wl.center, act=wl.act)
     to_dev = lambda b: torch.from_numpy(np.ascontiguousarray(b)).view(torch.bfloat16).to(dev)
 
@@ -357,9 +365,13 @@ def main():
         if r == 0:
             x_host_bits = xb
         w = to_dev(w_bits)
-        wp, ws, w1 = oq.prepare_weights(plan, w)
+        wsz = None
+        if g64:
+            wp, wsz, ws, w1 = oq.prepare_weights_g64(plan, w)
+        else:
+            wp, ws, w1 = oq.prepare_weights(plan, w)
         del w
-        s = {"x": to_dev(xb), "wp": wp, "ws": ws, "w1": w1,
+        s = {"x": to_dev(xb), "wp": wp, "ws": ws, "w1": w1, "wsz": wsz,
              "codes": torch.empty((T, wl.d // 2 if plan.packed else wl.d),
                                   dtype=torch.int8 if wl.act == "int8_absmax" else torch.uint8,
                                   device=dev),
@@ -375,7 +387,11 @@ def main():
                            stream=stream)
 
     def gemm(s):
-        if wl.act == "int8_absmax":
+        if g64:
+            oq.gemm_w4a4_g64(wl.act, s["codes"], s["scale"], s["wp"], s["wsz"], s["ws"],
+                             mean=s["mean"], w_rowsum=s["w1"] if wl.center else None, out=s["y"],
+                             stream=stream)
+        elif wl.act == "int8_absmax":
             oq.gemm_w4a8(s["codes"], s["scale"], s["wp"], s["ws"], mean=s["mean"],
                          w_rowsum=s["w1"] if wl.center else None, out=s["y"], stream=stream)
         elif wl.act == "int8_lloydmax":
@@ -456,8 +472,13 @@ def main():
         ev_in[k].record(s_in)
         stream.wait_event(ev_in[k])
         stream.wait_event(ev_out[k])         # step i - NB's output has left y_devs[k]
-        oq.linear(plan, x_devs[k], s0["wp"], s0["ws"], s0["w1"] if wl.center else None,
-                  workspace=workspace, out=y_devs[k], stream=stream)
+        if g64:
+            oq.linear_g64(plan, x_devs[k], s0["wp"], s0["wsz"], s0["ws"],
+                          s0["w1"] if wl.center else None, workspace=workspace, out=y_devs[k],
+                          stream=stream)
+        else:
+            oq.linear(plan, x_devs[k], s0["wp"], s0["ws"], s0["w1"] if wl.center else None,
+                      workspace=workspace, out=y_devs[k], stream=stream)
         ev_done[k].record(stream)
         s_out.wait_event(ev_done[k])
         with torch.cuda.stream(s_out):
@@ -496,7 +517,8 @@ def main():
     long_region = elapsed_ms > 1000.0
     bf16_peak = peaks.get("bf16_tflops_sustained" if long_region else "bf16_tflops",
                           peaks["bf16_tflops"])
-    tensor_peak = bf16_peak * (INT8_PER_BF16 if "lloydmax" not in wl.act else 1.0)
+    fp_gemm = "lloydmax" in wl.act or g64          # fp16 operands on the tensor cores
+    tensor_peak = bf16_peak * (INT8_PER_BF16 if not fp_gemm else 1.0)
     hbm_peak = peaks["hbm_gbs"]
     gemm_tops = ops / (gm_ms * 1e-3) / 1e12
     rq_gbs = rq_bytes / (rq_ms * 1e-3) / 1e9
@@ -508,9 +530,9 @@ def main():
     traffic_rq = tr_rq["bytes"] if tr_rq and tr_rq["sha"] == sha_of(kfile_rq) else None
     peak_note = (f"{peak_kind} {'sustained' if long_region else 'burst'} bf16 "
                  f"{bf16_peak} TFLOP/s" + (" x 2 (nominal int8/bf16 ratio)"
-                                           if "lloydmax" not in wl.act else ""))
+                                           if not fp_gemm else ""))
     gemm_roof = {"bound": "tensor", "achieved": gemm_tops, "peak": tensor_peak,
-                 "unit": "TOPS" if "lloydmax" not in wl.act else "TFLOP/s",
+                 "unit": "TOPS" if not fp_gemm else "TFLOP/s",
                  "frac": gemm_tops / tensor_peak, "traffic": traffic, "kernel": "k_gemm",
                  "peak_source": peak_note, "ms_per_launch": gm_ms}
     rq_roof = {"bound": "hbm", "achieved": rq_gbs, "peak": hbm_peak, "unit": "GB/s",
@@ -522,8 +544,7 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "int8" if "lloydmax" not in wl.act
-        else "f16", "data": "synthetic", "config": config_of(wl, T, world),
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8" if not fp_gemm else "f16", "data": "synthetic", "config": config_of(wl, T, world),
         "rotate_quantize_gbs": rq_gbs, "rotate_quantize_frac_hbm": rq_gbs / hbm_peak,
         "gemm_tops": gemm_tops, "gemm_frac_tensor": gemm_tops / tensor_peak,
         "roofline": dominant, "roofline_other": other,

@@ -193,6 +193,26 @@ oq_status oq_prepare_weights(const oq_plan* plan, const void* w_bf16, int64_t n_
                              int64_t ldw, uint8_t* w_packed, float* w_scale,
                              float* w_rowsum, void* stream);
 
+/* Offline preparation of asymmetric grouped INT4 weights (CentriQ §3 Eq. 2; §4.3 "Weight
+ * path": groups of g = 64 consecutive columns of the rotated weight W_R, round to nearest
+ * from the group minimum and maximum; App. B.2: codes stored as Q - 8; App. B.3 Tab. 3:
+ * grid {0..15}, 16-bit scale and zero point). Every row of W goes through the plan's rotation
+ * without centering; then per row o and group g:
+ *   sigma = fp16(max((max - min) / 15, 2^-14)),  z = fp16(-min / sigma),
+ *   Q = clamp(rint(w / sigma + z), 0, 15)        (float32, each step rounded to nearest)
+ * and w_1[o] = sum_k W[o,k] (fp32, before rotation).
+ *   plan      d % 64 == 0; its activation kind is not used here
+ *   w_bf16    [n_out, ldw] bf16, 16-byte aligned, ldw >= d, (ldw * 2) % 16 == 0
+ *   w_packed  uint8 [n_out, d/2] in the GEMM layout, nibble = (Q - 8) two's complement
+ *   w_sz      uint32 [d/64][n_out] (group-major): bits 0-15 fp16 sigma, bits 16-31 fp16 z
+ *   w_scale   float [n_out]: the per-row scale s_o of §4.3, 1 under round to nearest
+ *   w_rowsum  float [n_out]
+ * Allocates n_out * d * 4 bytes of stream-ordered scratch (cudaMallocAsync) for the rotated
+ * rows; errors as for oq_prepare_weights, OQ_ERR_INVALID_ARG if d % 64 != 0. */
+oq_status oq_prepare_weights_g64(const oq_plan* plan, const void* w_bf16, int64_t n_out,
+                                 int64_t ldw, uint8_t* w_packed, uint32_t* w_sz, float* w_scale,
+                                 float* w_rowsum, void* stream);
+
 /* W4A8 GEMM with the fused dequant epilogue (CentriQ Eq. 5 / Eq. 9):
  *   acc[t,o] = sum_k a[t,k] * w[o,k]                     (exact int32)
  *   y[t,o]   = bf16( a_scale[t] * w_scale[o] * acc + mean[t] * w_rowsum[o] + bias[o] )
@@ -218,6 +238,22 @@ oq_status oq_gemm_w4a4(const oq_plan* plan, oq_act_kind kind, const uint8_t* a_p
                        int64_t T, int64_t d_in, int64_t d_out, oq_out_kind out_kind,
                        void* out, void* stream);
 
+/* W4A4 GEMM against asymmetric grouped weights (oq_prepare_weights_g64), same epilogue:
+ *   w_hat[o,k] = fp16(sigma (Q - 8) + fp16(-sigma (z - 8)))   for k in group g = k / 64
+ *   acc[t,o]   = sum_k a[t,k] * w_hat[o,k]    (fp16 operands, fp32 accumulation)
+ *   y[t,o]     = bf16( a_scale[t] * w_scale[o] * acc + mean[t] * w_rowsum[o] + bias[o] )
+ * The zero-point correction of App. B.2 (sigma z' with z' = z - 8, against the group sums of
+ * the activation codes) is carried by the dequantized operand; the result is the same sum.
+ *   kind      OQ_ACT_INT4_ABSMAX or OQ_ACT_INT4_PERCENTILE; a_packed uint8 [T, d_in/2]
+ *   d_in      a multiple of 64; w_sz as written by oq_prepare_weights_g64
+ *   out       bf16 [T, d_out] (OQ_OUT_BF16) or float32 acc [T, d_out] (OQ_OUT_ACC)
+ *   other arguments as for oq_gemm_w4a8. */
+oq_status oq_gemm_w4a4_g64(oq_act_kind kind, const uint8_t* a_packed, const float* a_scale,
+                           const float* mean, const uint8_t* w_packed, const uint32_t* w_sz,
+                           const float* w_scale, const float* w_rowsum, const void* bias_bf16,
+                           int64_t T, int64_t d_in, int64_t d_out, oq_out_kind out_kind,
+                           void* out, void* stream);
+
 /* W4A8 GEMM for 8-bit Lloyd-Max codes (OQ_ACT_INT8_LLOYDMAX), same epilogue with
  * a_scale = sigma_t:
  *   acc[t,o] = sum_k c[codes[t,k]] * w[o,k]    (fp16 centroids and weights, fp32 accumulation)
@@ -241,6 +277,14 @@ oq_status oq_linear(const oq_plan* plan, const void* x_bf16, int64_t T, int64_t 
                     const uint8_t* w_packed, const float* w_scale, const float* w_rowsum,
                     const void* bias_bf16, int64_t d_out, void* y_bf16, void* workspace,
                     size_t workspace_bytes, void* stream);
+
+/* oq_linear against asymmetric grouped weights: oq_rotate_quantize into `workspace`, then
+ * oq_gemm_w4a4_g64. The plan's activation kind must be OQ_ACT_INT4_ABSMAX or
+ * OQ_ACT_INT4_PERCENTILE (else OQ_ERR_INVALID_ARG); workspace as for oq_linear. */
+oq_status oq_linear_g64(const oq_plan* plan, const void* x_bf16, int64_t T, int64_t ldx,
+                        const uint8_t* w_packed, const uint32_t* w_sz, const float* w_scale,
+                        const float* w_rowsum, const void* bias_bf16, int64_t d_out,
+                        void* y_bf16, void* workspace, size_t workspace_bytes, void* stream);
 
 /* Size in bytes of the library's static scratch array used by oq_linear_static_scratch. */
 #define OQ_STATIC_SCRATCH_BYTES (16u << 20)

@@ -71,6 +71,7 @@ class Workload:
     outlier_gain: float = 20.0
     heavy_frac: float = 0.0   # fraction of N(0,1) entries replaced by Student-t(3)
     seed: int = 0
+    weights: str = "int4_channel"   # "int4_channel" (symmetric per output channel) | "int4_g64"
     notes: str = field(default="", compare=False)
 
 
@@ -91,6 +92,9 @@ WORKLOADS = {
     # the same layer with CentriQ's percentile per-token scale (§4.2 "Scale and grid")
     "mlp_up_pct": Workload("mlp_up_pct", 4096, 3072, 12288, 1024, 1, "int4_percentile", True,
                            5.0),
+    # the same layer with CentriQ's weight format: asymmetric INT4 groups of 64 columns (§4.3)
+    "mlp_up_g64": Workload("mlp_up_g64", 4096, 3072, 12288, 1024, 1, "int4_absmax", True, 5.0,
+                           weights="int4_g64"),
 }
 
 

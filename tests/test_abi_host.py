@@ -98,3 +98,23 @@ def test_argument_validation_before_any_cuda_call(lib):
     st = lib.oq_gemm_w4a8(None, None, None, None, None, None, None, 16, 100, 256, 0, None, None)
     assert st == oq.OQ_ERR_INVALID_ARG
     assert b"d_in" in lib.oq_last_error()
+
+
+def test_grouped_weight_arguments_rejected_up_front(lib):
+    # grouped (g = 64) weights: activation kind, d_in % 64 and w_sz are checked before any launch
+    st = lib.oq_gemm_w4a4_g64(oq.ACT_KINDS["int4_lloydmax"], None, None, None, None, None, None,
+                              None, None, 16, 256, 256, 0, None, None)
+    assert st == oq.OQ_ERR_INVALID_ARG
+    assert b"INT4_ABSMAX" in lib.oq_last_error()
+    st = lib.oq_gemm_w4a4_g64(oq.ACT_KINDS["int4_absmax"], None, None, None, None, None, None,
+                              None, None, 16, 96, 256, 0, None, None)
+    assert st == oq.OQ_ERR_INVALID_ARG
+    assert b"64" in lib.oq_last_error()
+    st = lib.oq_gemm_w4a4_g64(oq.ACT_KINDS["int4_absmax"], None, None, None, None, None, None,
+                              None, None, 16, 256, 256, 0, None, None)
+    assert st == oq.OQ_ERR_INVALID_ARG
+    assert b"w_sz" in lib.oq_last_error()
+    assert lib.oq_prepare_weights_g64(None, None, 16, 256, None, None, None, None,
+                                      None) == oq.OQ_ERR_INVALID_ARG
+    assert lib.oq_linear_g64(None, None, 16, 256, None, None, None, None, None, 256, None, None,
+                             0, None) == oq.OQ_ERR_INVALID_ARG

@@ -50,6 +50,9 @@ SIGNATURES = [
     ("oq_linear_workspace_bytes", _SZ, [_P, _I64]),
     ("oq_linear", _I, [_P, _P, _I64, _I64, _P, _P, _P, _P, _I64, _P, _P, _SZ, _P]),
     ("oq_debug_wait_timeout", _I, [_U64, _P]),
+    ("oq_prepare_weights_g64", _I, [_P, _P, _I64, _I64, _P, _P, _P, _P, _P]),
+    ("oq_gemm_w4a4_g64", _I, [_I, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _P, _P]),
+    ("oq_linear_g64", _I, [_P, _P, _I64, _I64, _P, _P, _P, _P, _P, _I64, _P, _P, _SZ, _P]),
     ("oq_linear_static_scratch", _I, [_P, _P, _I64, _I64, _P, _P, _P, _P, _I64, _P, _P]),
 ]
 
@@ -298,6 +301,53 @@ def linear(plan: Plan, x, w_packed, w_scale, w_rowsum=None, bias=None, *, worksp
     _check(lib().oq_linear(plan.handle, _ptr(x), T, x.stride(0), _ptr(w_packed), _ptr(w_scale),
                            _ptr(w_rowsum), _ptr(bias), N, _ptr(out), _ptr(workspace),
                            workspace.numel() * workspace.element_size(), _stream(stream)))
+    return out
+
+
+def prepare_weights_g64(plan: Plan, w, *, stream=None):
+    """oq_prepare_weights_g64 on a bf16 [n_out, d] CUDA tensor: asymmetric INT4 groups of 64.
+
+    Returns (w_packed uint8 [n, d/2], w_sz int32 [d/64, n] of fp16 (sigma, z) pairs,
+    w_scale float32 [n] (ones), w_rowsum float32 [n])."""
+    import torch
+    n = w.shape[0]
+    wp = torch.empty((n, plan.d // 2), dtype=torch.uint8, device=w.device)
+    wsz = torch.empty((plan.d // 64, n), dtype=torch.int32, device=w.device)
+    ws = torch.empty(n, dtype=torch.float32, device=w.device)
+    w1 = torch.empty(n, dtype=torch.float32, device=w.device)
+    _check(lib().oq_prepare_weights_g64(plan.handle, _ptr(w), n, w.stride(0), _ptr(wp), _ptr(wsz),
+                                        _ptr(ws), _ptr(w1), _stream(stream)))
+    return wp, wsz, ws, w1
+
+
+def gemm_w4a4_g64(kind, a_packed, a_scale, w_packed, w_sz, w_scale, *, mean=None, w_rowsum=None,
+                  bias=None, out_kind=OUT_BF16, out=None, stream=None):
+    """oq_gemm_w4a4_g64: packed INT4 [T, K/2] codes x asymmetric grouped INT4 weights."""
+    import torch
+    T, K = a_packed.shape[0], a_packed.shape[1] * 2
+    N = w_packed.shape[0]
+    out = _out(T, N, out_kind, torch.float32, a_packed.device, out)
+    _check(lib().oq_gemm_w4a4_g64(ACT_KINDS[kind], _ptr(a_packed), _ptr(a_scale), _ptr(mean),
+                                  _ptr(w_packed), _ptr(w_sz), _ptr(w_scale), _ptr(w_rowsum),
+                                  _ptr(bias), T, K, N, out_kind, _ptr(out), _stream(stream)))
+    return out
+
+
+def linear_g64(plan: Plan, x, w_packed, w_sz, w_scale, w_rowsum=None, bias=None, *,
+               workspace=None, out=None, stream=None):
+    """oq_linear_g64: the whole layer against asymmetric grouped weights -> bf16 [T, N]."""
+    import torch
+    T = x.shape[0]
+    N = w_packed.shape[0]
+    need = plan.workspace_bytes(T)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=x.device)
+    if out is None:
+        out = torch.empty((T, N), dtype=torch.bfloat16, device=x.device)
+    _check(lib().oq_linear_g64(plan.handle, _ptr(x), T, x.stride(0), _ptr(w_packed), _ptr(w_sz),
+                               _ptr(w_scale), _ptr(w_rowsum), _ptr(bias), N, _ptr(out),
+                               _ptr(workspace), workspace.numel() * workspace.element_size(),
+                               _stream(stream)))
     return out
 
 

@@ -22,7 +22,8 @@ OBJ = os.path.join(ROOT, "_build", "obj")
 LIB_DIR = os.path.join(PKG, "lib")
 LIB = os.path.join(LIB_DIR, "liboq.so")
 
-SOURCES = ["oq_api.cu", "k_rotate_quant.cu", "k_gemm.cu", "oq_plan.cpp", "oq_static_scratch.cu"]
+SOURCES = ["oq_api.cu", "k_rotate_quant.cu", "k_gemm.cu", "k_weights_g64.cu", "oq_plan.cpp",
+           "oq_static_scratch.cu"]
 HEADERS = ["oq_internal.h", "ptx.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

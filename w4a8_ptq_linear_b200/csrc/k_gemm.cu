@@ -87,7 +87,9 @@ constexpr int NTHREADS = EPI0 + NEPI;
 
 template <int KIND, int CG>
 struct Cfg {
-  static constexpr bool FP = KIND == kGemmLloydMax || KIND == kGemmLloydMax8;  // kind::f16
+  static constexpr bool FP = KIND == kGemmLloydMax || KIND == kGemmLloydMax8 ||
+                             KIND == kGemmG64;                       // kind::f16
+  static constexpr bool X4F = KIND == kGemmLloydMax || KIND == kGemmG64;  // 4-bit codes -> fp16
   static constexpr int BK = FP ? 64 : 128;                          // 128 bytes of K per stage
   static constexpr bool XPACK = KIND != kGemmA8;
   static constexpr int XB = KIND == kGemmLloydMax8 ? BK : BK / 2;  // activation bytes per row
@@ -97,7 +99,7 @@ struct Cfg {
   // Ring depths. Loads from L2 take a few thousand cycles, so the packed ring, which the
   // converters free only after unpacking, must cover that latency at the MMA's pace.
   static constexpr int SX = XPACK ? 0 : (CG == 2 ? 5 : 4);         // activation ring (A8)
-  static constexpr int SP = CG == 1 ? 4 : (KIND == kGemmLloydMax ? 8 : 6);
+  static constexpr int SP = CG == 1 ? 4 : (X4F ? 8 : 6);
   static constexpr int S2 = (KIND == kGemmA4) ? (CG == 2 ? 3 : 2) : (CG == 2 ? 4 : 3);
   static constexpr int WT = BM * 128;                              // W operand tile
   static constexpr int XT = XR * 128;                              // X operand tile (this CTA)
@@ -116,8 +118,10 @@ struct Cfg {
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int OFF_LUT8 = OFF_MISC + 16;                   // 8-bit code -> fp16 table
   static constexpr int SMEM = OFF_LUT8 + (KIND == kGemmLloydMax8 ? 512 : 0) + 1024;
-  // 1/16 per widened INT4 operand (see "Integer widening")
-  static constexpr float ACC_SCALE = KIND == kGemmA4 ? 1.f / 256.f : 1.f / 16.f;
+  // 1/16 per widened INT4 operand (see "Integer widening"); the grouped weights are decoded
+  // to their real values and the activation codes to plain integers
+  static constexpr float ACC_SCALE =
+      KIND == kGemmA4 ? 1.f / 256.f : (KIND == kGemmG64 ? 1.f : 1.f / 16.f);
   static_assert(XT % 1024 == 0 && P_STAGE % 1024 == 0 && CONV_STAGE % 1024 == 0 &&
                 XP % 1024 == 0, "operand tiles must stay 1024-byte aligned");
   static_assert(SMEM <= 232448, "shared memory");
@@ -135,6 +139,7 @@ struct GemmParams {
   int out_acc;
   uint32_t lut[8];     // Lloyd-Max: fp16 low bytes (0-3) and high bytes (4-7) of c_0..c_15
   uint32_t lut8[128];  // 8-bit Lloyd-Max: fp16 centroids c_0..c_255, two per word
+  const uint32_t* w_sz;  // grouped weights: [K/64][N] words, fp16 sigma (low half), z (high)
   unsigned long long* err;
   unsigned long long limit_ns;
 };
@@ -278,6 +283,73 @@ __device__ __forceinline__ void convert_w_f16(const uint8_t* src, uint8_t* dst, 
     for (int m = 0; m < 4; ++m) {
       w_pair_f16(__byte_perm(w[m], 0u, 0x4140), P[m][0], Q[m][0]);
       w_pair_f16(__byte_perm(w[m], 0u, 0x4342), P[m][1], Q[m][1]);
+    }
+    uint8_t* row = d + j * RSTEP * 128;
+    *reinterpret_cast<uint4*>(row + (((4 * q + 0) ^ ph) << 4)) =
+        make_uint4(P[0][0], P[0][1], P[1][0], P[1][1]);
+    *reinterpret_cast<uint4*>(row + (((4 * q + 1) ^ ph) << 4)) =
+        make_uint4(P[2][0], P[2][1], P[3][0], P[3][1]);
+    *reinterpret_cast<uint4*>(row + (((4 * q + 2) ^ ph) << 4)) =
+        make_uint4(Q[0][0], Q[0][1], Q[1][0], Q[1][1]);
+    *reinterpret_cast<uint4*>(row + (((4 * q + 3) ^ ph) << 4)) =
+        make_uint4(Q[2][0], Q[2][1], Q[3][0], Q[3][1]);
+  }
+}
+
+// Grouped asymmetric weights (CentriQ §4.3 and App. B.2): the stored nibble is n = Q - 8
+// (two's complement), and row o of group g reconstructs as sigma (Q - z) = sigma n + m with
+// m = -sigma (z - 8), the zero-point correction sigma z' taken into the operand. Both nibbles
+// are first decoded exactly to n (1024 + (n + 8) - 1032; (1024 + 16 (n + 8)) / 16 - 72), then
+// one fused multiply-add per lane pair rounds sigma n + m to fp16 once.
+__device__ __forceinline__ void wg_pair_f16(uint32_t x, __half2 sg, __half2 mg, uint32_t& lo16,
+                                            uint32_t& hi16) {
+  const uint32_t l = (x & 0x000F000Fu) ^ 0x64086408u;
+  const uint32_t h = (x & 0x00F000F0u) ^ 0x64806480u;
+  const __half2 off_l = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));
+  const __half2 sixteenth = __halves2half2(__ushort_as_half(0x2C00), __ushort_as_half(0x2C00));
+  const __half2 off_h = __halves2half2(__ushort_as_half(0xD480), __ushort_as_half(0xD480));
+  const __half2 nl = __hsub2(*reinterpret_cast<const __half2*>(&l), off_l);           // n
+  const __half2 nh = __hfma2(*reinterpret_cast<const __half2*>(&h), sixteenth, off_h);  // n
+  __half2 vl = __hfma2(nl, sg, mg);
+  __half2 vh = __hfma2(nh, sg, mg);
+  lo16 = *reinterpret_cast<uint32_t*>(&vl);
+  hi16 = *reinterpret_cast<uint32_t*>(&vh);
+}
+
+// (sigma, z) word of one row and group -> the broadcast pairs (sigma, sigma) and (m, m),
+// m = -sigma (z - 8) formed in fp32 (z - 8 exact) and rounded to fp16 once more.
+__device__ __forceinline__ void group_consts(uint32_t sz, __half2& sg, __half2& mg) {
+  const __half s = __ushort_as_half((unsigned short)(sz & 0xFFFFu));
+  const __half z = __ushort_as_half((unsigned short)(sz >> 16));
+  const float sf = __half2float(s);
+  const float mf = sf * (8.f - __half2float(z));
+  sg = __halves2half2(s, s);
+  const __half m = __float2half_rn(mf);
+  mg = __halves2half2(m, m);
+}
+
+// Grouped weight rows in the GEMM layout (one group of 64 per stage) -> fp16 rows of the real
+// weights, swizzled as in convert_w_f16; sz0, sz1 are the (sigma, z) words of the thread's rows
+// ctid / 2 and ctid / 2 + NCG / 2 for this group.
+__device__ __forceinline__ void convert_wg_f16(const uint8_t* src, uint8_t* dst, int ctid,
+                                               uint32_t sz0, uint32_t sz1) {
+  constexpr int RSTEP = NCG / 2;
+  static_assert(BM / RSTEP == 2, "two weight rows per converter thread");
+  const int r0 = ctid >> 1, q = ctid & 1;
+  const uint8_t* s = src + r0 * 32 + q * 16;
+  uint8_t* d = dst + r0 * 128;
+  const int ph = r0 & 7;
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    __half2 sg, mg;
+    group_consts(j == 0 ? sz0 : sz1, sg, mg);
+    const uint4 in = *reinterpret_cast<const uint4*>(s + j * RSTEP * 32);
+    const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+    uint32_t P[4][2], Q[4][2];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      wg_pair_f16(__byte_perm(w[m], 0u, 0x4140), sg, mg, P[m][0], Q[m][0]);
+      wg_pair_f16(__byte_perm(w[m], 0u, 0x4342), sg, mg, P[m][1], Q[m][1]);
     }
     uint8_t* row = d + j * RSTEP * 128;
     *reinterpret_cast<uint4*>(row + (((4 * q + 0) ^ ph) << 4)) =
@@ -589,9 +661,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     int m, t0, nch;
     while (ok && it.next(m, t0, nch)) {
       const int rows = nch * CH / CG;   // activation rows of this CTA
+      const int krot = k_rotation(m, nkb);
       for (int step = 0; step < nkb; ++step, ++j) {
         if ((int)(j % NGROUP) != grp) continue;
         const int s = j % SP, c = j % S2;
+        uint32_t sz0 = 0u, sz1 = 0u;   // grouped weights: this k block's (sigma, z) words
+        if constexpr (KIND == kGemmG64) {
+          const int kb = (step + krot) % nkb;
+          const int o = m * UNIT + (int)rank * BM + (ctid >> 1);
+          const uint32_t* src = p.w_sz + (size_t)kb * (size_t)p.N;
+          if (o < p.N) sz0 = __ldg(src + o);
+          if (o + NCG / 2 < p.N) sz1 = __ldg(src + o + NCG / 2);
+        }
         bool w = !*s_abort &&
                  dev::mbar_wait(pfull_bar(s), (j / SP) & 1u, p.err, kSiteGemmFull, p.limit_ns);
         if (w)
@@ -608,6 +689,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if constexpr (KIND == kGemmLloydMax) {
           convert_w_f16(st + C::XP, cv, ctid);
           convert_lm_f16(st, cv + C::WT, ctid, lut, rows);
+        } else if constexpr (KIND == kGemmG64) {
+          convert_wg_f16(st + C::XP, cv, ctid, sz0, sz1);
+          convert_lm_f16(st, cv + C::WT, ctid, lut, rows);   // integer table: code -> n
         } else if constexpr (KIND == kGemmLloydMax8) {
           convert_w_f16(st + C::XP, cv, ctid);
           convert_lm8_f16(st, cv + C::WT, ctid, s_lut8, rows);
@@ -894,14 +978,17 @@ oq_status launch_gemm(const GemmArgs& g, cudaStream_t s) {
   p.N = (int)g.N;
   p.out_acc = g.out_acc;
   p.out = g.out;
+  p.w_sz = g.w_sz;
   if (g.kind == kGemmLloydMax8)
     for (int i = 0; i < 128; ++i)
       p.lut8[i] = (uint32_t)f16_bits(g.centroids8[2 * i]) |
                   ((uint32_t)f16_bits(g.centroids8[2 * i + 1]) << 16);
-  if (g.kind == kGemmLloydMax) {
+  if (g.kind == kGemmLloydMax || g.kind == kGemmG64) {
     uint8_t lo[16], hi[16];
     for (int i = 0; i < 16; ++i) {
-      const uint16_t b = f16_bits(g.centroids[i]);
+      // grouped weights take INT4 codes: the two's-complement nibble i decodes to i or i - 16
+      const float c = g.kind == kGemmG64 ? (float)(i < 8 ? i : i - 16) : g.centroids[i];
+      const uint16_t b = f16_bits(c);
       lo[i] = (uint8_t)(b & 0xFF);
       hi[i] = (uint8_t)(b >> 8);
     }
@@ -920,6 +1007,9 @@ oq_status launch_gemm(const GemmArgs& g, cudaStream_t s) {
       return small ? run<kGemmLloydMax, 1>(g, p, s) : run<kGemmLloydMax, 2>(g, p, s);
     case kGemmLloydMax8:
       return small ? run<kGemmLloydMax8, 1>(g, p, s) : run<kGemmLloydMax8, 2>(g, p, s);
+    case kGemmG64:
+      if (g.K % 64 || !g.w_sz) return fail(OQ_ERR_INVALID_ARG, "grouped weights need K % 64 == 0");
+      return small ? run<kGemmG64, 1>(g, p, s) : run<kGemmG64, 2>(g, p, s);
     default: return fail(OQ_ERR_INVALID_ARG, "unknown GEMM kind");
   }
 }

@@ -369,6 +369,16 @@ oq_status oq_rotate_quantize(const oq_plan* plan, const void* x_bf16, int64_t T,
 
 oq_status oq_prepare_weights(const oq_plan* plan, const void* w_bf16, int64_t n_out, int64_t ldw,
                              uint8_t* w_packed, float* w_scale, float* w_rowsum, void* stream) {
+  return oq_prepare_weights_rotated(plan, w_bf16, n_out, ldw, w_packed, w_scale, w_rowsum,
+                                    nullptr, static_cast<cudaStream_t>(stream));
+}
+}  // extern "C"
+
+namespace oq {
+// oq_prepare_weights, optionally keeping the rotated rows (float [n_out, d]) in `rot`
+oq_status oq_prepare_weights_rotated(const oq_plan* plan, const void* w_bf16, int64_t n_out,
+                                     int64_t ldw, uint8_t* w_packed, float* w_scale,
+                                     float* w_rowsum, float* rot, cudaStream_t stream) {
   if (!plan) return fail(OQ_ERR_INVALID_ARG, "NULL plan");
   if (n_out < 0 || n_out > 0x7FFFFFFF) return fail(OQ_ERR_INVALID_ARG, "n_out out of range");
   if (ldw < plan->d || (ldw * 2) % 16) return fail(OQ_ERR_MISALIGNED, "ldw must be >= d and a multiple of 8");
@@ -378,8 +388,54 @@ oq_status oq_prepare_weights(const oq_plan* plan, const void* w_bf16, int64_t n_
     return fail(OQ_ERR_MISALIGNED, "w and w_packed must be 16-byte aligned");
   oq_status st = check_plan_device(plan);
   if (st != OQ_OK) return st;
-  return rotate_quantize_impl(plan, w_bf16, n_out, ldw, w_packed, w_scale, nullptr, nullptr,
-                              w_rowsum, kRqInt4, 0, 1, static_cast<cudaStream_t>(stream));
+  return rotate_quantize_impl(plan, w_bf16, n_out, ldw, w_packed, w_scale, nullptr, rot,
+                              w_rowsum, kRqInt4, 0, 1, stream);
+}
+}  // namespace oq
+
+extern "C" {
+
+
+oq_status oq_prepare_weights_g64(const oq_plan* plan, const void* w_bf16, int64_t n_out,
+                                 int64_t ldw, uint8_t* w_packed, uint32_t* w_sz, float* w_scale,
+                                 float* w_rowsum, void* stream) {
+  if (!plan) return fail(OQ_ERR_INVALID_ARG, "NULL plan");
+  if (plan->d % 64) return fail(OQ_ERR_INVALID_ARG, "grouped weights need d %% 64 == 0");
+  if (n_out < 0 || n_out > 0x7FFFFFFF) return fail(OQ_ERR_INVALID_ARG, "n_out out of range");
+  if (n_out > 0 && !w_sz) return fail(OQ_ERR_INVALID_ARG, "NULL w_sz");
+  if (n_out == 0) return OQ_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  float* rot = nullptr;
+  cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&rot),
+                                  (size_t)n_out * (size_t)plan->d * sizeof(float), s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMallocAsync(rotated weights)");
+  // the rotation (and w_1) of oq_prepare_weights; its per-channel codes and scales are
+  // overwritten by the grouped quantizer below
+  oq_status st = oq_prepare_weights_rotated(plan, w_bf16, n_out, ldw, w_packed, w_scale,
+                                            w_rowsum, rot, s);
+  if (st == OQ_OK) st = launch_quant_g64(rot, n_out, plan->d, w_packed, w_sz, w_scale, s);
+  e = cudaFreeAsync(rot, s);
+  if (st == OQ_OK && e != cudaSuccess) return cuda_fail(e, "cudaFreeAsync(rotated weights)");
+  return st;
+}
+
+oq_status oq_gemm_w4a4_g64(oq_act_kind kind, const uint8_t* a_packed, const float* a_scale,
+                           const float* mean, const uint8_t* w_packed, const uint32_t* w_sz,
+                           const float* w_scale, const float* w_rowsum, const void* bias_bf16,
+                           int64_t T, int64_t d_in, int64_t d_out, oq_out_kind out_kind,
+                           void* out, void* stream) {
+  if (kind != OQ_ACT_INT4_ABSMAX && kind != OQ_ACT_INT4_PERCENTILE)
+    return fail(OQ_ERR_INVALID_ARG, "grouped weights take INT4_ABSMAX or INT4_PERCENTILE codes");
+  if (d_in % 64) return fail(OQ_ERR_INVALID_ARG, "grouped weights need d_in %% 64 == 0");
+  if (!w_sz) return fail(OQ_ERR_INVALID_ARG, "NULL w_sz");
+  oq_status st = check_gemm_args(a_packed, a_scale, mean, w_packed, w_scale, w_rowsum, bias_bf16,
+                                 T, d_in, d_out, (int)out_kind, out);
+  if (st != OQ_OK) return st;
+  GemmArgs g;
+  g.kind = kGemmG64; g.a = a_packed; g.a_scale = a_scale; g.mean = mean; g.w = w_packed;
+  g.w_sz = w_sz; g.w_scale = w_scale; g.w_rowsum = w_rowsum; g.bias = bias_bf16; g.T = T;
+  g.K = d_in; g.N = d_out; g.out_acc = out_kind == OQ_OUT_ACC; g.out = out;
+  return launch_gemm(g, static_cast<cudaStream_t>(stream));
 }
 
 oq_status oq_gemm_w4a8(const int8_t* a, const float* a_scale, const float* mean,
@@ -484,6 +540,31 @@ oq_status oq_linear(const oq_plan* plan, const void* x_bf16, int64_t T, int64_t 
   return oq_gemm_w4a4(plan, plan->act, static_cast<const uint8_t*>(codes), scale, m, w_packed,
                       w_scale, w_rowsum, bias_bf16, T, plan->d, d_out, OQ_OUT_BF16, y_bf16,
                       stream);
+}
+
+oq_status oq_linear_g64(const oq_plan* plan, const void* x_bf16, int64_t T, int64_t ldx,
+                        const uint8_t* w_packed, const uint32_t* w_sz, const float* w_scale,
+                        const float* w_rowsum, const void* bias_bf16, int64_t d_out,
+                        void* y_bf16, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!plan) return fail(OQ_ERR_INVALID_ARG, "NULL plan");
+  if (plan->act != OQ_ACT_INT4_ABSMAX && plan->act != OQ_ACT_INT4_PERCENTILE)
+    return fail(OQ_ERR_INVALID_ARG, "grouped weights need an INT4_ABSMAX or INT4_PERCENTILE plan");
+  if (T < 0) return fail(OQ_ERR_INVALID_ARG, "T out of range");
+  const size_t need = oq_linear_workspace_bytes(plan, T);
+  if (T > 0 && (!workspace || workspace_bytes < need))
+    return fail(OQ_ERR_INVALID_ARG, "workspace too small: need %zu bytes", need);
+  if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return fail(OQ_ERR_MISALIGNED, "workspace must be 256-byte aligned");
+  if (plan->center && !w_rowsum) return fail(OQ_ERR_INVALID_ARG, "centering needs w_rowsum");
+  const size_t code_bytes = (size_t)T * (plan->d / 2);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* scale = reinterpret_cast<float*>(ws + round256(code_bytes));
+  float* mean = reinterpret_cast<float*>(ws + round256(code_bytes) + round256((size_t)T * 4));
+  oq_status st = oq_rotate_quantize(plan, x_bf16, T, ldx, ws, scale, mean, nullptr, stream);
+  if (st != OQ_OK) return st;
+  return oq_gemm_w4a4_g64(plan->act, ws, scale, plan->center ? mean : nullptr, w_packed, w_sz,
+                          w_scale, w_rowsum, bias_bf16, T, plan->d, d_out, OQ_OUT_BF16, y_bf16,
+                          stream);
 }
 
 oq_status oq_debug_wait_timeout(uint64_t timeout_ns, void* stream) {

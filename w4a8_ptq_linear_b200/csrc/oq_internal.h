@@ -93,7 +93,9 @@ int rq_round1_index(int d, int j);
 int rq_round_buffer_index(int d, int p);
 
 // ---- GEMM ----------------------------------------------------------------------------------
-enum GemmKind : int { kGemmA8 = 0, kGemmA4 = 1, kGemmLloydMax = 2, kGemmLloydMax8 = 3 };
+// kGemmG64: INT4 codes (decoded to fp16 integers) against asymmetric g = 64 weights
+// dequantized to fp16 per (row, group) in the converters
+enum GemmKind : int { kGemmA8 = 0, kGemmA4 = 1, kGemmLloydMax = 2, kGemmLloydMax8 = 3, kGemmG64 = 4 };
 
 struct GemmArgs {
   int kind = kGemmA8;
@@ -109,8 +111,19 @@ struct GemmArgs {
   void* out = nullptr;
   float centroids[16] = {};
   float centroids8[256] = {};   // kGemmLloydMax8
+  const uint32_t* w_sz = nullptr;  // kGemmG64: [K/64][N] words, fp16 sigma (low), z (high)
 };
 oq_status launch_gemm(const GemmArgs& g, cudaStream_t s);
+
+// oq_prepare_weights that also writes the rotated rows (float [n_out, d]) to `rot` (if not null)
+oq_status oq_prepare_weights_rotated(const oq_plan* plan, const void* w_bf16, int64_t n_out,
+                                     int64_t ldw, uint8_t* w_packed, float* w_scale,
+                                     float* w_rowsum, float* rot, cudaStream_t stream);
+
+// Grouped asymmetric INT4 weights from rotated fp32 rows [n, d] (d % 64 == 0): codes Q - 8 in
+// the GEMM layout, (sigma, z) fp16 words [d/64][n], per-row scale 1.
+oq_status launch_quant_g64(const float* rot, int64_t n, int d, uint8_t* w_packed, uint32_t* w_sz,
+                           float* w_scale, cudaStream_t s);
 
 oq_status launch_debug_wait(unsigned long long timeout_ns, cudaStream_t s);
 
