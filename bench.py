@@ -45,10 +45,12 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic per launch from an ncu capture, valid only for the kernel source it was taken
 # on (sha256 of the .cu file at capture time); null once the kernel has changed.
 NCU_TRAFFIC = {
-    # ncu --set full of the CTA-pair kernel (TMA-store epilogue): dram read 17.373 MB + write 0.054 MB
-    ("dit_w4a8", "k_gemm"): {"sha": "46b41ab8fd129e4f0fffd487415f4d4283bb4672db876a2bdf3f7277377eb82b", "bytes": 17427456},
-    # ncu --set full of the two-token kernel: dram read 25.258 MB + write 0
-    ("dit_w4a8", "k_rotate_quant"): {"sha": "93e26d57a081f54e998e6a60544702af974645ab4a8686ba7cf31504ab486b2c", "bytes": 25258496},
+    # ncu --set full of the CTA-pair kernel (TMA-store epilogue): dram read 17.368 MB + write 0.113 MB
+    ("dit_w4a8", "k_gemm"): {"sha": "2245a3d68efb6a51fa03db639106dcbab4caca6e425a58ce9ae0eba8852b676a", "bytes": 17481728},
+    # ncu --set full of the two-token kernel: dram read 25.259 MB + write 0
+    ("dit_w4a8", "k_rotate_quant"): {"sha": "4939e9564cf117b03610c6f8cad5b10b8a15796cf0b4e685133a246067da9012", "bytes": 25258752},
+    # ncu --set full of the grouped-weight kind (first launch): dram read 27.974 MB + write 55.125 MB
+    ("mlp_up_g64", "k_gemm"): {"sha": "2245a3d68efb6a51fa03db639106dcbab4caca6e425a58ce9ae0eba8852b676a", "bytes": 83098880},
 }
 
 
