@@ -1163,13 +1163,14 @@ oq_status launch_rotate_quant(const RqArgs& a, cudaStream_t s) {
   cudaError_t ce = cudaGetDevice(&dev_id);
   if (ce != cudaSuccess) return cuda_fail(ce, "cudaGetDevice");
 
-  // launch shape per (device, d, h mode, rounds), computed once
+  // launch shape per (device, d, h mode, rounds, 8-bit Lloyd-Max), computed once
   static std::mutex mu;
-  static std::map<std::tuple<int, int, int, int>, LaunchCfg> cache;
+  static std::map<std::tuple<int, int, int, int, int>, LaunchCfg> cache;
+  const int lm8 = a.mode == kRqLloydMax8 ? 1 : 0;
   LaunchCfg cfg;
   {
     std::lock_guard<std::mutex> lock(mu);
-    auto key = std::make_tuple(dev_id, a.d, hlog2, a.rounds);
+    auto key = std::make_tuple(dev_id, a.d, hlog2, a.rounds, lm8);
     auto itc = cache.find(key);
     if (itc != cache.end()) {
       cfg = itc->second;
@@ -1180,7 +1181,8 @@ oq_status launch_rotate_quant(const RqArgs& a, cudaStream_t s) {
       const size_t row_stride = ((size_t)a.d * 2 + 127) & ~(size_t)127;
       if (a.d <= kPairMaxD) {
         // nbuf landing pairs, the interleaved words / transpose tiles, the round buffer,
-        // reductions + thresholds + barriers
+        // reductions + thresholds + barriers, the source-sign masks and, for 8-bit Lloyd-Max
+        // codes only, the 256 thresholds (1 KB less keeps 5 CTAs per SM at some widths)
         cfg.pair = 1;
         cfg.fn = a.rounds == 1 ? kern_pair_h<1>(hlog2) : kern_pair_h<2>(hlog2);
         cfg.nthr = nthr;
@@ -1189,7 +1191,8 @@ oq_status launch_rotate_quant(const RqArgs& a, cudaStream_t s) {
         cfg.nbuf = 1;
         cfg.smem = (size_t)cfg.nbuf * 2 * row_stride + (size_t)(nthr / 32) * 4096 +
                    (a.rounds == 2 ? (size_t)(nthr / 32) * 8192 : 0) + 224 * 4 +
-                   (hmode == 2 ? (size_t)(nthr / 32) * 4096 : 0) + (size_t)a.d * 2 + 1024;
+                   (hmode == 2 ? (size_t)(nthr / 32) * 4096 : 0) + (size_t)a.d * 2 +
+                   (lm8 ? 1024 : 0);
         int best_occ = 0;
         ce = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&best_occ, cfg.fn, nthr, cfg.smem);
         if (ce != cudaSuccess) return cuda_fail(ce, "occupancy(rotate_quant)");
