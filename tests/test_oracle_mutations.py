@@ -171,3 +171,58 @@ def test_weight_rotation_transposed_is_caught(monkeypatch):
         return y + (0 if bias is None else np.asarray(bias)[None, :])
     monkeypatch.setattr(Lm, "linear_unquantized", bad)
     assert _fails(TL.check_identity_quantizer, False, 1, False)
+
+
+# ---- grouped g = 64 weights ----------------------------------------------------------------
+
+import test_oracle_weights_g64 as TG  # noqa: E402
+from oracle import weights_g64 as Gm  # noqa: E402
+
+_asym_ok = Gm.asym_group_quantize
+_dequant_ok = Gm.dequantize
+_corr_ok = Gm.corrected_product
+
+
+def _asym_mutant(kind):
+    def asym_group_quantize(w, g=Gm.GROUP, bits=4, store=None, eps=Gm.EPS):
+        w = np.asarray(w, dtype=np.float64)
+        n, d = w.shape
+        top = 2 ** bits - 1
+        wg = w.reshape(n, d // g, g)
+        lo, hi = wg.min(axis=2), wg.max(axis=2)
+        sigma = np.maximum(hi - lo, eps) / (top + 1 if kind == "step_over_16" else top)
+        if store is not None:
+            sigma = np.maximum(sigma, Gm.SIGMA_MIN_F16).astype(store).astype(np.float64)
+        z = (lo if kind == "shift_sign" else -lo) / sigma
+        if store is not None:
+            z = z.astype(store).astype(np.float64)
+        rnd = np.floor if kind == "floor" else np.rint
+        q = np.clip(rnd(wg / sigma[..., None] + z[..., None]), 0, top).astype(np.int64)
+        return q.reshape(n, d), sigma, z
+    return asym_group_quantize
+
+
+def _pins_fail():
+    for t in (TG.test_reconstruction_error_and_extremes, TG.test_codes_are_the_nearest_grid_point,
+              TG.test_fp16_storage_codes_nearest_on_stored_grid,
+              TG.test_layer_reduces_to_unquantized_for_fine_weights):
+        if _fails(lambda: (t(), True)[1]):
+            return True
+    return False
+
+
+@pytest.mark.parametrize("kind", ["shift_sign", "floor", "step_over_16"])
+def test_grouped_quantizer_mistakes_are_caught(monkeypatch, kind):
+    monkeypatch.setattr(Gm, "asym_group_quantize", _asym_mutant(kind))
+    assert _pins_fail()
+
+
+def test_grouped_dequantize_and_correction_mistakes_are_caught(monkeypatch):
+    # sigma (Q + z) for sigma (Q - z)
+    monkeypatch.setattr(Gm, "dequantize", lambda q, s, z, g=Gm.GROUP: _dequant_ok(q, s, -z, g))
+    assert _pins_fail() or _fails(lambda: (TG.test_zero_point_correction_identity(), True)[1])
+    monkeypatch.setattr(Gm, "dequantize", _dequant_ok)
+    # z' = z instead of z - 8 in the App. B.2 correction
+    monkeypatch.setattr(Gm, "corrected_product",
+                        lambda a, q, s, z, g=Gm.GROUP: _corr_ok(a, q, s, z + 8.0, g))
+    assert _fails(lambda: (TG.test_zero_point_correction_identity(), True)[1])
