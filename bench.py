@@ -48,7 +48,7 @@ NCU_TRAFFIC = {
     # ncu --set full of the CTA-pair kernel (TMA-store epilogue): dram read 17.368 MB + write 0.113 MB
     ("dit_w4a8", "k_gemm"): {"sha": "2245a3d68efb6a51fa03db639106dcbab4caca6e425a58ce9ae0eba8852b676a", "bytes": 17481728},
     # ncu --set full of the two-token kernel: dram read 25.259 MB + write 0
-    ("dit_w4a8", "k_rotate_quant"): {"sha": "4939e9564cf117b03610c6f8cad5b10b8a15796cf0b4e685133a246067da9012", "bytes": 25258752},
+    ("dit_w4a8", "k_rotate_quant"): {"sha": "d0b7698240c307304d5df42966d972bbdef49d000e9013581a9acbac570631f6", "bytes": 25258752},
     # ncu --set full of the grouped-weight kind (first launch): dram read 27.974 MB + write 55.125 MB
     ("mlp_up_g64", "k_gemm"): {"sha": "2245a3d68efb6a51fa03db639106dcbab4caca6e425a58ce9ae0eba8852b676a", "bytes": 83098880},
 }
