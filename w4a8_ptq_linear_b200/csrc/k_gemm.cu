@@ -301,15 +301,20 @@ __device__ __forceinline__ void convert_w_f16(const uint8_t* src, uint8_t* dst, 
 // m = -sigma (z - 8), the zero-point correction sigma z' taken into the operand. Both nibbles
 // are first decoded exactly to n (1024 + (n + 8) - 1032; (1024 + 16 (n + 8)) / 16 - 72), then
 // one fused multiply-add per lane pair rounds sigma n + m to fp16 once.
-__device__ __forceinline__ void wg_pair_f16(uint32_t x, __half2 sg, __half2 mg, uint32_t& lo16,
-                                            uint32_t& hi16) {
+__device__ __forceinline__ void nib_pair_f16(uint32_t x, __half2& nl, __half2& nh) {
   const uint32_t l = (x & 0x000F000Fu) ^ 0x64086408u;
   const uint32_t h = (x & 0x00F000F0u) ^ 0x64806480u;
   const __half2 off_l = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));
   const __half2 sixteenth = __halves2half2(__ushort_as_half(0x2C00), __ushort_as_half(0x2C00));
   const __half2 off_h = __halves2half2(__ushort_as_half(0xD480), __ushort_as_half(0xD480));
-  const __half2 nl = __hsub2(*reinterpret_cast<const __half2*>(&l), off_l);           // n
-  const __half2 nh = __hfma2(*reinterpret_cast<const __half2*>(&h), sixteenth, off_h);  // n
+  nl = __hsub2(*reinterpret_cast<const __half2*>(&l), off_l);             // low nibbles
+  nh = __hfma2(*reinterpret_cast<const __half2*>(&h), sixteenth, off_h);  // high nibbles
+}
+
+__device__ __forceinline__ void wg_pair_f16(uint32_t x, __half2 sg, __half2 mg, uint32_t& lo16,
+                                            uint32_t& hi16) {
+  __half2 nl, nh;
+  nib_pair_f16(x, nl, nh);
   __half2 vl = __hfma2(nl, sg, mg);
   __half2 vh = __hfma2(nh, sg, mg);
   lo16 = *reinterpret_cast<uint32_t*>(&vl);
@@ -360,6 +365,39 @@ __device__ __forceinline__ void convert_wg_f16(const uint8_t* src, uint8_t* dst,
         make_uint4(Q[0][0], Q[0][1], Q[1][0], Q[1][1]);
     *reinterpret_cast<uint4*>(row + (((4 * q + 3) ^ ph) << 4)) =
         make_uint4(Q[2][0], Q[2][1], Q[3][0], Q[3][1]);
+  }
+}
+
+// INT4 activation code rows (natural nibble order, 32 bytes = 64 codes per stage) -> fp16
+// integer rows of 128 bytes, swizzled as in convert_lm_f16; the first `rows` rows (rounded up to
+// a pass of the group). Bytes j, j + 1 of a word decode exactly as in nib_pair_f16 to the lane
+// pairs (e_2j, e_2j+2) and (e_2j+1, e_2j+3), which two byte permutes interleave.
+__device__ __forceinline__ void convert_x4_f16(const uint8_t* src, uint8_t* dst, int ctid,
+                                               int rows) {
+  constexpr int RSTEP = NCG / 2;
+  const int r0 = ctid >> 1, q = ctid & 1;
+  const uint8_t* s = src + r0 * 32 + q * 16;
+  uint8_t* d = dst + r0 * 128;
+  const int ph = r0 & 7;
+#pragma unroll 1
+  for (int j = 0; j * RSTEP < rows; ++j) {
+    const uint4 in = *reinterpret_cast<const uint4*>(s + j * RSTEP * 32);
+    const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      uint32_t o[4];
+#pragma unroll
+      for (int hb = 0; hb < 2; ++hb) {
+        __half2 nl, nh;
+        nib_pair_f16(__byte_perm(w[k], 0u, hb ? 0x4342 : 0x4140), nl, nh);
+        const uint32_t a = *reinterpret_cast<uint32_t*>(&nl);
+        const uint32_t b = *reinterpret_cast<uint32_t*>(&nh);
+        o[2 * hb] = __byte_perm(a, b, 0x5410);
+        o[2 * hb + 1] = __byte_perm(a, b, 0x7632);
+      }
+      *reinterpret_cast<uint4*>(d + j * RSTEP * 128 + (((4 * q + k) ^ ph) << 4)) =
+          make_uint4(o[0], o[1], o[2], o[3]);
+    }
   }
 }
 
@@ -691,7 +729,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           convert_lm_f16(st, cv + C::WT, ctid, lut, rows);
         } else if constexpr (KIND == kGemmG64) {
           convert_wg_f16(st + C::XP, cv, ctid, sz0, sz1);
-          convert_lm_f16(st, cv + C::WT, ctid, lut, rows);   // integer table: code -> n
+          convert_x4_f16(st, cv + C::WT, ctid, rows);
         } else if constexpr (KIND == kGemmLloydMax8) {
           convert_w_f16(st + C::XP, cv, ctid);
           convert_lm8_f16(st, cv + C::WT, ctid, s_lut8, rows);
@@ -983,12 +1021,10 @@ oq_status launch_gemm(const GemmArgs& g, cudaStream_t s) {
     for (int i = 0; i < 128; ++i)
       p.lut8[i] = (uint32_t)f16_bits(g.centroids8[2 * i]) |
                   ((uint32_t)f16_bits(g.centroids8[2 * i + 1]) << 16);
-  if (g.kind == kGemmLloydMax || g.kind == kGemmG64) {
+  if (g.kind == kGemmLloydMax) {
     uint8_t lo[16], hi[16];
     for (int i = 0; i < 16; ++i) {
-      // grouped weights take INT4 codes: the two's-complement nibble i decodes to i or i - 16
-      const float c = g.kind == kGemmG64 ? (float)(i < 8 ? i : i - 16) : g.centroids[i];
-      const uint16_t b = f16_bits(c);
+      const uint16_t b = f16_bits(g.centroids[i]);
       lo[i] = (uint8_t)(b & 0xFF);
       hi[i] = (uint8_t)(b >> 8);
     }
