@@ -45,12 +45,12 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic per launch from an ncu capture, valid only for the kernel source it was taken
 # on (sha256 of the .cu file at capture time); null once the kernel has changed.
 NCU_TRAFFIC = {
-    # ncu --set full of the CTA-pair kernel (TMA-store epilogue): dram read 17.368 MB + write 0.050 MB
-    ("dit_w4a8", "k_gemm"): {"sha": "f4a043d531cf7140b917f1647fdb90a4be53cfe53e196aa3fb443cf4a78b657d", "bytes": 17417728},
+    # ncu --set full of the CTA-pair kernel (TMA-store epilogue): dram read 17.368 MB + write 0.037 MB
+    ("dit_w4a8", "k_gemm"): {"sha": "7150944b8b4e5abce3e1c8b823aae3a35488a0a0607921af58f132f85ef8694a", "bytes": 17405440},
     # ncu --set full of the two-token kernel: dram read 25.259 MB + write 0
     ("dit_w4a8", "k_rotate_quant"): {"sha": "d0b7698240c307304d5df42966d972bbdef49d000e9013581a9acbac570631f6", "bytes": 25258752},
-    # ncu --set full of the grouped-weight kind (first launch): dram read 27.993 MB + write 54.903 MB
-    ("mlp_up_g64", "k_gemm"): {"sha": "f4a043d531cf7140b917f1647fdb90a4be53cfe53e196aa3fb443cf4a78b657d", "bytes": 82895360},
+    # ncu --set full of the grouped-weight kind (first launch): dram read 28.036 MB + write 55.219 MB
+    ("mlp_up_g64", "k_gemm"): {"sha": "7150944b8b4e5abce3e1c8b823aae3a35488a0a0607921af58f132f85ef8694a", "bytes": 83255808},
 }
 
 

@@ -203,7 +203,10 @@ oq_status oq_prepare_weights(const oq_plan* plan, const void* w_bf16, int64_t n_
  * and w_1[o] = sum_k W[o,k] (fp32, before rotation).
  *   plan      d % 64 == 0; its activation kind is not used here
  *   w_bf16    [n_out, ldw] bf16, 16-byte aligned, ldw >= d, (ldw * 2) % 16 == 0
- *   w_packed  uint8 [n_out, d/2] in the GEMM layout, nibble = (Q - 8) two's complement
+ *   w_packed  uint8 [n_out, d/2] in the GEMM layout, nibble = (Q - 8) two's complement, with
+ *             the K order swapped inside every four columns: stored position p holds column
+ *             (p & ~3) | ((p & 1) << 1) | ((p >> 1) & 1), i.e. 0, 2, 1, 3 (the order in which
+ *             oq_gemm_w4a4_g64 decodes the activation codes)
  *   w_sz      uint32 [d/64][n_out] (group-major): bits 0-15 fp16 sigma, bits 16-31 fp16 z
  *   w_scale   float [n_out]: the per-row scale s_o of §4.3, 1 under round to nearest
  *   w_rowsum  float [n_out]

@@ -25,6 +25,13 @@ pytestmark = pytest.mark.gpu
 U16 = 2.0 ** -11
 
 
+def _k_order(d):
+    """Stored K order of the grouped weights: position p holds column pi(p), pi swapping bits 0
+    and 1 of the index (an involution), so natural = stored[:, pi] and stored = natural[:, pi]."""
+    k = np.arange(d)
+    return (k & ~3) | ((k & 1) << 1) | ((k >> 1) & 1)
+
+
 def _split_sz(wsz):
     """int32 [G, N] words -> (sigma, z) float64 [N, G]."""
     w = np.ascontiguousarray(wsz).view(np.uint32)
@@ -62,7 +69,7 @@ def test_prepare_weights_g64_bit_exact(n_out, d, h, rounds):
     q, s, z = G.asym_group_quantize_f32(rot)
     gs, gz = _split_sz(wsz.cpu().numpy())
     assert np.array_equal(gs, s) and np.array_equal(gz, z)
-    assert np.array_equal(unpack_w4_gemm(wp.cpu().numpy()), q - 8)
+    assert np.array_equal(unpack_w4_gemm(wp.cpu().numpy())[:, _k_order(d)], q - 8)
     assert np.all(ws.cpu().numpy() == 1.0)
     assert np.all(np.abs(w1.cpu().numpy() - w.sum(axis=1)) <= 1e-5 * np.abs(w).sum(axis=1))
     # every rotated weight is within half a grid step of its reconstruction (the fp16 shift
@@ -100,7 +107,8 @@ def test_g64_accumulators_and_epilogue(T, K, N):
     rng = np.random.default_rng(3 * T + K + N)
     a, q, s, z = _operands(rng, T, K, N)
     cu = lambda v: torch.from_numpy(np.ascontiguousarray(v)).cuda()
-    ap, wp, wsz = cu(oracle.pack_nibbles(a)), cu(pack_w4_gemm(q - 8)), cu(_pack_sz(s, z))
+    ap, wsz = cu(oracle.pack_nibbles(a)), cu(_pack_sz(s, z))
+    wp = cu(pack_w4_gemm((q - 8)[:, _k_order(K)]))
     ones = torch.ones(max(T, N), dtype=torch.float32, device="cuda")
     acc = oq.gemm_w4a4_g64("int4_absmax", ap, ones[:T], wp, wsz, ones[:N], out_kind=oq.OUT_ACC)
     alpha = rng.uniform(0.5, 2.0, T)

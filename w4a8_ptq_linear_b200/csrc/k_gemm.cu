@@ -371,7 +371,9 @@ __device__ __forceinline__ void convert_wg_f16(const uint8_t* src, uint8_t* dst,
 // INT4 activation code rows (natural nibble order, 32 bytes = 64 codes per stage) -> fp16
 // integer rows of 128 bytes, swizzled as in convert_lm_f16; the first `rows` rows (rounded up to
 // a pass of the group). Bytes j, j + 1 of a word decode exactly as in nib_pair_f16 to the lane
-// pairs (e_2j, e_2j+2) and (e_2j+1, e_2j+3), which two byte permutes interleave.
+// pairs (e_2j, e_2j+2) and (e_2j+1, e_2j+3), which are stored as they come: within every four
+// consecutive K positions the operand holds elements 0, 2, 1, 3. The grouped weights are stored
+// offline in the same K order, so the products pair up and the sum is unchanged.
 __device__ __forceinline__ void convert_x4_f16(const uint8_t* src, uint8_t* dst, int ctid,
                                                int rows) {
   constexpr int RSTEP = NCG / 2;
@@ -390,10 +392,8 @@ __device__ __forceinline__ void convert_x4_f16(const uint8_t* src, uint8_t* dst,
       for (int hb = 0; hb < 2; ++hb) {
         __half2 nl, nh;
         nib_pair_f16(__byte_perm(w[k], 0u, hb ? 0x4342 : 0x4140), nl, nh);
-        const uint32_t a = *reinterpret_cast<uint32_t*>(&nl);
-        const uint32_t b = *reinterpret_cast<uint32_t*>(&nh);
-        o[2 * hb] = __byte_perm(a, b, 0x5410);
-        o[2 * hb + 1] = __byte_perm(a, b, 0x7632);
+        o[2 * hb] = *reinterpret_cast<uint32_t*>(&nl);
+        o[2 * hb + 1] = *reinterpret_cast<uint32_t*>(&nh);
       }
       *reinterpret_cast<uint4*>(d + j * RSTEP * 128 + (((4 * q + k) ^ ph) << 4)) =
           make_uint4(o[0], o[1], o[2], o[3]);

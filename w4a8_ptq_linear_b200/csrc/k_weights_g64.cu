@@ -8,6 +8,11 @@
 //   Q = clamp(rint(w / sigma + z), 0, 15),  stored nibble Q - 8 (= Q xor 8).
 // Every step is one IEEE operation rounded to nearest (division, addition, conversion), so a
 // float32 restatement of the same steps reproduces the codes bit for bit.
+//
+// K order: the GEMM decodes INT4 activation codes into an operand that holds, within every four
+// consecutive K positions, elements 0, 2, 1, 3 (it skips an interleave). The grouped weights are
+// stored in that order too: stored position p holds column pi(p), pi swapping bits 0 and 1 of
+// the position (an involution that stays inside each group of 64).
 #include <cuda_fp16.h>
 
 #include <algorithm>
@@ -19,9 +24,9 @@ namespace {
 
 constexpr int kGroup = 64;
 
-// One warp per (row, group): lane l holds columns l and 32 + l of the group, i.e. position l of
-// the group's two 32-column blocks of the GEMM layout (byte j of a block: column j low nibble,
-// column 16 + j high nibble).
+// One warp per (row, group): lane l holds columns l and 32 + l of the group. Byte j of block b of
+// the GEMM layout holds stored positions 32b + j (low nibble) and 32b + 16 + j (high nibble),
+// i.e. columns 32b + pi(j) and 32b + 16 + pi(j).
 __global__ void __launch_bounds__(256) k_quant_g64(const float* __restrict__ rot, int64_t n,
                                                    int d, uint8_t* __restrict__ w_packed,
                                                    uint32_t* __restrict__ w_sz,
@@ -52,9 +57,13 @@ __global__ void __launch_bounds__(256) k_quant_g64(const float* __restrict__ rot
       return (uint32_t)fminf(fmaxf(v, 0.f), 15.f) ^ 8u;   // nibble of Q - 8
     };
     const uint32_t c0 = code(w0), c1 = code(w1);
-    const uint32_t a = __shfl_sync(0xffffffffu, c0, (lane + 16) & 31);   // c0 of lane l + 16
-    const uint32_t b = __shfl_sync(0xffffffffu, c1, (lane + 16) & 31);   // c1 of lane l - 16
-    const uint32_t byte = lane < 16 ? (c0 | (a << 4)) : (b | (c1 << 4));
+    const int j = lane & 15;
+    const int pj = (j & ~3) | ((j & 1) << 1) | ((j >> 1) & 1);   // pi(j)
+    const uint32_t lo0 = __shfl_sync(0xffffffffu, c0, pj);
+    const uint32_t hi0 = __shfl_sync(0xffffffffu, c0, 16 + pj);
+    const uint32_t lo1 = __shfl_sync(0xffffffffu, c1, pj);
+    const uint32_t hi1 = __shfl_sync(0xffffffffu, c1, 16 + pj);
+    const uint32_t byte = lane < 16 ? (lo0 | (hi0 << 4)) : (lo1 | (hi1 << 4));
     w_packed[row * (int64_t)(d / 2) + (int64_t)g * 32 + lane] = (uint8_t)byte;
     if (lane == 0) {
       w_sz[(int64_t)g * n + row] = (uint32_t)__half_as_ushort(s16) |
