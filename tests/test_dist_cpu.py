@@ -80,3 +80,23 @@ def test_reference_arm_runs_on_rank_zero_only():
     import synth
     args = argparse.Namespace(steps=1, warmup=0, gpus=2)
     assert bench.run_reference(args, synth.WORKLOADS["tiny"], rank=1) is None
+
+
+@pytest.mark.parametrize("name", ["mlp_up_g64", "tiny"])
+def test_bench_oracle_leg_is_the_layer_oracle(name):
+    # the CPU leg of bench.py (cpu_baseline and --impl reference) computes the layer oracle
+    import numpy as np
+    import bench
+    import oracle
+    import synth
+    from oracle import weights_g64
+    wl, xb, wb = synth.make_inputs(name, T=3)
+    x = synth.bf16_to_f64(xb)
+    got = bench.oracle_pass(wl, bench.oracle_setup(wl, xb, wb), x)
+    plan = oracle.rpbh_plan(wl.d, wl.h, wl.rounds, wl.seed)
+    if wl.weights == "int4_g64":
+        ref, _, _ = weights_g64.linear_forward_g64(x, synth.bf16_to_f64(wb), plan, wl.h, wl.act,
+                                                   wl.center)
+    else:
+        ref, _, _ = oracle.linear_forward(x, synth.bf16_to_f64(wb), plan, wl.h, wl.act, wl.center)
+    assert np.allclose(got, ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
