@@ -307,8 +307,9 @@ def linear(plan: Plan, x, w_packed, w_scale, w_rowsum=None, bias=None, *, worksp
 def prepare_weights_g64(plan: Plan, w, *, stream=None):
     """oq_prepare_weights_g64 on a bf16 [n_out, d] CUDA tensor: asymmetric INT4 groups of 64.
 
-    Returns (w_packed uint8 [n, d/2], w_sz int32 [d/64, n] of fp16 (sigma, z) pairs,
-    w_scale float32 [n] (ones), w_rowsum float32 [n])."""
+    Returns (w_packed uint8 [n, d/2]: Q - 8 nibbles in the GEMM layout, K order 0, 2, 1, 3
+    inside every four columns; w_sz int32 [d/64, n] of fp16 (sigma, z) pairs; w_scale float32
+    [n] (ones); w_rowsum float32 [n])."""
     import torch
     n = w.shape[0]
     wp = torch.empty((n, plan.d // 2), dtype=torch.uint8, device=w.device)
