@@ -211,7 +211,9 @@ oq_status oq_prepare_weights(const oq_plan* plan, const void* w_bf16, int64_t n_
  *   w_scale   float [n_out]: the per-row scale s_o of §4.3, 1 under round to nearest
  *   w_rowsum  float [n_out]
  * Allocates n_out * d * 4 bytes of stream-ordered scratch (cudaMallocAsync) for the rotated
- * rows; errors as for oq_prepare_weights, OQ_ERR_INVALID_ARG if d % 64 != 0. */
+ * rows; errors as for oq_prepare_weights, OQ_ERR_INVALID_ARG if d % 64 != 0. The fp16 storage
+ * bounds the format: a group whose range exceeds 15 * 65504 (sigma beyond fp16) is not
+ * representable and is not detected. */
 oq_status oq_prepare_weights_g64(const oq_plan* plan, const void* w_bf16, int64_t n_out,
                                  int64_t ldw, uint8_t* w_packed, uint32_t* w_sz, float* w_scale,
                                  float* w_rowsum, void* stream);
