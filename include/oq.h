@@ -167,6 +167,19 @@ void oq_plan_destroy(oq_plan* plan);
 oq_status oq_plan_get_rpbh(const oq_plan* plan, int round, int8_t* signs_host,
                            int32_t* perm_host);
 
+/* Host copies of the Lloyd-Max codebook a plan quantizes with (OrbitQuant PR #25 "Default
+ * changes": codebook v3, one table per width; FLUX.1-schnell-OrbitQuant-W4A4 model card,
+ * "Artifact Files": the Lloyd-Max codebooks ship with the rotation metadata as part of the
+ * quantized artifact). The table is the one the plan's kernels use: the 16-level N(0,1)
+ * codebook for OQ_ACT_INT4_LLOYDMAX, the 16-level width-d codebook for
+ * OQ_ACT_INT4_LLOYDMAX_WIDTH, the 256-level N(0,1) codebook for OQ_ACT_INT8_LLOYDMAX.
+ *   levels            16 or 256; must be the size of the plan's codebook
+ *   centroids_host    double[levels], ascending; thresholds_host double[levels - 1] midpoints
+ * OQ_ERR_INVALID_ARG for a NULL argument, a plan whose activation kind uses no codebook
+ * (absmax, percentile) or a levels value that is not the plan's. Host only. */
+oq_status oq_plan_get_codebook(const oq_plan* plan, int levels, double* centroids_host,
+                               double* thresholds_host);
+
 /* ---- compute ----------------------------------------------------------------------- */
 
 /* Fused center + RPBH + per-token scale + quantize (CentriQ §4.2, activation path, and
@@ -198,8 +211,10 @@ oq_status oq_prepare_weights(const oq_plan* plan, const void* w_bf16, int64_t n_
  * from the group minimum and maximum; App. B.2: codes stored as Q - 8; App. B.3 Tab. 3:
  * grid {0..15}, 16-bit scale and zero point). Every row of W goes through the plan's rotation
  * without centering; then per row o and group g:
- *   sigma = fp16(max((max - min) / 15, 2^-14)),  z = fp16(-min / sigma),
+ *   sigma = fp16(max((max - min) / 15, 2^-14, |min| / 2^15)),  z = fp16(-min / sigma),
  *   Q = clamp(rint(w / sigma + z), 0, 15)        (float32, each step rounded to nearest)
+ * (the |min| / 2^15 floor keeps |z| < 2^15 (1 + 2^-11), finite in fp16, for nearly constant
+ * groups far from zero)
  * and w_1[o] = sum_k W[o,k] (fp32, before rotation).
  *   plan      d % 64 == 0; its activation kind is not used here
  *   w_bf16    [n_out, ldw] bf16, 16-byte aligned, ldw >= d, (ldw * 2) % 16 == 0
@@ -212,8 +227,8 @@ oq_status oq_prepare_weights(const oq_plan* plan, const void* w_bf16, int64_t n_
  *   w_rowsum  float [n_out]
  * Allocates n_out * d * 4 bytes of stream-ordered scratch (cudaMallocAsync) for the rotated
  * rows; errors as for oq_prepare_weights, OQ_ERR_INVALID_ARG if d % 64 != 0. The fp16 storage
- * bounds the format: a group whose range exceeds 15 * 65504 (sigma beyond fp16) is not
- * representable and is not detected. */
+ * bounds the format: a group whose range exceeds 15 * 65504, or whose minimum exceeds 2^15 *
+ * 65504 in magnitude (sigma beyond fp16), is not representable and is not detected. */
 oq_status oq_prepare_weights_g64(const oq_plan* plan, const void* w_bf16, int64_t n_out,
                                  int64_t ldw, uint8_t* w_packed, uint32_t* w_sz, float* w_scale,
                                  float* w_rowsum, void* stream);
@@ -305,7 +320,10 @@ oq_status oq_linear_g64(const oq_plan* plan, const void* x_bf16, int64_t T, int6
  *     T <= 5447 tokens at d = 3072 with INT8 codes. Larger T returns OQ_ERR_INVALID_ARG
  *     with a message; split the batch or use oq_linear.
  *   - Set-up: the first call on a device looks up the array's device address (with that
- *     device current). Make that first call before any stream capture.
+ *     device current) and keeps it for the life of the process. Make that first call before
+ *     any stream capture. The kept address does not survive cudaDeviceReset (or any other
+ *     teardown of the device's primary context): after one, do not call this entry point
+ *     again in that process; use oq_linear.
  *   - Sharing: all calls on a device use the same array and leave their contents in it.
  *     Calls whose kernels overlap on the GPU (other streams, other host threads) race on it;
  *     the caller must serialise them. Nothing in the array needs to start at zero. */

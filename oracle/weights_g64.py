@@ -16,9 +16,12 @@ Mean Centering):
 Readings: sigma = max(max - min, eps) / (2^b - 1) and z = -min / sigma (HQQ-style min/max
 initialisation with a real shift); with 16-bit storage sigma and z are rounded to fp16 (the
 format of the tensor-core operand) and the codes are taken against the stored grid,
-Q = clip(round(w / sigma16 + z16), 0, 2^b - 1), round half to even; sigma is floored at 2^-14,
-the smallest normal fp16, so that the stored grid never degenerates; the activations that
-multiply these weights are the INT4 absmax (or percentile) codes.
+Q = clip(round(w / sigma16 + z16), 0, 2^b - 1), round half to even. Before rounding, sigma is
+floored at 2^-14 (the smallest normal fp16, so that the stored grid never degenerates) and at
+|min| / 2^15, so that the stored shift |z| = |min| / sigma16 stays below 2^15 (1 + 2^-11) and
+is finite in fp16 even for a nearly constant group far from zero; the grid still covers
+[min, max] because 15 sigma >= max - min. The activations that multiply these weights are the
+INT4 absmax (or percentile) codes.
 
 Parity: pinned (tests/test_oracle_weights_g64.py): the reconstruction error is at most
 sigma / 2 everywhere, group minima and maxima reconstruct exactly (exact storage), the codes
@@ -35,6 +38,7 @@ from .rpbh import rotate
 
 GROUP = 64
 SIGMA_MIN_F16 = 2.0 ** -14
+SHIFT_MAX = 2.0 ** 15      # 16-bit storage: sigma >= |min| / SHIFT_MAX keeps z finite
 
 
 def asym_group_quantize(w: np.ndarray, g: int = GROUP, bits: int = 4, store=None,
@@ -51,31 +55,13 @@ def asym_group_quantize(w: np.ndarray, g: int = GROUP, bits: int = 4, store=None
     lo, hi = wg.min(axis=2), wg.max(axis=2)
     sigma = np.maximum(hi - lo, eps) / top
     if store is not None:
-        sigma = np.maximum(sigma, SIGMA_MIN_F16).astype(store).astype(np.float64)
+        sigma = np.maximum(np.maximum(sigma, SIGMA_MIN_F16), np.abs(lo) / SHIFT_MAX)
+        sigma = sigma.astype(store).astype(np.float64)
     z = -lo / sigma
     if store is not None:
         z = z.astype(store).astype(np.float64)
     q = np.clip(np.rint(wg / sigma[..., None] + z[..., None]), 0, top).astype(np.int64)
     return q.reshape(n, d), sigma, z
-
-
-def asym_group_quantize_f32(w: np.ndarray, g: int = GROUP):
-    """The same codes, sigma and z with every step taken in float32, one IEEE operation at a
-    time (range, division by 15, the fp16 floor and rounding, -min / sigma, w / sigma + z,
-    round half to even): the precision in which the CUDA path takes these integer decisions.
-    Returns (Q int64 [N, d], sigma fp16-valued float64 [N, d/g], z likewise)."""
-    w = np.asarray(w, dtype=np.float32)
-    n, d = w.shape
-    if d % g:
-        raise ValueError("d must be a multiple of the group size")
-    wg = w.reshape(n, d // g, g)
-    lo, hi = wg.min(axis=2), wg.max(axis=2)
-    s = np.maximum((hi - lo) / np.float32(15), np.float32(SIGMA_MIN_F16))
-    sf = s.astype(np.float16).astype(np.float32)
-    zf = (-lo / sf).astype(np.float16).astype(np.float32)
-    v = np.rint(wg / sf[..., None] + zf[..., None])
-    q = np.clip(v, 0, 15).astype(np.int64)
-    return q.reshape(n, d), sf.astype(np.float64), zf.astype(np.float64)
 
 
 def dequantize(q: np.ndarray, sigma: np.ndarray, z: np.ndarray, g: int = GROUP) -> np.ndarray:

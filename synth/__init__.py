@@ -31,8 +31,8 @@ from dataclasses import dataclass, field
 import numpy as np
 
 __all__ = [
-    "Workload", "WORKLOADS", "f64_to_bf16", "bf16_to_f64", "make_x", "make_w", "make_bias",
-    "make_inputs", "sweep_points",
+    "Workload", "WORKLOADS", "f64_to_bf16", "bf16_to_f64", "make_x", "make_x_parallel", "make_w",
+    "make_bias", "make_inputs", "sweep_points",
 ]
 
 
@@ -40,13 +40,16 @@ def f64_to_bf16(a: np.ndarray) -> np.ndarray:
     """Round float64 values to bfloat16 bit patterns (round to nearest, ties to even).
 
     The value is first rounded to float32 by numpy (RNE), then the low 16 bits are rounded
-    away with ties to even. Non-finite values are not produced by the generators.
+    away with ties to even. Non-finite values are not produced by the generators (for finite
+    values the 32-bit sum below cannot wrap).
     """
     f = np.ascontiguousarray(np.asarray(a, dtype=np.float64).astype(np.float32))
-    u = f.view(np.uint32).astype(np.uint64)
-    lsb = (u >> np.uint64(16)) & np.uint64(1)
-    u = (u + np.uint64(0x7FFF) + lsb) >> np.uint64(16)
-    return u.astype(np.uint16)
+    u = f.view(np.uint32)
+    r = (u >> np.uint32(16)) & np.uint32(1)
+    r += np.uint32(0x7FFF)
+    r += u
+    r >>= np.uint32(16)
+    return r.astype(np.uint16)
 
 
 def bf16_to_f64(b: np.ndarray) -> np.ndarray:
@@ -123,8 +126,7 @@ def make_x(T: int, d: int, *, mean_var: float, heavy_frac: float = 0.0, outliers
         base = rng.standard_normal((BLK, d))
         if heavy_frac > 0.0:
             mask = rng.random((BLK, d)) < heavy_frac
-            heavy = rng.standard_t(3.0, size=(BLK, d))
-            base = np.where(mask, heavy, base)
+            base[mask] = rng.standard_t(3.0, size=int(mask.sum()))
         mu = rng.standard_normal((BLK, 1)) * np.sqrt(mean_var)
         x = base + mu
         if outlier_ch is not None:
@@ -132,6 +134,42 @@ def make_x(T: int, d: int, *, mean_var: float, heavy_frac: float = 0.0, outliers
         out[t:t + n] = f64_to_bf16(x[lo:lo + n])
         t += n
     return out
+
+
+def _fill_rows(job):
+    # worker of make_x_parallel: rows [r0, r1) of the shared array
+    from multiprocessing import shared_memory
+    name, T, d, r0, r1, kw = job
+    shm = shared_memory.SharedMemory(name=name)
+    try:
+        arr = np.ndarray((T, d), dtype=np.uint16, buffer=shm.buf)
+        arr[r0:r1] = make_x(r1 - r0, d, row_offset=r0, **kw)
+        del arr
+    finally:
+        shm.close()
+    return r1 - r0
+
+
+def make_x_parallel(T: int, d: int, *, workers: int | None = None, **kw) -> np.ndarray:
+    """``make_x(T, d, **kw)`` drawn by a pool of processes (the same bits: rows come from
+    generators keyed on their row block). The pool uses the spawn start method, which is safe
+    after CUDA has been initialised in the calling process."""
+    import multiprocessing as mp
+    import os
+    from multiprocessing import shared_memory
+    workers = workers or min(32, os.cpu_count() or 1)
+    if workers <= 1 or T * d < (1 << 24):
+        return make_x(T, d, **kw)
+    blk = 256 * max(1, -(-T // (256 * 4 * workers)))     # whole row blocks, ~4 jobs per worker
+    shm = shared_memory.SharedMemory(create=True, size=max(1, T * d * 2))
+    try:
+        jobs = [(shm.name, T, d, r, min(T, r + blk), kw) for r in range(0, T, blk)]
+        with mp.get_context("spawn").Pool(workers) as pool:
+            assert sum(pool.map(_fill_rows, jobs)) == T
+        return np.ndarray((T, d), dtype=np.uint16, buffer=shm.buf).copy()
+    finally:
+        shm.close()
+        shm.unlink()
 
 
 def make_w(n_out: int, d: int, *, seed: int = 0) -> np.ndarray:

@@ -75,3 +75,25 @@ def compare_codes(gpu_codes: np.ndarray, ref_codes: np.ndarray, exempt: np.ndarr
     """(number of differing codes outside the exemption, number of exempted positions)."""
     diff = gpu_codes != ref_codes
     return int(np.sum(diff & ~exempt)), int(np.sum(exempt))
+
+
+def fp16_boundary_mask(x: np.ndarray, floor: float = 0.0) -> np.ndarray:
+    """True where float64 x lies within 1e-5 * max(|x|, floor) of a rounding boundary of
+    fp16 (the midpoint between two neighbouring fp16 values), so that a computation that
+    reaches x with a relative error below 1e-5 may round it to either neighbour."""
+    x = np.asarray(x, dtype=np.float64)
+    f = x.astype(np.float16)
+    up = np.nextafter(f, np.float16(np.inf)).astype(np.float64)
+    dn = np.nextafter(f, np.float16(-np.inf)).astype(np.float64)
+    fd = f.astype(np.float64)
+    gap = np.minimum(np.abs(x - (fd + up) / 2), np.abs(x - (fd + dn) / 2))
+    return gap <= BOUNDARY_REL * np.maximum(np.abs(x), floor)
+
+
+def grid_boundary_mask(v: np.ndarray, lo: int, hi: int) -> np.ndarray:
+    """True where v lies within 1e-5 relative (floor 1/2) of a rounding boundary k + 1/2 with
+    lo <= k < hi, i.e. where round-half-even to the integers in [lo, hi] is decided by noise."""
+    v = np.asarray(v, dtype=np.float64)
+    b = np.floor(v) + 0.5
+    near = np.abs(v - b) <= BOUNDARY_REL * np.maximum(np.abs(b), 0.5)
+    return near & (b > lo) & (b < hi)

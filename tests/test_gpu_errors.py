@@ -56,3 +56,34 @@ def test_plan_rejects_other_device_or_bad_shape():
     s2, perm2 = oq.rpbh_tables(3072, 0, 5)
     assert np.array_equal(s, s2) and np.array_equal(perm, perm2)
     p.close()
+
+
+@pytest.mark.parametrize("act,d,levels", [("int4_lloydmax", 1920, 16),
+                                          ("int4_lloydmax_width", 1920, 16),
+                                          ("int4_lloydmax_width", 256, 16),
+                                          ("int8_lloydmax", 3072, 256)])
+def test_plan_codebook_is_the_oracle_table(act, d, levels):
+    # oq_plan_get_codebook returns the table the plan quantizes with; the oracle solves the
+    # same optimality conditions by Lloyd iteration (the library by Newton's method)
+    import oracle
+    import w4a8_ptq_linear_b200 as oq
+    p = oq.Plan(d, 128 if d % 128 == 0 else 64, 1, act=act)
+    c, t = p.codebook()
+    ref_c, ref_t = (oracle.lloyd_max_sphere(d) if act == "int4_lloydmax_width"
+                    else oracle.lloyd_max_gaussian_8bit() if levels == 256
+                    else oracle.lloyd_max_gaussian())
+    assert c.shape == (levels,) and t.shape == (levels - 1,)
+    assert np.abs(c - ref_c).max() < 1e-8 and np.abs(t - ref_t).max() < 1e-8
+    assert np.all(np.diff(c) > 0) and np.allclose(t, (c[1:] + c[:-1]) / 2, rtol=0, atol=1e-12)
+    # a wrong level count and a plan without a codebook are argument errors
+    wrong = np.empty(256 if levels == 16 else 16)
+    with pytest.raises(oq.OQError) as e:
+        oq._check(oq.lib().oq_plan_get_codebook(p.handle, wrong.size, wrong.ctypes.data,
+                                                wrong.ctypes.data))
+    assert e.value.status == oq.OQ_ERR_INVALID_ARG
+    p.close()
+    q = oq.Plan(256, 64, 1, act="int8_absmax")
+    with pytest.raises(oq.OQError) as e:
+        q.codebook()
+    assert e.value.status == oq.OQ_ERR_INVALID_ARG
+    q.close()

@@ -192,7 +192,8 @@ def _asym_mutant(kind):
         lo, hi = wg.min(axis=2), wg.max(axis=2)
         sigma = np.maximum(hi - lo, eps) / (top + 1 if kind == "step_over_16" else top)
         if store is not None:
-            sigma = np.maximum(sigma, Gm.SIGMA_MIN_F16).astype(store).astype(np.float64)
+            sigma = np.maximum(np.maximum(sigma, Gm.SIGMA_MIN_F16), np.abs(lo) / Gm.SHIFT_MAX)
+            sigma = sigma.astype(store).astype(np.float64)
         z = (lo if kind == "shift_sign" else -lo) / sigma
         if store is not None:
             z = z.astype(store).astype(np.float64)

@@ -112,15 +112,22 @@ def test_layer_reduces_to_unquantized_for_fine_weights():
     assert np.abs(y - y_exact).max() > 0                  # the weights really are quantized
 
 
-def test_f32_decision_agrees_with_the_definition():
-    # the float32 restatement gives the fp64 definition's codes except where the value sits
-    # within float32 rounding of a tie; sigma and z equal unless a fp16 boundary intervenes
-    rng = np.random.default_rng(10)
-    w = (rng.standard_normal((64, 512)) * 0.02).astype(np.float32).astype(np.float64)
-    q64, s64, z64 = G.asym_group_quantize(w, store=np.float16)
-    q32, s32, z32 = G.asym_group_quantize_f32(w)
-    same_grid = (s64 == s32) & (z64 == z32)
-    assert same_grid.mean() > 0.99
-    mask = np.repeat(same_grid, 64, axis=1)
-    assert np.mean(q64[mask] != q32[mask]) < 1e-4
-    assert q32.min() >= 0 and q32.max() <= 15
+def test_fp16_storage_keeps_the_shift_finite_for_constant_groups():
+    # a constant group c has range 0: sigma would be the 2^-14 floor and z = -c 2^14, past the
+    # fp16 maximum 65504 once |c| > 4; the |min| / 2^15 floor keeps z finite and the group still
+    # reconstructs to within half a grid step (below 2^-15 |c| where that floor is active)
+    for c in (5.0, -7.25, 300.0, -0.001, 4.0):
+        w = np.full((1, 64), c)
+        w[0, 5] = c * (1 + 2.0 ** -20)          # a range far below the floor
+        q, s, z = G.asym_group_quantize(w, store=np.float16)
+        assert np.all(np.isfinite(z)) and np.abs(z).max() <= 65504
+        assert np.array_equal(z.astype(np.float16).astype(np.float64), z)
+        assert s[0, 0] >= abs(c) / G.SHIFT_MAX * (1 - 2.0 ** -11)
+        err = np.abs(G.dequantize(q, s, z) - w)
+        assert err.max() <= s[0, 0] * (0.5 + 2.0 ** -11 * max(1.0, abs(z[0, 0]))) + 1e-300
+        if abs(c) >= 2.0:                       # the |min| / 2^15 floor is the active one
+            assert err.max() <= abs(c) * 2.0 ** -15
+    # a group whose minimum is far from zero with a normal range keeps sigma = range / 15
+    w = np.linspace(100.0, 100.5, 64)[None, :]
+    q, s, z = G.asym_group_quantize(w, store=np.float16)
+    assert s[0, 0] == np.float16(0.5 / 15) and abs(z[0, 0]) < 65504

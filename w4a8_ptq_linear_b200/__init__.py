@@ -42,6 +42,7 @@ SIGNATURES = [
     ("oq_plan_create", _I, [ctypes.POINTER(_P), _I, _I, _I, _U64, _I, _I]),
     ("oq_plan_destroy", None, [_P]),
     ("oq_plan_get_rpbh", _I, [_P, _I, _P, _P]),
+    ("oq_plan_get_codebook", _I, [_P, _I, _P, _P]),
     ("oq_rotate_quantize", _I, [_P, _P, _I64, _I64, _P, _P, _P, _P, _P]),
     ("oq_prepare_weights", _I, [_P, _P, _I64, _I64, _P, _P, _P, _P]),
     ("oq_gemm_w4a8", _I, [_P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _P, _P]),
@@ -194,6 +195,15 @@ class Plan:
         p = np.empty(self.d, np.int32)
         _check(lib().oq_plan_get_rpbh(self._h, round_, s.ctypes.data, p.ctypes.data))
         return s, p
+
+    def codebook(self):
+        """The plan's Lloyd-Max codebook (oq_plan_get_codebook): (centroids, thresholds),
+        16 or 256 levels by the plan's activation kind."""
+        levels = 256 if self.act == "int8_lloydmax" else 16
+        c = np.empty(levels, np.float64)
+        t = np.empty(levels - 1, np.float64)
+        _check(lib().oq_plan_get_codebook(self._h, levels, c.ctypes.data, t.ctypes.data))
+        return c, t
 
     @property
     def packed(self) -> bool:

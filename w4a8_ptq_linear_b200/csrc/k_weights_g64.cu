@@ -4,10 +4,11 @@
 // Offline step after the rotation: every row of the rotated weight W_R is cut into groups of 64
 // consecutive columns; round to nearest sets the group's scale and shift from its minimum and
 // maximum, both are stored in fp16, and the codes are taken against the stored grid:
-//   sigma = fp16(max((max - min) / 15, 2^-14)),  z = fp16(-min / sigma),
+//   sigma = fp16(max((max - min) / 15, 2^-14, |min| / 2^15)),  z = fp16(-min / sigma),
 //   Q = clamp(rint(w / sigma + z), 0, 15),  stored nibble Q - 8 (= Q xor 8).
-// Every step is one IEEE operation rounded to nearest (division, addition, conversion), so a
-// float32 restatement of the same steps reproduces the codes bit for bit.
+// The 2^-14 floor keeps the grid from collapsing (smallest normal fp16); the |min| / 2^15 floor
+// keeps the stored shift |z| below 2^15 (1 + 2^-11), finite in fp16, for a nearly constant group
+// far from zero. Every step is one float32 operation rounded to nearest.
 //
 // K order: the GEMM decodes INT4 activation codes into an operand that holds, within every four
 // consecutive K positions, elements 0, 2, 1, 3 (it skips an interleave). The grouped weights are
@@ -47,7 +48,8 @@ __global__ void __launch_bounds__(256) k_quant_g64(const float* __restrict__ rot
       lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
       hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
     }
-    const float s = fmaxf(__fdiv_rn(__fsub_rn(hi, lo), 15.f), 0x1p-14f);
+    const float s = fmaxf(fmaxf(__fdiv_rn(__fsub_rn(hi, lo), 15.f), 0x1p-14f),
+                          fabsf(lo) * 0x1p-15f);   // exact: a power-of-two scale
     const __half s16 = __float2half_rn(s);
     const float sf = __half2float(s16);
     const __half z16 = __float2half_rn(__fdiv_rn(-lo, sf));

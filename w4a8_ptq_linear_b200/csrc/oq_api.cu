@@ -330,6 +330,25 @@ oq_status oq_plan_get_rpbh(const oq_plan* plan, int round, int8_t* signs_host,
   return OQ_OK;
 }
 
+oq_status oq_plan_get_codebook(const oq_plan* plan, int levels, double* centroids_host,
+                               double* thresholds_host) {
+  if (!plan || !centroids_host || !thresholds_host)
+    return fail(OQ_ERR_INVALID_ARG, "NULL argument");
+  int have = 0;
+  if (plan->act == OQ_ACT_INT4_LLOYDMAX || plan->act == OQ_ACT_INT4_LLOYDMAX_WIDTH) have = 16;
+  if (plan->act == OQ_ACT_INT8_LLOYDMAX) have = 256;
+  if (have == 0)
+    return fail(OQ_ERR_INVALID_ARG, "the plan's activation kind (%d) uses no codebook",
+                (int)plan->act);
+  if (levels != have)
+    return fail(OQ_ERR_INVALID_ARG, "the plan's codebook has %d levels, not %d", have, levels);
+  const double* c = have == 16 ? plan->cb_c : plan->cb8_c;
+  const double* t = have == 16 ? plan->cb_t : plan->cb8_t;
+  std::memcpy(centroids_host, c, sizeof(double) * (size_t)have);
+  std::memcpy(thresholds_host, t, sizeof(double) * (size_t)(have - 1));
+  return OQ_OK;
+}
+
 static oq_status rotate_quantize_impl(const oq_plan* plan, const void* x, int64_t T, int64_t ldx,
                                       void* codes, float* scale, float* mean, float* rotated,
                                       float* rowsum, int mode, int center, int wlayout,

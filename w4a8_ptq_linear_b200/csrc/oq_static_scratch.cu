@@ -12,9 +12,11 @@
 // loads the library holds one copy until the process exits. In host code the variable's name
 // is only a host-side stand-in, not a device address. So on the first call on each device
 // (that device current) the address is fetched once with cudaGetSymbolAddress and cached.
-// That first call should therefore come before any stream capture. All calls on a device share
-// the one array: calls whose kernels overlap on the GPU (different streams, or several host
-// threads) race on it and must be serialised by the caller. The array keeps the previous call's
+// That first call should therefore come before any stream capture. The cached address belongs
+// to the device's primary context: cudaDeviceReset (or another teardown of that context) makes
+// it stale, so after one the entry point must not be called again in the process. All calls on
+// a device share the one array: calls whose kernels overlap on the GPU (different streams, or
+// several host threads) race on it and must be serialised by the caller. The array keeps the previous call's
 // contents. Nothing in it has to start at zero: the GEMM reads only codes, scales and means that
 // the rotate+quantize kernel of the same call has just written (rows past T are never read).
 #include <mutex>
