@@ -74,6 +74,10 @@ def parse():
                     help="time rotate+quantize alone at every point of the bandwidth sweep "
                          "(T x d x h x rounds x output), one JSON line per point")
     ap.add_argument("--sweep-iters", type=int, default=10)
+    ap.add_argument("--peaks", action="store_true",
+                    help="measure the dense tensor-core peaks on this GPU: the library's "
+                         "tcgen05 peak loop (kind::i8, kind::f16) and cuBLAS int8 / bf16 "
+                         "GEMMs at 8192^3, with the SM clock sampled")
     return ap.parse_args()
 
 
@@ -320,10 +324,77 @@ def run_sweep(args):
     return 0
 
 
+def run_peaks(args):
+    """Dense tensor-core peaks of this GPU, each timed with CUDA events on its stream after
+    warm-up, best of `reps`:
+      - tcgen05 loop: oq_mma_peak_loop, the GEMMs' own instruction (cta_group::2, M = N = 256)
+        issued back to back on shared-memory operands, one CTA pair per two SMs;
+      - cuBLAS: torch._int_mm (int8 x int8 -> int32) and torch.matmul (bf16) at 8192^3.
+    One JSON line per measurement, with the SM clock and throttle reasons sampled during it."""
+    import torch
+    import w4a8_ptq_linear_b200 as oq
+    dev = torch.device("cuda", 0)
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    reps = 10
+
+    def timed(fn, n_inner):
+        fn()
+        torch.cuda.synchronize()
+        best = None
+        with ClockSampler(uuid, enabled=not args.no_clocks) as clk:
+            for _ in range(reps):
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record()
+                for _ in range(n_inner):
+                    fn()
+                e1.record()
+                torch.cuda.synchronize()
+                ms = e0.elapsed_time(e1) / n_inner
+                best = ms if best is None else min(best, ms)
+        return best, clk.summary()
+
+    out = []
+    for kind, k_per in (("i8", 32), ("f16", 16)):
+        iters = 1 << 14
+        pairs = oq.mma_peak_loop(kind, iters)
+        ms, clocks = timed(lambda: oq.mma_peak_loop(kind, iters), 4)
+        ops = pairs * iters * 4 * 2.0 * 256 * 256 * k_per
+        st, code = oq.device_status()
+        if st != 0:
+            raise RuntimeError(f"device status {st} code {code:#x} in the peak loop")
+        out.append({"peak": f"tcgen05 kind::{kind} loop", "value": ops / (ms * 1e-3) / 1e12,
+                    "unit": "TOPS" if kind == "i8" else "TFLOP/s", "ms": ms, "pairs": pairs,
+                    "clocks": clocks})
+    n = 8192
+    a8 = torch.randint(-128, 128, (n, n), dtype=torch.int8, device=dev)
+    b8 = torch.randint(-128, 128, (n, n), dtype=torch.int8, device=dev)
+    ms, clocks = timed(lambda: torch._int_mm(a8, b8), 1)
+    out.append({"peak": "cuBLAS int8 GEMM (torch._int_mm) 8192^3",
+                "value": 2.0 * n ** 3 / (ms * 1e-3) / 1e12, "unit": "TOPS", "ms": ms,
+                "clocks": clocks})
+    del a8, b8
+    ab = torch.randn((n, n), dtype=torch.bfloat16, device=dev)
+    bb = torch.randn((n, n), dtype=torch.bfloat16, device=dev)
+    ms, clocks = timed(lambda: torch.matmul(ab, bb), 1)
+    out.append({"peak": "cuBLAS bf16 GEMM (torch.matmul) 8192^3",
+                "value": 2.0 * n ** 3 / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms": ms,
+                "clocks": clocks})
+    for o in out:
+        print(json.dumps(o), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     if args.sweep:
         return run_sweep(args)
+    if args.peaks:
+        return run_peaks(args)
     import synth
     wl = synth.WORKLOADS[args.workload]
     T = args.tokens or wl.T

@@ -332,6 +332,19 @@ oq_status oq_linear_static_scratch(const oq_plan* plan, const void* x_bf16, int6
                                    const float* w_rowsum, const void* bias_bf16, int64_t d_out,
                                    void* y_bf16, void* stream);
 
+/* ---- measurement ------------------------------------------------------------------- */
+
+/* Tensor-core peak loop, the roofline denominator of the GEMMs (the pages have no
+ * counterpart; they quote no B200 figure). One CTA pair per two SMs; the pair's leader issues
+ * iters x 4 back-to-back tcgen05.mma.cta_group::2 instructions (M = 256, N = 256, 128 bytes of
+ * K per group of four) on operand tiles resident in shared memory, into one TMEM accumulator,
+ * with no memory traffic. kind 0: kind::i8 (int8 x int8 -> int32, K = 32 per instruction);
+ * kind 1: kind::f16 (fp16 x fp16 -> fp32, K = 16). One launch performs
+ * pairs * iters * 4 * 2 * 256 * 256 * K operations; *pairs_out (may be NULL) receives pairs.
+ * Asynchronous on `stream`: time it with events there. iters in [1, 2^16], else
+ * OQ_ERR_INVALID_ARG. */
+oq_status oq_mma_peak_loop(int kind, int64_t iters, int* pairs_out, void* stream);
+
 /* Test hook for the bounded waits: launches one block that waits on an mbarrier nothing
  * will arrive on, for at most timeout_ns, then records a timeout and returns. The next
  * oq_device_status() reports OQ_ERR_DEVICE_TIMEOUT. The GPU stays usable. */

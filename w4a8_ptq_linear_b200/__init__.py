@@ -55,6 +55,7 @@ SIGNATURES = [
     ("oq_gemm_w4a4_g64", _I, [_I, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _P, _P]),
     ("oq_linear_g64", _I, [_P, _P, _I64, _I64, _P, _P, _P, _P, _P, _I64, _P, _P, _SZ, _P]),
     ("oq_linear_static_scratch", _I, [_P, _P, _I64, _I64, _P, _P, _P, _P, _I64, _P, _P]),
+    ("oq_mma_peak_loop", _I, [_I, _I64, _P, _P]),
 ]
 
 
@@ -380,6 +381,15 @@ def linear_static_scratch(plan: Plan, x, w_packed, w_scale, w_rowsum=None, bias=
                                           _ptr(w_scale), _ptr(w_rowsum), _ptr(bias), N,
                                           _ptr(out), _stream(stream)))
     return out
+
+
+def mma_peak_loop(kind: str, iters: int, stream=None) -> int:
+    """oq_mma_peak_loop: launches the tensor-core peak loop (kind "i8" or "f16") on the
+    stream; returns the number of CTA pairs, from which the operation count follows."""
+    pairs = ctypes.c_int(0)
+    _check(lib().oq_mma_peak_loop({"i8": 0, "f16": 1}[kind], iters, ctypes.byref(pairs),
+                                  _stream(stream)))
+    return pairs.value
 
 
 def debug_wait_timeout(timeout_ns: int, stream=None):

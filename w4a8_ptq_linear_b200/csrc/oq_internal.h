@@ -61,6 +61,7 @@ enum : uint32_t {
   kSiteGemmConv = 18,      // GEMM MMA: stage converted
   kSiteGemmAccum = 19,     // GEMM epilogue: accumulator ready
   kSiteGemmDrain = 20,     // GEMM: drain after an abort
+  kSitePeak = 21,          // tensor-core peak loop: completion of the MMAs
   kSiteDebug = 99          // oq_debug_wait_timeout
 };
 
@@ -126,5 +127,8 @@ oq_status launch_quant_g64(const float* rot, int64_t n, int d, uint8_t* w_packed
                            float* w_scale, cudaStream_t s);
 
 oq_status launch_debug_wait(unsigned long long timeout_ns, cudaStream_t s);
+
+// Tensor-core peak loop (kind 0: kind::i8, 1: kind::f16); *pairs_out = CTA pairs launched.
+oq_status launch_mma_peak(int kind, int64_t iters, int* pairs_out, cudaStream_t s);
 
 }  // namespace oq
