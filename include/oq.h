@@ -345,6 +345,16 @@ oq_status oq_linear_static_scratch(const oq_plan* plan, const void* x_bf16, int6
  * OQ_ERR_INVALID_ARG. */
 oq_status oq_mma_peak_loop(int kind, int64_t iters, int* pairs_out, void* stream);
 
+/* Inspection hook (host only, no device needed): the word layout a plan of width d, block h
+ * and seed gives the two-token rotate-quantize kernel (d <= 8192). Channel j of the
+ * interleaved row (both tokens' bf16 values in one 32-bit word) is kept in word word_host[j]
+ * (int32[d], caller-owned); bank = word % 32. The layout is an edge colouring chosen so that
+ * every warp-wide store of the interleave pass (thread t of a d/32-thread block stores
+ * channels 8c + k, c = t + m d/32, m = 0..3, k = 0..7) and every warp-wide round-1 gather
+ * (register i of the warp's lanes) touches distinct banks. OQ_ERR_INVALID_ARG if d or h is
+ * outside the two-token kernel's range. */
+oq_status oq_debug_pair_layout(int d, int h, uint64_t seed, int32_t* word_host);
+
 /* Test hook for the bounded waits: launches one block that waits on an mbarrier nothing
  * will arrive on, for at most timeout_ns, then records a timeout and returns. The next
  * oq_device_status() reports OQ_ERR_DEVICE_TIMEOUT. The GPU stays usable. */

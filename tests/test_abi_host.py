@@ -118,3 +118,41 @@ def test_grouped_weight_arguments_rejected_up_front(lib):
                                       None) == oq.OQ_ERR_INVALID_ARG
     assert lib.oq_linear_g64(None, None, 16, 256, None, None, None, None, None, 256, None, None,
                              0, None) == oq.OQ_ERR_INVALID_ARG
+
+
+def _gather_position(h, t, i):
+    """Rotated position that thread t, register i of a round's gather holds (the block
+    transform's arrangement: consecutive for h <= 128, strided within the warp's 1024 positions
+    for h >= 256)."""
+    if h <= 128:
+        return t * 32 + i
+    e2 = h // 32
+    w, lane = divmod(t, 32)
+    blk, kb = divmod(lane, e2)
+    ia, ib = divmod(i, e2)
+    return w * 1024 + blk * h + kb + e2 * ia + 32 * ib
+
+
+@pytest.mark.parametrize("d,h,seed", [(256, 64, 0), (3072, 1024, 0), (1920, 128, 0),
+                                      (1920, 64, 3), (4096, 256, 11), (8192, 512, 5),
+                                      (1280, 256, 0), (96, 32, 2), (32, 1, 9)])
+def test_pair_word_layout_is_bank_conflict_free(lib, d, h, seed):
+    # every warp-wide store of the interleave pass and every warp-wide round-1 gather touches
+    # distinct banks (bank = word % 32), and the words of distinct channels are distinct
+    word = oq.debug_pair_layout(d, h, seed)
+    nact = d // 32
+    nwarps = (nact + 31) // 32
+    assert len(set(word.tolist())) == d and word.min() >= 0 and word.max() < nwarps * 1024
+    bank = word % 32
+    for w in range(nwarps):
+        lanes = [t for t in range(32 * w, min(32 * w + 32, nact))]
+        for m in range(4):
+            for k in range(8):
+                chans = [8 * (t + m * nact) + k for t in lanes]
+                assert len(set(bank[chans].tolist())) == len(chans)
+    perm = oracle.rpbh_plan(d, h, 1, seed)[0][1].astype(np.int64)
+    for w in range(nwarps):
+        lanes = [t for t in range(32 * w, min(32 * w + 32, nact))]
+        for i in range(32):
+            chans = [perm[_gather_position(h, t, i)] for t in lanes]
+            assert len(set(bank[chans].tolist())) == len(chans)

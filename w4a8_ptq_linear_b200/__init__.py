@@ -56,6 +56,7 @@ SIGNATURES = [
     ("oq_linear_g64", _I, [_P, _P, _I64, _I64, _P, _P, _P, _P, _P, _I64, _P, _P, _SZ, _P]),
     ("oq_linear_static_scratch", _I, [_P, _P, _I64, _I64, _P, _P, _P, _P, _I64, _P, _P]),
     ("oq_mma_peak_loop", _I, [_I, _I64, _P, _P]),
+    ("oq_debug_pair_layout", _I, [_I, _I, _U64, _P]),
 ]
 
 
@@ -390,6 +391,14 @@ def mma_peak_loop(kind: str, iters: int, stream=None) -> int:
     _check(lib().oq_mma_peak_loop({"i8": 0, "f16": 1}[kind], iters, ctypes.byref(pairs),
                                   _stream(stream)))
     return pairs.value
+
+
+def debug_pair_layout(d: int, h: int, seed: int = 0):
+    """oq_debug_pair_layout: the word of every channel in the two-token kernel's
+    interleaved row (int32[d])."""
+    w = np.empty(d, np.int32)
+    _check(lib().oq_debug_pair_layout(d, h, seed, w.ctypes.data))
+    return w
 
 
 def debug_wait_timeout(timeout_ns: int, stream=None):

@@ -58,6 +58,8 @@ struct RqParams {
   float pct_mult;      // percentile: gamma / Phi^-1((1 + rho) / 2)
   const uint16_t* tab;   // rounds x d entries in kernel order
   const uint4* smask;    // round-1 source signs: bit 15 / 31 of word j/2 flips channel j
+  const uint4* slot;     // two-token kernel: byte offset of channel j's word, [j%8/4][j/8][j%4]
+  int land_bytes;        // two-token kernel: bytes of one landing buffer
   const float4* ones;    // c' = unnormalised round-1 transform of the all-ones vector
   void* codes;
   float* scale;
@@ -719,32 +721,28 @@ __global__ void __launch_bounds__(256, 2) k_rotate_quant_pair(const RqParams p) 
   const bool active = tid < nact;
   const uint32_t row_bytes = (uint32_t)d * 2u;
   const uint32_t row_stride = (row_bytes + 127u) & ~127u;
-  const uint32_t pair_bytes = 2u * row_stride;
-  constexpr int HMODE = HLOG2 <= 5 ? 0 : (HLOG2 <= 7 ? 1 : 2);
-  // [nbuf landing pairs (row A | row B)] [interleaved words, later the transpose tiles]
-  // [round buffer, two rounds only] [reductions, thresholds, barriers]
-  // [transpose tiles, h >= 256 only: their own region, so that no block barrier separates the
-  // gather from the transposes] [round-1 sign masks]
+  const size_t land_bytes = (size_t)p.land_bytes;
+  // [two landing buffers: a pair of rows (A | B) each; while a pass runs, its own buffer also
+  //  holds the warps' transpose tiles (h >= 256), so no barrier separates a warp's gather from
+  //  its transposes] [interleaved words, bank-aware layout: nwarps x 4 KB]
+  // [round buffer, two rounds only] [reductions, code cells, barriers, percentile lists,
+  //  8-bit Lloyd-Max thresholds]
   uint8_t* land = smem;
-  uint32_t* wbuf = reinterpret_cast<uint32_t*>(smem + (size_t)p.nbuf * pair_bytes);
-  float2* rbuf = reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(wbuf) + nwarps * 4096);
+  uint8_t* wbuf = smem + 2 * land_bytes;
+  float2* rbuf = reinterpret_cast<float2*>(wbuf + nwarps * 4096);
   float* red = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(rbuf) +
                                         (ROUNDS == 2 ? nwarps * 8192 : 0));
   // red: [0,16) sums, [16,32) statistic; then 32 Lloyd-Max code cells and the barriers
   float2* cells = reinterpret_cast<float2*>(red + 32);
   uint64_t* bars = reinterpret_cast<uint64_t*>(red + 96);
   float* pct_lists = red + 128;   // percentile: up to 8 warps x 2 tokens x 6 ranks
-  float* tiles = red + 224;       // h >= 256: nwarps x 1024 floats
-  uint4* s_mask = reinterpret_cast<uint4*>(tiles + (HMODE == 2 ? nwarps * 1024 : 0));
-  float* s_thr8 = reinterpret_cast<float*>(s_mask + d / 8);   // 8-bit Lloyd-Max thresholds
-  float* warp_tile = tiles + warp * 1024;
+  float* s_thr8 = red + 224;      // 8-bit Lloyd-Max thresholds
 
   if (tid < 32) cells[tid] = p.cells[tid];
-  for (int c = tid; c < d / 8; c += blockDim.x) s_mask[c] = __ldg(p.smask + c);
   if (p.mode == kRqLloydMax8)
     for (int k = tid; k < 256; k += blockDim.x) s_thr8[k] = __ldg(p.thr8 + k);
   if (tid == 0) {
-    for (int b = 0; b < p.nbuf; ++b) dev::mbar_init(dev::smem_u32(&bars[b]), 1);
+    for (int b = 0; b < 2; ++b) dev::mbar_init(dev::smem_u32(&bars[b]), 1);
     dev::fence_mbar_init();
   }
   __syncthreads();
@@ -755,13 +753,13 @@ __global__ void __launch_bounds__(256, 2) k_rotate_quant_pair(const RqParams p) 
   auto issue = [&](int b, int64_t q) {
     const int64_t ta = 2 * q, tb = (2 * q + 1 < T) ? 2 * q + 1 : 2 * q;
     const uint32_t bar = dev::smem_u32(&bars[b]);
-    uint8_t* dst = land + (size_t)b * pair_bytes;
+    uint8_t* dst = land + (size_t)b * land_bytes;
     dev::mbar_arrive_expect_tx(bar, 2u * row_bytes);
     dev::bulk_g2s(dev::smem_u32(dst), p.x + ta * p.ldx, row_bytes, bar);
     dev::bulk_g2s(dev::smem_u32(dst + row_stride), p.x + tb * p.ldx, row_bytes, bar);
   };
   if (tid == 0)
-    for (int b = 0; b < p.nbuf; ++b)
+    for (int b = 0; b < 2; ++b)
       if ((int64_t)blockIdx.x + (int64_t)b * G < NP) issue(b, (int64_t)blockIdx.x + (int64_t)b * G);
 
   const bool lm8 = p.mode == kRqLloydMax8;
@@ -770,9 +768,13 @@ __global__ void __launch_bounds__(256, 2) k_rotate_quant_pair(const RqParams p) 
   int it = 0;
   bool aborted = false;
   for (int64_t q = blockIdx.x; q < NP; q += G, ++it) {
-    const int b = it % p.nbuf;
+    const int b = it & 1;
+    uint8_t* lb = land + (size_t)b * land_bytes;
+    float* warp_tile = reinterpret_cast<float*>(lb) + warp * 1024;
     const int64_t ta = 2 * q;
     const bool has_b = ta + 1 < T;
+    // round-1 gather entries (byte offsets into the word buffer), L1-resident; loaded before
+    // the wait so that their latency overlaps it
     uint32_t t0[EP / 2];
 #pragma unroll
     for (int i = 0; i < EP / 2; ++i) t0[i] = 0u;
@@ -784,28 +786,34 @@ __global__ void __launch_bounds__(256, 2) k_rotate_quant_pair(const RqParams p) 
         t0[4 * i] = w.x; t0[4 * i + 1] = w.y; t0[4 * i + 2] = w.z; t0[4 * i + 3] = w.w;
       }
     }
-    int fail = !dev::mbar_wait(dev::smem_u32(&bars[b]), (uint32_t)(it / p.nbuf) & 1u, p.err,
+    int fail = !dev::mbar_wait(dev::smem_u32(&bars[b]), (uint32_t)(it >> 1) & 1u, p.err,
                                kSiteRqRow, p.limit_ns);
 
-    // ---- source-side signs, interleave A|B, row sums ----------------------------------
+    // ---- source-side signs, interleave A|B into the bank-aware word layout, row sums ------
+    // Channel 8c + k of both tokens becomes one word (A low, B high) at the byte offset the
+    // plan's slot table gives: the eight stores of a chunk, and the round-1 gathers below,
+    // each touch 32 distinct banks across the warp.
     float2 psum = make_float2(0.f, 0.f);
     if (active && !fail) {
-      const uint4* ra = reinterpret_cast<const uint4*>(land + (size_t)b * pair_bytes);
-      const uint4* rb = reinterpret_cast<const uint4*>(land + (size_t)b * pair_bytes + row_stride);
-      uint4* wv = reinterpret_cast<uint4*>(wbuf);
+      const uint4* ra = reinterpret_cast<const uint4*>(lb);
+      const uint4* rb = reinterpret_cast<const uint4*>(lb + row_stride);
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
         const int c = tid + m * nact;
         uint4 a = ra[c], bb = rb[c];
-        const uint4 mk = s_mask[c];
+        const uint4 mk = __ldg(p.smask + c);
+        const uint4 s0 = __ldg(p.slot + c), s1 = __ldg(p.slot + d / 8 + c);
         if (p.want_sum) psum = __fadd2_rn(psum, chunk_sums(a, bb));
         a.x ^= mk.x; a.y ^= mk.y; a.z ^= mk.z; a.w ^= mk.w;
         bb.x ^= mk.x; bb.y ^= mk.y; bb.z ^= mk.z; bb.w ^= mk.w;
-        // channels 8c..8c+3 -> words 4c..4c+3, channels 8c+4..8c+7 -> words d/2 + 4c..
-        wv[c] = make_uint4(__byte_perm(a.x, bb.x, 0x5410), __byte_perm(a.x, bb.x, 0x7632),
-                           __byte_perm(a.y, bb.y, 0x5410), __byte_perm(a.y, bb.y, 0x7632));
-        wv[d / 8 + c] = make_uint4(__byte_perm(a.z, bb.z, 0x5410), __byte_perm(a.z, bb.z, 0x7632),
-                                   __byte_perm(a.w, bb.w, 0x5410), __byte_perm(a.w, bb.w, 0x7632));
+        *reinterpret_cast<uint32_t*>(wbuf + s0.x) = __byte_perm(a.x, bb.x, 0x5410);
+        *reinterpret_cast<uint32_t*>(wbuf + s0.y) = __byte_perm(a.x, bb.x, 0x7632);
+        *reinterpret_cast<uint32_t*>(wbuf + s0.z) = __byte_perm(a.y, bb.y, 0x5410);
+        *reinterpret_cast<uint32_t*>(wbuf + s0.w) = __byte_perm(a.y, bb.y, 0x7632);
+        *reinterpret_cast<uint32_t*>(wbuf + s1.x) = __byte_perm(a.z, bb.z, 0x5410);
+        *reinterpret_cast<uint32_t*>(wbuf + s1.y) = __byte_perm(a.z, bb.z, 0x7632);
+        *reinterpret_cast<uint32_t*>(wbuf + s1.z) = __byte_perm(a.w, bb.w, 0x5410);
+        *reinterpret_cast<uint32_t*>(wbuf + s1.w) = __byte_perm(a.w, bb.w, 0x7632);
       }
     }
     if (p.want_sum) {
@@ -817,14 +825,12 @@ __global__ void __launch_bounds__(256, 2) k_rotate_quant_pair(const RqParams p) 
       aborted = true;
       break;
     }
-    // every thread is past its reads of landing pair b: refill it
-    if (tid == 0 && q + (int64_t)p.nbuf * G < NP) issue(b, q + (int64_t)p.nbuf * G);
 
     // ---- round 1: one gather for both tokens ---------------------------------------------
     float2 v[EP];
 #pragma unroll
     for (int i = 0; i < EP; ++i) {
-      const uint32_t w = active ? wbuf[entry(t0, i)] : 0u;
+      const uint32_t w = active ? *reinterpret_cast<const uint32_t*>(wbuf + entry(t0, i)) : 0u;
       v[i] = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
     }
     float2 mu = make_float2(0.f, 0.f);
@@ -907,6 +913,8 @@ __global__ void __launch_bounds__(256, 2) k_rotate_quant_pair(const RqParams p) 
     }
     if (lane == 0 && !pct) { red[16 + 2 * warp] = st.x; red[16 + 2 * warp + 1] = st.y; }
     __syncthreads();
+    // every thread is past its reads of landing buffer b (rows and transpose tiles): refill it
+    if (tid == 0 && q + 2 * G < NP) issue(b, q + 2 * G);
     st = make_float2(0.f, 0.f);
     if (pct) {
       switch (p.pct_r) {
@@ -1035,19 +1043,21 @@ __global__ void __launch_bounds__(256, 2) k_rotate_quant_pair(const RqParams p) 
     }
   }
 
+  // After an abort, wait (bounded) for the row loads this CTA still has in flight, so that no
+  // bulk copy lands in shared memory after the block has exited.
   if (aborted && tid == 0) {
-    for (int k = 0; k < p.nbuf; ++k) {
+    for (int k = 0; k < 2; ++k) {
       const int j = it + k;
       if ((int64_t)blockIdx.x + (int64_t)j * G >= NP) break;
-      dev::mbar_wait(dev::smem_u32(&bars[j % p.nbuf]), (uint32_t)(j / p.nbuf) & 1u, p.err,
-                     kSiteRqDrain, p.limit_ns);
+      dev::mbar_wait(dev::smem_u32(&bars[j & 1]), (uint32_t)(j >> 1) & 1u, p.err, kSiteRqDrain,
+                     p.limit_ns);
     }
   }
 }
 
 struct LaunchCfg {
   void* fn = nullptr;
-  int nthr = 0, nbuf = 0, grid_per_sm = 0, mask_smem = 0, pair = 0;
+  int nthr = 0, nbuf = 0, grid_per_sm = 0, mask_smem = 0, pair = 0, land_bytes = 0;
   size_t smem = 0;
 };
 
@@ -1100,8 +1110,8 @@ void* kern_pair_h(int hlog2) {
   }
 }
 
-// widths up to 8192 (at most 256 threads) run two tokens per pass
-constexpr int kPairMaxD = 8192;
+// widths up to kRqPairMaxD (at most 256 threads) run two tokens per pass
+constexpr int kPairMaxD = kRqPairMaxD;
 
 // CentriQ App. B.3 (Tab. 3): activation quantile rho and clip factor gamma*
 constexpr double kPctRho = 0.9995;
@@ -1128,14 +1138,6 @@ int64_t rq_gather_position(int h, int t, int i) {
   const int warp = t / 32, lane = t % 32;
   const int blk = lane / E2, kB = lane % E2, ia = i / E2, ib = i % E2;
   return (int64_t)warp * 1024 + (int64_t)blk * h + kB + E2 * ia + 32 * ib;
-}
-
-// Word of the staged input row that holds channel j. The pair kernel keeps channels
-// 8c..8c+3 in words 4c..4c+3 and channels 8c+4..8c+7 in words d/2 + 4c.. (each word carries
-// the channel of both tokens); the single-token kernel reads the bf16 row as it is.
-int rq_round1_index(int d, int j) {
-  if (d > kPairMaxD) return j;
-  return ((j >> 3) << 2) + (j & 3) + ((j & 4) ? d / 2 : 0);
 }
 
 // Index in the swizzled round buffer at which rotated position p is stored: float2 slots
@@ -1180,19 +1182,21 @@ oq_status launch_rotate_quant(const RqArgs& a, cudaStream_t s) {
       cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev_id);
       const size_t row_stride = ((size_t)a.d * 2 + 127) & ~(size_t)127;
       if (a.d <= kPairMaxD) {
-        // nbuf landing pairs, the interleaved words / transpose tiles, the round buffer,
-        // reductions + thresholds + barriers, the source-sign masks and, for 8-bit Lloyd-Max
-        // codes only, the 256 thresholds (1 KB less keeps 5 CTAs per SM at some widths)
+        // two landing buffers (each a row pair, and while its pass runs the warps' transpose
+        // tiles), the interleaved words, the round buffer, then reductions + code cells +
+        // barriers + percentile lists and, for 8-bit Lloyd-Max codes only, the 256 thresholds
         cfg.pair = 1;
         cfg.fn = a.rounds == 1 ? kern_pair_h<1>(hlog2) : kern_pair_h<2>(hlog2);
         cfg.nthr = nthr;
         ce = allow_max_dynamic_smem(cfg.fn);
         if (ce != cudaSuccess) return cuda_fail(ce, "cudaFuncSetAttribute(rotate_quant)");
-        cfg.nbuf = 1;
-        cfg.smem = (size_t)cfg.nbuf * 2 * row_stride + (size_t)(nthr / 32) * 4096 +
-                   (a.rounds == 2 ? (size_t)(nthr / 32) * 8192 : 0) + 224 * 4 +
-                   (hmode == 2 ? (size_t)(nthr / 32) * 4096 : 0) + (size_t)a.d * 2 +
-                   (lm8 ? 1024 : 0);
+        cfg.nbuf = 2;
+        const size_t nw = (size_t)(nthr / 32);
+        size_t land = 2 * row_stride;
+        if (hmode == 2) land = std::max(land, nw * 4096);
+        cfg.land_bytes = (int)((land + 127) & ~(size_t)127);
+        cfg.smem = 2 * (size_t)cfg.land_bytes + nw * 4096 + (a.rounds == 2 ? nw * 8192 : 0) +
+                   (size_t)(224 + (lm8 ? 256 : 0)) * 4;
         int best_occ = 0;
         ce = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&best_occ, cfg.fn, nthr, cfg.smem);
         if (ce != cudaSuccess) return cuda_fail(ce, "occupancy(rotate_quant)");
@@ -1255,6 +1259,9 @@ oq_status launch_rotate_quant(const RqArgs& a, cudaStream_t s) {
   }
   p.tab = a.tab;
   p.smask = reinterpret_cast<const uint4*>(a.smask);
+  p.slot = reinterpret_cast<const uint4*>(a.slot);
+  p.land_bytes = cfg.land_bytes;
+  if (cfg.pair && !a.slot) return fail(OQ_ERR_INVALID_ARG, "rotate_quant: plan has no word layout");
   p.ones = reinterpret_cast<const float4*>(a.ones);
   p.codes = a.codes;
   p.scale = a.scale;

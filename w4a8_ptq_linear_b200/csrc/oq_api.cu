@@ -231,6 +231,21 @@ oq_status oq_plan_create(oq_plan** out, int d, int h, int rounds, uint64_t seed,
   std::vector<uint16_t> tab((size_t)rounds * d);
   for (int r = 0; r < rounds; ++r)
     rpbh_round_tables(d, r, seed, p->signs.data() + (size_t)r * d, p->perm.data() + (size_t)r * d);
+  // Two-token kernel (d <= kRqPairMaxD): the interleaved row keeps channel j in word word[j]
+  // (bank-conflict-free stores and gathers); round-1 entries are byte offsets of those words.
+  // The single-token kernel reads the bf16 row as it is: entry = channel index.
+  const bool pair = d <= kRqPairMaxD;
+  std::vector<int> word;
+  if (pair) {
+    word = pair_word_layout(d, h, p->perm.data());
+    if (word.size() != (size_t)d) {
+      delete p;
+      return fail(OQ_ERR_UNSUPPORTED, "word layout failed for d=%d h=%d", d, h);
+    }
+  }
+  std::vector<uint32_t> slot(pair ? (size_t)d : 0);
+  for (int j = 0; pair && j < d; ++j)
+    slot[((size_t)((j % 8) / 4) * (d / 8) + j / 8) * 4 + j % 4] = 4u * (uint32_t)word[(size_t)j];
   for (int r = 0; r < rounds; ++r) {
     const int8_t* sg = p->signs.data() + (size_t)r * d;
     const int32_t* pm = p->perm.data() + (size_t)r * d;
@@ -238,7 +253,7 @@ oq_status oq_plan_create(oq_plan** out, int d, int h, int rounds, uint64_t seed,
       for (int i = 0; i < 32; ++i) {
         const int64_t q = rq_gather_position(h, t, i);
         // round 1 carries no sign: it is applied to the source channel (see below)
-        const int src = (r == 0) ? rq_round1_index(d, pm[q])
+        const int src = (r == 0) ? (pair ? 4 * word[(size_t)pm[q]] : pm[q])
                                  : (rq_round_buffer_index(d, pm[q]) | (sg[q] < 0 ? 0x8000 : 0));
         tab[(size_t)r * d + (size_t)t * 32 + i] = (uint16_t)src;
       }
@@ -271,13 +286,15 @@ oq_status oq_plan_create(oq_plan** out, int d, int h, int rounds, uint64_t seed,
   auto release = [&]() {
     if (p->d_tab) cudaFree(p->d_tab);
     if (p->d_smask) cudaFree(p->d_smask);
+    if (p->d_slot) cudaFree(p->d_slot);
     if (p->d_ones) cudaFree(p->d_ones);
     if (p->d_thr8) cudaFree(p->d_thr8);
     delete p;
   };
   if (cudaMalloc(&p->d_tab, tab.size() * sizeof(uint16_t)) != cudaSuccess ||
       cudaMalloc(&p->d_smask, smask.size() * sizeof(uint32_t)) != cudaSuccess ||
-      cudaMalloc(&p->d_ones, ones.size() * sizeof(float)) != cudaSuccess) {
+      cudaMalloc(&p->d_ones, ones.size() * sizeof(float)) != cudaSuccess ||
+      (pair && cudaMalloc(&p->d_slot, slot.size() * sizeof(uint32_t)) != cudaSuccess)) {
     release();
     return fail(OQ_ERR_NOMEM, "cudaMalloc plan tables");
   }
@@ -287,6 +304,8 @@ oq_status oq_plan_create(oq_plan** out, int d, int h, int rounds, uint64_t seed,
                    cudaMemcpyHostToDevice);
   if (e == cudaSuccess)
     e = cudaMemcpy(p->d_ones, ones.data(), ones.size() * sizeof(float), cudaMemcpyHostToDevice);
+  if (e == cudaSuccess && pair)
+    e = cudaMemcpy(p->d_slot, slot.data(), slot.size() * sizeof(uint32_t), cudaMemcpyHostToDevice);
   if (e == cudaSuccess && act == OQ_ACT_INT8_LLOYDMAX) {
     float thr[256];
     for (int k = 0; k < 255; ++k) thr[k] = (float)p->cb8_t[k];
@@ -308,12 +327,13 @@ oq_status oq_plan_create(oq_plan** out, int d, int h, int rounds, uint64_t seed,
 
 void oq_plan_destroy(oq_plan* plan) {
   if (!plan) return;
-  if (plan->d_tab || plan->d_smask || plan->d_ones || plan->d_thr8) {
+  if (plan->d_tab || plan->d_smask || plan->d_ones || plan->d_thr8 || plan->d_slot) {
     int cur = -1;
     cudaGetDevice(&cur);
     if (cur != plan->device) cudaSetDevice(plan->device);
     if (plan->d_tab) cudaFree(plan->d_tab);
     if (plan->d_smask) cudaFree(plan->d_smask);
+    if (plan->d_slot) cudaFree(plan->d_slot);
     if (plan->d_ones) cudaFree(plan->d_ones);
     if (plan->d_thr8) cudaFree(plan->d_thr8);
     if (cur != plan->device && cur >= 0) cudaSetDevice(cur);
@@ -327,6 +347,19 @@ oq_status oq_plan_get_rpbh(const oq_plan* plan, int round, int8_t* signs_host,
   if (round < 0 || round >= plan->rounds) return fail(OQ_ERR_INVALID_ARG, "round out of range");
   std::memcpy(signs_host, plan->signs.data() + (size_t)round * plan->d, plan->d);
   std::memcpy(perm_host, plan->perm.data() + (size_t)round * plan->d, plan->d * sizeof(int32_t));
+  return OQ_OK;
+}
+
+oq_status oq_debug_pair_layout(int d, int h, uint64_t seed, int32_t* word_host) {
+  if (!word_host) return fail(OQ_ERR_INVALID_ARG, "NULL output");
+  if (d < 32 || d > kRqPairMaxD || d % 32 || !pow2(h) || h > 1024 || d % h)
+    return fail(OQ_ERR_INVALID_ARG, "d=%d h=%d outside the two-token kernel's range", d, h);
+  std::vector<int8_t> sg((size_t)d);
+  std::vector<int32_t> pm((size_t)d);
+  rpbh_round_tables(d, 0, seed, sg.data(), pm.data());
+  const std::vector<int> word = pair_word_layout(d, h, pm.data());
+  if (word.size() != (size_t)d) return fail(OQ_ERR_UNSUPPORTED, "word layout failed");
+  for (int j = 0; j < d; ++j) word_host[j] = word[(size_t)j];
   return OQ_OK;
 }
 
@@ -356,6 +389,7 @@ static oq_status rotate_quantize_impl(const oq_plan* plan, const void* x, int64_
   RqArgs a;
   a.x = x; a.ldx = ldx; a.T = T; a.d = plan->d; a.h = plan->h; a.rounds = plan->rounds;
   a.center = center; a.mode = mode; a.tab = plan->d_tab; a.smask = plan->d_smask;
+  a.slot = plan->d_slot;
   a.ones = plan->d_ones; a.codes = codes; a.scale = scale;
   a.mean = mean; a.rotated = rotated; a.rowsum = rowsum; a.wlayout = wlayout;
   a.thr8 = plan->d_thr8;

@@ -20,6 +20,8 @@ struct oq_plan {
   uint16_t* d_tab = nullptr;    // device: rounds * d gather entries in kernel order,
                                 // source index (| (sign < 0) << 15 in round 2)
   uint32_t* d_smask = nullptr;  // device: d/2 words, round-1 sign of channel j at bit 15 / 31
+  uint32_t* d_slot = nullptr;   // device (d <= 8192): byte offset of channel j's word,
+                                // laid out [j % 8 / 4][j / 8][j % 4]
   float* d_ones = nullptr;      // device: d floats, unnormalised round-1 transform of ones
   double cb_c[16] = {}, cb_t[15] = {};
   double cb8_c[256] = {}, cb8_t[255] = {};   // 8-bit Lloyd-Max codebook
@@ -75,6 +77,7 @@ struct RqArgs {
   int d = 0, h = 0, rounds = 0, center = 0, mode = 0;
   const uint16_t* tab = nullptr;  // rounds * d
   const uint32_t* smask = nullptr;  // d/2 words: round-1 signs moved to the source channels
+  const uint32_t* slot = nullptr;   // d <= kRqPairMaxD: byte offsets of the channels' words
   const float* ones = nullptr;      // d floats: unnormalised round-1 transform of all ones
   void* codes = nullptr;
   float* scale = nullptr;
@@ -90,8 +93,13 @@ oq_status launch_rotate_quant(const RqArgs& a, cudaStream_t s);
 // round, where the staged input row keeps channel j, and where the fp32 round buffer keeps
 // rotated position p (the last two depend on which kernel shape width d uses).
 int64_t rq_gather_position(int h, int t, int i);
-int rq_round1_index(int d, int j);
 int rq_round_buffer_index(int d, int p);
+// Widths up to this run the two-token kernel; wider rows the single-token kernel.
+constexpr int kRqPairMaxD = 8192;
+// Two-token kernel: the word (32-bit slot of the interleaved row) of every channel, chosen so
+// that the interleave stores and the round-1 gathers of a warp are free of bank conflicts
+// (a 32-colour edge colouring of the bipartite store-group / gather-group multigraph).
+std::vector<int> pair_word_layout(int d, int h, const int32_t* perm0);
 
 // ---- GEMM ----------------------------------------------------------------------------------
 // kGemmG64: INT4 codes (decoded to fp16 integers) against asymmetric g = 64 weights

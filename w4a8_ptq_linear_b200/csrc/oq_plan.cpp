@@ -242,3 +242,83 @@ void lloyd_max_newton_256(double c256[256], double t255[255]) {
 }
 
 }  // namespace oq
+
+namespace oq {
+
+// Bank-aware word layout of the two-token kernel's interleaved row (widths d <= 8192).
+//
+// The interleave pass stores one 32-bit word per channel (both tokens' bf16 values) and the
+// round-1 gather loads one word per rotated position. Each warp-wide store instruction writes
+// a fixed set of channels (a "store group": thread t stores channels 8c + k, c = t + m nact,
+// for chunk m and k = 0..7), and each warp-wide gather instruction reads the channels of a
+// fixed set of rotated positions (a "gather group": register i of the warp's 32 lanes). A
+// channel lies in exactly one group of each kind, so the channels are the edges of a bipartite
+// multigraph between store groups and gather groups in which every node has degree <= 32.
+// By Koenig's edge-colouring theorem its edges can be coloured with 32 colours so that no two
+// edges at a node share a colour; with colour = shared-memory bank, every store and every
+// gather instruction then touches 32 distinct banks (no bank conflict). The colouring is built
+// edge by edge: an edge takes a colour free at both ends, or, when the free colours a (at the
+// store end) and b (at the gather end) differ, the a/b alternating path from the gather end is
+// recoloured first (in a bipartite graph it cannot reach the store end).
+// The word of channel ch is then 32 * store_group(ch) + colour(ch): unique, since the channels
+// of one store group have distinct colours.
+std::vector<int> pair_word_layout(int d, int h, const int32_t* perm0) {
+  const int nact = d / 32;                       // threads that own positions
+  const int nwarps = (nact + 31) / 32;
+  const int ng = nwarps * 32;                    // groups of each kind
+  std::vector<int> wg((size_t)d), rg((size_t)d, -1);
+  for (int ch = 0; ch < d; ++ch) {
+    const int c = ch / 8, k = ch % 8;
+    const int t = c % nact, m = c / nact;       // thread t, chunk m
+    wg[(size_t)ch] = ((t / 32) * 4 + m) * 8 + k;
+  }
+  for (int t = 0; t < nact; ++t)
+    for (int i = 0; i < 32; ++i) {
+      const int64_t q = rq_gather_position(h, t, i);
+      rg[(size_t)perm0[q]] = (t / 32) * 32 + i;
+    }
+  std::vector<int> at_w((size_t)ng * 32, -1), at_r((size_t)ng * 32, -1), col((size_t)d, -1);
+  auto free_at = [&](const std::vector<int>& at, int node) {
+    for (int c = 0; c < 32; ++c)
+      if (at[(size_t)node * 32 + c] < 0) return c;
+    return -1;
+  };
+  std::vector<int> path;
+  for (int ch = 0; ch < d; ++ch) {
+    const int u = wg[(size_t)ch], v = rg[(size_t)ch];
+    const int a = free_at(at_w, u), b = free_at(at_r, v);
+    if (a < 0 || b < 0) return {};              // degree above 32: cannot happen
+    if (at_r[(size_t)v * 32 + a] >= 0) {
+      // flip the a/b path that starts at v with its a-edge
+      path.clear();
+      int node = v, c = a;
+      bool on_gather_side = true;
+      while (true) {
+        const std::vector<int>& at = on_gather_side ? at_r : at_w;
+        const int e = at[(size_t)node * 32 + c];
+        if (e < 0) break;
+        path.push_back(e);
+        node = on_gather_side ? wg[(size_t)e] : rg[(size_t)e];
+        on_gather_side = !on_gather_side;
+        c = (c == a) ? b : a;
+      }
+      for (int e : path) {                       // clear, then recolour swapped
+        at_w[(size_t)wg[(size_t)e] * 32 + col[(size_t)e]] = -1;
+        at_r[(size_t)rg[(size_t)e] * 32 + col[(size_t)e]] = -1;
+      }
+      for (int e : path) {
+        col[(size_t)e] = (col[(size_t)e] == a) ? b : a;
+        at_w[(size_t)wg[(size_t)e] * 32 + col[(size_t)e]] = e;
+        at_r[(size_t)rg[(size_t)e] * 32 + col[(size_t)e]] = e;
+      }
+    }
+    col[(size_t)ch] = a;
+    at_w[(size_t)u * 32 + a] = ch;
+    at_r[(size_t)v * 32 + a] = ch;
+  }
+  std::vector<int> word((size_t)d);
+  for (int ch = 0; ch < d; ++ch) word[(size_t)ch] = 32 * wg[(size_t)ch] + col[(size_t)ch];
+  return word;
+}
+
+}  // namespace oq
