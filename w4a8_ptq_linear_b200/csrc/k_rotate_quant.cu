@@ -503,6 +503,9 @@ __global__ void __launch_bounds__(MAXT, 1) k_rotate_quant(const RqParams p) {
 // channel (A in the low half, B in the high half).
 // ================================================================================================
 
+// the two-token kernel's extra quantizer instantiation: 4-bit absmax codes in the GEMM layout
+constexpr int kPairInt4W = 5;
+
 template <int BIT>
 __device__ __forceinline__ void stage_pair(float2 (&v)[EP]) {
   constexpr int L = 1 << BIT;
@@ -710,7 +713,9 @@ __device__ __forceinline__ float2 pct_quantiles(const float* lists, int nwarps, 
                      fmaf(frac, ob[R - 2] - ob[R - 1], ob[R - 1]));
 }
 
-template <int HLOG2, int ROUNDS>
+// MODE: the quantizer (RqMode), or kPairInt4W for 4-bit absmax codes in the GEMM weight layout.
+// One instantiation per quantizer keeps each kernel's code small.
+template <int HLOG2, int ROUNDS, int MODE>
 __global__ void __launch_bounds__(256, 2) k_rotate_quant_pair(const RqParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const int d = p.d;
@@ -739,7 +744,7 @@ __global__ void __launch_bounds__(256, 2) k_rotate_quant_pair(const RqParams p) 
   float* s_thr8 = red + 224;      // 8-bit Lloyd-Max thresholds
 
   if (tid < 32) cells[tid] = p.cells[tid];
-  if (p.mode == kRqLloydMax8)
+  if constexpr (MODE == kRqLloydMax8)
     for (int k = tid; k < 256; k += blockDim.x) s_thr8[k] = __ldg(p.thr8 + k);
   if (tid == 0) {
     for (int b = 0; b < 2; ++b) dev::mbar_init(dev::smem_u32(&bars[b]), 1);
@@ -762,8 +767,8 @@ __global__ void __launch_bounds__(256, 2) k_rotate_quant_pair(const RqParams p) 
     for (int b = 0; b < 2; ++b)
       if ((int64_t)blockIdx.x + (int64_t)b * G < NP) issue(b, (int64_t)blockIdx.x + (int64_t)b * G);
 
-  const bool lm8 = p.mode == kRqLloydMax8;
-  const bool lm = p.mode == kRqLloydMax || lm8;   // RMS scale
+  constexpr bool lm8 = MODE == kRqLloydMax8;
+  constexpr bool lm = MODE == kRqLloydMax || lm8;   // RMS scale
   const float nrm = p.inv_norm;
   int it = 0;
   bool aborted = false;
@@ -786,6 +791,15 @@ __global__ void __launch_bounds__(256, 2) k_rotate_quant_pair(const RqParams p) 
         t0[4 * i] = w.x; t0[4 * i + 1] = w.y; t0[4 * i + 2] = w.z; t0[4 * i + 3] = w.w;
       }
     }
+    // the interleave's sign masks and word offsets (L1-resident), also before the wait
+    uint4 mks[4], sl0[4], sl1[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int c = active ? tid + m * nact : 0;
+      mks[m] = __ldg(p.smask + c);
+      sl0[m] = __ldg(p.slot + c);
+      sl1[m] = __ldg(p.slot + d / 8 + c);
+    }
     int fail = !dev::mbar_wait(dev::smem_u32(&bars[b]), (uint32_t)(it >> 1) & 1u, p.err,
                                kSiteRqRow, p.limit_ns);
 
@@ -801,8 +815,7 @@ __global__ void __launch_bounds__(256, 2) k_rotate_quant_pair(const RqParams p) 
       for (int m = 0; m < 4; ++m) {
         const int c = tid + m * nact;
         uint4 a = ra[c], bb = rb[c];
-        const uint4 mk = __ldg(p.smask + c);
-        const uint4 s0 = __ldg(p.slot + c), s1 = __ldg(p.slot + d / 8 + c);
+        const uint4 mk = mks[m], s0 = sl0[m], s1 = sl1[m];
         if (p.want_sum) psum = __fadd2_rn(psum, chunk_sums(a, bb));
         a.x ^= mk.x; a.y ^= mk.y; a.z ^= mk.z; a.w ^= mk.w;
         bb.x ^= mk.x; bb.y ^= mk.y; bb.z ^= mk.z; bb.w ^= mk.w;
@@ -889,8 +902,8 @@ __global__ void __launch_bounds__(256, 2) k_rotate_quant_pair(const RqParams p) 
 
     // ---- per-token statistics --------------------------------------------------------------
     float2 st = make_float2(0.f, 0.f);
-    const bool pct = p.mode == kRqPercentile;
-    if (pct) {
+    constexpr bool pct = MODE == kRqPercentile;
+    if constexpr (pct) {
       switch (p.pct_r) {
         case 2: pct_warp_lists<2>(v, active, lane, warp, pct_lists); break;
         case 3: pct_warp_lists<3>(v, active, lane, warp, pct_lists); break;
@@ -898,7 +911,7 @@ __global__ void __launch_bounds__(256, 2) k_rotate_quant_pair(const RqParams p) 
         case 5: pct_warp_lists<5>(v, active, lane, warp, pct_lists); break;
         default: pct_warp_lists<6>(v, active, lane, warp, pct_lists); break;
       }
-    } else if (lm) {
+    } else if constexpr (lm) {
 #pragma unroll
       for (int i = 0; i < EP; ++i) st = __ffma2_rn(v[i], v[i], st);
       st = warp_sum_pair(st);
@@ -916,7 +929,7 @@ __global__ void __launch_bounds__(256, 2) k_rotate_quant_pair(const RqParams p) 
     // every thread is past its reads of landing buffer b (rows and transpose tiles): refill it
     if (tid == 0 && q + 2 * G < NP) issue(b, q + 2 * G);
     st = make_float2(0.f, 0.f);
-    if (pct) {
+    if constexpr (pct) {
       switch (p.pct_r) {
         case 2: st = pct_quantiles<2>(pct_lists, nwarps, lane, p.pct_frac); break;
         case 3: st = pct_quantiles<3>(pct_lists, nwarps, lane, p.pct_frac); break;
@@ -947,12 +960,12 @@ __global__ void __launch_bounds__(256, 2) k_rotate_quant_pair(const RqParams p) 
 
     // ---- quantize + store ------------------------------------------------------------------
     uint8_t* codes = reinterpret_cast<uint8_t*>(p.codes);
-    if (lm) {
+    if constexpr (lm) {
       const float sa = fmaxf(sqrtf(st.x * nrm * nrm / (float)d), 1e-10f);
       const float sb = fmaxf(sqrtf(st.y * nrm * nrm / (float)d), 1e-10f);
       const float2 mult = make_float2(nrm * __frcp_rn(sa), nrm * __frcp_rn(sb));
       if (tid == 0) { p.scale[ta] = sa; if (has_b) p.scale[ta + 1] = sb; }
-      if (active && lm8) {
+      if (lm8 && active) {
         // 8-bit codes: the number of the 255 thresholds below u, by binary search in shared
         // memory; one byte per code, 32 consecutive codes per thread and token
         uint32_t wa[8], wb[8];
@@ -991,7 +1004,7 @@ __global__ void __launch_bounds__(256, 2) k_rotate_quant_pair(const RqParams p) 
               make_uint4(pb[0], pb[1], pb[2], pb[3]);
       }
     } else {
-      const float qmax = (p.mode == kRqInt8) ? 127.f : 7.f;
+      constexpr float qmax = (MODE == kRqInt8) ? 127.f : 7.f;
       // range: absmax, or gamma * sigma_hat for the percentile scale (its quantile times
       // gamma / Phi^-1((1 + rho) / 2)); both floored at eps
       const float rs = pct ? p.pct_mult : 1.f;
@@ -1010,13 +1023,13 @@ __global__ void __launch_bounds__(256, 2) k_rotate_quant_pair(const RqParams p) 
           float2 r1 = __ffma2_rn(v[4 * k + 1], mult, magic);
           float2 r2 = __ffma2_rn(v[4 * k + 2], mult, magic);
           float2 r3 = __ffma2_rn(v[4 * k + 3], mult, magic);
-          if (pct) {
+          if constexpr (pct) {
             r0 = clamp_code(r0); r1 = clamp_code(r1); r2 = clamp_code(r2); r3 = clamp_code(r3);
           }
           wa[k] = pack4(r0.x, r1.x, r2.x, r3.x);
           wb[k] = pack4(r0.y, r1.y, r2.y, r3.y);
         }
-        if (p.mode == kRqInt8) {
+        if constexpr (MODE == kRqInt8) {
           uint4* da = reinterpret_cast<uint4*>(codes + ta * (int64_t)d + base);
           da[0] = make_uint4(wa[0], wa[1], wa[2], wa[3]);
           da[1] = make_uint4(wa[4], wa[5], wa[6], wa[7]);
@@ -1025,7 +1038,7 @@ __global__ void __launch_bounds__(256, 2) k_rotate_quant_pair(const RqParams p) 
             db[0] = make_uint4(wb[0], wb[1], wb[2], wb[3]);
             db[1] = make_uint4(wb[4], wb[5], wb[6], wb[7]);
           }
-        } else if (p.wlayout) {
+        } else if constexpr (MODE == kPairInt4W) {
           *reinterpret_cast<uint4*>(codes + ta * (int64_t)(d / 2) + base / 2) = gemm_layout4(wa);
           if (has_b)
             *reinterpret_cast<uint4*>(codes + (ta + 1) * (int64_t)(d / 2) + base / 2) =
@@ -1089,24 +1102,31 @@ void* pick_kernel(int hlog2, bool big, int rounds) {
 }
 
 template <int HL, int R>
-void* kern_pair() {
-  return reinterpret_cast<void*>(&k_rotate_quant_pair<HL, R>);
+void* kern_pair(int mode) {
+  switch (mode) {
+    case kRqInt8: return reinterpret_cast<void*>(&k_rotate_quant_pair<HL, R, kRqInt8>);
+    case kRqInt4: return reinterpret_cast<void*>(&k_rotate_quant_pair<HL, R, kRqInt4>);
+    case kRqLloydMax: return reinterpret_cast<void*>(&k_rotate_quant_pair<HL, R, kRqLloydMax>);
+    case kRqPercentile: return reinterpret_cast<void*>(&k_rotate_quant_pair<HL, R, kRqPercentile>);
+    case kRqLloydMax8: return reinterpret_cast<void*>(&k_rotate_quant_pair<HL, R, kRqLloydMax8>);
+    default: return reinterpret_cast<void*>(&k_rotate_quant_pair<HL, R, kPairInt4W>);
+  }
 }
 
 template <int R>
-void* kern_pair_h(int hlog2) {
+void* kern_pair_h(int hlog2, int mode) {
   switch (hlog2) {
-    case 0: return kern_pair<0, R>();
-    case 1: return kern_pair<1, R>();
-    case 2: return kern_pair<2, R>();
-    case 3: return kern_pair<3, R>();
-    case 4: return kern_pair<4, R>();
-    case 5: return kern_pair<5, R>();
-    case 6: return kern_pair<6, R>();
-    case 7: return kern_pair<7, R>();
-    case 8: return kern_pair<8, R>();
-    case 9: return kern_pair<9, R>();
-    default: return kern_pair<10, R>();
+    case 0: return kern_pair<0, R>(mode);
+    case 1: return kern_pair<1, R>(mode);
+    case 2: return kern_pair<2, R>(mode);
+    case 3: return kern_pair<3, R>(mode);
+    case 4: return kern_pair<4, R>(mode);
+    case 5: return kern_pair<5, R>(mode);
+    case 6: return kern_pair<6, R>(mode);
+    case 7: return kern_pair<7, R>(mode);
+    case 8: return kern_pair<8, R>(mode);
+    case 9: return kern_pair<9, R>(mode);
+    default: return kern_pair<10, R>(mode);
   }
 }
 
@@ -1165,14 +1185,15 @@ oq_status launch_rotate_quant(const RqArgs& a, cudaStream_t s) {
   cudaError_t ce = cudaGetDevice(&dev_id);
   if (ce != cudaSuccess) return cuda_fail(ce, "cudaGetDevice");
 
-  // launch shape per (device, d, h mode, rounds, 8-bit Lloyd-Max), computed once
+  // launch shape per (device, d, h, rounds, quantizer), computed once
   static std::mutex mu;
   static std::map<std::tuple<int, int, int, int, int>, LaunchCfg> cache;
   const int lm8 = a.mode == kRqLloydMax8 ? 1 : 0;
+  const int pmode = (a.mode == kRqInt4 && a.wlayout) ? kPairInt4W : a.mode;
   LaunchCfg cfg;
   {
     std::lock_guard<std::mutex> lock(mu);
-    auto key = std::make_tuple(dev_id, a.d, hlog2, a.rounds, lm8);
+    auto key = std::make_tuple(dev_id, a.d, hlog2, a.rounds, pmode);
     auto itc = cache.find(key);
     if (itc != cache.end()) {
       cfg = itc->second;
@@ -1186,7 +1207,7 @@ oq_status launch_rotate_quant(const RqArgs& a, cudaStream_t s) {
         // tiles), the interleaved words, the round buffer, then reductions + code cells +
         // barriers + percentile lists and, for 8-bit Lloyd-Max codes only, the 256 thresholds
         cfg.pair = 1;
-        cfg.fn = a.rounds == 1 ? kern_pair_h<1>(hlog2) : kern_pair_h<2>(hlog2);
+        cfg.fn = a.rounds == 1 ? kern_pair_h<1>(hlog2, pmode) : kern_pair_h<2>(hlog2, pmode);
         cfg.nthr = nthr;
         ce = allow_max_dynamic_smem(cfg.fn);
         if (ce != cudaSuccess) return cuda_fail(ce, "cudaFuncSetAttribute(rotate_quant)");
