@@ -505,6 +505,8 @@ __global__ void __launch_bounds__(MAXT, 1) k_rotate_quant(const RqParams p) {
 
 // the two-token kernel's extra quantizer instantiation: 4-bit absmax codes in the GEMM layout
 constexpr int kPairInt4W = 5;
+// landing buffers of the two-token kernel (row pairs in flight per CTA)
+constexpr int kPairNbuf = 2;
 
 template <int BIT>
 __device__ __forceinline__ void stage_pair(float2 (&v)[EP]) {
@@ -727,13 +729,13 @@ __global__ void __launch_bounds__(256, 2) k_rotate_quant_pair(const RqParams p) 
   const uint32_t row_bytes = (uint32_t)d * 2u;
   const uint32_t row_stride = (row_bytes + 127u) & ~127u;
   const size_t land_bytes = (size_t)p.land_bytes;
-  // [two landing buffers: a pair of rows (A | B) each; while a pass runs, its own buffer also
+  // [kPairNbuf landing buffers: a pair of rows (A | B) each; while a pass runs, its own buffer also
   //  holds the warps' transpose tiles (h >= 256), so no barrier separates a warp's gather from
   //  its transposes] [interleaved words, bank-aware layout: nwarps x 4 KB]
   // [round buffer, two rounds only] [reductions, code cells, barriers, percentile lists,
   //  8-bit Lloyd-Max thresholds]
   uint8_t* land = smem;
-  uint8_t* wbuf = smem + 2 * land_bytes;
+  uint8_t* wbuf = smem + kPairNbuf * land_bytes;
   float2* rbuf = reinterpret_cast<float2*>(wbuf + nwarps * 4096);
   float* red = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(rbuf) +
                                         (ROUNDS == 2 ? nwarps * 8192 : 0));
@@ -747,7 +749,7 @@ __global__ void __launch_bounds__(256, 2) k_rotate_quant_pair(const RqParams p) 
   if constexpr (MODE == kRqLloydMax8)
     for (int k = tid; k < 256; k += blockDim.x) s_thr8[k] = __ldg(p.thr8 + k);
   if (tid == 0) {
-    for (int b = 0; b < 2; ++b) dev::mbar_init(dev::smem_u32(&bars[b]), 1);
+    for (int b = 0; b < kPairNbuf; ++b) dev::mbar_init(dev::smem_u32(&bars[b]), 1);
     dev::fence_mbar_init();
   }
   __syncthreads();
@@ -764,7 +766,7 @@ __global__ void __launch_bounds__(256, 2) k_rotate_quant_pair(const RqParams p) 
     dev::bulk_g2s(dev::smem_u32(dst + row_stride), p.x + tb * p.ldx, row_bytes, bar);
   };
   if (tid == 0)
-    for (int b = 0; b < 2; ++b)
+    for (int b = 0; b < kPairNbuf; ++b)
       if ((int64_t)blockIdx.x + (int64_t)b * G < NP) issue(b, (int64_t)blockIdx.x + (int64_t)b * G);
 
   constexpr bool lm8 = MODE == kRqLloydMax8;
@@ -773,7 +775,7 @@ __global__ void __launch_bounds__(256, 2) k_rotate_quant_pair(const RqParams p) 
   int it = 0;
   bool aborted = false;
   for (int64_t q = blockIdx.x; q < NP; q += G, ++it) {
-    const int b = it & 1;
+    const int b = it % kPairNbuf;
     uint8_t* lb = land + (size_t)b * land_bytes;
     float* warp_tile = reinterpret_cast<float*>(lb) + warp * 1024;
     const int64_t ta = 2 * q;
@@ -800,7 +802,7 @@ __global__ void __launch_bounds__(256, 2) k_rotate_quant_pair(const RqParams p) 
       sl0[m] = __ldg(p.slot + c);
       sl1[m] = __ldg(p.slot + d / 8 + c);
     }
-    int fail = !dev::mbar_wait(dev::smem_u32(&bars[b]), (uint32_t)(it >> 1) & 1u, p.err,
+    int fail = !dev::mbar_wait(dev::smem_u32(&bars[b]), (uint32_t)(it / kPairNbuf) & 1u, p.err,
                                kSiteRqRow, p.limit_ns);
 
     // ---- source-side signs, interleave A|B into the bank-aware word layout, row sums ------
@@ -927,7 +929,7 @@ __global__ void __launch_bounds__(256, 2) k_rotate_quant_pair(const RqParams p) 
     if (lane == 0 && !pct) { red[16 + 2 * warp] = st.x; red[16 + 2 * warp + 1] = st.y; }
     __syncthreads();
     // every thread is past its reads of landing buffer b (rows and transpose tiles): refill it
-    if (tid == 0 && q + 2 * G < NP) issue(b, q + 2 * G);
+    if (tid == 0 && q + kPairNbuf * G < NP) issue(b, q + kPairNbuf * G);
     st = make_float2(0.f, 0.f);
     if constexpr (pct) {
       switch (p.pct_r) {
@@ -1059,11 +1061,11 @@ __global__ void __launch_bounds__(256, 2) k_rotate_quant_pair(const RqParams p) 
   // After an abort, wait (bounded) for the row loads this CTA still has in flight, so that no
   // bulk copy lands in shared memory after the block has exited.
   if (aborted && tid == 0) {
-    for (int k = 0; k < 2; ++k) {
+    for (int k = 0; k < kPairNbuf; ++k) {
       const int j = it + k;
       if ((int64_t)blockIdx.x + (int64_t)j * G >= NP) break;
-      dev::mbar_wait(dev::smem_u32(&bars[j & 1]), (uint32_t)(j >> 1) & 1u, p.err, kSiteRqDrain,
-                     p.limit_ns);
+      dev::mbar_wait(dev::smem_u32(&bars[j % kPairNbuf]), (uint32_t)(j / kPairNbuf) & 1u, p.err,
+                     kSiteRqDrain, p.limit_ns);
     }
   }
 }
@@ -1211,12 +1213,12 @@ oq_status launch_rotate_quant(const RqArgs& a, cudaStream_t s) {
         cfg.nthr = nthr;
         ce = allow_max_dynamic_smem(cfg.fn);
         if (ce != cudaSuccess) return cuda_fail(ce, "cudaFuncSetAttribute(rotate_quant)");
-        cfg.nbuf = 2;
+        cfg.nbuf = kPairNbuf;
         const size_t nw = (size_t)(nthr / 32);
         size_t land = 2 * row_stride;
         if (hmode == 2) land = std::max(land, nw * 4096);
         cfg.land_bytes = (int)((land + 127) & ~(size_t)127);
-        cfg.smem = 2 * (size_t)cfg.land_bytes + nw * 4096 + (a.rounds == 2 ? nw * 8192 : 0) +
+        cfg.smem = kPairNbuf * (size_t)cfg.land_bytes + nw * 4096 + (a.rounds == 2 ? nw * 8192 : 0) +
                    (size_t)(224 + (lm8 ? 256 : 0)) * 4;
         int best_occ = 0;
         ce = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&best_occ, cfg.fn, nthr, cfg.smem);
