@@ -506,7 +506,7 @@ __global__ void __launch_bounds__(MAXT, 1) k_rotate_quant(const RqParams p) {
 // the two-token kernel's extra quantizer instantiation: 4-bit absmax codes in the GEMM layout
 constexpr int kPairInt4W = 5;
 // landing buffers of the two-token kernel (row pairs in flight per CTA)
-constexpr int kPairNbuf = 2;
+constexpr int kPairNbuf = 1;
 
 template <int BIT>
 __device__ __forceinline__ void stage_pair(float2 (&v)[EP]) {
