@@ -15,10 +15,13 @@ runs its own batch with no collective on the data path (weak scaling); the only 
 are the barriers around the timed region and the max-over-ranks of the time.
 
 Timing: CUDA events on the launching stream over exactly K steps, a barrier and a
-synchronize on both sides. Inputs rotate over 4 independent sets (about 270 MB, more than
-the 126 MB L2), so no step reads data a previous step left in L2. Per-kernel durations
-come from events recorded between the two launches of every timed step. nvidia-smi
-samples the SM clock and throttle reasons during the timed region.
+synchronize on both sides. The steps replay CUDA graphs of the library's launches (one graph
+of four steps, plus single steps for a remainder), so that no host-side launch gap falls
+between kernels. Inputs rotate over 4 independent sets (about 270 MB, more than the 126 MB
+L2), so no step reads data a previous step left in L2. Per-kernel durations come from graphs
+of each kernel alone over the same sets. The GEMM's roofline peak is the library's tcgen05
+peak loop for the GEMM's MMA kind, measured in the same run. nvidia-smi samples the SM clock
+and throttle reasons during the timed region.
 """
 from __future__ import annotations
 
@@ -38,7 +41,8 @@ sys.path.insert(0, ROOT)
 
 METRIC = "rotate+quantize GB/s (% of HBM peak); W4A8/W4A4 linear TOPS (% tensor peak)"
 RING = 4
-# nominal dense int8 / bf16 tensor throughput ratio on B200 (4.5 / 2.25 PFLOP/s)
+# nominal dense int8 / bf16 tensor throughput ratio on B200 (4.5 / 2.25 PFLOP/s), for the
+# peak the measured bf16 GEMM figure implies (reported beside the measured tcgen05 peak)
 INT8_PER_BF16 = 2.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -324,6 +328,29 @@ def run_sweep(args):
     return 0
 
 
+def measured_mma_peak(oq, kind, stream, iters=1 << 13, reps=3):
+    """(TOPS or TFLOP/s, ms) of the library's tcgen05 peak loop for `kind` ("i8" or "f16"),
+    best of `reps` launches timed with CUDA events on `stream`."""
+    import torch
+    k_per = 32 if kind == "i8" else 16
+    pairs = oq.mma_peak_loop(kind, iters, stream=stream)
+    best = None
+    for _ in range(reps):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        oq.mma_peak_loop(kind, iters, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1)
+        best = ms if best is None else min(best, ms)
+    st, code = oq.device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} code {code:#x} in the peak loop")
+    ops = pairs * iters * 4 * 2.0 * 256 * 256 * k_per
+    return ops / (best * 1e-3) / 1e12, best
+
+
 def run_peaks(args):
     """Dense tensor-core peaks of this GPU, each timed with CUDA events on its stream after
     warm-up, best of `reps`:
@@ -455,38 +482,59 @@ def main():
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
 
-    def step(s):
+    def step(s, st):
         oq.rotate_quantize(plan, s["x"], codes=s["codes"], scale=s["scale"], mean=s["mean"],
-                           stream=stream)
+                           stream=st)
 
-    def gemm(s):
+    def gemm(s, st):
         if g64:
             oq.gemm_w4a4_g64(wl.act, s["codes"], s["scale"], s["wp"], s["wsz"], s["ws"],
                              mean=s["mean"], w_rowsum=s["w1"] if wl.center else None, out=s["y"],
-                             stream=stream)
+                             stream=st)
         elif wl.act == "int8_absmax":
             oq.gemm_w4a8(s["codes"], s["scale"], s["wp"], s["ws"], mean=s["mean"],
-                         w_rowsum=s["w1"] if wl.center else None, out=s["y"], stream=stream)
+                         w_rowsum=s["w1"] if wl.center else None, out=s["y"], stream=st)
         elif wl.act == "int8_lloydmax":
             oq.gemm_w4a8_lloydmax(plan, s["codes"], s["scale"], s["wp"], s["ws"], mean=s["mean"],
                                   w_rowsum=s["w1"] if wl.center else None, out=s["y"],
-                                  stream=stream)
+                                  stream=st)
         else:
             oq.gemm_w4a4(plan, wl.act, s["codes"], s["scale"], s["wp"], s["ws"],
                          mean=s["mean"], w_rowsum=s["w1"] if wl.center else None, out=s["y"],
-                         stream=stream)
+                         stream=st)
 
     for i in range(max(3, args.warmup)):
         s = sets[i % RING]
-        step(s)
-        gemm(s)
+        step(s, stream)
+        gemm(s, stream)
     torch.cuda.synchronize()
     st, code = oq.device_status()
     if st != 0:
         raise RuntimeError(f"device status {st} code {code:#x} after warm-up")
 
+    # The timed steps replay CUDA graphs of the library's launches, so that no host-side launch
+    # gap falls between the kernels: g_ring holds the RING steps in order, g_one[r] one step.
+    cap_stream = torch.cuda.Stream(device=dev)
+
+    def capture(calls):
+        g = torch.cuda.CUDAGraph()
+        cap_stream.wait_stream(stream)
+        with torch.cuda.graph(g, stream=cap_stream):
+            cs = torch.cuda.current_stream()
+            for fn, s in calls:
+                fn(s, cs)
+        stream.wait_stream(cap_stream)
+        return g
+
+    g_ring = capture([(f, s) for s in sets for f in (step, gemm)])
+    g_one = [capture([(step, s), (gemm, s)]) for s in sets]
+    g_rq = capture([(step, s) for s in sets])        # the two kernels alone, for their
+    g_gm = capture([(gemm, s) for s in sets])        # average duration per launch
+    for _ in range(2):
+        g_ring.replay()
+    torch.cuda.synchronize()
+
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
     uuid = None
     try:
         uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
@@ -498,19 +546,28 @@ def main():
         t_start = torch.cuda.Event(enable_timing=True)
         t_end = torch.cuda.Event(enable_timing=True)
         t_start.record(stream)
-        for i in range(K):
-            s = sets[i % RING]
-            ev[i][0].record(stream)
-            step(s)
-            ev[i][1].record(stream)
-            gemm(s)
-            ev[i][2].record(stream)
+        for _ in range(K // RING):
+            g_ring.replay()
+        for r in range(K % RING):
+            g_one[r].replay()
         t_end.record(stream)
         torch.cuda.synchronize()
     barrier()
     elapsed_ms = t_start.elapsed_time(t_end)
-    rq_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / K
-    gm_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / K
+
+    def per_launch(g):
+        reps = max(1, -(-K // RING))
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / (reps * RING)
+
+    rq_ms = per_launch(g_rq)
+    gm_ms = per_launch(g_gm)
     st, code = oq.device_status()
     if st != 0:
         raise RuntimeError(f"device status {st} code {code:#x} after timing")
@@ -591,7 +648,11 @@ def main():
     bf16_peak = peaks.get("bf16_tflops_sustained" if long_region else "bf16_tflops",
                           peaks["bf16_tflops"])
     fp_gemm = "lloydmax" in wl.act or g64          # fp16 operands on the tensor cores
-    tensor_peak = bf16_peak * (INT8_PER_BF16 if not fp_gemm else 1.0)
+    rule_peak = bf16_peak * (INT8_PER_BF16 if not fp_gemm else 1.0)
+    # the dense tensor-core peak of this GPU for the GEMM's own MMA kind, measured now by the
+    # library's peak loop (the GEMM's instruction issued back to back on resident operands)
+    loop_kind = "f16" if fp_gemm else "i8"
+    tensor_peak, loop_ms = measured_mma_peak(oq, loop_kind, stream)
     hbm_peak = peaks["hbm_gbs"]
     gemm_tops = ops / (gm_ms * 1e-3) / 1e12
     rq_gbs = rq_bytes / (rq_ms * 1e-3) / 1e9
@@ -601,13 +662,17 @@ def main():
     kfile_rq = os.path.join(ROOT, "w4a8_ptq_linear_b200", "csrc", "k_rotate_quant.cu")
     tr_rq = NCU_TRAFFIC.get((wl.name, "k_rotate_quant"))
     traffic_rq = tr_rq["bytes"] if tr_rq and tr_rq["sha"] == sha_of(kfile_rq) else None
-    peak_note = (f"{peak_kind} {'sustained' if long_region else 'burst'} bf16 "
+    rule_note = (f"{peak_kind} {'sustained' if long_region else 'burst'} bf16 "
                  f"{bf16_peak} TFLOP/s" + (" x 2 (nominal int8/bf16 ratio)"
                                            if not fp_gemm else ""))
+    peak_note = (f"tcgen05 kind::{loop_kind} peak loop measured in this run "
+                 f"(oq_mma_peak_loop, one CTA pair per two SMs, {loop_ms:.3f} ms)")
     gemm_roof = {"bound": "tensor", "achieved": gemm_tops, "peak": tensor_peak,
                  "unit": "TOPS" if not fp_gemm else "TFLOP/s",
                  "frac": gemm_tops / tensor_peak, "traffic": traffic, "kernel": "k_gemm",
-                 "peak_source": peak_note, "ms_per_launch": gm_ms}
+                 "peak_source": peak_note, "ms_per_launch": gm_ms,
+                 "peak_rule": rule_peak, "frac_rule": gemm_tops / rule_peak,
+                 "peak_rule_source": rule_note}
     rq_roof = {"bound": "hbm", "achieved": rq_gbs, "peak": hbm_peak, "unit": "GB/s",
                "frac": rq_gbs / hbm_peak, "traffic": traffic_rq, "kernel": "k_rotate_quant",
                "peak_source": f"{peak_kind} copy bandwidth", "ms_per_launch": rq_ms,
@@ -620,6 +685,7 @@ def main():
         "scaling": "weak", "vs_baseline": None, "dtype": "int8" if not fp_gemm else "f16", "data": "synthetic", "config": config_of(wl, T, world),
         "rotate_quantize_gbs": rq_gbs, "rotate_quantize_frac_hbm": rq_gbs / hbm_peak,
         "gemm_tops": gemm_tops, "gemm_frac_tensor": gemm_tops / tensor_peak,
+        "timing": "steps and per-kernel averages replay CUDA graphs of the library's launches",
         "roofline": dominant, "roofline_other": other,
         "kernel_share": {"k_rotate_quant": rq_ms / (rq_ms + gm_ms),
                          "k_gemm": gm_ms / (rq_ms + gm_ms)},
