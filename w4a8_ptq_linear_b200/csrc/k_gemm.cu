@@ -914,7 +914,7 @@ int sm_count() {
 
 // Clusters of two CTAs that can be resident at once for a kernel and its shared memory (0 if
 // the query fails), computed once per kernel and device.
-int active_pairs(const void* kern, size_t smem) {
+int active_pairs_n(const void* kern, size_t smem, int nthreads) {
   static std::mutex mu;
   static std::map<std::pair<const void*, int>, int> cache;
   int dev = 0;
@@ -924,7 +924,7 @@ int active_pairs(const void* kern, size_t smem) {
   if (it != cache.end()) return it->second;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(2 * (unsigned)sm_count());
-  cfg.blockDim = dim3(NTHREADS);
+  cfg.blockDim = dim3((unsigned)nthreads);
   cfg.dynamicSmemBytes = smem;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -941,6 +941,8 @@ int active_pairs(const void* kern, size_t smem) {
   cache[{kern, dev}] = n;
   return n;
 }
+
+int active_pairs(const void* kern, size_t smem) { return active_pairs_n(kern, smem, NTHREADS); }
 
 template <int KIND, int CG>
 oq_status run(const GemmArgs& g, const GemmParams& p, cudaStream_t s) {
@@ -996,6 +998,426 @@ oq_status run(const GemmArgs& g, const GemmParams& p, cudaStream_t s) {
   return OQ_OK;
 }
 
+// ================================================================================================
+// W4A8 with the widened weights in tensor memory (CTA pairs, T > 128).
+//
+// The weight operand is the MMA's A; tcgen05.mma reads A from tensor memory as well as from
+// shared memory. Here the converter warps widen each 128-byte K block of their CTA's 128 weight
+// rows in registers (one row per thread: the thread's TMEM lane) and store it with tcgen05.st
+// into one of SA weight stages in TMEM, so the widened weights never pass through shared memory:
+// per K block and SM, shared memory carries only the packed weights (TMA write + converter read,
+// 16 KB) and the activations (TMA write + MMA read, 2 x 12 KB). TMEM holds two accumulators of
+// BN = 192 columns and SA = 4 weight stages of 32 columns (4 int8 per column): 512 columns.
+//
+// Schedule: the work is the flattened (channel tile, 32-token chunk) space; every CTA pair takes
+// an equal contiguous range of it and cuts its range, within each channel tile, into tiles of
+// at most BN tokens, as even as possible. All pairs then carry the same MMA work (within one
+// chunk), with no partial last wave.
+//
+// Warps: 0 packed-weight producer, 1 TMEM owner + MMA issuer, 2 activation producer, 3 idle,
+// 4-11 converters in two groups (warps 4-7 and 8-11, each covering the four TMEM lane quarters)
+// that take alternate K blocks, 12-19 epilogue (two per lane quarter).
+namespace ta {
+constexpr int BN = 192;              // tokens per tile at most (MMA N)
+constexpr int MAXCH = BN / CH;       // 32-token chunks per tile at most
+constexpr int XR = BN / 2;           // activation rows per CTA and stage
+constexpr int SX = 6;                // activation ring
+constexpr int SP = 8;                // packed weight ring
+constexpr int SA = 4;                // widened weight stages in TMEM
+constexpr int ACOL = 2 * BN;         // TMEM column of weight stage 0
+constexpr int TCOLS = 512;           // TMEM columns allocated
+constexpr int XT = XR * 128;         // activation stage bytes (128-byte swizzled rows)
+constexpr int WP = BM * 64;          // packed weight stage bytes (64-byte swizzled rows)
+constexpr int STG = 32 * 32 * 2;     // bf16 [32 tokens][32 channels] staging tile per warp
+// (NEPI = 256 epilogue threads, EPW = 2 per lane quarter, as in k_gemm)
+constexpr int OFF_X = 0;
+constexpr int OFF_P = OFF_X + SX * XT;
+constexpr int OFF_STG = OFF_P + SP * WP;
+constexpr int OFF_TOK = OFF_STG + (NEPI / 32) * STG;
+constexpr int OFF_BAR = OFF_TOK + BN * 8;
+constexpr int NBAR = 2 * SX + 2 * SP + 2 * SA + 4 + 1;
+constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+constexpr int SMEM = OFF_MISC + 16 + 1024;
+constexpr int NTHR = 640;
+constexpr int W_PROD_P = 0, W_MMA = 1, W_PROD_X = 2, W_CONV0 = 4, W_EPI0 = 12;
+static_assert(ACOL + SA * 32 <= TCOLS, "tensor memory budget");
+static_assert(XT % 1024 == 0 && OFF_P % 1024 == 0 && WP % 1024 == 0, "stage alignment");
+static_assert(SMEM <= 232448, "shared memory");
+static_assert(NTHR == (W_EPI0 * 32 + NEPI), "warp roles");
+
+// The tiles of one CTA pair: an equal share of the (channel tile, chunk) space, cut at channel
+// tile boundaries and into as-even-as-possible tiles of at most MAXCH chunks. Every role of the
+// pair walks the same sequence.
+struct RangeIter {
+  int cpm, cur, end;
+  __device__ RangeIter(int T, int n_o, int unit, int n_units) {
+    cpm = (T + CH - 1) / CH;
+    const long long total = (long long)n_o * cpm;
+    cur = (int)(total * unit / n_units);
+    end = (int)(total * (unit + 1) / n_units);
+  }
+  __device__ bool next(int& m, int& t0, int& nch) {
+    if (cur >= end) return false;
+    m = cur / cpm;
+    const int tc = cur - m * cpm;
+    const int run = min(end, (m + 1) * cpm) - cur;     // chunks left in this channel tile
+    const int ntiles = (run + MAXCH - 1) / MAXCH;
+    nch = (run + ntiles - 1) / ntiles;
+    t0 = tc * CH;
+    cur += nch;
+    return true;
+  }
+};
+}  // namespace ta
+
+__global__ void __launch_bounds__(ta::NTHR, 1)
+    k_gemm_a8t(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+               const __grid_constant__ CUtensorMap tm_y, const GemmParams p) {
+  using namespace ta;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  float2* s_tok = reinterpret_cast<float2*>(smem + OFF_TOK);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint32_t* s_misc = reinterpret_cast<uint32_t*>(smem + OFF_MISC);  // tmem, abort, epi flag
+  volatile uint32_t* s_abort = s_misc + 1;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = dev::cluster_ctarank();   // 0 = the pair's leader
+  constexpr int UNIT = 2 * BM;                     // channels per tile
+  const int n_o = (p.N + UNIT - 1) / UNIT;
+  const int nkb = (p.K + 127) / 128;
+  const int unit_index = (int)blockIdx.x / 2, n_units = (int)gridDim.x / 2;
+  auto tiles = [&]() { return RangeIter(p.T, n_o, unit_index, n_units); };
+
+  auto bar = [&](int i) { return dev::smem_u32(&bars[i]); };
+  auto xfull_bar = [&](int s) { return bar(s); };
+  auto xempty_bar = [&](int s) { return bar(SX + s); };
+  auto pfull_bar = [&](int s) { return bar(2 * SX + s); };
+  auto pempty_bar = [&](int s) { return bar(2 * SX + SP + s); };
+  auto wready_bar = [&](int c) { return bar(2 * SX + 2 * SP + c); };
+  auto wfree_bar = [&](int c) { return bar(2 * SX + 2 * SP + SA + c); };
+  auto tfull_bar = [&](int b) { return bar(2 * SX + 2 * SP + 2 * SA + b); };
+  auto tempty_bar = [&](int b) { return bar(2 * SX + 2 * SP + 2 * SA + 2 + b); };
+  const uint32_t drain_bar = bar(2 * SX + 2 * SP + 2 * SA + 4);
+  auto x_stage = [&](int s) { return smem + OFF_X + s * XT; };
+  auto p_stage = [&](int s) { return smem + OFF_P + s * WP; };
+  auto lead = [&](uint32_t a) { return dev::map_to_cta(a, 0); };
+
+  if (tid == 0) {
+    for (int s = 0; s < SX; ++s) {
+      dev::mbar_init(xfull_bar(s), 1);
+      dev::mbar_init(xempty_bar(s), 1);
+    }
+    for (int s = 0; s < SP; ++s) {
+      dev::mbar_init(pfull_bar(s), 1);
+      dev::mbar_init(pempty_bar(s), 4);      // the four warps of the converting group
+    }
+    for (int c = 0; c < SA; ++c) {
+      dev::mbar_init(wready_bar(c), 2 * 4);  // four converter warps of each CTA
+      dev::mbar_init(wfree_bar(c), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      dev::mbar_init(tfull_bar(b), 1);
+      dev::mbar_init(tempty_bar(b), 2 * (NEPI / 32));
+    }
+    dev::mbar_init(drain_bar, 1);
+    s_misc[1] = 0;
+    dev::fence_mbar_init_cluster();
+  }
+  if (warp == W_PROD_P && lane == 0) {
+    dev::prefetch_tmap(&tm_x);
+    dev::prefetch_tmap(&tm_w);
+  }
+  if (warp == W_EPI0 && lane == 0 && !p.out_acc) dev::prefetch_tmap(&tm_y);
+  if (warp == W_MMA) {
+    dev::tmem_alloc_pair(dev::smem_u32(&s_misc[0]), TCOLS);
+    dev::tmem_relinquish_pair();
+  }
+  dev::tc_fence_before();
+  dev::cluster_sync();   // barrier inits of both CTAs visible before any remote arrive
+  dev::tc_fence_after();
+  const uint32_t tmem = s_misc[0];
+  auto give_up = [&]() { *s_abort = 1; };
+
+  if (warp == W_PROD_P || warp == W_PROD_X) {
+    // ---------------- producers ----------------
+    const bool packed_role = warp == W_PROD_P;
+    if (lane == 0) {
+      const int ns = packed_role ? SP : SX;
+      uint32_t j = 0;
+      bool ok = true;
+      auto it = tiles();
+      int m, t0, nch;
+      while (ok && it.next(m, t0, nch)) {
+        const int o0 = m * UNIT + (int)rank * BM;            // this CTA's weight rows
+        const int x0 = t0 + (int)rank * (nch * CH / 2);      // this CTA's activation rows
+        const int krot = k_rotation(m, nkb);
+        for (int step = 0; step < nkb; ++step, ++j) {
+          const int kb = (step + krot) % nkb;
+          const int s = j % ns;
+          const uint32_t empty_b = packed_role ? pempty_bar(s) : xempty_bar(s);
+          const uint32_t full_b = packed_role ? pfull_bar(s) : xfull_bar(s);
+          if (*s_abort || !dev::mbar_wait(empty_b, ((j / ns) & 1u) ^ 1u, p.err, kSiteGemmEmpty,
+                                          p.limit_ns)) {
+            give_up();
+            ok = false;
+            break;
+          }
+          if (packed_role) {
+            dev::mbar_arrive_expect_tx(full_b, (uint32_t)WP);
+            dev::tma_load_2d(dev::smem_u32(p_stage(s)), &tm_w, kb * 64, o0, full_b);
+          } else {
+            // both halves complete on the leader's barrier, which expects the bytes of both
+            if (rank == 0) dev::mbar_arrive_expect_tx(full_b, (uint32_t)(2 * XT));
+            dev::tma_load_2d_pair(dev::smem_u32(x_stage(s)), &tm_x, kb * 128, x0, lead(full_b));
+          }
+        }
+      }
+      if (!ok && (packed_role || rank == 0)) {
+        for (uint32_t i = (j >= (uint32_t)ns ? j - ns : 0); i < j; ++i)
+          dev::mbar_wait(packed_role ? pfull_bar(i % ns) : xfull_bar(i % ns), (i / ns) & 1u, p.err,
+                         kSiteGemmDrain, p.limit_ns);
+      }
+    }
+  } else if (warp == W_MMA) {
+    // ---------------- MMA issuer (the leader's lane 0) ----------------
+    if (lane == 0 && rank == 0) {
+      uint32_t j = 0, it_n = 0;
+      bool ok = true, issued = false;
+      auto it = tiles();
+      int m, t0, nch;
+      for (; ok && it.next(m, t0, nch); ++it_n) {
+        const uint32_t idesc = dev::idesc_i8(UNIT, nch * CH);
+        const int b = it_n & 1;
+        if (*s_abort || !dev::mbar_wait(tempty_bar(b), ((it_n >> 1) & 1u) ^ 1u, p.err,
+                                        kSiteGemmAccum, p.limit_ns)) {
+          give_up();
+          ok = false;
+          break;
+        }
+        dev::tc_fence_after();
+        const uint32_t dt = tmem + (uint32_t)(b * BN);
+        for (int step = 0; step < nkb; ++step, ++j) {
+          const int c = j % SA, sx = j % SX;
+          bool w = !*s_abort &&
+                   dev::mbar_wait(wready_bar(c), (j / SA) & 1u, p.err, kSiteGemmConv, p.limit_ns);
+          if (w) w = dev::mbar_wait(xfull_bar(sx), (j / SX) & 1u, p.err, kSiteGemmFull, p.limit_ns);
+          if (!w) {
+            give_up();
+            ok = false;
+            break;
+          }
+          dev::tc_fence_after();
+          const uint32_t at = tmem + (uint32_t)(ACOL + c * 32);
+          const uint32_t bx = dev::smem_u32(x_stage(sx));
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            dev::mma_i8_pair_ta(dt, at + kk * 8, dev::sdesc_sw128(bx + kk * 32), idesc,
+                                (step | kk) != 0);
+          issued = true;
+          dev::mma_commit_pair(wfree_bar(c));
+          dev::mma_commit_pair(xempty_bar(sx));
+        }
+        if (!ok) break;
+        dev::mma_commit_pair(tfull_bar(b));
+      }
+      if (!ok && issued) {  // wait for the MMAs in flight before TMEM is freed
+        dev::mma_commit_pair(drain_bar);
+        dev::mbar_wait(drain_bar, 0, p.err, kSiteGemmDrain, p.limit_ns);
+      }
+    }
+  } else if (warp >= W_CONV0 && warp < W_EPI0) {
+    // ---------------- converters: packed weights -> int8 16 n -> TMEM ----------------
+    // Thread (quarter q, lane l) owns weight row r = 32 q + l, i.e. TMEM lane r. The packed
+    // stage holds 64-byte rows whose four 16-byte groups were swizzled by TMA (group g of row r
+    // at ((g ^ ((r >> 1) & 3)) << 4)), so that the warp's row-wise reads hit distinct banks.
+    // Group g (32 elements) widens to columns 8g..8g+3 (low nibbles, elements 32g..32g+15) and
+    // 8g+4..8g+7 (high nibbles, elements 32g+16..32g+31).
+    const int grp = (warp - W_CONV0) >> 2, q = warp & 3;
+    const int r = q * 32 + lane;
+    const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
+    uint32_t j = 0;
+    bool ok = true;
+    auto it = tiles();
+    int m, t0, nch;
+    while (ok && it.next(m, t0, nch)) {
+      for (int step = 0; step < nkb; ++step, ++j) {
+        if ((int)(j & 1u) != grp) continue;
+        const int s = j % SP, c = j % SA;
+        bool w = !*s_abort &&
+                 dev::mbar_wait(pfull_bar(s), (j / SP) & 1u, p.err, kSiteGemmFull, p.limit_ns);
+        if (w)
+          w = dev::mbar_wait(wfree_bar(c), ((j / SA) & 1u) ^ 1u, p.err, kSiteGemmConv, p.limit_ns);
+        w = __all_sync(0xffffffffu, w);
+        if (!w) {
+          give_up();
+          ok = false;
+          break;
+        }
+        const uint8_t* row = p_stage(s) + r * 64;
+        const int ph = (r >> 1) & 3;
+        uint32_t o[32];
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const uint4 in = *reinterpret_cast<const uint4*>(row + ((g ^ ph) << 4));
+          o[8 * g + 0] = (in.x << 4) & 0xF0F0F0F0u;
+          o[8 * g + 1] = (in.y << 4) & 0xF0F0F0F0u;
+          o[8 * g + 2] = (in.z << 4) & 0xF0F0F0F0u;
+          o[8 * g + 3] = (in.w << 4) & 0xF0F0F0F0u;
+          o[8 * g + 4] = in.x & 0xF0F0F0F0u;
+          o[8 * g + 5] = in.y & 0xF0F0F0F0u;
+          o[8 * g + 6] = in.z & 0xF0F0F0F0u;
+          o[8 * g + 7] = in.w & 0xF0F0F0F0u;
+        }
+        __syncwarp();              // the warp's reads of the packed stage are done
+        if (lane == 0) dev::mbar_arrive(pempty_bar(s));
+        dev::tmem_st32(tmem + lane_addr + (uint32_t)(ACOL + c * 32), o);
+        dev::tmem_wait_st();
+        dev::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) dev::mbar_arrive_cluster(lead(wready_bar(c)));
+      }
+    }
+  } else if (warp >= W_EPI0) {
+    // ---------------- epilogue ----------------
+    const int etid = tid - W_EPI0 * 32;
+    uint8_t* stg = smem + OFF_STG + (warp - W_EPI0) * STG;
+    const int q = warp & 3;
+    const int half = (warp - W_EPI0) >> 2;
+    const int o_local = q * 32 + lane;
+    const bool ep_lead = etid == 0;
+    uint32_t it_n = 0;
+    bool ok = true;
+    auto it = tiles();
+    int m, t0, nch;
+    for (; ok && it.next(m, t0, nch); ++it_n) {
+      const int o0 = m * UNIT + (int)rank * BM;
+      const int b = it_n & 1;
+      const int o = o0 + o_local;
+      const bool has_o = o < p.N;
+      const float sw = has_o ? p.w_scale[o] * (1.f / 16.f) : 0.f;
+      const float w1 = (has_o && p.mean) ? p.w_rowsum[o] : 0.f;
+      const float bb = (has_o && p.bias) ? __bfloat162float(p.bias[o]) : 0.f;
+      const int ncols = nch * CH;
+      for (int i = etid; i < ncols; i += NEPI) {
+        const int t = t0 + i;
+        s_tok[i] = make_float2((t < p.T) ? p.a_scale[t] : 0.f,
+                               (t < p.T && p.mean) ? p.mean[t] : 0.f);
+      }
+      if (ep_lead) {
+        const bool ready = !*s_abort && dev::mbar_wait(tfull_bar(b), (it_n >> 1) & 1u, p.err,
+                                                       kSiteGemmAccum, p.limit_ns);
+        if (!ready) give_up();
+        s_misc[2] = ready ? 1u : 0u;
+      }
+      dev::named_bar(1, NEPI);
+      ok = *reinterpret_cast<volatile uint32_t*>(&s_misc[2]) != 0;
+      if (ok) dev::tc_fence_after();
+      const int t_end = min(ncols, p.T - t0);
+      const int nmine = (nch - half + EPW - 1) / EPW;
+      if (ok && nmine == 0) {
+        dev::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) dev::mbar_arrive_cluster(lead(tempty_bar(b)));
+      }
+#pragma unroll 1
+      for (int cc = 0; ok && cc < nmine; ++cc) {
+        const int c = half + cc * EPW;
+        uint32_t r[32];
+        dev::tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * BN + c * 32), r);
+        dev::tmem_wait_ld();
+        if (cc == nmine - 1) {
+          dev::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) dev::mbar_arrive_cluster(lead(tempty_bar(b)));
+        }
+        if (o0 + q * 32 >= p.N) continue;
+        const int n_valid = t_end - c * 32;
+        if (p.out_acc) {
+          int32_t* dst = reinterpret_cast<int32_t*>(p.out) + (int64_t)(t0 + c * 32) * p.N + o;
+#pragma unroll
+          for (int jj = 0; jj < 32; ++jj)
+            if (has_o && jj < n_valid) dst[(int64_t)jj * p.N] = (int32_t)r[jj] >> 4;
+        } else {
+          const float4* tk4 = reinterpret_cast<const float4*>(s_tok + c * 32);
+          const float2 sw2 = make_float2(sw, sw), w12 = make_float2(w1, w1);
+          const float2 bb2 = make_float2(bb, bb);
+          uint32_t yb[16];
+#pragma unroll
+          for (int jj = 0; jj < 32; jj += 2) {
+            const float4 tk = tk4[jj / 2];
+            const float2 s2 = __fmul2_rn(make_float2(tk.x, tk.z), sw2);
+            const float2 c2 = __ffma2_rn(make_float2(tk.y, tk.w), w12, bb2);
+            const float2 a2 = make_float2((float)(int32_t)r[jj], (float)(int32_t)r[jj + 1]);
+            const __nv_bfloat162 y = __float22bfloat162_rn(__ffma2_rn(a2, s2, c2));
+            yb[jj / 2] = *reinterpret_cast<const uint32_t*>(&y);
+          }
+          if (lane == 0) dev::bulk_wait_all_read();
+          __syncwarp();
+#pragma unroll
+          for (int jj = 0; jj < 32; jj += 2) {
+            *reinterpret_cast<uint16_t*>(stg + jj * 64 + lane * 2) = (uint16_t)(yb[jj / 2] & 0xFFFFu);
+            *reinterpret_cast<uint16_t*>(stg + (jj + 1) * 64 + lane * 2) = (uint16_t)(yb[jj / 2] >> 16);
+          }
+          dev::fence_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            dev::tma_store_2d(&tm_y, dev::smem_u32(stg), o0 + q * 32, t0 + c * 32);
+            dev::bulk_commit();
+          }
+        }
+      }
+      dev::named_bar(1, NEPI);
+    }
+    if (lane == 0) dev::bulk_wait_all();
+  }
+
+  dev::tc_fence_before();
+  dev::cluster_sync();  // no MMA, remote arrive or TMEM access of either CTA is still pending
+  if (warp == W_MMA) {
+    dev::tc_fence_after();
+    dev::tmem_dealloc_pair(tmem, TCOLS);
+  }
+}
+
+oq_status run_a8t(const GemmArgs& g, const GemmParams& p, cudaStream_t s) {
+  using namespace ta;
+  CUtensorMap tx, tw, ty;
+  bool ok = true;
+  if (!g.out_acc)
+    ok &= make_map_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.out, (uint64_t)g.N, (uint64_t)g.T,
+                      (uint64_t)g.N * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE);
+  else
+    std::memset(&ty, 0, sizeof(ty));
+  ok &= make_map_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.a, (uint64_t)g.K, (uint64_t)g.T,
+                    (uint64_t)g.K, 128, XR, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= make_map_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.w, (uint64_t)g.K / 2, (uint64_t)g.N,
+                    (uint64_t)g.K / 2, 64, BM, CU_TENSOR_MAP_SWIZZLE_64B);
+  if (!ok) return fail(OQ_ERR_CUDA, "cuTensorMapEncodeTiled failed or unavailable");
+  auto kern = &k_gemm_a8t;
+  const cudaError_t attr_err = allow_max_dynamic_smem(reinterpret_cast<const void*>(kern));
+  if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute(gemm_a8t)");
+  const int pairs = active_pairs_n(reinterpret_cast<const void*>(kern), SMEM, NTHR);
+  if (pairs <= 0) return fail(OQ_ERR_UNSUPPORTED, "gemm: no CTA pair fits on this device");
+  const int64_t chunks = ((g.N + 2 * BM - 1) / (2 * BM)) * ((g.T + CH - 1) / CH);
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3((unsigned)(2 * std::min<int64_t>(chunks, pairs)));
+  cfg.blockDim = dim3(NTHR);
+  cfg.dynamicSmemBytes = SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t le = cudaLaunchKernelEx(&cfg, kern, tx, tw, ty, p);
+  if (le != cudaSuccess) return cuda_fail(le, "launch gemm_a8t");
+  return OQ_OK;
+}
+
 uint16_t f16_bits(float f) {
   const __half h = __float2half_rn(f);
   return *reinterpret_cast<const uint16_t*>(&h);
@@ -1037,7 +1459,7 @@ oq_status launch_gemm(const GemmArgs& g, cudaStream_t s) {
   // up to 128 tokens: single CTAs on 128-channel tiles; beyond: CTA pairs on 256 channels
   const bool small = g.T <= 128;
   switch (g.kind) {
-    case kGemmA8: return small ? run<kGemmA8, 1>(g, p, s) : run<kGemmA8, 2>(g, p, s);
+    case kGemmA8: return small ? run<kGemmA8, 1>(g, p, s) : run_a8t(g, p, s);
     case kGemmA4: return small ? run<kGemmA4, 1>(g, p, s) : run<kGemmA4, 2>(g, p, s);
     case kGemmLloydMax:
       return small ? run<kGemmLloydMax, 1>(g, p, s) : run<kGemmLloydMax, 2>(g, p, s);
