@@ -1006,8 +1006,16 @@ oq_status run(const GemmArgs& g, const GemmParams& p, cudaStream_t s) {
 // rows in registers (one row per thread: the thread's TMEM lane) and store it with tcgen05.st
 // into one of SA weight stages in TMEM, so the widened weights never pass through shared memory:
 // per K block and SM, shared memory carries only the packed weights (TMA write + converter read,
-// 16 KB) and the activations (TMA write + MMA read, 2 x 12 KB). TMEM holds two accumulators of
-// BN = 192 columns and SA = 4 weight stages of 32 columns (4 int8 per column): 512 columns.
+// 16 KB) and the activations (TMA write + MMA read, 2 x 16 KB).
+//
+// Pipeline depth. The completion of an MMA reaches an mbarrier (tcgen05.commit) several hundred
+// nanoseconds after the tensor pipe finishes it, and a stage can only be refilled after that
+// arrive; with four stages in flight the MMA issue rate halves. So TMEM holds one accumulator
+// of BN = 256 columns and SA = 8 weight stages (2.3 us of MMA work at the N = 256 rate), and the
+// activation ring has as many stages. One commit per K block frees both the weight stage and
+// the activation stage of that block. The accumulator is not double-buffered: the next tile's
+// MMAs wait until the epilogue warps have read it (each releases it after its last
+// tcgen05.ld, before that chunk's stores), a fraction of a microsecond per tile of 24 K blocks.
 //
 // Schedule: the work is the flattened (channel tile, 32-token chunk) space; every CTA pair takes
 // an equal contiguous range of it and cuts its range, within each channel tile, into tiles of
@@ -1018,29 +1026,28 @@ oq_status run(const GemmArgs& g, const GemmParams& p, cudaStream_t s) {
 // 4-11 converters in two groups (warps 4-7 and 8-11, each covering the four TMEM lane quarters)
 // that take alternate K blocks, 12-19 epilogue (two per lane quarter).
 namespace ta {
-constexpr int BN = 192;              // tokens per tile at most (MMA N)
+constexpr int BN = 256;              // tokens per tile at most (MMA N)
 constexpr int MAXCH = BN / CH;       // 32-token chunks per tile at most
 constexpr int XR = BN / 2;           // activation rows per CTA and stage
-constexpr int SX = 6;                // activation ring
+constexpr int SK = 8;                // K-block stages: weight stages in TMEM and activation ring
 constexpr int SP = 8;                // packed weight ring
-constexpr int SA = 4;                // widened weight stages in TMEM
-constexpr int ACOL = 2 * BN;         // TMEM column of weight stage 0
+constexpr int ACOL = BN;             // TMEM column of weight stage 0 (after the accumulator)
 constexpr int TCOLS = 512;           // TMEM columns allocated
 constexpr int XT = XR * 128;         // activation stage bytes (128-byte swizzled rows)
 constexpr int WP = BM * 64;          // packed weight stage bytes (64-byte swizzled rows)
 constexpr int STG = 32 * 32 * 2;     // bf16 [32 tokens][32 channels] staging tile per warp
 // (NEPI = 256 epilogue threads, EPW = 2 per lane quarter, as in k_gemm)
 constexpr int OFF_X = 0;
-constexpr int OFF_P = OFF_X + SX * XT;
+constexpr int OFF_P = OFF_X + SK * XT;
 constexpr int OFF_STG = OFF_P + SP * WP;
 constexpr int OFF_TOK = OFF_STG + (NEPI / 32) * STG;
 constexpr int OFF_BAR = OFF_TOK + BN * 8;
-constexpr int NBAR = 2 * SX + 2 * SP + 2 * SA + 4 + 1;
+constexpr int NBAR = 3 * SK + 2 * SP + 2 + 1;
 constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
 constexpr int SMEM = OFF_MISC + 16 + 1024;
 constexpr int NTHR = 640;
 constexpr int W_PROD_P = 0, W_MMA = 1, W_PROD_X = 2, W_CONV0 = 4, W_EPI0 = 12;
-static_assert(ACOL + SA * 32 <= TCOLS, "tensor memory budget");
+static_assert(ACOL + SK * 32 <= TCOLS, "tensor memory budget");
 static_assert(XT % 1024 == 0 && OFF_P % 1024 == 0 && WP % 1024 == 0, "stage alignment");
 static_assert(SMEM <= 232448, "shared memory");
 static_assert(NTHR == (W_EPI0 * 32 + NEPI), "warp roles");
@@ -1091,36 +1098,29 @@ __global__ void __launch_bounds__(ta::NTHR, 1)
   auto tiles = [&]() { return RangeIter(p.T, n_o, unit_index, n_units); };
 
   auto bar = [&](int i) { return dev::smem_u32(&bars[i]); };
-  auto xfull_bar = [&](int s) { return bar(s); };
-  auto xempty_bar = [&](int s) { return bar(SX + s); };
-  auto pfull_bar = [&](int s) { return bar(2 * SX + s); };
-  auto pempty_bar = [&](int s) { return bar(2 * SX + SP + s); };
-  auto wready_bar = [&](int c) { return bar(2 * SX + 2 * SP + c); };
-  auto wfree_bar = [&](int c) { return bar(2 * SX + 2 * SP + SA + c); };
-  auto tfull_bar = [&](int b) { return bar(2 * SX + 2 * SP + 2 * SA + b); };
-  auto tempty_bar = [&](int b) { return bar(2 * SX + 2 * SP + 2 * SA + 2 + b); };
-  const uint32_t drain_bar = bar(2 * SX + 2 * SP + 2 * SA + 4);
+  auto xfull_bar = [&](int s) { return bar(s); };             // activation stage landed
+  auto wready_bar = [&](int s) { return bar(SK + s); };       // weight stage in TMEM
+  auto kfree_bar = [&](int s) { return bar(2 * SK + s); };    // K block s consumed by the MMAs
+  auto pfull_bar = [&](int s) { return bar(3 * SK + s); };
+  auto pempty_bar = [&](int s) { return bar(3 * SK + SP + s); };
+  const uint32_t tfull = bar(3 * SK + 2 * SP), tempty = bar(3 * SK + 2 * SP + 1);
+  const uint32_t drain_bar = bar(3 * SK + 2 * SP + 2);
   auto x_stage = [&](int s) { return smem + OFF_X + s * XT; };
   auto p_stage = [&](int s) { return smem + OFF_P + s * WP; };
   auto lead = [&](uint32_t a) { return dev::map_to_cta(a, 0); };
 
   if (tid == 0) {
-    for (int s = 0; s < SX; ++s) {
+    for (int s = 0; s < SK; ++s) {
       dev::mbar_init(xfull_bar(s), 1);
-      dev::mbar_init(xempty_bar(s), 1);
+      dev::mbar_init(wready_bar(s), 2 * 4);  // four converter warps of each CTA
+      dev::mbar_init(kfree_bar(s), 1);
     }
     for (int s = 0; s < SP; ++s) {
       dev::mbar_init(pfull_bar(s), 1);
       dev::mbar_init(pempty_bar(s), 4);      // the four warps of the converting group
     }
-    for (int c = 0; c < SA; ++c) {
-      dev::mbar_init(wready_bar(c), 2 * 4);  // four converter warps of each CTA
-      dev::mbar_init(wfree_bar(c), 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-      dev::mbar_init(tfull_bar(b), 1);
-      dev::mbar_init(tempty_bar(b), 2 * (NEPI / 32));
-    }
+    dev::mbar_init(tfull, 1);
+    dev::mbar_init(tempty, 2 * (NEPI / 32));
     dev::mbar_init(drain_bar, 1);
     s_misc[1] = 0;
     dev::fence_mbar_init_cluster();
@@ -1144,7 +1144,7 @@ __global__ void __launch_bounds__(ta::NTHR, 1)
     // ---------------- producers ----------------
     const bool packed_role = warp == W_PROD_P;
     if (lane == 0) {
-      const int ns = packed_role ? SP : SX;
+      const int ns = packed_role ? SP : SK;
       uint32_t j = 0;
       bool ok = true;
       auto it = tiles();
@@ -1156,7 +1156,9 @@ __global__ void __launch_bounds__(ta::NTHR, 1)
         for (int step = 0; step < nkb; ++step, ++j) {
           const int kb = (step + krot) % nkb;
           const int s = j % ns;
-          const uint32_t empty_b = packed_role ? pempty_bar(s) : xempty_bar(s);
+          // a packed stage is free once its group has read it; an activation stage once the
+          // MMAs of its K block have completed
+          const uint32_t empty_b = packed_role ? pempty_bar(s) : kfree_bar(s);
           const uint32_t full_b = packed_role ? pfull_bar(s) : xfull_bar(s);
           if (*s_abort || !dev::mbar_wait(empty_b, ((j / ns) & 1u) ^ 1u, p.err, kSiteGemmEmpty,
                                           p.limit_ns)) {
@@ -1189,20 +1191,18 @@ __global__ void __launch_bounds__(ta::NTHR, 1)
       int m, t0, nch;
       for (; ok && it.next(m, t0, nch); ++it_n) {
         const uint32_t idesc = dev::idesc_i8(UNIT, nch * CH);
-        const int b = it_n & 1;
-        if (*s_abort || !dev::mbar_wait(tempty_bar(b), ((it_n >> 1) & 1u) ^ 1u, p.err,
-                                        kSiteGemmAccum, p.limit_ns)) {
+        if (*s_abort || !dev::mbar_wait(tempty, (it_n & 1u) ^ 1u, p.err, kSiteGemmAccum,
+                                        p.limit_ns)) {
           give_up();
           ok = false;
           break;
         }
         dev::tc_fence_after();
-        const uint32_t dt = tmem + (uint32_t)(b * BN);
         for (int step = 0; step < nkb; ++step, ++j) {
-          const int c = j % SA, sx = j % SX;
+          const int c = j % SK;
           bool w = !*s_abort &&
-                   dev::mbar_wait(wready_bar(c), (j / SA) & 1u, p.err, kSiteGemmConv, p.limit_ns);
-          if (w) w = dev::mbar_wait(xfull_bar(sx), (j / SX) & 1u, p.err, kSiteGemmFull, p.limit_ns);
+                   dev::mbar_wait(wready_bar(c), (j / SK) & 1u, p.err, kSiteGemmConv, p.limit_ns);
+          if (w) w = dev::mbar_wait(xfull_bar(c), (j / SK) & 1u, p.err, kSiteGemmFull, p.limit_ns);
           if (!w) {
             give_up();
             ok = false;
@@ -1210,17 +1210,16 @@ __global__ void __launch_bounds__(ta::NTHR, 1)
           }
           dev::tc_fence_after();
           const uint32_t at = tmem + (uint32_t)(ACOL + c * 32);
-          const uint32_t bx = dev::smem_u32(x_stage(sx));
+          const uint32_t bx = dev::smem_u32(x_stage(c));
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            dev::mma_i8_pair_ta(dt, at + kk * 8, dev::sdesc_sw128(bx + kk * 32), idesc,
+            dev::mma_i8_pair_ta(tmem, at + kk * 8, dev::sdesc_sw128(bx + kk * 32), idesc,
                                 (step | kk) != 0);
           issued = true;
-          dev::mma_commit_pair(wfree_bar(c));
-          dev::mma_commit_pair(xempty_bar(sx));
+          dev::mma_commit_pair(kfree_bar(c));
         }
         if (!ok) break;
-        dev::mma_commit_pair(tfull_bar(b));
+        dev::mma_commit_pair(tfull);
       }
       if (!ok && issued) {  // wait for the MMAs in flight before TMEM is freed
         dev::mma_commit_pair(drain_bar);
@@ -1233,7 +1232,8 @@ __global__ void __launch_bounds__(ta::NTHR, 1)
     // stage holds 64-byte rows whose four 16-byte groups were swizzled by TMA (group g of row r
     // at ((g ^ ((r >> 1) & 3)) << 4)), so that the warp's row-wise reads hit distinct banks.
     // Group g (32 elements) widens to columns 8g..8g+3 (low nibbles, elements 32g..32g+15) and
-    // 8g+4..8g+7 (high nibbles, elements 32g+16..32g+31).
+    // 8g+4..8g+7 (high nibbles, elements 32g+16..32g+31). The widening happens before the wait
+    // for the weight stage to be free, so that only the TMEM store follows that wait.
     const int grp = (warp - W_CONV0) >> 2, q = warp & 3;
     const int r = q * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
@@ -1244,11 +1244,9 @@ __global__ void __launch_bounds__(ta::NTHR, 1)
     while (ok && it.next(m, t0, nch)) {
       for (int step = 0; step < nkb; ++step, ++j) {
         if ((int)(j & 1u) != grp) continue;
-        const int s = j % SP, c = j % SA;
+        const int s = j % SP, c = j % SK;
         bool w = !*s_abort &&
                  dev::mbar_wait(pfull_bar(s), (j / SP) & 1u, p.err, kSiteGemmFull, p.limit_ns);
-        if (w)
-          w = dev::mbar_wait(wfree_bar(c), ((j / SA) & 1u) ^ 1u, p.err, kSiteGemmConv, p.limit_ns);
         w = __all_sync(0xffffffffu, w);
         if (!w) {
           give_up();
@@ -1272,6 +1270,15 @@ __global__ void __launch_bounds__(ta::NTHR, 1)
         }
         __syncwarp();              // the warp's reads of the packed stage are done
         if (lane == 0) dev::mbar_arrive(pempty_bar(s));
+        w = !*s_abort &&
+            dev::mbar_wait(kfree_bar(c), ((j / SK) & 1u) ^ 1u, p.err, kSiteGemmConv, p.limit_ns);
+        w = __all_sync(0xffffffffu, w);
+        if (!w) {
+          give_up();
+          ok = false;
+          break;
+        }
+        dev::tc_fence_after();
         dev::tmem_st32(tmem + lane_addr + (uint32_t)(ACOL + c * 32), o);
         dev::tmem_wait_st();
         dev::tc_fence_before();
@@ -1281,6 +1288,8 @@ __global__ void __launch_bounds__(ta::NTHR, 1)
     }
   } else if (warp >= W_EPI0) {
     // ---------------- epilogue ----------------
+    // Each warp releases the accumulator (the next tile's MMAs wait for that) right after its
+    // last tcgen05.ld of the tile, before that chunk's scaling and stores.
     const int etid = tid - W_EPI0 * 32;
     uint8_t* stg = smem + OFF_STG + (warp - W_EPI0) * STG;
     const int q = warp & 3;
@@ -1293,7 +1302,6 @@ __global__ void __launch_bounds__(ta::NTHR, 1)
     int m, t0, nch;
     for (; ok && it.next(m, t0, nch); ++it_n) {
       const int o0 = m * UNIT + (int)rank * BM;
-      const int b = it_n & 1;
       const int o = o0 + o_local;
       const bool has_o = o < p.N;
       const float sw = has_o ? p.w_scale[o] * (1.f / 16.f) : 0.f;
@@ -1306,7 +1314,7 @@ __global__ void __launch_bounds__(ta::NTHR, 1)
                                (t < p.T && p.mean) ? p.mean[t] : 0.f);
       }
       if (ep_lead) {
-        const bool ready = !*s_abort && dev::mbar_wait(tfull_bar(b), (it_n >> 1) & 1u, p.err,
+        const bool ready = !*s_abort && dev::mbar_wait(tfull, it_n & 1u, p.err,
                                                        kSiteGemmAccum, p.limit_ns);
         if (!ready) give_up();
         s_misc[2] = ready ? 1u : 0u;
@@ -1315,22 +1323,22 @@ __global__ void __launch_bounds__(ta::NTHR, 1)
       ok = *reinterpret_cast<volatile uint32_t*>(&s_misc[2]) != 0;
       if (ok) dev::tc_fence_after();
       const int t_end = min(ncols, p.T - t0);
-      const int nmine = (nch - half + EPW - 1) / EPW;
+      const int nmine = (nch - half + EPW - 1) / EPW;   // chunks half, half + EPW, ...
       if (ok && nmine == 0) {
         dev::tc_fence_before();
         __syncwarp();
-        if (lane == 0) dev::mbar_arrive_cluster(lead(tempty_bar(b)));
+        if (lane == 0) dev::mbar_arrive_cluster(lead(tempty));
       }
 #pragma unroll 1
       for (int cc = 0; ok && cc < nmine; ++cc) {
         const int c = half + cc * EPW;
         uint32_t r[32];
-        dev::tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * BN + c * 32), r);
+        dev::tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(c * 32), r);
         dev::tmem_wait_ld();
-        if (cc == nmine - 1) {
+        if (cc == nmine - 1) {   // this warp's part of the accumulator is read: release it
           dev::tc_fence_before();
           __syncwarp();
-          if (lane == 0) dev::mbar_arrive_cluster(lead(tempty_bar(b)));
+          if (lane == 0) dev::mbar_arrive_cluster(lead(tempty));
         }
         if (o0 + q * 32 >= p.N) continue;
         const int n_valid = t_end - c * 32;
@@ -1368,7 +1376,7 @@ __global__ void __launch_bounds__(ta::NTHR, 1)
           }
         }
       }
-      dev::named_bar(1, NEPI);
+      dev::named_bar(1, NEPI);   // s_tok of this tile is no longer read
     }
     if (lane == 0) dev::bulk_wait_all();
   }
