@@ -1426,6 +1426,390 @@ oq_status run_a8t(const GemmArgs& g, const GemmParams& p, cudaStream_t s) {
   return OQ_OK;
 }
 
+// ================================================================================================
+// W4A8 with the widened weights in shared memory and double-buffered accumulators (CTA pairs,
+// T > 128). The variant the W4A8 layer runs.
+//
+// The converter warps load the packed INT4 weights of each 128-byte K block straight from L2
+// (the prepared weights stay L2-resident) into registers, widen them to the int8 16 n and store
+// them into a stage of widened weights in the 128-byte-swizzled K-major layout the MMA reads.
+// There is no shared-memory ring of packed weights: its space goes to deeper rings. The loads
+// of a K block are issued before the converter waits for its stage to be free, and that wait
+// (the converters run ahead of the MMA) hides the L2 latency.
+//
+// Pipeline depth. The completion of an MMA reaches an mbarrier (tcgen05.commit) several hundred
+// nanoseconds after the tensor pipe finishes it, and a stage is refilled only after that
+// arrive. SK = 6 stages of widened weights and of activations (1.7 us of MMA work at N = 256)
+// keep the pipe fed; one commit per K block frees both stages of that block. TMEM holds two
+// accumulators of 256 columns, so the epilogue of one tile overlaps the next tile's MMAs.
+//
+// Schedule: as in the tensor-memory variant, every CTA pair takes an equal contiguous range of
+// the (channel tile, 32-token chunk) space, cut into tiles of at most 256 tokens.
+//
+// Warps: 0 activation producer, 1 TMEM owner + MMA issuer, 2-3 idle, 4-11 converters in two
+// groups of four that take alternate K blocks, 12-19 epilogue (two per TMEM lane quarter).
+namespace sa {
+constexpr int BN = 256;              // tokens per tile at most (MMA N)
+constexpr int MAXCH = BN / CH;
+constexpr int XR = BN / 2;           // activation rows per CTA and stage
+constexpr int SK = 6;                // K-block stages: widened weights and activations
+constexpr int WT = BM * 128;         // widened weight stage bytes
+constexpr int XT = XR * 128;         // activation stage bytes
+constexpr int TCOLS = 2 * BN;        // two accumulators
+constexpr int STG = 32 * 32 * 2;     // bf16 [32 tokens][32 channels] staging tile per warp
+constexpr int OFF_W = 0;
+constexpr int OFF_X = OFF_W + SK * WT;
+constexpr int OFF_STG = OFF_X + SK * XT;
+constexpr int OFF_TOK = OFF_STG + (NEPI / 32) * STG;
+constexpr int OFF_BAR = OFF_TOK + BN * 8;
+constexpr int NBAR = 3 * SK + 4 + 1;
+constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+constexpr int SMEM = OFF_MISC + 16 + 1024;
+constexpr int NTHR = 640;
+constexpr int W_PROD_X = 0, W_MMA = 1, W_CONV0 = 4, W_EPI0 = 12;
+static_assert(WT % 1024 == 0 && XT % 1024 == 0 && OFF_X % 1024 == 0, "stage alignment");
+static_assert(SMEM <= 232448, "shared memory");
+static_assert(NTHR == (W_EPI0 * 32 + NEPI), "warp roles");
+}  // namespace sa
+
+// A walk over one CTA pair's K blocks in the order every role processes them.
+struct KWalk {
+  ta::RangeIter rit;
+  int m = 0, t0 = 0, nch = 0, step = 0, nkb;
+  bool live;
+  __device__ KWalk(int T, int n_o, int unit, int n_units, int nkb_)
+      : rit(T, n_o, unit, n_units), nkb(nkb_) {
+    live = rit.next(m, t0, nch);
+  }
+  __device__ void advance() {
+    if (live && ++step == nkb) {
+      step = 0;
+      live = rit.next(m, t0, nch);
+    }
+  }
+};
+
+__global__ void __launch_bounds__(sa::NTHR, 1)
+    k_gemm_a8s(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_y,
+               const uint8_t* __restrict__ wpk, const GemmParams p) {
+  using namespace sa;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  float2* s_tok = reinterpret_cast<float2*>(smem + OFF_TOK);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint32_t* s_misc = reinterpret_cast<uint32_t*>(smem + OFF_MISC);  // tmem, abort, epi flag
+  volatile uint32_t* s_abort = s_misc + 1;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = dev::cluster_ctarank();   // 0 = the pair's leader
+  constexpr int UNIT = 2 * BM;                     // channels per tile
+  const int n_o = (p.N + UNIT - 1) / UNIT;
+  const int nkb = (p.K + 127) / 128;
+  const int unit_index = (int)blockIdx.x / 2, n_units = (int)gridDim.x / 2;
+  auto tiles = [&]() { return ta::RangeIter(p.T, n_o, unit_index, n_units); };
+
+  auto bar = [&](int i) { return dev::smem_u32(&bars[i]); };
+  auto xfull_bar = [&](int s) { return bar(s); };             // activation stage landed
+  auto wready_bar = [&](int s) { return bar(SK + s); };       // widened weight stage stored
+  auto kfree_bar = [&](int s) { return bar(2 * SK + s); };    // K block s consumed by the MMAs
+  auto tfull_bar = [&](int b) { return bar(3 * SK + b); };
+  auto tempty_bar = [&](int b) { return bar(3 * SK + 2 + b); };
+  const uint32_t drain_bar = bar(3 * SK + 4);
+  auto w_stage = [&](int s) { return smem + OFF_W + s * WT; };
+  auto x_stage = [&](int s) { return smem + OFF_X + s * XT; };
+  auto lead = [&](uint32_t a) { return dev::map_to_cta(a, 0); };
+
+  if (tid == 0) {
+    for (int s = 0; s < SK; ++s) {
+      dev::mbar_init(xfull_bar(s), 1);
+      dev::mbar_init(wready_bar(s), 2 * 4);  // four converter warps of each CTA
+      dev::mbar_init(kfree_bar(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      dev::mbar_init(tfull_bar(b), 1);
+      dev::mbar_init(tempty_bar(b), 2 * (NEPI / 32));
+    }
+    dev::mbar_init(drain_bar, 1);
+    s_misc[1] = 0;
+    dev::fence_mbar_init_cluster();
+  }
+  if (warp == W_PROD_X && lane == 0) dev::prefetch_tmap(&tm_x);
+  if (warp == W_EPI0 && lane == 0 && !p.out_acc) dev::prefetch_tmap(&tm_y);
+  if (warp == W_MMA) {
+    dev::tmem_alloc_pair(dev::smem_u32(&s_misc[0]), TCOLS);
+    dev::tmem_relinquish_pair();
+  }
+  dev::tc_fence_before();
+  dev::cluster_sync();   // barrier inits of both CTAs visible before any remote arrive
+  dev::tc_fence_after();
+  const uint32_t tmem = s_misc[0];
+  auto give_up = [&]() { *s_abort = 1; };
+
+  if (warp == W_PROD_X) {
+    // ---------------- activation producer ----------------
+    if (lane == 0) {
+      uint32_t j = 0;
+      bool ok = true;
+      auto it = tiles();
+      int m, t0, nch;
+      while (ok && it.next(m, t0, nch)) {
+        const int x0 = t0 + (int)rank * (nch * CH / 2);      // this CTA's activation rows
+        const int krot = k_rotation(m, nkb);
+        for (int step = 0; step < nkb; ++step, ++j) {
+          const int kb = (step + krot) % nkb;
+          const int s = j % SK;
+          if (!dev::mbar_wait(kfree_bar(s), ((j / SK) & 1u) ^ 1u, p.err, kSiteGemmEmpty,
+                              p.limit_ns) || *s_abort) {
+            give_up();
+            ok = false;
+            break;
+          }
+          // both halves complete on the leader's barrier, which expects the bytes of both
+          if (rank == 0) dev::mbar_arrive_expect_tx(xfull_bar(s), (uint32_t)(2 * XT));
+          dev::tma_load_2d_pair(dev::smem_u32(x_stage(s)), &tm_x, kb * 128, x0, lead(xfull_bar(s)));
+        }
+      }
+      if (!ok && rank == 0) {
+        for (uint32_t i = (j >= (uint32_t)SK ? j - SK : 0); i < j; ++i)
+          dev::mbar_wait(xfull_bar(i % SK), (i / SK) & 1u, p.err, kSiteGemmDrain, p.limit_ns);
+      }
+    }
+  } else if (warp == W_MMA) {
+    // ---------------- MMA issuer (the leader's lane 0) ----------------
+    if (lane == 0 && rank == 0) {
+      uint32_t j = 0, it_n = 0;
+      bool ok = true, issued = false;
+      auto it = tiles();
+      int m, t0, nch;
+      for (; ok && it.next(m, t0, nch); ++it_n) {
+        const uint32_t idesc = dev::idesc_i8(UNIT, nch * CH);
+        const int b = it_n & 1;
+        if (!dev::mbar_wait(tempty_bar(b), ((it_n >> 1) & 1u) ^ 1u, p.err, kSiteGemmAccum,
+                            p.limit_ns) || *s_abort) {
+          give_up();
+          ok = false;
+          break;
+        }
+        dev::tc_fence_after();
+        const uint32_t dt = tmem + (uint32_t)(b * BN);
+        for (int step = 0; step < nkb; ++step, ++j) {
+          const int c = j % SK;
+          const uint32_t par = (j / SK) & 1u;
+          if (!dev::mbar_wait(wready_bar(c), par, p.err, kSiteGemmConv, p.limit_ns) ||
+              !dev::mbar_wait(xfull_bar(c), par, p.err, kSiteGemmFull, p.limit_ns)) {
+            give_up();
+            ok = false;
+            break;
+          }
+          dev::tc_fence_after();
+          const uint32_t aw = dev::smem_u32(w_stage(c));
+          const uint32_t bx = dev::smem_u32(x_stage(c));
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            dev::mma_i8_pair(dt, dev::sdesc_sw128(aw + kk * 32), dev::sdesc_sw128(bx + kk * 32),
+                             idesc, (step | kk) != 0);
+          issued = true;
+          dev::mma_commit_pair(kfree_bar(c));
+        }
+        if (!ok) break;
+        dev::mma_commit_pair(tfull_bar(b));
+      }
+      if (!ok && issued) {  // wait for the MMAs in flight before TMEM is freed
+        dev::mma_commit_pair(drain_bar);
+        dev::mbar_wait(drain_bar, 0, p.err, kSiteGemmDrain, p.limit_ns);
+      }
+    }
+  } else if (warp >= W_CONV0 && warp < W_EPI0) {
+    // ---------------- converters: packed weights (L2) -> int8 16 n -> shared memory -------
+    // Group g takes the K blocks j = g, g + 2, ... Thread ctid of a group takes 16-byte packed
+    // group q = ctid & 3 of rows r0 + 32 i (r0 = ctid >> 2, i = 0..3): its low nibbles become
+    // chunk 2q and its high nibbles chunk 2q + 1 of the row's 128 widened bytes, stored at
+    // chunk index ^ (row & 7) (the 128-byte swizzle), the same for every i.
+    const int grp = (warp - W_CONV0) >> 2;
+    const int ctid = ((warp - W_CONV0) & 3) * 32 + lane;
+    const int r0 = ctid >> 2, q = ctid & 3;
+    const int ph = r0 & 7;
+    const int64_t kbytes = p.K / 2;                  // packed bytes per weight row
+    KWalk wk(p.T, n_o, unit_index, n_units, nkb);
+    if (grp == 1) wk.advance();
+    bool ok = true;
+    for (uint32_t j = (uint32_t)grp; ok && wk.live; j += 2) {
+      const int kb = (wk.step + k_rotation(wk.m, nkb)) % nkb;
+      const int o0 = wk.m * UNIT + (int)rank * BM;
+      const int64_t col = (int64_t)kb * 64 + q * 16;
+      uint4 in[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int o = o0 + r0 + 32 * i;
+        in[i] = (o < p.N && col < kbytes)
+                    ? __ldg(reinterpret_cast<const uint4*>(wpk + (int64_t)o * kbytes + col))
+                    : make_uint4(0u, 0u, 0u, 0u);
+      }
+      const int c = j % SK;
+      bool w = dev::mbar_wait(kfree_bar(c), ((j / SK) & 1u) ^ 1u, p.err, kSiteGemmConv,
+                              p.limit_ns) && !*s_abort;
+      w = __all_sync(0xffffffffu, w);
+      if (!w) {
+        give_up();
+        ok = false;
+        break;
+      }
+      uint8_t* dst = w_stage(c);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        uint8_t* rowp = dst + (r0 + 32 * i) * 128;
+        *reinterpret_cast<uint4*>(rowp + (((2 * q) ^ ph) << 4)) =
+            make_uint4((in[i].x << 4) & 0xF0F0F0F0u, (in[i].y << 4) & 0xF0F0F0F0u,
+                       (in[i].z << 4) & 0xF0F0F0F0u, (in[i].w << 4) & 0xF0F0F0F0u);
+        *reinterpret_cast<uint4*>(rowp + (((2 * q + 1) ^ ph) << 4)) =
+            make_uint4(in[i].x & 0xF0F0F0F0u, in[i].y & 0xF0F0F0F0u, in[i].z & 0xF0F0F0F0u,
+                       in[i].w & 0xF0F0F0F0u);
+      }
+      dev::fence_async_smem();   // this thread's stores -> visible to the tensor cores
+      __syncwarp();
+      if (lane == 0) dev::mbar_arrive_cluster(lead(wready_bar(c)));
+      wk.advance();
+      wk.advance();
+    }
+  } else if (warp >= W_EPI0) {
+    // ---------------- epilogue ----------------
+    const int etid = tid - W_EPI0 * 32;
+    uint8_t* stg = smem + OFF_STG + (warp - W_EPI0) * STG;
+    const int q = warp & 3;
+    const int half = (warp - W_EPI0) >> 2;
+    const int o_local = q * 32 + lane;
+    const bool ep_lead = etid == 0;
+    uint32_t it_n = 0;
+    bool ok = true;
+    auto it = tiles();
+    int m, t0, nch;
+    for (; ok && it.next(m, t0, nch); ++it_n) {
+      const int o0 = m * UNIT + (int)rank * BM;
+      const int b = it_n & 1;
+      const int o = o0 + o_local;
+      const bool has_o = o < p.N;
+      const float sw = has_o ? p.w_scale[o] * (1.f / 16.f) : 0.f;
+      const float w1 = (has_o && p.mean) ? p.w_rowsum[o] : 0.f;
+      const float bb = (has_o && p.bias) ? __bfloat162float(p.bias[o]) : 0.f;
+      const int ncols = nch * CH;
+      for (int i = etid; i < ncols; i += NEPI) {
+        const int t = t0 + i;
+        s_tok[i] = make_float2((t < p.T) ? p.a_scale[t] : 0.f,
+                               (t < p.T && p.mean) ? p.mean[t] : 0.f);
+      }
+      if (ep_lead) {
+        const bool ready = dev::mbar_wait(tfull_bar(b), (it_n >> 1) & 1u, p.err,
+                                          kSiteGemmAccum, p.limit_ns) && !*s_abort;
+        if (!ready) give_up();
+        s_misc[2] = ready ? 1u : 0u;
+      }
+      dev::named_bar(1, NEPI);
+      ok = *reinterpret_cast<volatile uint32_t*>(&s_misc[2]) != 0;
+      if (ok) dev::tc_fence_after();
+      const int t_end = min(ncols, p.T - t0);
+      const int nmine = (nch - half + EPW - 1) / EPW;
+      if (ok && nmine == 0) {
+        dev::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) dev::mbar_arrive_cluster(lead(tempty_bar(b)));
+      }
+#pragma unroll 1
+      for (int cc = 0; ok && cc < nmine; ++cc) {
+        const int c = half + cc * EPW;
+        uint32_t r[32];
+        dev::tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * BN + c * 32), r);
+        dev::tmem_wait_ld();
+        if (cc == nmine - 1) {
+          dev::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) dev::mbar_arrive_cluster(lead(tempty_bar(b)));
+        }
+        if (o0 + q * 32 >= p.N) continue;
+        const int n_valid = t_end - c * 32;
+        if (p.out_acc) {
+          int32_t* dst = reinterpret_cast<int32_t*>(p.out) + (int64_t)(t0 + c * 32) * p.N + o;
+#pragma unroll
+          for (int jj = 0; jj < 32; ++jj)
+            if (has_o && jj < n_valid) dst[(int64_t)jj * p.N] = (int32_t)r[jj] >> 4;
+        } else {
+          const float4* tk4 = reinterpret_cast<const float4*>(s_tok + c * 32);
+          const float2 sw2 = make_float2(sw, sw), w12 = make_float2(w1, w1);
+          const float2 bb2 = make_float2(bb, bb);
+          uint32_t yb[16];
+#pragma unroll
+          for (int jj = 0; jj < 32; jj += 2) {
+            const float4 tk = tk4[jj / 2];
+            const float2 s2 = __fmul2_rn(make_float2(tk.x, tk.z), sw2);
+            const float2 c2 = __ffma2_rn(make_float2(tk.y, tk.w), w12, bb2);
+            const float2 a2 = make_float2((float)(int32_t)r[jj], (float)(int32_t)r[jj + 1]);
+            const __nv_bfloat162 y = __float22bfloat162_rn(__ffma2_rn(a2, s2, c2));
+            yb[jj / 2] = *reinterpret_cast<const uint32_t*>(&y);
+          }
+          if (lane == 0) dev::bulk_wait_all_read();
+          __syncwarp();
+#pragma unroll
+          for (int jj = 0; jj < 32; jj += 2) {
+            *reinterpret_cast<uint16_t*>(stg + jj * 64 + lane * 2) = (uint16_t)(yb[jj / 2] & 0xFFFFu);
+            *reinterpret_cast<uint16_t*>(stg + (jj + 1) * 64 + lane * 2) = (uint16_t)(yb[jj / 2] >> 16);
+          }
+          dev::fence_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            dev::tma_store_2d(&tm_y, dev::smem_u32(stg), o0 + q * 32, t0 + c * 32);
+            dev::bulk_commit();
+          }
+        }
+      }
+      dev::named_bar(1, NEPI);   // s_tok of this tile is no longer read
+    }
+    if (lane == 0) dev::bulk_wait_all();
+  }
+
+  dev::tc_fence_before();
+  dev::cluster_sync();  // no MMA, remote arrive or TMEM access of either CTA is still pending
+  if (warp == W_MMA) {
+    dev::tc_fence_after();
+    dev::tmem_dealloc_pair(tmem, TCOLS);
+  }
+}
+
+oq_status run_a8s(const GemmArgs& g, const GemmParams& p, cudaStream_t s) {
+  using namespace sa;
+  CUtensorMap tx, ty;
+  bool ok = true;
+  if (!g.out_acc)
+    ok &= make_map_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.out, (uint64_t)g.N, (uint64_t)g.T,
+                      (uint64_t)g.N * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE);
+  else
+    std::memset(&ty, 0, sizeof(ty));
+  ok &= make_map_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.a, (uint64_t)g.K, (uint64_t)g.T,
+                    (uint64_t)g.K, 128, XR, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!ok) return fail(OQ_ERR_CUDA, "cuTensorMapEncodeTiled failed or unavailable");
+  auto kern = &k_gemm_a8s;
+  const cudaError_t attr_err = allow_max_dynamic_smem(reinterpret_cast<const void*>(kern));
+  if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute(gemm_a8s)");
+  const int pairs = active_pairs_n(reinterpret_cast<const void*>(kern), SMEM, NTHR);
+  if (pairs <= 0) return fail(OQ_ERR_UNSUPPORTED, "gemm: no CTA pair fits on this device");
+  const int64_t chunks = ((g.N + 2 * BM - 1) / (2 * BM)) * ((g.T + CH - 1) / CH);
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3((unsigned)(2 * std::min<int64_t>(chunks, pairs)));
+  cfg.blockDim = dim3(NTHR);
+  cfg.dynamicSmemBytes = SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const uint8_t* wpk = g.w;
+  const cudaError_t le = cudaLaunchKernelEx(&cfg, kern, tx, ty, wpk, p);
+  if (le != cudaSuccess) return cuda_fail(le, "launch gemm_a8s");
+  return OQ_OK;
+}
+
 uint16_t f16_bits(float f) {
   const __half h = __float2half_rn(f);
   return *reinterpret_cast<const uint16_t*>(&h);
@@ -1467,7 +1851,7 @@ oq_status launch_gemm(const GemmArgs& g, cudaStream_t s) {
   // up to 128 tokens: single CTAs on 128-channel tiles; beyond: CTA pairs on 256 channels
   const bool small = g.T <= 128;
   switch (g.kind) {
-    case kGemmA8: return small ? run<kGemmA8, 1>(g, p, s) : run_a8t(g, p, s);
+    case kGemmA8: return small ? run<kGemmA8, 1>(g, p, s) : run_a8s(g, p, s);
     case kGemmA4: return small ? run<kGemmA4, 1>(g, p, s) : run<kGemmA4, 2>(g, p, s);
     case kGemmLloydMax:
       return small ? run<kGemmLloydMax, 1>(g, p, s) : run<kGemmLloydMax, 2>(g, p, s);
