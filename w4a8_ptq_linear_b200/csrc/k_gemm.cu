@@ -1446,8 +1446,11 @@ oq_status run_a8t(const GemmArgs& g, const GemmParams& p, cudaStream_t s) {
 // Schedule: as in the tensor-memory variant, every CTA pair takes an equal contiguous range of
 // the (channel tile, 32-token chunk) space, cut into tiles of at most 256 tokens.
 //
-// Warps: 0 activation producer, 1 TMEM owner + MMA issuer, 2-3 idle, 4-11 converters in two
-// groups of four that take alternate K blocks, 12-19 epilogue (two per TMEM lane quarter).
+// Warps: 1 TMEM owner + MMA issuer, 5 activation producer, eight converters in two groups of
+// four that take alternate K blocks, 12-19 epilogue (two per TMEM lane quarter), 9 and 11 idle.
+// A warp's scheduler is warp % 4: the single MMA thread shares its scheduler only with the
+// producer and the two epilogue warps of lane quarter 1; the converters (warps 0, 2-4, 6-8, 10)
+// use the other three schedulers, so that their work never delays an MMA issue.
 namespace sa {
 constexpr int BN = 256;              // tokens per tile at most (MMA N)
 constexpr int MAXCH = BN / CH;
@@ -1466,7 +1469,15 @@ constexpr int NBAR = 3 * SK + 4 + 1;
 constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
 constexpr int SMEM = OFF_MISC + 16 + 1024;
 constexpr int NTHR = 640;
-constexpr int W_PROD_X = 0, W_MMA = 1, W_CONV0 = 4, W_EPI0 = 12;
+constexpr int W_PROD_X = 5, W_MMA = 1, W_EPI0 = 12;
+// converter index (0..7) of a warp, -1 for the other roles
+__device__ __forceinline__ int conv_index(int w) {
+  switch (w) {
+    case 0: return 0; case 2: return 1; case 3: return 2; case 4: return 3;
+    case 6: return 4; case 7: return 5; case 8: return 6; case 10: return 7;
+    default: return -1;
+  }
+}
 static_assert(WT % 1024 == 0 && XT % 1024 == 0 && OFF_X % 1024 == 0, "stage alignment");
 static_assert(SMEM <= 232448, "shared memory");
 static_assert(NTHR == (W_EPI0 * 32 + NEPI), "warp roles");
@@ -1620,14 +1631,14 @@ __global__ void __launch_bounds__(sa::NTHR, 1)
         dev::mbar_wait(drain_bar, 0, p.err, kSiteGemmDrain, p.limit_ns);
       }
     }
-  } else if (warp >= W_CONV0 && warp < W_EPI0) {
+  } else if (conv_index(warp) >= 0) {
     // ---------------- converters: packed weights (L2) -> int8 16 n -> shared memory -------
     // Group g takes the K blocks j = g, g + 2, ... Thread ctid of a group takes 16-byte packed
     // group q = ctid & 3 of rows r0 + 32 i (r0 = ctid >> 2, i = 0..3): its low nibbles become
     // chunk 2q and its high nibbles chunk 2q + 1 of the row's 128 widened bytes, stored at
     // chunk index ^ (row & 7) (the 128-byte swizzle), the same for every i.
-    const int grp = (warp - W_CONV0) >> 2;
-    const int ctid = ((warp - W_CONV0) & 3) * 32 + lane;
+    const int grp = conv_index(warp) >> 2;
+    const int ctid = (conv_index(warp) & 3) * 32 + lane;
     const int r0 = ctid >> 2, q = ctid & 3;
     const int ph = r0 & 7;
     const int64_t kbytes = p.K / 2;                  // packed bytes per weight row
