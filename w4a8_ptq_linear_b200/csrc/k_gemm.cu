@@ -1446,8 +1446,10 @@ oq_status run_a8t(const GemmArgs& g, const GemmParams& p, cudaStream_t s) {
 // Schedule: as in the tensor-memory variant, every CTA pair takes an equal contiguous range of
 // the (channel tile, 32-token chunk) space, cut into tiles of at most 256 tokens.
 //
-// Warps: 1 TMEM owner + MMA issuer, 5 activation producer, eight converters in two groups of
-// four that take alternate K blocks, 12-19 epilogue (two per TMEM lane quarter), 9 and 11 idle.
+// Warps: 1 TMEM owner + MMA issuer, 5 activation producer, eight converters in four groups of
+// two that take every fourth K block (four K blocks convert at once: a conversion is bound by
+// the latency of its L2 loads, the stores and the hand-off, not by its work), 12-19 epilogue
+// (two per TMEM lane quarter), 9 and 11 idle.
 // A warp's scheduler is warp % 4: the single MMA thread shares its scheduler only with the
 // producer and the two epilogue warps of lane quarter 1; the converters (warps 0, 2-4, 6-8, 10)
 // use the other three schedulers, so that their work never delays an MMA issue.
@@ -1534,7 +1536,7 @@ __global__ void __launch_bounds__(sa::NTHR, 1)
   if (tid == 0) {
     for (int s = 0; s < SK; ++s) {
       dev::mbar_init(xfull_bar(s), 1);
-      dev::mbar_init(wready_bar(s), 2 * 4);  // four converter warps of each CTA
+      dev::mbar_init(wready_bar(s), 2 * 2);  // two converter warps of each CTA
       dev::mbar_init(kfree_bar(s), 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -1633,26 +1635,28 @@ __global__ void __launch_bounds__(sa::NTHR, 1)
     }
   } else if (conv_index(warp) >= 0) {
     // ---------------- converters: packed weights (L2) -> int8 16 n -> shared memory -------
-    // Group g takes the K blocks j = g, g + 2, ... Thread ctid of a group takes 16-byte packed
-    // group q = ctid & 3 of rows r0 + 32 i (r0 = ctid >> 2, i = 0..3): its low nibbles become
+    // Group g takes the K blocks j = g, g + 4, ... Thread ctid of a group takes 16-byte packed
+    // group q = ctid & 3 of rows r0 + 16 i (r0 = ctid >> 2, i = 0..7): its low nibbles become
     // chunk 2q and its high nibbles chunk 2q + 1 of the row's 128 widened bytes, stored at
     // chunk index ^ (row & 7) (the 128-byte swizzle), the same for every i.
-    const int grp = conv_index(warp) >> 2;
-    const int ctid = (conv_index(warp) & 3) * 32 + lane;
+    constexpr int NCG_A = 64, RS = 16, NRI = BM / RS;   // threads per group, row step, rows
+    const int grp = conv_index(warp) >> 1;
+    const int ctid = (conv_index(warp) & 1) * 32 + lane;
     const int r0 = ctid >> 2, q = ctid & 3;
     const int ph = r0 & 7;
     const int64_t kbytes = p.K / 2;                  // packed bytes per weight row
+    static_assert(NCG_A / 4 == RS, "one pass of a group covers RS rows");
     KWalk wk(p.T, n_o, unit_index, n_units, nkb);
-    if (grp == 1) wk.advance();
+    for (int g = 0; g < grp; ++g) wk.advance();
     bool ok = true;
-    for (uint32_t j = (uint32_t)grp; ok && wk.live; j += 2) {
+    for (uint32_t j = (uint32_t)grp; ok && wk.live; j += 4) {
       const int kb = (wk.step + k_rotation(wk.m, nkb)) % nkb;
       const int o0 = wk.m * UNIT + (int)rank * BM;
       const int64_t col = (int64_t)kb * 64 + q * 16;
-      uint4 in[4];
+      uint4 in[NRI];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int o = o0 + r0 + 32 * i;
+      for (int i = 0; i < NRI; ++i) {
+        const int o = o0 + r0 + RS * i;
         in[i] = (o < p.N && col < kbytes)
                     ? __ldg(reinterpret_cast<const uint4*>(wpk + (int64_t)o * kbytes + col))
                     : make_uint4(0u, 0u, 0u, 0u);
@@ -1668,8 +1672,8 @@ __global__ void __launch_bounds__(sa::NTHR, 1)
       }
       uint8_t* dst = w_stage(c);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        uint8_t* rowp = dst + (r0 + 32 * i) * 128;
+      for (int i = 0; i < NRI; ++i) {
+        uint8_t* rowp = dst + (r0 + RS * i) * 128;
         *reinterpret_cast<uint4*>(rowp + (((2 * q) ^ ph) << 4)) =
             make_uint4((in[i].x << 4) & 0xF0F0F0F0u, (in[i].y << 4) & 0xF0F0F0F0u,
                        (in[i].z << 4) & 0xF0F0F0F0u, (in[i].w << 4) & 0xF0F0F0F0u);
@@ -1680,8 +1684,7 @@ __global__ void __launch_bounds__(sa::NTHR, 1)
       dev::fence_async_smem();   // this thread's stores -> visible to the tensor cores
       __syncwarp();
       if (lane == 0) dev::mbar_arrive_cluster(lead(wready_bar(c)));
-      wk.advance();
-      wk.advance();
+      for (int g = 0; g < 4; ++g) wk.advance();
     }
   } else if (warp >= W_EPI0) {
     // ---------------- epilogue ----------------
