@@ -85,6 +85,8 @@ constexpr int EPW = NEPI / 128;               // epilogue warps per TMEM lane qu
 constexpr int EPI0 = CONV0 + NCONV;  // first epilogue thread
 constexpr int NTHREADS = EPI0 + NEPI;
 
+constexpr int kMaxPairs = 160;   // CTA pairs a balanced schedule describes at most
+
 template <int KIND, int CG>
 struct Cfg {
   static constexpr bool FP = KIND == kGemmLloydMax || KIND == kGemmLloydMax8 ||
@@ -142,6 +144,9 @@ struct GemmParams {
   const uint32_t* w_sz;  // grouped weights: [K/64][N] words, fp16 sigma (low half), z (high)
   unsigned long long* err;
   unsigned long long limit_ns;
+  // balanced schedules: CTA pair u takes the flattened (channel tile, 32-token chunk) range
+  // [sched[u], sched[u + 1])
+  int sched[kMaxPairs + 1];
 };
 
 // ---- schedule ----------------------------------------------------------------------------------
@@ -998,70 +1003,19 @@ oq_status run(const GemmArgs& g, const GemmParams& p, cudaStream_t s) {
   return OQ_OK;
 }
 
-// ================================================================================================
-// W4A8 with the widened weights in tensor memory (CTA pairs, T > 128).
-//
-// The weight operand is the MMA's A; tcgen05.mma reads A from tensor memory as well as from
-// shared memory. Here the converter warps widen each 128-byte K block of their CTA's 128 weight
-// rows in registers (one row per thread: the thread's TMEM lane) and store it with tcgen05.st
-// into one of SA weight stages in TMEM, so the widened weights never pass through shared memory:
-// per K block and SM, shared memory carries only the packed weights (TMA write + converter read,
-// 16 KB) and the activations (TMA write + MMA read, 2 x 16 KB).
-//
-// Pipeline depth. The completion of an MMA reaches an mbarrier (tcgen05.commit) several hundred
-// nanoseconds after the tensor pipe finishes it, and a stage can only be refilled after that
-// arrive; with four stages in flight the MMA issue rate halves. So TMEM holds one accumulator
-// of BN = 256 columns and SA = 8 weight stages (2.3 us of MMA work at the N = 256 rate), and the
-// activation ring has as many stages. One commit per K block frees both the weight stage and
-// the activation stage of that block. The accumulator is not double-buffered: the next tile's
-// MMAs wait until the epilogue warps have read it (each releases it after its last
-// tcgen05.ld, before that chunk's stores), a fraction of a microsecond per tile of 24 K blocks.
-//
-// Schedule: the work is the flattened (channel tile, 32-token chunk) space; every CTA pair takes
-// an equal contiguous range of it and cuts its range, within each channel tile, into tiles of
-// at most BN tokens, as even as possible. All pairs then carry the same MMA work (within one
-// chunk), with no partial last wave.
-//
-// Warps: 0 packed-weight producer, 1 TMEM owner + MMA issuer, 2 activation producer, 3 idle,
-// 4-11 converters in two groups (warps 4-7 and 8-11, each covering the four TMEM lane quarters)
-// that take alternate K blocks, 12-19 epilogue (two per lane quarter).
+// ---- balanced schedule of the CTA-pair GEMM -----------------------------------------------------
 namespace ta {
-constexpr int BN = 256;              // tokens per tile at most (MMA N)
-constexpr int MAXCH = BN / CH;       // 32-token chunks per tile at most
-constexpr int XR = BN / 2;           // activation rows per CTA and stage
-constexpr int SK = 8;                // K-block stages: weight stages in TMEM and activation ring
-constexpr int SP = 8;                // packed weight ring
-constexpr int ACOL = BN;             // TMEM column of weight stage 0 (after the accumulator)
-constexpr int TCOLS = 512;           // TMEM columns allocated
-constexpr int XT = XR * 128;         // activation stage bytes (128-byte swizzled rows)
-constexpr int WP = BM * 64;          // packed weight stage bytes (64-byte swizzled rows)
-constexpr int STG = 32 * 32 * 2;     // bf16 [32 tokens][32 channels] staging tile per warp
-// (NEPI = 256 epilogue threads, EPW = 2 per lane quarter, as in k_gemm)
-constexpr int OFF_X = 0;
-constexpr int OFF_P = OFF_X + SK * XT;
-constexpr int OFF_STG = OFF_P + SP * WP;
-constexpr int OFF_TOK = OFF_STG + (NEPI / 32) * STG;
-constexpr int OFF_BAR = OFF_TOK + BN * 8;
-constexpr int NBAR = 3 * SK + 2 * SP + 2 + 1;
-constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-constexpr int SMEM = OFF_MISC + 16 + 1024;
-constexpr int NTHR = 640;
-constexpr int W_PROD_P = 0, W_MMA = 1, W_PROD_X = 2, W_CONV0 = 4, W_EPI0 = 12;
-static_assert(ACOL + SK * 32 <= TCOLS, "tensor memory budget");
-static_assert(XT % 1024 == 0 && OFF_P % 1024 == 0 && WP % 1024 == 0, "stage alignment");
-static_assert(SMEM <= 232448, "shared memory");
-static_assert(NTHR == (W_EPI0 * 32 + NEPI), "warp roles");
+constexpr int MAXCH = 256 / CH;      // 32-token chunks per tile at most
 
-// The tiles of one CTA pair: an equal share of the (channel tile, chunk) space, cut at channel
-// tile boundaries and into as-even-as-possible tiles of at most MAXCH chunks. Every role of the
-// pair walks the same sequence.
+// The tiles of one CTA pair: its range [sched[u], sched[u + 1]) of the flattened (channel tile,
+// chunk) space, cut at channel tile boundaries and into as-even-as-possible tiles of at most
+// MAXCH chunks. Every role of the pair walks the same sequence.
 struct RangeIter {
   int cpm, cur, end;
-  __device__ RangeIter(int T, int n_o, int unit, int n_units) {
+  __device__ RangeIter(int T, const int* sched, int unit) {
     cpm = (T + CH - 1) / CH;
-    const long long total = (long long)n_o * cpm;
-    cur = (int)(total * unit / n_units);
-    end = (int)(total * (unit + 1) / n_units);
+    cur = sched[unit];
+    end = sched[unit + 1];
   }
   __device__ bool next(int& m, int& t0, int& nch) {
     if (cur >= end) return false;
@@ -1076,355 +1030,6 @@ struct RangeIter {
   }
 };
 }  // namespace ta
-
-__global__ void __launch_bounds__(ta::NTHR, 1)
-    k_gemm_a8t(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
-               const __grid_constant__ CUtensorMap tm_y, const GemmParams p) {
-  using namespace ta;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  float2* s_tok = reinterpret_cast<float2*>(smem + OFF_TOK);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
-  uint32_t* s_misc = reinterpret_cast<uint32_t*>(smem + OFF_MISC);  // tmem, abort, epi flag
-  volatile uint32_t* s_abort = s_misc + 1;
-
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const uint32_t rank = dev::cluster_ctarank();   // 0 = the pair's leader
-  constexpr int UNIT = 2 * BM;                     // channels per tile
-  const int n_o = (p.N + UNIT - 1) / UNIT;
-  const int nkb = (p.K + 127) / 128;
-  const int unit_index = (int)blockIdx.x / 2, n_units = (int)gridDim.x / 2;
-  auto tiles = [&]() { return RangeIter(p.T, n_o, unit_index, n_units); };
-
-  auto bar = [&](int i) { return dev::smem_u32(&bars[i]); };
-  auto xfull_bar = [&](int s) { return bar(s); };             // activation stage landed
-  auto wready_bar = [&](int s) { return bar(SK + s); };       // weight stage in TMEM
-  auto kfree_bar = [&](int s) { return bar(2 * SK + s); };    // K block s consumed by the MMAs
-  auto pfull_bar = [&](int s) { return bar(3 * SK + s); };
-  auto pempty_bar = [&](int s) { return bar(3 * SK + SP + s); };
-  const uint32_t tfull = bar(3 * SK + 2 * SP), tempty = bar(3 * SK + 2 * SP + 1);
-  const uint32_t drain_bar = bar(3 * SK + 2 * SP + 2);
-  auto x_stage = [&](int s) { return smem + OFF_X + s * XT; };
-  auto p_stage = [&](int s) { return smem + OFF_P + s * WP; };
-  auto lead = [&](uint32_t a) { return dev::map_to_cta(a, 0); };
-
-  if (tid == 0) {
-    for (int s = 0; s < SK; ++s) {
-      dev::mbar_init(xfull_bar(s), 1);
-      dev::mbar_init(wready_bar(s), 2 * 4);  // four converter warps of each CTA
-      dev::mbar_init(kfree_bar(s), 1);
-    }
-    for (int s = 0; s < SP; ++s) {
-      dev::mbar_init(pfull_bar(s), 1);
-      dev::mbar_init(pempty_bar(s), 4);      // the four warps of the converting group
-    }
-    dev::mbar_init(tfull, 1);
-    dev::mbar_init(tempty, 2 * (NEPI / 32));
-    dev::mbar_init(drain_bar, 1);
-    s_misc[1] = 0;
-    dev::fence_mbar_init_cluster();
-  }
-  if (warp == W_PROD_P && lane == 0) {
-    dev::prefetch_tmap(&tm_x);
-    dev::prefetch_tmap(&tm_w);
-  }
-  if (warp == W_EPI0 && lane == 0 && !p.out_acc) dev::prefetch_tmap(&tm_y);
-  if (warp == W_MMA) {
-    dev::tmem_alloc_pair(dev::smem_u32(&s_misc[0]), TCOLS);
-    dev::tmem_relinquish_pair();
-  }
-  dev::tc_fence_before();
-  dev::cluster_sync();   // barrier inits of both CTAs visible before any remote arrive
-  dev::tc_fence_after();
-  const uint32_t tmem = s_misc[0];
-  auto give_up = [&]() { *s_abort = 1; };
-
-  if (warp == W_PROD_P || warp == W_PROD_X) {
-    // ---------------- producers ----------------
-    const bool packed_role = warp == W_PROD_P;
-    if (lane == 0) {
-      const int ns = packed_role ? SP : SK;
-      uint32_t j = 0;
-      bool ok = true;
-      auto it = tiles();
-      int m, t0, nch;
-      while (ok && it.next(m, t0, nch)) {
-        const int o0 = m * UNIT + (int)rank * BM;            // this CTA's weight rows
-        const int x0 = t0 + (int)rank * (nch * CH / 2);      // this CTA's activation rows
-        const int krot = k_rotation(m, nkb);
-        for (int step = 0; step < nkb; ++step, ++j) {
-          const int kb = (step + krot) % nkb;
-          const int s = j % ns;
-          // a packed stage is free once its group has read it; an activation stage once the
-          // MMAs of its K block have completed
-          const uint32_t empty_b = packed_role ? pempty_bar(s) : kfree_bar(s);
-          const uint32_t full_b = packed_role ? pfull_bar(s) : xfull_bar(s);
-          if (*s_abort || !dev::mbar_wait(empty_b, ((j / ns) & 1u) ^ 1u, p.err, kSiteGemmEmpty,
-                                          p.limit_ns)) {
-            give_up();
-            ok = false;
-            break;
-          }
-          if (packed_role) {
-            dev::mbar_arrive_expect_tx(full_b, (uint32_t)WP);
-            dev::tma_load_2d(dev::smem_u32(p_stage(s)), &tm_w, kb * 64, o0, full_b);
-          } else {
-            // both halves complete on the leader's barrier, which expects the bytes of both
-            if (rank == 0) dev::mbar_arrive_expect_tx(full_b, (uint32_t)(2 * XT));
-            dev::tma_load_2d_pair(dev::smem_u32(x_stage(s)), &tm_x, kb * 128, x0, lead(full_b));
-          }
-        }
-      }
-      if (!ok && (packed_role || rank == 0)) {
-        for (uint32_t i = (j >= (uint32_t)ns ? j - ns : 0); i < j; ++i)
-          dev::mbar_wait(packed_role ? pfull_bar(i % ns) : xfull_bar(i % ns), (i / ns) & 1u, p.err,
-                         kSiteGemmDrain, p.limit_ns);
-      }
-    }
-  } else if (warp == W_MMA) {
-    // ---------------- MMA issuer (the leader's lane 0) ----------------
-    if (lane == 0 && rank == 0) {
-      uint32_t j = 0, it_n = 0;
-      bool ok = true, issued = false;
-      auto it = tiles();
-      int m, t0, nch;
-      for (; ok && it.next(m, t0, nch); ++it_n) {
-        const uint32_t idesc = dev::idesc_i8(UNIT, nch * CH);
-        if (*s_abort || !dev::mbar_wait(tempty, (it_n & 1u) ^ 1u, p.err, kSiteGemmAccum,
-                                        p.limit_ns)) {
-          give_up();
-          ok = false;
-          break;
-        }
-        dev::tc_fence_after();
-        for (int step = 0; step < nkb; ++step, ++j) {
-          const int c = j % SK;
-          bool w = !*s_abort &&
-                   dev::mbar_wait(wready_bar(c), (j / SK) & 1u, p.err, kSiteGemmConv, p.limit_ns);
-          if (w) w = dev::mbar_wait(xfull_bar(c), (j / SK) & 1u, p.err, kSiteGemmFull, p.limit_ns);
-          if (!w) {
-            give_up();
-            ok = false;
-            break;
-          }
-          dev::tc_fence_after();
-          const uint32_t at = tmem + (uint32_t)(ACOL + c * 32);
-          const uint32_t bx = dev::smem_u32(x_stage(c));
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            dev::mma_i8_pair_ta(tmem, at + kk * 8, dev::sdesc_sw128(bx + kk * 32), idesc,
-                                (step | kk) != 0);
-          issued = true;
-          dev::mma_commit_pair(kfree_bar(c));
-        }
-        if (!ok) break;
-        dev::mma_commit_pair(tfull);
-      }
-      if (!ok && issued) {  // wait for the MMAs in flight before TMEM is freed
-        dev::mma_commit_pair(drain_bar);
-        dev::mbar_wait(drain_bar, 0, p.err, kSiteGemmDrain, p.limit_ns);
-      }
-    }
-  } else if (warp >= W_CONV0 && warp < W_EPI0) {
-    // ---------------- converters: packed weights -> int8 16 n -> TMEM ----------------
-    // Thread (quarter q, lane l) owns weight row r = 32 q + l, i.e. TMEM lane r. The packed
-    // stage holds 64-byte rows whose four 16-byte groups were swizzled by TMA (group g of row r
-    // at ((g ^ ((r >> 1) & 3)) << 4)), so that the warp's row-wise reads hit distinct banks.
-    // Group g (32 elements) widens to columns 8g..8g+3 (low nibbles, elements 32g..32g+15) and
-    // 8g+4..8g+7 (high nibbles, elements 32g+16..32g+31). The widening happens before the wait
-    // for the weight stage to be free, so that only the TMEM store follows that wait.
-    const int grp = (warp - W_CONV0) >> 2, q = warp & 3;
-    const int r = q * 32 + lane;
-    const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
-    uint32_t j = 0;
-    bool ok = true;
-    auto it = tiles();
-    int m, t0, nch;
-    while (ok && it.next(m, t0, nch)) {
-      for (int step = 0; step < nkb; ++step, ++j) {
-        if ((int)(j & 1u) != grp) continue;
-        const int s = j % SP, c = j % SK;
-        bool w = !*s_abort &&
-                 dev::mbar_wait(pfull_bar(s), (j / SP) & 1u, p.err, kSiteGemmFull, p.limit_ns);
-        w = __all_sync(0xffffffffu, w);
-        if (!w) {
-          give_up();
-          ok = false;
-          break;
-        }
-        const uint8_t* row = p_stage(s) + r * 64;
-        const int ph = (r >> 1) & 3;
-        uint32_t o[32];
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const uint4 in = *reinterpret_cast<const uint4*>(row + ((g ^ ph) << 4));
-          o[8 * g + 0] = (in.x << 4) & 0xF0F0F0F0u;
-          o[8 * g + 1] = (in.y << 4) & 0xF0F0F0F0u;
-          o[8 * g + 2] = (in.z << 4) & 0xF0F0F0F0u;
-          o[8 * g + 3] = (in.w << 4) & 0xF0F0F0F0u;
-          o[8 * g + 4] = in.x & 0xF0F0F0F0u;
-          o[8 * g + 5] = in.y & 0xF0F0F0F0u;
-          o[8 * g + 6] = in.z & 0xF0F0F0F0u;
-          o[8 * g + 7] = in.w & 0xF0F0F0F0u;
-        }
-        __syncwarp();              // the warp's reads of the packed stage are done
-        if (lane == 0) dev::mbar_arrive(pempty_bar(s));
-        w = !*s_abort &&
-            dev::mbar_wait(kfree_bar(c), ((j / SK) & 1u) ^ 1u, p.err, kSiteGemmConv, p.limit_ns);
-        w = __all_sync(0xffffffffu, w);
-        if (!w) {
-          give_up();
-          ok = false;
-          break;
-        }
-        dev::tc_fence_after();
-        dev::tmem_st32(tmem + lane_addr + (uint32_t)(ACOL + c * 32), o);
-        dev::tmem_wait_st();
-        dev::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) dev::mbar_arrive_cluster(lead(wready_bar(c)));
-      }
-    }
-  } else if (warp >= W_EPI0) {
-    // ---------------- epilogue ----------------
-    // Each warp releases the accumulator (the next tile's MMAs wait for that) right after its
-    // last tcgen05.ld of the tile, before that chunk's scaling and stores.
-    const int etid = tid - W_EPI0 * 32;
-    uint8_t* stg = smem + OFF_STG + (warp - W_EPI0) * STG;
-    const int q = warp & 3;
-    const int half = (warp - W_EPI0) >> 2;
-    const int o_local = q * 32 + lane;
-    const bool ep_lead = etid == 0;
-    uint32_t it_n = 0;
-    bool ok = true;
-    auto it = tiles();
-    int m, t0, nch;
-    for (; ok && it.next(m, t0, nch); ++it_n) {
-      const int o0 = m * UNIT + (int)rank * BM;
-      const int o = o0 + o_local;
-      const bool has_o = o < p.N;
-      const float sw = has_o ? p.w_scale[o] * (1.f / 16.f) : 0.f;
-      const float w1 = (has_o && p.mean) ? p.w_rowsum[o] : 0.f;
-      const float bb = (has_o && p.bias) ? __bfloat162float(p.bias[o]) : 0.f;
-      const int ncols = nch * CH;
-      for (int i = etid; i < ncols; i += NEPI) {
-        const int t = t0 + i;
-        s_tok[i] = make_float2((t < p.T) ? p.a_scale[t] : 0.f,
-                               (t < p.T && p.mean) ? p.mean[t] : 0.f);
-      }
-      if (ep_lead) {
-        const bool ready = !*s_abort && dev::mbar_wait(tfull, it_n & 1u, p.err,
-                                                       kSiteGemmAccum, p.limit_ns);
-        if (!ready) give_up();
-        s_misc[2] = ready ? 1u : 0u;
-      }
-      dev::named_bar(1, NEPI);
-      ok = *reinterpret_cast<volatile uint32_t*>(&s_misc[2]) != 0;
-      if (ok) dev::tc_fence_after();
-      const int t_end = min(ncols, p.T - t0);
-      const int nmine = (nch - half + EPW - 1) / EPW;   // chunks half, half + EPW, ...
-      if (ok && nmine == 0) {
-        dev::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) dev::mbar_arrive_cluster(lead(tempty));
-      }
-#pragma unroll 1
-      for (int cc = 0; ok && cc < nmine; ++cc) {
-        const int c = half + cc * EPW;
-        uint32_t r[32];
-        dev::tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(c * 32), r);
-        dev::tmem_wait_ld();
-        if (cc == nmine - 1) {   // this warp's part of the accumulator is read: release it
-          dev::tc_fence_before();
-          __syncwarp();
-          if (lane == 0) dev::mbar_arrive_cluster(lead(tempty));
-        }
-        if (o0 + q * 32 >= p.N) continue;
-        const int n_valid = t_end - c * 32;
-        if (p.out_acc) {
-          int32_t* dst = reinterpret_cast<int32_t*>(p.out) + (int64_t)(t0 + c * 32) * p.N + o;
-#pragma unroll
-          for (int jj = 0; jj < 32; ++jj)
-            if (has_o && jj < n_valid) dst[(int64_t)jj * p.N] = (int32_t)r[jj] >> 4;
-        } else {
-          const float4* tk4 = reinterpret_cast<const float4*>(s_tok + c * 32);
-          const float2 sw2 = make_float2(sw, sw), w12 = make_float2(w1, w1);
-          const float2 bb2 = make_float2(bb, bb);
-          uint32_t yb[16];
-#pragma unroll
-          for (int jj = 0; jj < 32; jj += 2) {
-            const float4 tk = tk4[jj / 2];
-            const float2 s2 = __fmul2_rn(make_float2(tk.x, tk.z), sw2);
-            const float2 c2 = __ffma2_rn(make_float2(tk.y, tk.w), w12, bb2);
-            const float2 a2 = make_float2((float)(int32_t)r[jj], (float)(int32_t)r[jj + 1]);
-            const __nv_bfloat162 y = __float22bfloat162_rn(__ffma2_rn(a2, s2, c2));
-            yb[jj / 2] = *reinterpret_cast<const uint32_t*>(&y);
-          }
-          if (lane == 0) dev::bulk_wait_all_read();
-          __syncwarp();
-#pragma unroll
-          for (int jj = 0; jj < 32; jj += 2) {
-            *reinterpret_cast<uint16_t*>(stg + jj * 64 + lane * 2) = (uint16_t)(yb[jj / 2] & 0xFFFFu);
-            *reinterpret_cast<uint16_t*>(stg + (jj + 1) * 64 + lane * 2) = (uint16_t)(yb[jj / 2] >> 16);
-          }
-          dev::fence_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            dev::tma_store_2d(&tm_y, dev::smem_u32(stg), o0 + q * 32, t0 + c * 32);
-            dev::bulk_commit();
-          }
-        }
-      }
-      dev::named_bar(1, NEPI);   // s_tok of this tile is no longer read
-    }
-    if (lane == 0) dev::bulk_wait_all();
-  }
-
-  dev::tc_fence_before();
-  dev::cluster_sync();  // no MMA, remote arrive or TMEM access of either CTA is still pending
-  if (warp == W_MMA) {
-    dev::tc_fence_after();
-    dev::tmem_dealloc_pair(tmem, TCOLS);
-  }
-}
-
-oq_status run_a8t(const GemmArgs& g, const GemmParams& p, cudaStream_t s) {
-  using namespace ta;
-  CUtensorMap tx, tw, ty;
-  bool ok = true;
-  if (!g.out_acc)
-    ok &= make_map_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.out, (uint64_t)g.N, (uint64_t)g.T,
-                      (uint64_t)g.N * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE);
-  else
-    std::memset(&ty, 0, sizeof(ty));
-  ok &= make_map_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.a, (uint64_t)g.K, (uint64_t)g.T,
-                    (uint64_t)g.K, 128, XR, CU_TENSOR_MAP_SWIZZLE_128B);
-  ok &= make_map_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.w, (uint64_t)g.K / 2, (uint64_t)g.N,
-                    (uint64_t)g.K / 2, 64, BM, CU_TENSOR_MAP_SWIZZLE_64B);
-  if (!ok) return fail(OQ_ERR_CUDA, "cuTensorMapEncodeTiled failed or unavailable");
-  auto kern = &k_gemm_a8t;
-  const cudaError_t attr_err = allow_max_dynamic_smem(reinterpret_cast<const void*>(kern));
-  if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute(gemm_a8t)");
-  const int pairs = active_pairs_n(reinterpret_cast<const void*>(kern), SMEM, NTHR);
-  if (pairs <= 0) return fail(OQ_ERR_UNSUPPORTED, "gemm: no CTA pair fits on this device");
-  const int64_t chunks = ((g.N + 2 * BM - 1) / (2 * BM)) * ((g.T + CH - 1) / CH);
-  cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3((unsigned)(2 * std::min<int64_t>(chunks, pairs)));
-  cfg.blockDim = dim3(NTHR);
-  cfg.dynamicSmemBytes = SMEM;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  const cudaError_t le = cudaLaunchKernelEx(&cfg, kern, tx, tw, ty, p);
-  if (le != cudaSuccess) return cuda_fail(le, "launch gemm_a8t");
-  return OQ_OK;
-}
 
 // ================================================================================================
 // W4A8 with the widened weights in shared memory and double-buffered accumulators (CTA pairs,
@@ -1443,8 +1048,9 @@ oq_status run_a8t(const GemmArgs& g, const GemmParams& p, cudaStream_t s) {
 // keep the pipe fed; one commit per K block frees both stages of that block. TMEM holds two
 // accumulators of 256 columns, so the epilogue of one tile overlaps the next tile's MMAs.
 //
-// Schedule: as in the tensor-memory variant, every CTA pair takes an equal contiguous range of
-// the (channel tile, 32-token chunk) space, cut into tiles of at most 256 tokens.
+// Schedule: every CTA pair takes a contiguous range of the (channel tile, 32-token chunk) space,
+// cut into tiles of at most 256 tokens; the host chooses the ranges so that the largest
+// per-pair cost (chunks plus a fixed cost per tile) is as small as possible (balance_ranges).
 //
 // Warps: 1 TMEM owner + MMA issuer, 5 activation producer, eight converters in four groups of
 // two that take every fourth K block (four K blocks convert at once: a conversion is bound by
@@ -1455,7 +1061,6 @@ oq_status run_a8t(const GemmArgs& g, const GemmParams& p, cudaStream_t s) {
 // use the other three schedulers, so that their work never delays an MMA issue.
 namespace sa {
 constexpr int BN = 256;              // tokens per tile at most (MMA N)
-constexpr int MAXCH = BN / CH;
 constexpr int XR = BN / 2;           // activation rows per CTA and stage
 constexpr int SK = 6;                // K-block stages: widened weights and activations
 constexpr int WT = BM * 128;         // widened weight stage bytes
@@ -1490,8 +1095,8 @@ struct KWalk {
   ta::RangeIter rit;
   int m = 0, t0 = 0, nch = 0, step = 0, nkb;
   bool live;
-  __device__ KWalk(int T, int n_o, int unit, int n_units, int nkb_)
-      : rit(T, n_o, unit, n_units), nkb(nkb_) {
+  __device__ KWalk(int T, const int* sched, int unit, int nkb_)
+      : rit(T, sched, unit), nkb(nkb_) {
     live = rit.next(m, t0, nch);
   }
   __device__ void advance() {
@@ -1517,10 +1122,9 @@ __global__ void __launch_bounds__(sa::NTHR, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = dev::cluster_ctarank();   // 0 = the pair's leader
   constexpr int UNIT = 2 * BM;                     // channels per tile
-  const int n_o = (p.N + UNIT - 1) / UNIT;
   const int nkb = (p.K + 127) / 128;
-  const int unit_index = (int)blockIdx.x / 2, n_units = (int)gridDim.x / 2;
-  auto tiles = [&]() { return ta::RangeIter(p.T, n_o, unit_index, n_units); };
+  const int unit_index = (int)blockIdx.x / 2;
+  auto tiles = [&]() { return ta::RangeIter(p.T, p.sched, unit_index); };
 
   auto bar = [&](int i) { return dev::smem_u32(&bars[i]); };
   auto xfull_bar = [&](int s) { return bar(s); };             // activation stage landed
@@ -1646,7 +1250,7 @@ __global__ void __launch_bounds__(sa::NTHR, 1)
     const int ph = r0 & 7;
     const int64_t kbytes = p.K / 2;                  // packed bytes per weight row
     static_assert(NCG_A / 4 == RS, "one pass of a group covers RS rows");
-    KWalk wk(p.T, n_o, unit_index, n_units, nkb);
+    KWalk wk(p.T, p.sched, unit_index, nkb);
     for (int g = 0; g < grp; ++g) wk.advance();
     bool ok = true;
     for (uint32_t j = (uint32_t)grp; ok && wk.live; j += 4) {
@@ -1788,8 +1392,59 @@ __global__ void __launch_bounds__(sa::NTHR, 1)
   }
 }
 
-oq_status run_a8s(const GemmArgs& g, const GemmParams& p, cudaStream_t s) {
+// The CTA pairs' ranges of the flattened (channel tile, 32-token chunk) space. A range costs
+// its chunks plus kTileCost for every tile it is cut into (at most maxch chunks, never across a
+// channel tile): a tile's K loop costs nearly the same whatever its width (measured: the issue
+// loop, not the tensor pipe, sets the time per K block), so the tile count dominates and a cut
+// that would add a narrow tile is avoided. The largest cost over the pairs is minimised by
+// bisection on a bound C with a greedy cover that stretches every range while its cost stays
+// within C. Computed once per shape.
+constexpr int kTileCost = 8;
+
+void balance_ranges(int n_o, int cpm, int pairs, int maxch, int* starts) {
+  static std::mutex mu;
+  static std::map<std::tuple<int, int, int, int>, std::vector<int>> cache;
+  std::lock_guard<std::mutex> lock(mu);
+  const auto key = std::make_tuple(n_o, cpm, pairs, maxch);
+  auto it = cache.find(key);
+  if (it == cache.end()) {
+    const int64_t total = (int64_t)n_o * cpm;
+    // cost of [a, b): chunks + kTileCost * tiles, tiles counted per channel-tile piece
+    auto cover = [&](int64_t cmax, std::vector<int>* out) {
+      int64_t pos = 0;
+      for (int u = 0; u < pairs; ++u) {
+        if (out) (*out)[u] = (int)pos;
+        int64_t cost = 0, end = pos;
+        while (end < total) {
+          // extend by one chunk: a new tile starts at a channel-tile boundary or after maxch
+          // chunks of the current piece
+          const int64_t m = end / cpm, piece_start = std::max(pos, m * cpm);
+          const int64_t len = end - piece_start;            // chunks of this piece so far
+          const int64_t add = 1 + ((len % maxch == 0) ? kTileCost : 0);
+          if (cost + add > cmax) break;
+          cost += add;
+          ++end;
+        }
+        pos = end;
+      }
+      if (out) (*out)[pairs] = (int)total;
+      return pos >= total;
+    };
+    int64_t lo = 1 + kTileCost, hi = total + kTileCost * (total + maxch - 1) / maxch + 1;
+    while (lo < hi) {
+      const int64_t mid = (lo + hi) / 2;
+      if (cover(mid, nullptr)) hi = mid; else lo = mid + 1;
+    }
+    std::vector<int> v((size_t)pairs + 1);
+    cover(lo, &v);
+    it = cache.emplace(key, std::move(v)).first;
+  }
+  std::copy(it->second.begin(), it->second.end(), starts);
+}
+
+oq_status run_a8s(const GemmArgs& g, const GemmParams& p_in, cudaStream_t s) {
   using namespace sa;
+  GemmParams p = p_in;
   CUtensorMap tx, ty;
   bool ok = true;
   if (!g.out_acc)
@@ -1803,11 +1458,15 @@ oq_status run_a8s(const GemmArgs& g, const GemmParams& p, cudaStream_t s) {
   auto kern = &k_gemm_a8s;
   const cudaError_t attr_err = allow_max_dynamic_smem(reinterpret_cast<const void*>(kern));
   if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute(gemm_a8s)");
-  const int pairs = active_pairs_n(reinterpret_cast<const void*>(kern), SMEM, NTHR);
+  int pairs = active_pairs_n(reinterpret_cast<const void*>(kern), SMEM, NTHR);
   if (pairs <= 0) return fail(OQ_ERR_UNSUPPORTED, "gemm: no CTA pair fits on this device");
-  const int64_t chunks = ((g.N + 2 * BM - 1) / (2 * BM)) * ((g.T + CH - 1) / CH);
+  const int n_o = (int)((g.N + 2 * BM - 1) / (2 * BM));
+  const int cpm = (int)((g.T + CH - 1) / CH);
+  const int64_t chunks = (int64_t)n_o * cpm;
+  pairs = (int)std::min<int64_t>(std::min<int64_t>(chunks, pairs), kMaxPairs);
+  balance_ranges(n_o, cpm, pairs, BN / CH, p.sched);
   cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3((unsigned)(2 * std::min<int64_t>(chunks, pairs)));
+  cfg.gridDim = dim3((unsigned)(2 * pairs));
   cfg.blockDim = dim3(NTHR);
   cfg.dynamicSmemBytes = SMEM;
   cfg.stream = s;
