@@ -1072,7 +1072,7 @@ constexpr int OFF_X = OFF_W + SK * WT;
 constexpr int OFF_STG = OFF_X + SK * XT;
 constexpr int OFF_TOK = OFF_STG + (NEPI / 32) * STG;
 constexpr int OFF_BAR = OFF_TOK + BN * 8;
-constexpr int NBAR = 3 * SK + 4 + 1;
+constexpr int NBAR = 2 * SK + 4 + 1;
 constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
 constexpr int SMEM = OFF_MISC + 16 + 1024;
 constexpr int NTHR = 640;
@@ -1126,22 +1126,23 @@ __global__ void __launch_bounds__(sa::NTHR, 1)
   const int unit_index = (int)blockIdx.x / 2;
   auto tiles = [&]() { return ta::RangeIter(p.T, p.sched, unit_index); };
 
+  // ready[s]: K block s is in place, i.e. both activation halves landed (TMA bytes on the
+  // leader's barrier, armed by the leader's producer) and the four converter warps of the pair
+  // stored its widened weights: one wait per K block for the MMA thread
   auto bar = [&](int i) { return dev::smem_u32(&bars[i]); };
-  auto xfull_bar = [&](int s) { return bar(s); };             // activation stage landed
-  auto wready_bar = [&](int s) { return bar(SK + s); };       // widened weight stage stored
-  auto kfree_bar = [&](int s) { return bar(2 * SK + s); };    // K block s consumed by the MMAs
-  auto tfull_bar = [&](int b) { return bar(3 * SK + b); };
-  auto tempty_bar = [&](int b) { return bar(3 * SK + 2 + b); };
-  const uint32_t drain_bar = bar(3 * SK + 4);
+  auto ready_bar = [&](int s) { return bar(s); };
+  auto kfree_bar = [&](int s) { return bar(SK + s); };        // K block s consumed by the MMAs
+  auto tfull_bar = [&](int b) { return bar(2 * SK + b); };
+  auto tempty_bar = [&](int b) { return bar(2 * SK + 2 + b); };
+  const uint32_t drain_bar = bar(2 * SK + 4);
   auto w_stage = [&](int s) { return smem + OFF_W + s * WT; };
   auto x_stage = [&](int s) { return smem + OFF_X + s * XT; };
   auto lead = [&](uint32_t a) { return dev::map_to_cta(a, 0); };
 
   if (tid == 0) {
     for (int s = 0; s < SK; ++s) {
-      dev::mbar_init(xfull_bar(s), 1);
-      dev::mbar_init(wready_bar(s), 2 * 2);  // two converter warps of each CTA
-      dev::mbar_init(kfree_bar(s), 1);
+      dev::mbar_init(ready_bar(s), 1 + 2 * 2);  // the leader's producer + two converter warps
+      dev::mbar_init(kfree_bar(s), 1);           // of each CTA
     }
     for (int b = 0; b < 2; ++b) {
       dev::mbar_init(tfull_bar(b), 1);
@@ -1183,13 +1184,16 @@ __global__ void __launch_bounds__(sa::NTHR, 1)
             break;
           }
           // both halves complete on the leader's barrier, which expects the bytes of both
-          if (rank == 0) dev::mbar_arrive_expect_tx(xfull_bar(s), (uint32_t)(2 * XT));
-          dev::tma_load_2d_pair(dev::smem_u32(x_stage(s)), &tm_x, kb * 128, x0, lead(xfull_bar(s)));
+          if (rank == 0) dev::mbar_arrive_expect_tx(ready_bar(s), (uint32_t)(2 * XT));
+          dev::tma_load_2d_pair(dev::smem_u32(x_stage(s)), &tm_x, kb * 128, x0, lead(ready_bar(s)));
         }
       }
+      // after an abort the landed bytes of the loads in flight can no longer be told apart from
+      // the converters' arrivals: wait (bounded) for the stages' completions, which also covers
+      // the bytes; a stage whose converter arrivals never come gives up at the time limit
       if (!ok && rank == 0) {
         for (uint32_t i = (j >= (uint32_t)SK ? j - SK : 0); i < j; ++i)
-          dev::mbar_wait(xfull_bar(i % SK), (i / SK) & 1u, p.err, kSiteGemmDrain, p.limit_ns);
+          dev::mbar_wait(ready_bar(i % SK), (i / SK) & 1u, p.err, kSiteGemmDrain, p.limit_ns);
       }
     }
   } else if (warp == W_MMA) {
@@ -1213,8 +1217,7 @@ __global__ void __launch_bounds__(sa::NTHR, 1)
         for (int step = 0; step < nkb; ++step, ++j) {
           const int c = j % SK;
           const uint32_t par = (j / SK) & 1u;
-          if (!dev::mbar_wait(wready_bar(c), par, p.err, kSiteGemmConv, p.limit_ns) ||
-              !dev::mbar_wait(xfull_bar(c), par, p.err, kSiteGemmFull, p.limit_ns)) {
+          if (!dev::mbar_wait(ready_bar(c), par, p.err, kSiteGemmFull, p.limit_ns)) {
             give_up();
             ok = false;
             break;
@@ -1287,7 +1290,7 @@ __global__ void __launch_bounds__(sa::NTHR, 1)
       }
       dev::fence_async_smem();   // this thread's stores -> visible to the tensor cores
       __syncwarp();
-      if (lane == 0) dev::mbar_arrive_cluster(lead(wready_bar(c)));
+      if (lane == 0) dev::mbar_arrive_cluster(lead(ready_bar(c)));
       for (int g = 0; g < 4; ++g) wk.advance();
     }
   } else if (warp >= W_EPI0) {
