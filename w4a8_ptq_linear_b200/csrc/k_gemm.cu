@@ -1214,24 +1214,36 @@ __global__ void __launch_bounds__(sa::NTHR, 1)
         }
         dev::tc_fence_after();
         const uint32_t dt = tmem + (uint32_t)(b * BN);
-        for (int step = 0; step < nkb; ++step, ++j) {
-          const int c = j % SK;
-          const uint32_t par = (j / SK) & 1u;
-          if (!dev::mbar_wait(ready_bar(c), par, p.err, kSiteGemmFull, p.limit_ns)) {
+        // two K blocks per iteration: the waits, the fence and the loop overhead of the single
+        // issuing thread are paid once for eight MMAs (the tensor pipe idles while it runs them)
+        for (int step = 0; step < nkb; step += 2, j += 2) {
+          const int nb = min(2, nkb - step);
+          const int c0 = j % SK, c1 = (j + 1) % SK;
+          if (!dev::mbar_wait(ready_bar(c0), (j / SK) & 1u, p.err, kSiteGemmFull, p.limit_ns) ||
+              (nb == 2 && !dev::mbar_wait(ready_bar(c1), ((j + 1) / SK) & 1u, p.err,
+                                          kSiteGemmFull, p.limit_ns))) {
             give_up();
             ok = false;
             break;
           }
           dev::tc_fence_after();
-          const uint32_t aw = dev::smem_u32(w_stage(c));
-          const uint32_t bx = dev::smem_u32(x_stage(c));
+          const uint32_t aw0 = dev::smem_u32(w_stage(c0)), bx0 = dev::smem_u32(x_stage(c0));
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            dev::mma_i8_pair(dt, dev::sdesc_sw128(aw + kk * 32), dev::sdesc_sw128(bx + kk * 32),
+            dev::mma_i8_pair(dt, dev::sdesc_sw128(aw0 + kk * 32), dev::sdesc_sw128(bx0 + kk * 32),
                              idesc, (step | kk) != 0);
           issued = true;
-          dev::mma_commit_pair(kfree_bar(c));
+          dev::mma_commit_pair(kfree_bar(c0));
+          if (nb == 2) {
+            const uint32_t aw1 = dev::smem_u32(w_stage(c1)), bx1 = dev::smem_u32(x_stage(c1));
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              dev::mma_i8_pair(dt, dev::sdesc_sw128(aw1 + kk * 32),
+                               dev::sdesc_sw128(bx1 + kk * 32), idesc, 1);
+            dev::mma_commit_pair(kfree_bar(c1));
+          }
         }
+        if (ok) j -= (uint32_t)(((nkb + 1) / 2) * 2 - nkb);   // an odd K loop used one block less
         if (!ok) break;
         dev::mma_commit_pair(tfull_bar(b));
       }
