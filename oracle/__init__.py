@@ -27,7 +27,8 @@ from .rpbh import (splitmix64_at, rpbh_plan, sylvester_hadamard, rotate, unrotat
 from .lloyd_max import (lloyd_max_gaussian, lloyd_max_gaussian_8bit, lloyd_max_mse,
                         lloyd_max_sphere, sphere_marginal)
 from .quant import (EPS, PCT_RHO, PCT_GAMMA, center, absmax_quantize, lloyd_max_quantize,
-                    percentile_quantize, pack_nibbles, unpack_nibbles)
+                    percentile_quantize, pack_nibbles, unpack_nibbles, pack_pairs,
+                    unpack_pairs)
 from .linear import (quantize_activations, prepare_weights, gemm_int, gemm_lloyd_max,
                      epilogue, linear_forward, linear_unquantized)
 
@@ -37,7 +38,7 @@ __all__ = [
     "lloyd_max_mse", "lloyd_max_sphere",
     "sphere_marginal", "EPS", "center",
     "absmax_quantize", "lloyd_max_quantize", "percentile_quantize", "PCT_RHO", "PCT_GAMMA",
-    "pack_nibbles", "unpack_nibbles",
+    "pack_nibbles", "unpack_nibbles", "pack_pairs", "unpack_pairs",
     "quantize_activations", "prepare_weights", "gemm_int", "gemm_lloyd_max", "epilogue",
     "linear_forward", "linear_unquantized",
 ]

@@ -7,6 +7,8 @@ What the pages fix:
   from the unquantized weight (here in float64).
 - CentriQ §4.2, Eq. 5 and App. B.2, Eq. 9: y_t = W_hat Q_a(Q x_t^c) + mean_t * w_1 + b, with
   the rank-1 term and the bias added in the GEMM epilogue.
+- W4A2 (CentriQ App. C.1, Tab. 4): the same layer with b = 2 activations (percentile range,
+  grid {-1, 0, 1}); the integer GEMM and the epilogue are unchanged.
 - Weights: symmetric INT4 per output channel on the pre-rotated weight W_R = W Q^T
   (grid {-7..7}, CentriQ Eq. 1 applied to the rows of W_R; the task fixes per-channel INT4).
 
@@ -48,6 +50,8 @@ def quantize_activations(x: np.ndarray, plan, h: int, act: str, center_tokens: b
         codes, scale = lloyd_max_quantize(z, thresholds)
     elif act == "int4_percentile":
         codes, scale = percentile_quantize(z, 7)
+    elif act == "int2_percentile":
+        codes, scale = percentile_quantize(z, 1)       # b = 2: grid {-1, 0, 1}
     else:
         raise ValueError(act)
     return {"rotated": z, "codes": codes, "scale": scale, "mean": mean}

@@ -227,3 +227,29 @@ def test_grouped_dequantize_and_correction_mistakes_are_caught(monkeypatch):
     monkeypatch.setattr(Gm, "corrected_product",
                         lambda a, q, s, z, g=Gm.GROUP: _corr_ok(a, q, s, z + 8.0, g))
     assert _fails(lambda: (TG.test_zero_point_correction_identity(), True)[1])
+
+
+def test_a2_mistakes_are_caught(monkeypatch):
+    # the 2-bit packing with the element order reversed inside a byte
+    def bad_pack(v):
+        v = np.asarray(v, dtype=np.int64) & 0x3
+        return (v[..., 3::4] | (v[..., 2::4] << 2) | (v[..., 1::4] << 4)
+                | (v[..., 0::4] << 6)).astype(np.uint8)
+    with monkeypatch.context() as m:
+        m.setattr(Qm, "pack_pairs", bad_pack)
+        assert _fails(TQ.check_pairs)
+    # the layer's A2 kind on the b-bit count 2^b - 1 = 3 instead of 2^(b-1) - 1 = 1
+    real = Lm.percentile_quantize
+    with monkeypatch.context() as m:
+        m.setattr(Lm, "percentile_quantize", lambda z, qmax: real(z, 3 if qmax == 1 else qmax))
+        assert _fails(TQ.check_layer_a2)
+    # a ternary threshold at alpha instead of alpha / 2 (a floor instead of a rounding)
+    def bad_pct(z, qmax, rho=Qm.PCT_RHO, gamma=Qm.PCT_GAMMA, eps=Qm.EPS):
+        z = np.asarray(z, dtype=np.float64)
+        q = np.quantile(np.abs(z), rho, axis=1)
+        alpha = np.maximum(gamma * q / Qm.ndtri((1.0 + rho) / 2.0), eps) / qmax
+        c = np.clip(np.trunc(z / alpha[:, None]), -qmax, qmax).astype(np.int64)
+        return c, alpha
+    with monkeypatch.context() as m:
+        m.setattr(Qm, "percentile_quantize", bad_pct)
+        assert _fails(TQ.check_ternary, np.random.default_rng(8).standard_normal((4, 1024)) * 2.0)

@@ -174,3 +174,69 @@ def test_percentile_clips_outliers():
     assert s[k] <= quantile <= s[k + 2]
     assert q[0, 17] == 7
     assert q.min() >= -7 and q.max() <= 7
+
+
+# ---- A2: the b = 2 grid of CentriQ Eq. 1 (W4A2, App. C.1 Tab. 4; Tab. 3 scale) ----------------
+
+def check_pairs():
+    """2-bit packing: hand-written bytes and a round trip."""
+    v = np.array([[1, 0, -1, 0, -1, -1, -1, -1, 0, 1, 0, 1]])
+    b = [[0b00110001, 0xFF, 0b01000100]]
+    ok = Qm.pack_pairs(v).tolist() == b
+    ok &= Qm.unpack_pairs(np.array(b, np.uint8)).tolist() == v.tolist()
+    s = np.random.default_rng(5).integers(-1, 2, (5, 64))
+    ok &= bool(np.array_equal(Qm.unpack_pairs(Qm.pack_pairs(s)), s))
+    return ok
+
+
+def check_ternary(z):
+    """qmax = 1: the nearest point of {-1, 0, 1} is sign(z) where |z| > alpha / 2, else 0
+    (round half to even sends |z| = alpha / 2 to 0), and alpha is gamma sigma_hat itself."""
+    q, alpha = Qm.percentile_quantize(z, 1)
+    _, alpha7 = Qm.percentile_quantize(z, 7)
+    ref = np.where(np.abs(z) > alpha[:, None] / 2, np.sign(z), 0).astype(np.int64)
+    return bool(np.allclose(alpha, 7 * alpha7, rtol=1e-15) and np.array_equal(q, ref))
+
+
+def check_layer_a2():
+    """The layer oracle's A2 kind: percentile codes on the grid {-1, 0, 1}."""
+    from oracle import linear as L, rpbh_plan
+    x = np.random.default_rng(9).standard_normal((3, 256)) + 2.0
+    qa = L.quantize_activations(x, rpbh_plan(256, 64, 1, 0), 64, "int2_percentile", True)
+    q, a = Qm.percentile_quantize(qa["rotated"], 1)
+    return bool(set(np.unique(qa["codes"])) <= {-1, 0, 1} and np.array_equal(q, qa["codes"])
+                and np.allclose(a, qa["scale"], rtol=0))
+
+
+def test_pack_pairs():
+    # element 4j + i in bits 2i, 2i + 1 of byte j, two's complement (-1 = 0b11)
+    assert check_pairs()
+    with pytest.raises(ValueError):
+        Qm.pack_pairs(np.zeros((1, 6), np.int64))
+
+
+@pytest.mark.parametrize("n", [256, 3072])
+def test_ternary_percentile_definition(n):
+    # qmax = 1: the same quantile and clip (Tab. 3 is one setting for every b), grid {-1, 0, 1}
+    z = np.random.default_rng(n + 1).standard_normal((5, n)) * np.array([[0.5], [1], [3], [7], [1e-3]])
+    assert check_percentile(z, qmax=1)
+
+
+def test_ternary_codes_closed_form():
+    rng = np.random.default_rng(8)
+    assert check_ternary(rng.standard_normal((4, 1024)) * 2.0)
+    # exact half steps go to 0, and anything past 1.5 alpha clips to +-1: two of the smallest
+    # magnitudes become +-alpha / 2 and one becomes an outlier; alpha / 2 lies far below the
+    # quantile's order statistics, so alpha only moves with the outlier (by one rank)
+    z2 = rng.standard_normal((1, 4000))
+    small = np.argsort(np.abs(z2[0]))[:3]
+    z2[0, small[2]] = 1e3
+    _, a = Qm.percentile_quantize(z2, 1)
+    z2[0, small[0]], z2[0, small[1]] = a[0] / 2, -a[0] / 2
+    q2, a2 = Qm.percentile_quantize(z2, 1)
+    assert a2[0] == a[0]
+    assert q2[0, small[0]] == 0 and q2[0, small[1]] == 0 and q2[0, small[2]] == 1
+
+
+def test_layer_oracle_accepts_a2():
+    assert check_layer_a2()
