@@ -40,7 +40,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "rotate+quantize GB/s (% of HBM peak); W4A8/W4A4 linear TOPS (% tensor peak)"
-RING = 4
+RING = 4            # independent input sets at least; more when a set is small (see ring_size)
+L2_BYTES = 126 << 20   # B200 L2
 # nominal dense int8 / bf16 tensor throughput ratio on B200 (4.5 / 2.25 PFLOP/s), for the
 # peak the measured bf16 GEMM figure implies (reported beside the measured tcgen05 peak)
 INT8_PER_BF16 = 2.0
@@ -66,7 +67,9 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="dit_w4a8",
                     choices=["tiny", "dit_w4a8", "dit_lm8", "narrow_lm", "narrow_lm_w", "mlp_up",
-                             "mlp_up_pct", "mlp_up_g64"])
+                             "mlp_up_pct", "mlp_up_a2", "mlp_up_g64"])
+    ap.add_argument("--fused", action="store_true",
+                    help="time the single-launch layer (oq_linear_fused; INT8 absmax, T <= 256)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="override the token count (small cases for profiler captures)")
     ap.add_argument("--e2e-steps", type=int, default=100)
@@ -267,19 +270,38 @@ def run_reference(args, wl, rank):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
-            "config": config_of(wl, wl.T, args.gpus),
+            "config": config_of(wl, args.tokens or wl.T, args.gpus, fused=args.fused),
             "cpu_baseline": {"value": v, "unit": "TOPS", "cores": blas_threads(),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": v, "unit": "TOPS", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 
 
-def config_of(wl, T, n):
-    return {"workload": wl.name, "T": T, "d_in": wl.d, "d_out": wl.n_out, "h": wl.h,
-            "rounds": wl.rounds, "act": wl.act, "center": wl.center,
-            "weights": "int4" if wl.weights == "int4_channel" else wl.weights,
-            "l2": f"inputs rotate over {RING} sets larger than L2 together",
-            "parallelism": "replicas" if n == 1 else f"dp{n} (tokens split, no collective)"}
+def set_bytes(wl, T):
+    """Device bytes of one input set: activations, prepared weights, codes, scales, output."""
+    code = (T * wl.d if wl.act.startswith("int8")
+            else T * wl.d // 4 if wl.act.startswith("int2") else T * wl.d // 2)
+    return T * wl.d * 2 + wl.n_out * wl.d // 2 + 12 * wl.n_out + code + 8 * T + T * wl.n_out * 2
+
+
+def ring_size(wl, T, l2_bytes):
+    """Input sets the timed steps rotate over: at least RING, and together at least twice the
+    L2, so that every step reads its weights and activations from HBM as a layer of a real
+    model would (capped at 256 sets)."""
+    return int(min(256, max(RING, -(-2 * l2_bytes // set_bytes(wl, T)))))
+
+
+def config_of(wl, T, n, ring=None, l2_bytes=L2_BYTES, fused=False):
+    ring = ring_size(wl, T, l2_bytes) if ring is None else ring
+    c = {"workload": wl.name, "T": T, "d_in": wl.d, "d_out": wl.n_out, "h": wl.h,
+         "rounds": wl.rounds, "act": wl.act, "center": wl.center,
+         "weights": "int4" if wl.weights == "int4_channel" else wl.weights,
+         "l2": (f"inputs rotate over {ring} sets, {ring * set_bytes(wl, T) / 1e6:.0f} MB "
+                f"together, larger than the {l2_bytes / 1e6:.0f} MB L2"),
+         "parallelism": "replicas" if n == 1 else f"dp{n} (tokens split, no collective)"}
+    if fused:
+        c["path"] = "single launch (oq_linear_fused)"
+    return c
 
 
 # ---- GPU leg ---------------------------------------------------------------------------------
@@ -455,10 +477,14 @@ def main():
     plan = oq.Plan(wl.d, wl.h, wl.rounds, seed=wl.seed, center=wl.center, act=wl.act)
     to_dev = lambda b: torch.from_numpy(np.ascontiguousarray(b)).view(torch.bfloat16).to(dev)
 
-    # RING independent sets: activations, prepared weights, codes, scales, outputs
+    # independent sets: activations, prepared weights, codes, scales, outputs
+    ring = ring_size(wl, T, L2_BYTES)
+    fused = args.fused
+    if fused and (wl.act != "int8_absmax" or g64 or T > 256):
+        raise SystemExit("--fused takes INT8 absmax workloads with per-channel weights, T <= 256")
     sets = []
     x_host_bits = None
-    for r in range(RING):
+    for r in range(ring):
         xb = synth.make_x(T, wl.d, mean_var=wl.mean_var, heavy_frac=wl.heavy_frac,
                           outliers=wl.outliers, outlier_gain=wl.outlier_gain,
                           seed=input_seed(wl.seed, rank, r))
@@ -472,27 +498,39 @@ def main():
             wp, ws, w1 = oq.prepare_weights(plan, w)
         del w
         s = {"x": to_dev(xb), "wp": wp, "ws": ws, "w1": w1, "wsz": wsz,
-             "codes": torch.empty((T, wl.d // 2 if plan.packed else wl.d),
+             "codes": torch.empty((T, plan.code_row_bytes),
                                   dtype=torch.int8 if wl.act == "int8_absmax" else torch.uint8,
                                   device=dev),
              "scale": torch.empty(T, dtype=torch.float32, device=dev),
              "mean": torch.empty(T, dtype=torch.float32, device=dev) if wl.center else None,
              "y": torch.empty((T, wl.n_out), dtype=torch.bfloat16, device=dev)}
+        if fused:
+            s["wsb"] = torch.empty(max(plan.workspace_bytes(T), 256), dtype=torch.uint8,
+                                   device=dev)
         sets.append(s)
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
 
     def step(s, st):
+        if fused:   # the whole layer in one launch
+            oq.linear_fused(plan, s["x"], s["wp"], s["ws"], s["w1"] if wl.center else None,
+                            workspace=s["wsb"], out=s["y"], stream=st)
+            return
         oq.rotate_quantize(plan, s["x"], codes=s["codes"], scale=s["scale"], mean=s["mean"],
                            stream=st)
 
     def gemm(s, st):
+        if fused:
+            return
         if g64:
             oq.gemm_w4a4_g64(wl.act, s["codes"], s["scale"], s["wp"], s["wsz"], s["ws"],
                              mean=s["mean"], w_rowsum=s["w1"] if wl.center else None, out=s["y"],
                              stream=st)
         elif wl.act == "int8_absmax":
             oq.gemm_w4a8(s["codes"], s["scale"], s["wp"], s["ws"], mean=s["mean"],
+                         w_rowsum=s["w1"] if wl.center else None, out=s["y"], stream=st)
+        elif wl.act == "int2_percentile":
+            oq.gemm_w4a2(s["codes"], s["scale"], s["wp"], s["ws"], mean=s["mean"],
                          w_rowsum=s["w1"] if wl.center else None, out=s["y"], stream=st)
         elif wl.act == "int8_lloydmax":
             oq.gemm_w4a8_lloydmax(plan, s["codes"], s["scale"], s["wp"], s["ws"], mean=s["mean"],
@@ -504,7 +542,7 @@ def main():
                          stream=st)
 
     for i in range(max(3, args.warmup)):
-        s = sets[i % RING]
+        s = sets[i % ring]
         step(s, stream)
         gemm(s, stream)
     torch.cuda.synchronize()
@@ -513,7 +551,7 @@ def main():
         raise RuntimeError(f"device status {st} code {code:#x} after warm-up")
 
     # The timed steps replay CUDA graphs of the library's launches, so that no host-side launch
-    # gap falls between the kernels: g_ring holds the RING steps in order, g_one[r] one step.
+    # gap falls between the kernels: g_ring holds the ring's steps in order, g_one[r] one step.
     cap_stream = torch.cuda.Stream(device=dev)
 
     def capture(calls):
@@ -529,7 +567,7 @@ def main():
     g_ring = capture([(f, s) for s in sets for f in (step, gemm)])
     g_one = [capture([(step, s), (gemm, s)]) for s in sets]
     g_rq = capture([(step, s) for s in sets])        # the two kernels alone, for their
-    g_gm = capture([(gemm, s) for s in sets])        # average duration per launch
+    g_gm = None if fused else capture([(gemm, s) for s in sets])   # average duration per launch
     for _ in range(2):
         g_ring.replay()
     torch.cuda.synchronize()
@@ -546,9 +584,9 @@ def main():
         t_start = torch.cuda.Event(enable_timing=True)
         t_end = torch.cuda.Event(enable_timing=True)
         t_start.record(stream)
-        for _ in range(K // RING):
+        for _ in range(K // ring):
             g_ring.replay()
-        for r in range(K % RING):
+        for r in range(K % ring):
             g_one[r].replay()
         t_end.record(stream)
         torch.cuda.synchronize()
@@ -556,7 +594,7 @@ def main():
     elapsed_ms = t_start.elapsed_time(t_end)
 
     def per_launch(g):
-        reps = max(1, -(-K // RING))
+        reps = max(1, -(-K // ring))
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
@@ -564,10 +602,10 @@ def main():
             g.replay()
         e1.record(stream)
         torch.cuda.synchronize()
-        return e0.elapsed_time(e1) / (reps * RING)
+        return e0.elapsed_time(e1) / (reps * ring)
 
     rq_ms = per_launch(g_rq)
-    gm_ms = per_launch(g_gm)
+    gm_ms = per_launch(g_gm) if g_gm is not None else 0.0
     st, code = oq.device_status()
     if st != 0:
         raise RuntimeError(f"device status {st} code {code:#x} after timing")
@@ -607,8 +645,9 @@ def main():
                           s0["w1"] if wl.center else None, workspace=workspace, out=y_devs[k],
                           stream=stream)
         else:
-            oq.linear(plan, x_devs[k], s0["wp"], s0["ws"], s0["w1"] if wl.center else None,
-                      workspace=workspace, out=y_devs[k], stream=stream)
+            layer = oq.linear_fused if fused else oq.linear
+            layer(plan, x_devs[k], s0["wp"], s0["ws"], s0["w1"] if wl.center else None,
+                  workspace=workspace, out=y_devs[k], stream=stream)
         ev_done[k].record(stream)
         s_out.wait_event(ev_done[k])
         with torch.cuda.stream(s_out):
@@ -641,7 +680,8 @@ def main():
     ops = 2.0 * T * wl.d * wl.n_out
     ms_per_step = elapsed_ms / K
     value = whole_job_rate(ops, world, ms_per_step) / 1e12
-    code_bytes = T * wl.d if wl.act.startswith("int8") else T * wl.d // 2
+    code_bytes = (T * wl.d if wl.act.startswith("int8")
+                  else T * wl.d // 4 if wl.act.startswith("int2") else T * wl.d // 2)
     rq_bytes = T * wl.d * 2 + code_bytes + 4 * T * (2 if wl.center else 1)
     peaks, peak_kind = load_peaks()
     long_region = elapsed_ms > 1000.0
@@ -654,7 +694,7 @@ def main():
     loop_kind = "f16" if fp_gemm else "i8"
     tensor_peak, loop_ms = measured_mma_peak(oq, loop_kind, stream)
     hbm_peak = peaks["hbm_gbs"]
-    gemm_tops = ops / (gm_ms * 1e-3) / 1e12
+    gemm_tops = ops / (max(gm_ms, 1e-9) * 1e-3) / 1e12
     rq_gbs = rq_bytes / (rq_ms * 1e-3) / 1e9
     kfile = os.path.join(ROOT, "w4a8_ptq_linear_b200", "csrc", "k_gemm.cu")
     tr = NCU_TRAFFIC.get((wl.name, "k_gemm"))
@@ -679,20 +719,38 @@ def main():
                "algorithmic_bytes": rq_bytes}
     dominant = gemm_roof if gm_ms >= rq_ms else rq_roof
     other = rq_roof if dominant is gemm_roof else gemm_roof
+    shares = {"k_rotate_quant": rq_ms / (rq_ms + gm_ms), "k_gemm": gm_ms / (rq_ms + gm_ms)}
+    if fused:
+        # one kernel does everything: its HBM floor is reading x and the packed weights and
+        # writing y and the workspace's codes, scales and means once
+        layer_bytes = (T * wl.d * 2 + wl.n_out * wl.d // 2 + wl.n_out * 4 * (2 if wl.center else 1)
+                       + T * wl.n_out * 2 + code_bytes + 4 * T * (2 if wl.center else 1))
+        f_gbs = layer_bytes / (rq_ms * 1e-3) / 1e9
+        f_tops = ops / (rq_ms * 1e-3) / 1e12
+        dominant = {"bound": "hbm", "achieved": f_gbs, "peak": hbm_peak, "unit": "GB/s",
+                    "frac": f_gbs / hbm_peak, "traffic": None, "kernel": "k_linear_fused",
+                    "peak_source": f"{peak_kind} copy bandwidth", "ms_per_launch": rq_ms,
+                    "algorithmic_bytes": layer_bytes}
+        other = {"bound": "tensor", "achieved": f_tops, "peak": tensor_peak, "unit": "TOPS",
+                 "frac": f_tops / tensor_peak, "kernel": "k_linear_fused",
+                 "peak_source": peak_note, "ms_per_launch": rq_ms}
+        shares = {"k_linear_fused": 1.0}
     line = {
         "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "int8" if not fp_gemm else "f16", "data": "synthetic", "config": config_of(wl, T, world),
-        "rotate_quantize_gbs": rq_gbs, "rotate_quantize_frac_hbm": rq_gbs / hbm_peak,
-        "gemm_tops": gemm_tops, "gemm_frac_tensor": gemm_tops / tensor_peak,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8" if not fp_gemm else "f16",
+        "data": "synthetic", "config": config_of(wl, T, world, ring, fused=fused),
+        "rotate_quantize_gbs": None if fused else rq_gbs,
+        "rotate_quantize_frac_hbm": None if fused else rq_gbs / hbm_peak,
+        "gemm_tops": None if fused else gemm_tops,
+        "gemm_frac_tensor": None if fused else gemm_tops / tensor_peak,
         "timing": "steps and per-kernel averages replay CUDA graphs of the library's launches",
         "roofline": dominant, "roofline_other": other,
-        "kernel_share": {"k_rotate_quant": rq_ms / (rq_ms + gm_ms),
-                         "k_gemm": gm_ms / (rq_ms + gm_ms)},
+        "kernel_share": shares,
         "e2e": {"value": whole_job_rate(ops, world, e2e_ms) / 1e12, "unit": "TOPS",
                 "h2d_bytes_per_step": T * wl.d * 2, "d2h_bytes_per_step": T * wl.n_out * 2,
                 "ms_per_step": e2e_ms, "steps": args.e2e_steps},
-        "gpu_launches": 2 * K,
+        "gpu_launches": (1 if fused else 2) * K,
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -35,6 +35,8 @@
  *   - 4-bit activation codes: uint8 [rows, d/2], element 2j in bits 0-3 of byte j and
  *     element 2j+1 in bits 4-7; absmax codes are two's-complement nibbles in -7..7,
  *     Lloyd-Max codes are indices 0..15 into the ascending codebook;
+ *   - 2-bit activation codes (A2): uint8 [rows, d/4], element 4j + i in bits 2i, 2i + 1 of
+ *     byte j, two's complement in -1..1;
  *   - prepared INT4 weights (the GEMM layout): uint8 [d_out, d_in/2] of two's-complement
  *     nibbles in -7..7; every row is split into 16-byte groups, and byte j of group g holds
  *     element 32g + j in bits 0-3 and element 32g + 16 + j in bits 4-7. The GEMM widens a
@@ -75,7 +77,8 @@ typedef enum {
   OQ_ACT_INT4_LLOYDMAX = 2,  /* A4: sigma_t = RMS(z_t), nearest of 16 N(0,1) centroids   */
   OQ_ACT_INT4_PERCENTILE = 3, /* A4: percentile range (below), codes clipped to -7..7    */
   OQ_ACT_INT4_LLOYDMAX_WIDTH = 4, /* A4: as LLOYDMAX with the width-d codebook (below)   */
-  OQ_ACT_INT8_LLOYDMAX = 5   /* A8: sigma_t = RMS(z_t), nearest of 256 N(0,1) centroids  */
+  OQ_ACT_INT8_LLOYDMAX = 5,  /* A8: sigma_t = RMS(z_t), nearest of 256 N(0,1) centroids  */
+  OQ_ACT_INT2_PERCENTILE = 6 /* A2: percentile range, codes clipped to -1..1 (below)      */
 } oq_act_kind;
 /* OQ_ACT_INT8_LLOYDMAX (OrbitQuant PR #25 "Default changes": the 8-bit Lloyd-Max activations
  * that absmax INT8 replaced as the A8 default): codes are uint8 [T, d] indices 0..255 into the
@@ -95,6 +98,15 @@ typedef enum {
  * codes = clip(round(z / alpha_t), -7, 7). The codes and the GEMM are those of
  * OQ_ACT_INT4_ABSMAX; only the scale differs. Limit: d <= 8192 (the quantile needs the
  * d - floor(rho (d - 1)) <= 6 largest magnitudes, kept per thread). */
+
+/* OQ_ACT_INT2_PERCENTILE (CentriQ Eq. 1 with b = 2, the activation grid of its W4A2 results,
+ * App. C.1 Tab. 4; scale of App. B.3 Tab. 3, which is one setting for every b): the range of
+ * OQ_ACT_INT4_PERCENTILE, alpha_t = max(gamma sigma_hat_t, 1e-10) / 1, and
+ * codes = clip(round(z / alpha_t), -1, 1), i.e. sign(z) where |z| > alpha_t / 2, else 0.
+ * Codes are uint8 [T, d/4]: element 4j + i in bits 2i, 2i + 1 of byte j, two's complement
+ * (-1 = 0b11). The pages only simulate 2-bit activations (CentriQ §7: no fused kernel supports
+ * them yet), so this storage is the library's own. GEMM: oq_gemm_w4a2. Limits: d <= 8192 (as
+ * the percentile scale) and d % 64 == 0 (a token's codes are whole 16-byte rows). */
 
 typedef enum {
   OQ_OUT_BF16 = 0,           /* dequantised, rank-1 and bias added, rounded to bf16      */
@@ -186,8 +198,8 @@ oq_status oq_plan_get_codebook(const oq_plan* plan, int levels, double* centroid
  * App. B.2, where one prologue centers each token, rotates it and quantizes it with one scale
  * per token; OrbitQuant PR #25 "Runtime work": the pre-rotation runs as a single kernel).
  *   x_bf16       [T, ldx] bf16, ldx >= d, (ldx * 2) % 16 == 0
- *   codes        int8 [T, d] (A8 absmax), uint8 [T, d] (8-bit Lloyd-Max) or uint8 [T, d/2]
- *                (A4 kinds)
+ *   codes        int8 [T, d] (A8 absmax), uint8 [T, d] (8-bit Lloyd-Max), uint8 [T, d/2]
+ *                (A4 kinds) or uint8 [T, d/4] (A2)
  *   scale        float [T]: alpha_t (absmax kinds) or sigma_t (Lloyd-Max)
  *   mean         float [T] per-token mean; required iff the plan centers, else ignored
  *   rotated_f32  float [T, d] normalised rotated (centered) values, or NULL (test output) */
@@ -274,6 +286,17 @@ oq_status oq_gemm_w4a4_g64(oq_act_kind kind, const uint8_t* a_packed, const floa
                            int64_t T, int64_t d_in, int64_t d_out, oq_out_kind out_kind,
                            void* out, void* stream);
 
+/* W4A2 GEMM (CentriQ App. C.1: W4A2) for OQ_ACT_INT2_PERCENTILE codes, same epilogue as
+ * oq_gemm_w4a8:
+ *   acc[t,o] = sum_k a[t,k] * w[o,k]    (a in -1..1, w in -7..7; exact int32)
+ *   a_packed  uint8 [T, d_in/4] (four codes per byte, see OQ_ACT_INT2_PERCENTILE)
+ *   d_in      a multiple of 64 (else OQ_ERR_INVALID_ARG)
+ *   other arguments and out as for oq_gemm_w4a8. */
+oq_status oq_gemm_w4a2(const uint8_t* a_packed, const float* a_scale, const float* mean,
+                       const uint8_t* w_packed, const float* w_scale, const float* w_rowsum,
+                       const void* bias_bf16, int64_t T, int64_t d_in, int64_t d_out,
+                       oq_out_kind out_kind, void* out, void* stream);
+
 /* W4A8 GEMM for 8-bit Lloyd-Max codes (OQ_ACT_INT8_LLOYDMAX), same epilogue with
  * a_scale = sigma_t:
  *   acc[t,o] = sum_k c[codes[t,k]] * w[o,k]    (fp16 centroids and weights, fp32 accumulation)
@@ -297,6 +320,20 @@ oq_status oq_linear(const oq_plan* plan, const void* x_bf16, int64_t T, int64_t 
                     const uint8_t* w_packed, const float* w_scale, const float* w_rowsum,
                     const void* bias_bf16, int64_t d_out, void* y_bf16, void* workspace,
                     size_t workspace_bytes, void* stream);
+
+/* The whole layer in ONE launch, for small token counts (CentriQ App. B.2: the activation path
+ * runs as the prologue of the INT4 GEMM). Same arguments, workspace and result as oq_linear,
+ * bit for bit: the kernel first rotates and quantizes the tokens into `workspace` (every CTA takes a
+ * share of the token pairs), passes one grid-wide barrier, then runs a split-K GEMM in which a
+ * cluster of CTAs shares each 128-channel tile and adds its int32 partial sums through
+ * distributed shared memory before the epilogue.
+ * Limits: the plan's kind must be OQ_ACT_INT8_ABSMAX and d <= 8192 with d % 128 == 0;
+ * 1 <= T <= 256; the channel tiles' clusters must all fit on the device at once (the launch is
+ * cooperative). Outside them it returns OQ_ERR_UNSUPPORTED and launches nothing. */
+oq_status oq_linear_fused(const oq_plan* plan, const void* x_bf16, int64_t T, int64_t ldx,
+                          const uint8_t* w_packed, const float* w_scale, const float* w_rowsum,
+                          const void* bias_bf16, int64_t d_out, void* y_bf16, void* workspace,
+                          size_t workspace_bytes, void* stream);
 
 /* oq_linear against asymmetric grouped weights: oq_rotate_quantize into `workspace`, then
  * oq_gemm_w4a4_g64. The plan's activation kind must be OQ_ACT_INT4_ABSMAX or

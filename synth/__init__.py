@@ -67,7 +67,7 @@ class Workload:
     h: int
     rounds: int
     act: str            # "int8_absmax" | "int4_absmax" | "int4_lloydmax" | "int4_percentile"
-                        # | "int4_lloydmax_width" | "int8_lloydmax"
+                        # | "int4_lloydmax_width" | "int8_lloydmax" | "int2_percentile"
     center: bool
     mean_var: float     # variance of the per-token mean offset
     outliers: int = 0   # channels scaled by outlier_gain (tiny workload)
@@ -95,6 +95,8 @@ WORKLOADS = {
     # the same layer with CentriQ's percentile per-token scale (§4.2 "Scale and grid")
     "mlp_up_pct": Workload("mlp_up_pct", 4096, 3072, 12288, 1024, 1, "int4_percentile", True,
                            5.0),
+    # the same layer with 2-bit activations (CentriQ's W4A2: grid {-1, 0, 1}, percentile scale)
+    "mlp_up_a2": Workload("mlp_up_a2", 4096, 3072, 12288, 1024, 1, "int2_percentile", True, 5.0),
     # the same layer with CentriQ's weight format: asymmetric INT4 groups of 64 columns (§4.3)
     "mlp_up_g64": Workload("mlp_up_g64", 4096, 3072, 12288, 1024, 1, "int4_absmax", True, 5.0,
                            weights="int4_g64"),

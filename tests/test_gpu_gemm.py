@@ -62,6 +62,35 @@ def test_w4a4_absmax_accumulators_bit_exact(T, K, N):
     assert np.array_equal(acc.cpu().numpy().astype(np.int64), ref)
 
 
+@pytest.mark.parametrize("T,K,N", SHAPES)
+def test_w4a2_accumulators_bit_exact(T, K, N):
+    import torch
+    import w4a8_ptq_linear_b200 as oq
+    rng = np.random.default_rng(5 * T + K + N)
+    a, w = _codes(rng, T, K, N, 1)
+    a[1, :] = -1
+    w[1, :] = -7
+    ap = torch.from_numpy(oracle.pack_pairs(a)).cuda()
+    wp = torch.from_numpy(pack_w4_gemm(w)).cuda()
+    ones = torch.ones(max(T, N), dtype=torch.float32, device="cuda")
+    acc = oq.gemm_w4a2(ap, ones[:T], wp, ones[:N], out_kind=oq.OUT_ACC)
+    torch.cuda.synchronize()
+    assert oq.device_status()[0] == 0
+    ref = oracle.gemm_int(a, w).astype(np.int64)
+    assert np.array_equal(acc.cpu().numpy().astype(np.int64), ref)
+
+
+def test_w4a2_rejects_width_not_multiple_of_64():
+    import torch
+    import w4a8_ptq_linear_b200 as oq
+    ap = torch.zeros((8, 24), dtype=torch.uint8, device="cuda")     # K = 96
+    wp = torch.zeros((16, 48), dtype=torch.uint8, device="cuda")
+    ones = torch.ones(16, dtype=torch.float32, device="cuda")
+    with pytest.raises(oq.OQError) as e:
+        oq.gemm_w4a2(ap, ones[:8], wp, ones, out_kind=oq.OUT_ACC)
+    assert e.value.status == oq.OQ_ERR_INVALID_ARG
+
+
 @pytest.mark.parametrize("T,K,N", [(64, 256, 256), (200, 384, 272), (130, 1920, 1920),
                                    (2560, 1536, 2560)])
 def test_lloyd_max_accumulators(T, K, N):
@@ -85,14 +114,15 @@ def test_lloyd_max_accumulators(T, K, N):
     plan.close()
 
 
-@pytest.mark.parametrize("kind", ["int8_absmax", "int4_absmax", "int4_lloydmax"])
+@pytest.mark.parametrize("kind", ["int8_absmax", "int4_absmax", "int4_lloydmax",
+                                  "int2_percentile"])
 @pytest.mark.parametrize("with_mean,with_bias", [(False, False), (True, True), (True, False)])
 def test_epilogue_matches_oracle(kind, with_mean, with_bias):
     import torch
     import w4a8_ptq_linear_b200 as oq
     T, K, N = 260, 512, 384
     rng = np.random.default_rng(11)
-    amax = 127 if kind == "int8_absmax" else 7
+    amax = {"int8_absmax": 127, "int2_percentile": 1}.get(kind, 7)
     if kind == "int4_lloydmax":
         a = rng.integers(0, 16, (T, K))
     else:
@@ -111,6 +141,10 @@ def test_epilogue_matches_oracle(kind, with_mean, with_bias):
     wp = cuda(pack_w4_gemm(w))
     if kind == "int8_absmax":
         y = oq.gemm_w4a8(cuda(a.astype(np.int8)), cuda(scale), wp, cuda(s_w), mean=mean_t,
+                         w_rowsum=w1_t, bias=bias_t)
+        acc = oracle.gemm_int(a, w)
+    elif kind == "int2_percentile":
+        y = oq.gemm_w4a2(cuda(oracle.pack_pairs(a)), cuda(scale), wp, cuda(s_w), mean=mean_t,
                          w_rowsum=w1_t, bias=bias_t)
         acc = oracle.gemm_int(a, w)
     else:

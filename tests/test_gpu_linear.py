@@ -43,7 +43,8 @@ def _gpu_layer(wl, xb, wb, bias_bits=None):
 
 @pytest.mark.parametrize("name,T", [("tiny", 64), ("dit_w4a8", 300), ("dit_lm8", 300),
                                     ("narrow_lm", 257),
-                                    ("narrow_lm_w", 257), ("mlp_up", 130), ("mlp_up_pct", 130)])
+                                    ("narrow_lm_w", 257), ("mlp_up", 130), ("mlp_up_pct", 130),
+                                    ("mlp_up_a2", 130), ("mlp_up_a2", 1)])
 def test_layer_matches_oracle(name, T):
     wl, xb, wb = synth.make_inputs(name, T=T)
     y = _gpu_layer(wl, xb, wb)
@@ -60,7 +61,7 @@ def test_layer_with_bias():
 
 
 @pytest.mark.parametrize("name", ["dit_w4a8", "dit_lm8", "narrow_lm", "narrow_lm_w", "mlp_up",
-                                  "mlp_up_pct"])
+                                  "mlp_up_pct", "mlp_up_a2"])
 def test_full_size_layer_on_sampled_rows(name):
     wl, xb, wb = synth.make_inputs(name)
     y = _gpu_layer(wl, xb, wb)

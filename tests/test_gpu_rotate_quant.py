@@ -44,6 +44,13 @@ CASES = [
     (31, 6144, 1024, 1, "int4_percentile", True),
     (20, 8192, 512, 1, "int4_percentile", True),
     (7, 256, 64, 1, "int4_percentile", False),
+    # 2-bit activations (CentriQ W4A2: the percentile range, grid {-1, 0, 1}, four codes a byte)
+    (257, 3072, 1024, 1, "int2_percentile", True),
+    (130, 1920, 128, 2, "int2_percentile", False),
+    (45, 4096, 256, 2, "int2_percentile", True),
+    (20, 8192, 512, 1, "int2_percentile", True),
+    (7, 256, 64, 1, "int2_percentile", False),
+    (301, 1024, 1, 1, "int2_percentile", False),
     # the width-d Lloyd-Max codebook (codebook v3 tables per width)
     (130, 1920, 128, 2, "int4_lloydmax_width", False),
     (33, 256, 32, 1, "int4_lloydmax_width", True),
@@ -101,6 +108,10 @@ def test_rotate_quantize_matches_oracle(T, d, h, rounds, act, center):
     elif act in ("int4_absmax", "int4_percentile"):
         gpu = oracle.unpack_nibbles(out["codes"], signed=True)
         ex = absmax_boundary_mask(ref["rotated"], ref["scale"], 7)
+    elif act == "int2_percentile":
+        assert out["codes"].shape == (T, d // 4)
+        gpu = oracle.unpack_pairs(out["codes"])
+        ex = absmax_boundary_mask(ref["rotated"], ref["scale"], 1)
     else:
         gpu = oracle.unpack_nibbles(out["codes"], signed=False)
         thr = (oracle.lloyd_max_sphere(d)[1] if act == "int4_lloydmax_width"
@@ -167,7 +178,8 @@ def test_row_pitch_larger_than_width():
     plan.close()
 
 
-def test_percentile_clips_outliers_and_handles_flat_tokens():
+@pytest.mark.parametrize("act", ["int4_percentile", "int2_percentile"])
+def test_percentile_clips_outliers_and_handles_flat_tokens(act):
     # CentriQ §4.2: the percentile range leaves the largest magnitudes past +-7 alpha, which
     # clip to +-7; tokens with few distinct magnitudes exercise ties in the order statistics
     import torch
@@ -182,19 +194,21 @@ def test_percentile_clips_outliers_and_handles_flat_tokens():
     x[3, 5] = 2.0                       # one non-zero channel
     x[4] = np.where(np.arange(d) % 2 == 0, 1.0, -1.0)   # flat magnitudes
     xb = synth.f64_to_bf16(x)
-    plan = oq.Plan(d, h, 1, act="int4_percentile")
+    plan = oq.Plan(d, h, 1, act=act)
     codes, scale, _, rot = oq.rotate_quantize(plan, to_torch_bf16(xb), rotated=True)
     torch.cuda.synchronize()
     ref = oracle.quantize_activations(synth.bf16_to_f64(xb), oracle.rpbh_plan(d, h, 1, 0), h,
-                                      "int4_percentile", False)
+                                      act, False)
+    qmax = 7 if act == "int4_percentile" else 1
     s = scale.cpu().numpy().astype(np.float64)
     nz = ref["scale"] > 1e-9
     assert np.all(np.abs(s[nz] / ref["scale"][nz] - 1) <= ROT_TOL)
     assert np.all(np.abs(s[~nz] - ref["scale"][~nz]) <= 1e-16)
-    gpu = oracle.unpack_nibbles(codes.cpu().numpy(), signed=True)
-    ex = absmax_boundary_mask(ref["rotated"], ref["scale"], 7)
+    gpu = (oracle.unpack_nibbles(codes.cpu().numpy(), signed=True) if qmax == 7
+           else oracle.unpack_pairs(codes.cpu().numpy()))
+    ex = absmax_boundary_mask(ref["rotated"], ref["scale"], qmax)
     bad, _ = compare_codes(gpu, ref["codes"], ex)
     assert bad == 0
-    assert np.abs(gpu[0]).max() == 7 and np.all(gpu[2] == 0)
+    assert np.abs(gpu[0]).max() == qmax and np.all(gpu[2] == 0)
     plan.close()
 

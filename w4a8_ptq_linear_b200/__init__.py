@@ -7,7 +7,7 @@ There is no CPU fallback: if the library is missing, importing works but every c
 call raises ``OQError``.
 
 The function names follow the C ABI: ``rotate_quantize``, ``prepare_weights``,
-``gemm_w4a8``, ``gemm_w4a4``, ``linear`` (oq_rotate_quantize, oq_prepare_weights, ...).
+``gemm_w4a8``, ``gemm_w4a4``, ``gemm_w4a2``, ``linear`` (oq_rotate_quantize, oq_prepare_weights, ...).
 """
 from __future__ import annotations
 
@@ -23,7 +23,7 @@ LIB_PATH = os.path.join(_PKG, "lib", "liboq.so")
 OQ_OK, OQ_ERR_INVALID_ARG, OQ_ERR_UNSUPPORTED, OQ_ERR_MISALIGNED = 0, 1, 2, 3
 OQ_ERR_CUDA, OQ_ERR_DEVICE_TIMEOUT, OQ_ERR_NOMEM = 4, 5, 6
 ACT_KINDS = {"int8_absmax": 0, "int4_absmax": 1, "int4_lloydmax": 2, "int4_percentile": 3,
-             "int4_lloydmax_width": 4, "int8_lloydmax": 5}
+             "int4_lloydmax_width": 4, "int8_lloydmax": 5, "int2_percentile": 6}
 OUT_BF16, OUT_ACC = 0, 1
 
 # (name, restype, argtypes) of every exported entry point
@@ -47,6 +47,7 @@ SIGNATURES = [
     ("oq_prepare_weights", _I, [_P, _P, _I64, _I64, _P, _P, _P, _P]),
     ("oq_gemm_w4a8", _I, [_P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _P, _P]),
     ("oq_gemm_w4a4", _I, [_P, _I, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _P, _P]),
+    ("oq_gemm_w4a2", _I, [_P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _P, _P]),
     ("oq_gemm_w4a8_lloydmax", _I, [_P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _P, _P]),
     ("oq_linear_workspace_bytes", _SZ, [_P, _I64]),
     ("oq_linear", _I, [_P, _P, _I64, _I64, _P, _P, _P, _P, _I64, _P, _P, _SZ, _P]),
@@ -54,6 +55,7 @@ SIGNATURES = [
     ("oq_prepare_weights_g64", _I, [_P, _P, _I64, _I64, _P, _P, _P, _P, _P]),
     ("oq_gemm_w4a4_g64", _I, [_I, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _P, _P]),
     ("oq_linear_g64", _I, [_P, _P, _I64, _I64, _P, _P, _P, _P, _P, _I64, _P, _P, _SZ, _P]),
+    ("oq_linear_fused", _I, [_P, _P, _I64, _I64, _P, _P, _P, _P, _I64, _P, _P, _SZ, _P]),
     ("oq_linear_static_scratch", _I, [_P, _P, _I64, _I64, _P, _P, _P, _P, _I64, _P, _P]),
     ("oq_mma_peak_loop", _I, [_I, _I64, _P, _P]),
     ("oq_debug_pair_layout", _I, [_I, _I, _U64, _P]),
@@ -211,6 +213,13 @@ class Plan:
     def packed(self) -> bool:
         return self.act not in ("int8_absmax", "int8_lloydmax")
 
+    @property
+    def code_row_bytes(self) -> int:
+        """Bytes of one token's codes: d (8-bit kinds), d/2 (4-bit) or d/4 (2-bit)."""
+        if not self.packed:
+            return self.d
+        return self.d // 4 if self.act == "int2_percentile" else self.d // 2
+
     def workspace_bytes(self, T: int) -> int:
         return int(lib().oq_linear_workspace_bytes(self._h, T))
 
@@ -224,7 +233,7 @@ def rotate_quantize(plan: Plan, x, *, codes=None, scale=None, mean=None, rotated
     T, ldx = x.shape[0], x.stride(0)
     dev = x.device
     if codes is None:
-        codes = torch.empty((T, plan.d // 2 if plan.packed else plan.d),
+        codes = torch.empty((T, plan.code_row_bytes),
                             dtype=torch.int8 if plan.act == "int8_absmax" else torch.uint8,
                             device=dev)
     if scale is None:
@@ -286,6 +295,19 @@ def gemm_w4a4(plan, kind, a_packed, a_scale, w_packed, w_scale, *, mean=None, w_
     return out
 
 
+def gemm_w4a2(a_packed, a_scale, w_packed, w_scale, *, mean=None, w_rowsum=None, bias=None,
+              out_kind=OUT_BF16, out=None, stream=None):
+    """oq_gemm_w4a2: 2-bit codes [T, K/4] (four per byte) x packed INT4 [N, K/2] weights."""
+    import torch
+    T, K = a_packed.shape[0], a_packed.shape[1] * 4
+    N = w_packed.shape[0]
+    out = _out(T, N, out_kind, torch.int32, a_packed.device, out)
+    _check(lib().oq_gemm_w4a2(_ptr(a_packed), _ptr(a_scale), _ptr(mean), _ptr(w_packed),
+                              _ptr(w_scale), _ptr(w_rowsum), _ptr(bias), T, K, N, out_kind,
+                              _ptr(out), _stream(stream)))
+    return out
+
+
 def gemm_w4a8_lloydmax(plan, codes, sigma, w_packed, w_scale, *, mean=None, w_rowsum=None,
                        bias=None, out_kind=OUT_BF16, out=None, stream=None):
     """oq_gemm_w4a8_lloydmax: uint8 [T, K] 8-bit Lloyd-Max codes x packed INT4."""
@@ -313,6 +335,24 @@ def linear(plan: Plan, x, w_packed, w_scale, w_rowsum=None, bias=None, *, worksp
     _check(lib().oq_linear(plan.handle, _ptr(x), T, x.stride(0), _ptr(w_packed), _ptr(w_scale),
                            _ptr(w_rowsum), _ptr(bias), N, _ptr(out), _ptr(workspace),
                            workspace.numel() * workspace.element_size(), _stream(stream)))
+    return out
+
+
+def linear_fused(plan: Plan, x, w_packed, w_scale, w_rowsum=None, bias=None, *, workspace=None,
+                 out=None, stream=None):
+    """oq_linear_fused: the whole layer in one launch (T <= 256, INT8 absmax plans)."""
+    import torch
+    T = x.shape[0]
+    N = w_packed.shape[0]
+    need = plan.workspace_bytes(T)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=x.device)
+    if out is None:
+        out = torch.empty((T, N), dtype=torch.bfloat16, device=x.device)
+    _check(lib().oq_linear_fused(plan.handle, _ptr(x), T, x.stride(0), _ptr(w_packed),
+                                 _ptr(w_scale), _ptr(w_rowsum), _ptr(bias), N, _ptr(out),
+                                 _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                 _stream(stream)))
     return out
 
 

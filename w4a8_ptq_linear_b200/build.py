@@ -23,8 +23,8 @@ LIB_DIR = os.path.join(PKG, "lib")
 LIB = os.path.join(LIB_DIR, "liboq.so")
 
 SOURCES = ["oq_api.cu", "k_rotate_quant.cu", "k_gemm.cu", "k_weights_g64.cu", "oq_plan.cpp",
-           "oq_static_scratch.cu", "k_peak.cu"]
-HEADERS = ["oq_internal.h", "ptx.cuh"]
+           "oq_static_scratch.cu", "k_peak.cu", "k_linear_fused.cu"]
+HEADERS = ["oq_internal.h", "ptx.cuh", "rq_device.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -48,13 +48,15 @@
 // high nibble. A two's-complement nibble moved to the high half of a byte is the int8 16 n,
 // so a group widens to two 16-byte int8 chunks with one shift and two masks per word. The
 // 4-bit activations (element 2j low, 2j + 1 high in byte j) widen the same way plus two byte
-// permutes. The products are then 16 or 256 times the true ones; the int32 sums stay exact
-// (|16 * 127 * 7| K < 2^31 for K <= 32768) and the epilogue folds 1/16 or 1/256 into its
-// scale, which is exact in floating point.
+// permutes. A 2-bit code moved to the top two bits of a byte is the int8 64 c. The products
+// are then 16, 256 or 1024 times the true ones; the int32 sums stay exact (|16 * 127 * 7| K
+// and |1024 * 7| K stay below 2^31 for K <= 32768) and the epilogue folds 1/16, 1/256 or
+// 1/1024 into its scale, which is exact in floating point.
 //
 // Kinds:
 //   A8       X int8 straight from TMA, W int4 -> 16 W int8; tcgen05.mma.kind::i8, exact int32.
 //   A4       X int4 -> 16 X int8, W int4 -> 16 W int8; kind::i8.
+//   A2       X 2-bit -> 64 X int8 (four codes per byte), W as A4; kind::i8.
 //   LloydMax X code -> fp16 centroid (register table via prmt), W int4 -> 16 W fp16 (exact);
 //            kind::f16 with fp32 accumulation.
 //   LloydMax8 X 8-bit code -> fp16 centroid through a 256-entry table in shared memory, W as
@@ -94,7 +96,8 @@ struct Cfg {
   static constexpr bool X4F = KIND == kGemmLloydMax || KIND == kGemmG64;  // 4-bit codes -> fp16
   static constexpr int BK = FP ? 64 : 128;                          // 128 bytes of K per stage
   static constexpr bool XPACK = KIND != kGemmA8;
-  static constexpr int XB = KIND == kGemmLloydMax8 ? BK : BK / 2;  // activation bytes per row
+  static constexpr int XB =                                          // activation bytes per row
+      KIND == kGemmLloydMax8 ? BK : (KIND == kGemmA2 ? BK / 4 : BK / 2);
   static constexpr int BNMAX = 128 * CG;                           // tokens per tile, at most
   static constexpr int MAXCH = BNMAX / CH;                         // chunks per tile, at most
   static constexpr int XR = 128;                                   // activation rows per CTA
@@ -102,7 +105,8 @@ struct Cfg {
   // converters free only after unpacking, must cover that latency at the MMA's pace.
   static constexpr int SX = XPACK ? 0 : (CG == 2 ? 5 : 4);         // activation ring (A8)
   static constexpr int SP = CG == 1 ? 4 : (X4F ? 8 : 6);
-  static constexpr int S2 = (KIND == kGemmA4) ? (CG == 2 ? 3 : 2) : (CG == 2 ? 4 : 3);
+  static constexpr int S2 =
+      (KIND == kGemmA4 || KIND == kGemmA2) ? (CG == 2 ? 3 : 2) : (CG == 2 ? 4 : 3);
   static constexpr int WT = BM * 128;                              // W operand tile
   static constexpr int XT = XR * 128;                              // X operand tile (this CTA)
   static constexpr int WP = BM * (BK / 2);                         // packed W per stage
@@ -120,10 +124,12 @@ struct Cfg {
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int OFF_LUT8 = OFF_MISC + 16;                   // 8-bit code -> fp16 table
   static constexpr int SMEM = OFF_LUT8 + (KIND == kGemmLloydMax8 ? 512 : 0) + 1024;
-  // 1/16 per widened INT4 operand (see "Integer widening"); the grouped weights are decoded
-  // to their real values and the activation codes to plain integers
+  // 1/16 per widened INT4 operand and 1/64 per widened 2-bit one (see "Integer widening"); the
+  // grouped weights are decoded to their real values and the activation codes to plain integers
   static constexpr float ACC_SCALE =
-      KIND == kGemmA4 ? 1.f / 256.f : (KIND == kGemmG64 ? 1.f : 1.f / 16.f);
+      KIND == kGemmA4 ? 1.f / 256.f
+                      : (KIND == kGemmA2 ? 1.f / 1024.f : (KIND == kGemmG64 ? 1.f : 1.f / 16.f));
+  static constexpr int ACC_SHIFT = KIND == kGemmA4 ? 8 : (KIND == kGemmA2 ? 10 : 4);
   static_assert(XT % 1024 == 0 && P_STAGE % 1024 == 0 && CONV_STAGE % 1024 == 0 &&
                 XP % 1024 == 0, "operand tiles must stay 1024-byte aligned");
   static_assert(SMEM <= 232448, "shared memory");
@@ -249,6 +255,39 @@ __device__ __forceinline__ void convert_x_i8(const uint8_t* src, uint8_t* dst, i
     nib8_to_i8x16(in.y, a.z, a.w);
     nib8_to_i8x16(in.z, b.x, b.y);
     nib8_to_i8x16(in.w, b.z, b.w);
+    *reinterpret_cast<uint4*>(da + j * RSTEP * 128) = a;
+    *reinterpret_cast<uint4*>(db + j * RSTEP * 128) = b;
+  }
+}
+
+// 2-bit activation rows (element e in bits 2e, 2e + 1 of a 32-bit word, two's complement; 32
+// packed bytes = 128 codes per stage) -> int8 rows of 64 times the codes, swizzled as in
+// convert_w_i8, the
+// first `rows` rows (rounded up to a pass of the group). Thread ctid takes packed bytes
+// 8q .. 8q + 7 (q = ctid & 3) of its rows: codes 32q .. 32q + 31, chunks 2q and 2q + 1.
+__device__ __forceinline__ void pairs16_to_i8x64(uint32_t w, uint4& o) {
+  // field i of every byte moved to that byte's top two bits: 64 times element 4j + i in byte j
+  const uint32_t a0 = (w << 6) & 0xC0C0C0C0u, a1 = (w << 4) & 0xC0C0C0C0u;
+  const uint32_t a2 = (w << 2) & 0xC0C0C0C0u, a3 = w & 0xC0C0C0C0u;
+  const uint32_t l01 = __byte_perm(a0, a1, 0x5140), h01 = __byte_perm(a0, a1, 0x7362);
+  const uint32_t l23 = __byte_perm(a2, a3, 0x5140), h23 = __byte_perm(a2, a3, 0x7362);
+  o = make_uint4(__byte_perm(l01, l23, 0x5410), __byte_perm(l01, l23, 0x7632),
+                 __byte_perm(h01, h23, 0x5410), __byte_perm(h01, h23, 0x7632));
+}
+
+__device__ __forceinline__ void convert_x2_i8(const uint8_t* src, uint8_t* dst, int ctid,
+                                              int rows) {
+  constexpr int RSTEP = NCG / 4;
+  const int r0 = ctid >> 2, q = ctid & 3;
+  const uint8_t* s = src + r0 * 32 + q * 8;
+  uint8_t* da = dst + r0 * 128 + (((2 * q) ^ (r0 & 7)) << 4);
+  uint8_t* db = dst + r0 * 128 + (((2 * q + 1) ^ (r0 & 7)) << 4);
+#pragma unroll 1
+  for (int j = 0; j * RSTEP < rows; ++j) {
+    const uint2 in = *reinterpret_cast<const uint2*>(s + j * RSTEP * 32);
+    uint4 a, b;
+    pairs16_to_i8x64(in.x, a);
+    pairs16_to_i8x64(in.y, b);
     *reinterpret_cast<uint4*>(da + j * RSTEP * 128) = a;
     *reinterpret_cast<uint4*>(db + j * RSTEP * 128) = b;
   }
@@ -741,6 +780,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         } else {
           convert_w_i8(st + C::XP, cv, ctid);
           if constexpr (KIND == kGemmA4) convert_x_i8(st, cv + C::WT, ctid, rows);
+          if constexpr (KIND == kGemmA2) convert_x2_i8(st, cv + C::WT, ctid, rows);
         }
         dev::fence_async_smem();  // this thread's tiles -> visible to the tensor cores
         __syncwarp();             // the warp's reads of the packed stage and writes are done
@@ -821,7 +861,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             int32_t* dst = reinterpret_cast<int32_t*>(p.out) + (int64_t)(t0 + c * 32) * p.N + o;
 #pragma unroll
             for (int jj = 0; jj < 32; ++jj)
-              if (has_o && jj < n_valid) dst[(int64_t)jj * p.N] = (int32_t)r[jj] >> (KIND == kGemmA4 ? 8 : 4);
+              if (has_o && jj < n_valid) dst[(int64_t)jj * p.N] = (int32_t)r[jj] >> C::ACC_SHIFT;
           }
         } else {
           // two tokens at a time as f32x2: y = acc * (alpha_t s_w) + (mean_t w_1 + b), into
@@ -1505,6 +1545,12 @@ uint16_t f16_bits(float f) {
 
 }  // namespace
 
+bool tma_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner,
+                uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                CUtensorMapSwizzle sw) {
+  return make_map_2d(m, dt, base, inner, outer, row_bytes, box_inner, box_outer, sw);
+}
+
 oq_status launch_gemm(const GemmArgs& g, cudaStream_t s) {
   if (g.T == 0) return OQ_OK;
   GemmParams p{};
@@ -1541,6 +1587,9 @@ oq_status launch_gemm(const GemmArgs& g, cudaStream_t s) {
   switch (g.kind) {
     case kGemmA8: return small ? run<kGemmA8, 1>(g, p, s) : run_a8s(g, p, s);
     case kGemmA4: return small ? run<kGemmA4, 1>(g, p, s) : run<kGemmA4, 2>(g, p, s);
+    case kGemmA2:
+      if (g.K % 64) return fail(OQ_ERR_INVALID_ARG, "2-bit activations need K %% 64 == 0");
+      return small ? run<kGemmA2, 1>(g, p, s) : run<kGemmA2, 2>(g, p, s);
     case kGemmLloydMax:
       return small ? run<kGemmLloydMax, 1>(g, p, s) : run<kGemmLloydMax, 2>(g, p, s);
     case kGemmLloydMax8:

@@ -1,0 +1,460 @@
+// The whole layer in one launch for small token counts: center + RPBH + quantize and the W4A8
+// GEMM with its epilogue, for INT8 absmax activations against per-channel INT4 weights.
+//
+// CentriQ App. B.2 runs the activation path as a prologue of its INT4 GEMM: the token tile is
+// loaded once, centered, rotated and quantized with one scale per token, then multiplied. The
+// per-token scale needs the whole rotated token, and at the DiT widths a tile of whole tokens
+// does not fit on chip beside the GEMM's operands, so here the prologue is a phase of the same
+// kernel instead of a stage of every tile:
+//
+//   phase A  every CTA rotates and quantizes its share of the token pairs with the two-token
+//            body of the standalone kernel (rq_device.cuh), writing codes, scales and means;
+//            meanwhile the CTA's remaining warps widen its slice of the packed INT4 weights
+//            (which do not depend on phase A) into the tensor-core layout in shared memory;
+//   grid     one grid-wide barrier (a cooperative launch, so every CTA is resident) publishes
+//            the codes; they are read back from L2 by TMA while still resident there;
+//   phase B  split-K GEMM: a cluster of S CTAs owns one 128-channel tile, CTA r of the cluster
+//            its K blocks [r ks, (r + 1) ks), all T <= 256 tokens at once (MMA M = 128
+//            channels, N = T rounded up to 32, kind::i8 into TMEM), the code tiles streaming
+//            through a ring of ns stages. Each CTA moves its int32
+//            partial sums to shared memory; after a cluster barrier CTA r adds the S partials of
+//            its share of the tokens through distributed shared memory and applies the
+//            epilogue of CentriQ Eq. 5 / Eq. 9.
+//
+// Integer partial sums add exactly in any order, and the epilogue takes the same float steps
+// as the two-kernel path (scale alpha_t * s_w / 16, offset mean_t * w_1 + b, one fused
+// multiply-add, one rounding to bf16), so both paths return the same bits.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cooperative_groups.h>
+
+#include <algorithm>
+#include <map>
+#include <mutex>
+#include <tuple>
+
+#include "oq_internal.h"
+#include "ptx.cuh"
+#include "rq_device.cuh"
+
+namespace oq {
+
+bool tma_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner,
+                uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                CUtensorMapSwizzle sw);
+
+namespace {
+
+constexpr int FT = 256;           // threads per CTA
+constexpr int FM = 128;           // output channels per cluster (MMA M)
+constexpr int FWT = FM * 128;     // widened weight bytes of one K block (128 rows x 128 B)
+constexpr int kFusedMaxT = 256;   // tokens of one launch at most (MMA N, TMEM columns)
+constexpr int kFusedMaxS = 8;     // CTAs per cluster at most (portable cluster size)
+constexpr int kFusedMaxNs = 8;    // code-tile stages at most
+
+struct FusedParams {
+  RqParams rq;                    // phase A: codes int8 [T, K], scale [T], mean [T]
+  const uint8_t* w;               // packed INT4 weights [N, K/2], GEMM layout
+  const float* w_scale;
+  const float* w_rowsum;          // null without centering
+  const __nv_bfloat16* bias;      // may be null
+  __nv_bfloat16* y;               // [T, N]
+  int T, K, N, npad, ks, nkb, ns, rq_threads;
+  int off_u, off_bar;             // shared-memory offsets of the union region and the barriers
+  unsigned long long* err;
+  unsigned long long limit_ns;
+};
+
+// This CTA's weight tile, widened in place. At launch one TMA load per K block k brings the
+// packed rows (GEMM layout, 64 bytes = 128 elements per row) into the upper half of the K
+// block's 16 KB of widened weights; here they become int8 rows of 16 w in the 128-byte-swizzled
+// K-major layout of the MMA's A operand (as the GEMM's converters), written over the whole
+// 16 KB. Each of the nt participating threads (t = 0 .. nt - 1) first reads its packed groups
+// of the K block into registers, then, after a named barrier over the nt threads, writes them
+// widened, so that no write overtakes a read of the same block. Rows past N arrive as zeros.
+constexpr uint32_t kWidenBarrier = 2;
+constexpr int kWidenMaxItems = 4;   // packed 16-byte groups per thread and K block (nt >= 128)
+static_assert(FM * 4 <= kWidenMaxItems * (FT / 2), "widening threads: at least half the block");
+
+__device__ __forceinline__ void widen_weights(uint8_t* ww, int nk, int t, int nt) {
+  for (int k = 0; k < nk; ++k) {
+    uint8_t* blk = ww + k * FWT;
+    const uint8_t* packed = blk + FWT / 2;
+    uint4 in[kWidenMaxItems];
+#pragma unroll
+    for (int j = 0; j < kWidenMaxItems; ++j) {
+      const int i = t + j * nt;   // group q = i & 3 of row i >> 2
+      if (i < FM * 4) in[j] = *reinterpret_cast<const uint4*>(packed + i * 16);
+    }
+    dev::named_bar(kWidenBarrier, nt);
+#pragma unroll
+    for (int j = 0; j < kWidenMaxItems; ++j) {
+      const int i = t + j * nt;
+      if (i >= FM * 4) break;
+      const int row = i >> 2, q = i & 3;
+      const uint4 v = in[j];
+      const uint4 lo = make_uint4((v.x << 4) & 0xF0F0F0F0u, (v.y << 4) & 0xF0F0F0F0u,
+                                  (v.z << 4) & 0xF0F0F0F0u, (v.w << 4) & 0xF0F0F0F0u);
+      const uint4 hi = make_uint4(v.x & 0xF0F0F0F0u, v.y & 0xF0F0F0F0u, v.z & 0xF0F0F0F0u,
+                                  v.w & 0xF0F0F0F0u);
+      uint8_t* dst = blk + row * 128;
+      *reinterpret_cast<uint4*>(dst + (((2 * q) ^ (row & 7)) << 4)) = lo;
+      *reinterpret_cast<uint4*>(dst + (((2 * q + 1) ^ (row & 7)) << 4)) = hi;
+    }
+  }
+}
+
+template <int HLOG2, int ROUNDS>
+__global__ void __launch_bounds__(FT, 1)
+    k_linear_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+                   const __grid_constant__ FusedParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* ww = smem;                          // widened weights, ks K blocks
+  uint8_t* u = smem + p.off_u;                 // phase A scratch | X tiles | partial sums
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.off_bar);
+  // bars: full[ns], empty[ns], done, wfull; then the TMEM base and the abort flag
+  uint32_t* misc = reinterpret_cast<uint32_t*>(bars + 2 * kFusedMaxNs + 2);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int S = (int)dev::cluster_nctarank();
+  const int r = (int)dev::cluster_ctarank();
+  const int o0 = ((int)blockIdx.x / S) * FM;   // the cluster's channel tile
+  const int kb0 = r * p.ks;
+  const int nk = max(0, min(p.nkb, kb0 + p.ks) - kb0);
+  const int npad = p.npad;
+  const int ns = p.ns;
+  auto full = [&](int st) { return dev::smem_u32(&bars[st]); };
+  auto empty = [&](int st) { return dev::smem_u32(&bars[kFusedMaxNs + st]); };
+  const uint32_t done = dev::smem_u32(&bars[2 * kFusedMaxNs]);
+  const uint32_t wfull = dev::smem_u32(&bars[2 * kFusedMaxNs + 1]);
+  const int stage_bytes = npad * 128;
+
+  if (tid == 0) {
+    for (int st = 0; st < ns; ++st) {
+      dev::mbar_init(full(st), 1);
+      dev::mbar_init(empty(st), 1);
+    }
+    dev::mbar_init(done, 1);
+    dev::mbar_init(wfull, 1);
+    misc[1] = 0u;
+    dev::fence_mbar_init();
+    dev::prefetch_tmap(&tm_x);
+    // the packed weights do not depend on phase A: their loads fly while it runs
+    dev::mbar_arrive_expect_tx(wfull, (uint32_t)(nk * (FWT / 2)));
+    for (int k = 0; k < nk; ++k)
+      dev::tma_load_2d(dev::smem_u32(ww + k * FWT + FWT / 2), &tm_w, (kb0 + k) * 64, o0, wfull);
+  }
+  if (warp == 1) {
+    dev::tmem_alloc(dev::smem_u32(&misc[0]), kFusedMaxT);
+    dev::tmem_relinquish();
+  }
+  dev::tc_fence_before();
+  __syncthreads();
+  dev::tc_fence_after();
+  const uint32_t tmem = misc[0];
+
+  // ---- phase A: rotate-quantize the token pairs; widen this CTA's weights ------------------
+  const int nrq = p.rq_threads;
+  if (tid < nrq)
+    rq_pair_body<HLOG2, ROUNDS, kRqInt8>(p.rq, u, (int)blockIdx.x, (int)gridDim.x, nrq, true);
+  // the widening threads: the four or more warps phase A leaves idle, else all after phase A;
+  // their first thread waits for the packed weights, the others meet it at the named barrier
+  const int w0 = FT - nrq >= FT / 2 ? nrq : 0;
+  if (tid >= w0) {
+    if (tid == w0 && nk > 0 && !dev::mbar_wait(wfull, 0, p.err, kSiteFusedLoad, p.limit_ns))
+      misc[1] = 1u;
+    dev::named_bar(kWidenBarrier, FT - w0);
+    widen_weights(ww, nk, tid - w0, FT - w0);
+  }
+  // this thread's generic shared-memory writes (widened weights, phase A scratch) are ordered
+  // before the tensor core's reads and the TMA writes that follow the barrier below
+  dev::fence_async_smem();
+  // every CTA's codes, scales and means are written (the grid barrier orders them before what
+  // follows in every CTA)
+  cooperative_groups::this_grid().sync();
+
+  // ---- phase B: split-K GEMM ---------------------------------------------------------------
+  int issued = 0;   // code tiles this CTA's producer issued (thread 0)
+  if (tid == 0 && nk > 0) {
+    dev::fence_async_global();   // the codes acquired above, before the TMA reads them
+    for (int k = 0; k < nk; ++k) {
+      const int st = k % ns;
+      if (k >= ns && !dev::mbar_wait(empty(st), (uint32_t)((k / ns) - 1) & 1u, p.err,
+                                     kSiteGemmEmpty, p.limit_ns)) {
+        misc[1] = 1u;
+        break;
+      }
+      if (*reinterpret_cast<volatile uint32_t*>(&misc[1]) != 0u) break;
+      dev::mbar_arrive_expect_tx(full(st), (uint32_t)stage_bytes);
+      dev::tma_load_2d(dev::smem_u32(u + st * stage_bytes), &tm_x, (kb0 + k) * 128, 0, full(st));
+      issued = k + 1;
+    }
+  }
+  if (warp == 1 && lane == 0) {
+    const uint32_t idesc = dev::idesc_i8(FM, npad);
+    for (int k = 0; k < nk; ++k) {
+      const int st = k % ns;
+      if (!dev::mbar_wait(full(st), (uint32_t)(k / ns) & 1u, p.err, kSiteFusedLoad,
+                          p.limit_ns)) {
+        misc[1] = 1u;
+        break;
+      }
+      dev::tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t ad = dev::sdesc_sw128(dev::smem_u32(ww + k * FWT) + kk * 32);
+        const uint64_t bd = dev::sdesc_sw128(dev::smem_u32(u + st * stage_bytes) + kk * 32);
+        dev::mma_i8(tmem, ad, bd, idesc, (k | kk) != 0);
+      }
+      dev::mma_commit(empty(st));   // the stage is free once these MMAs have read it
+    }
+    dev::mma_commit(done);   // arrives once every MMA issued above has completed
+  }
+
+  // ---- partial sums: TMEM -> shared memory (int32 [npad tokens][128 channels]) -------------
+  {
+    bool ok = true;
+    if (lane == 0) ok = dev::mbar_wait(done, 0, p.err, kSiteFusedMma, p.limit_ns);
+    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    dev::tc_fence_after();
+    const bool valid = ok && nk > 0 && *reinterpret_cast<volatile uint32_t*>(&misc[1]) == 0u;
+    int32_t* part = reinterpret_cast<int32_t*>(u);   // the X tiles are consumed
+    const int q = warp & 3, o_local = q * 32 + lane;
+    for (int c = warp >> 2; c < npad / 32; c += 2) {
+      uint32_t v[32];
+      dev::tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(c * 32), v);
+      dev::tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 32; ++j) part[(c * 32 + j) * FM + o_local] = valid ? (int32_t)v[j] : 0;
+    }
+  }
+  dev::tc_fence_before();
+  __syncwarp();
+  dev::cluster_sync();   // every CTA's partial sums are in its shared memory
+
+  // ---- cluster reduction and epilogue: CTA r takes tokens [t0, t1) -------------------------
+  {
+    const int tps = (p.T + S - 1) / S;
+    const int t0 = r * tps, t1 = min(p.T, t0 + tps);
+    const int c4 = lane * 4;                 // four channels of the tile per thread
+    const int o = o0 + c4;
+    float sw[4], w1[4], bb[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const bool has = o + i < p.N;
+      sw[i] = has ? p.w_scale[o + i] * (1.f / 16.f) : 0.f;   // 1/16: the widened weights
+      w1[i] = (has && p.w_rowsum) ? p.w_rowsum[o + i] : 0.f;
+      bb[i] = (has && p.bias) ? __bfloat162float(p.bias[o + i]) : 0.f;
+    }
+    const uint32_t part0 = dev::smem_u32(u);
+    for (int t = t0 + warp; t < t1; t += FT / 32) {
+      const uint32_t off = part0 + (uint32_t)((t * FM + c4) * 4);
+      int32_t acc[4] = {0, 0, 0, 0};
+      for (int s = 0; s < S; ++s) {
+        const uint4 v = dev::ld_cluster_v4(dev::map_to_cta(off, (uint32_t)s));
+        acc[0] += (int32_t)v.x; acc[1] += (int32_t)v.y;
+        acc[2] += (int32_t)v.z; acc[3] += (int32_t)v.w;
+      }
+      // written by other CTAs in phase A: read at L2 (the grid barrier ordered them)
+      const float alpha = __ldcg(p.rq.scale + t);
+      const float mu = p.rq.mean ? __ldcg(p.rq.mean + t) : 0.f;
+      uint32_t yb[2];
+#pragma unroll
+      for (int i = 0; i < 4; i += 2) {
+        const float2 s2 = __fmul2_rn(make_float2(alpha, alpha), make_float2(sw[i], sw[i + 1]));
+        const float2 c2 = __ffma2_rn(make_float2(mu, mu), make_float2(w1[i], w1[i + 1]),
+                                     make_float2(bb[i], bb[i + 1]));
+        const float2 a2 = make_float2((float)acc[i], (float)acc[i + 1]);
+        const __nv_bfloat162 yv = __float22bfloat162_rn(__ffma2_rn(a2, s2, c2));
+        yb[i / 2] = *reinterpret_cast<const uint32_t*>(&yv);
+      }
+      if (o < p.N)   // N % 16 == 0: the four channels lie all inside or all outside
+        *reinterpret_cast<uint2*>(p.y + (int64_t)t * p.N + o) = make_uint2(yb[0], yb[1]);
+    }
+  }
+  __syncwarp();
+  dev::cluster_sync();   // no CTA leaves while another still reads its partial sums
+
+  // after an abort, loads already issued may still land: wait for them (bounded) before the
+  // block exits (a stage's barrier is at most one phase past its last issued load)
+  if (tid == 0 && misc[1] != 0u) {
+    for (int k = max(0, issued - ns); k < issued; ++k)
+      dev::mbar_wait(full(k % ns), (uint32_t)(k / ns) & 1u, p.err, kSiteGemmDrain, p.limit_ns);
+    if (nk > 0) dev::mbar_wait(wfull, 0, p.err, kSiteGemmDrain, p.limit_ns);
+  }
+  if (warp == 1) {
+    dev::tc_fence_after();
+    dev::tmem_dealloc(tmem, kFusedMaxT);
+  }
+}
+
+template <int HL, int R>
+const void* fused_kern() {
+  return reinterpret_cast<const void*>(&k_linear_fused<HL, R>);
+}
+
+template <int R>
+const void* fused_kern_h(int hlog2) {
+  switch (hlog2) {
+    case 0: return fused_kern<0, R>();
+    case 1: return fused_kern<1, R>();
+    case 2: return fused_kern<2, R>();
+    case 3: return fused_kern<3, R>();
+    case 4: return fused_kern<4, R>();
+    case 5: return fused_kern<5, R>();
+    case 6: return fused_kern<6, R>();
+    case 7: return fused_kern<7, R>();
+    case 8: return fused_kern<8, R>();
+    case 9: return fused_kern<9, R>();
+    default: return fused_kern<10, R>();
+  }
+}
+
+// Shared memory of a launch: widened weights, the union region, barriers, alignment slack.
+struct FusedShape {
+  int ks = 0, S = 0, ns = 0, off_u = 0, off_bar = 0;
+  size_t smem = 0;
+};
+
+// ks K blocks per CTA: the widened weights, then the union of the phase A scratch, the partial
+// sums and as many code-tile stages (up to ks) as the shared memory leaves room for; ns = 0 if
+// not even one stage fits.
+FusedShape fused_shape(int ks, int nkb, int npad, size_t rq_smem, size_t max_smem) {
+  FusedShape f;
+  f.ks = ks;
+  f.S = (nkb + ks - 1) / ks;
+  f.off_u = ks * FWT;
+  const size_t tail = (2 * kFusedMaxNs + 2) * 8 + 16 + 1024;   // barriers, misc, alignment
+  const size_t stage = (size_t)npad * 128;
+  const size_t fixed = std::max(rq_smem, (size_t)npad * FM * 4);
+  const size_t room = max_smem > f.off_u + tail ? max_smem - f.off_u - tail : 0;
+  int ns = std::min(std::min(ks, kFusedMaxNs), (int)(room / stage));
+  size_t uz = std::max(fixed, (size_t)ns * stage);
+  uz = (uz + 1023) & ~(size_t)1023;
+  if (uz > room) ns = 0;
+  f.ns = ns;
+  f.off_bar = f.off_u + (int)uz;
+  f.smem = (size_t)f.off_bar + tail;
+  return f;
+}
+
+}  // namespace
+
+oq_status launch_linear_fused(const FusedArgs& a, cudaStream_t s) {
+  if (a.T <= 0 || a.T > kFusedMaxT)
+    return fail(OQ_ERR_UNSUPPORTED, "single-launch layer: T must be in [1, %d]", kFusedMaxT);
+  if (a.rq.mode != kRqInt8)
+    return fail(OQ_ERR_UNSUPPORTED, "single-launch layer: INT8 absmax activations only");
+  if (a.N % 16 || a.K % 128)
+    return fail(OQ_ERR_UNSUPPORTED, "single-launch layer: d_in %% 128 == 0, d_out %% 16 == 0");
+  FusedParams p{};
+  int rq_threads = 0;
+  size_t rq_smem = 0;
+  oq_status st = rq_pair_setup(a.rq, p.rq, rq_threads, rq_smem);
+  if (st != OQ_OK) return st;
+  if (rq_threads > FT) return fail(OQ_ERR_UNSUPPORTED, "single-launch layer: d too large");
+  int hlog2 = 0;
+  while ((1 << hlog2) < a.rq.h) ++hlog2;
+  const void* fn = a.rq.rounds == 1 ? fused_kern_h<1>(hlog2) : fused_kern_h<2>(hlog2);
+  cudaError_t ce = allow_max_dynamic_smem(fn);
+  if (ce != cudaSuccess) return cuda_fail(ce, "cudaFuncSetAttribute(linear_fused)");
+
+  int dev = 0, max_smem = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  const int npad = ((int)a.T + 31) / 32 * 32;
+  const int nkb = (int)(a.K / 128);
+  const int n_o = (int)((a.N + FM - 1) / FM);
+
+  // The smallest K share per CTA (most CTAs) whose cluster fits the portable size, whose shared
+  // memory fits, and whose clusters can all be resident at once (the grid barrier needs that).
+  // Computed once per (device, kernel, T rounded, K, N).
+  static std::mutex mu;
+  static std::map<std::tuple<int, const void*, int, int, int, size_t>, FusedShape> cache;
+  FusedShape f;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    const auto key = std::make_tuple(dev, fn, npad, nkb, n_o, rq_smem);
+    auto it = cache.find(key);
+    if (it != cache.end()) {
+      f = it->second;
+    } else {
+      for (int ks = (nkb + kFusedMaxS - 1) / kFusedMaxS; ks <= nkb; ++ks) {
+        const FusedShape c = fused_shape(ks, nkb, npad, rq_smem, (size_t)max_smem);
+        if (c.ns < 1 || c.smem > (size_t)max_smem) break;   // only grows with ks
+        if ((c.S - 1) * ks >= nkb) continue;          // a CTA would get no K block
+        cudaLaunchConfig_t cfg{};
+        cfg.gridDim = dim3((unsigned)(n_o * c.S));
+        cfg.blockDim = dim3(FT);
+        cfg.dynamicSmemBytes = c.smem;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = (unsigned)c.S;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int nclusters = 0;
+        if (cudaOccupancyMaxActiveClusters(&nclusters, fn, &cfg) != cudaSuccess) {
+          cudaGetLastError();
+          nclusters = 0;
+        }
+        if (nclusters >= n_o) {
+          f = c;
+          break;
+        }
+      }
+      cache[key] = f;
+    }
+  }
+  if (f.ks == 0)
+    return fail(OQ_ERR_UNSUPPORTED, "single-launch layer: %d channel tiles do not fit at once",
+                n_o);
+
+  CUtensorMap tx, tw;
+  if (!tma_map_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.rq.codes, (uint64_t)a.K, (uint64_t)a.T,
+                  (uint64_t)a.K, 128, (uint32_t)npad, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !tma_map_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.w, (uint64_t)a.K / 2, (uint64_t)a.N,
+                  (uint64_t)a.K / 2, 64, FM, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return fail(OQ_ERR_CUDA, "cuTensorMapEncodeTiled failed or unavailable");
+  p.w = a.w;
+  p.w_scale = a.w_scale;
+  p.w_rowsum = a.w_rowsum;
+  p.bias = reinterpret_cast<const __nv_bfloat16*>(a.bias);
+  p.y = reinterpret_cast<__nv_bfloat16*>(a.y);
+  p.T = (int)a.T;
+  p.K = (int)a.K;
+  p.N = (int)a.N;
+  p.npad = npad;
+  p.ks = f.ks;
+  p.ns = f.ns;
+  p.nkb = nkb;
+  p.rq_threads = rq_threads;
+  p.off_u = f.off_u;
+  p.off_bar = f.off_bar;
+  p.err = device_error_word();
+  if (!p.err) return fail(OQ_ERR_CUDA, "device error word unavailable");
+  p.limit_ns = kWaitLimitNs;
+
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3((unsigned)(n_o * f.S));
+  cfg.blockDim = dim3(FT);
+  cfg.dynamicSmemBytes = f.smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)f.S;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeCooperative;
+  attr[1].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  void* args[] = {&tx, &tw, &p};
+  ce = cudaLaunchKernelExC(&cfg, fn, args);
+  if (ce != cudaSuccess) return cuda_fail(ce, "launch linear_fused");
+  return OQ_OK;
+}
+
+}  // namespace oq

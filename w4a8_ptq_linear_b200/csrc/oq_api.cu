@@ -202,12 +202,15 @@ oq_status oq_plan_create(oq_plan** out, int d, int h, int rounds, uint64_t seed,
   if (rounds != 1 && rounds != 2) return fail(OQ_ERR_INVALID_ARG, "rounds=%d not in {1,2}", rounds);
   if (act != OQ_ACT_INT8_ABSMAX && act != OQ_ACT_INT4_ABSMAX && act != OQ_ACT_INT4_LLOYDMAX &&
       act != OQ_ACT_INT4_PERCENTILE && act != OQ_ACT_INT4_LLOYDMAX_WIDTH &&
-      act != OQ_ACT_INT8_LLOYDMAX)
+      act != OQ_ACT_INT8_LLOYDMAX && act != OQ_ACT_INT2_PERCENTILE)
     return fail(OQ_ERR_INVALID_ARG, "unknown activation kind %d", (int)act);
   if (act == OQ_ACT_INT4_PERCENTILE && d > 8192)
     return fail(OQ_ERR_UNSUPPORTED, "the percentile scale supports d <= 8192 (d=%d)", d);
   if (act == OQ_ACT_INT8_LLOYDMAX && d > 8192)
     return fail(OQ_ERR_UNSUPPORTED, "8-bit Lloyd-Max codes support d <= 8192 (d=%d)", d);
+  if (act == OQ_ACT_INT2_PERCENTILE && (d > 8192 || d % 64))
+    return fail(d % 64 ? OQ_ERR_INVALID_ARG : OQ_ERR_UNSUPPORTED,
+                "2-bit activations need d %% 64 == 0 and d <= 8192 (d=%d)", d);
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
@@ -413,6 +416,7 @@ oq_status oq_rotate_quantize(const oq_plan* plan, const void* x_bf16, int64_t T,
   const int mode = plan->act == OQ_ACT_INT8_ABSMAX       ? kRqInt8
                    : plan->act == OQ_ACT_INT4_ABSMAX     ? kRqInt4
                    : plan->act == OQ_ACT_INT4_PERCENTILE ? kRqPercentile
+                   : plan->act == OQ_ACT_INT2_PERCENTILE ? kRqPercentile2
                    : plan->act == OQ_ACT_INT8_LLOYDMAX   ? kRqLloydMax8
                                                          : kRqLloydMax;   // either codebook
   return rotate_quantize_impl(plan, x_bf16, T, ldx, codes, scale, plan->center ? mean : nullptr,
@@ -530,6 +534,21 @@ oq_status oq_gemm_w4a4(const oq_plan* plan, oq_act_kind kind, const uint8_t* a_p
   return launch_gemm(g, static_cast<cudaStream_t>(stream));
 }
 
+oq_status oq_gemm_w4a2(const uint8_t* a_packed, const float* a_scale, const float* mean,
+                       const uint8_t* w_packed, const float* w_scale, const float* w_rowsum,
+                       const void* bias_bf16, int64_t T, int64_t d_in, int64_t d_out,
+                       oq_out_kind out_kind, void* out, void* stream) {
+  if (d_in % 64) return fail(OQ_ERR_INVALID_ARG, "2-bit activations need d_in %% 64 == 0");
+  oq_status st = check_gemm_args(a_packed, a_scale, mean, w_packed, w_scale, w_rowsum, bias_bf16,
+                                 T, d_in, d_out, (int)out_kind, out);
+  if (st != OQ_OK) return st;
+  GemmArgs g;
+  g.kind = kGemmA2; g.a = a_packed; g.a_scale = a_scale; g.mean = mean; g.w = w_packed;
+  g.w_scale = w_scale; g.w_rowsum = w_rowsum; g.bias = bias_bf16; g.T = T; g.K = d_in;
+  g.N = d_out; g.out_acc = out_kind == OQ_OUT_ACC; g.out = out;
+  return launch_gemm(g, static_cast<cudaStream_t>(stream));
+}
+
 oq_status oq_gemm_w4a8_lloydmax(const oq_plan* plan, const uint8_t* codes, const float* sigma,
                                 const float* mean, const uint8_t* w_packed, const float* w_scale,
                                 const float* w_rowsum, const void* bias_bf16, int64_t T,
@@ -555,10 +574,15 @@ static bool codes8(const oq_plan* plan) {
   return plan->act == OQ_ACT_INT8_ABSMAX || plan->act == OQ_ACT_INT8_LLOYDMAX;
 }
 
+// bytes of one token's codes: d (8-bit kinds), d / 2 (4-bit) or d / 4 (2-bit)
+static size_t code_row_bytes(const oq_plan* plan) {
+  if (codes8(plan)) return (size_t)plan->d;
+  return plan->act == OQ_ACT_INT2_PERCENTILE ? (size_t)plan->d / 4 : (size_t)plan->d / 2;
+}
+
 size_t oq_linear_workspace_bytes(const oq_plan* plan, int64_t T) {
   if (!plan || T < 0) return 0;
-  const size_t code_bytes =
-      codes8(plan) ? (size_t)T * plan->d : (size_t)T * (plan->d / 2);
+  const size_t code_bytes = (size_t)T * code_row_bytes(plan);
   return round256(code_bytes) + 2 * round256((size_t)T * 4);
 }
 
@@ -574,8 +598,7 @@ oq_status oq_linear(const oq_plan* plan, const void* x_bf16, int64_t T, int64_t 
   if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return fail(OQ_ERR_MISALIGNED, "workspace must be 256-byte aligned");
   if (plan->center && !w_rowsum) return fail(OQ_ERR_INVALID_ARG, "centering needs w_rowsum");
-  const size_t code_bytes =
-      codes8(plan) ? (size_t)T * plan->d : (size_t)T * (plan->d / 2);
+  const size_t code_bytes = (size_t)T * code_row_bytes(plan);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   void* codes = ws;
   float* scale = reinterpret_cast<float*>(ws + round256(code_bytes));
@@ -590,9 +613,50 @@ oq_status oq_linear(const oq_plan* plan, const void* x_bf16, int64_t T, int64_t 
     return oq_gemm_w4a8_lloydmax(plan, static_cast<const uint8_t*>(codes), scale, m, w_packed,
                                  w_scale, w_rowsum, bias_bf16, T, plan->d, d_out, OQ_OUT_BF16,
                                  y_bf16, stream);
+  if (plan->act == OQ_ACT_INT2_PERCENTILE)
+    return oq_gemm_w4a2(static_cast<const uint8_t*>(codes), scale, m, w_packed, w_scale,
+                        w_rowsum, bias_bf16, T, plan->d, d_out, OQ_OUT_BF16, y_bf16, stream);
   return oq_gemm_w4a4(plan, plan->act, static_cast<const uint8_t*>(codes), scale, m, w_packed,
                       w_scale, w_rowsum, bias_bf16, T, plan->d, d_out, OQ_OUT_BF16, y_bf16,
                       stream);
+}
+
+oq_status oq_linear_fused(const oq_plan* plan, const void* x_bf16, int64_t T, int64_t ldx,
+                          const uint8_t* w_packed, const float* w_scale, const float* w_rowsum,
+                          const void* bias_bf16, int64_t d_out, void* y_bf16, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  if (!plan) return fail(OQ_ERR_INVALID_ARG, "NULL plan");
+  if (plan->act != OQ_ACT_INT8_ABSMAX)
+    return fail(OQ_ERR_UNSUPPORTED, "the single-launch layer takes INT8_ABSMAX plans");
+  if (T < 1 || T > 256) return fail(OQ_ERR_UNSUPPORTED, "the single-launch layer takes 1 <= T <= 256");
+  const size_t need = oq_linear_workspace_bytes(plan, T);
+  if (!workspace || workspace_bytes < need)
+    return fail(OQ_ERR_INVALID_ARG, "workspace too small: need %zu bytes", need);
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u)
+    return fail(OQ_ERR_MISALIGNED, "workspace must be 256-byte aligned");
+  if (plan->center && !w_rowsum) return fail(OQ_ERR_INVALID_ARG, "centering needs w_rowsum");
+  if (ldx < plan->d || (ldx * 2) % 16) return fail(OQ_ERR_MISALIGNED, "ldx must be >= d and a multiple of 8");
+  if (!x_bf16 || !aligned16(x_bf16)) return fail(OQ_ERR_MISALIGNED, "x must be 16-byte aligned");
+  oq_status st = check_gemm_args(workspace, reinterpret_cast<const float*>(workspace), nullptr,
+                                 w_packed, w_scale, w_rowsum, bias_bf16, T, plan->d, d_out,
+                                 OQ_OUT_BF16, y_bf16);
+  if (st != OQ_OK) return st;
+  st = check_plan_device(plan);
+  if (st != OQ_OK) return st;
+  const size_t code_bytes = (size_t)T * code_row_bytes(plan);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  FusedArgs f;
+  RqArgs& a = f.rq;
+  a.x = x_bf16; a.ldx = ldx; a.T = T; a.d = plan->d; a.h = plan->h; a.rounds = plan->rounds;
+  a.center = plan->center; a.mode = kRqInt8; a.tab = plan->d_tab; a.smask = plan->d_smask;
+  a.slot = plan->d_slot; a.ones = plan->d_ones; a.codes = ws;
+  a.scale = reinterpret_cast<float*>(ws + round256(code_bytes));
+  a.mean = plan->center ? reinterpret_cast<float*>(ws + round256(code_bytes) +
+                                                   round256((size_t)T * 4))
+                        : nullptr;
+  f.w = w_packed; f.w_scale = w_scale; f.w_rowsum = plan->center ? w_rowsum : nullptr;
+  f.bias = bias_bf16; f.y = y_bf16; f.T = T; f.K = plan->d; f.N = d_out;
+  return launch_linear_fused(f, static_cast<cudaStream_t>(stream));
 }
 
 oq_status oq_linear_g64(const oq_plan* plan, const void* x_bf16, int64_t T, int64_t ldx,

@@ -64,12 +64,14 @@ enum : uint32_t {
   kSiteGemmAccum = 19,     // GEMM epilogue: accumulator ready
   kSiteGemmDrain = 20,     // GEMM: drain after an abort
   kSitePeak = 21,          // tensor-core peak loop: completion of the MMAs
+  kSiteFusedLoad = 22,     // single-launch layer: activation codes loaded
+  kSiteFusedMma = 23,      // single-launch layer: partial sums complete
   kSiteDebug = 99          // oq_debug_wait_timeout
 };
 
 // ---- rotate + quantize ---------------------------------------------------------------------
 enum RqMode : int { kRqInt8 = 0, kRqInt4 = 1, kRqLloydMax = 2, kRqPercentile = 3,
-                     kRqLloydMax8 = 4 };
+                     kRqLloydMax8 = 4, kRqPercentile2 = 5 };
 
 struct RqArgs {
   const void* x = nullptr;   // bf16 [T, ldx]
@@ -104,7 +106,8 @@ std::vector<int> pair_word_layout(int d, int h, const int32_t* perm0);
 // ---- GEMM ----------------------------------------------------------------------------------
 // kGemmG64: INT4 codes (decoded to fp16 integers) against asymmetric g = 64 weights
 // dequantized to fp16 per (row, group) in the converters
-enum GemmKind : int { kGemmA8 = 0, kGemmA4 = 1, kGemmLloydMax = 2, kGemmLloydMax8 = 3, kGemmG64 = 4 };
+enum GemmKind : int { kGemmA8 = 0, kGemmA4 = 1, kGemmLloydMax = 2, kGemmLloydMax8 = 3, kGemmG64 = 4,
+                      kGemmA2 = 5 };
 
 struct GemmArgs {
   int kind = kGemmA8;
@@ -123,6 +126,19 @@ struct GemmArgs {
   const uint32_t* w_sz = nullptr;  // kGemmG64: [K/64][N] words, fp16 sigma (low), z (high)
 };
 oq_status launch_gemm(const GemmArgs& g, cudaStream_t s);
+
+// The whole layer in one launch (T <= 256, INT8 absmax activations, per-channel weights):
+// rotate-quantize into rq.codes / rq.scale / rq.mean, then the GEMM and epilogue into y.
+struct FusedArgs {
+  RqArgs rq;                        // the activation path, codes int8 [T, K] in the workspace
+  const uint8_t* w = nullptr;       // uint8 [N, K/2], GEMM layout
+  const float* w_scale = nullptr;
+  const float* w_rowsum = nullptr;  // null unless the plan centers
+  const void* bias = nullptr;       // bf16 [N] or null
+  void* y = nullptr;                // bf16 [T, N]
+  int64_t T = 0, K = 0, N = 0;
+};
+oq_status launch_linear_fused(const FusedArgs& a, cudaStream_t s);
 
 // oq_prepare_weights that also writes the rotated rows (float [n_out, d]) to `rot` (if not null)
 oq_status oq_prepare_weights_rotated(const oq_plan* plan, const void* w_bf16, int64_t n_out,
