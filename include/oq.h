@@ -315,7 +315,9 @@ size_t oq_linear_workspace_bytes(const oq_plan* plan, int64_t T);
 /* The whole layer: oq_rotate_quantize into `workspace`, then the GEMM for the plan's
  * activation kind, on one stream. y_bf16 is [T, d_out] bf16. workspace must hold
  * oq_linear_workspace_bytes(plan, T) bytes, 256-byte aligned; it is scratch owned by the
- * caller and overwritten. */
+ * caller and overwritten. For INT8 absmax plans and 1 <= T <= 256 the call runs as one launch
+ * (oq_linear_fused) wherever that path applies; the result and the workspace's contents are
+ * the same bits either way. */
 oq_status oq_linear(const oq_plan* plan, const void* x_bf16, int64_t T, int64_t ldx,
                     const uint8_t* w_packed, const float* w_scale, const float* w_rowsum,
                     const void* bias_bf16, int64_t d_out, void* y_bf16, void* workspace,

@@ -35,6 +35,15 @@ def test_library_exports_every_declared_symbol(lib):
     assert set(names) == bound, "binding and header disagree"
 
 
+def test_checked_build_exports_the_same_symbols(lib):
+    # the bounds-checked variant (-DOQ_CHECKED) is the same ABI
+    from w4a8_ptq_linear_b200 import build
+    path = build.build(checked=True)
+    checked = oq.load(path)
+    for n in declared_symbols():
+        assert hasattr(checked, n), n
+
+
 def test_status_strings(lib):
     for code, name in [(0, "OQ_OK"), (1, "OQ_ERR_INVALID_ARG"), (5, "OQ_ERR_DEVICE_TIMEOUT")]:
         assert lib.oq_status_string(code).decode() == name

@@ -51,8 +51,12 @@ def test_fused_layer_equals_two_kernel_path_and_oracle(d, n_out, h, rounds, cent
     need = max(plan.workspace_bytes(T), 256)
     ws_f = torch.full((need,), 0xA5, dtype=torch.uint8, device="cuda")
     y_f = oq.linear_fused(plan, x, wp, ws, w1, b, workspace=ws_f)
-    y_2 = oq.linear(plan, x, wp, ws, w1, b)
+    y_l = oq.linear(plan, x, wp, ws, w1, b)          # dispatches to the single launch
     codes, scale, mean, _ = oq.rotate_quantize(plan, x)
+    y_2 = oq.gemm_w4a8(codes, scale, wp, ws, mean=mean, w_rowsum=w1 if center else None,
+                       bias=b)                       # the two-kernel path, call by call
+    torch.cuda.synchronize()
+    assert torch.equal(y_l, y_f)
     torch.cuda.synchronize()
     st, code = oq.device_status()
     assert st == 0, hex(code)

@@ -19,6 +19,8 @@ import numpy as np
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "lib", "liboq.so")
+# the bounds-checked build (python -m w4a8_ptq_linear_b200.build --checked)
+LIB_CHECKED_PATH = os.path.join(_PKG, "lib", "liboq_checked.so")
 
 OQ_OK, OQ_ERR_INVALID_ARG, OQ_ERR_UNSUPPORTED, OQ_ERR_MISALIGNED = 0, 1, 2, 3
 OQ_ERR_CUDA, OQ_ERR_DEVICE_TIMEOUT, OQ_ERR_NOMEM = 4, 5, 6
@@ -69,7 +71,6 @@ class OQError(RuntimeError):
 
 
 _lib = None
-_load_error = None
 
 
 def _status_name(s: int) -> str:
@@ -79,20 +80,43 @@ def _status_name(s: int) -> str:
     return names.get(s, f"status {s}")
 
 
+def load(path: str):
+    """A ctypes handle on a build of the library at `path`, with every signature set."""
+    if not os.path.exists(path):
+        raise OQError(OQ_ERR_UNSUPPORTED,
+                      f"{path} is not built: run python -m w4a8_ptq_linear_b200.build")
+    L = ctypes.CDLL(path)
+    for name, res, args in SIGNATURES:
+        f = getattr(L, name)
+        f.restype = res
+        f.argtypes = args
+    return L
+
+
 def lib():
     """The loaded ctypes library; raises OQError if it is not built."""
-    global _lib, _load_error
+    global _lib
     if _lib is None:
-        if not os.path.exists(LIB_PATH):
-            raise OQError(OQ_ERR_UNSUPPORTED,
-                          f"{LIB_PATH} is not built: run python -m w4a8_ptq_linear_b200.build")
-        L = ctypes.CDLL(LIB_PATH)
-        for name, res, args in SIGNATURES:
-            f = getattr(L, name)
-            f.restype = res
-            f.argtypes = args
-        _lib = L
+        _lib = load(LIB_PATH)
     return _lib
+
+
+class using:
+    """Within the block, every call of this module goes to the library build `handle` (for
+    example ``load(LIB_CHECKED_PATH)``); plans must be created and used inside one build."""
+
+    def __init__(self, handle):
+        self.handle = handle
+
+    def __enter__(self):
+        global _lib
+        self.saved = lib()
+        _lib = self.handle
+        return self.handle
+
+    def __exit__(self, *exc):
+        global _lib
+        _lib = self.saved
 
 
 def _check(status: int):

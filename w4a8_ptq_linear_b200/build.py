@@ -21,6 +21,10 @@ CSRC = os.path.join(PKG, "csrc")
 OBJ = os.path.join(ROOT, "_build", "obj")
 LIB_DIR = os.path.join(PKG, "lib")
 LIB = os.path.join(LIB_DIR, "liboq.so")
+# the bounds-checked variant (-DOQ_CHECKED): every table-driven device index is range-checked
+# and the first violation is reported through the device error word
+OBJ_CHECKED = os.path.join(ROOT, "_build", "obj_checked")
+LIB_CHECKED = os.path.join(LIB_DIR, "liboq_checked.so")
 
 SOURCES = ["oq_api.cu", "k_rotate_quant.cu", "k_gemm.cu", "k_weights_g64.cu", "oq_plan.cpp",
            "oq_static_scratch.cu", "k_peak.cu", "k_linear_fused.cu"]
@@ -41,23 +45,25 @@ def _flags():
                    "--expt-relaxed-constexpr"]
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = [os.path.join(CSRC, f) for f in SOURCES + HEADERS]
     deps += [os.path.join(ROOT, "include", "oq.h"), os.path.abspath(__file__)]
     return any(os.path.getmtime(p) > t for p in deps)
 
 
-def build(force: bool = False, verbose: bool = False, extra=None) -> str:
-    """Compile every source to an object, then link lib/liboq.so. Returns the .so path."""
-    if not force and not _stale():
+def build(force: bool = False, verbose: bool = False, extra=None, checked: bool = False) -> str:
+    """Compile every source to an object, then link lib/liboq.so (lib/liboq_checked.so with
+    checked=True). Returns the .so path."""
+    LIB, OBJ = (LIB_CHECKED, OBJ_CHECKED) if checked else (globals()["LIB"], globals()["OBJ"])
+    if not force and not _stale(LIB):
         return LIB
     os.makedirs(OBJ, exist_ok=True)
     os.makedirs(LIB_DIR, exist_ok=True)
     cc = nvcc()
-    extra = list(extra or [])
+    extra = list(extra or []) + (["-DOQ_CHECKED"] if checked else [])
 
     def compile_one(src):
         obj = os.path.join(OBJ, os.path.splitext(src)[0] + ".o")
@@ -89,7 +95,9 @@ if __name__ == "__main__":
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose", action="store_true")
     ap.add_argument("--ptxas-v", action="store_true", help="print register/smem usage")
+    ap.add_argument("--checked", action="store_true", help="the bounds-checked variant")
     a = ap.parse_args()
     extra = ["-Xptxas", "-v"] if a.ptxas_v else []
-    print(build(force=a.force or a.ptxas_v, verbose=a.verbose or a.ptxas_v, extra=extra))
+    print(build(force=a.force or a.ptxas_v, verbose=a.verbose or a.ptxas_v, extra=extra,
+                checked=a.checked))
     sys.exit(0)

@@ -60,7 +60,7 @@ struct FusedParams {
   const __nv_bfloat16* bias;      // may be null
   __nv_bfloat16* y;               // [T, N]
   int T, K, N, npad, ks, nkb, ns, rq_threads;
-  int off_u, off_bar;             // shared-memory offsets of the union region and the barriers
+  int off_u, off_bar, off_tok;    // shared-memory offsets: union region, barriers, token scales
   unsigned long long* err;
   unsigned long long limit_ns;
 };
@@ -75,6 +75,7 @@ struct FusedParams {
 constexpr uint32_t kWidenBarrier = 2;
 constexpr int kWidenMaxItems = 4;   // packed 16-byte groups per thread and K block (nt >= 128)
 static_assert(FM * 4 <= kWidenMaxItems * (FT / 2), "widening threads: at least half the block");
+static_assert((2 * kFusedMaxNs + 2) * 8 + 8 <= 256, "barriers and misc fit their 256 bytes");
 
 __device__ __forceinline__ void widen_weights(uint8_t* ww, int nk, int t, int nt) {
   for (int k = 0; k < nk; ++k) {
@@ -186,6 +187,10 @@ __global__ void __launch_bounds__(FT, 1)
         break;
       }
       if (*reinterpret_cast<volatile uint32_t*>(&misc[1]) != 0u) break;
+      if (!OQ_IN_BOUNDS((st + 1) * stage_bytes <= p.off_bar - p.off_u, p.err, kSiteBoundsFused)) {
+        misc[1] = 1u;
+        break;
+      }
       dev::mbar_arrive_expect_tx(full(st), (uint32_t)stage_bytes);
       dev::tma_load_2d(dev::smem_u32(u + st * stage_bytes), &tm_x, (kb0 + k) * 128, 0, full(st));
       issued = k + 1;
@@ -212,16 +217,30 @@ __global__ void __launch_bounds__(FT, 1)
     dev::mma_commit(done);   // arrives once every MMA issued above has completed
   }
 
+  // This CTA's share of the tokens for the reduction: [t0, t1).
+  const int tps = (p.T + S - 1) / S;
+  const int t0 = min(p.T, r * tps), t1 = min(p.T, t0 + tps);
+  // their scales and means (written by other CTAs in phase A, ordered by the grid barrier),
+  // read at L2 while the MMAs run; the cluster barrier below publishes them to the CTA
+  float2* s_tok = reinterpret_cast<float2*>(smem + p.off_tok);
+  for (int t = t0 + tid; t < t1; t += FT)
+    if (OQ_IN_BOUNDS(t - t0 < kFusedMaxT, p.err, kSiteBoundsFused))
+      s_tok[t - t0] = make_float2(__ldcg(p.rq.scale + t), p.rq.mean ? __ldcg(p.rq.mean + t) : 0.f);
+
   // ---- partial sums: TMEM -> shared memory (int32 [npad tokens][128 channels]) -------------
+  // A token's 128 partial sums are 512 contiguous bytes, so that the reduction below reads
+  // whole rows from the other CTAs' shared memory; the stores of a warp (32 channels of one
+  // token) are 128 contiguous bytes.
   {
     bool ok = true;
     if (lane == 0) ok = dev::mbar_wait(done, 0, p.err, kSiteFusedMma, p.limit_ns);
     ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
     dev::tc_fence_after();
     const bool valid = ok && nk > 0 && *reinterpret_cast<volatile uint32_t*>(&misc[1]) == 0u;
-    int32_t* part = reinterpret_cast<int32_t*>(u);   // the X tiles are consumed
-    const int q = warp & 3, o_local = q * 32 + lane;
-    for (int c = warp >> 2; c < npad / 32; c += 2) {
+    int32_t* part = reinterpret_cast<int32_t*>(u);   // the code tiles are consumed
+    const int q = warp & 3, o_local = q * 32 + lane;   // TMEM lane quarter of this warp
+    const bool fits = OQ_IN_BOUNDS(npad * FM * 4 <= p.off_bar - p.off_u, p.err, kSiteBoundsFused);
+    for (int c = warp >> 2; fits && c < npad / 32; c += 2) {
       uint32_t v[32];
       dev::tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(c * 32), v);
       dev::tmem_wait_ld();
@@ -233,44 +252,52 @@ __global__ void __launch_bounds__(FT, 1)
   __syncwarp();
   dev::cluster_sync();   // every CTA's partial sums are in its shared memory
 
-  // ---- cluster reduction and epilogue: CTA r takes tokens [t0, t1) -------------------------
+  // ---- cluster reduction and epilogue ------------------------------------------------------
+  // Thread: four consecutive channels of one token per item, the S partial sums of the
+  // cluster's CTAs loaded together; a warp reads one token's whole row from each CTA and
+  // writes 256 contiguous bytes of y. y = bf16(acc * (alpha_t s_w / 16) + (mean_t w_1 + b)).
   {
-    const int tps = (p.T + S - 1) / S;
-    const int t0 = r * tps, t1 = min(p.T, t0 + tps);
-    const int c4 = lane * 4;                 // four channels of the tile per thread
+    const int c4 = lane * 4;
     const int o = o0 + c4;
+    const bool has = o < p.N;   // N % 16 == 0: the four channels lie all inside or all outside
     float sw[4], w1[4], bb[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const bool has = o + i < p.N;
       sw[i] = has ? p.w_scale[o + i] * (1.f / 16.f) : 0.f;   // 1/16: the widened weights
       w1[i] = (has && p.w_rowsum) ? p.w_rowsum[o + i] : 0.f;
       bb[i] = (has && p.bias) ? __bfloat162float(p.bias[o + i]) : 0.f;
     }
-    const uint32_t part0 = dev::smem_u32(u);
-    for (int t = t0 + warp; t < t1; t += FT / 32) {
-      const uint32_t off = part0 + (uint32_t)((t * FM + c4) * 4);
+    const uint32_t part0 = dev::smem_u32(u) + (uint32_t)(c4 * 4);
+    uint32_t peer[kFusedMaxS];
+#pragma unroll
+    for (int sr = 0; sr < kFusedMaxS; ++sr)
+      peer[sr] = sr < S ? dev::map_to_cta(part0, (uint32_t)sr) : 0u;
+    const bool fits = OQ_IN_BOUNDS(t1 <= npad && t1 - t0 <= kFusedMaxT, p.err, kSiteBoundsFused);
+    for (int t = t0 + warp; fits && t < t1; t += FT / 32) {
+      const uint32_t off = (uint32_t)(t * FM * 4);
+      uint4 v[kFusedMaxS];
+#pragma unroll
+      for (int sr = 0; sr < kFusedMaxS; ++sr)
+        if (sr < S) v[sr] = dev::ld_cluster_v4(peer[sr] + off);
       int32_t acc[4] = {0, 0, 0, 0};
-      for (int s = 0; s < S; ++s) {
-        const uint4 v = dev::ld_cluster_v4(dev::map_to_cta(off, (uint32_t)s));
-        acc[0] += (int32_t)v.x; acc[1] += (int32_t)v.y;
-        acc[2] += (int32_t)v.z; acc[3] += (int32_t)v.w;
-      }
-      // written by other CTAs in phase A: read at L2 (the grid barrier ordered them)
-      const float alpha = __ldcg(p.rq.scale + t);
-      const float mu = p.rq.mean ? __ldcg(p.rq.mean + t) : 0.f;
+#pragma unroll
+      for (int sr = 0; sr < kFusedMaxS; ++sr)
+        if (sr < S) {
+          acc[0] += (int32_t)v[sr].x; acc[1] += (int32_t)v[sr].y;
+          acc[2] += (int32_t)v[sr].z; acc[3] += (int32_t)v[sr].w;
+        }
+      const float2 tk = s_tok[t - t0];
       uint32_t yb[2];
 #pragma unroll
       for (int i = 0; i < 4; i += 2) {
-        const float2 s2 = __fmul2_rn(make_float2(alpha, alpha), make_float2(sw[i], sw[i + 1]));
-        const float2 c2 = __ffma2_rn(make_float2(mu, mu), make_float2(w1[i], w1[i + 1]),
+        const float2 s2 = __fmul2_rn(make_float2(tk.x, tk.x), make_float2(sw[i], sw[i + 1]));
+        const float2 c2 = __ffma2_rn(make_float2(tk.y, tk.y), make_float2(w1[i], w1[i + 1]),
                                      make_float2(bb[i], bb[i + 1]));
         const float2 a2 = make_float2((float)acc[i], (float)acc[i + 1]);
         const __nv_bfloat162 yv = __float22bfloat162_rn(__ffma2_rn(a2, s2, c2));
         yb[i / 2] = *reinterpret_cast<const uint32_t*>(&yv);
       }
-      if (o < p.N)   // N % 16 == 0: the four channels lie all inside or all outside
-        *reinterpret_cast<uint2*>(p.y + (int64_t)t * p.N + o) = make_uint2(yb[0], yb[1]);
+      if (has) *reinterpret_cast<uint2*>(p.y + (int64_t)t * p.N + o) = make_uint2(yb[0], yb[1]);
     }
   }
   __syncwarp();
@@ -313,7 +340,7 @@ const void* fused_kern_h(int hlog2) {
 
 // Shared memory of a launch: widened weights, the union region, barriers, alignment slack.
 struct FusedShape {
-  int ks = 0, S = 0, ns = 0, off_u = 0, off_bar = 0;
+  int ks = 0, S = 0, ns = 0, off_u = 0, off_bar = 0, off_tok = 0;
   size_t smem = 0;
 };
 
@@ -325,7 +352,8 @@ FusedShape fused_shape(int ks, int nkb, int npad, size_t rq_smem, size_t max_sme
   f.ks = ks;
   f.S = (nkb + ks - 1) / ks;
   f.off_u = ks * FWT;
-  const size_t tail = (2 * kFusedMaxNs + 2) * 8 + 16 + 1024;   // barriers, misc, alignment
+  // barriers and misc (256 B), the token scales and means (8 B a token), alignment slack
+  const size_t tail = 256 + 8 * kFusedMaxT + 1024;
   const size_t stage = (size_t)npad * 128;
   const size_t fixed = std::max(rq_smem, (size_t)npad * FM * 4);
   const size_t room = max_smem > f.off_u + tail ? max_smem - f.off_u - tail : 0;
@@ -335,6 +363,7 @@ FusedShape fused_shape(int ks, int nkb, int npad, size_t rq_smem, size_t max_sme
   if (uz > room) ns = 0;
   f.ns = ns;
   f.off_bar = f.off_u + (int)uz;
+  f.off_tok = f.off_bar + 256;
   f.smem = (size_t)f.off_bar + tail;
   return f;
 }
@@ -433,6 +462,7 @@ oq_status launch_linear_fused(const FusedArgs& a, cudaStream_t s) {
   p.rq_threads = rq_threads;
   p.off_u = f.off_u;
   p.off_bar = f.off_bar;
+  p.off_tok = f.off_tok;
   p.err = device_error_word();
   if (!p.err) return fail(OQ_ERR_CUDA, "device error word unavailable");
   p.limit_ns = kWaitLimitNs;

@@ -149,8 +149,12 @@ oq_status oq_device_status(int clear, uint64_t* code_out) {
     e = cudaMemset(w, 0, sizeof(v));
     if (e != cudaSuccess) return cuda_fail(e, "clear device error word");
   }
-  if (v) return fail(OQ_ERR_DEVICE_TIMEOUT, "device wait gave up: site %u block %u",
-                     (unsigned)((v >> 32) & 0xFFFF), (unsigned)(v & 0xFFFFFFFFu));
+  const unsigned site = (unsigned)((v >> 32) & 0xFFFF);
+  if (v && site >= kSiteBounds)
+    return fail(OQ_ERR_INVALID_ARG, "index out of range (checked build): site %#x block %u", site,
+                (unsigned)(v & 0xFFFFFFFFu));
+  if (v) return fail(OQ_ERR_DEVICE_TIMEOUT, "device wait gave up: site %u block %u", site,
+                     (unsigned)(v & 0xFFFFFFFFu));
   return OQ_OK;
 }
 
@@ -598,6 +602,15 @@ oq_status oq_linear(const oq_plan* plan, const void* x_bf16, int64_t T, int64_t 
   if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return fail(OQ_ERR_MISALIGNED, "workspace must be 256-byte aligned");
   if (plan->center && !w_rowsum) return fail(OQ_ERR_INVALID_ARG, "centering needs w_rowsum");
+  // Up to 256 tokens of an INT8 absmax layer run as one launch where the device holds all of
+  // its clusters at once (same results bit for bit); otherwise the two kernels below.
+  if (plan->act == OQ_ACT_INT8_ABSMAX && T >= 1 && T <= 256 && plan->d <= 8192 &&
+      plan->d % 128 == 0 && d_out % 16 == 0) {
+    const oq_status fs = oq_linear_fused(plan, x_bf16, T, ldx, w_packed, w_scale, w_rowsum,
+                                         bias_bf16, d_out, y_bf16, workspace, workspace_bytes,
+                                         stream);
+    if (fs != OQ_ERR_UNSUPPORTED) return fs;
+  }
   const size_t code_bytes = (size_t)T * code_row_bytes(plan);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   void* codes = ws;

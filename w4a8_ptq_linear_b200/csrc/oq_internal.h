@@ -66,7 +66,14 @@ enum : uint32_t {
   kSitePeak = 21,          // tensor-core peak loop: completion of the MMAs
   kSiteFusedLoad = 22,     // single-launch layer: activation codes loaded
   kSiteFusedMma = 23,      // single-launch layer: partial sums complete
-  kSiteDebug = 99          // oq_debug_wait_timeout
+  kSiteDebug = 99,         // oq_debug_wait_timeout
+  // checked builds (-DOQ_CHECKED): an index outside its buffer (sites >= kSiteBounds)
+  kSiteBounds = 0x100,
+  kSiteBoundsRqRow = 0x101,      // single-token kernel: round-1 gather from the staged row
+  kSiteBoundsRqRound2 = 0x102,   // round-2 gather from the round buffer
+  kSiteBoundsPairSlot = 0x103,   // two-token kernel: interleave store into the word buffer
+  kSiteBoundsPairGather = 0x104, // two-token kernel: round-1 gather from the word buffer
+  kSiteBoundsFused = 0x120       // single-launch layer: ring stage, partial sums, token share
 };
 
 // ---- rotate + quantize ---------------------------------------------------------------------

@@ -27,6 +27,15 @@ __device__ __forceinline__ void report(unsigned long long* err, uint32_t site) {
   atomicCAS(err, 0ull, v);
 }
 
+// Checked builds (-DOQ_CHECKED): OQ_IN_BOUNDS(cond, err, site) is cond, and a false cond
+// reports `site` to the error word (first error wins); the caller then skips the access.
+// Release builds compile it to true and check nothing.
+#ifdef OQ_CHECKED
+#define OQ_IN_BOUNDS(cond, err, site) ((cond) ? true : (::oq::dev::report((err), (site)), false))
+#else
+#define OQ_IN_BOUNDS(cond, err, site) true
+#endif
+
 // ---- mbarrier ------------------------------------------------------------------------------
 // Invalidate an mbarrier before its shared memory is used for anything else.
 __device__ __forceinline__ void mbar_inval(uint32_t bar) {

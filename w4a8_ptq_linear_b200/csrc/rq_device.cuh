@@ -313,7 +313,9 @@ __global__ void __launch_bounds__(MAXT, 1) k_rotate_quant(const RqParams p) {
     const uint16_t* row = reinterpret_cast<const uint16_t*>(rowbuf + (size_t)b * row_stride);
 #pragma unroll
     for (int i = 0; i < EP; ++i) {
-      const uint32_t hb = active ? (uint32_t)row[entry(t0, i)] : 0u;
+      const uint32_t ei = entry(t0, i);
+      const uint32_t hb =
+          active && OQ_IN_BOUNDS(ei < (uint32_t)d, p.err, kSiteBoundsRqRow) ? (uint32_t)row[ei] : 0u;
       el(v, i) = __uint_as_float(hb << 16);
     }
     float mu = 0.f;
@@ -359,7 +361,10 @@ __global__ void __launch_bounds__(MAXT, 1) k_rotate_quant(const RqParams p) {
 #pragma unroll
       for (int i = 0; i < EP; ++i) {
         const uint32_t e = entry(t1, i);
-        const float g = active ? rbuf[e & 0x7FFFu] : 0.f;
+        const float g = active && OQ_IN_BOUNDS((e & 0x7FFFu) < (uint32_t)d, p.err,
+                                               kSiteBoundsRqRound2)
+                            ? rbuf[e & 0x7FFFu]
+                            : 0.f;
         el(v, i) = __uint_as_float(__float_as_uint(g) ^ ((e & 0x8000u) << 16));
       }
       if constexpr (kAlias) __syncthreads();  // every warp is done reading the round buffer
@@ -830,6 +835,20 @@ __device__ __forceinline__ void rq_pair_body(const RqParams& p, uint8_t* smem, i
         if (p.want_sum) psum = __fadd2_rn(psum, chunk_sums(a, bb));
         a.x ^= mk.x; a.y ^= mk.y; a.z ^= mk.z; a.w ^= mk.w;
         bb.x ^= mk.x; bb.y ^= mk.y; bb.z ^= mk.z; bb.w ^= mk.w;
+#ifdef OQ_CHECKED
+        {
+          const uint32_t lim = (uint32_t)(nwarps * 4096 - 4);
+          const uint32_t offs[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+          const uint32_t vals[8] = {__byte_perm(a.x, bb.x, 0x5410), __byte_perm(a.x, bb.x, 0x7632),
+                                    __byte_perm(a.y, bb.y, 0x5410), __byte_perm(a.y, bb.y, 0x7632),
+                                    __byte_perm(a.z, bb.z, 0x5410), __byte_perm(a.z, bb.z, 0x7632),
+                                    __byte_perm(a.w, bb.w, 0x5410), __byte_perm(a.w, bb.w, 0x7632)};
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            if (OQ_IN_BOUNDS(offs[k] <= lim && (offs[k] & 3u) == 0u, p.err, kSiteBoundsPairSlot))
+              *reinterpret_cast<uint32_t*>(wbuf + offs[k]) = vals[k];
+        }
+#else
         *reinterpret_cast<uint32_t*>(wbuf + s0.x) = __byte_perm(a.x, bb.x, 0x5410);
         *reinterpret_cast<uint32_t*>(wbuf + s0.y) = __byte_perm(a.x, bb.x, 0x7632);
         *reinterpret_cast<uint32_t*>(wbuf + s0.z) = __byte_perm(a.y, bb.y, 0x5410);
@@ -838,6 +857,7 @@ __device__ __forceinline__ void rq_pair_body(const RqParams& p, uint8_t* smem, i
         *reinterpret_cast<uint32_t*>(wbuf + s1.y) = __byte_perm(a.z, bb.z, 0x7632);
         *reinterpret_cast<uint32_t*>(wbuf + s1.z) = __byte_perm(a.w, bb.w, 0x5410);
         *reinterpret_cast<uint32_t*>(wbuf + s1.w) = __byte_perm(a.w, bb.w, 0x7632);
+#endif
       }
     }
     if (p.want_sum) {
@@ -854,7 +874,12 @@ __device__ __forceinline__ void rq_pair_body(const RqParams& p, uint8_t* smem, i
     float2 v[EP];
 #pragma unroll
     for (int i = 0; i < EP; ++i) {
-      const uint32_t w = active ? *reinterpret_cast<const uint32_t*>(wbuf + entry(t0, i)) : 0u;
+      const uint32_t ei = entry(t0, i);
+      const uint32_t w =
+          active && OQ_IN_BOUNDS(ei <= (uint32_t)(nwarps * 4096 - 4) && (ei & 3u) == 0u, p.err,
+                                 kSiteBoundsPairGather)
+              ? *reinterpret_cast<const uint32_t*>(wbuf + ei)
+              : 0u;
       v[i] = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
     }
     float2 mu = make_float2(0.f, 0.f);
@@ -903,7 +928,10 @@ __device__ __forceinline__ void rq_pair_body(const RqParams& p, uint8_t* smem, i
 #pragma unroll
       for (int i = 0; i < EP; ++i) {
         const uint32_t e = entry(t1, i);
-        const float2 g = active ? rbuf[e & 0x7FFFu] : make_float2(0.f, 0.f);
+        const float2 g = active && OQ_IN_BOUNDS((e & 0x7FFFu) < (uint32_t)d, p.err,
+                                                kSiteBoundsRqRound2)
+                             ? rbuf[e & 0x7FFFu]
+                             : make_float2(0.f, 0.f);
         const uint32_t sb = (e & 0x8000u) << 16;
         v[i] = make_float2(__uint_as_float(__float_as_uint(g.x) ^ sb),
                            __uint_as_float(__float_as_uint(g.y) ^ sb));
