@@ -48,14 +48,16 @@ INT8_PER_BF16 = 2.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM traffic per launch from an ncu capture, valid only for the kernel source it was taken
-# on (sha256 of the .cu file at capture time); null once the kernel has changed.
+# on (sha256 of the kernel's source files at capture time); null once they have changed.
 NCU_TRAFFIC = {
-    # ncu --set full of the CTA-pair kernel (TMA-store epilogue): dram read 17.368 MB + write 0.037 MB
-    ("dit_w4a8", "k_gemm"): {"sha": "7150944b8b4e5abce3e1c8b823aae3a35488a0a0607921af58f132f85ef8694a", "bytes": 17405440},
-    # ncu --set full of the two-token kernel: dram read 25.259 MB + write 0
-    ("dit_w4a8", "k_rotate_quant"): {"sha": "d0b7698240c307304d5df42966d972bbdef49d000e9013581a9acbac570631f6", "bytes": 25258752},
-    # ncu --set full of the grouped-weight kind (first launch): dram read 28.036 MB + write 55.219 MB
-    ("mlp_up_g64", "k_gemm"): {"sha": "7150944b8b4e5abce3e1c8b823aae3a35488a0a0607921af58f132f85ef8694a", "bytes": 83255808},
+    # ncu --set full of k_gemm_a8s (profiles/k_gemm_dit_w4a8.md): dram read 17.378 MB + write 0.011 MB
+    ("dit_w4a8", "k_gemm"): {"sha": "57d6a95b6e663f6eca36d39da6dddc172dc2774c1522eebbe7c745c474d5505d", "bytes": 17389312},
+    # ncu --set full of k_rotate_quant_pair<10, 1, 0> (profiles/k_rotate_quant_dit_w4a8.md):
+    # dram read 18.938 MB + write 0
+    ("dit_w4a8", "k_rotate_quant"): {"sha": "87f6c6be20e09a9f5081d57f6b571448a18a68ae3a8e277a1e60ed8cb6d4ea6f", "bytes": 18937600},
+    # ncu --set full of k_linear_fused<10, 1> at T = 256 (profiles/k_linear_fused_t256.md):
+    # dram read 3.297 MB + write 0
+    ("dit_w4a8@T256", "k_linear_fused"): {"sha": "01bce53c38dc9ed004cf5db98c81bf0d6da5dd5d56ab7d549ff822ffecec2474", "bytes": 3297280},
 }
 
 
@@ -118,9 +120,34 @@ def whole_job_rate(units_per_rank, world, ms):
     return units_per_rank * world / (ms * 1e-3)
 
 
-def sha_of(path):
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()
+def sha_of(*paths):
+    """sha256 of the kernel sources a traffic figure was taken with (concatenated)."""
+    h = hashlib.sha256()
+    for path in paths:
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def csrc(name):
+    return os.path.join(ROOT, "w4a8_ptq_linear_b200", "csrc", name)
+
+
+# the sources each kernel's DRAM traffic depends on
+KERNEL_SOURCES = {
+    "k_gemm": ("k_gemm.cu", "ptx.cuh"),
+    "k_rotate_quant": ("rq_device.cuh", "k_rotate_quant.cu", "ptx.cuh"),
+    "k_linear_fused": ("k_linear_fused.cu", "rq_device.cuh", "ptx.cuh"),
+}
+
+
+def ncu_traffic(workload, kernel):
+    """DRAM bytes per launch from the committed ncu capture, or None once the kernel's sources
+    have changed since it was taken."""
+    tr = NCU_TRAFFIC.get((workload, kernel))
+    if not tr:
+        return None
+    return tr["bytes"] if tr["sha"] == sha_of(*[csrc(f) for f in KERNEL_SOURCES[kernel]]) else None
 
 
 # ---- clocks ---------------------------------------------------------------------------------
@@ -408,7 +435,8 @@ def run_peaks(args):
         return best, clk.summary()
 
     out = []
-    for kind, k_per in (("i8", 32), ("f16", 16)):
+    group_us = {}
+    for kind, k_per in (("i8", 32), ("f16", 16), ("i8_serial", 32)):
         iters = 1 << 14
         pairs = oq.mma_peak_loop(kind, iters)
         ms, clocks = timed(lambda: oq.mma_peak_loop(kind, iters), 4)
@@ -416,9 +444,15 @@ def run_peaks(args):
         st, code = oq.device_status()
         if st != 0:
             raise RuntimeError(f"device status {st} code {code:#x} in the peak loop")
-        out.append({"peak": f"tcgen05 kind::{kind} loop", "value": ops / (ms * 1e-3) / 1e12,
-                    "unit": "TOPS" if kind == "i8" else "TFLOP/s", "ms": ms, "pairs": pairs,
-                    "clocks": clocks})
+        group_us[kind] = ms * 1e3 / iters
+        line = {"peak": f"tcgen05 kind::{kind} loop", "value": ops / (ms * 1e-3) / 1e12,
+                "unit": "TOPS" if kind != "f16" else "TFLOP/s", "ms": ms, "pairs": pairs,
+                "us_per_group_of_four": group_us[kind], "clocks": clocks}
+        if kind == "i8_serial":
+            # each group waited for before the next: the extra time per group is the latency
+            # from the end of the MMAs to the completion the issuing thread sees
+            line["completion_latency_us"] = group_us["i8_serial"] - group_us["i8"]
+        out.append(line)
     n = 8192
     a8 = torch.randint(-128, 128, (n, n), dtype=torch.int8, device=dev)
     b8 = torch.randint(-128, 128, (n, n), dtype=torch.int8, device=dev)
@@ -696,12 +730,8 @@ def main():
     hbm_peak = peaks["hbm_gbs"]
     gemm_tops = ops / (max(gm_ms, 1e-9) * 1e-3) / 1e12
     rq_gbs = rq_bytes / (rq_ms * 1e-3) / 1e9
-    kfile = os.path.join(ROOT, "w4a8_ptq_linear_b200", "csrc", "k_gemm.cu")
-    tr = NCU_TRAFFIC.get((wl.name, "k_gemm"))
-    traffic = tr["bytes"] if tr and tr["sha"] == sha_of(kfile) else None
-    kfile_rq = os.path.join(ROOT, "w4a8_ptq_linear_b200", "csrc", "k_rotate_quant.cu")
-    tr_rq = NCU_TRAFFIC.get((wl.name, "k_rotate_quant"))
-    traffic_rq = tr_rq["bytes"] if tr_rq and tr_rq["sha"] == sha_of(kfile_rq) else None
+    traffic = ncu_traffic(wl.name, "k_gemm")
+    traffic_rq = ncu_traffic(wl.name, "k_rotate_quant")
     rule_note = (f"{peak_kind} {'sustained' if long_region else 'burst'} bf16 "
                  f"{bf16_peak} TFLOP/s" + (" x 2 (nominal int8/bf16 ratio)"
                                            if not fp_gemm else ""))
@@ -728,7 +758,9 @@ def main():
         f_gbs = layer_bytes / (rq_ms * 1e-3) / 1e9
         f_tops = ops / (rq_ms * 1e-3) / 1e12
         dominant = {"bound": "hbm", "achieved": f_gbs, "peak": hbm_peak, "unit": "GB/s",
-                    "frac": f_gbs / hbm_peak, "traffic": None, "kernel": "k_linear_fused",
+                    "frac": f_gbs / hbm_peak,
+                    "traffic": ncu_traffic(f"{wl.name}@T{T}", "k_linear_fused"),
+                    "kernel": "k_linear_fused",
                     "peak_source": f"{peak_kind} copy bandwidth", "ms_per_launch": rq_ms,
                     "algorithmic_bytes": layer_bytes}
         other = {"bound": "tensor", "achieved": f_tops, "peak": tensor_peak, "unit": "TOPS",

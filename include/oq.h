@@ -378,7 +378,10 @@ oq_status oq_linear_static_scratch(const oq_plan* plan, const void* x_bf16, int6
  * iters x 4 back-to-back tcgen05.mma.cta_group::2 instructions (M = 256, N = 256, 128 bytes of
  * K per group of four) on operand tiles resident in shared memory, into one TMEM accumulator,
  * with no memory traffic. kind 0: kind::i8 (int8 x int8 -> int32, K = 32 per instruction);
- * kind 1: kind::f16 (fp16 x fp16 -> fp32, K = 16). One launch performs
+ * kind 1: kind::f16 (fp16 x fp16 -> fp32, K = 16); kind 2: kind::i8 with each group of four
+ * committed to an mbarrier and waited for before the next is issued, so that its time per
+ * group minus kind 0's is the MMA-to-completion latency seen by the issuing thread. One launch
+ * performs
  * pairs * iters * 4 * 2 * 256 * 256 * K operations; *pairs_out (may be NULL) receives pairs.
  * Asynchronous on `stream`: time it with events there. iters in [1, 2^16], else
  * OQ_ERR_INVALID_ARG. */

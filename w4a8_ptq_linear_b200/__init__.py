@@ -449,11 +449,12 @@ def linear_static_scratch(plan: Plan, x, w_packed, w_scale, w_rowsum=None, bias=
 
 
 def mma_peak_loop(kind: str, iters: int, stream=None) -> int:
-    """oq_mma_peak_loop: launches the tensor-core peak loop (kind "i8" or "f16") on the
-    stream; returns the number of CTA pairs, from which the operation count follows."""
+    """oq_mma_peak_loop: launches the tensor-core peak loop (kind "i8", "f16", or "i8_serial":
+    each group of four MMAs waited for before the next) on the stream; returns the number of
+    CTA pairs, from which the operation count follows."""
     pairs = ctypes.c_int(0)
-    _check(lib().oq_mma_peak_loop({"i8": 0, "f16": 1}[kind], iters, ctypes.byref(pairs),
-                                  _stream(stream)))
+    _check(lib().oq_mma_peak_loop({"i8": 0, "f16": 1, "i8_serial": 2}[kind], iters,
+                                  ctypes.byref(pairs), _stream(stream)))
     return pairs.value
 
 

@@ -1084,32 +1084,36 @@ struct RangeIter {
 //
 // Pipeline depth. The completion of an MMA reaches an mbarrier (tcgen05.commit) several hundred
 // nanoseconds after the tensor pipe finishes it, and a stage is refilled only after that
-// arrive. SK = 6 stages of widened weights and of activations (1.7 us of MMA work at N = 256)
-// keep the pipe fed; one commit per K block frees both stages of that block. TMEM holds two
-// accumulators of 256 columns, so the epilogue of one tile overlaps the next tile's MMAs.
+// arrive. SK = 3 stages of two 128-byte K blocks of widened weights and activations (1.7 us of
+// MMA work at N = 256) keep the pipe fed. The single MMA thread pays a fixed cost per stage
+// (its wait, fence and commit), so a stage carries two K blocks: eight MMAs per wait. TMEM
+// holds two accumulators of 256 columns, so the epilogue of one tile overlaps the next tile's
+// MMAs.
 //
 // Schedule: every CTA pair takes a contiguous range of the (channel tile, 32-token chunk) space,
 // cut into tiles of at most 256 tokens; the host chooses the ranges so that the largest
 // per-pair cost (chunks plus a fixed cost per tile) is as small as possible (balance_ranges).
 //
-// Warps: 1 TMEM owner + MMA issuer, 5 activation producer, eight converters in four groups of
-// two that take every fourth K block (four K blocks convert at once: a conversion is bound by
-// the latency of its L2 loads, the stores and the hand-off, not by its work), 12-19 epilogue
-// (two per TMEM lane quarter), 9 and 11 idle.
+// Warps: 1 TMEM owner + MMA issuer, 5 activation producer, eight converters in two groups of
+// four that take every other stage (two stages convert at once: a conversion is bound by the
+// latency of its L2 loads, the stores and the hand-off, not by its work), 12-19 epilogue (two
+// per TMEM lane quarter), 9 and 11 idle.
 // A warp's scheduler is warp % 4: the single MMA thread shares its scheduler only with the
 // producer and the two epilogue warps of lane quarter 1; the converters (warps 0, 2-4, 6-8, 10)
 // use the other three schedulers, so that their work never delays an MMA issue.
 namespace sa {
 constexpr int BN = 256;              // tokens per tile at most (MMA N)
 constexpr int XR = BN / 2;           // activation rows per CTA and stage
-constexpr int SK = 6;                // K-block stages: widened weights and activations
-constexpr int WT = BM * 128;         // widened weight stage bytes
-constexpr int XT = XR * 128;         // activation stage bytes
+constexpr int KSUB = 2;              // 128-byte K blocks per stage
+constexpr int SK = 3;                // stages: widened weights and activations
+constexpr int WT = BM * 128;         // widened weight bytes of one K block
+constexpr int XT = XR * 128;         // activation bytes of one K block (this CTA's rows)
+constexpr int WS = KSUB * WT, XS = KSUB * XT;   // stage bytes
 constexpr int TCOLS = 2 * BN;        // two accumulators
 constexpr int STG = 32 * 32 * 2;     // bf16 [32 tokens][32 channels] staging tile per warp
 constexpr int OFF_W = 0;
-constexpr int OFF_X = OFF_W + SK * WT;
-constexpr int OFF_STG = OFF_X + SK * XT;
+constexpr int OFF_X = OFF_W + SK * WS;
+constexpr int OFF_STG = OFF_X + SK * XS;
 constexpr int OFF_TOK = OFF_STG + (NEPI / 32) * STG;
 constexpr int OFF_BAR = OFF_TOK + BN * 8;
 constexpr int NBAR = 2 * SK + 4 + 1;
@@ -1117,6 +1121,7 @@ constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
 constexpr int SMEM = OFF_MISC + 16 + 1024;
 constexpr int NTHR = 640;
 constexpr int W_PROD_X = 5, W_MMA = 1, W_EPI0 = 12;
+constexpr int CONV_GROUPS = 2;       // converter groups (of four warps); group g takes stages g mod 2
 // converter index (0..7) of a warp, -1 for the other roles
 __device__ __forceinline__ int conv_index(int w) {
   switch (w) {
@@ -1163,26 +1168,28 @@ __global__ void __launch_bounds__(sa::NTHR, 1)
   const uint32_t rank = dev::cluster_ctarank();   // 0 = the pair's leader
   constexpr int UNIT = 2 * BM;                     // channels per tile
   const int nkb = (p.K + 127) / 128;
+  const int nst = (nkb + KSUB - 1) / KSUB;        // stages per tile (a K loop)
   const int unit_index = (int)blockIdx.x / 2;
   auto tiles = [&]() { return ta::RangeIter(p.T, p.sched, unit_index); };
 
-  // ready[s]: K block s is in place, i.e. both activation halves landed (TMA bytes on the
-  // leader's barrier, armed by the leader's producer) and the four converter warps of the pair
-  // stored its widened weights: one wait per K block for the MMA thread
+  // ready[s]: stage s is in place, i.e. both activation halves of its K blocks landed (TMA
+  // bytes on the leader's barrier, armed by the leader's producer) and the converter warps of
+  // both CTAs stored its widened weights: one wait per stage for the MMA thread
   auto bar = [&](int i) { return dev::smem_u32(&bars[i]); };
   auto ready_bar = [&](int s) { return bar(s); };
-  auto kfree_bar = [&](int s) { return bar(SK + s); };        // K block s consumed by the MMAs
+  auto kfree_bar = [&](int s) { return bar(SK + s); };        // stage s consumed by the MMAs
   auto tfull_bar = [&](int b) { return bar(2 * SK + b); };
   auto tempty_bar = [&](int b) { return bar(2 * SK + 2 + b); };
   const uint32_t drain_bar = bar(2 * SK + 4);
-  auto w_stage = [&](int s) { return smem + OFF_W + s * WT; };
-  auto x_stage = [&](int s) { return smem + OFF_X + s * XT; };
+  auto w_stage = [&](int s) { return smem + OFF_W + s * WS; };
+  auto x_stage = [&](int s) { return smem + OFF_X + s * XS; };
   auto lead = [&](uint32_t a) { return dev::map_to_cta(a, 0); };
 
   if (tid == 0) {
     for (int s = 0; s < SK; ++s) {
-      dev::mbar_init(ready_bar(s), 1 + 2 * 2);  // the leader's producer + two converter warps
-      dev::mbar_init(kfree_bar(s), 1);           // of each CTA
+      // the leader's producer + the converter warps of a group in each CTA
+      dev::mbar_init(ready_bar(s), 1 + 2 * (8 / CONV_GROUPS));
+      dev::mbar_init(kfree_bar(s), 1);
     }
     for (int b = 0; b < 2; ++b) {
       dev::mbar_init(tfull_bar(b), 1);
@@ -1213,9 +1220,9 @@ __global__ void __launch_bounds__(sa::NTHR, 1)
       int m, t0, nch;
       while (ok && it.next(m, t0, nch)) {
         const int x0 = t0 + (int)rank * (nch * CH / 2);      // this CTA's activation rows
-        const int krot = k_rotation(m, nkb);
-        for (int step = 0; step < nkb; ++step, ++j) {
-          const int kb = (step + krot) % nkb;
+        const int krot = k_rotation(m, nst);
+        for (int step = 0; step < nst; ++step, ++j) {
+          const int kb0 = ((step + krot) % nst) * KSUB;        // first K block of the stage
           const int s = j % SK;
           if (!dev::mbar_wait(kfree_bar(s), ((j / SK) & 1u) ^ 1u, p.err, kSiteGemmEmpty,
                               p.limit_ns) || *s_abort) {
@@ -1223,9 +1230,13 @@ __global__ void __launch_bounds__(sa::NTHR, 1)
             ok = false;
             break;
           }
-          // both halves complete on the leader's barrier, which expects the bytes of both
-          if (rank == 0) dev::mbar_arrive_expect_tx(ready_bar(s), (uint32_t)(2 * XT));
-          dev::tma_load_2d_pair(dev::smem_u32(x_stage(s)), &tm_x, kb * 128, x0, lead(ready_bar(s)));
+          // both halves complete on the leader's barrier, which expects the bytes of both; a K
+          // block past the end of K (an odd count) lands as zeros and still counts its bytes
+          if (rank == 0) dev::mbar_arrive_expect_tx(ready_bar(s), (uint32_t)(2 * XS));
+#pragma unroll
+          for (int u = 0; u < KSUB; ++u)
+            dev::tma_load_2d_pair(dev::smem_u32(x_stage(s) + u * XT), &tm_x, (kb0 + u) * 128, x0,
+                                  lead(ready_bar(s)));
         }
       }
       // after an abort the landed bytes of the loads in flight can no longer be told apart from
@@ -1254,36 +1265,31 @@ __global__ void __launch_bounds__(sa::NTHR, 1)
         }
         dev::tc_fence_after();
         const uint32_t dt = tmem + (uint32_t)(b * BN);
-        // two K blocks per iteration: the waits, the fence and the loop overhead of the single
-        // issuing thread are paid once for eight MMAs (the tensor pipe idles while it runs them)
-        for (int step = 0; step < nkb; step += 2, j += 2) {
-          const int nb = min(2, nkb - step);
-          const int c0 = j % SK, c1 = (j + 1) % SK;
-          if (!dev::mbar_wait(ready_bar(c0), (j / SK) & 1u, p.err, kSiteGemmFull, p.limit_ns) ||
-              (nb == 2 && !dev::mbar_wait(ready_bar(c1), ((j + 1) / SK) & 1u, p.err,
-                                          kSiteGemmFull, p.limit_ns))) {
+        // one wait, one fence and one commit per stage of KSUB K blocks (4 KSUB MMAs): the
+        // single issuing thread's fixed cost per wait is what sets the pace, not the tensor pipe
+        const int krot = k_rotation(m, nst);
+        for (int step = 0; step < nst; ++step, ++j) {
+          const int c = j % SK;
+          const int kb0 = ((step + krot) % nst) * KSUB;
+          if (!dev::mbar_wait(ready_bar(c), (j / SK) & 1u, p.err, kSiteGemmFull, p.limit_ns)) {
             give_up();
             ok = false;
             break;
           }
           dev::tc_fence_after();
-          const uint32_t aw0 = dev::smem_u32(w_stage(c0)), bx0 = dev::smem_u32(x_stage(c0));
+          const uint32_t aw = dev::smem_u32(w_stage(c)), bx = dev::smem_u32(x_stage(c));
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            dev::mma_i8_pair(dt, dev::sdesc_sw128(aw0 + kk * 32), dev::sdesc_sw128(bx0 + kk * 32),
-                             idesc, (step | kk) != 0);
-          issued = true;
-          dev::mma_commit_pair(kfree_bar(c0));
-          if (nb == 2) {
-            const uint32_t aw1 = dev::smem_u32(w_stage(c1)), bx1 = dev::smem_u32(x_stage(c1));
+          for (int u = 0; u < KSUB; ++u) {
+            if (kb0 + u >= nkb) break;   // past the end of K: zeros, nothing to add
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-              dev::mma_i8_pair(dt, dev::sdesc_sw128(aw1 + kk * 32),
-                               dev::sdesc_sw128(bx1 + kk * 32), idesc, 1);
-            dev::mma_commit_pair(kfree_bar(c1));
+              dev::mma_i8_pair(dt, dev::sdesc_sw128(aw + u * WT + kk * 32),
+                               dev::sdesc_sw128(bx + u * XT + kk * 32), idesc,
+                               (step | u | kk) != 0);
           }
+          issued = true;
+          dev::mma_commit_pair(kfree_bar(c));
         }
-        if (ok) j -= (uint32_t)(((nkb + 1) / 2) * 2 - nkb);   // an odd K loop used one block less
         if (!ok) break;
         dev::mma_commit_pair(tfull_bar(b));
       }
@@ -1294,31 +1300,36 @@ __global__ void __launch_bounds__(sa::NTHR, 1)
     }
   } else if (conv_index(warp) >= 0) {
     // ---------------- converters: packed weights (L2) -> int8 16 n -> shared memory -------
-    // Group g takes the K blocks j = g, g + 4, ... Thread ctid of a group takes 16-byte packed
-    // group q = ctid & 3 of rows r0 + 16 i (r0 = ctid >> 2, i = 0..7): its low nibbles become
-    // chunk 2q and its high nibbles chunk 2q + 1 of the row's 128 widened bytes, stored at
-    // chunk index ^ (row & 7) (the 128-byte swizzle), the same for every i.
-    constexpr int NCG_A = 64, RS = 16, NRI = BM / RS;   // threads per group, row step, rows
-    const int grp = conv_index(warp) >> 1;
-    const int ctid = (conv_index(warp) & 1) * 32 + lane;
+    // Group g (four warps) takes the stages j = g, g + CONV_GROUPS, ... Thread ctid of a group
+    // takes 16-byte packed group q = ctid & 3 of rows r0 + 32 i (r0 = ctid >> 2, i = 0..3) in
+    // each K block of the stage: its low nibbles become chunk 2q and its high nibbles chunk
+    // 2q + 1 of the row's 128 widened bytes, stored at chunk index ^ (row & 7) (the 128-byte
+    // swizzle), the same for every i. All loads of the stage are issued before the wait for a
+    // free stage.
+    constexpr int NCG_A = 32 * (8 / CONV_GROUPS), RS = NCG_A / 4, NRI = BM / RS;
+    const int grp = conv_index(warp) / (8 / CONV_GROUPS);
+    const int ctid = (conv_index(warp) % (8 / CONV_GROUPS)) * 32 + lane;
     const int r0 = ctid >> 2, q = ctid & 3;
     const int ph = r0 & 7;
     const int64_t kbytes = p.K / 2;                  // packed bytes per weight row
-    static_assert(NCG_A / 4 == RS, "one pass of a group covers RS rows");
-    KWalk wk(p.T, p.sched, unit_index, nkb);
+    static_assert(RS % 8 == 0, "rows of a thread share the swizzle phase");
+    KWalk wk(p.T, p.sched, unit_index, nst);
     for (int g = 0; g < grp; ++g) wk.advance();
     bool ok = true;
-    for (uint32_t j = (uint32_t)grp; ok && wk.live; j += 4) {
-      const int kb = (wk.step + k_rotation(wk.m, nkb)) % nkb;
+    for (uint32_t j = (uint32_t)grp; ok && wk.live; j += CONV_GROUPS) {
+      const int kb0 = ((wk.step + k_rotation(wk.m, nst)) % nst) * KSUB;
       const int o0 = wk.m * UNIT + (int)rank * BM;
-      const int64_t col = (int64_t)kb * 64 + q * 16;
-      uint4 in[NRI];
+      uint4 in[KSUB][NRI];
 #pragma unroll
-      for (int i = 0; i < NRI; ++i) {
-        const int o = o0 + r0 + RS * i;
-        in[i] = (o < p.N && col < kbytes)
-                    ? __ldg(reinterpret_cast<const uint4*>(wpk + (int64_t)o * kbytes + col))
-                    : make_uint4(0u, 0u, 0u, 0u);
+      for (int u = 0; u < KSUB; ++u) {
+        const int64_t col = (int64_t)(kb0 + u) * 64 + q * 16;
+#pragma unroll
+        for (int i = 0; i < NRI; ++i) {
+          const int o = o0 + r0 + RS * i;
+          in[u][i] = (o < p.N && col < kbytes)
+                         ? __ldg(reinterpret_cast<const uint4*>(wpk + (int64_t)o * kbytes + col))
+                         : make_uint4(0u, 0u, 0u, 0u);
+        }
       }
       const int c = j % SK;
       bool w = dev::mbar_wait(kfree_bar(c), ((j / SK) & 1u) ^ 1u, p.err, kSiteGemmConv,
@@ -1329,21 +1340,25 @@ __global__ void __launch_bounds__(sa::NTHR, 1)
         ok = false;
         break;
       }
-      uint8_t* dst = w_stage(c);
 #pragma unroll
-      for (int i = 0; i < NRI; ++i) {
-        uint8_t* rowp = dst + (r0 + RS * i) * 128;
-        *reinterpret_cast<uint4*>(rowp + (((2 * q) ^ ph) << 4)) =
-            make_uint4((in[i].x << 4) & 0xF0F0F0F0u, (in[i].y << 4) & 0xF0F0F0F0u,
-                       (in[i].z << 4) & 0xF0F0F0F0u, (in[i].w << 4) & 0xF0F0F0F0u);
-        *reinterpret_cast<uint4*>(rowp + (((2 * q + 1) ^ ph) << 4)) =
-            make_uint4(in[i].x & 0xF0F0F0F0u, in[i].y & 0xF0F0F0F0u, in[i].z & 0xF0F0F0F0u,
-                       in[i].w & 0xF0F0F0F0u);
+      for (int u = 0; u < KSUB; ++u) {
+        uint8_t* dst = w_stage(c) + u * WT;
+#pragma unroll
+        for (int i = 0; i < NRI; ++i) {
+          uint8_t* rowp = dst + (r0 + RS * i) * 128;
+          const uint4 v = in[u][i];
+          *reinterpret_cast<uint4*>(rowp + (((2 * q) ^ ph) << 4)) =
+              make_uint4((v.x << 4) & 0xF0F0F0F0u, (v.y << 4) & 0xF0F0F0F0u,
+                         (v.z << 4) & 0xF0F0F0F0u, (v.w << 4) & 0xF0F0F0F0u);
+          *reinterpret_cast<uint4*>(rowp + (((2 * q + 1) ^ ph) << 4)) =
+              make_uint4(v.x & 0xF0F0F0F0u, v.y & 0xF0F0F0F0u, v.z & 0xF0F0F0F0u,
+                         v.w & 0xF0F0F0F0u);
+        }
       }
       dev::fence_async_smem();   // this thread's stores -> visible to the tensor cores
       __syncwarp();
       if (lane == 0) dev::mbar_arrive_cluster(lead(ready_bar(c)));
-      for (int g = 0; g < 4; ++g) wk.advance();
+      for (int g = 0; g < CONV_GROUPS; ++g) wk.advance();
     }
   } else if (warp >= W_EPI0) {
     // ---------------- epilogue ----------------

@@ -8,6 +8,11 @@
 // else runs: no loads, no conversion, no epilogue, so the time is the tensor pipe's own.
 // The operands hold pseudo-random values (random int8, or fp16 of moderate magnitude), not
 // zeros, so that the datapath toggles as it does on real data.
+//
+// Kind 2 (kind::i8, serialised) issues the same groups but commits each one to an mbarrier and
+// waits for that arrive before issuing the next: its time per group minus kind 0's is the
+// latency from the end of an MMA group to the completion seen by the issuing thread, the figure
+// that sizes the GEMM's operand rings.
 #include <algorithm>
 #include <map>
 #include <mutex>
@@ -33,13 +38,14 @@ __device__ __forceinline__ uint32_t mix32(uint32_t x) {
   return x;
 }
 
-template <bool FP>
+template <bool FP, bool SERIAL>
 __global__ void __launch_bounds__(kPeakThreads, 1)
     k_mma_peak(int64_t iters, unsigned long long* err, unsigned long long limit_ns) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t* done = reinterpret_cast<uint64_t*>(smem + 2 * kTile);
+  uint64_t* step = reinterpret_cast<uint64_t*>(smem + 2 * kTile + 16);   // serial kind
   uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + 2 * kTile + 8);
   const int tid = threadIdx.x;
   const uint32_t rank = dev::cluster_ctarank();
@@ -58,6 +64,7 @@ __global__ void __launch_bounds__(kPeakThreads, 1)
   dev::fence_async_smem();
   if (tid == 0) {
     dev::mbar_init(dev::smem_u32(done), 1);
+    dev::mbar_init(dev::smem_u32(step), 1);
     dev::fence_mbar_init_cluster();
   }
   if (tid < 32) {
@@ -82,6 +89,11 @@ __global__ void __launch_bounds__(kPeakThreads, 1)
         else
           dev::mma_i8_pair(tmem, ad, bd, idesc, (it | kk) != 0);
       }
+      if constexpr (SERIAL) {   // the group's completion, seen by this thread
+        dev::mma_commit_pair(dev::smem_u32(step));
+        if (!dev::mbar_wait(dev::smem_u32(step), (uint32_t)(it & 1), err, kSitePeak, limit_ns))
+          break;
+      }
     }
     dev::mma_commit_pair(dev::smem_u32(done));   // arrives on both CTAs' barriers
   }
@@ -98,8 +110,9 @@ __global__ void __launch_bounds__(kPeakThreads, 1)
 }  // namespace
 
 oq_status launch_mma_peak(int kind, int64_t iters, int* pairs_out, cudaStream_t s) {
-  const void* fn = kind == 0 ? reinterpret_cast<const void*>(&k_mma_peak<false>)
-                             : reinterpret_cast<const void*>(&k_mma_peak<true>);
+  const void* fn = kind == 0   ? reinterpret_cast<const void*>(&k_mma_peak<false, false>)
+                   : kind == 1 ? reinterpret_cast<const void*>(&k_mma_peak<true, false>)
+                               : reinterpret_cast<const void*>(&k_mma_peak<false, true>);
   cudaError_t e = allow_max_dynamic_smem(fn);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(mma_peak)");
   int dev = 0, nsm = 0;
@@ -128,8 +141,9 @@ oq_status launch_mma_peak(int kind, int64_t iters, int* pairs_out, cudaStream_t 
   unsigned long long* err = device_error_word();
   if (!err) return fail(OQ_ERR_CUDA, "device error word unavailable");
   const unsigned long long limit = kWaitLimitNs;
-  e = kind == 0 ? cudaLaunchKernelEx(&cfg, &k_mma_peak<false>, iters, err, limit)
-                : cudaLaunchKernelEx(&cfg, &k_mma_peak<true>, iters, err, limit);
+  e = kind == 0   ? cudaLaunchKernelEx(&cfg, &k_mma_peak<false, false>, iters, err, limit)
+      : kind == 1 ? cudaLaunchKernelEx(&cfg, &k_mma_peak<true, false>, iters, err, limit)
+                  : cudaLaunchKernelEx(&cfg, &k_mma_peak<false, true>, iters, err, limit);
   if (e != cudaSuccess) return cuda_fail(e, "launch mma_peak");
   if (pairs_out) *pairs_out = pairs;
   return OQ_OK;
@@ -138,9 +152,10 @@ oq_status launch_mma_peak(int kind, int64_t iters, int* pairs_out, cudaStream_t 
 }  // namespace oq
 
 extern "C" oq_status oq_mma_peak_loop(int kind, int64_t iters, int* pairs_out, void* stream) {
-  if (kind != 0 && kind != 1) return oq::fail(OQ_ERR_INVALID_ARG, "kind must be 0 (i8) or 1 (f16)");
-  // 2^16 groups of four MMAs take about 20 ms at the nominal rate, far inside the 2 s bound on
-  // the completion wait (a wait that gave up must never be followed by the TMEM release while
+  if (kind < 0 || kind > 2)
+    return oq::fail(OQ_ERR_INVALID_ARG, "kind must be 0 (i8), 1 (f16) or 2 (i8, serialised)");
+  // 2^16 groups of four MMAs take about 20 ms at the nominal rate (about 70 ms serialised), far
+  // inside the 2 s bound on the completion wait (a wait that gave up must never be followed by the TMEM release while
   // MMAs still run)
   if (iters < 1 || iters > (int64_t)1 << 16)
     return oq::fail(OQ_ERR_INVALID_ARG, "iters out of [1, 2^16]");
