@@ -730,8 +730,10 @@ def main():
     hbm_peak = peaks["hbm_gbs"]
     gemm_tops = ops / (max(gm_ms, 1e-9) * 1e-3) / 1e12
     rq_gbs = rq_bytes / (rq_ms * 1e-3) / 1e9
-    traffic = ncu_traffic(wl.name, "k_gemm")
-    traffic_rq = ncu_traffic(wl.name, "k_rotate_quant")
+    # captures are of the workload at its own token count (or T = 256 for the single launch)
+    tkey = wl.name if T == wl.T else f"{wl.name}@T{T}"
+    traffic = ncu_traffic(tkey, "k_gemm")
+    traffic_rq = ncu_traffic(tkey, "k_rotate_quant")
     rule_note = (f"{peak_kind} {'sustained' if long_region else 'burst'} bf16 "
                  f"{bf16_peak} TFLOP/s" + (" x 2 (nominal int8/bf16 ratio)"
                                            if not fp_gemm else ""))
@@ -759,7 +761,7 @@ def main():
         f_tops = ops / (rq_ms * 1e-3) / 1e12
         dominant = {"bound": "hbm", "achieved": f_gbs, "peak": hbm_peak, "unit": "GB/s",
                     "frac": f_gbs / hbm_peak,
-                    "traffic": ncu_traffic(f"{wl.name}@T{T}", "k_linear_fused"),
+                    "traffic": ncu_traffic(tkey, "k_linear_fused"),
                     "kernel": "k_linear_fused",
                     "peak_source": f"{peak_kind} copy bandwidth", "ms_per_launch": rq_ms,
                     "algorithmic_bytes": layer_bytes}

@@ -16,10 +16,10 @@
 //   phase B  split-K GEMM: a cluster of S CTAs owns one 128-channel tile, CTA r of the cluster
 //            its K blocks [r ks, (r + 1) ks), all T <= 256 tokens at once (MMA M = 128
 //            channels, N = T rounded up to 32, kind::i8 into TMEM), the code tiles streaming
-//            through a ring of ns stages. Each CTA stores its int32 partial sums of every
-//            token into the shared memory of the CTA that owns the token (distributed shared
-//            memory); after a cluster barrier CTA r adds the S partial rows of its tokens and
-//            applies the epilogue of CentriQ Eq. 5 / Eq. 9.
+//            through a ring of ns stages. Each CTA moves its int32
+//            partial sums to shared memory; after a cluster barrier CTA r adds the S partials of
+//            its share of the tokens through distributed shared memory and applies the
+//            epilogue of CentriQ Eq. 5 / Eq. 9.
 //
 // Integer partial sums add exactly in any order, and the epilogue takes the same float steps
 // as the two-kernel path (scale alpha_t * s_w / 16, offset mean_t * w_1 + b, one fused
@@ -227,48 +227,35 @@ __global__ void __launch_bounds__(FT, 1)
     if (OQ_IN_BOUNDS(t - t0 < kFusedMaxT, p.err, kSiteBoundsFused))
       s_tok[t - t0] = make_float2(__ldcg(p.rq.scale + t), p.rq.mean ? __ldcg(p.rq.mean + t) : 0.f);
 
-  // ---- partial sums: TMEM -> the owners' shared memory --------------------------------------
-  // CTA r' of the cluster owns tokens [r' tps, (r' + 1) tps) and receives, in its union region,
-  // one row of 128 int32 partial sums per (source CTA, owned token): slot [s][t - t0'][o]. Once
-  // every CTA's MMAs are complete (the cluster barrier below: the union regions hold no code
-  // tiles any more), each thread stores its channel's sums of 32 tokens straight from TMEM
-  // into the owners' shared memory (a warp's stores for one token are 128 contiguous bytes);
-  // remote stores do not wait for a reply, so the exchange costs one more barrier, and the
-  // reduction reads only local shared memory.
+  // ---- partial sums: TMEM -> shared memory (int32 [npad tokens][128 channels]) -------------
+  // A token's 128 partial sums are 512 contiguous bytes, so that the reduction below reads
+  // whole rows from the other CTAs' shared memory; the stores of a warp (32 channels of one
+  // token) are 128 contiguous bytes.
   {
     bool ok = true;
     if (lane == 0) ok = dev::mbar_wait(done, 0, p.err, kSiteFusedMma, p.limit_ns);
     ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-    dev::tc_fence_before();
-    __syncwarp();
-    dev::cluster_sync();   // every CTA's MMAs are complete
     dev::tc_fence_after();
     const bool valid = ok && nk > 0 && *reinterpret_cast<volatile uint32_t*>(&misc[1]) == 0u;
+    int32_t* part = reinterpret_cast<int32_t*>(u);   // the code tiles are consumed
     const int q = warp & 3, o_local = q * 32 + lane;   // TMEM lane quarter of this warp
-    const uint32_t u0 = dev::smem_u32(u);
-    const bool fits = OQ_IN_BOUNDS(S * tps * FM * 4 <= p.off_bar - p.off_u, p.err,
-                                   kSiteBoundsFused);
-    for (int c = warp >> 2; fits && c < npad / 32 && c * 32 < p.T; c += 2) {
+    const bool fits = OQ_IN_BOUNDS(npad * FM * 4 <= p.off_bar - p.off_u, p.err, kSiteBoundsFused);
+    for (int c = warp >> 2; fits && c < npad / 32; c += 2) {
       uint32_t v[32];
       dev::tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(c * 32), v);
       dev::tmem_wait_ld();
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const int t = c * 32 + j;
-        if (t >= p.T) break;
-        const int owner = t / tps;
-        const uint32_t off = (uint32_t)(((r * tps + (t - owner * tps)) * FM + o_local) * 4);
-        dev::st_cluster_u32(dev::map_to_cta(u0 + off, (uint32_t)owner), valid ? v[j] : 0u);
-      }
+      for (int j = 0; j < 32; ++j) part[(c * 32 + j) * FM + o_local] = valid ? (int32_t)v[j] : 0;
     }
   }
+  dev::tc_fence_before();
   __syncwarp();
-  dev::cluster_sync();   // every partial row is in its owner's shared memory
+  dev::cluster_sync();   // every CTA's partial sums are in its shared memory
 
-  // ---- reduction and epilogue: this CTA's tokens [t0, t1) ---------------------------------
-  // Thread: four consecutive channels of one token per item, the S partial rows added from
-  // local shared memory; a warp writes 256 contiguous bytes of y.
-  // y = bf16(acc * (alpha_t s_w / 16) + (mean_t w_1 + b)).
+  // ---- cluster reduction and epilogue ------------------------------------------------------
+  // Thread: four consecutive channels of one token per item, the S partial sums of the
+  // cluster's CTAs loaded together; a warp reads one token's whole row from each CTA and
+  // writes 256 contiguous bytes of y. y = bf16(acc * (alpha_t s_w / 16) + (mean_t w_1 + b)).
   {
     const int c4 = lane * 4;
     const int o = o0 + c4;
@@ -280,14 +267,24 @@ __global__ void __launch_bounds__(FT, 1)
       w1[i] = (has && p.w_rowsum) ? p.w_rowsum[o + i] : 0.f;
       bb[i] = (has && p.bias) ? __bfloat162float(p.bias[o + i]) : 0.f;
     }
-    const int32_t* slots = reinterpret_cast<const int32_t*>(u);
-    for (int t = t0 + warp; t < t1; t += FT / 32) {
+    const uint32_t part0 = dev::smem_u32(u) + (uint32_t)(c4 * 4);
+    uint32_t peer[kFusedMaxS];
+#pragma unroll
+    for (int sr = 0; sr < kFusedMaxS; ++sr)
+      peer[sr] = sr < S ? dev::map_to_cta(part0, (uint32_t)sr) : 0u;
+    const bool fits = OQ_IN_BOUNDS(t1 <= npad && t1 - t0 <= kFusedMaxT, p.err, kSiteBoundsFused);
+    for (int t = t0 + warp; fits && t < t1; t += FT / 32) {
+      const uint32_t off = (uint32_t)(t * FM * 4);
+      uint4 v[kFusedMaxS];
+#pragma unroll
+      for (int sr = 0; sr < kFusedMaxS; ++sr)
+        if (sr < S) v[sr] = dev::ld_cluster_v4(peer[sr] + off);
       int32_t acc[4] = {0, 0, 0, 0};
 #pragma unroll
       for (int sr = 0; sr < kFusedMaxS; ++sr)
         if (sr < S) {
-          const int4 v = *reinterpret_cast<const int4*>(slots + (sr * tps + (t - t0)) * FM + c4);
-          acc[0] += v.x; acc[1] += v.y; acc[2] += v.z; acc[3] += v.w;
+          acc[0] += (int32_t)v[sr].x; acc[1] += (int32_t)v[sr].y;
+          acc[2] += (int32_t)v[sr].z; acc[3] += (int32_t)v[sr].w;
         }
       const float2 tk = s_tok[t - t0];
       uint32_t yb[2];
@@ -303,6 +300,8 @@ __global__ void __launch_bounds__(FT, 1)
       if (has) *reinterpret_cast<uint2*>(p.y + (int64_t)t * p.N + o) = make_uint2(yb[0], yb[1]);
     }
   }
+  __syncwarp();
+  dev::cluster_sync();   // no CTA leaves while another still reads its partial sums
 
   // after an abort, loads already issued may still land: wait for them (bounded) before the
   // block exits (a stage's barrier is at most one phase past its last issued load)
@@ -348,7 +347,7 @@ struct FusedShape {
 // ks K blocks per CTA: the widened weights, then the union of the phase A scratch, the partial
 // sums and as many code-tile stages (up to ks) as the shared memory leaves room for; ns = 0 if
 // not even one stage fits.
-FusedShape fused_shape(int ks, int nkb, int npad, int T, size_t rq_smem, size_t max_smem) {
+FusedShape fused_shape(int ks, int nkb, int npad, size_t rq_smem, size_t max_smem) {
   FusedShape f;
   f.ks = ks;
   f.S = (nkb + ks - 1) / ks;
@@ -356,9 +355,7 @@ FusedShape fused_shape(int ks, int nkb, int npad, int T, size_t rq_smem, size_t 
   // barriers and misc (256 B), the token scales and means (8 B a token), alignment slack
   const size_t tail = 256 + 8 * kFusedMaxT + 1024;
   const size_t stage = (size_t)npad * 128;
-  // the owners' receive slots: S source rows for each of the ceil(T / S) owned tokens
-  const size_t slots = (size_t)f.S * (size_t)((T + f.S - 1) / f.S) * FM * 4;
-  const size_t fixed = std::max(rq_smem, slots);
+  const size_t fixed = std::max(rq_smem, (size_t)npad * FM * 4);
   const size_t room = max_smem > f.off_u + tail ? max_smem - f.off_u - tail : 0;
   int ns = std::min(std::min(ks, kFusedMaxNs), (int)(room / stage));
   size_t uz = std::max(fixed, (size_t)ns * stage);
@@ -407,13 +404,13 @@ oq_status launch_linear_fused(const FusedArgs& a, cudaStream_t s) {
   FusedShape f;
   {
     std::lock_guard<std::mutex> lock(mu);
-    const auto key = std::make_tuple(dev, fn, (int)a.T, nkb, n_o, rq_smem);
+    const auto key = std::make_tuple(dev, fn, npad, nkb, n_o, rq_smem);
     auto it = cache.find(key);
     if (it != cache.end()) {
       f = it->second;
     } else {
       for (int ks = (nkb + kFusedMaxS - 1) / kFusedMaxS; ks <= nkb; ++ks) {
-        const FusedShape c = fused_shape(ks, nkb, npad, (int)a.T, rq_smem, (size_t)max_smem);
+        const FusedShape c = fused_shape(ks, nkb, npad, rq_smem, (size_t)max_smem);
         if (c.ns < 1 || c.smem > (size_t)max_smem) break;   // only grows with ks
         if ((c.S - 1) * ks >= nkb) continue;          // a CTA would get no K block
         cudaLaunchConfig_t cfg{};

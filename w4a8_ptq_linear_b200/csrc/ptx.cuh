@@ -113,10 +113,6 @@ __device__ __forceinline__ uint4 ld_cluster_v4(uint32_t cluster_addr) {
                : "memory");
   return v;
 }
-// One 32-bit word to a shared::cluster address (possibly another CTA's shared memory).
-__device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v) {
-  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
-}
 // Address, in the shared::cluster window, of the same shared-memory offset in CTA `rank`.
 __device__ __forceinline__ uint32_t map_to_cta(uint32_t saddr, uint32_t rank) {
   uint32_t r;
