@@ -218,3 +218,41 @@ def test_lloyd_max_8bit_accumulators_and_epilogue(T, K, N):
     assert rel_fro(y.float().cpu().numpy().astype(np.float64), ref) <= OUT_TOL
     plan.close()
 
+
+
+@pytest.mark.parametrize("T", [1, 37, 128, 200, 256])
+@pytest.mark.parametrize("with_mean,with_bias", [(False, False), (True, True)])
+def test_small_t_w4a8_split_k_matches_oracle(T, with_mean, with_bias):
+    # up to 256 tokens the W4A8 GEMM with a bf16 result runs split-K over clusters, the int32
+    # partial sums added through distributed shared memory; the result is compared with the
+    # oracle's epilogue on the same codes, and with the same call one token at a time
+    import torch
+    import w4a8_ptq_linear_b200 as oq
+    K, N = 3072, 3072
+    rng = np.random.default_rng(100 + T)
+    a = rng.integers(-127, 128, (T, K))
+    w = rng.integers(-7, 8, (N, K))
+    scale = rng.uniform(0.001, 0.1, T).astype(np.float32)
+    s_w = rng.uniform(0.001, 0.05, N).astype(np.float32)
+    mean = rng.normal(0, 3, T).astype(np.float32)
+    w1 = rng.normal(0, 1, N).astype(np.float32)
+    bias_bits = synth.make_bias(N, seed=4)
+    cuda = lambda v: torch.from_numpy(v).cuda()
+    mean_t = cuda(mean) if with_mean else None
+    w1_t = cuda(w1) if with_mean else None
+    bias_t = to_torch_bf16(bias_bits) if with_bias else None
+    at, wp = cuda(a.astype(np.int8)), cuda(pack_w4_gemm(w))
+    y = oq.gemm_w4a8(at, cuda(scale), wp, cuda(s_w), mean=mean_t, w_rowsum=w1_t, bias=bias_t)
+    torch.cuda.synchronize()
+    assert oq.device_status()[0] == 0
+    ref = oracle.epilogue(oracle.gemm_int(a, w), scale.astype(np.float64),
+                          s_w.astype(np.float64), mean.astype(np.float64) if with_mean else None,
+                          w1.astype(np.float64) if with_mean else None,
+                          synth.bf16_to_f64(bias_bits) if with_bias else None)
+    got = y.float().cpu().numpy().astype(np.float64)
+    assert rel_fro(got, ref) < 3e-3
+    # token rows are independent: the first row alone gives the same bits
+    y1 = oq.gemm_w4a8(at[:1], cuda(scale[:1]), wp, cuda(s_w),
+                      mean=mean_t[:1] if with_mean else None, w_rowsum=w1_t, bias=bias_t)
+    torch.cuda.synchronize()
+    assert torch.equal(y1[0], y[0])

@@ -1599,6 +1599,12 @@ oq_status launch_gemm(const GemmArgs& g, cudaStream_t s) {
   p.limit_ns = kWaitLimitNs;
   // up to 128 tokens: single CTAs on 128-channel tiles; beyond: CTA pairs on 256 channels
   const bool small = g.T <= 128;
+  // W4A8 with a bf16 result and up to 256 tokens: the split-K cluster GEMM, which spreads
+  // the K loop over the whole device instead of one tile per channel block
+  if (g.kind == kGemmA8 && !g.out_acc && g.T <= 256) {
+    const oq_status st = launch_gemm_splitk(g, s);
+    if (st != OQ_ERR_UNSUPPORTED) return st;
+  }
   switch (g.kind) {
     case kGemmA8: return small ? run<kGemmA8, 1>(g, p, s) : run_a8s(g, p, s);
     case kGemmA4: return small ? run<kGemmA4, 1>(g, p, s) : run<kGemmA4, 2>(g, p, s);

@@ -51,6 +51,7 @@ constexpr int FWT = FM * 128;     // widened weight bytes of one K block (128 ro
 constexpr int kFusedMaxT = 256;   // tokens of one launch at most (MMA N, TMEM columns)
 constexpr int kFusedMaxS = 8;     // CTAs per cluster at most (portable cluster size)
 constexpr int kFusedMaxNs = 8;    // code-tile stages at most
+constexpr int kTokUnroll = 4;     // tokens per warp in flight in the cluster reduction
 
 struct FusedParams {
   RqParams rq;                    // phase A: codes int8 [T, K], scale [T], mean [T]
@@ -105,7 +106,9 @@ __device__ __forceinline__ void widen_weights(uint8_t* ww, int nk, int t, int nt
   }
 }
 
-template <int HLOG2, int ROUNDS>
+// FUSED = false: the GEMM alone (phase B) on codes, scales and means a previous launch wrote;
+// no grid barrier, no cooperative launch; every thread widens the weights once they land.
+template <int HLOG2, int ROUNDS, bool FUSED>
 __global__ void __launch_bounds__(FT, 1)
     k_linear_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                    const __grid_constant__ FusedParams p) {
@@ -156,9 +159,10 @@ __global__ void __launch_bounds__(FT, 1)
   const uint32_t tmem = misc[0];
 
   // ---- phase A: rotate-quantize the token pairs; widen this CTA's weights ------------------
-  const int nrq = p.rq_threads;
-  if (tid < nrq)
-    rq_pair_body<HLOG2, ROUNDS, kRqInt8>(p.rq, u, (int)blockIdx.x, (int)gridDim.x, nrq, true);
+  const int nrq = FUSED ? p.rq_threads : 0;
+  if constexpr (FUSED)
+    if (tid < nrq)
+      rq_pair_body<HLOG2, ROUNDS, kRqInt8>(p.rq, u, (int)blockIdx.x, (int)gridDim.x, nrq, true);
   // the widening threads: the four or more warps phase A leaves idle, else all after phase A;
   // their first thread waits for the packed weights, the others meet it at the named barrier
   const int w0 = FT - nrq >= FT / 2 ? nrq : 0;
@@ -171,14 +175,18 @@ __global__ void __launch_bounds__(FT, 1)
   // this thread's generic shared-memory writes (widened weights, phase A scratch) are ordered
   // before the tensor core's reads and the TMA writes that follow the barrier below
   dev::fence_async_smem();
-  // every CTA's codes, scales and means are written (the grid barrier orders them before what
-  // follows in every CTA)
-  cooperative_groups::this_grid().sync();
+  if constexpr (FUSED) {
+    // every CTA's codes, scales and means are written (the grid barrier orders them before
+    // what follows in every CTA)
+    cooperative_groups::this_grid().sync();
+  } else {
+    __syncthreads();   // the widened weights, before the MMA thread reads them
+  }
 
   // ---- phase B: split-K GEMM ---------------------------------------------------------------
   int issued = 0;   // code tiles this CTA's producer issued (thread 0)
   if (tid == 0 && nk > 0) {
-    dev::fence_async_global();   // the codes acquired above, before the TMA reads them
+    if constexpr (FUSED) dev::fence_async_global();   // the codes acquired above, before TMA
     for (int k = 0; k < nk; ++k) {
       const int st = k % ns;
       if (k >= ns && !dev::mbar_wait(empty(st), (uint32_t)((k / ns) - 1) & 1u, p.err,
@@ -273,31 +281,43 @@ __global__ void __launch_bounds__(FT, 1)
     for (int sr = 0; sr < kFusedMaxS; ++sr)
       peer[sr] = sr < S ? dev::map_to_cta(part0, (uint32_t)sr) : 0u;
     const bool fits = OQ_IN_BOUNDS(t1 <= npad && t1 - t0 <= kFusedMaxT, p.err, kSiteBoundsFused);
-    for (int t = t0 + warp; fits && t < t1; t += FT / 32) {
-      const uint32_t off = (uint32_t)(t * FM * 4);
-      uint4 v[kFusedMaxS];
+    // kTokUnroll tokens per warp and iteration: their S x kTokUnroll remote loads are all in
+    // flight together (a remote load takes about as long as the rest of the iteration)
+    for (int tb = t0 + warp; fits && tb < t1; tb += kTokUnroll * (FT / 32)) {
+      uint4 v[kTokUnroll][kFusedMaxS];
 #pragma unroll
-      for (int sr = 0; sr < kFusedMaxS; ++sr)
-        if (sr < S) v[sr] = dev::ld_cluster_v4(peer[sr] + off);
-      int32_t acc[4] = {0, 0, 0, 0};
+      for (int uu = 0; uu < kTokUnroll; ++uu) {
+        const int t = tb + uu * (FT / 32);
+        const uint32_t off = (uint32_t)(t * FM * 4);
 #pragma unroll
-      for (int sr = 0; sr < kFusedMaxS; ++sr)
-        if (sr < S) {
-          acc[0] += (int32_t)v[sr].x; acc[1] += (int32_t)v[sr].y;
-          acc[2] += (int32_t)v[sr].z; acc[3] += (int32_t)v[sr].w;
-        }
-      const float2 tk = s_tok[t - t0];
-      uint32_t yb[2];
-#pragma unroll
-      for (int i = 0; i < 4; i += 2) {
-        const float2 s2 = __fmul2_rn(make_float2(tk.x, tk.x), make_float2(sw[i], sw[i + 1]));
-        const float2 c2 = __ffma2_rn(make_float2(tk.y, tk.y), make_float2(w1[i], w1[i + 1]),
-                                     make_float2(bb[i], bb[i + 1]));
-        const float2 a2 = make_float2((float)acc[i], (float)acc[i + 1]);
-        const __nv_bfloat162 yv = __float22bfloat162_rn(__ffma2_rn(a2, s2, c2));
-        yb[i / 2] = *reinterpret_cast<const uint32_t*>(&yv);
+        for (int sr = 0; sr < kFusedMaxS; ++sr)
+          if (sr < S && t < t1) v[uu][sr] = dev::ld_cluster_v4(peer[sr] + off);
       }
-      if (has) *reinterpret_cast<uint2*>(p.y + (int64_t)t * p.N + o) = make_uint2(yb[0], yb[1]);
+#pragma unroll
+      for (int uu = 0; uu < kTokUnroll; ++uu) {
+        const int t = tb + uu * (FT / 32);
+        if (t >= t1) break;
+        int32_t acc[4] = {0, 0, 0, 0};
+#pragma unroll
+        for (int sr = 0; sr < kFusedMaxS; ++sr)
+          if (sr < S) {
+            acc[0] += (int32_t)v[uu][sr].x; acc[1] += (int32_t)v[uu][sr].y;
+            acc[2] += (int32_t)v[uu][sr].z; acc[3] += (int32_t)v[uu][sr].w;
+          }
+        const float2 tk = s_tok[t - t0];
+        uint32_t yb[2];
+#pragma unroll
+        for (int i = 0; i < 4; i += 2) {
+          const float2 s2 = __fmul2_rn(make_float2(tk.x, tk.x), make_float2(sw[i], sw[i + 1]));
+          const float2 c2 = __ffma2_rn(make_float2(tk.y, tk.y), make_float2(w1[i], w1[i + 1]),
+                                       make_float2(bb[i], bb[i + 1]));
+          const float2 a2 = make_float2((float)acc[i], (float)acc[i + 1]);
+          const __nv_bfloat162 yv = __float22bfloat162_rn(__ffma2_rn(a2, s2, c2));
+          yb[i / 2] = *reinterpret_cast<const uint32_t*>(&yv);
+        }
+        if (has)
+          *reinterpret_cast<uint2*>(p.y + (int64_t)t * p.N + o) = make_uint2(yb[0], yb[1]);
+      }
     }
   }
   __syncwarp();
@@ -318,7 +338,7 @@ __global__ void __launch_bounds__(FT, 1)
 
 template <int HL, int R>
 const void* fused_kern() {
-  return reinterpret_cast<const void*>(&k_linear_fused<HL, R>);
+  return reinterpret_cast<const void*>(&k_linear_fused<HL, R, true>);
 }
 
 template <int R>
@@ -368,37 +388,23 @@ FusedShape fused_shape(int ks, int nkb, int npad, size_t rq_smem, size_t max_sme
   return f;
 }
 
-}  // namespace
-
-oq_status launch_linear_fused(const FusedArgs& a, cudaStream_t s) {
-  if (a.T <= 0 || a.T > kFusedMaxT)
-    return fail(OQ_ERR_UNSUPPORTED, "single-launch layer: T must be in [1, %d]", kFusedMaxT);
-  if (a.rq.mode != kRqInt8)
-    return fail(OQ_ERR_UNSUPPORTED, "single-launch layer: INT8 absmax activations only");
-  if (a.N % 16 || a.K % 128)
-    return fail(OQ_ERR_UNSUPPORTED, "single-launch layer: d_in %% 128 == 0, d_out %% 16 == 0");
-  FusedParams p{};
-  int rq_threads = 0;
-  size_t rq_smem = 0;
-  oq_status st = rq_pair_setup(a.rq, p.rq, rq_threads, rq_smem);
-  if (st != OQ_OK) return st;
-  if (rq_threads > FT) return fail(OQ_ERR_UNSUPPORTED, "single-launch layer: d too large");
-  int hlog2 = 0;
-  while ((1 << hlog2) < a.rq.h) ++hlog2;
-  const void* fn = a.rq.rounds == 1 ? fused_kern_h<1>(hlog2) : fused_kern_h<2>(hlog2);
+// Shape, tensor maps and launch of the kernel `fn` (the single launch, or with
+// cooperative = false the GEMM alone) for T tokens, K x N weights; p holds everything else.
+oq_status launch_shaped(const void* fn, bool cooperative, FusedParams& p, const void* codes,
+                        const uint8_t* w, int64_t T, int64_t K, int64_t N, size_t rq_smem,
+                        cudaStream_t s) {
   cudaError_t ce = allow_max_dynamic_smem(fn);
   if (ce != cudaSuccess) return cuda_fail(ce, "cudaFuncSetAttribute(linear_fused)");
-
   int dev = 0, max_smem = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-  const int npad = ((int)a.T + 31) / 32 * 32;
-  const int nkb = (int)(a.K / 128);
-  const int n_o = (int)((a.N + FM - 1) / FM);
+  const int npad = ((int)T + 31) / 32 * 32;
+  const int nkb = (int)(K / 128);
+  const int n_o = (int)((N + FM - 1) / FM);
 
-  // The smallest K share per CTA (most CTAs) whose cluster fits the portable size, whose shared
-  // memory fits, and whose clusters can all be resident at once (the grid barrier needs that).
-  // Computed once per (device, kernel, T rounded, K, N).
+  // The smallest K share per CTA (most CTAs) whose cluster fits the portable size and whose
+  // shared memory fits; for the single launch its clusters must also all be resident at once
+  // (the grid barrier needs that). Computed once per (device, kernel, T rounded, K, N).
   static std::mutex mu;
   static std::map<std::tuple<int, const void*, int, int, int, size_t>, FusedShape> cache;
   FusedShape f;
@@ -429,6 +435,8 @@ oq_status launch_linear_fused(const FusedArgs& a, cudaStream_t s) {
           cudaGetLastError();
           nclusters = 0;
         }
+        // the GEMM alone needs no co-residency: any size that launches at all will do, but
+        // the clusters that fit at once bound its parallelism the same way
         if (nclusters >= n_o) {
           f = c;
           break;
@@ -442,24 +450,18 @@ oq_status launch_linear_fused(const FusedArgs& a, cudaStream_t s) {
                 n_o);
 
   CUtensorMap tx, tw;
-  if (!tma_map_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.rq.codes, (uint64_t)a.K, (uint64_t)a.T,
-                  (uint64_t)a.K, 128, (uint32_t)npad, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !tma_map_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.w, (uint64_t)a.K / 2, (uint64_t)a.N,
-                  (uint64_t)a.K / 2, 64, FM, CU_TENSOR_MAP_SWIZZLE_NONE))
+  if (!tma_map_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, (uint64_t)K, (uint64_t)T,
+                  (uint64_t)K, 128, (uint32_t)npad, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !tma_map_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, w, (uint64_t)K / 2, (uint64_t)N,
+                  (uint64_t)K / 2, 64, FM, CU_TENSOR_MAP_SWIZZLE_NONE))
     return fail(OQ_ERR_CUDA, "cuTensorMapEncodeTiled failed or unavailable");
-  p.w = a.w;
-  p.w_scale = a.w_scale;
-  p.w_rowsum = a.w_rowsum;
-  p.bias = reinterpret_cast<const __nv_bfloat16*>(a.bias);
-  p.y = reinterpret_cast<__nv_bfloat16*>(a.y);
-  p.T = (int)a.T;
-  p.K = (int)a.K;
-  p.N = (int)a.N;
+  p.T = (int)T;
+  p.K = (int)K;
+  p.N = (int)N;
   p.npad = npad;
   p.ks = f.ks;
   p.ns = f.ns;
   p.nkb = nkb;
-  p.rq_threads = rq_threads;
   p.off_u = f.off_u;
   p.off_bar = f.off_bar;
   p.off_tok = f.off_tok;
@@ -480,11 +482,54 @@ oq_status launch_linear_fused(const FusedArgs& a, cudaStream_t s) {
   attr[1].id = cudaLaunchAttributeCooperative;
   attr[1].val.cooperative = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 2;
+  cfg.numAttrs = cooperative ? 2 : 1;
   void* args[] = {&tx, &tw, &p};
   ce = cudaLaunchKernelExC(&cfg, fn, args);
   if (ce != cudaSuccess) return cuda_fail(ce, "launch linear_fused");
   return OQ_OK;
+}
+
+}  // namespace
+
+oq_status launch_linear_fused(const FusedArgs& a, cudaStream_t s) {
+  if (a.T <= 0 || a.T > kFusedMaxT)
+    return fail(OQ_ERR_UNSUPPORTED, "single-launch layer: T must be in [1, %d]", kFusedMaxT);
+  if (a.rq.mode != kRqInt8)
+    return fail(OQ_ERR_UNSUPPORTED, "single-launch layer: INT8 absmax activations only");
+  if (a.N % 16 || a.K % 128)
+    return fail(OQ_ERR_UNSUPPORTED, "single-launch layer: d_in %% 128 == 0, d_out %% 16 == 0");
+  FusedParams p{};
+  int rq_threads = 0;
+  size_t rq_smem = 0;
+  oq_status st = rq_pair_setup(a.rq, p.rq, rq_threads, rq_smem);
+  if (st != OQ_OK) return st;
+  if (rq_threads > FT) return fail(OQ_ERR_UNSUPPORTED, "single-launch layer: d too large");
+  int hlog2 = 0;
+  while ((1 << hlog2) < a.rq.h) ++hlog2;
+  const void* fn = a.rq.rounds == 1 ? fused_kern_h<1>(hlog2) : fused_kern_h<2>(hlog2);
+  p.w = a.w;
+  p.w_scale = a.w_scale;
+  p.w_rowsum = a.w_rowsum;
+  p.bias = reinterpret_cast<const __nv_bfloat16*>(a.bias);
+  p.y = reinterpret_cast<__nv_bfloat16*>(a.y);
+  p.rq_threads = rq_threads;
+  return launch_shaped(fn, true, p, a.rq.codes, a.w, a.T, a.K, a.N, rq_smem, s);
+}
+
+oq_status launch_gemm_splitk(const GemmArgs& g, cudaStream_t s) {
+  if (g.kind != kGemmA8 || g.out_acc || g.T < 1 || g.T > kFusedMaxT || g.N % 16 || g.K % 128)
+    return fail(OQ_ERR_UNSUPPORTED, "split-K GEMM: W4A8, bf16 output, T <= %d", kFusedMaxT);
+  FusedParams p{};
+  p.rq.scale = const_cast<float*>(g.a_scale);
+  p.rq.mean = const_cast<float*>(g.mean);
+  p.w = g.w;
+  p.w_scale = g.w_scale;
+  p.w_rowsum = g.mean ? g.w_rowsum : nullptr;
+  p.bias = reinterpret_cast<const __nv_bfloat16*>(g.bias);
+  p.y = reinterpret_cast<__nv_bfloat16*>(g.out);
+  p.rq_threads = 0;
+  const void* fn = reinterpret_cast<const void*>(&k_linear_fused<0, 1, false>);
+  return launch_shaped(fn, false, p, g.a, g.w, g.T, g.K, g.N, 0, s);
 }
 
 }  // namespace oq

@@ -146,6 +146,9 @@ struct FusedArgs {
   int64_t T = 0, K = 0, N = 0;
 };
 oq_status launch_linear_fused(const FusedArgs& a, cudaStream_t s);
+// The same kernel's split-K GEMM alone (W4A8, bf16 output, 1 <= T <= 256) on codes a previous
+// launch wrote; OQ_ERR_UNSUPPORTED (nothing launched) outside that or when it does not fit.
+oq_status launch_gemm_splitk(const GemmArgs& g, cudaStream_t s);
 
 // oq_prepare_weights that also writes the rotated rows (float [n_out, d]) to `rot` (if not null)
 oq_status oq_prepare_weights_rotated(const oq_plan* plan, const void* w_bf16, int64_t n_out,
