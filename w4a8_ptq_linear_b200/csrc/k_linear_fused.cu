@@ -485,6 +485,12 @@ oq_status launch_shaped(const void* fn, bool cooperative, FusedParams& p, const 
   cfg.numAttrs = cooperative ? 2 : 1;
   void* args[] = {&tx, &tw, &p};
   ce = cudaLaunchKernelExC(&cfg, fn, args);
+  if (ce == cudaErrorCooperativeLaunchTooLarge) {
+    // the device cannot hold every CTA at once right now (e.g. a partitioned or shared GPU):
+    // nothing was launched, and the caller takes the two-kernel path
+    cudaGetLastError();
+    return fail(OQ_ERR_UNSUPPORTED, "single-launch layer: the grid does not fit at once");
+  }
   if (ce != cudaSuccess) return cuda_fail(ce, "launch linear_fused");
   return OQ_OK;
 }
