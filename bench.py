@@ -50,14 +50,17 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic per launch from an ncu capture, valid only for the kernel source it was taken
 # on (sha256 of the kernel's source files at capture time); null once they have changed.
 NCU_TRAFFIC = {
-    # ncu --set full of k_gemm_a8s (profiles/k_gemm_dit_w4a8.md): dram read 17.378 MB + write 0.011 MB
-    ("dit_w4a8", "k_gemm"): {"sha": "57d6a95b6e663f6eca36d39da6dddc172dc2774c1522eebbe7c745c474d5505d", "bytes": 17389312},
+    # ncu --set full of k_gemm_a8s (profiles/k_gemm_dit_w4a8.md): dram read 17.378 MB + write 0.028 MB
+    ("dit_w4a8", "k_gemm"): {"sha": "1cd5718ddffa4e06462ea9fe112d66be691be407e62728f26e7033b23e0691b6", "bytes": 17406464},
     # ncu --set full of k_rotate_quant_pair<10, 1, 0> (profiles/k_rotate_quant_dit_w4a8.md):
-    # dram read 18.938 MB + write 0
-    ("dit_w4a8", "k_rotate_quant"): {"sha": "87f6c6be20e09a9f5081d57f6b571448a18a68ae3a8e277a1e60ed8cb6d4ea6f", "bytes": 18937600},
+    # dram read 25.228 MB + write 0
+    ("dit_w4a8", "k_rotate_quant"): {"sha": "c534d56c906ecaea13e6eb1bf5a09d276c178e7568b1ee867101212c9195590c", "bytes": 25228032},
     # ncu --set full of k_linear_fused<10, 1, 1> at T = 256 (profiles/k_linear_fused_t256.md):
     # dram read 3.294 MB + write 0
     ("dit_w4a8@T256", "k_linear_fused"): {"sha": "e880d62c1be09afc48025f28a0c5807979a49e39f6a692781810bf370db3c231", "bytes": 3293696},
+    # ncu --set full of the split-K GEMM k_linear_fused<0, 1, 0> at T = 256
+    # (profiles/k_gemm_splitk_t256.md): dram read 5.558 MB + write 0
+    ("dit_w4a8@T256", "k_gemm"): {"sha": "e880d62c1be09afc48025f28a0c5807979a49e39f6a692781810bf370db3c231", "bytes": 5558016, "sources": "k_linear_fused"},
 }
 
 
@@ -147,7 +150,8 @@ def ncu_traffic(workload, kernel):
     tr = NCU_TRAFFIC.get((workload, kernel))
     if not tr:
         return None
-    return tr["bytes"] if tr["sha"] == sha_of(*[csrc(f) for f in KERNEL_SOURCES[kernel]]) else None
+    files = KERNEL_SOURCES[tr.get("sources", kernel)]
+    return tr["bytes"] if tr["sha"] == sha_of(*[csrc(f) for f in files]) else None
 
 
 # ---- clocks ---------------------------------------------------------------------------------
