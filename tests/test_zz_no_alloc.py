@@ -4,9 +4,9 @@ Some callers cannot allocate device scratch: plug-ins inside a framework that ow
 memory, or paths that may not call cudaMalloc. For them the library keeps its own fixed
 scratch array. This file checks that the entry point gives bit for bit the layer output of
 oq_linear with a caller-owned workspace (the same kernels on the same inputs, only the scratch
-pointer differs) on two calls in a row, the first with more tokens than the second, so that
-the second call's scales and means sit where the first call left codes: it must not be
-disturbed by what the first left in the shared array. It also checks that the entry point
+pointer differs) on three calls in a row, each with fewer tokens than the one before, so that
+a call's scales and means sit where the previous call left codes: it must not be disturbed by
+what the earlier calls left in the shared array. It also checks that the entry point
 refuses a batch too large for the array. It is collected last so that a failure here comes
 after every other test has run.
 """
@@ -39,7 +39,8 @@ def test_static_scratch_matches_linear_on_consecutive_calls(name):
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     # two calls in a row, different tokens; the first is larger, so the regions of the shared
     # array that hold the second call's scales and means move
-    for call, (T, seed) in enumerate(((2000, 11), (777, 12))):
+    # (a third call of 100 tokens takes the single-launch path for INT8 absmax plans)
+    for call, (T, seed) in enumerate(((2000, 11), (777, 12), (100, 13))):
         assert plan.workspace_bytes(T) <= STATIC_SCRATCH_BYTES
         xb = synth.make_x(T, wl.d, mean_var=wl.mean_var, heavy_frac=wl.heavy_frac, seed=seed)
         x = to_torch_bf16(xb)
