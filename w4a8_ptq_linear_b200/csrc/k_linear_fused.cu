@@ -16,14 +16,17 @@
 //   phase B  split-K GEMM: a cluster of S CTAs owns one 128-channel tile, CTA r of the cluster
 //            its K blocks [r ks, (r + 1) ks), all T <= 256 tokens at once (MMA M = 128
 //            channels, N = T rounded up to 32, kind::i8 into TMEM), the code tiles streaming
-//            through a ring of ns stages. Each CTA moves its int32
-//            partial sums to shared memory; after a cluster barrier CTA r adds the S partials of
-//            its share of the tokens through distributed shared memory and applies the
-//            epilogue of CentriQ Eq. 5 / Eq. 9.
+//            through a ring of ns stages. Each CTA moves its int32 partial sums to shared
+//            memory; after a cluster barrier CTA r adds the S partials of its share of the
+//            tokens through distributed shared memory and applies the epilogue of CentriQ
+//            Eq. 5 / Eq. 9.
 //
 // Integer partial sums add exactly in any order, and the epilogue takes the same float steps
 // as the two-kernel path (scale alpha_t * s_w / 16, offset mean_t * w_1 + b, one fused
 // multiply-add, one rounding to bf16), so both paths return the same bits.
+//
+// With FUSED = false the same kernel is the split-K W4A8 GEMM alone for up to 256 tokens
+// (phase B on codes an earlier launch wrote): an ordinary cluster launch, no grid barrier.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cooperative_groups.h>
