@@ -57,10 +57,10 @@ NCU_TRAFFIC = {
     ("dit_w4a8", "k_rotate_quant"): {"sha": "c534d56c906ecaea13e6eb1bf5a09d276c178e7568b1ee867101212c9195590c", "bytes": 25228032},
     # ncu --set full of k_linear_fused<10, 1, 1> at T = 256 (profiles/k_linear_fused_t256.md):
     # dram read 3.294 MB + write 0
-    ("dit_w4a8@T256", "k_linear_fused"): {"sha": "e880d62c1be09afc48025f28a0c5807979a49e39f6a692781810bf370db3c231", "bytes": 3293696},
+    ("dit_w4a8@T256", "k_linear_fused"): {"sha": "856c3aff665e8befa7f38a057243027f3e6b7be028c0851d2217298e2e2dce17", "bytes": 3293696},
     # ncu --set full of the split-K GEMM k_linear_fused<0, 1, 0> at T = 256
     # (profiles/k_gemm_splitk_t256.md): dram read 5.558 MB + write 0
-    ("dit_w4a8@T256", "k_gemm"): {"sha": "e880d62c1be09afc48025f28a0c5807979a49e39f6a692781810bf370db3c231", "bytes": 5558016, "sources": "k_linear_fused"},
+    ("dit_w4a8@T256", "k_gemm"): {"sha": "856c3aff665e8befa7f38a057243027f3e6b7be028c0851d2217298e2e2dce17", "bytes": 5558016, "sources": "k_linear_fused"},
 }
 
 
