@@ -279,7 +279,8 @@ def run_reference(args, wl, rank):
         return None
     import numpy as np
     import synth
-    wl_, x_bits, w_bits = synth.make_inputs(wl.name, T=min(wl.T, 1024))
+    T = args.tokens or wl.T
+    wl_, x_bits, w_bits = synth.make_inputs(wl.name, T=min(T, 1024))
     setup = oracle_setup(wl, x_bits, w_bits)
     xs = synth.bf16_to_f64(x_bits)
     # size each step so that warm-up + K steps take about two minutes in total
@@ -296,12 +297,12 @@ def run_reference(args, wl, rank):
     el = time.perf_counter() - t0
     ops = 2.0 * n * wl.d * wl.n_out * args.steps
     v = ops / el / 1e12
-    sample = f"{n} tokens per step of the {wl.T}-token workload (float64 NumPy oracle)"
+    sample = f"{n} tokens per step of the {T}-token workload (float64 NumPy oracle)"
     return {"metric": METRIC, "value": v, "unit": "TOPS", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
-            "config": config_of(wl, args.tokens or wl.T, args.gpus, fused=args.fused),
+            "config": config_of(wl, T, args.gpus, fused=args.fused),
             "cpu_baseline": {"value": v, "unit": "TOPS", "cores": blas_threads(),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": v, "unit": "TOPS", "h2d_bytes_per_step": 0,
