@@ -252,7 +252,10 @@ oq_status oq_prepare_weights_g64(const oq_plan* plan, const void* w_bf16, int64_
  *   mean      float [T] or NULL (no rank-1 term; w_rowsum may then be NULL)
  *   w_packed  uint8 [d_out, d_in/2] in the GEMM layout; w_scale float [d_out]
  *   bias_bf16 bf16 [d_out] or NULL
- *   out       bf16 [T, d_out] (OQ_OUT_BF16) or int32 [T, d_out] (OQ_OUT_ACC) */
+ *   out       bf16 [T, d_out] (OQ_OUT_BF16) or int32 [T, d_out] (OQ_OUT_ACC)
+ * For 1 <= T <= 256 with a bf16 result (d_in % 128 == 0) the call runs a split-K cluster GEMM
+ * whose int32 partial sums are added exactly in distributed shared memory; the result is the
+ * same either way. */
 oq_status oq_gemm_w4a8(const int8_t* a, const float* a_scale, const float* mean,
                        const uint8_t* w_packed, const float* w_scale, const float* w_rowsum,
                        const void* bias_bf16, int64_t T, int64_t d_in, int64_t d_out,
