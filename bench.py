@@ -45,6 +45,8 @@ L2_BYTES = 126 << 20   # B200 L2
 # nominal dense int8 / bf16 tensor throughput ratio on B200 (4.5 / 2.25 PFLOP/s), for the
 # peak the measured bf16 GEMM figure implies (reported beside the measured tcgen05 peak)
 INT8_PER_BF16 = 2.0
+# activation kinds the single-launch layer takes
+FUSED_ACTS = ("int8_absmax", "int4_absmax", "int4_percentile")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM traffic per launch from an ncu capture, valid only for the kernel source it was taken
@@ -52,15 +54,15 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 NCU_TRAFFIC = {
     # ncu --set full of k_gemm_a8s (profiles/k_gemm_dit_w4a8.md): dram read 17.378 MB + write 0.028 MB
     ("dit_w4a8", "k_gemm"): {"sha": "1cd5718ddffa4e06462ea9fe112d66be691be407e62728f26e7033b23e0691b6", "bytes": 17406464},
-    # ncu --set full of k_rotate_quant_pair<10, 1, 0> (profiles/k_rotate_quant_dit_w4a8.md):
-    # dram read 25.228 MB + write 0
-    ("dit_w4a8", "k_rotate_quant"): {"sha": "c534d56c906ecaea13e6eb1bf5a09d276c178e7568b1ee867101212c9195590c", "bytes": 25228032},
-    # ncu --set full of k_linear_fused<10, 1, 1> at T = 256 (profiles/k_linear_fused_t256.md):
+    # ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum of k_rotate_quant_pair<10, 1, 0>
+    # (profiles/k_rotate_quant_dit_w4a8.md): dram read 25.229 MB + write 0
+    ("dit_w4a8", "k_rotate_quant"): {"sha": "4b015d18928769dad475d94b8ec7157548036b65a5e9d65eb4b1d2098617a6c8", "bytes": 25229312},
+    # the same metrics of k_linear_fused<10, 1, 1, 0> at T = 256 (profiles/k_linear_fused_t256.md):
     # dram read 3.294 MB + write 0
-    ("dit_w4a8@T256", "k_linear_fused"): {"sha": "856c3aff665e8befa7f38a057243027f3e6b7be028c0851d2217298e2e2dce17", "bytes": 3293696},
-    # ncu --set full of the split-K GEMM k_linear_fused<0, 1, 0> at T = 256
+    ("dit_w4a8@T256", "k_linear_fused"): {"sha": "c1317b878b243d1843dcf021d4be390047c19d8c206cae3e50b9f1f5877ffa60", "bytes": 3294464},
+    # the same metrics of the split-K GEMM k_linear_fused<0, 1, 0, 0> at T = 256
     # (profiles/k_gemm_splitk_t256.md): dram read 5.558 MB + write 0
-    ("dit_w4a8@T256", "k_gemm"): {"sha": "856c3aff665e8befa7f38a057243027f3e6b7be028c0851d2217298e2e2dce17", "bytes": 5558016, "sources": "k_linear_fused"},
+    ("dit_w4a8@T256", "k_gemm"): {"sha": "c1317b878b243d1843dcf021d4be390047c19d8c206cae3e50b9f1f5877ffa60", "bytes": 5558272, "sources": "k_linear_fused"},
 }
 
 
@@ -71,10 +73,11 @@ def parse():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="dit_w4a8",
-                    choices=["tiny", "dit_w4a8", "dit_lm8", "narrow_lm", "narrow_lm_w", "mlp_up",
-                             "mlp_up_pct", "mlp_up_a2", "mlp_up_g64"])
+                    choices=["tiny", "dit_w4a8", "dit_a4", "dit_lm8", "narrow_lm", "narrow_lm_w",
+                             "mlp_up", "mlp_up_pct", "mlp_up_a2", "mlp_up_g64"])
     ap.add_argument("--fused", action="store_true",
-                    help="time the single-launch layer (oq_linear_fused; INT8 absmax, T <= 256)")
+                    help="time the single-launch layer (oq_linear_fused; INT8 absmax, INT4 "
+                         "absmax or percentile activations, T <= 256)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="override the token count (small cases for profiler captures)")
     ap.add_argument("--e2e-steps", type=int, default=100)
@@ -519,8 +522,9 @@ def main():
     # independent sets: activations, prepared weights, codes, scales, outputs
     ring = ring_size(wl, T, L2_BYTES)
     fused = args.fused
-    if fused and (wl.act != "int8_absmax" or g64 or T > 256):
-        raise SystemExit("--fused takes INT8 absmax workloads with per-channel weights, T <= 256")
+    if fused and (wl.act not in FUSED_ACTS or g64 or T > 256):
+        raise SystemExit("--fused takes INT8 absmax or INT4 absmax / percentile workloads with "
+                         "per-channel weights, T <= 256")
     sets = []
     x_host_bits = None
     for r in range(ring):
@@ -759,9 +763,9 @@ def main():
     shares = {"k_rotate_quant": rq_ms / (rq_ms + gm_ms), "k_gemm": gm_ms / (rq_ms + gm_ms)}
     if fused:
         # one kernel does everything: its HBM floor is reading x and the packed weights and
-        # writing y and the workspace's codes, scales and means once
+        # writing y and the workspace's codes (one byte each), scales and means once
         layer_bytes = (T * wl.d * 2 + wl.n_out * wl.d // 2 + wl.n_out * 4 * (2 if wl.center else 1)
-                       + T * wl.n_out * 2 + code_bytes + 4 * T * (2 if wl.center else 1))
+                       + T * wl.n_out * 2 + T * wl.d + 4 * T * (2 if wl.center else 1))
         f_gbs = layer_bytes / (rq_ms * 1e-3) / 1e9
         f_tops = ops / (rq_ms * 1e-3) / 1e12
         dominant = {"bound": "hbm", "achieved": f_gbs, "peak": hbm_peak, "unit": "GB/s",

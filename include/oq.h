@@ -312,15 +312,18 @@ oq_status oq_gemm_w4a8_lloydmax(const oq_plan* plan, const uint8_t* codes, const
                                 int64_t d_in, int64_t d_out, oq_out_kind out_kind, void* out,
                                 void* stream);
 
-/* Bytes of device workspace oq_linear needs for T tokens (codes, scales, means). */
+/* Bytes of device workspace oq_linear needs for T tokens (codes, scales, means). Where the
+ * single launch may run (OQ_ACT_INT8_ABSMAX, OQ_ACT_INT4_ABSMAX and OQ_ACT_INT4_PERCENTILE
+ * plans, 1 <= T <= 256) the code region holds one byte per code. */
 size_t oq_linear_workspace_bytes(const oq_plan* plan, int64_t T);
 
 /* The whole layer: oq_rotate_quantize into `workspace`, then the GEMM for the plan's
  * activation kind, on one stream. y_bf16 is [T, d_out] bf16. workspace must hold
  * oq_linear_workspace_bytes(plan, T) bytes, 256-byte aligned; it is scratch owned by the
- * caller and overwritten. For INT8 absmax plans and 1 <= T <= 256 the call runs as one launch
- * (oq_linear_fused) wherever that path applies; the result and the workspace's contents are
- * the same bits either way. */
+ * caller and overwritten. For INT8 absmax and INT4 (absmax, percentile) plans and
+ * 1 <= T <= 256 the call runs as one launch (oq_linear_fused) wherever that path applies; the
+ * result, and the scales and means in the workspace, are the same bits either way (INT4 codes
+ * are left one per byte by the single launch, two per byte by the two kernels). */
 oq_status oq_linear(const oq_plan* plan, const void* x_bf16, int64_t T, int64_t ldx,
                     const uint8_t* w_packed, const float* w_scale, const float* w_rowsum,
                     const void* bias_bf16, int64_t d_out, void* y_bf16, void* workspace,
@@ -332,7 +335,10 @@ oq_status oq_linear(const oq_plan* plan, const void* x_bf16, int64_t T, int64_t 
  * share of the token pairs), passes one grid-wide barrier, then runs a split-K GEMM in which a
  * cluster of CTAs shares each 128-channel tile and adds its int32 partial sums through
  * distributed shared memory before the epilogue.
- * Limits: the plan's kind must be OQ_ACT_INT8_ABSMAX and d <= 8192 with d % 128 == 0;
+ * INT4 codes are written one two's-complement byte per code (the INT8 layout, values -7..7) and
+ * multiplied by the same kind::i8 GEMM; their integer sums are those of oq_gemm_w4a4.
+ * Limits: the plan's kind must be OQ_ACT_INT8_ABSMAX, OQ_ACT_INT4_ABSMAX or
+ * OQ_ACT_INT4_PERCENTILE, and d <= 8192 with d % 128 == 0;
  * 1 <= T <= 256; the channel tiles' clusters must all fit on the device at once (the launch is
  * cooperative). Outside them it returns OQ_ERR_UNSUPPORTED and launches nothing. */
 oq_status oq_linear_fused(const oq_plan* plan, const void* x_bf16, int64_t T, int64_t ldx,

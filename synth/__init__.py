@@ -17,6 +17,7 @@ activations", OrbitQuant PR #25 "Benchmark subsets"):
                 N(0, var 2), four outlier channels scaled x20; W ~ N(0, 1/d).
 - ``dit_w4a8``  T=4096, d=N=3072, h=1024, 1 round, A8; X ~ N(0,1) with 1% of entries replaced
                 by Student-t(3) draws, plus a per-token mean N(0, var 3); W ~ N(0, 1/d).
+- ``dit_a4``    the ``dit_w4a8`` layer with centered A4 absmax activations (CentriQ's W4A4).
 - ``narrow_lm`` T=8192, d=N=1920, h=128, 2 rounds, A4 Lloyd-Max; X and W as ``dit_w4a8``.
 - ``mlp_up``    T=4096, d=3072, N=12288, h=1024, 1 round, centered A4 absmax; X ~ N(0,1)
                 + per-token mean N(0, var 5); W ~ N(0, 1/d).
@@ -86,6 +87,9 @@ WORKLOADS = {
     # PR #25 compares absmax INT8 against)
     "dit_lm8": Workload("dit_lm8", 4096, 3072, 3072, 1024, 1, "int8_lloydmax", False, 3.0,
                         heavy_frac=0.01),
+    # the same layer with CentriQ's centered INT4 activations (W4A4)
+    "dit_a4": Workload("dit_a4", 4096, 3072, 3072, 1024, 1, "int4_absmax", True, 3.0,
+                       heavy_frac=0.01),
     "narrow_lm": Workload("narrow_lm", 8192, 1920, 1920, 128, 2, "int4_lloydmax", False, 3.0,
                           heavy_frac=0.01),
     # the same layer with the width-d codebook (per-width tables, codebook v3)

@@ -39,7 +39,8 @@ def test_static_scratch_matches_linear_on_consecutive_calls(name):
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     # two calls in a row, different tokens; the first is larger, so the regions of the shared
     # array that hold the second call's scales and means move
-    # (a third call of 100 tokens takes the single-launch path for INT8 absmax plans)
+    # (a third call of 100 tokens takes the single-launch path for the DiT plan; the MLP-up
+    # layer's 96 channel tiles do not fit on the device at once, so it takes the two kernels)
     for call, (T, seed) in enumerate(((2000, 11), (777, 12), (100, 13))):
         assert plan.workspace_bytes(T) <= STATIC_SCRATCH_BYTES
         xb = synth.make_x(T, wl.d, mean_var=wl.mean_var, heavy_frac=wl.heavy_frac, seed=seed)

@@ -364,7 +364,8 @@ def linear(plan: Plan, x, w_packed, w_scale, w_rowsum=None, bias=None, *, worksp
 
 def linear_fused(plan: Plan, x, w_packed, w_scale, w_rowsum=None, bias=None, *, workspace=None,
                  out=None, stream=None):
-    """oq_linear_fused: the whole layer in one launch (T <= 256, INT8 absmax plans)."""
+    """oq_linear_fused: the whole layer in one launch (T <= 256; INT8 absmax, INT4 absmax and
+    INT4 percentile plans)."""
     import torch
     T = x.shape[0]
     N = w_packed.shape[0]

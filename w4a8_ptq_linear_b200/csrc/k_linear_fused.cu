@@ -1,5 +1,7 @@
-// The whole layer in one launch for small token counts: center + RPBH + quantize and the W4A8
-// GEMM with its epilogue, for INT8 absmax activations against per-channel INT4 weights.
+// The whole layer in one launch for small token counts: center + RPBH + quantize and the
+// integer GEMM with its epilogue, for INT8 absmax or INT4 (absmax, percentile) activations
+// against per-channel INT4 weights. INT4 codes are written one byte per code, so that every
+// kind runs the same kind::i8 GEMM on them (their integer sums are those of the 4-bit GEMM).
 //
 // CentriQ App. B.2 runs the activation path as a prologue of its INT4 GEMM: the token tile is
 // loaded once, centered, rotated and quantized with one scale per token, then multiplied. The
@@ -8,7 +10,8 @@
 // kernel instead of a stage of every tile:
 //
 //   phase A  every CTA rotates and quantizes its share of the token pairs with the two-token
-//            body of the standalone kernel (rq_device.cuh), writing codes, scales and means;
+//            body of the standalone kernel (rq_device.cuh), writing codes (one byte each),
+//            scales and means;
 //            meanwhile the CTA's remaining warps widen its slice of the packed INT4 weights
 //            (which do not depend on phase A) into the tensor-core layout in shared memory;
 //   grid     one grid-wide barrier (a cooperative launch, so every CTA is resident) publishes
@@ -23,7 +26,10 @@
 //
 // Integer partial sums add exactly in any order, and the epilogue takes the same float steps
 // as the two-kernel path (scale alpha_t * s_w / 16, offset mean_t * w_1 + b, one fused
-// multiply-add, one rounding to bf16), so both paths return the same bits.
+// multiply-add, one rounding to bf16), so both paths return the same bits. For INT4 codes the
+// two-kernel path's GEMM widens both operands (sums of 256 w x, scale s_w / 256) where this one
+// widens the weights only (16 w x, s_w / 16): the factors are exact powers of two, so the
+// product that enters the fused multiply-add, and hence the result, is the same.
 //
 // With FUSED = false the same kernel is the split-K W4A8 GEMM alone for up to 256 tokens
 // (phase B on codes an earlier launch wrote): an ordinary cluster launch, no grid barrier.
@@ -111,7 +117,8 @@ __device__ __forceinline__ void widen_weights(uint8_t* ww, int nk, int t, int nt
 
 // FUSED = false: the GEMM alone (phase B) on codes, scales and means a previous launch wrote;
 // no grid barrier, no cooperative launch; every thread widens the weights once they land.
-template <int HLOG2, int ROUNDS, bool FUSED>
+// MODE: phase A's quantizer (kRqInt8, kPairInt4B or kPairPct4B).
+template <int HLOG2, int ROUNDS, bool FUSED, int MODE>
 __global__ void __launch_bounds__(FT, 1)
     k_linear_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                    const __grid_constant__ FusedParams p) {
@@ -165,7 +172,7 @@ __global__ void __launch_bounds__(FT, 1)
   const int nrq = FUSED ? p.rq_threads : 0;
   if constexpr (FUSED)
     if (tid < nrq)
-      rq_pair_body<HLOG2, ROUNDS, kRqInt8>(p.rq, u, (int)blockIdx.x, (int)gridDim.x, nrq, true);
+      rq_pair_body<HLOG2, ROUNDS, MODE>(p.rq, u, (int)blockIdx.x, (int)gridDim.x, nrq, true);
   // the widening threads: the four or more warps phase A leaves idle, else all after phase A;
   // their first thread waits for the packed weights, the others meet it at the named barrier
   const int w0 = FT - nrq >= FT / 2 ? nrq : 0;
@@ -339,26 +346,31 @@ __global__ void __launch_bounds__(FT, 1)
   }
 }
 
-template <int HL, int R>
+template <int HL, int R, int M>
 const void* fused_kern() {
-  return reinterpret_cast<const void*>(&k_linear_fused<HL, R, true>);
+  return reinterpret_cast<const void*>(&k_linear_fused<HL, R, true, M>);
 }
 
-template <int R>
+template <int R, int M>
 const void* fused_kern_h(int hlog2) {
   switch (hlog2) {
-    case 0: return fused_kern<0, R>();
-    case 1: return fused_kern<1, R>();
-    case 2: return fused_kern<2, R>();
-    case 3: return fused_kern<3, R>();
-    case 4: return fused_kern<4, R>();
-    case 5: return fused_kern<5, R>();
-    case 6: return fused_kern<6, R>();
-    case 7: return fused_kern<7, R>();
-    case 8: return fused_kern<8, R>();
-    case 9: return fused_kern<9, R>();
-    default: return fused_kern<10, R>();
+    case 0: return fused_kern<0, R, M>();
+    case 1: return fused_kern<1, R, M>();
+    case 2: return fused_kern<2, R, M>();
+    case 3: return fused_kern<3, R, M>();
+    case 4: return fused_kern<4, R, M>();
+    case 5: return fused_kern<5, R, M>();
+    case 6: return fused_kern<6, R, M>();
+    case 7: return fused_kern<7, R, M>();
+    case 8: return fused_kern<8, R, M>();
+    case 9: return fused_kern<9, R, M>();
+    default: return fused_kern<10, R, M>();
   }
+}
+
+template <int M>
+const void* fused_kern_m(int rounds, int hlog2) {
+  return rounds == 1 ? fused_kern_h<1, M>(hlog2) : fused_kern_h<2, M>(hlog2);
 }
 
 // Shared memory of a launch: widened weights, the union region, barriers, alignment slack.
@@ -503,8 +515,9 @@ oq_status launch_shaped(const void* fn, bool cooperative, FusedParams& p, const 
 oq_status launch_linear_fused(const FusedArgs& a, cudaStream_t s) {
   if (a.T <= 0 || a.T > kFusedMaxT)
     return fail(OQ_ERR_UNSUPPORTED, "single-launch layer: T must be in [1, %d]", kFusedMaxT);
-  if (a.rq.mode != kRqInt8)
-    return fail(OQ_ERR_UNSUPPORTED, "single-launch layer: INT8 absmax activations only");
+  if (a.rq.mode != kRqInt8 && a.rq.mode != kRqInt4 && a.rq.mode != kRqPercentile)
+    return fail(OQ_ERR_UNSUPPORTED,
+                "single-launch layer: INT8 absmax, INT4 absmax or INT4 percentile activations");
   if (a.N % 16 || a.K % 128)
     return fail(OQ_ERR_UNSUPPORTED, "single-launch layer: d_in %% 128 == 0, d_out %% 16 == 0");
   FusedParams p{};
@@ -515,7 +528,9 @@ oq_status launch_linear_fused(const FusedArgs& a, cudaStream_t s) {
   if (rq_threads > FT) return fail(OQ_ERR_UNSUPPORTED, "single-launch layer: d too large");
   int hlog2 = 0;
   while ((1 << hlog2) < a.rq.h) ++hlog2;
-  const void* fn = a.rq.rounds == 1 ? fused_kern_h<1>(hlog2) : fused_kern_h<2>(hlog2);
+  const void* fn = a.rq.mode == kRqInt8 ? fused_kern_m<kRqInt8>(a.rq.rounds, hlog2)
+                   : a.rq.mode == kRqInt4 ? fused_kern_m<kPairInt4B>(a.rq.rounds, hlog2)
+                                          : fused_kern_m<kPairPct4B>(a.rq.rounds, hlog2);
   p.w = a.w;
   p.w_scale = a.w_scale;
   p.w_rowsum = a.w_rowsum;
@@ -537,7 +552,7 @@ oq_status launch_gemm_splitk(const GemmArgs& g, cudaStream_t s) {
   p.bias = reinterpret_cast<const __nv_bfloat16*>(g.bias);
   p.y = reinterpret_cast<__nv_bfloat16*>(g.out);
   p.rq_threads = 0;
-  const void* fn = reinterpret_cast<const void*>(&k_linear_fused<0, 1, false>);
+  const void* fn = reinterpret_cast<const void*>(&k_linear_fused<0, 1, false, kRqInt8>);
   return launch_shaped(fn, false, p, g.a, g.w, g.T, g.K, g.N, 0, s);
 }
 

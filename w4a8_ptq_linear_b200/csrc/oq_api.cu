@@ -584,10 +584,23 @@ static size_t code_row_bytes(const oq_plan* plan) {
   return plan->act == OQ_ACT_INT2_PERCENTILE ? (size_t)plan->d / 4 : (size_t)plan->d / 2;
 }
 
+// the activation kinds the single-launch layer takes (it writes their codes one byte each)
+static bool fused_kind(const oq_plan* plan) {
+  return plan->act == OQ_ACT_INT8_ABSMAX || plan->act == OQ_ACT_INT4_ABSMAX ||
+         plan->act == OQ_ACT_INT4_PERCENTILE;
+}
+constexpr int64_t kFusedMaxTokens = 256;
+
+// bytes of oq_linear's code region for T tokens: one byte per code wherever the single launch
+// may run, the kind's own rows otherwise
+static size_t linear_code_bytes(const oq_plan* plan, int64_t T) {
+  if (fused_kind(plan) && T >= 1 && T <= kFusedMaxTokens) return (size_t)T * (size_t)plan->d;
+  return (size_t)T * code_row_bytes(plan);
+}
+
 size_t oq_linear_workspace_bytes(const oq_plan* plan, int64_t T) {
   if (!plan || T < 0) return 0;
-  const size_t code_bytes = (size_t)T * code_row_bytes(plan);
-  return round256(code_bytes) + 2 * round256((size_t)T * 4);
+  return round256(linear_code_bytes(plan, T)) + 2 * round256((size_t)T * 4);
 }
 
 oq_status oq_linear(const oq_plan* plan, const void* x_bf16, int64_t T, int64_t ldx,
@@ -602,16 +615,17 @@ oq_status oq_linear(const oq_plan* plan, const void* x_bf16, int64_t T, int64_t 
   if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return fail(OQ_ERR_MISALIGNED, "workspace must be 256-byte aligned");
   if (plan->center && !w_rowsum) return fail(OQ_ERR_INVALID_ARG, "centering needs w_rowsum");
-  // Up to 256 tokens of an INT8 absmax layer run as one launch where the device holds all of
-  // its clusters at once (same results bit for bit); otherwise the two kernels below.
-  if (plan->act == OQ_ACT_INT8_ABSMAX && T >= 1 && T <= 256 && plan->d <= 8192 &&
+  // Up to 256 tokens of an INT8 absmax or INT4 (absmax, percentile) layer run as one launch
+  // where the device holds all of its clusters at once (same results bit for bit); otherwise
+  // the two kernels below.
+  if (fused_kind(plan) && T >= 1 && T <= kFusedMaxTokens && plan->d <= 8192 &&
       plan->d % 128 == 0 && d_out % 16 == 0) {
     const oq_status fs = oq_linear_fused(plan, x_bf16, T, ldx, w_packed, w_scale, w_rowsum,
                                          bias_bf16, d_out, y_bf16, workspace, workspace_bytes,
                                          stream);
     if (fs != OQ_ERR_UNSUPPORTED) return fs;
   }
-  const size_t code_bytes = (size_t)T * code_row_bytes(plan);
+  const size_t code_bytes = linear_code_bytes(plan, T);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   void* codes = ws;
   float* scale = reinterpret_cast<float*>(ws + round256(code_bytes));
@@ -639,9 +653,11 @@ oq_status oq_linear_fused(const oq_plan* plan, const void* x_bf16, int64_t T, in
                           const void* bias_bf16, int64_t d_out, void* y_bf16, void* workspace,
                           size_t workspace_bytes, void* stream) {
   if (!plan) return fail(OQ_ERR_INVALID_ARG, "NULL plan");
-  if (plan->act != OQ_ACT_INT8_ABSMAX)
-    return fail(OQ_ERR_UNSUPPORTED, "the single-launch layer takes INT8_ABSMAX plans");
-  if (T < 1 || T > 256) return fail(OQ_ERR_UNSUPPORTED, "the single-launch layer takes 1 <= T <= 256");
+  if (!fused_kind(plan))
+    return fail(OQ_ERR_UNSUPPORTED,
+                "the single-launch layer takes INT8_ABSMAX, INT4_ABSMAX or INT4_PERCENTILE plans");
+  if (T < 1 || T > kFusedMaxTokens)
+    return fail(OQ_ERR_UNSUPPORTED, "the single-launch layer takes 1 <= T <= 256");
   const size_t need = oq_linear_workspace_bytes(plan, T);
   if (!workspace || workspace_bytes < need)
     return fail(OQ_ERR_INVALID_ARG, "workspace too small: need %zu bytes", need);
@@ -656,12 +672,16 @@ oq_status oq_linear_fused(const oq_plan* plan, const void* x_bf16, int64_t T, in
   if (st != OQ_OK) return st;
   st = check_plan_device(plan);
   if (st != OQ_OK) return st;
-  const size_t code_bytes = (size_t)T * code_row_bytes(plan);
+  const size_t code_bytes = linear_code_bytes(plan, T);   // T * d: one byte per code
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   FusedArgs f;
   RqArgs& a = f.rq;
   a.x = x_bf16; a.ldx = ldx; a.T = T; a.d = plan->d; a.h = plan->h; a.rounds = plan->rounds;
-  a.center = plan->center; a.mode = kRqInt8; a.tab = plan->d_tab; a.smask = plan->d_smask;
+  a.center = plan->center;
+  a.mode = plan->act == OQ_ACT_INT8_ABSMAX   ? kRqInt8
+           : plan->act == OQ_ACT_INT4_ABSMAX ? kRqInt4
+                                             : kRqPercentile;
+  a.tab = plan->d_tab; a.smask = plan->d_smask;
   a.slot = plan->d_slot; a.ones = plan->d_ones; a.codes = ws;
   a.scale = reinterpret_cast<float*>(ws + round256(code_bytes));
   a.mean = plan->center ? reinterpret_cast<float*>(ws + round256(code_bytes) +

@@ -486,6 +486,11 @@ __global__ void __launch_bounds__(MAXT, 1) k_rotate_quant(const RqParams p) {
 // the two-token kernel's extra quantizer instantiation: 4-bit absmax codes in the GEMM layout
 constexpr int kPairInt4W = 16;   // outside the RqMode values
 static_assert(kPairInt4W > kRqPercentile2, "weight-layout mode must not alias a quantizer");
+// the single launch's 4-bit quantizers (absmax, percentile): the same codes as kRqInt4 and
+// kRqPercentile, stored one two's-complement byte per code (the INT8 layout) for its kind::i8
+// split-K GEMM
+constexpr int kPairInt4B = 17;
+constexpr int kPairPct4B = 18;
 // landing buffers of the two-token kernel (row pairs in flight per CTA)
 constexpr int kPairNbuf = 1;
 
@@ -941,7 +946,7 @@ __device__ __forceinline__ void rq_pair_body(const RqParams& p, uint8_t* smem, i
 
     // ---- per-token statistics --------------------------------------------------------------
     float2 st = make_float2(0.f, 0.f);
-    constexpr bool pct = MODE == kRqPercentile || MODE == kRqPercentile2;
+    constexpr bool pct = MODE == kRqPercentile || MODE == kRqPercentile2 || MODE == kPairPct4B;
     if constexpr (pct) {
       switch (p.pct_r) {
         case 2: pct_warp_lists<2>(v, active, lane, warp, pct_lists); break;
@@ -1070,7 +1075,7 @@ __device__ __forceinline__ void rq_pair_body(const RqParams& p, uint8_t* smem, i
           wa[k] = pack4(r0.x, r1.x, r2.x, r3.x);
           wb[k] = pack4(r0.y, r1.y, r2.y, r3.y);
         }
-        if constexpr (MODE == kRqInt8) {
+        if constexpr (MODE == kRqInt8 || MODE == kPairInt4B || MODE == kPairPct4B) {
           uint4* da = reinterpret_cast<uint4*>(codes + ta * (int64_t)d + base);
           da[0] = make_uint4(wa[0], wa[1], wa[2], wa[3]);
           da[1] = make_uint4(wa[4], wa[5], wa[6], wa[7]);
