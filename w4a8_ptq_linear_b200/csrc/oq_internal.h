@@ -134,10 +134,12 @@ struct GemmArgs {
 };
 oq_status launch_gemm(const GemmArgs& g, cudaStream_t s);
 
-// The whole layer in one launch (T <= 256, INT8 absmax activations, per-channel weights):
-// rotate-quantize into rq.codes / rq.scale / rq.mean, then the GEMM and epilogue into y.
+// The whole layer in one launch (T <= 256; INT8 absmax, INT4 absmax or INT4 percentile
+// activations, rq.mode kRqInt8 / kRqInt4 / kRqPercentile; per-channel weights): rotate-quantize
+// into rq.codes / rq.scale / rq.mean, then the GEMM and epilogue into y.
 struct FusedArgs {
-  RqArgs rq;                        // the activation path, codes int8 [T, K] in the workspace
+  RqArgs rq;                        // the activation path, codes int8 [T, K] (one byte per
+                                    // code for every kind) in the workspace
   const uint8_t* w = nullptr;       // uint8 [N, K/2], GEMM layout
   const float* w_scale = nullptr;
   const float* w_rowsum = nullptr;  // null unless the plan centers
