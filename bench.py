@@ -59,10 +59,10 @@ NCU_TRAFFIC = {
     ("dit_w4a8", "k_rotate_quant"): {"sha": "4b015d18928769dad475d94b8ec7157548036b65a5e9d65eb4b1d2098617a6c8", "bytes": 25229312},
     # the same metrics of k_linear_fused<10, 1, 1, 0> at T = 256 (profiles/k_linear_fused_t256.md):
     # dram read 3.294 MB + write 0
-    ("dit_w4a8@T256", "k_linear_fused"): {"sha": "c1317b878b243d1843dcf021d4be390047c19d8c206cae3e50b9f1f5877ffa60", "bytes": 3294464},
+    ("dit_w4a8@T256", "k_linear_fused"): {"sha": "8d5c5d5381a3e22bfb7dd801e3c23b1639653c392cdaf29e5f574263b7ab32a9", "bytes": 3294464},
     # the same metrics of the split-K GEMM k_linear_fused<0, 1, 0, 0> at T = 256
     # (profiles/k_gemm_splitk_t256.md): dram read 5.558 MB + write 0
-    ("dit_w4a8@T256", "k_gemm"): {"sha": "c1317b878b243d1843dcf021d4be390047c19d8c206cae3e50b9f1f5877ffa60", "bytes": 5558272, "sources": "k_linear_fused"},
+    ("dit_w4a8@T256", "k_gemm"): {"sha": "8d5c5d5381a3e22bfb7dd801e3c23b1639653c392cdaf29e5f574263b7ab32a9", "bytes": 5558272, "sources": "k_linear_fused"},
 }
 
 

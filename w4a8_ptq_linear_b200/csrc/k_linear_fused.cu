@@ -57,7 +57,7 @@ namespace {
 constexpr int FT = 256;           // threads per CTA
 constexpr int FM = 128;           // output channels per cluster (MMA M)
 constexpr int FWT = FM * 128;     // widened weight bytes of one K block (128 rows x 128 B)
-constexpr int kFusedMaxT = 256;   // tokens of one launch at most (MMA N, TMEM columns)
+constexpr int kFusedMaxT = kFusedMaxTokens;   // tokens of one launch at most
 constexpr int kFusedMaxS = 8;     // CTAs per cluster at most (portable cluster size)
 constexpr int kFusedMaxNs = 8;    // code-tile stages at most
 constexpr int kTokUnroll = 4;     // tokens per warp in flight in the cluster reduction

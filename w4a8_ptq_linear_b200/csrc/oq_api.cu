@@ -589,7 +589,6 @@ static bool fused_kind(const oq_plan* plan) {
   return plan->act == OQ_ACT_INT8_ABSMAX || plan->act == OQ_ACT_INT4_ABSMAX ||
          plan->act == OQ_ACT_INT4_PERCENTILE;
 }
-constexpr int64_t kFusedMaxTokens = 256;
 
 // bytes of oq_linear's code region for T tokens: one byte per code wherever the single launch
 // may run, the kind's own rows otherwise
@@ -618,7 +617,7 @@ oq_status oq_linear(const oq_plan* plan, const void* x_bf16, int64_t T, int64_t 
   // Up to 256 tokens of an INT8 absmax or INT4 (absmax, percentile) layer run as one launch
   // where the device holds all of its clusters at once (same results bit for bit); otherwise
   // the two kernels below.
-  if (fused_kind(plan) && T >= 1 && T <= kFusedMaxTokens && plan->d <= 8192 &&
+  if (fused_kind(plan) && T >= 1 && T <= kFusedMaxTokens && plan->d <= kRqPairMaxD &&
       plan->d % 128 == 0 && d_out % 16 == 0) {
     const oq_status fs = oq_linear_fused(plan, x_bf16, T, ldx, w_packed, w_scale, w_rowsum,
                                          bias_bf16, d_out, y_bf16, workspace, workspace_bytes,

@@ -105,6 +105,8 @@ int64_t rq_gather_position(int h, int t, int i);
 int rq_round_buffer_index(int d, int p);
 // Widths up to this run the two-token kernel; wider rows the single-token kernel.
 constexpr int kRqPairMaxD = 8192;
+// tokens of one single-launch layer call at most (its MMA N and TMEM columns)
+constexpr int kFusedMaxTokens = 256;
 // Two-token kernel: the word (32-bit slot of the interleaved row) of every channel, chosen so
 // that the interleave stores and the round-1 gathers of a warp are free of bank conflicts
 // (a 32-colour edge colouring of the bipartite store-group / gather-group multigraph).
